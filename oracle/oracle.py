@@ -1,0 +1,245 @@
+"""numpy-level wrapper around the scalar C oracle (test infrastructure only).
+
+Every function takes and returns dense numpy arrays; BF16 values travel as
+their uint16 bit patterns.  The arithmetic is all in ``pwq_oracle.c``; this
+module only allocates outputs and composes the per-format calls (for NVFP4:
+the group amax over sibling tensors, then quantisation with that amax).
+
+Formats and readings: see the header of ``pwq_oracle.c`` (block-scaled FP8,
+MXFP8 and NVFP4 as defined on "Low Precision RL", "Choose a precision", and
+the verl NVFP4 QAT article, sections 2.3-2.4 and 3.3).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        F = ctypes.c_float
+        L.or_fp_env_ok.restype = ctypes.c_int
+        L.or_bf16_round.restype = ctypes.c_uint16
+        L.or_bf16_round.argtypes = [F]
+        L.or_e4m3_encode.restype = ctypes.c_uint8
+        L.or_e4m3_encode.argtypes = [ctypes.c_double]
+        L.or_e4m3_decode.restype = ctypes.c_double
+        L.or_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.or_e2m1_encode.restype = ctypes.c_uint8
+        L.or_e2m1_encode.argtypes = [ctypes.c_double]
+        L.or_e2m1_decode.restype = ctypes.c_double
+        L.or_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.or_ue8m0_exponent.restype = ctypes.c_int
+        L.or_ue8m0_exponent.argtypes = [F]
+        for name in ("or_bf16_round_array", "or_e4m3_encode_array",
+                     "or_e2m1_encode_array", "or_ue8m0_byte_array"):
+            getattr(L, name).argtypes = [P, P, I64]
+            getattr(L, name).restype = None
+        L.or_fp8_block_quant.argtypes = [P, I64, I64, I64, P, P]
+        L.or_fp8_block_dequant.argtypes = [P, P, I64, I64, I64, P]
+        L.or_mxfp8_quant.argtypes = [P, I64, I64, I64, P, P]
+        L.or_mxfp8_dequant.argtypes = [P, P, I64, I64, I64, P]
+        L.or_amax_bf16.argtypes = [P, I64]
+        L.or_amax_bf16.restype = F
+        L.or_nvfp4_global_scale.argtypes = [F]
+        L.or_nvfp4_global_scale.restype = F
+        L.or_nvfp4_quant.argtypes = [P, I64, I64, F, P, P]
+        L.or_nvfp4_dequant.argtypes = [P, P, F, I64, I64, P]
+        L.or_nvfp4_fake_quant.argtypes = [P, I64, I64, F, P]
+        for name in ("or_fp8_block_quant", "or_fp8_block_dequant", "or_mxfp8_quant",
+                     "or_mxfp8_dequant", "or_nvfp4_quant", "or_nvfp4_dequant",
+                     "or_nvfp4_fake_quant"):
+            getattr(L, name).restype = None
+        _LIB = L
+    return _LIB
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == dtype, (a.dtype, dtype)
+    return a
+
+
+def fp_env_ok():
+    return bool(lib().or_fp_env_ok())
+
+
+# ---------------------------------------------------------------- codecs
+
+def bf16_round(v):
+    v = _c(np.asarray(v, dtype=np.float32), np.float32)
+    out = np.empty(v.shape, np.uint16)
+    lib().or_bf16_round_array(_p(v), _p(out), v.size)
+    return out
+
+
+def e4m3_encode(v):
+    v = _c(np.asarray(v, dtype=np.float32), np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().or_e4m3_encode_array(_p(v), _p(out), v.size)
+    return out
+
+
+def e2m1_encode(v):
+    v = _c(np.asarray(v, dtype=np.float32), np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().or_e2m1_encode_array(_p(v), _p(out), v.size)
+    return out
+
+
+def ue8m0_byte(amax):
+    a = _c(np.asarray(amax, dtype=np.float32), np.float32)
+    out = np.empty(a.shape, np.uint8)
+    lib().or_ue8m0_byte_array(_p(a), _p(out), a.size)
+    return out
+
+
+def e4m3_decode(code):
+    return float(lib().or_e4m3_decode(int(code)))
+
+
+def e2m1_decode(code):
+    return float(lib().or_e2m1_decode(int(code)))
+
+
+def bf16_to_f32(bits):
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------- FP8 block
+
+def _bmn(x):
+    if x.ndim == 2:
+        return 1, x.shape[0], x.shape[1]
+    assert x.ndim == 3
+    return x.shape
+
+
+def fp8_block_quant(x_bits):
+    """x_bits: uint16 [M][N] or [B][M][N].  Returns (codes u8, scales f32
+    [B][ceil(M/128)][ceil(N/128)]) with the input's leading shape."""
+    x = _c(x_bits, np.uint16)
+    B, M, N = _bmn(x)
+    q = np.empty(x.shape, np.uint8)
+    s = np.empty((B, -(-M // 128), -(-N // 128)), np.float32)
+    if x.size:
+        lib().or_fp8_block_quant(_p(x), B, M, N, _p(q), _p(s))
+    if x.ndim == 2:
+        s = s[0]
+    return q, s
+
+
+def fp8_block_dequant(q, s):
+    q = _c(q, np.uint8)
+    s = _c(s, np.float32)
+    B, M, N = _bmn(q)
+    y = np.empty(q.shape, np.uint16)
+    if q.size:
+        lib().or_fp8_block_dequant(_p(q), _p(s), B, M, N, _p(y))
+    return y
+
+
+# ---------------------------------------------------------------- MXFP8
+
+def mxfp8_quant(x_bits):
+    x = _c(x_bits, np.uint16)
+    B, M, N = _bmn(x)
+    assert N % 32 == 0
+    q = np.empty(x.shape, np.uint8)
+    e = np.empty(x.shape[:-1] + (N // 32,), np.uint8)
+    if x.size:
+        lib().or_mxfp8_quant(_p(x), B, M, N, _p(q), _p(e))
+    return q, e
+
+
+def mxfp8_dequant(q, e):
+    q = _c(q, np.uint8)
+    e = _c(e, np.uint8)
+    B, M, N = _bmn(q)
+    y = np.empty(q.shape, np.uint16)
+    if q.size:
+        lib().or_mxfp8_dequant(_p(q), _p(e), B, M, N, _p(y))
+    return y
+
+
+# ---------------------------------------------------------------- NVFP4
+
+def amax_bf16(x_bits):
+    x = _c(x_bits, np.uint16)
+    return float(np.float32(lib().or_amax_bf16(_p(x), x.size)))
+
+
+def nvfp4_group_amax(members):
+    """A = max |x| over every element of every member of a sibling group."""
+    return float(np.float32(max([amax_bf16(m) for m in members] + [0.0])))
+
+
+def nvfp4_global_scale(group_amax):
+    return float(np.float32(lib().or_nvfp4_global_scale(np.float32(group_amax))))
+
+
+def _as_2d(x):
+    return x.reshape(-1, x.shape[-1])
+
+
+def nvfp4_quant(x_bits, group_amax):
+    """One member tensor [..., M, N] with its group's amax.  Returns
+    (packed u8 [..., N/2], sb u8 [..., N/16], gs f32)."""
+    x = _c(x_bits, np.uint16)
+    N = x.shape[-1]
+    assert N % 16 == 0
+    x2 = _as_2d(x)
+    packed = np.empty(x.shape[:-1] + (N // 2,), np.uint8)
+    sb = np.empty(x.shape[:-1] + (N // 16,), np.uint8)
+    if x.size:
+        lib().or_nvfp4_quant(_p(x2), x2.shape[0], N, np.float32(group_amax), _p(packed), _p(sb))
+    return packed, sb, nvfp4_global_scale(group_amax)
+
+
+def nvfp4_dequant(packed, sb, gs, N):
+    packed = _c(packed, np.uint8)
+    sb = _c(sb, np.uint8)
+    M = packed.size // (N // 2) if N else 0
+    y = np.empty(packed.shape[:-1] + (N,), np.uint16)
+    if y.size:
+        lib().or_nvfp4_dequant(_p(packed), _p(sb), np.float32(gs), M, N, _p(y))
+    return y
+
+
+def nvfp4_fake_quant(x_bits, group_amax):
+    x = _c(x_bits, np.uint16)
+    N = x.shape[-1]
+    x2 = _as_2d(x)
+    y = np.empty(x.shape, np.uint16)
+    if x.size:
+        lib().or_nvfp4_fake_quant(_p(x2), x2.shape[0], N, np.float32(group_amax), _p(y))
+    return y
+
+
+def nvfp4_quant_group(members):
+    """Quantise a sibling group (list of member arrays sharing one amax)."""
+    A = nvfp4_group_amax(members)
+    return A, [nvfp4_quant(m, A) for m in members]
+
+
+def unpack_e2m1(packed):
+    """Packed bytes -> one code per element (element 2j from the low nibble)."""
+    packed = np.asarray(packed, np.uint8)
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = packed & 0xF
+    out[..., 1::2] = packed >> 4
+    return out
