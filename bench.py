@@ -1,0 +1,484 @@
+"""Benchmark: the whole block-scaled quantisation path on the Qwen3-4B-shaped
+weight sweep (36 decoder layers x 7 BF16 weight tensors, 3.633 G elements,
+seeded synthetic N(0, 0.02) weights), on N GPUs of one node.
+
+One step takes every element of the sweep through every row of the path:
+  fp8_block_quant -> fp8_block_dequant         (128x128 tiles, FP32 scales)
+  mxfp8_quant     -> mxfp8_dequant             (1x32, UE8M0)
+  nvfp4_quant (q/k/v and gate/up siblings share the global amax) -> nvfp4_dequant
+  nvfp4_fake_quant (siblings; the straight-through backward needs no kernel)
+Each op kind is captured once in a CUDA graph (one node per call, 36 layers)
+and the step replays the graphs back to back on one stream; CUDA events
+between them give the per-op device times.  Inputs (7.3 GB) are larger than
+the 126 MB L2, so no flush is needed between steps.
+
+`value` = elements of the sweep taken through the whole path per second,
+summed over ranks (weak scaling: every rank sweeps its own seeded layers; the
+path needs no collective).  `e2e` = the same metric through the public Python
+API with the BF16 weights in pinned host memory, one layer at a time: H2D
+copy, every op, and a D2H read of the quantised artefacts (codes + scales of
+the three formats) inside the timed region.
+
+`--impl reference` times the CPU oracle (single thread, as it stands) on a
+bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized elements/s and achieved HBM GB/s (% of B200 peak) per format"
+WORKLOAD = "qwen3_4b_weight_sweep_36x7"
+FALLBACK_HBM_GBS = 6650.0
+
+# algorithmic HBM bytes per element: one read of every input, one write of
+# every output (NVFP4 amax re-read not counted: the ideal is one pass)
+BYTES_PER_ELEM = {
+    "fp8_block_quant": 2 + 1 + 4 / 16384,
+    "fp8_block_dequant": 1 + 4 / 16384 + 2,
+    "mxfp8_quant": 2 + 1 + 1 / 32,
+    "mxfp8_dequant": 1 + 1 / 32 + 2,
+    "nvfp4_quant": 2 + 0.5 + 1 / 16,
+    "nvfp4_dequant": 0.5 + 1 / 16 + 2,
+    "nvfp4_fake_quant": 2 + 2,
+}
+# our kernels launched per call (memsets are not counted)
+KERNELS_PER_CALL = {"fp8_block_quant": 1, "fp8_block_dequant": 1, "mxfp8_quant": 1, "mxfp8_dequant": 1,
+                    "nvfp4_quant": 2, "nvfp4_dequant": 1, "nvfp4_fake_quant": 2}
+OPS = list(BYTES_PER_ELEM)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="pwq", choices=["pwq", "reference"])
+    ap.add_argument("--layers", type=int, default=36)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        load = [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ workload
+
+def make_layers(n_layers, device, rank):
+    import workloads as W
+    layers = []
+    for L in range(n_layers):
+        # every rank sweeps its own seeded layers (weak scaling)
+        layers.append(W.qwen3_4b_layer(L + 1000 * rank, device=device))
+    return layers
+
+
+def layer_elems():
+    import workloads as W
+    return sum(r * c for _, (r, c) in W.QWEN3_4B_LAYER)
+
+
+class Buffers:
+    """Pre-allocated outputs for every op of every layer."""
+
+    def __init__(self, layers, P, torch):
+        import workloads as W
+        self.fp8 = []
+        self.mx = []
+        self.nv = []
+        self.y = []
+        self.ws = []
+        dev = layers[0]["q_proj"].device
+        for lay in layers:
+            self.fp8.append({n: (torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev),
+                                 torch.empty((-(-x.shape[0] // 128), -(-x.shape[1] // 128)),
+                                             dtype=torch.float32, device=dev)) for n, x in lay.items()})
+            self.mx.append({n: (torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev),
+                                torch.empty((x.shape[0], x.shape[1] // 32), dtype=torch.uint8, device=dev))
+                            for n, x in lay.items()})
+            nv = {}
+            for g in W.QWEN3_4B_GROUPS:
+                nv[g] = ([torch.empty((lay[n].shape[0], lay[n].shape[1] // 2), dtype=torch.uint8, device=dev)
+                          for n in g],
+                         [torch.empty((lay[n].shape[0], lay[n].shape[1] // 16), dtype=torch.float8_e4m3fn,
+                                      device=dev) for n in g],
+                         torch.empty(1, dtype=torch.float32, device=dev))
+            self.nv.append(nv)
+        # one BF16 output set shared by every dequant / fake-quant (largest layer)
+        self.y = {n: torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for n, x in layers[0].items()}
+
+
+def op_calls(op, layers, buf, P):
+    """Closures for every call of one op kind over all layers."""
+    import workloads as W
+    calls = []
+    for i, lay in enumerate(layers):
+        if op == "fp8_block_quant":
+            for n, x in lay.items():
+                q, s = buf.fp8[i][n]
+                calls.append(lambda x=x, q=q, s=s: P.fp8_block_quant(x, out=q, scale=s))
+        elif op == "fp8_block_dequant":
+            for n in lay:
+                q, s = buf.fp8[i][n]
+                calls.append(lambda q=q, s=s, y=buf.y[n]: P.fp8_block_dequant(q, s, out=y))
+        elif op == "mxfp8_quant":
+            for n, x in lay.items():
+                q, e = buf.mx[i][n]
+                calls.append(lambda x=x, q=q, e=e: P.mxfp8_quant(x, out=q, scale=e))
+        elif op == "mxfp8_dequant":
+            for n in lay:
+                q, e = buf.mx[i][n]
+                calls.append(lambda q=q, e=e, y=buf.y[n]: P.mxfp8_dequant(q, e, out=y))
+        elif op == "nvfp4_quant":
+            for g in W.QWEN3_4B_GROUPS:
+                pk, sb, gs = buf.nv[i][g]
+                xs = [lay[n] for n in g]
+                calls.append(lambda xs=xs, pk=pk, sb=sb, gs=gs: P.nvfp4_quant(xs, out=pk, sb=sb, global_scale=gs))
+        elif op == "nvfp4_dequant":
+            for g in W.QWEN3_4B_GROUPS:
+                pk, sb, gs = buf.nv[i][g]
+                for k, n in enumerate(g):
+                    calls.append(lambda p=pk[k], s=sb[k], gs=gs, y=buf.y[n]: P.nvfp4_dequant(p, s, gs, out=y))
+        elif op == "nvfp4_fake_quant":
+            for g in W.QWEN3_4B_GROUPS:
+                xs = [lay[n] for n in g]
+                ys = [buf.y[n] for n in g]
+                calls.append(lambda xs=xs, ys=ys: P.nvfp4_fake_quant(xs, out=ys))
+    return calls
+
+
+def capture(calls, torch):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for c in calls:           # warm up outside the graph (workspace pool, attributes)
+            c()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    return g
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def cpu_sample_elems():
+    import workloads as W
+    return sum(r * c for n, (r, c) in W.QWEN3_4B_LAYER if n in ("q_proj", "k_proj", "v_proj", "o_proj"))
+
+
+def run_oracle_path(xs_bits, O):
+    """The oracle over the same path for a list of member tensors (one
+    sibling group)."""
+    for x in xs_bits:
+        q, s = O.fp8_block_quant(x)
+        O.fp8_block_dequant(q, s)
+        q, e = O.mxfp8_quant(x)
+        O.mxfp8_dequant(q, e)
+    A = O.nvfp4_group_amax(xs_bits)
+    for x in xs_bits:
+        pk, sb, gs = O.nvfp4_quant(x, A)
+        O.nvfp4_dequant(pk, sb, gs, x.shape[-1])
+        O.nvfp4_fake_quant(x, A)
+
+
+def cpu_baseline(layer_cpu_bits):
+    from oracle import oracle as O
+    groups = [["q_proj", "k_proj", "v_proj"], ["o_proj"]]
+    n = cpu_sample_elems()
+    t0 = time.perf_counter()
+    for g in groups:
+        run_oracle_path([layer_cpu_bits[k] for k in g], O)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "elem/s", "cores": 1, "kind": "oracle",
+            "sample": "layer 0 q/k/v (one NVFP4 sibling group) + o_proj: %d elements through every op "
+                      "of the path, single-threaded scalar C oracle, %.1f s" % (n, dt)}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    args = parse()
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    if args.impl == "reference":
+        return main_reference(args, rank, world, torch, dist)
+
+    import precision_weight_quantization_b200 as P
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hbm_peak, peak_kind = peaks()
+
+    layers = make_layers(args.layers, dev, rank)
+    buf = Buffers(layers, P, torch)
+    elems_per_step = layer_elems() * args.layers
+    graphs = {op: capture(op_calls(op, layers, buf, P), torch) for op in OPS}
+    ncalls = {op: len(op_calls(op, layers[:1], buf, P)) * args.layers for op in OPS}
+    launches_per_step = sum(ncalls[op] * KERNELS_PER_CALL[op] for op in OPS)
+
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        for k, op in enumerate(OPS):
+            if evs is not None:
+                evs[k].record(stream)
+            graphs[op].replay()
+        if evs is not None:
+            evs[len(OPS)].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    per_op_ms = {op: 0.0 for op in OPS}
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(len(OPS) + 1)] for _ in range(args.steps)]
+    with Clocks(local) as clk:
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            step(evsets[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    for evs in evsets:
+        for k, op in enumerate(OPS):
+            per_op_ms[op] += evs[k].elapsed_time(evs[k + 1]) / args.steps
+    ms_per_step = total_ms / args.steps
+    t = torch.tensor([ms_per_step], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = elems_per_step * world / (ms_max / 1e3)
+
+    per_op = {}
+    for op in OPS:
+        ms = per_op_ms[op]
+        gbs = elems_per_step * BYTES_PER_ELEM[op] / (ms / 1e3) / 1e9
+        per_op[op] = {"ms": round(ms, 4), "elem_per_s": elems_per_step / (ms / 1e3), "alg_gbs": round(gbs, 1),
+                      "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "calls": ncalls[op],
+                      "bytes_per_elem": round(BYTES_PER_ELEM[op], 5)}
+    dom = max(OPS, key=lambda o: per_op_ms[o])
+    dom_gbs = per_op[dom]["alg_gbs"]
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(dom_gbs / hbm_peak, 4), "traffic": None, "peak_kind": peak_kind,
+                "note": "achieved = algorithmic bytes of all %d calls / their total device time per step "
+                        "(launch gaps included)" % ncalls[dom]}
+
+    line = {"metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "layers": args.layers, "elements_per_rank": elems_per_step,
+                       "tensors": "q 4096x2560, k/v 1024x2560, o 2560x4096, gate/up 9728x2560, down 2560x9728",
+                       "path": "fp8_block q+dq, mxfp8 q+dq, nvfp4 q (qkv, gate/up siblings)+dq, "
+                               "nvfp4 fake-quant (siblings)",
+                       "l2": "inputs larger than L2 (7.3 GB per rank), no flush",
+                       "launch": "one CUDA graph per op kind, replayed back to back",
+                       "parallelism": "dp%d (independent sweeps)" % world},
+            "per_op": per_op, "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary() if rank == 0 else None}
+
+    if not args.no_e2e:
+        line["e2e"] = e2e(args, layers, P, torch, dev, world, dist, elems_per_step)
+    del graphs
+    if rank == 0 and not args.no_cpu_baseline:
+        import workloads as W
+        lay0 = {n: W.bits(x) for n, x in layers[0].items() if n in ("q_proj", "k_proj", "v_proj", "o_proj")}
+        line["cpu_baseline"] = cpu_baseline(lay0)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
+    """Same path through the public API, host-resident weights: per layer an
+    H2D copy from pinned memory, every op, and a D2H read of the codes and
+    scales of the three formats."""
+    import workloads as W
+    host_in = {n: x.cpu().pin_memory() for n, x in layers[0].items()}
+    dx = {n: torch.empty_like(x) for n, x in layers[0].items()}
+    out_bytes = 0
+    host_out = {}
+    for n, x in layers[0].items():
+        M, N = x.shape
+        host_out[n] = [torch.empty((M, N), dtype=torch.uint8).pin_memory(),
+                       torch.empty((-(-M // 128), -(-N // 128)), dtype=torch.float32).pin_memory(),
+                       torch.empty((M, N), dtype=torch.uint8).pin_memory(),
+                       torch.empty((M, N // 32), dtype=torch.uint8).pin_memory(),
+                       torch.empty((M, N // 2), dtype=torch.uint8).pin_memory(),
+                       torch.empty((M, N // 16), dtype=torch.uint8).pin_memory()]
+        out_bytes += sum(t.numel() * t.element_size() for t in host_out[n])
+    in_bytes = sum(t.numel() * 2 for t in host_in.values())
+    stream = torch.cuda.current_stream()
+
+    def one_layer():
+        for n in dx:
+            dx[n].copy_(host_in[n], non_blocking=True)
+        res = {}
+        for n, x in dx.items():
+            q, s = P.fp8_block_quant(x)
+            P.fp8_block_dequant(q, s)
+            mq, me = P.mxfp8_quant(x)
+            P.mxfp8_dequant(mq, me)
+            res[n] = [q, s, mq, me]
+        for g in W.QWEN3_4B_GROUPS:
+            xs = [dx[n] for n in g]
+            pk, sb, gs = P.nvfp4_quant(xs)
+            for k, n in enumerate(g):
+                P.nvfp4_dequant(pk[k], sb[k], gs)
+                res[n] += [pk[k], sb[k]]
+            P.nvfp4_fake_quant(xs)
+        for n, ts in res.items():
+            for h, d in zip(host_out[n], ts):
+                h.copy_(d.view(h.dtype) if d.dtype != h.dtype and d.element_size() == h.element_size() else d,
+                        non_blocking=True)
+
+    steps = max(1, min(args.steps, 3))
+    for _ in range(1):
+        for _ in range(args.layers):
+            one_layer()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        for _ in range(args.layers):
+            one_layer()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": elems_per_step * world / (ms / 1e3), "unit": "elem/s",
+            "h2d_bytes_per_step": in_bytes * args.layers, "d2h_bytes_per_step": out_bytes * args.layers,
+            "ms_per_step": ms, "steps": steps,
+            "note": "public Python API, one layer at a time from pinned host memory (the same host "
+                    "buffer feeds every layer), codes+scales of the three formats read back"}
+
+
+def main_reference(args, rank, world, torch, dist):
+    """The CPU oracle, as it stands, on a bounded sample of the same workload."""
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    import workloads as W
+    from oracle import oracle as O
+    lay = W.qwen3_4b_layer(0, device="cpu")
+    # per step: a 256-row slice of each q/k/v member (one sibling group) = 1.57 M elements
+    sample = [W.bits(lay[n][:256]) for n in ("q_proj", "k_proj", "v_proj")]
+    n = sum(x.size for x in sample)
+    for _ in range(args.warmup):
+        run_oracle_path(sample, O)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run_oracle_path(sample, O)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = n / dt
+    line = {"metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "layers": args.layers,
+                       "sample_per_step": "256 rows of q/k/v of layer 0 (%d elements)" % n},
+            "cpu_baseline": {"value": value, "unit": "elem/s", "cores": 1, "kind": "oracle",
+                             "sample": "256-row slices of q/k/v (one sibling group) through every op, "
+                                       "single-threaded scalar C oracle"},
+            "e2e": {"value": value, "unit": "elem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,273 @@
+/*
+ * pwq.h -- C ABI of libpwq: block-scaled quantisation of BF16 tensors on
+ * NVIDIA B200 (sm_100a), in the three formats of "Low Precision RL"
+ * ("Choose a precision" table):
+ *
+ *   FP8 block-wise  128x128 tiles, one FP32 scale per tile, E4M3 codes
+ *   MXFP8           1x32 blocks along a row, UE8M0 (power-of-two) scale byte,
+ *                   E4M3 codes
+ *   NVFP4           1x16 blocks along a row, E4M3 block scale, one FP32 global
+ *                   scale per group, E2M1 codes packed two per byte
+ *
+ * plus NVFP4 fake-quantisation (quantise then dequantise, BF16 out) as used
+ * by quantisation-aware training (verl NVFP4 QAT article, section 2.3), with
+ * q/k/v or gate/up siblings sharing one global amax (same article, 2.4).
+ *
+ * ---------------------------------------------------------------------
+ * Conventions shared by every call
+ * ---------------------------------------------------------------------
+ * Tensors.  A pwq_tensor describes a row-major [batch][rows][cols] array
+ * whose last dimension is contiguous.  Strides are counted in storage units
+ * of that array: 2-byte units for BF16, bytes for E4M3 codes, bytes for
+ * packed E2M1 codes (one byte holds two elements).  `cols` is always the
+ * logical number of elements per row.  batch >= 1 (batch > 1 is a stack of
+ * independent matrices, e.g. the experts of a MoE layer).
+ *
+ * Memory.  Every data pointer is a device pointer.  The caller owns every
+ * buffer, including outputs and workspace; the library allocates nothing,
+ * keeps no state between calls and never synchronises.
+ *
+ * Alignment.  Base pointers of BF16 / code / packed tensors must be 16-byte
+ * aligned and their row and batch strides multiples of 16 bytes, else
+ * PWQ_ERR_ALIGN (there is no unaligned slow path).  Scale arrays are dense
+ * (layouts below) and need only their natural alignment.
+ *
+ * Streams.  Every call enqueues its kernels on `stream` (NULL = the legacy
+ * default stream) and returns; the status covers host-side validation and
+ * the launch itself (cudaGetLastError right after each launch).  Device code
+ * never traps; a bounded wait that gives up records a code readable with
+ * pwq_device_error().
+ *
+ * Empty tensors (batch, rows or cols equal to 0) return PWQ_OK and launch
+ * nothing.  Outputs may not overlap inputs or each other (PWQ_ERR_OVERLAP),
+ * except that nvfp4_fake_quant accepts y == x exactly (in place).
+ *
+ * Numerics.  Built without fast math (-ftz=false -prec-div=true
+ * -prec-sqrt=true -fmad=false); every rounding below is IEEE
+ * round-to-nearest-even, as the NVFP4 QDQ review thread on vime pull
+ * request #503 requires (fast math refused).  fl() is one binary32 rounding,
+ * bf16() rounds binary32 to BF16, e4m3() rounds to E4M3 (FN variant, max 448)
+ * saturating, e2m1() rounds to {0,0.5,1,1.5,2,3,4,6} saturating; ties go to
+ * the even code; the sign of zero is kept.  NaN and Inf inputs are outside
+ * the contract.
+ */
+#ifndef PWQ_H
+#define PWQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (same object as cudaStream_t). */
+typedef struct CUstream_st* pwq_stream_t;
+
+typedef enum pwq_status {
+    PWQ_OK = 0,
+    PWQ_ERR_NULL = 1,      /* a required pointer is NULL */
+    PWQ_ERR_ALIGN = 2,     /* base pointer or stride not 16-byte aligned */
+    PWQ_ERR_SHAPE = 3,     /* negative extent, mismatched shapes, cols % 32 (MXFP8) or % 16 (NVFP4) != 0 */
+    PWQ_ERR_STRIDE = 4,    /* row stride < row length, or batch stride < rows * row stride */
+    PWQ_ERR_OVERLAP = 5,   /* an output overlaps an input or another output */
+    PWQ_ERR_WORKSPACE = 6, /* workspace NULL or smaller than nvfp4_workspace_size() */
+    PWQ_ERR_CUDA = 7,      /* a CUDA runtime call or a kernel launch failed */
+    PWQ_ERR_ARG = 8        /* other bad argument: sibling count, batch mismatch, too many tensors */
+} pwq_status;
+
+typedef struct pwq_tensor {
+    void*   ptr;           /* device address of element [0][0][0] */
+    int64_t batch;         /* B */
+    int64_t rows;          /* M */
+    int64_t cols;          /* N, logical elements per row */
+    int64_t batch_stride;  /* storage units between [b][0][0] and [b+1][0][0] */
+    int64_t row_stride;    /* storage units between [b][m][0] and [b][m+1][0] */
+} pwq_tensor;
+
+/* Largest number of sibling tensors in one NVFP4 group. */
+#define PWQ_MAX_SIBLINGS 8
+
+/* ===================================================================== */
+/* FP8 block-wise (DeepSeek-style), 128x128 tiles                        */
+/* ===================================================================== */
+
+/* fp8_block_quant
+ * Source: "Low Precision RL", "Choose a precision" table (FP8 block-wise:
+ * 128x128, FP32 scales) and "Modes" 2 ("Unified block-wise FP8");
+ * "低精度训练与 Rollout", "FP8 训练 + FP8 Rollout" (FP32 block scales via
+ * NVTE_FP8_BLOCK_SCALING_FP32_SCALES=1).
+ * For each 128x128 tile (edge tiles cover only the elements that exist):
+ *   amax = max |x| over the tile, s = fl(amax / 448),
+ *   q = e4m3(fl(x / s)) for every element (s == 0: q = +-0 with x's sign).
+ * x      BF16 [B][M][N], any N >= 1.
+ * q      E4M3 codes, same [B][M][N] shape, caller-allocated.
+ * scale  FP32, dense [B][ceil(M/128)][ceil(N/128)]; s is the dequantisation
+ *        multiplier (x ~= dec(q) * s).
+ * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE (q shape != x shape), _STRIDE,
+ * _OVERLAP, _CUDA. */
+pwq_status fp8_block_quant(const pwq_tensor* x, const pwq_tensor* q, float* scale,
+                           pwq_stream_t stream);
+
+/* fp8_block_dequant
+ * Source: "低精度训练与 Rollout", "FP8 训练 + FP8 Rollout" (FP8 weights are
+ * dequantised to BF16 before each weight update and on checkpoint save).
+ *   y = bf16(fl(dec(q) * s)) with s the element's tile scale.
+ * q      E4M3 codes [B][M][N]; scale FP32 dense [B][ceil(M/128)][ceil(N/128)].
+ * y      BF16 [B][M][N], caller-allocated.
+ * Errors as fp8_block_quant. */
+pwq_status fp8_block_dequant(const pwq_tensor* q, const float* scale, const pwq_tensor* y,
+                             pwq_stream_t stream);
+
+/* ===================================================================== */
+/* MXFP8, 1x32 blocks, UE8M0 scale                                        */
+/* ===================================================================== */
+
+/* mxfp8_quant
+ * Source: "Low Precision RL", "Choose a precision" table (MXFP8: 1x32, UE8M0
+ * scales) and "Modes" 3 ("Unified MXFP8": power-of-two UE8M0 scales packed
+ * as uint8, weights float8_e4m3fn; converter quantises tensors whose last
+ * dimension is divisible by 32).
+ * For each block of 32 consecutive elements of a row:
+ *   e = min{k integer : amax <= 448 * 2^k} clamped to [-127, 127]
+ *       (amax = 0 gives -127), scale byte = e + 127,
+ *   q = e4m3(x * 2^-e) (the scaling is exact; no element saturates).
+ * x      BF16 [B][M][N] with N % 32 == 0 (else PWQ_ERR_SHAPE).
+ * q      E4M3 codes [B][M][N].
+ * scale  uint8, dense [B][M][N/32].
+ * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _STRIDE, _OVERLAP, _CUDA. */
+pwq_status mxfp8_quant(const pwq_tensor* x, const pwq_tensor* q, uint8_t* scale,
+                       pwq_stream_t stream);
+
+/* mxfp8_dequant
+ *   y = bf16(fl(dec(q) * 2^e)), e = scale byte - 127.
+ * q E4M3 [B][M][N] (N % 32 == 0); scale uint8 dense [B][M][N/32];
+ * y BF16 [B][M][N].  Errors as mxfp8_quant. */
+pwq_status mxfp8_dequant(const pwq_tensor* q, const uint8_t* scale, const pwq_tensor* y,
+                         pwq_stream_t stream);
+
+/* ===================================================================== */
+/* NVFP4, 1x16 blocks, two-level scale                                    */
+/* ===================================================================== */
+/*
+ * Source: verl NVFP4 QAT article, section 2.3 (global scale = amax / (6 *
+ * 448) in FP32, per-16 block scale in E4M3 precision, nearest E2M1 value,
+ * multiply back to dequantise), 2.4 (q/k/v and gate/up fusion siblings share
+ * the group's maximum amax), 2.5 / 3.3 (export: packed uint8 codes,
+ * E4M3 weight_scale per 16 elements, FP32 weight_scale_2 = amax /
+ * (6.0 * 448.0)); "Low Precision RL", "Choose a precision" table and
+ * "Modes" 4 (NVFP4: E2M1, 1x16, two-level FP8 + FP32 scales).
+ *
+ * Groups.  A call takes n_siblings (1..PWQ_MAX_SIBLINGS) tensors x[0..n-1]
+ * with the same batch B; group b is {x[i][b] : all i}.  A plain tensor is
+ * n_siblings = 1; batched experts give one group per expert.
+ *   A_b  = max |x| over every element of group b (or amax_in[b] if given),
+ *   gs_b = fl(A_b / 2688)                       (2688 = 6 * 448),
+ * and for each block of 16 consecutive elements of a row, with block
+ * amax a:
+ *   sb = e4m3(fl(a / fl(6 * gs_b)))             (gs_b == 0: sb = 0),
+ *   d  = fl(dec(sb) * gs_b),
+ *   c  = e2m1(fl(x / d))                        (d == 0: c = +-0),
+ * and the dequantised value is y = bf16(fl((dec(c) * dec(sb)) * gs_b)).
+ * Packed codes: element 2j of a row in the low nibble of byte j, 2j+1 in
+ * the high nibble; bit 3 of a nibble is the sign.
+ *
+ * Workspace.  When amax_in is NULL the group amax is reduced on the device
+ * into caller-provided workspace of at least nvfp4_workspace_size() bytes
+ * (256-byte aligned is best; 4-byte aligned is required).  Its contents on
+ * entry do not matter.  When amax_in is given, workspace may be NULL.
+ */
+
+/* Bytes of workspace an NVFP4 call over these siblings needs (4 * B rounded
+ * up to 256).  x points to n_siblings descriptors; returns 0 on bad input. */
+size_t nvfp4_workspace_size(int n_siblings, const pwq_tensor* x);
+
+/* nvfp4_group_amax: A_b for every group, as FP32, into amax_out[B] (device).
+ * This is the one value a data-parallel caller must all-reduce (MAX) when a
+ * group is sharded across devices, before nvfp4_quant with amax_in.
+ * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE (cols % 16), _STRIDE, _ARG, _CUDA. */
+pwq_status nvfp4_group_amax(const pwq_tensor* x, int n_siblings, float* amax_out,
+                            pwq_stream_t stream);
+
+/* nvfp4_quant
+ * x            n_siblings BF16 descriptors [B][M_i][N_i], N_i % 16 == 0.
+ * q_packed     n_siblings descriptors of packed codes, [B][M_i][N_i] logical
+ *              shape (N_i / 2 bytes per row).
+ * sb           host array of n_siblings device pointers, each a dense
+ *              uint8 [B][M_i][N_i/16] array of E4M3 block scales.
+ * global_scale FP32 [B] device output: gs_b (the dequant multiplier).
+ * amax_in      optional FP32 [B] device input: precomputed / all-reduced /
+ *              cached group amax; NULL = reduce it here (needs workspace).
+ * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _STRIDE, _OVERLAP, _WORKSPACE,
+ * _ARG, _CUDA. */
+pwq_status nvfp4_quant(const pwq_tensor* x, int n_siblings, const pwq_tensor* q_packed,
+                       uint8_t* const* sb, float* global_scale, const float* amax_in,
+                       void* workspace, size_t workspace_bytes, pwq_stream_t stream);
+
+/* nvfp4_dequant: one tensor.
+ * q_packed  packed codes [B][M][N] logical shape; sb dense uint8 [B][M][N/16];
+ * global_scale FP32 [B]; y BF16 [B][M][N].
+ * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _STRIDE, _OVERLAP, _CUDA. */
+pwq_status nvfp4_dequant(const pwq_tensor* q_packed, const uint8_t* sb,
+                         const float* global_scale, const pwq_tensor* y, pwq_stream_t stream);
+
+/* nvfp4_fake_quant: y = dequant(quant(x)) for every sibling, BF16 in and
+ * out, without writing codes or scales; bitwise equal to nvfp4_dequant of
+ * nvfp4_quant.  y[i] may be exactly x[i] (in place).  The backward of
+ * fake-quantisation is the straight-through estimator (grad_x = grad_y, no
+ * gradient for the scales; verl NVFP4 QAT article, section 2.3), which
+ * needs no kernel.
+ * amax_out optional FP32 [B] device output: the group amax that was used.
+ * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _STRIDE, _OVERLAP, _WORKSPACE,
+ * _ARG, _CUDA. */
+pwq_status nvfp4_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_siblings,
+                            const float* amax_in, float* amax_out, void* workspace,
+                            size_t workspace_bytes, pwq_stream_t stream);
+
+/* ===================================================================== */
+/* Diagnostics                                                            */
+/* ===================================================================== */
+
+/* Human-readable name of a status code (static string). */
+const char* pwq_status_string(pwq_status status);
+
+/* One line on the most recent failure in the calling thread: the argument
+ * that failed validation, or the CUDA error name and message. */
+const char* pwq_last_error_detail(void);
+
+/* Build description: target architecture and the exact-math compiler flags
+ * (static string). */
+const char* pwq_build_info(void);
+
+/* Reads and clears the device-side error word of the current device
+ * (synchronous; 0 = no error; bit 0 = a TMA load wait gave up).  Returns
+ * PWQ_ERR_NULL or PWQ_ERR_CUDA on failure. */
+pwq_status pwq_device_error(uint32_t* code);
+
+/* Exhaustive self-check of the device arithmetic against CUDA's IEEE
+ * division (__fdiv_rn), for every BF16 numerator x and every divisor the
+ * formats can produce:
+ *   which = 0  FP8 block: divisors s = fl(a / 448), a every positive BF16;
+ *              compares e4m3 codes and binary32 quotients.
+ *   which = 1  NVFP4: divisors d = fl(dec(sb) * fl(a / 2688)) for every
+ *              positive BF16 a and every non-zero E4M3 sb; compares e2m1
+ *              codes.
+ * counts (device, 4 x uint64, zeroed by the call): [0] pairs checked,
+ * [1] code mismatches, [2] binary32 quotient mismatches (which = 0 only,
+ * where the quotient is a normal number), [3] pairs that took the
+ * division fallback.  Asynchronous on `stream`. */
+pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream);
+
+/* Runs the device codecs over 2^32 / 2^k inputs starting at `first`
+ * (uint32 bit patterns of binary32 values, `count` of them, stepping by 1)
+ * and writes: e4m3 codes (count bytes), e2m1 codes (count bytes, one code
+ * per byte), bf16 bit patterns (count x uint16).  Any of the outputs may be
+ * NULL.  Used to compare the device conversions with the oracle. */
+pwq_status pwq_selftest_codecs(uint32_t first, uint32_t count, uint8_t* e4m3, uint8_t* e2m1,
+                               uint16_t* bf16, pwq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PWQ_H */

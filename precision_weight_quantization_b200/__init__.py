@@ -1,0 +1,283 @@
+"""B200-native block-scaled quantisation of BF16 tensors: FP8 block-wise
+(128x128, FP32 scales), MXFP8 (1x32, UE8M0) and NVFP4 (1x16, E4M3 block
+scale + FP32 global scale), quantise / dequantise / fake-quantise.
+
+Formats as listed on "Low Precision RL" ("Choose a precision" table); NVFP4
+fake-quantisation with sibling-shared global amax and the straight-through
+backward as described in the verl NVFP4 QAT article (sections 2.3, 2.4).
+
+This module is argument marshalling only: every step runs in libpwq's CUDA
+kernels (include/pwq.h).  PyTorch supplies device memory and the stream.
+Functions take CUDA tensors ([M, N] or batched [B, M, N], last dimension
+contiguous) and return newly allocated outputs unless ``out=`` buffers are
+given.  Nothing synchronises.
+"""
+import ctypes
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+from ._lib import (LIB_PATH, PWQ_MAX_SIBLINGS, PwqError, PwqTensor, check, lib,  # noqa: F401
+                   status_string)
+
+__all__ = [
+    "fp8_block_quant", "fp8_block_dequant", "mxfp8_quant", "mxfp8_dequant",
+    "nvfp4_group_amax", "nvfp4_quant", "nvfp4_dequant", "nvfp4_fake_quant",
+    "nvfp4_workspace_size", "NVFP4FakeQuantSTE", "nvfp4_fake_quant_ste", "build_info",
+    "device_error", "PwqError", "LIB_PATH",
+]
+
+_CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _bmn(t: torch.Tensor, name: str):
+    if t.dim() == 2:
+        M, N = t.shape
+        return 1, M, N, M * t.stride(0), t.stride(0)
+    if t.dim() == 3:
+        B, M, N = t.shape
+        return B, M, N, t.stride(0), t.stride(1)
+    raise ValueError("%s must be 2-D [M, N] or 3-D [B, M, N], got shape %s" % (name, tuple(t.shape)))
+
+
+def _desc(t: torch.Tensor, name: str, packed: bool = False) -> PwqTensor:
+    """pwq_tensor for a [M, N] / [B, M, N] CUDA tensor.  For packed E2M1 codes
+    (uint8, two per byte) the logical column count is twice the byte count."""
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    B, M, N, bs, rs = _bmn(t, name)
+    if N > 1 and t.stride(-1) != 1:
+        raise ValueError("%s: last dimension must be contiguous" % name)
+    return PwqTensor(t.data_ptr(), B, M, 2 * N if packed else N, bs, rs)
+
+
+def _lead(x: torch.Tensor):
+    return tuple(x.shape[:-2]) if x.dim() == 3 else ()
+
+
+def _check_dtype(t, dtypes, name):
+    if t.dtype not in dtypes:
+        raise TypeError("%s must have dtype in %s, got %s" % (name, dtypes, t.dtype))
+
+
+# ---------------------------------------------------------------- FP8 block-wise
+
+def fp8_block_quant(x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """128x128 block-wise FP8: returns (codes float8_e4m3fn [.., M, N],
+    scale float32 [.., ceil(M/128), ceil(N/128)]) with s = fl(amax/448)."""
+    _check_dtype(x, (torch.bfloat16,), "x")
+    M, N = x.shape[-2:]
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    if scale is None:
+        scale = torch.empty(_lead(x) + (-(-M // 128), -(-N // 128)), dtype=torch.float32, device=x.device)
+    _check_dtype(out, _CODE_DTYPES, "out")
+    dx, dq = _desc(x, "x"), _desc(out, "out")
+    check(lib.fp8_block_quant(ctypes.byref(dx), ctypes.byref(dq), scale.data_ptr(), _stream(x)),
+          "fp8_block_quant")
+    return out, scale
+
+
+def fp8_block_dequant(q: torch.Tensor, scale: torch.Tensor,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """BF16 y = bf16(fl(dec(q) * s)) for FP8 block-wise codes and scales."""
+    _check_dtype(q, _CODE_DTYPES, "q")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if not scale.is_contiguous() or scale.dtype != torch.float32:
+        raise ValueError("scale must be a contiguous float32 tensor")
+    dq, dy = _desc(q, "q"), _desc(out, "out")
+    check(lib.fp8_block_dequant(ctypes.byref(dq), scale.data_ptr(), ctypes.byref(dy), _stream(q)),
+          "fp8_block_dequant")
+    return out
+
+
+# ---------------------------------------------------------------- MXFP8
+
+def mxfp8_quant(x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MXFP8 1x32: returns (codes float8_e4m3fn [.., M, N], UE8M0 scale bytes
+    uint8 [.., M, N/32])."""
+    _check_dtype(x, (torch.bfloat16,), "x")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    if scale is None:
+        scale = torch.empty(x.shape[:-1] + (x.shape[-1] // 32,), dtype=torch.uint8, device=x.device)
+    dx, dq = _desc(x, "x"), _desc(out, "out")
+    check(lib.mxfp8_quant(ctypes.byref(dx), ctypes.byref(dq), scale.data_ptr(), _stream(x)), "mxfp8_quant")
+    return out, scale
+
+
+def mxfp8_dequant(q: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _check_dtype(q, _CODE_DTYPES, "q")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if not scale.is_contiguous():
+        raise ValueError("scale must be contiguous")
+    dq, dy = _desc(q, "q"), _desc(out, "out")
+    check(lib.mxfp8_dequant(ctypes.byref(dq), scale.data_ptr(), ctypes.byref(dy), _stream(q)),
+          "mxfp8_dequant")
+    return out
+
+
+# ---------------------------------------------------------------- NVFP4
+
+def _siblings(xs) -> List[torch.Tensor]:
+    if isinstance(xs, torch.Tensor):
+        xs = [xs]
+    xs = list(xs)
+    if not 1 <= len(xs) <= PWQ_MAX_SIBLINGS:
+        raise ValueError("1..%d sibling tensors expected" % PWQ_MAX_SIBLINGS)
+    for i, x in enumerate(xs):
+        _check_dtype(x, (torch.bfloat16,), "x[%d]" % i)
+    return xs
+
+
+def _desc_array(ts, name, packed=False):
+    arr = (PwqTensor * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = _desc(t, "%s[%d]" % (name, i), packed)
+    return arr
+
+
+def _batch(x: torch.Tensor) -> int:
+    return x.shape[0] if x.dim() == 3 else 1
+
+
+def nvfp4_workspace_size(xs) -> int:
+    xs = _siblings(xs)
+    return int(lib.nvfp4_workspace_size(len(xs), _desc_array(xs, "x")))
+
+
+def _workspace(xs, arr) -> torch.Tensor:
+    n = int(lib.nvfp4_workspace_size(len(xs), arr))
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=xs[0].device)
+
+
+def nvfp4_group_amax(xs, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Group amax A_b = max |x| over all siblings' batch slice b, float32 [B].
+    This is the value to all-reduce (MAX) when a group is sharded."""
+    xs = _siblings(xs)
+    if out is None:
+        out = torch.empty(_batch(xs[0]), dtype=torch.float32, device=xs[0].device)
+    arr = _desc_array(xs, "x")
+    check(lib.nvfp4_group_amax(arr, len(xs), out.data_ptr(), _stream(xs[0])), "nvfp4_group_amax")
+    return out
+
+
+def nvfp4_quant(xs, amax: Optional[torch.Tensor] = None, out=None, sb=None,
+                global_scale: Optional[torch.Tensor] = None):
+    """NVFP4 quantisation of a sibling group (one tensor or a list sharing
+    one global amax per batch index).  Returns (packed codes list uint8
+    [.., M, N/2], block scales list float8_e4m3fn [.., M, N/16], global
+    scales float32 [B]).  ``amax`` (float32 [B]) replaces the on-device
+    group amax reduction (cached or all-reduced value)."""
+    single = isinstance(xs, torch.Tensor)
+    xs = _siblings(xs)
+    dev = xs[0].device
+    B = _batch(xs[0])
+    if out is None:
+        out = [torch.empty(x.shape[:-1] + (x.shape[-1] // 2,), dtype=torch.uint8, device=dev) for x in xs]
+    if sb is None:
+        sb = [torch.empty(x.shape[:-1] + (x.shape[-1] // 16,), dtype=torch.float8_e4m3fn, device=dev)
+              for x in xs]
+    if global_scale is None:
+        global_scale = torch.empty(B, dtype=torch.float32, device=dev)
+    for t in sb:
+        if not t.is_contiguous():
+            raise ValueError("block scale tensors must be contiguous")
+    ax = _desc_array(xs, "x")
+    aq = _desc_array(out, "out", packed=True)
+    sbp = (ctypes.c_void_p * len(xs))(*[t.data_ptr() for t in sb])
+    ws = None if amax is not None else _workspace(xs, ax)
+    check(lib.nvfp4_quant(ax, len(xs), aq, sbp, global_scale.data_ptr(),
+                          amax.data_ptr() if amax is not None else None,
+                          ws.data_ptr() if ws is not None else None,
+                          ws.numel() if ws is not None else 0, _stream(xs[0])), "nvfp4_quant")
+    if single:
+        return out[0], sb[0], global_scale
+    return out, sb, global_scale
+
+
+def nvfp4_dequant(packed: torch.Tensor, sb: torch.Tensor, global_scale: torch.Tensor,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """BF16 y = bf16(fl((dec(c) * dec(sb)) * gs)) for one NVFP4 tensor."""
+    _check_dtype(packed, (torch.uint8,), "packed")
+    if out is None:
+        out = torch.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=torch.bfloat16,
+                          device=packed.device)
+    if not sb.is_contiguous() or not global_scale.is_contiguous():
+        raise ValueError("sb and global_scale must be contiguous")
+    dq, dy = _desc(packed, "packed", packed=True), _desc(out, "out")
+    check(lib.nvfp4_dequant(ctypes.byref(dq), sb.data_ptr(), global_scale.data_ptr(), ctypes.byref(dy),
+                            _stream(packed)), "nvfp4_dequant")
+    return out
+
+
+def nvfp4_fake_quant(xs, amax: Optional[torch.Tensor] = None, out=None, inplace: bool = False,
+                     amax_out: Optional[torch.Tensor] = None):
+    """NVFP4 QDQ of a sibling group: BF16 outputs equal to
+    nvfp4_dequant(nvfp4_quant(x)), without materialising codes.  Returns the
+    output tensor (single input) or list of outputs."""
+    single = isinstance(xs, torch.Tensor)
+    xs = _siblings(xs)
+    if out is None:
+        out = xs if inplace else [torch.empty_like(x) for x in xs]
+    elif isinstance(out, torch.Tensor):
+        out = [out]
+    ax = _desc_array(xs, "x")
+    ay = _desc_array(out, "out")
+    ws = None if amax is not None else _workspace(xs, ax)
+    check(lib.nvfp4_fake_quant(ax, ay, len(xs), amax.data_ptr() if amax is not None else None,
+                               amax_out.data_ptr() if amax_out is not None else None,
+                               ws.data_ptr() if ws is not None else None,
+                               ws.numel() if ws is not None else 0, _stream(xs[0])), "nvfp4_fake_quant")
+    return out[0] if single else out
+
+
+class NVFP4FakeQuantSTE(torch.autograd.Function):
+    """Fake-quantised forward, straight-through backward: grad_x = grad_y and
+    no gradient for the amax (verl NVFP4 QAT article, section 2.3)."""
+
+    @staticmethod
+    def forward(ctx, x: torch.Tensor, amax: Optional[torch.Tensor] = None):
+        return nvfp4_fake_quant(x, amax=amax)
+
+    @staticmethod
+    def backward(ctx, grad_y):
+        return grad_y, None
+
+
+class _SiblingSTE(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, amax, *xs):
+        return tuple(nvfp4_fake_quant(list(xs), amax=amax))
+
+    @staticmethod
+    def backward(ctx, *grads):
+        return (None,) + tuple(grads)
+
+
+def nvfp4_fake_quant_ste(xs: Sequence[torch.Tensor], amax: Optional[torch.Tensor] = None):
+    """Sibling-group fake-quantisation with the straight-through backward."""
+    if isinstance(xs, torch.Tensor):
+        return NVFP4FakeQuantSTE.apply(xs, amax)
+    return list(_SiblingSTE.apply(amax, *xs))
+
+
+# ---------------------------------------------------------------- diagnostics
+
+def build_info() -> str:
+    return lib.pwq_build_info().decode()
+
+
+def device_error() -> int:
+    """Reads and clears the device-side error word (synchronous)."""
+    code = ctypes.c_uint32(0)
+    check(lib.pwq_device_error(ctypes.byref(code)), "pwq_device_error")
+    return int(code.value)

@@ -1,0 +1,322 @@
+// fp8_block.cu -- FP8 block-wise quantise / dequantise: 128x128 tiles, one
+// FP32 scale per tile (s = fl(amax / 448), the dequant multiplier), E4M3
+// codes.  Source: "Low Precision RL", "Choose a precision" table and
+// "Modes" 2 (DeepSeek-style 128x128 block-wise FP8 with FP32 scales);
+// "低精度训练与 Rollout", "FP8 训练 + FP8 Rollout" (FP32 block scales; FP8
+// weights dequantised to BF16 on weight update).
+//
+// Quantise: a persistent grid (2 CTAs per SM) walks the tiles.  Each tile is
+// brought into shared memory by one 3-D TMA box load (cp.async.bulk.tensor,
+// no multicast) whose out-of-range part is zero-filled -- zeros never raise
+// the amax, so ragged edge tiles need no masking on the load side.  A ring
+// of kStages tile buffers keeps the next tiles in flight while the current
+// one is reduced: every thread copies its 64 elements to registers, the CTA
+// reduces the tile amax (shuffles + one barrier), the freed buffer is
+// immediately refilled, and the codes are computed from registers with one
+// correctly rounded reciprocal per tile plus an FMA residual correction per
+// element (proved equal to IEEE division by the exhaustive self-test).
+#include <algorithm>
+#include <cuda.h>
+
+#include "pwq_internal.h"
+
+namespace pwq {
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kThreads = 256;
+constexpr int kStages = 3;
+constexpr int kTileBytes = kTile * kTile * 2;  // BF16
+constexpr int kChunksPerThread = kTile * kTile / 8 / kThreads;  // 8
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Device-side error word of this library (bit kErrTmaTimeout: a TMA wait
+// gave up).  Read and cleared by pwq_device_error().
+__device__ uint32_t g_device_error = 0u;
+
+struct QuantArgs {
+    char* q;
+    int64_t q_bs, q_rs;   // bytes
+    float* scale;         // dense [B][TM][TN]
+    int rows, cols;
+    int tiles_m, tiles_n;
+    uint32_t total_tiles;
+};
+
+__device__ __forceinline__ void tile_coords(uint32_t t, const QuantArgs& a, int& b, int& tm, int& tn) {
+    const uint32_t per_b = (uint32_t)a.tiles_m * (uint32_t)a.tiles_n;
+    b = (int)(t / per_b);
+    const uint32_t rem = t - (uint32_t)b * per_b;
+    tm = (int)(rem / (uint32_t)a.tiles_n);
+    tn = (int)(rem - (uint32_t)tm * (uint32_t)a.tiles_n);
+}
+
+__device__ __forceinline__ void issue_tile(const CUtensorMap* tmap, uint32_t dst, uint32_t bar, uint32_t t,
+                                           const QuantArgs& a) {
+    int b, tm, tn;
+    tile_coords(t, a, b, tm, tn);
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    tma_load_3d(dst, tmap, bar, tn * kTile, tm * kTile, b);
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    __shared__ __align__(8) uint64_t bars[kStages];
+    __shared__ uint32_t red[2][kThreads / 32];
+
+    const uint32_t tid = threadIdx.x;
+    // the ring starts at the first 1024-byte boundary of dynamic shared memory
+    const uint32_t pad = (1024u - (smem_addr(smem) & 1023u)) & 1023u;
+    unsigned char* ring = smem + pad;
+    const uint32_t smem0 = smem_addr(ring);
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const uint32_t first = blockIdx.x, step = gridDim.x;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            const uint32_t t = first + (uint32_t)s * step;
+            if (t < a.total_tiles) issue_tile(&tmap, smem0 + s * kTileBytes, smem_addr(&bars[s]), t, a);
+        }
+    }
+
+    // thread -> (row, 16-byte column chunk) pairs: chunk j covers row
+    // (tid >> 4) + 16 j, columns (tid & 15) * 8 .. + 7
+    const int ccol = (int)(tid & 15u) * 8;
+    const int row0 = (int)(tid >> 4);
+
+    uint32_t it = 0;
+    for (uint32_t t = first; t < a.total_tiles; t += step, ++it) {
+        const uint32_t s = it % kStages;
+        const uint32_t parity = (it / kStages) & 1u;
+        const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity, kWaitLimitNs);
+        const unsigned char* buf = ring + s * kTileBytes;
+        uint4 v[kChunksPerThread];
+        uint32_t m = 0u;
+#pragma unroll
+        for (int j = 0; j < kChunksPerThread; ++j) {
+            v[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (ok) v[j] = *reinterpret_cast<const uint4*>(buf + (row0 + 16 * j) * (kTile * 2) + ccol * 2);
+            m = max(m, amax_bits8(v[j]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((tid & 31u) == 0u) red[it & 1u][tid >> 5] = m;
+        // one barrier: publishes the warp maxima, ends every read of buffer
+        // s, and makes a timed-out wait a CTA-uniform decision
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_device_error, kErrTmaTimeout);
+                // let every issued copy land before shared memory is released
+                for (uint32_t k = 0; k < (uint32_t)kStages; ++k) {
+                    if (t + k * step < a.total_tiles)
+                        (void)mbar_wait_bounded(smem_addr(&bars[(it + k) % kStages]),
+                                                ((it + k) / kStages) & 1u, kWaitLimitNs);
+                }
+            }
+            return;
+        }
+        if (tid == 0) {
+            const uint32_t tn = t + (uint32_t)kStages * step;
+            if (tn < a.total_tiles) issue_tile(&tmap, smem0 + s * kTileBytes, smem_addr(&bars[s]), tn, a);
+        }
+        uint32_t am = red[it & 1u][0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) am = max(am, red[it & 1u][w]);
+
+        const float amax = __uint_as_float(am << 16);
+        const float sc = __fdiv_rn(amax, 448.0f);
+        const float rc = __frcp_rn(sc);
+        const bool fast = div_fast_ok(sc, rc);
+
+        int b, tm, tn;
+        tile_coords(t, a, b, tm, tn);
+        if (tid == 0) a.scale[t] = sc;
+        const int rows_here = min(kTile, a.rows - tm * kTile);
+        const int cols_here = min(kTile, a.cols - tn * kTile);
+        char* qtile = a.q + (int64_t)b * a.q_bs + (int64_t)tm * kTile * a.q_rs + (int64_t)tn * kTile;
+#pragma unroll
+        for (int j = 0; j < kChunksPerThread; ++j) {
+            const int r = row0 + 16 * j;
+            uint2 out;
+            out.x = e4m3x4(quotient(bf16_lo(v[j].x), sc, rc, fast), quotient(bf16_hi(v[j].x), sc, rc, fast),
+                           quotient(bf16_lo(v[j].y), sc, rc, fast), quotient(bf16_hi(v[j].y), sc, rc, fast));
+            out.y = e4m3x4(quotient(bf16_lo(v[j].z), sc, rc, fast), quotient(bf16_hi(v[j].z), sc, rc, fast),
+                           quotient(bf16_lo(v[j].w), sc, rc, fast), quotient(bf16_hi(v[j].w), sc, rc, fast));
+            if (r < rows_here) {
+                char* dst = qtile + (int64_t)r * a.q_rs + ccol;
+                if (ccol + 8 <= cols_here) {
+                    st_v2(dst, out);
+                } else if (ccol < cols_here) {
+                    for (int e = 0; e < cols_here - ccol; ++e)
+                        dst[e] = (char)((e < 4 ? out.x >> (8 * e) : out.y >> (8 * (e - 4))) & 0xffu);
+                }
+            }
+        }
+    }
+}
+
+// Dequantise: 8 codes (8 bytes) -> 8 BF16 (16 bytes) per chunk; the
+// chunk's tile scale is a cached 4-byte load.  Ragged row tails (cols not a
+// multiple of 8) take a byte-wise path.
+struct DequantArgs {
+    const char* q;
+    char* y;
+    const float* scale;
+    int64_t q_bs, q_rs, y_bs, y_rs;
+    FastDiv cpr;      // chunks per row, ceil(N / 8)
+    FastDiv rows;     // M
+    int cols, tiles_m, tiles_n;
+    uint32_t total;
+};
+
+constexpr int kDqUnroll = 4;
+
+__global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const DequantArgs a) {
+    const uint32_t stride = gridDim.x * blockDim.x;
+    for (uint32_t base = blockIdx.x * blockDim.x + threadIdx.x; base < a.total;
+         base += stride * kDqUnroll) {
+        uint2 v[kDqUnroll];
+        float sc[kDqUnroll];
+        char* yp[kDqUnroll];
+        int nvalid[kDqUnroll];
+#pragma unroll
+        for (int u = 0; u < kDqUnroll; ++u) {
+            const uint32_t c = base + u * stride;
+            const uint32_t r = fdiv(c, a.cpr);
+            const int col = (int)(c - r * a.cpr.d) * 8;
+            const uint32_t b = fdiv(r, a.rows);
+            const int mrow = (int)(r - b * a.rows.d);
+            const char* qp = a.q + (int64_t)b * a.q_bs + (int64_t)mrow * a.q_rs + col;
+            yp[u] = a.y + (int64_t)b * a.y_bs + (int64_t)mrow * a.y_rs + (int64_t)col * 2;
+            nvalid[u] = (c < a.total) ? min(8, a.cols - col) : 0;
+            v[u] = make_uint2(0u, 0u);
+            sc[u] = 0.0f;
+            if (nvalid[u] > 0) {
+                sc[u] = __ldg(a.scale + ((int64_t)b * a.tiles_m + (mrow >> 7)) * a.tiles_n + (col >> 7));
+                if (nvalid[u] == 8) {
+                    v[u] = ld_stream_v2(qp);
+                } else {
+                    uint32_t w[2] = {0u, 0u};
+                    for (int e = 0; e < nvalid[u]; ++e)
+                        w[e >> 2] |= (uint32_t)(unsigned char)qp[e] << (8 * (e & 3));
+                    v[u] = make_uint2(w[0], w[1]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kDqUnroll; ++u) {
+            if (nvalid[u] <= 0) continue;
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const uint32_t pair = ((h < 2 ? v[u].x : v[u].y) >> (16 * (h & 1))) & 0xffffu;
+                const float2 f = e4m3x2_decode(pair);
+                w[h] = pack_bf16x2(__fmul_rn(f.x, sc[u]), __fmul_rn(f.y, sc[u]));
+            }
+            if (nvalid[u] == 8) {
+                st_v4(yp[u], make_uint4(w[0], w[1], w[2], w[3]));
+            } else {
+                unsigned short* y16 = reinterpret_cast<unsigned short*>(yp[u]);
+                for (int e = 0; e < nvalid[u]; ++e)
+                    y16[e] = (unsigned short)((w[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+            }
+        }
+    }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+}  // namespace
+
+cudaError_t read_and_clear_device_error(uint32_t* code) {
+    uint32_t zero = 0u;
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_device_error, sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t));
+}
+
+cudaError_t launch_fp8_block_quant(const View& x, const View& q, float* scale, cudaStream_t s) {
+    EncodeTiledFn encode = encode_tiled_fn();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap tmap;
+    const cuuint64_t dims[3] = {(cuuint64_t)x.cols, (cuuint64_t)x.rows, (cuuint64_t)x.batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)x.rstride,
+                                   (cuuint64_t)(x.batch > 1 ? x.bstride : x.rows * x.rstride)};
+    const cuuint32_t box[3] = {kTile, kTile, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x.ptr, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+    QuantArgs a;
+    a.q = q.ptr;
+    a.q_bs = q.bstride;
+    a.q_rs = q.rstride;
+    a.scale = scale;
+    a.rows = (int)x.rows;
+    a.cols = (int)x.cols;
+    a.tiles_m = (int)((x.rows + kTile - 1) / kTile);
+    a.tiles_n = (int)((x.cols + kTile - 1) / kTile);
+    a.total_tiles = (uint32_t)(x.batch * a.tiles_m * a.tiles_n);
+
+    const size_t smem = (size_t)kStages * kTileBytes + 1024;
+    static int configured[64] = {0};
+    const int dev = current_device();
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(fp8_block_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        configured[dev] = 1;
+    }
+    const int grid = (int)std::min<int64_t>(a.total_tiles, (int64_t)sm_count(dev) * 2);
+    fp8_block_quant_kernel<<<grid, kThreads, smem, s>>>(tmap, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_block_dequant(const View& q, const float* scale, const View& y, cudaStream_t s) {
+    DequantArgs a;
+    a.q = q.ptr;
+    a.y = y.ptr;
+    a.scale = scale;
+    a.q_bs = q.bstride;
+    a.q_rs = q.rstride;
+    a.y_bs = y.bstride;
+    a.y_rs = y.rstride;
+    const int64_t cpr = (q.cols + 7) / 8;
+    a.cpr = make_fastdiv((uint32_t)cpr);
+    a.rows = make_fastdiv((uint32_t)q.rows);
+    a.cols = (int)q.cols;
+    a.tiles_m = (int)((q.rows + kTile - 1) / kTile);
+    a.tiles_n = (int)((q.cols + kTile - 1) / kTile);
+    a.total = (uint32_t)(q.batch * q.rows * cpr);
+    const int64_t span = int64_t(kThreads) * kDqUnroll;
+    const int grid = persistent_grid((a.total + span - 1) / span, 8);
+    fp8_block_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace pwq

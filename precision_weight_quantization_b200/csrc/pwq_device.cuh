@@ -1,0 +1,257 @@
+// pwq_device.cuh -- device helpers shared by the libpwq kernels (sm_100a).
+//
+// Conversions use the sm_100a hardware converters:
+//   cvt.rn.satfinite.e4m3x2.f32   binary32 pair -> two E4M3 bytes (RNE, saturating)
+//   cvt.rn.satfinite.e2m1x2.f32   binary32 pair -> two E2M1 nibbles (RNE, saturating)
+//   cvt.rn.f16x2.e4m3x2 / .e2m1x2 exact decode to binary16
+//   cvt.rn.bf16x2.f32             binary32 pair -> BF16 pair (RNE, subnormals kept)
+// Their rounding, saturation and sign-of-zero behaviour is checked against
+// the CPU oracle over whole input ranges by the codec self-test.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace pwq {
+
+// ---------------------------------------------------------------- BF16 lanes
+
+// Low / high BF16 of a packed 32-bit word, widened exactly to binary32.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Max of |x| over the 8 BF16 values of a 16-byte chunk, as BF16 magnitude
+// bits.  For finite values the magnitude order equals the unsigned order of
+// the low 15 bits, so the max is two SIMD halfword maxes.
+__device__ __forceinline__ uint32_t amax_bits8(uint4 v) {
+    const uint32_t m = 0x7fff7fffu;
+    uint32_t a = __vmaxu2(v.x & m, v.y & m);
+    uint32_t b = __vmaxu2(v.z & m, v.w & m);
+    uint32_t c = __vmaxu2(a, b);
+    return max(c & 0xffffu, c >> 16);
+}
+
+// Pack two binary32 into a BF16x2 word (lo in bits 0..15), RNE.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---------------------------------------------------------------- E4M3
+
+// Two binary32 -> two E4M3 codes in a 16-bit value (lo in bits 0..7).
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Four binary32 -> four E4M3 codes in a 32-bit word (element 0 in byte 0).
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+    return e4m3x2(a, b) | (e4m3x2(c, d) << 16);
+}
+
+// Two E4M3 codes (lo in bits 0..7) -> exact binary32 values.
+__device__ __forceinline__ float2 e4m3x2_decode(uint32_t codes16) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)codes16));
+    float2 f;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(f.x) : "h"((unsigned short)(h2 & 0xffffu)));
+    asm("cvt.f32.f16 %0, %1;" : "=f"(f.y) : "h"((unsigned short)(h2 >> 16)));
+    return f;
+}
+
+// One E4M3 code -> exact binary32 value.
+__device__ __forceinline__ float e4m3_decode(uint32_t code) { return e4m3x2_decode(code & 0xffu).x; }
+
+// ---------------------------------------------------------------- E2M1
+
+// Two binary32 -> one byte of two E2M1 codes (lo element in bits 0..3).
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Byte of two E2M1 codes -> two exact binary32 values (lo nibble first).
+__device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}" : "=r"(h2) : "r"(byte));
+    float2 f;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(f.x) : "h"((unsigned short)(h2 & 0xffffu)));
+    asm("cvt.f32.f16 %0, %1;" : "=f"(f.y) : "h"((unsigned short)(h2 >> 16)));
+    return f;
+}
+
+// ---------------------------------------------------------------- division
+
+// Correctly rounded binary32 quotient x / s from the correctly rounded
+// reciprocal r = RN(1/s): one product and one residual correction with
+// fused multiply-adds (Markstein's correction step; P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990).  The caller uses it only when
+// `div_fast_ok(s, r)` holds; over every BF16 numerator and every divisor the
+// formats produce, its results are checked bit for bit against __fdiv_rn by
+// pwq_selftest_division.
+__device__ __forceinline__ float div_rcp_correct(float x, float s, float r) {
+    float q0 = __fmul_rn(x, r);
+    float res = __fmaf_rn(-q0, s, x);
+    return __fmaf_rn(res, r, q0);
+}
+
+// The fast quotient is used only when the divisor and its reciprocal are
+// both normal binary32 numbers (exponent field in 1..254).
+__device__ __forceinline__ bool div_fast_ok(float s, float r) {
+    uint32_t es = (__float_as_uint(s) >> 23) & 0xffu;
+    uint32_t er = (__float_as_uint(r) >> 23) & 0xffu;
+    return (es - 1u) < 254u && (er - 1u) < 254u;
+}
+
+// fl(x / s) with the zero-scale reading: s == 0 gives a zero of x's sign.
+__device__ __forceinline__ float quotient(float x, float s, float r, bool fast) {
+    if (fast) return div_rcp_correct(x, s, r);
+    if (s == 0.0f) return __uint_as_float(__float_as_uint(x) & 0x80000000u);
+    return __fdiv_rn(x, s);
+}
+
+// ---------------------------------------------------------------- UE8M0
+
+// e = min{k : amax <= 448 * 2^k} from the BF16 magnitude bits of amax,
+// clamped to [-127, 127] (amax = 0 gives -127).  With amax = sig * 2^(E-msb)
+// and sig an integer whose top bit is bit msb: 448 * 2^(E-8) = 1.75 * 2^E,
+// so e = E - 8 when sig <= 1.75 * 2^msb and E - 7 otherwise.
+__device__ __forceinline__ int ue8m0_exponent(uint32_t amax_bits16) {
+    if (amax_bits16 == 0u) return -127;
+    uint32_t ef = amax_bits16 >> 7, mant = amax_bits16 & 0x7fu;
+    uint32_t sig = ef ? (0x80u | mant) : mant;
+    int msb = 31 - __clz(sig);
+    int E = (int)(ef ? ef : 1u) - 127 - 7 + msb;
+    int e = E - 8 + ((4u * sig <= (7u << msb)) ? 0 : 1);
+    return max(-127, min(127, e));
+}
+
+// 2^k as binary32 for k in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float exp2i(int k) {
+    return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// ---------------------------------------------------------------- loads / stores
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void st_v2(void* p, uint2 v) {
+    asm volatile("st.global.v2.u32 [%0], {%1, %2};" :: "l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+__device__ __forceinline__ void st_u32(void* p, uint32_t v) {
+    asm volatile("st.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+// ---------------------------------------------------------------- fast division by a constant
+
+// Unsigned 32-bit division by a runtime constant d >= 1 (round-up magic
+// multiplier; T. Granlund and P. Montgomery, "Division by invariant integers
+// using multiplication", PLDI 1994): q = (umulhi(n, m) + n) >> l with
+// l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1.
+struct FastDiv {
+    uint32_t d, m, l;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+    FastDiv f;
+    f.d = d;
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    f.l = l;
+    f.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+    uint32_t t = __umulhi(n, f.m);
+    return (uint32_t)(((uint64_t)t + n) >> f.l);
+}
+
+// ---------------------------------------------------------------- device error word
+
+// Bits of the device error word set by kernels whose bounded waits give up.
+constexpr uint32_t kErrTmaTimeout = 1u;
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- mbarrier / TMA
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    return done != 0;
+}
+
+// Waits for the phase with the given parity to complete; gives up after
+// `limit_ns` nanoseconds of wall time and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// 3-D tiled TMA load (no multicast) of the box at (x, y, z) into shared
+// memory, completing `bar`'s transaction count.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar,
+                                           int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        :: "r"(dst), "l"(tmap), "r"(bar), "r"(x), "r"(y), "r"(z) : "memory");
+}
+
+}  // namespace pwq

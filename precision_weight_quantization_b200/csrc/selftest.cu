@@ -1,0 +1,98 @@
+// selftest.cu -- exhaustive checks of the device arithmetic the kernels use.
+//
+// Division: the quantisers replace the per-element IEEE division by one
+// correctly rounded reciprocal per tile/block and an FMA residual correction
+// (pwq_device.cuh).  The numerators are BF16 values and the divisors come
+// from small finite sets (FP8 block-wise: fl(a / 448); NVFP4:
+// fl(dec(sb) * fl(a / 2688)), a a positive BF16, sb a non-zero E4M3 code), so
+// every (numerator, divisor) pair can be enumerated and compared with CUDA's
+// IEEE division __fdiv_rn in well under a second.
+//
+// Codecs: writes the hardware conversions of a range of binary32 inputs so
+// the host can compare them with the CPU oracle.
+#include "pwq_internal.h"
+
+namespace pwq {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ bool bf16_is_finite(uint32_t b) { return ((b >> 7) & 0xffu) != 0xffu; }
+
+// One divisor per CTA; every finite BF16 numerator.
+template <int kWhich>
+__global__ void __launch_bounds__(kThreads) selftest_division_kernel(unsigned long long* counts) {
+    float d;
+    if (kWhich == 0) {
+        const uint32_t a = blockIdx.x + 1u;            // positive finite BF16 0x0001..0x7f7f
+        d = __fdiv_rn(__uint_as_float(a << 16), 448.0f);
+    } else {
+        const uint32_t a = blockIdx.x + 1u;
+        const uint32_t sb = blockIdx.y + 1u;           // E4M3 0x01..0x7e
+        const float gs = __fdiv_rn(__uint_as_float(a << 16), 2688.0f);
+        d = __fmul_rn(e4m3_decode(sb), gs);
+    }
+    const float r = __frcp_rn(d);
+    const bool fast = div_fast_ok(d, r);
+    unsigned long long n = 0, code_bad = 0, quot_bad = 0;
+    for (uint32_t xb = threadIdx.x; xb < 65536u; xb += kThreads) {
+        if (!bf16_is_finite(xb)) continue;
+        const float x = __uint_as_float(xb << 16);
+        const float qf = quotient(x, d, r, fast);
+        const float qr = (d == 0.0f) ? __uint_as_float((xb << 16) & 0x80000000u) : __fdiv_rn(x, d);
+        ++n;
+        if (kWhich == 0) {
+            code_bad += (e4m3x2(qf, 0.0f) & 0xffu) != (e4m3x2(qr, 0.0f) & 0xffu);
+            const uint32_t ef = (__float_as_uint(qr) >> 23) & 0xffu;
+            if (ef != 0u) quot_bad += __float_as_uint(qf) != __float_as_uint(qr);
+        } else {
+            code_bad += (e2m1x2(qf, 0.0f) & 0xfu) != (e2m1x2(qr, 0.0f) & 0xfu);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n += __shfl_xor_sync(0xffffffffu, n, o);
+        code_bad += __shfl_xor_sync(0xffffffffu, code_bad, o);
+        quot_bad += __shfl_xor_sync(0xffffffffu, quot_bad, o);
+    }
+    if ((threadIdx.x & 31u) == 0u) {
+        atomicAdd(counts + 0, n);
+        atomicAdd(counts + 1, code_bad);
+        atomicAdd(counts + 2, quot_bad);
+        if (!fast) atomicAdd(counts + 3, n);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+selftest_codecs_kernel(uint32_t first, uint32_t count, uint8_t* e4m3, uint8_t* e2m1, uint16_t* bf16) {
+    const uint32_t stride = gridDim.x * blockDim.x;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride) {
+        const float f = __uint_as_float(first + i);
+        if (e4m3) e4m3[i] = (uint8_t)(e4m3x2(f, 0.0f) & 0xffu);
+        if (e2m1) e2m1[i] = (uint8_t)(e2m1x2(f, 0.0f) & 0xfu);
+        if (bf16) bf16[i] = (uint16_t)(pack_bf16x2(f, 0.0f) & 0xffffu);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_selftest_division(int which, unsigned long long* counts, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(counts, 0, 4 * sizeof(unsigned long long), s);
+    if (e != cudaSuccess) return e;
+    if (which == 0) {
+        selftest_division_kernel<0><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
+    } else {
+        selftest_division_kernel<1><<<dim3(0x7f7f, 0x7e), kThreads, 0, s>>>(counts);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_codecs(uint32_t first, uint32_t count, uint8_t* e4m3, uint8_t* e2m1,
+                                   uint16_t* bf16, cudaStream_t s) {
+    if (count == 0) return cudaSuccess;
+    const int grid = persistent_grid((count + kThreads - 1) / kThreads, 8);
+    selftest_codecs_kernel<<<grid, kThreads, 0, s>>>(first, count, e4m3, e2m1, bf16);
+    return cudaGetLastError();
+}
+
+}  // namespace pwq

@@ -1,0 +1,149 @@
+"""C ABI boundary tests that need no GPU: the shared library loads, exports
+every function include/pwq.h declares, reports its exact-math build, and
+rejects bad arguments with the documented status before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pwq.h")
+
+
+def _lib():
+    from precision_weight_quantization_b200 import build
+    build.build()
+    import precision_weight_quantization_b200._lib as L
+    return L
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_header_declares_the_named_entry_points():
+    names = declared_functions()
+    for n in ["fp8_block_quant", "fp8_block_dequant", "mxfp8_quant", "mxfp8_dequant",
+              "nvfp4_quant", "nvfp4_dequant", "nvfp4_fake_quant", "nvfp4_group_amax",
+              "nvfp4_workspace_size", "pwq_status_string", "pwq_build_info"]:
+        assert n in names, n
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib()
+    raw = ctypes.CDLL(L.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(raw, n)]
+    assert not missing, missing
+
+
+def test_build_is_exact_math():
+    L = _lib()
+    info = L.lib.pwq_build_info().decode()
+    assert "sm_100a" in info
+    for flag in ("-ftz=false", "-prec-div=true", "-prec-sqrt=true", "-fmad=false"):
+        assert flag in info
+    assert "no --use_fast_math" in info
+
+
+def test_status_strings():
+    L = _lib()
+    assert L.status_string(0) == "PWQ_OK"
+    assert L.status_string(L.PWQ_ERR_OVERLAP) == "PWQ_ERR_OVERLAP"
+    assert L.status_string(99) == "PWQ_ERR_UNKNOWN"
+
+
+def T(L, ptr, b, m, n, bs, rs):
+    return L.PwqTensor(ptr, b, m, n, bs, rs)
+
+
+def test_validation_errors_without_gpu():
+    L = _lib()
+    lib = L.lib
+    by = ctypes.byref
+    base = 1 << 40                       # never dereferenced: validation fails first
+    x = T(L, base, 1, 256, 512, 256 * 512, 512)
+    q = T(L, base + (1 << 30), 1, 256, 512, 256 * 512, 512)
+    s = base + (1 << 31)
+    # null descriptors and pointers
+    assert lib.fp8_block_quant(None, by(q), s, None) == L.PWQ_ERR_NULL
+    assert lib.fp8_block_quant(by(x), by(q), None, None) == L.PWQ_ERR_NULL
+    xn = T(L, None, 1, 256, 512, 256 * 512, 512)
+    assert lib.fp8_block_quant(by(xn), by(q), s, None) == L.PWQ_ERR_NULL
+    # alignment
+    xa = T(L, base + 8, 1, 256, 512, 256 * 512, 512)
+    assert lib.fp8_block_quant(by(xa), by(q), s, None) == L.PWQ_ERR_ALIGN
+    xr = T(L, base, 1, 256, 512, 256 * 516, 516)          # 1032-byte rows: not 16-aligned
+    assert lib.fp8_block_quant(by(xr), by(q), s, None) == L.PWQ_ERR_ALIGN
+    assert lib.fp8_block_quant(by(x), by(q), s + 2, None) == L.PWQ_ERR_ALIGN
+    # stride too small
+    xs = T(L, base, 1, 256, 512, 256 * 256, 256)
+    assert lib.fp8_block_quant(by(xs), by(q), s, None) == L.PWQ_ERR_STRIDE
+    xb = T(L, base, 2, 256, 512, 100 * 512, 512)
+    qb = T(L, base + (1 << 30), 2, 256, 512, 256 * 512, 512)
+    assert lib.fp8_block_quant(by(xb), by(qb), s, None) == L.PWQ_ERR_STRIDE
+    # shape mismatch, negative extents
+    q2 = T(L, base + (1 << 30), 1, 128, 512, 128 * 512, 512)
+    assert lib.fp8_block_quant(by(x), by(q2), s, None) == L.PWQ_ERR_SHAPE
+    xneg = T(L, base, 1, -1, 512, 0, 512)
+    assert lib.fp8_block_quant(by(xneg), by(xneg), s, None) == L.PWQ_ERR_SHAPE
+    # overlap: codes written over the input, scales written over the codes
+    qo = T(L, base + 4096, 1, 256, 512, 256 * 512, 512)
+    assert lib.fp8_block_quant(by(x), by(qo), s, None) == L.PWQ_ERR_OVERLAP
+    assert lib.fp8_block_quant(by(x), by(q), base + (1 << 30) + 64, None) == L.PWQ_ERR_OVERLAP
+    # MXFP8 / NVFP4 divisibility
+    x33 = T(L, base, 1, 4, 48, 4 * 48, 48)
+    q33 = T(L, base + (1 << 30), 1, 4, 48, 4 * 48, 48)
+    assert lib.mxfp8_quant(by(x33), by(q33), s, None) == L.PWQ_ERR_SHAPE
+    x24 = T(L, base, 1, 4, 24, 4 * 24, 24)
+    assert lib.nvfp4_group_amax(by(x24), 1, s, None) == L.PWQ_ERR_SHAPE
+    # empty tensors are a no-op that succeeds (no CUDA call is made)
+    xe = T(L, None, 1, 0, 512, 0, 512)
+    assert lib.fp8_block_quant(by(xe), by(xe), None, None) == L.PWQ_OK
+    assert lib.mxfp8_quant(by(xe), by(xe), None, None) == L.PWQ_OK
+
+
+def test_nvfp4_validation_without_gpu():
+    L = _lib()
+    lib = L.lib
+    base = 1 << 40
+    xs = (L.PwqTensor * 2)(T(L, base, 1, 64, 256, 64 * 256, 256),
+                           T(L, base + (1 << 24), 1, 32, 256, 32 * 256, 256))
+    qs = (L.PwqTensor * 2)(T(L, base + (1 << 30), 1, 64, 256, 64 * 128, 128),
+                           T(L, base + (1 << 30) + (1 << 24), 1, 32, 256, 32 * 128, 128))
+    sb = (ctypes.c_void_p * 2)(base + (2 << 30), base + (2 << 30) + (1 << 24))
+    gs = base + (3 << 30)
+    ws = base + (4 << 30)
+    assert lib.nvfp4_workspace_size(2, xs) == 256
+    # sibling count
+    assert lib.nvfp4_quant(xs, 0, qs, sb, gs, None, ws, 256, None) == L.PWQ_ERR_ARG
+    assert lib.nvfp4_quant(xs, 9, qs, sb, gs, None, ws, 256, None) == L.PWQ_ERR_ARG
+    # workspace required without amax_in
+    assert lib.nvfp4_quant(xs, 2, qs, sb, gs, None, None, 0, None) == L.PWQ_ERR_WORKSPACE
+    assert lib.nvfp4_quant(xs, 2, qs, sb, gs, None, ws, 2, None) == L.PWQ_ERR_WORKSPACE
+    # batch mismatch between siblings
+    xm = (L.PwqTensor * 2)(xs[0], T(L, base + (1 << 24), 2, 32, 256, 32 * 256, 256))
+    assert lib.nvfp4_quant(xm, 2, qs, sb, gs, None, ws, 256, None) == L.PWQ_ERR_ARG
+    # fake-quant: exact alias allowed (validation passes to the launch), partial overlap not
+    ys = (L.PwqTensor * 2)(T(L, base + 32, 1, 64, 256, 64 * 256, 256), xs[1])
+    assert lib.nvfp4_fake_quant(xs, ys, 2, None, None, ws, 256, None) == L.PWQ_ERR_OVERLAP
+    xe = (L.PwqTensor * 2)(xs[0], T(L, base + (1 << 24), 1, 64, 256, 64 * 256, 256))
+    ys2 = (L.PwqTensor * 2)(xe[1], xe[0])                # outputs swapped onto the other input
+    assert lib.nvfp4_fake_quant(xe, ys2, 2, None, None, ws, 256, None) == L.PWQ_ERR_OVERLAP
+    assert lib.nvfp4_fake_quant(xe, xe, 2, None, None, xs[0].ptr + 64, 256, None) == L.PWQ_ERR_OVERLAP
+    # overlap of the block scales with an input
+    sbo = (ctypes.c_void_p * 2)(base + 64, base + (2 << 30) + (1 << 24))
+    assert lib.nvfp4_quant(xs, 2, qs, sbo, gs, None, ws, 256, None) == L.PWQ_ERR_OVERLAP
+
+
+def test_python_binding_names_match_the_abi():
+    import precision_weight_quantization_b200 as P
+    for n in ["fp8_block_quant", "fp8_block_dequant", "mxfp8_quant", "mxfp8_dequant", "nvfp4_quant",
+              "nvfp4_dequant", "nvfp4_fake_quant", "nvfp4_group_amax", "nvfp4_workspace_size"]:
+        assert callable(getattr(P, n))
+    with pytest.raises(ValueError):
+        import torch
+        P.fp8_block_quant(torch.zeros(4, 4, dtype=torch.bfloat16))    # CPU tensor refused
