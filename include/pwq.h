@@ -27,10 +27,11 @@
  * buffer, including outputs and workspace; the library allocates nothing,
  * keeps no state between calls and never synchronises.
  *
- * Alignment.  Base pointers of BF16 / code / packed tensors must be 16-byte
- * aligned and their row and batch strides multiples of 16 bytes, else
- * PWQ_ERR_ALIGN (there is no unaligned slow path).  Scale arrays are dense
- * (layouts below) and need only their natural alignment.
+ * Alignment.  BF16 tensors: base pointer 16-byte aligned, row and batch
+ * strides multiples of 16 bytes.  E4M3 code and packed E2M1 tensors: base
+ * pointer and strides multiples of 8 bytes.  Otherwise PWQ_ERR_ALIGN (there
+ * is no unaligned slow path).  Scale arrays are dense (layouts below) and
+ * need only their natural alignment.
  *
  * Streams.  Every call enqueues its kernels on `stream` (NULL = the legacy
  * default stream) and returns; the status covers host-side validation and
@@ -67,7 +68,7 @@ typedef struct CUstream_st* pwq_stream_t;
 typedef enum pwq_status {
     PWQ_OK = 0,
     PWQ_ERR_NULL = 1,      /* a required pointer is NULL */
-    PWQ_ERR_ALIGN = 2,     /* base pointer or stride not 16-byte aligned */
+    PWQ_ERR_ALIGN = 2,     /* base pointer or stride not aligned as stated below */
     PWQ_ERR_SHAPE = 3,     /* negative extent, mismatched shapes, cols % 32 (MXFP8) or % 16 (NVFP4) != 0 */
     PWQ_ERR_STRIDE = 4,    /* row stride < row length, or batch stride < rows * row stride */
     PWQ_ERR_OVERLAP = 5,   /* an output overlaps an input or another output */
@@ -245,21 +246,21 @@ const char* pwq_build_info(void);
 pwq_status pwq_device_error(uint32_t* code);
 
 /* Exhaustive self-check of the device arithmetic against CUDA's IEEE
- * division (__fdiv_rn), for every BF16 numerator x and every divisor the
- * formats can produce:
- *   which = 0  FP8 block: divisors s = fl(a / 448), a every positive BF16;
- *              compares e4m3 codes and binary32 quotients.
+ * division (__fdiv_rn), for every divisor the formats can produce and every
+ * finite BF16 numerator that can be paired with it:
+ *   which = 0  FP8 block: divisors s = fl(a / 448), a every positive finite
+ *              BF16; numerators |x| <= a.  Compares E4M3 codes.
  *   which = 1  NVFP4: divisors d = fl(dec(sb) * fl(a / 2688)) for every
- *              positive BF16 a and every non-zero E4M3 sb; compares e2m1
- *              codes.
+ *              positive finite BF16 a and every non-zero E4M3 sb;
+ *              numerators |x| <= 16 d.  Compares E2M1 codes.
  * counts (device, 4 x uint64, zeroed by the call): [0] pairs checked,
- * [1] code mismatches, [2] binary32 quotient mismatches (which = 0 only,
- * where the quotient is a normal number), [3] pairs that took the
- * division fallback.  Asynchronous on `stream`. */
+ * [1] code mismatches, [2] binary32 quotient mismatches where the IEEE
+ * quotient is a normal number, [3] pairs that took the IEEE-division
+ * fallback instead of the reciprocal path.  Asynchronous on `stream`. */
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream);
 
-/* Runs the device codecs over 2^32 / 2^k inputs starting at `first`
- * (uint32 bit patterns of binary32 values, `count` of them, stepping by 1)
+/* Runs the device codecs over `count` consecutive binary32 bit patterns
+ * starting at `first`
  * and writes: e4m3 codes (count bytes), e2m1 codes (count bytes, one code
  * per byte), bf16 bit patterns (count x uint16).  Any of the outputs may be
  * NULL.  Used to compare the device conversions with the oracle. */

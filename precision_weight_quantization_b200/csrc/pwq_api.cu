@@ -93,8 +93,11 @@ pwq_status check_tensor(const pwq_tensor* t, Kind k, View* v, Extent* ext, const
         return PWQ_OK;
     }
     if (!t->ptr) return fail(PWQ_ERR_NULL, name);
-    if ((uintptr_t)t->ptr % 16 != 0 || (t->row_stride * unit) % 16 != 0 ||
-        (t->batch > 1 && (t->batch_stride * unit) % 16 != 0))
+    // BF16 rows are moved in 16-byte vectors (and by TMA); code rows in
+    // 8-byte (E4M3) or 4-byte (packed E2M1) pieces
+    const int64_t align = (k == Kind::kBF16) ? 16 : 8;
+    if ((uintptr_t)t->ptr % align != 0 || (t->row_stride * unit) % align != 0 ||
+        (t->batch > 1 && (t->batch_stride * unit) % align != 0))
         return fail(PWQ_ERR_ALIGN, name);
     if (t->row_stride < row_units || (t->batch > 1 && t->batch_stride < t->rows * t->row_stride))
         return fail(PWQ_ERR_STRIDE, name);

@@ -88,31 +88,41 @@ __device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
 
 // ---------------------------------------------------------------- division
 
-// Correctly rounded binary32 quotient x / s from the correctly rounded
-// reciprocal r = RN(1/s): one product and one residual correction with
-// fused multiply-adds (Markstein's correction step; P. Markstein,
-// "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990).  The caller uses it only when
-// `div_fast_ok(s, r)` holds; over every BF16 numerator and every divisor the
-// formats produce, its results are checked bit for bit against __fdiv_rn by
-// pwq_selftest_division.
+// Binary32 quotient x / s from the correctly rounded reciprocal r = RN(1/s):
+// one product and one residual correction with fused multiply-adds
+// (Markstein's correction step; P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990).  The residual x - q0*s is exact only while it does not underflow,
+// so the caller takes this path only for a positive divisor whose
+// reciprocal is normal (div_fast_ok) and a numerator that is zero or at
+// least 2^-100 in magnitude (num_fast_ok).  The quotient's sign is set from
+// x (s > 0), which keeps -0 / s = -0.  Over every BF16 numerator and every
+// divisor the formats produce, pwq_selftest_division checks the codes this
+// gives against IEEE division (__fdiv_rn), and the binary32 quotients
+// wherever the IEEE quotient is normal.
 __device__ __forceinline__ float div_rcp_correct(float x, float s, float r) {
     float q0 = __fmul_rn(x, r);
     float res = __fmaf_rn(-q0, s, x);
-    return __fmaf_rn(res, r, q0);
+    float q = __fmaf_rn(res, r, q0);
+    return __uint_as_float(__float_as_uint(q) | (__float_as_uint(x) & 0x80000000u));
 }
 
-// The fast quotient is used only when the divisor and its reciprocal are
-// both normal binary32 numbers (exponent field in 1..254).
+// Divisor condition: s and RN(1/s) are both normal binary32 numbers.
 __device__ __forceinline__ bool div_fast_ok(float s, float r) {
     uint32_t es = (__float_as_uint(s) >> 23) & 0xffu;
     uint32_t er = (__float_as_uint(r) >> 23) & 0xffu;
     return (es - 1u) < 254u && (er - 1u) < 254u;
 }
 
+// Numerator condition: x == +-0 or |x| >= 2^-100.
+__device__ __forceinline__ bool num_fast_ok(float x) {
+    const uint32_t ax = __float_as_uint(x) & 0x7fffffffu;
+    return ax >= 0x0d800000u || ax == 0u;
+}
+
 // fl(x / s) with the zero-scale reading: s == 0 gives a zero of x's sign.
 __device__ __forceinline__ float quotient(float x, float s, float r, bool fast) {
-    if (fast) return div_rcp_correct(x, s, r);
+    if (fast && num_fast_ok(x)) return div_rcp_correct(x, s, r);
     if (s == 0.0f) return __uint_as_float(__float_as_uint(x) & 0x80000000u);
     return __fdiv_rn(x, s);
 }

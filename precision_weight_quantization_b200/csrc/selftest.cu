@@ -19,47 +19,54 @@ constexpr int kThreads = 256;
 
 __device__ __forceinline__ bool bf16_is_finite(uint32_t b) { return ((b >> 7) & 0xffu) != 0xffu; }
 
-// One divisor per CTA; every finite BF16 numerator.
+// One divisor per CTA; every finite BF16 numerator the format can pair with
+// it: |x| <= a for FP8 block-wise (x is in the tile whose amax is a), and
+// |x| <= 16 d for NVFP4 (x / d stays below 6 / (1 - 2^-4) for an E4M3-normal
+// block scale and below 9.1 for a subnormal one).
 template <int kWhich>
 __global__ void __launch_bounds__(kThreads) selftest_division_kernel(unsigned long long* counts) {
-    float d;
+    float d, xmax;
     if (kWhich == 0) {
         const uint32_t a = blockIdx.x + 1u;            // positive finite BF16 0x0001..0x7f7f
-        d = __fdiv_rn(__uint_as_float(a << 16), 448.0f);
+        xmax = __uint_as_float(a << 16);
+        d = __fdiv_rn(xmax, 448.0f);
     } else {
         const uint32_t a = blockIdx.x + 1u;
         const uint32_t sb = blockIdx.y + 1u;           // E4M3 0x01..0x7e
         const float gs = __fdiv_rn(__uint_as_float(a << 16), 2688.0f);
         d = __fmul_rn(e4m3_decode(sb), gs);
+        xmax = __fmul_rn(16.0f, d);
     }
     const float r = __frcp_rn(d);
     const bool fast = div_fast_ok(d, r);
-    unsigned long long n = 0, code_bad = 0, quot_bad = 0;
+    unsigned long long n = 0, code_bad = 0, quot_bad = 0, slow = 0;
     for (uint32_t xb = threadIdx.x; xb < 65536u; xb += kThreads) {
         if (!bf16_is_finite(xb)) continue;
         const float x = __uint_as_float(xb << 16);
+        if (!(fabsf(x) <= xmax)) continue;
         const float qf = quotient(x, d, r, fast);
         const float qr = (d == 0.0f) ? __uint_as_float((xb << 16) & 0x80000000u) : __fdiv_rn(x, d);
         ++n;
-        if (kWhich == 0) {
+        slow += !(fast && num_fast_ok(x));
+        if (kWhich == 0)
             code_bad += (e4m3x2(qf, 0.0f) & 0xffu) != (e4m3x2(qr, 0.0f) & 0xffu);
-            const uint32_t ef = (__float_as_uint(qr) >> 23) & 0xffu;
-            if (ef != 0u) quot_bad += __float_as_uint(qf) != __float_as_uint(qr);
-        } else {
+        else
             code_bad += (e2m1x2(qf, 0.0f) & 0xfu) != (e2m1x2(qr, 0.0f) & 0xfu);
-        }
+        const uint32_t ef = (__float_as_uint(qr) >> 23) & 0xffu;
+        if (ef != 0u) quot_bad += __float_as_uint(qf) != __float_as_uint(qr);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         n += __shfl_xor_sync(0xffffffffu, n, o);
         code_bad += __shfl_xor_sync(0xffffffffu, code_bad, o);
         quot_bad += __shfl_xor_sync(0xffffffffu, quot_bad, o);
+        slow += __shfl_xor_sync(0xffffffffu, slow, o);
     }
     if ((threadIdx.x & 31u) == 0u) {
         atomicAdd(counts + 0, n);
         atomicAdd(counts + 1, code_bad);
         atomicAdd(counts + 2, quot_bad);
-        if (!fast) atomicAdd(counts + 3, n);
+        atomicAdd(counts + 3, slow);
     }
 }
 

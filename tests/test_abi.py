@@ -74,7 +74,7 @@ def test_validation_errors_without_gpu():
     xn = T(L, None, 1, 256, 512, 256 * 512, 512)
     assert lib.fp8_block_quant(by(xn), by(q), s, None) == L.PWQ_ERR_NULL
     # alignment
-    xa = T(L, base + 8, 1, 256, 512, 256 * 512, 512)
+    xa = T(L, base + 8, 1, 256, 512, 256 * 512, 512)                 # BF16 base must be 16-aligned
     assert lib.fp8_block_quant(by(xa), by(q), s, None) == L.PWQ_ERR_ALIGN
     xr = T(L, base, 1, 256, 512, 256 * 516, 516)          # 1032-byte rows: not 16-aligned
     assert lib.fp8_block_quant(by(xr), by(q), s, None) == L.PWQ_ERR_ALIGN
