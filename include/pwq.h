@@ -248,15 +248,17 @@ pwq_status pwq_device_error(uint32_t* code);
 /* Exhaustive self-check of the device arithmetic against CUDA's IEEE
  * division (__fdiv_rn), for every divisor the formats can produce and every
  * finite BF16 numerator that can be paired with it:
- *   which = 0  FP8 block: divisors s = fl(a / 448), a every positive finite
- *              BF16; numerators |x| <= a.  Compares E4M3 codes.
- *   which = 1  NVFP4: divisors d = fl(dec(sb) * fl(a / 2688)) for every
+ *   which = 0  FP8 block code divisor s = fl(a / 448), a every positive
+ *              finite BF16; numerators |x| <= a.  Compares E4M3 codes.
+ *   which = 1  NVFP4 code divisor d = fl(dec(sb) * fl(a / 2688)) for every
  *              positive finite BF16 a and every non-zero E4M3 sb;
  *              numerators |x| <= 16 d.  Compares E2M1 codes.
+ *   which = 2  NVFP4 block-scale divisor fl(6 * fl(a / 2688)); numerators
+ *              |x| <= a.  Compares E4M3 codes.
  * counts (device, 4 x uint64, zeroed by the call): [0] pairs checked,
- * [1] code mismatches, [2] binary32 quotient mismatches where the IEEE
- * quotient is a normal number, [3] pairs that took the IEEE-division
- * fallback instead of the reciprocal path.  Asynchronous on `stream`. */
+ * [1] code mismatches, [2] binary32 quotient mismatches where |x| >= 2^-100
+ * and the IEEE quotient is normal, [3] pairs whose divisor takes the
+ * IEEE-division path instead of the reciprocal path.  Asynchronous. */
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream);
 
 /* Runs the device codecs over `count` consecutive binary32 bit patterns

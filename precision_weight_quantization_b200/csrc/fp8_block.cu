@@ -59,6 +59,20 @@ __device__ __forceinline__ void issue_tile(const CUtensorMap* tmap, uint32_t dst
     tma_load_3d(dst, tmap, bar, tn * kTile, tm * kTile, b);
 }
 
+// E4M3 codes of a thread's 8 chunks (64 elements) for tile scale s with
+// r = RN(1/s); kFast selects the reciprocal path for the whole tile.
+template <bool kFast>
+__device__ __forceinline__ void encode_chunks(const uint4 (&v)[kChunksPerThread], float s, float r,
+                                              uint2 (&out)[kChunksPerThread]) {
+#pragma unroll
+    for (int j = 0; j < kChunksPerThread; ++j) {
+        float q[8];
+        quotients8<kFast>(v[j], s, r, q);
+        out[j].x = e4m3x4(q[0], q[1], q[2], q[3]);
+        out[j].y = e4m3x4(q[4], q[5], q[6], q[7]);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
 fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs a) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -131,7 +145,11 @@ fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs
         const float amax = __uint_as_float(am << 16);
         const float sc = __fdiv_rn(amax, 448.0f);
         const float rc = __frcp_rn(sc);
-        const bool fast = div_fast_ok(sc, rc);
+        uint2 out[kChunksPerThread];
+        if (div_fast_ok(sc))   // CTA-uniform
+            encode_chunks<true>(v, sc, rc, out);
+        else
+            encode_chunks<false>(v, sc, rc, out);
 
         int b, tm, tn;
         tile_coords(t, a, b, tm, tn);
@@ -139,91 +157,97 @@ fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs
         const int rows_here = min(kTile, a.rows - tm * kTile);
         const int cols_here = min(kTile, a.cols - tn * kTile);
         char* qtile = a.q + (int64_t)b * a.q_bs + (int64_t)tm * kTile * a.q_rs + (int64_t)tn * kTile;
+        if (rows_here == kTile && cols_here == kTile) {
 #pragma unroll
-        for (int j = 0; j < kChunksPerThread; ++j) {
-            const int r = row0 + 16 * j;
-            uint2 out;
-            out.x = e4m3x4(quotient(bf16_lo(v[j].x), sc, rc, fast), quotient(bf16_hi(v[j].x), sc, rc, fast),
-                           quotient(bf16_lo(v[j].y), sc, rc, fast), quotient(bf16_hi(v[j].y), sc, rc, fast));
-            out.y = e4m3x4(quotient(bf16_lo(v[j].z), sc, rc, fast), quotient(bf16_hi(v[j].z), sc, rc, fast),
-                           quotient(bf16_lo(v[j].w), sc, rc, fast), quotient(bf16_hi(v[j].w), sc, rc, fast));
-            if (r < rows_here) {
+            for (int j = 0; j < kChunksPerThread; ++j)
+                st_v2(qtile + (int64_t)(row0 + 16 * j) * a.q_rs + ccol, out[j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < kChunksPerThread; ++j) {
+                const int r = row0 + 16 * j;
+                if (r >= rows_here || ccol >= cols_here) continue;
                 char* dst = qtile + (int64_t)r * a.q_rs + ccol;
                 if (ccol + 8 <= cols_here) {
-                    st_v2(dst, out);
-                } else if (ccol < cols_here) {
+                    st_v2(dst, out[j]);
+                } else {
                     for (int e = 0; e < cols_here - ccol; ++e)
-                        dst[e] = (char)((e < 4 ? out.x >> (8 * e) : out.y >> (8 * (e - 4))) & 0xffu);
+                        dst[e] = (char)((e < 4 ? out[j].x >> (8 * e) : out[j].y >> (8 * (e - 4))) & 0xffu);
                 }
             }
         }
     }
 }
 
-// Dequantise: 8 codes (8 bytes) -> 8 BF16 (16 bytes) per chunk; the
-// chunk's tile scale is a cached 4-byte load.  Ragged row tails (cols not a
-// multiple of 8) take a byte-wise path.
+// Dequantise: a persistent grid walks the tiles; the tile scale is one
+// load per tile.  Thread t owns 16-code chunks at column (t & 7) * 16 of
+// rows (t >> 3) + 32 j, j = 0..3: a 16-byte code load becomes two 16-byte
+// BF16 stores.  Edge tiles take a masked element-wise path.
 struct DequantArgs {
     const char* q;
     char* y;
-    const float* scale;
-    int64_t q_bs, q_rs, y_bs, y_rs;
-    FastDiv cpr;      // chunks per row, ceil(N / 8)
-    FastDiv rows;     // M
-    int cols, tiles_m, tiles_n;
-    uint32_t total;
+    const float* scale;   // dense [B][TM][TN]
+    int64_t q_bs, q_rs, y_bs, y_rs;  // bytes
+    int rows, cols, tiles_m, tiles_n;
+    uint32_t total_tiles;
+    int vec16;            // code rows 16-byte aligned (else two 8-byte loads)
 };
 
-constexpr int kDqUnroll = 4;
+constexpr int kDqRowsPerPass = kThreads / 8;         // 32
+constexpr int kDqChunks = kTile / kDqRowsPerPass;     // 4
+
+__device__ __forceinline__ uint4 dequant8(uint2 codes, float s) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const uint32_t pair = ((h < 2 ? codes.x : codes.y) >> (16 * (h & 1))) & 0xffffu;
+        const float2 f = e4m3x2_decode(pair);
+        w[h] = pack_bf16x2(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const DequantArgs a) {
-    const uint32_t stride = gridDim.x * blockDim.x;
-    for (uint32_t base = blockIdx.x * blockDim.x + threadIdx.x; base < a.total;
-         base += stride * kDqUnroll) {
-        uint2 v[kDqUnroll];
-        float sc[kDqUnroll];
-        char* yp[kDqUnroll];
-        int nvalid[kDqUnroll];
+    const int ccol = (int)(threadIdx.x & 7u) * 16;
+    const int row0 = (int)(threadIdx.x >> 3);
+    const uint32_t per_b = (uint32_t)a.tiles_m * (uint32_t)a.tiles_n;
+    for (uint32_t t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
+        const uint32_t b = t / per_b;
+        const uint32_t rem = t - b * per_b;
+        const int tm = (int)(rem / (uint32_t)a.tiles_n);
+        const int tn = (int)(rem - (uint32_t)tm * (uint32_t)a.tiles_n);
+        const float sc = __ldg(a.scale + t);
+        const char* qt = a.q + (int64_t)b * a.q_bs + (int64_t)tm * kTile * a.q_rs + (int64_t)tn * kTile;
+        char* yt = a.y + (int64_t)b * a.y_bs + (int64_t)tm * kTile * a.y_rs + (int64_t)tn * kTile * 2;
+        const int rows_here = min(kTile, a.rows - tm * kTile);
+        const int cols_here = min(kTile, a.cols - tn * kTile);
+        if (rows_here == kTile && cols_here == kTile) {
+            uint4 v[kDqChunks];
 #pragma unroll
-        for (int u = 0; u < kDqUnroll; ++u) {
-            const uint32_t c = base + u * stride;
-            const uint32_t r = fdiv(c, a.cpr);
-            const int col = (int)(c - r * a.cpr.d) * 8;
-            const uint32_t b = fdiv(r, a.rows);
-            const int mrow = (int)(r - b * a.rows.d);
-            const char* qp = a.q + (int64_t)b * a.q_bs + (int64_t)mrow * a.q_rs + col;
-            yp[u] = a.y + (int64_t)b * a.y_bs + (int64_t)mrow * a.y_rs + (int64_t)col * 2;
-            nvalid[u] = (c < a.total) ? min(8, a.cols - col) : 0;
-            v[u] = make_uint2(0u, 0u);
-            sc[u] = 0.0f;
-            if (nvalid[u] > 0) {
-                sc[u] = __ldg(a.scale + ((int64_t)b * a.tiles_m + (mrow >> 7)) * a.tiles_n + (col >> 7));
-                if (nvalid[u] == 8) {
-                    v[u] = ld_stream_v2(qp);
+            for (int j = 0; j < kDqChunks; ++j) {
+                const char* src = qt + (int64_t)(row0 + kDqRowsPerPass * j) * a.q_rs + ccol;
+                if (a.vec16) {
+                    v[j] = ld_stream_v4(src);
                 } else {
-                    uint32_t w[2] = {0u, 0u};
-                    for (int e = 0; e < nvalid[u]; ++e)
-                        w[e >> 2] |= (uint32_t)(unsigned char)qp[e] << (8 * (e & 3));
-                    v[u] = make_uint2(w[0], w[1]);
+                    const uint2 lo = ld_stream_v2(src), hi = ld_stream_v2(src + 8);
+                    v[j] = make_uint4(lo.x, lo.y, hi.x, hi.y);
                 }
             }
-        }
 #pragma unroll
-        for (int u = 0; u < kDqUnroll; ++u) {
-            if (nvalid[u] <= 0) continue;
-            uint32_t w[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const uint32_t pair = ((h < 2 ? v[u].x : v[u].y) >> (16 * (h & 1))) & 0xffffu;
-                const float2 f = e4m3x2_decode(pair);
-                w[h] = pack_bf16x2(__fmul_rn(f.x, sc[u]), __fmul_rn(f.y, sc[u]));
+            for (int j = 0; j < kDqChunks; ++j) {
+                char* dst = yt + (int64_t)(row0 + kDqRowsPerPass * j) * a.y_rs + ccol * 2;
+                st_v4(dst, dequant8(make_uint2(v[j].x, v[j].y), sc));
+                st_v4(dst + 16, dequant8(make_uint2(v[j].z, v[j].w), sc));
             }
-            if (nvalid[u] == 8) {
-                st_v4(yp[u], make_uint4(w[0], w[1], w[2], w[3]));
-            } else {
-                unsigned short* y16 = reinterpret_cast<unsigned short*>(yp[u]);
-                for (int e = 0; e < nvalid[u]; ++e)
-                    y16[e] = (unsigned short)((w[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+        } else {
+            for (int j = 0; j < kDqChunks; ++j) {
+                const int r = row0 + kDqRowsPerPass * j;
+                if (r >= rows_here) break;
+                const unsigned char* src = reinterpret_cast<const unsigned char*>(qt + (int64_t)r * a.q_rs);
+                unsigned short* dst = reinterpret_cast<unsigned short*>(yt + (int64_t)r * a.y_rs);
+                for (int c = ccol; c < min(ccol + 16, cols_here); ++c) {
+                    const float f = __fmul_rn(e4m3_decode(src[c]), sc);
+                    dst[c] = (unsigned short)(pack_bf16x2(f, 0.0f) & 0xffffu);
+                }
             }
         }
     }
@@ -306,15 +330,13 @@ cudaError_t launch_fp8_block_dequant(const View& q, const float* scale, const Vi
     a.q_rs = q.rstride;
     a.y_bs = y.bstride;
     a.y_rs = y.rstride;
-    const int64_t cpr = (q.cols + 7) / 8;
-    a.cpr = make_fastdiv((uint32_t)cpr);
-    a.rows = make_fastdiv((uint32_t)q.rows);
+    a.rows = (int)q.rows;
     a.cols = (int)q.cols;
     a.tiles_m = (int)((q.rows + kTile - 1) / kTile);
     a.tiles_n = (int)((q.cols + kTile - 1) / kTile);
-    a.total = (uint32_t)(q.batch * q.rows * cpr);
-    const int64_t span = int64_t(kThreads) * kDqUnroll;
-    const int grid = persistent_grid((a.total + span - 1) / span, 8);
+    a.total_tiles = (uint32_t)(q.batch * a.tiles_m * a.tiles_n);
+    a.vec16 = ((uintptr_t)q.ptr % 16 == 0) && (q.rstride % 16 == 0) && (q.batch == 1 || q.bstride % 16 == 0);
+    const int grid = persistent_grid(a.total_tiles, 8);
     fp8_block_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }

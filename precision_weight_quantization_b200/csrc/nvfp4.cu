@@ -15,10 +15,13 @@
 //      128-bit load each, amax combined with one shuffle).  It walks the
 //      tensor in the reverse order of pass 1 so that the most recently read
 //      data -- still in the 126 MB L2 -- is consumed first.
-// Division: each block's divisor d gets one correctly rounded reciprocal;
-// the per-element quotient is the reciprocal product plus one FMA residual
-// correction (pwq_device.cuh), which the self-test proves equal to IEEE
-// division over every BF16 numerator and every reachable divisor.
+// Division: a group has at most 127 distinct code divisors d = fl(dec(sb) *
+// gs), so each CTA tabulates d and RN(1/d) for every block-scale code in
+// shared memory once; the block scale itself divides by fl(6 gs), whose
+// reciprocal is also formed once.  Per element the quotient is the
+// reciprocal product plus one FMA residual correction (pwq_device.cuh),
+// which the self-test proves to give IEEE division's codes over every BF16
+// numerator and every reachable divisor.
 #include <algorithm>
 
 #include "pwq_internal.h"
@@ -104,35 +107,30 @@ struct EncodeArgs {
     float* amax_out;            // [B] or null
 };
 
-// Codes (quant) or dequantised BF16 (fake) for one 8-element half block.
-// `m` is the 16-element block amax (BF16 magnitude bits), `gs`/`six_gs` the
-// group's global scale and fl(6 * gs).
-struct HalfBlock {
-    uint32_t sb;     // E4M3 block scale byte
-    uint32_t codes;  // 8 nibbles, element 0 in bits 0..3
-    float sbv;       // dec(sb)
+// Per-group constants of the encode pass, for every E4M3 block-scale code
+// k: d_k = fl(dec(k) * gs) (the code divisor), r_k = RN(1/d_k) when d_k is
+// in the reciprocal path's range (else 0: IEEE division), and dec(k).
+struct ScaleTable {
+    float4 e[128];
 };
 
-__device__ __forceinline__ HalfBlock encode_half(uint4 v, uint32_t m, float gs, float six_gs) {
-    HalfBlock h;
-    const float amax_b = __uint_as_float(m << 16);
-    h.sb = (gs == 0.0f) ? 0u : (e4m3x2(__fdiv_rn(amax_b, six_gs), 0.0f) & 0xffu);
-    h.sbv = e4m3_decode(h.sb);
-    const float d = __fmul_rn(h.sbv, gs);
-    const float r = __frcp_rn(d);
-    const bool fast = div_fast_ok(d, r);
+__device__ __forceinline__ void fill_scale_table(ScaleTable& t, float gs) {
+    for (uint32_t k = threadIdx.x; k < 128u; k += blockDim.x) {
+        const float dec = e4m3_decode(k);  // k = 0x7f (NaN) is never produced
+        const float d = __fmul_rn(dec, gs);
+        t.e[k] = make_float4(d, div_fast_ok(d) ? __frcp_rn(d) : 0.0f, dec, 0.0f);
+    }
+}
+
+// E2M1 codes of one 8-element half block (element 0 in bits 0..3).
+__device__ __forceinline__ uint32_t codes_half(uint4 v, float d, float r) {
     float q[8];
-    q[0] = quotient(bf16_lo(v.x), d, r, fast);
-    q[1] = quotient(bf16_hi(v.x), d, r, fast);
-    q[2] = quotient(bf16_lo(v.y), d, r, fast);
-    q[3] = quotient(bf16_hi(v.y), d, r, fast);
-    q[4] = quotient(bf16_lo(v.z), d, r, fast);
-    q[5] = quotient(bf16_hi(v.z), d, r, fast);
-    q[6] = quotient(bf16_lo(v.w), d, r, fast);
-    q[7] = quotient(bf16_hi(v.w), d, r, fast);
-    h.codes = e2m1x2(q[0], q[1]) | (e2m1x2(q[2], q[3]) << 8) | (e2m1x2(q[4], q[5]) << 16) |
-              (e2m1x2(q[6], q[7]) << 24);
-    return h;
+    if (r != 0.0f)
+        quotients8<true>(v, d, r, q);
+    else
+        quotients8<false>(v, d, r, q);
+    return e2m1x2(q[0], q[1]) | (e2m1x2(q[2], q[3]) << 8) | (e2m1x2(q[4], q[5]) << 16) |
+           (e2m1x2(q[6], q[7]) << 24);
 }
 
 // y = bf16(fl((dec(c) * dec(sb)) * gs)) for the 8 codes of a half block.
@@ -148,14 +146,19 @@ __device__ __forceinline__ uint4 dequant_half(uint32_t codes, float sbv, float g
 
 template <bool kFake>
 __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs a) {
+    __shared__ ScaleTable tab;
     const uint32_t b = blockIdx.y;
     const float A = a.amax_in ? a.amax_in[b] : __uint_as_float(a.amax_bits[b]);
     const float gs = __fdiv_rn(A, 2688.0f);
     const float six_gs = __fmul_rn(6.0f, gs);
+    const float r6 = __frcp_rn(six_gs);
+    const bool fast6 = div_fast_ok(six_gs);
+    fill_scale_table(tab, gs);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         if (a.gs_out) a.gs_out[b] = gs;
         if (a.amax_out) a.amax_out[b] = A;
     }
+    __syncthreads();
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -190,7 +193,12 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
                 const uint32_t j = base + u * 32u + lane;
                 uint32_t m = amax_bits8(v[u]);
                 m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-                const HalfBlock h = encode_half(v[u], m, gs, six_gs);
+                // block scale sb = e4m3(fl(amax_b / fl(6 gs)))
+                const float amax_b = __uint_as_float(m << 16);
+                const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
+                const uint32_t sb = e4m3x2(ratio, 0.0f) & 0xffu;
+                const float4 e = tab.e[sb];
+                const uint32_t codes = codes_half(v[u], e.x, e.y);
                 if (j < S.chunks) {
                     const uint32_t c = cc[u];
                     int64_t oo;
@@ -201,10 +209,10 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
                         oo = (int64_t)r * S.o_rs + (int64_t)(c - r * S.cpr.d) * (kFake ? 16 : 4);
                     }
                     if (kFake) {
-                        st_v4(ob + oo, dequant_half(h.codes, h.sbv, gs));
+                        st_v4(ob + oo, dequant_half(codes, e.z, gs));
                     } else {
-                        st_u32(ob + oo, h.codes);
-                        if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)h.sb;
+                        st_u32(ob + oo, codes);
+                        if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)sb;
                     }
                 }
             }

@@ -415,7 +415,7 @@ pwq_status nvfp4_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_sibl
 
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream) {
     if (!counts) return fail(PWQ_ERR_NULL, "counts");
-    if (which != 0 && which != 1) return fail(PWQ_ERR_ARG, "which");
+    if (which < 0 || which > 2) return fail(PWQ_ERR_ARG, "which");
     return from_cuda(pwq::launch_selftest_division(which, counts, (cudaStream_t)stream));
 }
 

@@ -88,43 +88,55 @@ __device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
 
 // ---------------------------------------------------------------- division
 
-// Binary32 quotient x / s from the correctly rounded reciprocal r = RN(1/s):
-// one product and one residual correction with fused multiply-adds
-// (Markstein's correction step; P. Markstein, "Computation of elementary
-// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
-// 1990).  The residual x - q0*s is exact only while it does not underflow,
-// so the caller takes this path only for a positive divisor whose
-// reciprocal is normal (div_fast_ok) and a numerator that is zero or at
-// least 2^-100 in magnitude (num_fast_ok).  The quotient's sign is set from
-// x (s > 0), which keeps -0 / s = -0.  Over every BF16 numerator and every
-// divisor the formats produce, pwq_selftest_division checks the codes this
-// gives against IEEE division (__fdiv_rn), and the binary32 quotients
-// wherever the IEEE quotient is normal.
-__device__ __forceinline__ float div_rcp_correct(float x, float s, float r) {
+// Quotient x / s for a positive block divisor s, from the correctly rounded
+// reciprocal r = RN(1/s): one product and one residual correction with
+// fused multiply-adds (Markstein's correction step; P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990).  The quotient's sign is set
+// from x, which keeps -0 / s = -0.
+//
+// It is used for a whole tile or block when 2^-64 <= s <= 2^126 (then s and
+// r are normal).  Within that range:
+//   |x| >= 2^-100: the residual x - q0*s is exact and the result is the IEEE
+//                  quotient, bit for bit;
+//   |x| <  2^-100: |x / s| < 2^-36 and every intermediate stays below 2^-30,
+//                  so the E4M3 / E2M1 code is +-0 exactly as with IEEE
+//                  division (the binary32 quotient itself may differ in its
+//                  last subnormal bits, and is never stored).
+// pwq_selftest_division checks both statements over every BF16 numerator
+// and every divisor the formats produce, against __fdiv_rn.
+__device__ __forceinline__ float div_fast(float x, float s, float r) {
     float q0 = __fmul_rn(x, r);
     float res = __fmaf_rn(-q0, s, x);
     float q = __fmaf_rn(res, r, q0);
     return __uint_as_float(__float_as_uint(q) | (__float_as_uint(x) & 0x80000000u));
 }
 
-// Divisor condition: s and RN(1/s) are both normal binary32 numbers.
-__device__ __forceinline__ bool div_fast_ok(float s, float r) {
-    uint32_t es = (__float_as_uint(s) >> 23) & 0xffu;
-    uint32_t er = (__float_as_uint(r) >> 23) & 0xffu;
-    return (es - 1u) < 254u && (er - 1u) < 254u;
-}
+__device__ __forceinline__ bool div_fast_ok(float s) { return s >= 0x1p-64f && s <= 0x1p126f; }
 
-// Numerator condition: x == +-0 or |x| >= 2^-100.
-__device__ __forceinline__ bool num_fast_ok(float x) {
-    const uint32_t ax = __float_as_uint(x) & 0x7fffffffu;
-    return ax >= 0x0d800000u || ax == 0u;
-}
-
-// fl(x / s) with the zero-scale reading: s == 0 gives a zero of x's sign.
-__device__ __forceinline__ float quotient(float x, float s, float r, bool fast) {
-    if (fast && num_fast_ok(x)) return div_rcp_correct(x, s, r);
+// Outside that range: IEEE division, with the zero-scale reading (s == 0
+// gives a zero of x's sign).
+__device__ __forceinline__ float div_slow(float x, float s) {
     if (s == 0.0f) return __uint_as_float(__float_as_uint(x) & 0x80000000u);
     return __fdiv_rn(x, s);
+}
+
+template <bool kFast>
+__device__ __forceinline__ float quotient(float x, float s, float r) {
+    return kFast ? div_fast(x, s, r) : div_slow(x, s);
+}
+
+// The 8 quotients of a 16-byte BF16 chunk.
+template <bool kFast>
+__device__ __forceinline__ void quotients8(uint4 v, float s, float r, float q[8]) {
+    q[0] = quotient<kFast>(bf16_lo(v.x), s, r);
+    q[1] = quotient<kFast>(bf16_hi(v.x), s, r);
+    q[2] = quotient<kFast>(bf16_lo(v.y), s, r);
+    q[3] = quotient<kFast>(bf16_hi(v.y), s, r);
+    q[4] = quotient<kFast>(bf16_lo(v.z), s, r);
+    q[5] = quotient<kFast>(bf16_hi(v.z), s, r);
+    q[6] = quotient<kFast>(bf16_lo(v.w), s, r);
+    q[7] = quotient<kFast>(bf16_hi(v.w), s, r);
 }
 
 // ---------------------------------------------------------------- UE8M0

@@ -20,40 +20,50 @@ constexpr int kThreads = 256;
 __device__ __forceinline__ bool bf16_is_finite(uint32_t b) { return ((b >> 7) & 0xffu) != 0xffu; }
 
 // One divisor per CTA; every finite BF16 numerator the format can pair with
-// it: |x| <= a for FP8 block-wise (x is in the tile whose amax is a), and
-// |x| <= 16 d for NVFP4 (x / d stays below 6 / (1 - 2^-4) for an E4M3-normal
-// block scale and below 9.1 for a subnormal one).
+// it:
+//   kWhich 0  FP8 block-wise code divisor s = fl(a / 448), |x| <= a (x is in
+//             the tile whose amax is a);
+//   kWhich 1  NVFP4 code divisor d = fl(dec(sb) * fl(a / 2688)), |x| <= 16 d
+//             (x / d stays below 6 / (1 - 2^-4) for an E4M3-normal block
+//             scale and below 9.1 for a subnormal one);
+//   kWhich 2  NVFP4 block-scale divisor fl(6 * fl(a / 2688)), |x| <= a (the
+//             block amax never exceeds the group amax a).
+// The kernels' path (reciprocal or IEEE, chosen by the divisor) is compared
+// with __fdiv_rn: codes for every pair, binary32 quotients where |x| >=
+// 2^-100 and the IEEE quotient is normal.
 template <int kWhich>
 __global__ void __launch_bounds__(kThreads) selftest_division_kernel(unsigned long long* counts) {
+    const uint32_t a = blockIdx.x + 1u;                // positive finite BF16 0x0001..0x7f7f
+    const float av = __uint_as_float(a << 16);
     float d, xmax;
     if (kWhich == 0) {
-        const uint32_t a = blockIdx.x + 1u;            // positive finite BF16 0x0001..0x7f7f
-        xmax = __uint_as_float(a << 16);
-        d = __fdiv_rn(xmax, 448.0f);
-    } else {
-        const uint32_t a = blockIdx.x + 1u;
+        d = __fdiv_rn(av, 448.0f);
+        xmax = av;
+    } else if (kWhich == 1) {
         const uint32_t sb = blockIdx.y + 1u;           // E4M3 0x01..0x7e
-        const float gs = __fdiv_rn(__uint_as_float(a << 16), 2688.0f);
-        d = __fmul_rn(e4m3_decode(sb), gs);
+        d = __fmul_rn(e4m3_decode(sb), __fdiv_rn(av, 2688.0f));
         xmax = __fmul_rn(16.0f, d);
+    } else {
+        d = __fmul_rn(6.0f, __fdiv_rn(av, 2688.0f));
+        xmax = av;
     }
     const float r = __frcp_rn(d);
-    const bool fast = div_fast_ok(d, r);
+    const bool fast = div_fast_ok(d);
     unsigned long long n = 0, code_bad = 0, quot_bad = 0, slow = 0;
     for (uint32_t xb = threadIdx.x; xb < 65536u; xb += kThreads) {
         if (!bf16_is_finite(xb)) continue;
         const float x = __uint_as_float(xb << 16);
         if (!(fabsf(x) <= xmax)) continue;
-        const float qf = quotient(x, d, r, fast);
+        const float qf = fast ? quotient<true>(x, d, r) : quotient<false>(x, d, r);
         const float qr = (d == 0.0f) ? __uint_as_float((xb << 16) & 0x80000000u) : __fdiv_rn(x, d);
         ++n;
-        slow += !(fast && num_fast_ok(x));
-        if (kWhich == 0)
-            code_bad += (e4m3x2(qf, 0.0f) & 0xffu) != (e4m3x2(qr, 0.0f) & 0xffu);
-        else
+        slow += !fast;
+        if (kWhich == 1)
             code_bad += (e2m1x2(qf, 0.0f) & 0xfu) != (e2m1x2(qr, 0.0f) & 0xfu);
+        else
+            code_bad += (e4m3x2(qf, 0.0f) & 0xffu) != (e4m3x2(qr, 0.0f) & 0xffu);
         const uint32_t ef = (__float_as_uint(qr) >> 23) & 0xffu;
-        if (ef != 0u) quot_bad += __float_as_uint(qf) != __float_as_uint(qr);
+        if (ef != 0u && fabsf(x) >= 0x1p-100f) quot_bad += __float_as_uint(qf) != __float_as_uint(qr);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -86,11 +96,12 @@ selftest_codecs_kernel(uint32_t first, uint32_t count, uint8_t* e4m3, uint8_t* e
 cudaError_t launch_selftest_division(int which, unsigned long long* counts, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(counts, 0, 4 * sizeof(unsigned long long), s);
     if (e != cudaSuccess) return e;
-    if (which == 0) {
+    if (which == 0)
         selftest_division_kernel<0><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
-    } else {
+    else if (which == 1)
         selftest_division_kernel<1><<<dim3(0x7f7f, 0x7e), kThreads, 0, s>>>(counts);
-    }
+    else
+        selftest_division_kernel<2><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
     return cudaGetLastError();
 }
 

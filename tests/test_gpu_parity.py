@@ -368,16 +368,16 @@ def test_dsv3_experts_and_activation_full_size(P):
 
 # ------------------------------------------------------------------ device arithmetic self-tests
 
-@pytest.mark.parametrize("which", [0, 1], ids=["fp8_divisors", "nvfp4_divisors"])
+@pytest.mark.parametrize("which", [0, 1, 2], ids=["fp8_divisors", "nvfp4_divisors", "nvfp4_scale_divisors"])
 def test_division_exhaustive(P, which):
     counts = torch.zeros(4, dtype=torch.int64, device=DEV)
     P.check(P.lib.pwq_selftest_division(which, counts.data_ptr(), None), "pwq_selftest_division")
     torch.cuda.synchronize()
     n, code_bad, quot_bad, fallback = counts.tolist()
-    print("division self-test", ["fp8", "nvfp4"][which], "pairs", n, "code mismatches", code_bad,
+    print("division self-test", ["fp8", "nvfp4", "nvfp4_sb"][which], "pairs", n, "code mismatches", code_bad,
           "quotient mismatches", quot_bad, "fallback pairs", fallback)
-    if which == 0:
-        # FP8: every tile amax a (positive finite BF16) with every |x| <= a
+    if which in (0, 2):
+        # every divisor's amax a (positive finite BF16) with every |x| <= a
         assert n == sum(2 * (a + 1) for a in range(1, 0x7F80))
     else:
         assert n > 65280 * 0x7F7F
