@@ -225,6 +225,32 @@ pwq_status nvfp4_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_sibl
                             const float* amax_in, float* amax_out, void* workspace,
                             size_t workspace_bytes, pwq_stream_t stream);
 
+/* nvfp4_fake_quant_noalloc
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory.  Such callers include code running
+ * inside a framework or plugin host that owns all device memory and offers
+ * no allocator, real-time loops that forbid allocation after start-up, and
+ * steps where a cudaMalloc would be unacceptable because it can implicitly
+ * synchronise the device.  It computes exactly what nvfp4_fake_quant
+ * computes, with the same arguments minus the workspace: the per-group amax
+ * scratch lives in a file-scope device array of the library instead.
+ * Limits and behaviour:
+ *   - at most 4096 groups (batch) per call when amax_in is NULL; larger
+ *     batches return PWQ_ERR_SHAPE (with amax_in the scratch is unused);
+ *   - the array takes 16 KB on every device that loads the library, held
+ *     until the process exits;
+ *   - the first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture;
+ *   - every call shares the one array and it keeps the last call's contents
+ *     (each call clears the words it needs before using them), so calls
+ *     that may overlap on the GPU -- on different streams without ordering
+ *     between them, or from several host threads -- race: order them;
+ *   - it calls no cudaMalloc, cudaFree or other allocating routine.
+ * Errors as nvfp4_fake_quant, except that there is no PWQ_ERR_WORKSPACE. */
+pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, int n_siblings,
+                                    const float* amax_in, float* amax_out, pwq_stream_t stream);
+
 /* ===================================================================== */
 /* Diagnostics                                                            */
 /* ===================================================================== */

@@ -23,6 +23,7 @@
 // which the self-test proves to give IEEE division's codes over every BF16
 // numerator and every reachable divisor.
 #include <algorithm>
+#include <mutex>
 
 #include "pwq_internal.h"
 
@@ -366,6 +367,35 @@ cudaError_t launch_nvfp4_dequant(const View& q, const uint8_t* sb, const float* 
     const int grid = persistent_grid((a.total + span - 1) / span, 8);
     nvfp4_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- scratch for callers that cannot allocate
+
+// Group-amax scratch of nvfp4_fake_quant_noalloc: one word per group, in a
+// file-scope device array.  Every device that loads the library holds these
+// kStaticScratchGroups * 4 bytes until the process exits.
+__device__ __align__(256) uint32_t g_static_amax[kStaticScratchGroups];
+
+cudaError_t static_amax_scratch(uint32_t** ptr) {
+    // In host code g_static_amax names a host-side stand-in, not the device
+    // array: the device address is looked up once per device, with that
+    // device current, and cached.
+    constexpr int kMaxDevices = 64;
+    static uint32_t* addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_amax);
+        if (e != cudaSuccess) return e;
+        addr[dev] = static_cast<uint32_t*>(p);
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
 }
 
 }  // namespace pwq

@@ -411,6 +411,62 @@ pwq_status nvfp4_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_sibl
                                               amax_in, nullptr, amax_out, s));
 }
 
+// ------------------------------------------------------------------ no-allocation variant
+
+// nvfp4_fake_quant with the group-amax scratch in a file-scope device array
+// (csrc/nvfp4.cu) instead of caller workspace; see include/pwq.h.
+pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, int n_siblings,
+                                    const float* amax_in, float* amax_out, pwq_stream_t stream) {
+    View vx[PWQ_MAX_SIBLINGS], vy[PWQ_MAX_SIBLINGS];
+    Extent ex[PWQ_MAX_SIBLINGS + 1], ey[PWQ_MAX_SIBLINGS];
+    bool all_empty;
+    pwq_status st = check_siblings(x, n_siblings, vx, ex, &all_empty);
+    if (st != PWQ_OK) return st;
+    if (!y) return fail(PWQ_ERR_NULL, "y");
+    for (int i = 0; i < n_siblings; ++i) {
+        if (!same_shape(&x[i], &y[i])) return fail(PWQ_ERR_SHAPE, "y[i] shape != x[i] shape");
+        if ((st = check_tensor(&y[i], Kind::kBF16, &vy[i], &ey[i], "y[i]")) != PWQ_OK) return st;
+    }
+    if (all_empty || x[0].batch == 0) return PWQ_OK;
+    const int64_t B = x[0].batch;
+    if (!amax_in && B > pwq::kStaticScratchGroups)
+        return fail(PWQ_ERR_SHAPE, "batch exceeds the 4096-group static scratch of nvfp4_fake_quant_noalloc");
+    for (int i = 0; i < n_siblings; ++i) {
+        for (int j = 0; j < n_siblings; ++j) {
+            if (i == j && exact_alias(&x[i], &y[i])) continue;
+            if (overlaps(ey[i], ex[j])) return fail(PWQ_ERR_OVERLAP, "y[i] overlaps an input");
+        }
+        for (int j = i + 1; j < n_siblings; ++j)
+            if (overlaps(ey[i], ey[j])) return fail(PWQ_ERR_OVERLAP, "two outputs overlap");
+    }
+    int n_in = n_siblings;
+    if (amax_in) {
+        if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
+        ex[n_in++] = extent_of(amax_in, (size_t)B * 4);
+    }
+    if (amax_out) {
+        if ((uintptr_t)amax_out % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_out");
+        const Extent eo = extent_of(amax_out, (size_t)B * 4);
+        for (int j = 0; j < n_in; ++j)
+            if (overlaps(eo, ex[j])) return fail(PWQ_ERR_OVERLAP, "amax_out overlaps an input");
+        for (int i = 0; i < n_siblings; ++i)
+            if (overlaps(eo, ey[i])) return fail(PWQ_ERR_OVERLAP, "amax_out overlaps y");
+    }
+    if (amax_in)
+        for (int i = 0; i < n_siblings; ++i)
+            if (overlaps(ey[i], ex[n_siblings])) return fail(PWQ_ERR_OVERLAP, "y overlaps amax_in");
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t* amax_bits = nullptr;
+    if (!amax_in) {
+        cudaError_t e = pwq::static_amax_scratch(&amax_bits);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = pwq::launch_nvfp4_amax(vx, n_siblings, amax_bits, s);  // clears the words first
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return from_cuda(pwq::launch_nvfp4_encode(vx, n_siblings, vy, nullptr, true, amax_bits, amax_in, nullptr,
+                                              amax_out, s));
+}
+
 // ------------------------------------------------------------------ self-tests
 
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream) {

@@ -37,6 +37,11 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
 cudaError_t launch_nvfp4_dequant(const View& q, const uint8_t* sb, const float* gs, const View& y,
                                  cudaStream_t s);
 
+// Device address (on the current device) of the file-scope group-amax
+// scratch used by nvfp4_fake_quant_noalloc; kStaticScratchGroups words.
+constexpr int64_t kStaticScratchGroups = 4096;
+cudaError_t static_amax_scratch(uint32_t** ptr);
+
 // Reads and clears the device error word (synchronous).
 cudaError_t read_and_clear_device_error(uint32_t* code);
 

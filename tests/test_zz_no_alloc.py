@@ -1,0 +1,51 @@
+"""GPU test of nvfp4_fake_quant_noalloc, the entry point for callers that
+cannot allocate device memory (for example code inside a framework or plugin
+host that owns all device memory, or a step where cudaMalloc's implicit
+synchronisation is not acceptable).  It must give exactly what the
+workspace-taking nvfp4_fake_quant gives.
+
+Two calls in a row: the second group's amax is far smaller than the first's,
+so a scratch array that still held the first call's maxima would change the
+second call's output.  The file is named so that pytest collects it last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_entry_point_matches_workspace_entry_point_twice():
+    import precision_weight_quantization_b200 as P
+    from precision_weight_quantization_b200._lib import PwqTensor, lib
+
+    f = lib.nvfp4_fake_quant_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.POINTER(PwqTensor), ctypes.POINTER(PwqTensor), ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    dev = torch.device("cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    for call, (seed, std) in enumerate(((11, 40.0), (12, 0.003))):
+        # a batched sibling pair: 3 groups, each {x0[b], x1[b]}
+        xs = [W.random_bf16((3, 64, 512), seed=seed, std=std, device=dev),
+              W.random_bf16((3, 32, 512), seed=seed + 100, std=std, device=dev)]
+        ys = [torch.full_like(x, float("nan")) for x in xs]
+        amax_out = torch.full((3,), -1.0, dtype=torch.float32, device=dev)
+        ax = (PwqTensor * 2)(*[P._desc(x, "x") for x in xs])
+        ay = (PwqTensor * 2)(*[P._desc(y, "y") for y in ys])
+        st = f(ax, ay, 2, None, amax_out.data_ptr(), stream)
+        assert st == 0, (call, P.status_string(st), lib.pwq_last_error_detail().decode())
+
+        ref_amax = torch.empty(3, dtype=torch.float32, device=dev)
+        ref = P.nvfp4_fake_quant(xs, amax_out=ref_amax)
+        torch.cuda.synchronize()
+        # tolerance 0: bit-identical BF16 outputs and amax
+        for y, r in zip(ys, ref):
+            assert torch.equal(y.view(torch.int16), r.view(torch.int16)), call
+        assert torch.equal(amax_out, ref_amax), call
+        expect = torch.stack([torch.maximum(xs[0][b].float().abs().max(), xs[1][b].float().abs().max())
+                              for b in range(3)])
+        assert torch.equal(amax_out, expect), call
