@@ -92,8 +92,7 @@ __device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
 // reciprocal r = RN(1/s): one product and one residual correction with
 // fused multiply-adds (Markstein's correction step; P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990).  The quotient's sign is set
-// from x, which keeps -0 / s = -0.
+// processor", IBM J. Res. Dev. 34(1), 1990).
 //
 // It is used for a whole tile or block when 2^-64 <= s <= 2^126 (then s and
 // r are normal).  Within that range:
@@ -105,14 +104,56 @@ __device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
 //                  last subnormal bits, and is never stored).
 // pwq_selftest_division checks both statements over every BF16 numerator
 // and every divisor the formats produce, against __fdiv_rn.
+//
+// Written with the negated numerator nx = -x and negated reciprocal nr = -r:
+//   q0 = nx * nr (= x * r),  e = q0 * s + nx (= q0 * s - x, exact),
+//   q  = e * nr + q0 (= q0 - e * r),
+// the same roundings as q0 + (x - q0 * s) * r, but the final product
+// (+0) * nr = -0 carries the sign of zero through: -0 / s gives -0 and +0 / s
+// gives +0 with no extra instruction.
 __device__ __forceinline__ float div_fast(float x, float s, float r) {
-    float q0 = __fmul_rn(x, r);
-    float res = __fmaf_rn(-q0, s, x);
-    float q = __fmaf_rn(res, r, q0);
-    return __uint_as_float(__float_as_uint(q) | (__float_as_uint(x) & 0x80000000u));
+    const float nx = -x, nr = -r;
+    const float q0 = __fmul_rn(nx, nr);
+    const float e = __fmaf_rn(q0, s, nx);
+    return __fmaf_rn(e, nr, q0);
 }
 
 __device__ __forceinline__ bool div_fast_ok(float s) { return s >= 0x1p-64f && s <= 0x1p126f; }
+
+// Packed binary32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes).
+__device__ __forceinline__ uint64_t f32x2_bits(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    return f32x2_bits(__float_as_uint(lo), __float_as_uint(hi));
+}
+__device__ __forceinline__ float2 f32x2_split(uint64_t v) {
+    float2 f;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+    return f;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// div_fast on the two BF16 values of a packed word w (low half first):
+// s2 = {s, s}, nr2 = {-r, -r}.  The negated numerators come straight from
+// the BF16 bits (widening and sign flip in one integer operation each).
+__device__ __forceinline__ float2 div_fast_bf16x2(uint32_t w, uint64_t s2, uint64_t nr2) {
+    const uint64_t nx = f32x2_bits((w << 16) + 0x80000000u, (w & 0xffff0000u) ^ 0x80000000u);
+    const uint64_t q0 = mul_f32x2(nx, nr2);
+    const uint64_t e = fma_f32x2(q0, s2, nx);
+    return f32x2_split(fma_f32x2(e, nr2, q0));
+}
 
 // Outside that range: IEEE division, with the zero-scale reading (s == 0
 // gives a zero of x's sign).
@@ -126,17 +167,23 @@ __device__ __forceinline__ float quotient(float x, float s, float r) {
     return kFast ? div_fast(x, s, r) : div_slow(x, s);
 }
 
+// The quotients of the two BF16 values of a packed word.
+template <bool kFast>
+__device__ __forceinline__ float2 quotient_bf16x2(uint32_t w, float s, float r) {
+    if (kFast) return div_fast_bf16x2(w, f32x2(s, s), f32x2(-r, -r));
+    return make_float2(div_slow(bf16_lo(w), s), div_slow(bf16_hi(w), s));
+}
+
 // The 8 quotients of a 16-byte BF16 chunk.
 template <bool kFast>
 __device__ __forceinline__ void quotients8(uint4 v, float s, float r, float q[8]) {
-    q[0] = quotient<kFast>(bf16_lo(v.x), s, r);
-    q[1] = quotient<kFast>(bf16_hi(v.x), s, r);
-    q[2] = quotient<kFast>(bf16_lo(v.y), s, r);
-    q[3] = quotient<kFast>(bf16_hi(v.y), s, r);
-    q[4] = quotient<kFast>(bf16_lo(v.z), s, r);
-    q[5] = quotient<kFast>(bf16_hi(v.z), s, r);
-    q[6] = quotient<kFast>(bf16_lo(v.w), s, r);
-    q[7] = quotient<kFast>(bf16_hi(v.w), s, r);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 p = quotient_bf16x2<kFast>(w[i], s, r);
+        q[2 * i] = p.x;
+        q[2 * i + 1] = p.y;
+    }
 }
 
 // ---------------------------------------------------------------- UE8M0

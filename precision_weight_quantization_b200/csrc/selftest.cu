@@ -50,20 +50,34 @@ __global__ void __launch_bounds__(kThreads) selftest_division_kernel(unsigned lo
     const float r = __frcp_rn(d);
     const bool fast = div_fast_ok(d);
     unsigned long long n = 0, code_bad = 0, quot_bad = 0, slow = 0;
-    for (uint32_t xb = threadIdx.x; xb < 65536u; xb += kThreads) {
-        if (!bf16_is_finite(xb)) continue;
-        const float x = __uint_as_float(xb << 16);
-        if (!(fabsf(x) <= xmax)) continue;
-        const float qf = fast ? quotient<true>(x, d, r) : quotient<false>(x, d, r);
-        const float qr = (d == 0.0f) ? __uint_as_float((xb << 16) & 0x80000000u) : __fdiv_rn(x, d);
-        ++n;
-        slow += !fast;
-        if (kWhich == 1)
-            code_bad += (e2m1x2(qf, 0.0f) & 0xfu) != (e2m1x2(qr, 0.0f) & 0xfu);
-        else
-            code_bad += (e4m3x2(qf, 0.0f) & 0xffu) != (e4m3x2(qr, 0.0f) & 0xffu);
-        const uint32_t ef = (__float_as_uint(qr) >> 23) & 0xffu;
-        if (ef != 0u && fabsf(x) >= 0x1p-100f) quot_bad += __float_as_uint(qf) != __float_as_uint(qr);
+    // numerators in BF16 pairs, through the same functions the kernels call:
+    // the packed pair path for code divisors, the scalar one for fl(6 gs)
+    for (uint32_t wi = threadIdx.x; wi < 32768u; wi += kThreads) {
+        const uint32_t w = (2u * wi) | ((2u * wi + 1u) << 16);
+        float2 qp;
+        if (kWhich == 2) {
+            qp.x = fast ? quotient<true>(bf16_lo(w), d, r) : quotient<false>(bf16_lo(w), d, r);
+            qp.y = fast ? quotient<true>(bf16_hi(w), d, r) : quotient<false>(bf16_hi(w), d, r);
+        } else {
+            qp = fast ? quotient_bf16x2<true>(w, d, r) : quotient_bf16x2<false>(w, d, r);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t xb = 2u * wi + (uint32_t)h;
+            if (!bf16_is_finite(xb)) continue;
+            const float x = __uint_as_float(xb << 16);
+            if (!(fabsf(x) <= xmax)) continue;
+            const float qf = h ? qp.y : qp.x;
+            const float qr = (d == 0.0f) ? __uint_as_float((xb << 16) & 0x80000000u) : __fdiv_rn(x, d);
+            ++n;
+            slow += !fast;
+            if (kWhich == 1)
+                code_bad += (e2m1x2(qf, 0.0f) & 0xfu) != (e2m1x2(qr, 0.0f) & 0xfu);
+            else
+                code_bad += (e4m3x2(qf, 0.0f) & 0xffu) != (e4m3x2(qr, 0.0f) & 0xffu);
+            const uint32_t ef = (__float_as_uint(qr) >> 23) & 0xffu;
+            if (ef != 0u && fabsf(x) >= 0x1p-100f) quot_bad += __float_as_uint(qf) != __float_as_uint(qr);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
