@@ -49,8 +49,9 @@ BYTES_PER_ELEM = {
     "nvfp4_fake_quant": 2 + 2,
 }
 # our kernels launched per call (memsets are not counted)
+# (NVFP4 quantise / fake-quantise is one single-pass kernel after a memset)
 KERNELS_PER_CALL = {"fp8_block_quant": 1, "fp8_block_dequant": 1, "mxfp8_quant": 1, "mxfp8_dequant": 1,
-                    "nvfp4_quant": 2, "nvfp4_dequant": 1, "nvfp4_fake_quant": 2}
+                    "nvfp4_quant": 1, "nvfp4_dequant": 1, "nvfp4_fake_quant": 1}
 OPS = list(BYTES_PER_ELEM)
 
 
@@ -63,6 +64,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=36)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-tensor", action="store_true",
+                    help="one call per tensor / sibling group instead of one grouped call per layer")
     return ap.parse_args()
 
 
@@ -174,8 +177,50 @@ class Buffers:
         self.y = {n: torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for n, x in layers[0].items()}
 
 
-def op_calls(op, layers, buf, P):
-    """Closures for every call of one op kind over all layers."""
+def op_calls(op, layers, buf, P, grouped=True):
+    """Closures for every call of one op kind over all layers: one grouped
+    call per layer (all 7 tensors / all 4 sibling groups in one launch), or
+    with grouped=False one call per tensor / per group."""
+    import workloads as W
+    if not grouped:
+        return op_calls_per_tensor(op, layers, buf, P)
+    calls = []
+    for i, lay in enumerate(layers):
+        names = list(lay)
+        if op == "fp8_block_quant":
+            calls.append(lambda xs=[lay[n] for n in names], q=[buf.fp8[i][n][0] for n in names],
+                         s=[buf.fp8[i][n][1] for n in names]: P.fp8_block_quant_grouped(xs, out=q, scale=s))
+        elif op == "fp8_block_dequant":
+            calls.append(lambda q=[buf.fp8[i][n][0] for n in names], s=[buf.fp8[i][n][1] for n in names],
+                         y=[buf.y[n] for n in names]: P.fp8_block_dequant_grouped(q, s, out=y))
+        elif op == "mxfp8_quant":
+            calls.append(lambda xs=[lay[n] for n in names], q=[buf.mx[i][n][0] for n in names],
+                         e=[buf.mx[i][n][1] for n in names]: P.mxfp8_quant_grouped(xs, out=q, scale=e))
+        elif op == "mxfp8_dequant":
+            calls.append(lambda q=[buf.mx[i][n][0] for n in names], e=[buf.mx[i][n][1] for n in names],
+                         y=[buf.y[n] for n in names]: P.mxfp8_dequant_grouped(q, e, out=y))
+        elif op == "nvfp4_quant":
+            gs_ = W.QWEN3_4B_GROUPS
+            calls.append(lambda xs=[[lay[n] for n in g] for g in gs_], pk=[buf.nv[i][g][0] for g in gs_],
+                         sb=[buf.nv[i][g][1] for g in gs_], gsc=[buf.nv[i][g][2] for g in gs_]:
+                         P.nvfp4_quant_grouped(xs, out=pk, sb=sb, global_scale=gsc))
+        elif op == "nvfp4_dequant":
+            pk, sb, gs, ys = [], [], [], []
+            for g in W.QWEN3_4B_GROUPS:
+                for k, n in enumerate(g):
+                    pk.append(buf.nv[i][g][0][k])
+                    sb.append(buf.nv[i][g][1][k])
+                    gs.append(buf.nv[i][g][2])
+                    ys.append(buf.y[n])
+            calls.append(lambda pk=pk, sb=sb, gs=gs, ys=ys: P.nvfp4_dequant_grouped(pk, sb, gs, out=ys))
+        elif op == "nvfp4_fake_quant":
+            gs_ = W.QWEN3_4B_GROUPS
+            calls.append(lambda xs=[[lay[n] for n in g] for g in gs_], ys=[[buf.y[n] for n in g] for g in gs_]:
+                         P.nvfp4_fake_quant_grouped(xs, out=ys))
+    return calls
+
+
+def op_calls_per_tensor(op, layers, buf, P):
     import workloads as W
     calls = []
     for i, lay in enumerate(layers):
@@ -291,8 +336,9 @@ def main():
     layers = make_layers(args.layers, dev, rank)
     buf = Buffers(layers, P, torch)
     elems_per_step = layer_elems() * args.layers
-    graphs = {op: capture(op_calls(op, layers, buf, P), torch) for op in OPS}
-    ncalls = {op: len(op_calls(op, layers[:1], buf, P)) * args.layers for op in OPS}
+    grouped = not args.per_tensor
+    graphs = {op: capture(op_calls(op, layers, buf, P, grouped), torch) for op in OPS}
+    ncalls = {op: len(op_calls(op, layers[:1], buf, P, grouped)) * args.layers for op in OPS}
     launches_per_step = sum(ncalls[op] * KERNELS_PER_CALL[op] for op in OPS)
 
     stream = torch.cuda.current_stream()
@@ -356,7 +402,8 @@ def main():
                        "path": "fp8_block q+dq, mxfp8 q+dq, nvfp4 q (qkv, gate/up siblings)+dq, "
                                "nvfp4 fake-quant (siblings)",
                        "l2": "inputs larger than L2 (7.3 GB per rank), no flush",
-                       "launch": "one CUDA graph per op kind, replayed back to back",
+                       "launch": ("one grouped call per op per layer" if grouped else "one call per tensor") +
+                                 "; one CUDA graph per op kind, replayed back to back",
                        "parallelism": "dp%d (independent sweeps)" % world},
             "per_op": per_op, "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary() if rank == 0 else None}

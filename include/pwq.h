@@ -173,14 +173,19 @@ pwq_status mxfp8_dequant(const pwq_tensor* q, const uint8_t* scale, const pwq_te
  * Packed codes: element 2j of a row in the low nibble of byte j, 2j+1 in
  * the high nibble; bit 3 of a nibble is the sign.
  *
- * Workspace.  When amax_in is NULL the group amax is reduced on the device
- * into caller-provided workspace of at least nvfp4_workspace_size() bytes
- * (256-byte aligned is best; 4-byte aligned is required).  Its contents on
- * entry do not matter.  When amax_in is given, workspace may be NULL.
+ * Single pass.  When amax_in is NULL, quantise and fake-quantise run as one
+ * launch: a queue of amax items and encode items, ordered so that the amax
+ * of the next group (or batch index) is reduced while the current one is
+ * encoded from data still in L2.  The per-group amax words, completion
+ * counters and queue head live in caller-provided workspace of at least
+ * nvfp4_workspace_size() / nvfp4_workspace_size_grouped() bytes (4-byte
+ * aligned; 256-byte aligned is best).  Its contents on entry do not matter.
+ * When amax_in is given, workspace may be NULL.
  */
 
-/* Bytes of workspace an NVFP4 call over these siblings needs (4 * B rounded
- * up to 256).  x points to n_siblings descriptors; returns 0 on bad input. */
+/* Bytes of workspace an NVFP4 quantise / fake-quantise call over these
+ * siblings needs: 4 * (2 * min(B, 2048) + 1), rounded up to 256.  x points
+ * to n_siblings descriptors; returns 0 on bad input. */
 size_t nvfp4_workspace_size(int n_siblings, const pwq_tensor* x);
 
 /* nvfp4_group_amax: A_b for every group, as FP32, into amax_out[B] (device).
@@ -225,6 +230,56 @@ pwq_status nvfp4_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_sibl
                             const float* amax_in, float* amax_out, void* workspace,
                             size_t workspace_bytes, pwq_stream_t stream);
 
+/* ===================================================================== */
+/* Grouped calls: a list of independent tensors in one launch             */
+/* ===================================================================== */
+/*
+ * Source: verl NVFP4 QAT article, section 2.5 (the exporter buffers one
+ * decoder layer's parameters and quantises the layer at once) and section
+ * 3.3 (per-parameter export inside the weight-update stream); "Low Precision
+ * RL", "Unified training recipe" (weights re-quantised on every weight
+ * update).  Each grouped call computes exactly what the single-tensor call
+ * computes for every tensor of the list, with one kernel launch per
+ * PWQ_LAUNCH_TENSORS tensors, so small tensors (k/v projections) no longer
+ * pay a launch and a ramp each.  n is the list length (0 .. PWQ_MAX_GROUPED;
+ * 0 is a no-op); x, q, y are host arrays of n descriptors; scale, sb and
+ * global_scale are host arrays of n device pointers with the per-tensor
+ * layouts of the single-tensor calls.  No output may overlap any input or
+ * another output of the list.  Errors: as the single-tensor calls, plus
+ * PWQ_ERR_ARG for n out of range.
+ */
+#define PWQ_MAX_GROUPED 256
+#define PWQ_LAUNCH_TENSORS 16
+
+pwq_status fp8_block_quant_grouped(int n, const pwq_tensor* x, const pwq_tensor* q,
+                                   float* const* scale, pwq_stream_t stream);
+pwq_status fp8_block_dequant_grouped(int n, const pwq_tensor* q, const float* const* scale,
+                                     const pwq_tensor* y, pwq_stream_t stream);
+pwq_status mxfp8_quant_grouped(int n, const pwq_tensor* x, const pwq_tensor* q,
+                               uint8_t* const* scale, pwq_stream_t stream);
+pwq_status mxfp8_dequant_grouped(int n, const pwq_tensor* q, const uint8_t* const* scale,
+                                 const pwq_tensor* y, pwq_stream_t stream);
+pwq_status nvfp4_dequant_grouped(int n, const pwq_tensor* q_packed, const uint8_t* const* sb,
+                                 const float* const* global_scale, const pwq_tensor* y,
+                                 pwq_stream_t stream);
+
+/* NVFP4 over several sibling groups (e.g. {q,k,v}, {o}, {gate,up}, {down}
+ * of one layer): group g has group_sizes[g] consecutive members of x (and
+ * of q_packed / sb / y), 1 <= group_sizes[g] <= PWQ_MAX_SIBLINGS, at most
+ * PWQ_MAX_GROUPED members in all; members of a group share one batch B_g and
+ * one amax per batch index.  global_scale[g] (quantise) and amax_out[g]
+ * (fake-quantise; the array or any entry may be NULL) are per-group FP32
+ * [B_g] device arrays.  The amax is always reduced on the device: workspace
+ * of at least nvfp4_workspace_size_grouped() bytes is required. */
+size_t nvfp4_workspace_size_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x);
+pwq_status nvfp4_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                               const pwq_tensor* q_packed, uint8_t* const* sb,
+                               float* const* global_scale, void* workspace,
+                               size_t workspace_bytes, pwq_stream_t stream);
+pwq_status nvfp4_fake_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                                    const pwq_tensor* y, float* const* amax_out, void* workspace,
+                                    size_t workspace_bytes, pwq_stream_t stream);
+
 /* nvfp4_fake_quant_noalloc
  * The pages have no counterpart to this entry point; it exists for callers
  * that cannot allocate device memory.  Such callers include code running
@@ -267,7 +322,8 @@ const char* pwq_last_error_detail(void);
 const char* pwq_build_info(void);
 
 /* Reads and clears the device-side error word of the current device
- * (synchronous; 0 = no error; bit 0 = a TMA load wait gave up).  Returns
+ * (synchronous; 0 = no error; bit 0 = a TMA load wait gave up, bit 1 = an
+ * NVFP4 single-pass encode item gave up waiting for its group amax).  Returns
  * PWQ_ERR_NULL or PWQ_ERR_CUDA on failure. */
 pwq_status pwq_device_error(uint32_t* code);
 
@@ -281,6 +337,10 @@ pwq_status pwq_device_error(uint32_t* code);
  *              numerators |x| <= 16 d.  Compares E2M1 codes.
  *   which = 2  NVFP4 block-scale divisor fl(6 * fl(a / 2688)); numerators
  *              |x| <= a.  Compares E4M3 codes.
+ *   which = 3  FP8 tile scale s = fl(a / 448) as the kernels form it, for
+ *              every BF16 amax a >= 0: [0] = values checked, [1] = [2] =
+ *              binary32 mismatches against __fdiv_rn (s is stored, so it
+ *              must be exact), [3] = values taking the IEEE path.
  * counts (device, 4 x uint64, zeroed by the call): [0] pairs checked,
  * [1] code mismatches, [2] binary32 quotient mismatches where |x| >= 2^-100
  * and the IEEE quotient is normal, [3] pairs whose divisor takes the

@@ -24,7 +24,9 @@ __all__ = [
     "fp8_block_quant", "fp8_block_dequant", "mxfp8_quant", "mxfp8_dequant",
     "nvfp4_group_amax", "nvfp4_quant", "nvfp4_dequant", "nvfp4_fake_quant",
     "nvfp4_workspace_size", "NVFP4FakeQuantSTE", "nvfp4_fake_quant_ste", "build_info",
-    "device_error", "PwqError", "LIB_PATH",
+    "device_error", "PwqError", "LIB_PATH", "fp8_block_quant_grouped", "fp8_block_dequant_grouped",
+    "mxfp8_quant_grouped", "mxfp8_dequant_grouped", "nvfp4_dequant_grouped", "nvfp4_quant_grouped",
+    "nvfp4_fake_quant_grouped",
 ]
 
 _CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
@@ -268,6 +270,123 @@ def nvfp4_fake_quant_ste(xs: Sequence[torch.Tensor], amax: Optional[torch.Tensor
     if isinstance(xs, torch.Tensor):
         return NVFP4FakeQuantSTE.apply(xs, amax)
     return list(_SiblingSTE.apply(amax, *xs))
+
+
+# ---------------------------------------------------------------- grouped calls (one launch per list)
+
+def _ptrs(ts):
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def fp8_block_quant_grouped(xs: Sequence[torch.Tensor], out=None, scale=None):
+    """fp8_block_quant of every tensor of a list (a layer's weights) in one
+    launch.  Returns (codes list, scales list)."""
+    xs = list(xs)
+    for i, x in enumerate(xs):
+        _check_dtype(x, (torch.bfloat16,), "x[%d]" % i)
+    if out is None:
+        out = [torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device) for x in xs]
+    if scale is None:
+        scale = [torch.empty(_lead(x) + (-(-x.shape[-2] // 128), -(-x.shape[-1] // 128)), dtype=torch.float32,
+                             device=x.device) for x in xs]
+    if xs:
+        check(lib.fp8_block_quant_grouped(len(xs), _desc_array(xs, "x"), _desc_array(out, "out"), _ptrs(scale),
+                                          _stream(xs[0])), "fp8_block_quant_grouped")
+    return out, scale
+
+
+def fp8_block_dequant_grouped(qs: Sequence[torch.Tensor], scales: Sequence[torch.Tensor], out=None):
+    qs = list(qs)
+    if out is None:
+        out = [torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) for q in qs]
+    if qs:
+        check(lib.fp8_block_dequant_grouped(len(qs), _desc_array(qs, "q"), _ptrs(scales), _desc_array(out, "out"),
+                                            _stream(qs[0])), "fp8_block_dequant_grouped")
+    return out
+
+
+def mxfp8_quant_grouped(xs: Sequence[torch.Tensor], out=None, scale=None):
+    xs = list(xs)
+    if out is None:
+        out = [torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device) for x in xs]
+    if scale is None:
+        scale = [torch.empty(x.shape[:-1] + (x.shape[-1] // 32,), dtype=torch.uint8, device=x.device) for x in xs]
+    if xs:
+        check(lib.mxfp8_quant_grouped(len(xs), _desc_array(xs, "x"), _desc_array(out, "out"), _ptrs(scale),
+                                      _stream(xs[0])), "mxfp8_quant_grouped")
+    return out, scale
+
+
+def mxfp8_dequant_grouped(qs: Sequence[torch.Tensor], scales: Sequence[torch.Tensor], out=None):
+    qs = list(qs)
+    if out is None:
+        out = [torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) for q in qs]
+    if qs:
+        check(lib.mxfp8_dequant_grouped(len(qs), _desc_array(qs, "q"), _ptrs(scales), _desc_array(out, "out"),
+                                        _stream(qs[0])), "mxfp8_dequant_grouped")
+    return out
+
+
+def nvfp4_dequant_grouped(packed: Sequence[torch.Tensor], sb: Sequence[torch.Tensor],
+                          global_scale: Sequence[torch.Tensor], out=None):
+    packed = list(packed)
+    if out is None:
+        out = [torch.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=torch.bfloat16, device=p.device)
+               for p in packed]
+    if packed:
+        check(lib.nvfp4_dequant_grouped(len(packed), _desc_array(packed, "packed", packed=True), _ptrs(sb),
+                                        _ptrs(global_scale), _desc_array(out, "out"), _stream(packed[0])),
+              "nvfp4_dequant_grouped")
+    return out
+
+
+def _groups(groups):
+    groups = [_siblings(g) for g in groups]
+    flat = [x for g in groups for x in g]
+    sizes = (ctypes.c_int * len(groups))(*[len(g) for g in groups])
+    return groups, flat, sizes
+
+
+def nvfp4_quant_grouped(groups: Sequence[Sequence[torch.Tensor]], out=None, sb=None, global_scale=None):
+    """NVFP4 quantisation of several sibling groups (e.g. a layer's {q,k,v},
+    {o}, {gate,up}, {down}) in one single-pass launch.  Returns (packed
+    codes per group, block scales per group, global scales per group)."""
+    groups, flat, sizes = _groups(groups)
+    dev = flat[0].device
+    if out is None:
+        out = [[torch.empty(x.shape[:-1] + (x.shape[-1] // 2,), dtype=torch.uint8, device=dev) for x in g]
+               for g in groups]
+    if sb is None:
+        sb = [[torch.empty(x.shape[:-1] + (x.shape[-1] // 16,), dtype=torch.float8_e4m3fn, device=dev) for x in g]
+              for g in groups]
+    if global_scale is None:
+        global_scale = [torch.empty(_batch(g[0]), dtype=torch.float32, device=dev) for g in groups]
+    ax = _desc_array(flat, "x")
+    ws_bytes = int(lib.nvfp4_workspace_size_grouped(len(groups), sizes, ax))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    check(lib.nvfp4_quant_grouped(len(groups), sizes, ax, _desc_array([p for g in out for p in g], "out", packed=True),
+                                  _ptrs([s for g in sb for s in g]), _ptrs(global_scale), ws.data_ptr(), ws.numel(),
+                                  _stream(flat[0])), "nvfp4_quant_grouped")
+    return out, sb, global_scale
+
+
+def nvfp4_fake_quant_grouped(groups: Sequence[Sequence[torch.Tensor]], out=None, inplace: bool = False,
+                             amax_out=None):
+    """NVFP4 fake-quantisation of several sibling groups in one single-pass
+    launch.  Returns the BF16 outputs per group."""
+    groups, flat, sizes = _groups(groups)
+    dev = flat[0].device
+    if out is None:
+        out = groups if inplace else [[torch.empty_like(x) for x in g] for g in groups]
+    ax = _desc_array(flat, "x")
+    ws_bytes = int(lib.nvfp4_workspace_size_grouped(len(groups), sizes, ax))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    ao = None
+    if amax_out is not None:
+        ao = (ctypes.c_void_p * len(groups))(*[a.data_ptr() if a is not None else None for a in amax_out])
+    check(lib.nvfp4_fake_quant_grouped(len(groups), sizes, ax, _desc_array([y for g in out for y in g], "out"), ao,
+                                       ws.data_ptr(), ws.numel(), _stream(flat[0])), "nvfp4_fake_quant_grouped")
+    return out
 
 
 # ---------------------------------------------------------------- diagnostics

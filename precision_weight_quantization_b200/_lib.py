@@ -39,6 +39,8 @@ class PwqError(RuntimeError):
 _P = ctypes.c_void_p
 _T = ctypes.POINTER(PwqTensor)
 _S = ctypes.c_int
+_PP = ctypes.POINTER(ctypes.c_void_p)
+_IP = ctypes.POINTER(ctypes.c_int)
 _SIG = {
     "fp8_block_quant": (_S, [_T, _T, _P, _P]),
     "fp8_block_dequant": (_S, [_T, _P, _T, _P]),
@@ -50,6 +52,14 @@ _SIG = {
                          ctypes.c_size_t, _P]),
     "nvfp4_dequant": (_S, [_T, _P, _P, _T, _P]),
     "nvfp4_fake_quant": (_S, [_T, _T, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
+    "fp8_block_quant_grouped": (_S, [ctypes.c_int, _T, _T, _PP, _P]),
+    "fp8_block_dequant_grouped": (_S, [ctypes.c_int, _T, _PP, _T, _P]),
+    "mxfp8_quant_grouped": (_S, [ctypes.c_int, _T, _T, _PP, _P]),
+    "mxfp8_dequant_grouped": (_S, [ctypes.c_int, _T, _PP, _T, _P]),
+    "nvfp4_dequant_grouped": (_S, [ctypes.c_int, _T, _PP, _PP, _T, _P]),
+    "nvfp4_workspace_size_grouped": (ctypes.c_size_t, [ctypes.c_int, _IP, _T]),
+    "nvfp4_quant_grouped": (_S, [ctypes.c_int, _IP, _T, _T, _PP, _PP, _P, ctypes.c_size_t, _P]),
+    "nvfp4_fake_quant_grouped": (_S, [ctypes.c_int, _IP, _T, _T, _PP, _P, ctypes.c_size_t, _P]),
     "pwq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "pwq_last_error_detail": (ctypes.c_char_p, []),
     "pwq_build_info": (ctypes.c_char_p, []),

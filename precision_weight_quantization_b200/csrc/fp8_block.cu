@@ -5,16 +5,20 @@
 // "低精度训练与 Rollout", "FP8 训练 + FP8 Rollout" (FP32 block scales; FP8
 // weights dequantised to BF16 on weight update).
 //
-// Quantise: a persistent grid (2 CTAs per SM) walks the tiles.  Each tile is
-// brought into shared memory by one 3-D TMA box load (cp.async.bulk.tensor,
-// no multicast) whose out-of-range part is zero-filled -- zeros never raise
-// the amax, so ragged edge tiles need no masking on the load side.  A ring
-// of kStages tile buffers keeps the next tiles in flight while the current
-// one is reduced: every thread copies its 64 elements to registers, the CTA
-// reduces the tile amax (shuffles + one barrier), the freed buffer is
-// immediately refilled, and the codes are computed from registers with one
-// correctly rounded reciprocal per tile plus an FMA residual correction per
-// element (proved equal to IEEE division by the exhaustive self-test).
+// Both kernels take a list of up to kMaxLaunchTensors independent tensors
+// (one decoder layer's weights, say) and walk the concatenation of their
+// tiles with a persistent grid, so a whole list costs one launch.
+//
+// Quantise: 2 CTAs per SM.  Each tile is brought into shared memory by one
+// 3-D TMA box load (cp.async.bulk.tensor, no multicast) from its tensor's
+// map; the out-of-range part of an edge tile is zero-filled, and zeros never
+// raise the amax, so the load side needs no masking.  A ring of kStages tile
+// buffers keeps the next tiles in flight while the current one is reduced:
+// every thread copies its 64 elements to registers, one barrier publishes
+// the warp maxima and frees the buffer, which is refilled at once, and the
+// codes are computed from registers with one correctly rounded reciprocal
+// per tile plus an FMA residual correction per element (proved to give the
+// IEEE-division codes by the exhaustive self-test).
 #include <algorithm>
 #include <cuda.h>
 
@@ -34,30 +38,49 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // gave up).  Read and cleared by pwq_device_error().
 __device__ uint32_t g_device_error = 0u;
 
-struct QuantArgs {
-    char* q;
-    int64_t q_bs, q_rs;   // bytes
+// One tensor of a grouped launch (byte strides).
+struct TileTensor {
+    char* q;              // E4M3 codes: quant output, dequant input
+    char* y;              // dequant: BF16 output
+    int64_t q_bs, q_rs, y_bs, y_rs;
     float* scale;         // dense [B][TM][TN]
     int rows, cols;
-    int tiles_m, tiles_n;
-    uint32_t total_tiles;
+    uint32_t tile_begin;  // first tile of this tensor in the launch
+    FastDiv tiles_n;      // tiles per tile row (TN)
+    FastDiv tiles_mn;     // tiles per batch matrix (TM * TN)
+    int vec16;            // dequant: code rows 16-byte aligned
 };
 
-__device__ __forceinline__ void tile_coords(uint32_t t, const QuantArgs& a, int& b, int& tm, int& tn) {
-    const uint32_t per_b = (uint32_t)a.tiles_m * (uint32_t)a.tiles_n;
-    b = (int)(t / per_b);
-    const uint32_t rem = t - (uint32_t)b * per_b;
-    tm = (int)(rem / (uint32_t)a.tiles_n);
-    tn = (int)(rem - (uint32_t)tm * (uint32_t)a.tiles_n);
+struct TileLoc {
+    int i;                // tensor
+    uint32_t lt;          // tile within the tensor (= its scale index)
+    int b, tm, tn;
+};
+
+template <class Args>
+__device__ __forceinline__ TileLoc locate(const Args& a, uint32_t tile) {
+    int i = 0;
+    for (int k = 1; k < a.n; ++k)
+        if (tile >= a.t[k].tile_begin) i = k;
+    const TileTensor& T = a.t[i];
+    TileLoc L;
+    L.i = i;
+    L.lt = tile - T.tile_begin;
+    const uint32_t b = fdiv(L.lt, T.tiles_mn);
+    const uint32_t rem = L.lt - b * T.tiles_mn.d;
+    const uint32_t tm = fdiv(rem, T.tiles_n);
+    L.b = (int)b;
+    L.tm = (int)tm;
+    L.tn = (int)(rem - tm * T.tiles_n.d);
+    return L;
 }
 
-__device__ __forceinline__ void issue_tile(const CUtensorMap* tmap, uint32_t dst, uint32_t bar, uint32_t t,
-                                           const QuantArgs& a) {
-    int b, tm, tn;
-    tile_coords(t, a, b, tm, tn);
-    mbar_arrive_expect_tx(bar, kTileBytes);
-    tma_load_3d(dst, tmap, bar, tn * kTile, tm * kTile, b);
-}
+struct QuantArgs {
+    CUtensorMap tmap[kMaxLaunchTensors];
+    TileTensor t[kMaxLaunchTensors];
+    int n;
+    uint32_t total_tiles;
+};
 
 // E4M3 codes of a thread's 8 chunks (64 elements) for tile scale s with
 // r = RN(1/s); kFast selects the reciprocal path for the whole tile.
@@ -74,9 +97,10 @@ __device__ __forceinline__ void encode_chunks(const uint4 (&v)[kChunksPerThread]
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
-fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs a) {
-    extern __shared__ __align__(1024) unsigned char smem[];
+fp8_block_quant_kernel(const __grid_constant__ QuantArgs a) {
+    extern __shared__ unsigned char smem[];
     __shared__ __align__(8) uint64_t bars[kStages];
+    __shared__ TileLoc meta[kStages];
     __shared__ uint32_t red[2][kThreads / 32];
 
     const uint32_t tid = threadIdx.x;
@@ -90,11 +114,21 @@ fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs
     }
     __syncthreads();
 
+    // thread 0 locates a tile, records it for the consumers (visible to them
+    // once they observe the barrier phase) and starts its TMA load
+    auto issue = [&](uint32_t t, uint32_t s) {
+        const TileLoc L = locate(a, t);
+        meta[s] = L;
+        const uint32_t bar = smem_addr(&bars[s]);
+        mbar_arrive_expect_tx(bar, kTileBytes);
+        tma_load_3d(smem0 + s * kTileBytes, &a.tmap[L.i], bar, L.tn * kTile, L.tm * kTile, L.b);
+    };
+
     const uint32_t first = blockIdx.x, step = gridDim.x;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             const uint32_t t = first + (uint32_t)s * step;
-            if (t < a.total_tiles) issue_tile(&tmap, smem0 + s * kTileBytes, smem_addr(&bars[s]), t, a);
+            if (t < a.total_tiles) issue(t, (uint32_t)s);
         }
     }
 
@@ -109,6 +143,7 @@ fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs
         const uint32_t parity = (it / kStages) & 1u;
         const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity, kWaitLimitNs);
         const unsigned char* buf = ring + s * kTileBytes;
+        const TileLoc L = meta[s];
         uint4 v[kChunksPerThread];
         uint32_t m = 0u;
 #pragma unroll
@@ -121,7 +156,7 @@ fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((tid & 31u) == 0u) red[it & 1u][tid >> 5] = m;
         // one barrier: publishes the warp maxima, ends every read of buffer
-        // s, and makes a timed-out wait a CTA-uniform decision
+        // s and of meta[s], and makes a timed-out wait a CTA-uniform decision
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 atomicOr(&g_device_error, kErrTmaTimeout);
@@ -136,14 +171,13 @@ fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs
         }
         if (tid == 0) {
             const uint32_t tn = t + (uint32_t)kStages * step;
-            if (tn < a.total_tiles) issue_tile(&tmap, smem0 + s * kTileBytes, smem_addr(&bars[s]), tn, a);
+            if (tn < a.total_tiles) issue(tn, s);
         }
         uint32_t am = red[it & 1u][0];
 #pragma unroll
         for (int w = 1; w < kThreads / 32; ++w) am = max(am, red[it & 1u][w]);
 
-        const float amax = __uint_as_float(am << 16);
-        const float sc = __fdiv_rn(amax, 448.0f);
+        const float sc = fp8_tile_scale(__uint_as_float(am << 16));
         const float rc = __frcp_rn(sc);
         uint2 out[kChunksPerThread];
         if (div_fast_ok(sc))   // CTA-uniform
@@ -151,22 +185,21 @@ fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs
         else
             encode_chunks<false>(v, sc, rc, out);
 
-        int b, tm, tn;
-        tile_coords(t, a, b, tm, tn);
-        if (tid == 0) a.scale[t] = sc;
-        const int rows_here = min(kTile, a.rows - tm * kTile);
-        const int cols_here = min(kTile, a.cols - tn * kTile);
-        char* qtile = a.q + (int64_t)b * a.q_bs + (int64_t)tm * kTile * a.q_rs + (int64_t)tn * kTile;
+        const TileTensor& T = a.t[L.i];
+        if (tid == 0) T.scale[L.lt] = sc;
+        const int rows_here = min(kTile, T.rows - L.tm * kTile);
+        const int cols_here = min(kTile, T.cols - L.tn * kTile);
+        char* qtile = T.q + (int64_t)L.b * T.q_bs + (int64_t)L.tm * kTile * T.q_rs + (int64_t)L.tn * kTile;
         if (rows_here == kTile && cols_here == kTile) {
 #pragma unroll
             for (int j = 0; j < kChunksPerThread; ++j)
-                st_v2(qtile + (int64_t)(row0 + 16 * j) * a.q_rs + ccol, out[j]);
+                st_v2(qtile + (int64_t)(row0 + 16 * j) * T.q_rs + ccol, out[j]);
         } else {
 #pragma unroll
             for (int j = 0; j < kChunksPerThread; ++j) {
                 const int r = row0 + 16 * j;
                 if (r >= rows_here || ccol >= cols_here) continue;
-                char* dst = qtile + (int64_t)r * a.q_rs + ccol;
+                char* dst = qtile + (int64_t)r * T.q_rs + ccol;
                 if (ccol + 8 <= cols_here) {
                     st_v2(dst, out[j]);
                 } else {
@@ -178,18 +211,14 @@ fp8_block_quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantArgs
     }
 }
 
-// Dequantise: a persistent grid walks the tiles; the tile scale is one
-// load per tile.  Thread t owns 16-code chunks at column (t & 7) * 16 of
-// rows (t >> 3) + 32 j, j = 0..3: a 16-byte code load becomes two 16-byte
+// Dequantise: a persistent grid walks the tiles of the list; the tile scale
+// is one load per tile.  Thread t owns 16-code chunks at column (t & 7) * 16
+// of rows (t >> 3) + 32 j, j = 0..3: a 16-byte code load becomes two 16-byte
 // BF16 stores.  Edge tiles take a masked element-wise path.
 struct DequantArgs {
-    const char* q;
-    char* y;
-    const float* scale;   // dense [B][TM][TN]
-    int64_t q_bs, q_rs, y_bs, y_rs;  // bytes
-    int rows, cols, tiles_m, tiles_n;
+    TileTensor t[kMaxLaunchTensors];
+    int n;
     uint32_t total_tiles;
-    int vec16;            // code rows 16-byte aligned (else two 8-byte loads)
 };
 
 constexpr int kDqRowsPerPass = kThreads / 8;         // 32
@@ -206,26 +235,23 @@ __device__ __forceinline__ uint4 dequant8(uint2 codes, float s) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const DequantArgs a) {
+__global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const __grid_constant__ DequantArgs a) {
     const int ccol = (int)(threadIdx.x & 7u) * 16;
     const int row0 = (int)(threadIdx.x >> 3);
-    const uint32_t per_b = (uint32_t)a.tiles_m * (uint32_t)a.tiles_n;
     for (uint32_t t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
-        const uint32_t b = t / per_b;
-        const uint32_t rem = t - b * per_b;
-        const int tm = (int)(rem / (uint32_t)a.tiles_n);
-        const int tn = (int)(rem - (uint32_t)tm * (uint32_t)a.tiles_n);
-        const float sc = __ldg(a.scale + t);
-        const char* qt = a.q + (int64_t)b * a.q_bs + (int64_t)tm * kTile * a.q_rs + (int64_t)tn * kTile;
-        char* yt = a.y + (int64_t)b * a.y_bs + (int64_t)tm * kTile * a.y_rs + (int64_t)tn * kTile * 2;
-        const int rows_here = min(kTile, a.rows - tm * kTile);
-        const int cols_here = min(kTile, a.cols - tn * kTile);
+        const TileLoc L = locate(a, t);
+        const TileTensor& T = a.t[L.i];
+        const float sc = __ldg(T.scale + L.lt);
+        const char* qt = T.q + (int64_t)L.b * T.q_bs + (int64_t)L.tm * kTile * T.q_rs + (int64_t)L.tn * kTile;
+        char* yt = T.y + (int64_t)L.b * T.y_bs + (int64_t)L.tm * kTile * T.y_rs + (int64_t)L.tn * kTile * 2;
+        const int rows_here = min(kTile, T.rows - L.tm * kTile);
+        const int cols_here = min(kTile, T.cols - L.tn * kTile);
         if (rows_here == kTile && cols_here == kTile) {
             uint4 v[kDqChunks];
 #pragma unroll
             for (int j = 0; j < kDqChunks; ++j) {
-                const char* src = qt + (int64_t)(row0 + kDqRowsPerPass * j) * a.q_rs + ccol;
-                if (a.vec16) {
+                const char* src = qt + (int64_t)(row0 + kDqRowsPerPass * j) * T.q_rs + ccol;
+                if (T.vec16) {
                     v[j] = ld_stream_v4(src);
                 } else {
                     const uint2 lo = ld_stream_v2(src), hi = ld_stream_v2(src + 8);
@@ -234,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const Dequa
             }
 #pragma unroll
             for (int j = 0; j < kDqChunks; ++j) {
-                char* dst = yt + (int64_t)(row0 + kDqRowsPerPass * j) * a.y_rs + ccol * 2;
+                char* dst = yt + (int64_t)(row0 + kDqRowsPerPass * j) * T.y_rs + ccol * 2;
                 st_v4(dst, dequant8(make_uint2(v[j].x, v[j].y), sc));
                 st_v4(dst + 16, dequant8(make_uint2(v[j].z, v[j].w), sc));
             }
@@ -242,8 +268,8 @@ __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const Dequa
             for (int j = 0; j < kDqChunks; ++j) {
                 const int r = row0 + kDqRowsPerPass * j;
                 if (r >= rows_here) break;
-                const unsigned char* src = reinterpret_cast<const unsigned char*>(qt + (int64_t)r * a.q_rs);
-                unsigned short* dst = reinterpret_cast<unsigned short*>(yt + (int64_t)r * a.y_rs);
+                const unsigned char* src = reinterpret_cast<const unsigned char*>(qt + (int64_t)r * T.q_rs);
+                unsigned short* dst = reinterpret_cast<unsigned short*>(yt + (int64_t)r * T.y_rs);
                 for (int c = ccol; c < min(ccol + 16, cols_here); ++c) {
                     const float f = __fmul_rn(e4m3_decode(src[c]), sc);
                     dst[c] = (unsigned short)(pack_bf16x2(f, 0.0f) & 0xffffu);
@@ -273,6 +299,27 @@ EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
+// Fills the per-tensor descriptor; returns the tensor's tile count.
+uint32_t fill_tile_tensor(TileTensor& T, const Job& j, bool quant, uint32_t tile_begin) {
+    const View& q = quant ? j.out : j.in;
+    T.q = q.ptr;
+    T.q_bs = q.bstride;
+    T.q_rs = q.rstride;
+    T.y = quant ? nullptr : j.out.ptr;
+    T.y_bs = quant ? 0 : j.out.bstride;
+    T.y_rs = quant ? 0 : j.out.rstride;
+    T.scale = static_cast<float*>(j.scale);
+    T.rows = (int)q.rows;
+    T.cols = (int)q.cols;
+    const uint32_t tm = (uint32_t)((q.rows + kTile - 1) / kTile);
+    const uint32_t tn = (uint32_t)((q.cols + kTile - 1) / kTile);
+    T.tile_begin = tile_begin;
+    T.tiles_n = make_fastdiv(tn);
+    T.tiles_mn = make_fastdiv(tm * tn);
+    T.vec16 = ((uintptr_t)q.ptr % 16 == 0) && (q.rstride % 16 == 0) && (q.batch == 1 || q.bstride % 16 == 0);
+    return (uint32_t)q.batch * tm * tn;
+}
+
 }  // namespace
 
 cudaError_t read_and_clear_device_error(uint32_t* code) {
@@ -282,31 +329,9 @@ cudaError_t read_and_clear_device_error(uint32_t* code) {
     return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t));
 }
 
-cudaError_t launch_fp8_block_quant(const View& x, const View& q, float* scale, cudaStream_t s) {
+cudaError_t launch_fp8_block_quant(const Job* jobs, int n, cudaStream_t s) {
     EncodeTiledFn encode = encode_tiled_fn();
     if (!encode) return cudaErrorNotSupported;
-    CUtensorMap tmap;
-    const cuuint64_t dims[3] = {(cuuint64_t)x.cols, (cuuint64_t)x.rows, (cuuint64_t)x.batch};
-    const cuuint64_t strides[2] = {(cuuint64_t)x.rstride,
-                                   (cuuint64_t)(x.batch > 1 ? x.bstride : x.rows * x.rstride)};
-    const cuuint32_t box[3] = {kTile, kTile, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x.ptr, dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-
-    QuantArgs a;
-    a.q = q.ptr;
-    a.q_bs = q.bstride;
-    a.q_rs = q.rstride;
-    a.scale = scale;
-    a.rows = (int)x.rows;
-    a.cols = (int)x.cols;
-    a.tiles_m = (int)((x.rows + kTile - 1) / kTile);
-    a.tiles_n = (int)((x.cols + kTile - 1) / kTile);
-    a.total_tiles = (uint32_t)(x.batch * a.tiles_m * a.tiles_n);
-
     const size_t smem = (size_t)kStages * kTileBytes + 1024;
     static int configured[64] = {0};
     const int dev = current_device();
@@ -316,29 +341,48 @@ cudaError_t launch_fp8_block_quant(const View& x, const View& q, float* scale, c
         if (e != cudaSuccess) return e;
         configured[dev] = 1;
     }
-    const int grid = (int)std::min<int64_t>(a.total_tiles, (int64_t)sm_count(dev) * 2);
-    fp8_block_quant_kernel<<<grid, kThreads, smem, s>>>(tmap, a);
-    return cudaGetLastError();
+    for (int j0 = 0; j0 < n; j0 += kMaxLaunchTensors) {
+        QuantArgs a;
+        a.n = std::min(n - j0, kMaxLaunchTensors);
+        uint32_t tiles = 0;
+        for (int k = 0; k < a.n; ++k) {
+            const Job& j = jobs[j0 + k];
+            const View& x = j.in;
+            const cuuint64_t dims[3] = {(cuuint64_t)x.cols, (cuuint64_t)x.rows, (cuuint64_t)x.batch};
+            const cuuint64_t strides[2] = {(cuuint64_t)x.rstride,
+                                           (cuuint64_t)(x.batch > 1 ? x.bstride : x.rows * x.rstride)};
+            const cuuint32_t box[3] = {kTile, kTile, 1};
+            const cuuint32_t estr[3] = {1, 1, 1};
+            CUresult cr = encode(&a.tmap[k], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x.ptr, dims, strides, box, estr,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+            tiles += fill_tile_tensor(a.t[k], j, true, tiles);
+        }
+        a.total_tiles = tiles;
+        if (tiles == 0) continue;
+        const int grid = (int)std::min<int64_t>(tiles, (int64_t)sm_count(dev) * 2);
+        fp8_block_quant_kernel<<<grid, kThreads, smem, s>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
-cudaError_t launch_fp8_block_dequant(const View& q, const float* scale, const View& y, cudaStream_t s) {
-    DequantArgs a;
-    a.q = q.ptr;
-    a.y = y.ptr;
-    a.scale = scale;
-    a.q_bs = q.bstride;
-    a.q_rs = q.rstride;
-    a.y_bs = y.bstride;
-    a.y_rs = y.rstride;
-    a.rows = (int)q.rows;
-    a.cols = (int)q.cols;
-    a.tiles_m = (int)((q.rows + kTile - 1) / kTile);
-    a.tiles_n = (int)((q.cols + kTile - 1) / kTile);
-    a.total_tiles = (uint32_t)(q.batch * a.tiles_m * a.tiles_n);
-    a.vec16 = ((uintptr_t)q.ptr % 16 == 0) && (q.rstride % 16 == 0) && (q.batch == 1 || q.bstride % 16 == 0);
-    const int grid = persistent_grid(a.total_tiles, 8);
-    fp8_block_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
-    return cudaGetLastError();
+cudaError_t launch_fp8_block_dequant(const Job* jobs, int n, cudaStream_t s) {
+    for (int j0 = 0; j0 < n; j0 += kMaxLaunchTensors) {
+        DequantArgs a;
+        a.n = std::min(n - j0, kMaxLaunchTensors);
+        uint32_t tiles = 0;
+        for (int k = 0; k < a.n; ++k) tiles += fill_tile_tensor(a.t[k], jobs[j0 + k], false, tiles);
+        a.total_tiles = tiles;
+        if (tiles == 0) continue;
+        const int grid = persistent_grid(tiles, 8);
+        fp8_block_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace pwq

@@ -3,12 +3,17 @@
 // "Modes" 3 (MXFP8: 1x32 blocks, power-of-two UE8M0 scales packed as uint8,
 // float8_e4m3fn weights).
 //
-// HBM-bound elementwise kernels: each thread owns 8-element chunks (16 B of
-// BF16, one 128-bit load), four consecutive lanes form one 32-element block
-// and combine their amax with two butterfly shuffles.  The scale is a power
-// of two, so x * 2^-e is an exact multiply and no division is needed.
-// Persistent grids (a few CTAs per SM) walk the tensor in warp-sized spans
-// with U independent 128-bit loads in flight per thread.
+// HBM-bound elementwise kernels over a list of up to kMaxLaunchTensors
+// tensors per launch.  Each thread owns 8-element chunks (16 B of BF16, one
+// 128-bit load); four consecutive lanes form one 32-element block and
+// combine their amax with two butterfly shuffles.  The scale is a power of
+// two, so x * 2^-e is an exact multiply and no division is needed.  A
+// persistent grid walks the concatenated chunk ranges in warp-sized spans of
+// kUnroll * 32 chunks (kUnroll independent 128-bit loads in flight per
+// thread); every tensor's range is padded to a whole number of spans so a
+// span never straddles two tensors.
+#include <algorithm>
+
 #include "pwq_internal.h"
 
 namespace pwq {
@@ -16,47 +21,65 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
+constexpr uint32_t kSpan = 32u * kUnroll;   // chunks per warp span
 
-struct Rows {
-    int64_t bstride, rstride;
-    FastDiv per_batch;  // rows per batch matrix (M)
-    __device__ __forceinline__ int64_t offset(uint32_t r) const {
-        uint32_t b = fdiv(r, per_batch);
-        return (int64_t)b * bstride + (int64_t)(r - b * per_batch.d) * rstride;
+struct ChunkTensor {
+    const char* in;
+    char* out;
+    int64_t in_bs, in_rs, out_bs, out_rs;   // bytes
+    uint8_t* e;            // dense [B][M][N/32] scale bytes
+    uint32_t chunks;       // B * M * N / 8
+    uint32_t slot_begin;   // first chunk slot of this tensor (multiple of kSpan)
+    FastDiv cpr;           // chunks per row (N / 8)
+    FastDiv rows;          // M
+    int dense;             // both operands dense: chunk c at in + c*in_chunk, out + c*out_chunk
+};
+
+struct ChunkArgs {
+    ChunkTensor t[kMaxLaunchTensors];
+    int n;
+    uint32_t total_slots;
+};
+
+__device__ __forceinline__ int span_tensor(const ChunkArgs& a, uint32_t slot) {
+    int i = 0;
+    for (int k = 1; k < a.n; ++k)
+        if (slot >= a.t[k].slot_begin) i = k;
+    return i;
+}
+
+// Byte offsets of chunk c of T (input chunk in_chunk bytes, output out_chunk).
+__device__ __forceinline__ void chunk_offsets(const ChunkTensor& T, uint32_t c, int in_chunk, int out_chunk,
+                                              int64_t& io, int64_t& oo) {
+    if (T.dense) {
+        io = (int64_t)c * in_chunk;
+        oo = (int64_t)c * out_chunk;
+    } else {
+        const uint32_t r = fdiv(c, T.cpr);           // row over all batches
+        const uint32_t k = c - r * T.cpr.d;
+        const uint32_t b = fdiv(r, T.rows);
+        const uint32_t m = r - b * T.rows.d;
+        io = (int64_t)b * T.in_bs + (int64_t)m * T.in_rs + (int64_t)k * in_chunk;
+        oo = (int64_t)b * T.out_bs + (int64_t)m * T.out_rs + (int64_t)k * out_chunk;
     }
-};
+}
 
-struct MxQuantArgs {
-    const char* x;
-    char* q;
-    uint8_t* e;            // dense [rows][N/32]
-    Rows xr, qr;
-    FastDiv cpr;           // 8-element chunks per row (N / 8)
-    uint32_t total;        // chunks in this launch
-    int dense;             // x and q both dense: chunk c lives at x + 16c, q + 8c
-};
-
-__global__ void __launch_bounds__(kThreads) mxfp8_quant_kernel(const MxQuantArgs a) {
+__global__ void __launch_bounds__(kThreads) mxfp8_quant_kernel(const __grid_constant__ ChunkArgs a) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-    for (uint32_t base = gwarp * 32u * kUnroll; base < a.total; base += nwarps * 32u * kUnroll) {
+    for (uint32_t slot = gwarp * kSpan; slot < a.total_slots; slot += nwarps * kSpan) {
+        const ChunkTensor& T = a.t[span_tensor(a, slot)];
+        const uint32_t base = slot - T.slot_begin;
         uint4 v[kUnroll];
-        int64_t xo[kUnroll], qo[kUnroll];
+        int64_t qo[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const uint32_t c = base + u * 32u + lane;
-            if (a.dense) {
-                xo[u] = (int64_t)c * 16;
-                qo[u] = (int64_t)c * 8;
-            } else {
-                const uint32_t r = fdiv(c, a.cpr);
-                const uint32_t k = c - r * a.cpr.d;
-                xo[u] = a.xr.offset(r) + (int64_t)k * 16;
-                qo[u] = a.qr.offset(r) + (int64_t)k * 8;
-            }
+            int64_t xo;
+            chunk_offsets(T, c, 16, 8, xo, qo[u]);
             v[u] = make_uint4(0u, 0u, 0u, 0u);
-            if (c < a.total) v[u] = ld_stream_v4(a.x + xo[u]);
+            if (c < T.chunks) v[u] = ld_stream_v4(T.in + xo);
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -71,54 +94,39 @@ __global__ void __launch_bounds__(kThreads) mxfp8_quant_kernel(const MxQuantArgs
                            __fmul_rn(bf16_lo(v[u].y), inv), __fmul_rn(bf16_hi(v[u].y), inv));
             out.y = e4m3x4(__fmul_rn(bf16_lo(v[u].z), inv), __fmul_rn(bf16_hi(v[u].z), inv),
                            __fmul_rn(bf16_lo(v[u].w), inv), __fmul_rn(bf16_hi(v[u].w), inv));
-            if (c < a.total) {
-                st_v2(a.q + qo[u], out);
-                if ((lane & 3u) == 0u) a.e[c >> 2] = (uint8_t)(e + 127);
+            if (c < T.chunks) {
+                st_v2(T.out + qo[u], out);
+                if ((lane & 3u) == 0u) T.e[c >> 2] = (uint8_t)(e + 127);
             }
         }
     }
 }
 
-struct MxDequantArgs {
-    const char* q;
-    char* y;
-    const uint8_t* e;      // dense [rows][N/32]
-    Rows qr, yr;
-    FastDiv cpr;
-    uint32_t total;
-    int dense;
-};
-
-__global__ void __launch_bounds__(kThreads) mxfp8_dequant_kernel(const MxDequantArgs a) {
-    const uint32_t stride = gridDim.x * blockDim.x;
-    uint32_t c0 = blockIdx.x * blockDim.x + threadIdx.x;
-    for (uint32_t base = c0; base < a.total; base += stride * kUnroll) {
+__global__ void __launch_bounds__(kThreads) mxfp8_dequant_kernel(const __grid_constant__ ChunkArgs a) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t slot = gwarp * kSpan; slot < a.total_slots; slot += nwarps * kSpan) {
+        const ChunkTensor& T = a.t[span_tensor(a, slot)];
+        const uint32_t base = slot - T.slot_begin;
         uint2 v[kUnroll];
         uint32_t eb[kUnroll];
         int64_t yo[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * stride;
+            const uint32_t c = base + u * 32u + lane;
             int64_t qo;
-            if (a.dense) {
-                qo = (int64_t)c * 8;
-                yo[u] = (int64_t)c * 16;
-            } else {
-                const uint32_t r = fdiv(c, a.cpr);
-                const uint32_t k = c - r * a.cpr.d;
-                qo = a.qr.offset(r) + (int64_t)k * 8;
-                yo[u] = a.yr.offset(r) + (int64_t)k * 16;
-            }
+            chunk_offsets(T, c, 8, 16, qo, yo[u]);
             v[u] = make_uint2(0u, 0u);
             eb[u] = 127u;
-            if (c < a.total) {
-                v[u] = ld_stream_v2(a.q + qo);
-                eb[u] = __ldg(a.e + (c >> 2));
+            if (c < T.chunks) {
+                v[u] = ld_stream_v2(T.in + qo);
+                eb[u] = __ldg(T.e + (c >> 2));
             }
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * stride;
+            const uint32_t c = base + u * 32u + lane;
             const float p2 = exp2i((int)eb[u] - 127);
             uint4 out;
             float2 f;
@@ -130,68 +138,63 @@ __global__ void __launch_bounds__(kThreads) mxfp8_dequant_kernel(const MxDequant
             out.z = pack_bf16x2(__fmul_rn(f.x, p2), __fmul_rn(f.y, p2));
             f = e4m3x2_decode(v[u].y >> 16);
             out.w = pack_bf16x2(__fmul_rn(f.x, p2), __fmul_rn(f.y, p2));
-            if (c < a.total) st_v4(a.y + yo[u], out);
+            if (c < T.chunks) st_v4(T.out + yo[u], out);
         }
     }
 }
 
-bool dense_view(const View& v, int64_t elem_bytes_per_row) {
-    return v.rstride == elem_bytes_per_row && (v.batch == 1 || v.bstride == v.rows * v.rstride);
+bool dense_view(const View& v, int64_t row_bytes) {
+    return v.rstride == row_bytes && (v.batch == 1 || v.bstride == v.rows * v.rstride);
 }
 
-// Splits a launch over whole batch matrices so that each launch has fewer
-// than 2^31 chunks (chunk indices stay 32-bit).
-template <class F>
-cudaError_t for_batch_ranges(int64_t batch, int64_t chunks_per_batch, F&& f) {
-    const int64_t cap = (int64_t(1) << 31) - 1;
-    const int64_t per = chunks_per_batch > 0 ? std::max<int64_t>(1, cap / chunks_per_batch) : batch;
-    for (int64_t b0 = 0; b0 < batch; b0 += per) {
-        cudaError_t err = f(b0, std::min(batch, b0 + per));
-        if (err != cudaSuccess) return err;
+// quant: in = BF16 x, out = codes; dequant: in = codes, out = BF16 y
+template <bool kQuant>
+cudaError_t launch_mx(const Job* jobs, int n, cudaStream_t s) {
+    const uint64_t kMaxSlots = uint64_t(1) << 31;   // chunk indices stay 32-bit
+    for (int j0 = 0; j0 < n;) {
+        ChunkArgs a;
+        a.n = 0;
+        uint32_t slots = 0;
+        for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
+            const Job& j = jobs[j0 + a.n];
+            const View& xv = kQuant ? j.in : j.out;
+            const uint64_t padded = ((uint64_t)(xv.batch * xv.rows * (xv.cols / 8)) + kSpan - 1) / kSpan * kSpan;
+            if (a.n > 0 && slots + padded > kMaxSlots) break;
+            ChunkTensor& T = a.t[a.n];
+            const View& x = kQuant ? j.in : j.out;   // the BF16 side
+            const View& q = kQuant ? j.out : j.in;   // the code side
+            T.in = j.in.ptr;
+            T.out = j.out.ptr;
+            T.in_bs = j.in.bstride;
+            T.in_rs = j.in.rstride;
+            T.out_bs = j.out.bstride;
+            T.out_rs = j.out.rstride;
+            T.e = static_cast<uint8_t*>(j.scale);
+            T.chunks = (uint32_t)(x.batch * x.rows * (x.cols / 8));
+            T.slot_begin = slots;
+            T.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
+            T.rows = make_fastdiv((uint32_t)std::max<int64_t>(1, x.rows));
+            T.dense = dense_view(x, x.cols * 2) && dense_view(q, q.cols);
+            slots += (uint32_t)padded;
+        }
+        j0 += a.n;
+        a.total_slots = slots;
+        if (slots == 0) continue;
+        const int grid = persistent_grid((slots + kThreads * kUnroll - 1) / (kThreads * kUnroll), 8);
+        if (kQuant)
+            mxfp8_quant_kernel<<<grid, kThreads, 0, s>>>(a);
+        else
+            mxfp8_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
 
 }  // namespace
 
-cudaError_t launch_mxfp8_quant(const View& x, const View& q, uint8_t* scale, cudaStream_t s) {
-    const int64_t cpr = x.cols / 8;
-    const bool dense = dense_view(x, x.cols * 2) && dense_view(q, q.cols);
-    return for_batch_ranges(x.batch, x.rows * cpr, [&](int64_t b0, int64_t b1) {
-        MxQuantArgs a;
-        a.x = x.ptr + b0 * x.bstride;
-        a.q = q.ptr + b0 * q.bstride;
-        a.e = scale + b0 * x.rows * (x.cols / 32);
-        a.xr = Rows{x.bstride, x.rstride, make_fastdiv((uint32_t)x.rows)};
-        a.qr = Rows{q.bstride, q.rstride, make_fastdiv((uint32_t)x.rows)};
-        a.cpr = make_fastdiv((uint32_t)cpr);
-        a.total = (uint32_t)((b1 - b0) * x.rows * cpr);
-        a.dense = dense;
-        const int64_t span = int64_t(kThreads) * kUnroll;
-        const int grid = persistent_grid((a.total + span - 1) / span, 8);
-        mxfp8_quant_kernel<<<grid, kThreads, 0, s>>>(a);
-        return cudaGetLastError();
-    });
-}
+cudaError_t launch_mxfp8_quant(const Job* jobs, int n, cudaStream_t s) { return launch_mx<true>(jobs, n, s); }
 
-cudaError_t launch_mxfp8_dequant(const View& q, const uint8_t* scale, const View& y, cudaStream_t s) {
-    const int64_t cpr = q.cols / 8;
-    const bool dense = dense_view(q, q.cols) && dense_view(y, y.cols * 2);
-    return for_batch_ranges(q.batch, q.rows * cpr, [&](int64_t b0, int64_t b1) {
-        MxDequantArgs a;
-        a.q = q.ptr + b0 * q.bstride;
-        a.y = y.ptr + b0 * y.bstride;
-        a.e = scale + b0 * q.rows * (q.cols / 32);
-        a.qr = Rows{q.bstride, q.rstride, make_fastdiv((uint32_t)q.rows)};
-        a.yr = Rows{y.bstride, y.rstride, make_fastdiv((uint32_t)q.rows)};
-        a.cpr = make_fastdiv((uint32_t)cpr);
-        a.total = (uint32_t)((b1 - b0) * q.rows * cpr);
-        a.dense = dense;
-        const int64_t span = int64_t(kThreads) * kUnroll;
-        const int grid = persistent_grid((a.total + span - 1) / span, 8);
-        mxfp8_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
-        return cudaGetLastError();
-    });
-}
+cudaError_t launch_mxfp8_dequant(const Job* jobs, int n, cudaStream_t s) { return launch_mx<false>(jobs, n, s); }
 
 }  // namespace pwq

@@ -221,56 +221,317 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
     }
 }
 
-struct DequantArgs {
+// Dequantise: a grouped chunk walk like MXFP8's.  Per 8-element chunk: 4
+// packed bytes in, 16 bytes of BF16 out; the chunk's block scale and its
+// batch index's global scale are cached loads.
+constexpr uint32_t kSpan = 32u * kUnroll;   // chunks per warp span
+
+struct DqTensor {
     const char* q;        // packed codes
     char* y;              // BF16
+    int64_t q_bs, q_rs, y_bs, y_rs;
     const uint8_t* sb;    // dense [B][M][N/16]
     const float* gs;      // [B]
-    int64_t q_bs, q_rs, y_bs, y_rs;
+    uint32_t chunks;      // B * M * N / 8
+    uint32_t slot_begin;  // multiple of kSpan
     FastDiv cpr;          // chunks per row (N / 8)
-    FastDiv per_batch;    // chunks per batch slab (M * N / 8)
+    FastDiv per_batch;    // chunks per batch matrix (M * N / 8)
     FastDiv rows;         // M
-    uint32_t total;
     int dense;
 };
 
-__global__ void __launch_bounds__(kThreads) nvfp4_dequant_kernel(const DequantArgs a) {
-    const uint32_t stride = gridDim.x * blockDim.x;
-    for (uint32_t base = blockIdx.x * blockDim.x + threadIdx.x; base < a.total;
-         base += stride * kUnroll) {
+struct DequantArgs {
+    DqTensor t[kMaxLaunchTensors];
+    int n;
+    uint32_t total_slots;
+};
+
+__global__ void __launch_bounds__(kThreads) nvfp4_dequant_kernel(const __grid_constant__ DequantArgs a) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t slot = gwarp * kSpan; slot < a.total_slots; slot += nwarps * kSpan) {
+        int ti = 0;
+        for (int k = 1; k < a.n; ++k)
+            if (slot >= a.t[k].slot_begin) ti = k;
+        const DqTensor& T = a.t[ti];
+        const uint32_t base = slot - T.slot_begin;
         uint32_t codes[kUnroll], sbyte[kUnroll], bidx[kUnroll];
         int64_t yo[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * stride;
-            const uint32_t b = fdiv(c, a.per_batch);
+            const uint32_t c = base + u * 32u + lane;
+            const uint32_t b = fdiv(c, T.per_batch);
             int64_t qo;
-            if (a.dense) {
+            if (T.dense) {
                 qo = (int64_t)c * 4;
                 yo[u] = (int64_t)c * 16;
             } else {
-                const uint32_t r = fdiv(c, a.cpr);          // global row
-                const uint32_t k = c - r * a.cpr.d;
-                const uint32_t mrow = r - b * a.rows.d;
-                qo = (int64_t)b * a.q_bs + (int64_t)mrow * a.q_rs + (int64_t)k * 4;
-                yo[u] = (int64_t)b * a.y_bs + (int64_t)mrow * a.y_rs + (int64_t)k * 16;
+                const uint32_t r = fdiv(c, T.cpr);          // row over all batches
+                const uint32_t k = c - r * T.cpr.d;
+                const uint32_t mrow = r - b * T.rows.d;
+                qo = (int64_t)b * T.q_bs + (int64_t)mrow * T.q_rs + (int64_t)k * 4;
+                yo[u] = (int64_t)b * T.y_bs + (int64_t)mrow * T.y_rs + (int64_t)k * 16;
             }
             bidx[u] = b;
             codes[u] = 0u;
             sbyte[u] = 0u;
-            if (c < a.total) {
-                codes[u] = ld_stream_u32(a.q + qo);
-                sbyte[u] = __ldg(a.sb + (c >> 1));
+            if (c < T.chunks) {
+                codes[u] = ld_stream_u32(T.q + qo);
+                sbyte[u] = __ldg(T.sb + (c >> 1));
             }
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * stride;
-            if (c < a.total) {
-                const float gs = __ldg(a.gs + bidx[u]);
-                st_v4(a.y + yo[u], dequant_half(codes[u], e4m3_decode(sbyte[u]), gs));
+            const uint32_t c = base + u * 32u + lane;
+            if (c < T.chunks) {
+                const float gs = __ldg(T.gs + bidx[u]);
+                st_v4(T.y + yo[u], dequant_half(codes[u], e4m3_decode(sbyte[u]), gs));
             }
         }
+    }
+}
+
+// ---------------------------------------------------------------- single-pass quantise / fake-quantise
+//
+// One launch covers up to kMaxLaunchTensors members in up to as many sibling
+// groups, every batch index of a group being one "instance" with its own
+// amax.  The work is a queue of items of kItemChunks chunks of one member's
+// batch slab: amax items A(i, k) and encode items E(i, k) of instance i.  The
+// queue order is
+//     A(0) A(1) E(0) A(2) E(1) ... A(I-1) E(I-2) E(I-1)
+// so while the encode items of instance i run (ALU-heavy, reading data that
+// is still in L2), the amax items of instance i+1 keep HBM busy.  CTAs take
+// items from a global atomic counter.  An encode item waits (bounded) until
+// all amax items of its instance are done; those items all sit earlier in
+// the queue, were taken by running CTAs that never wait on later items, and
+// so finish: there is no deadlock whatever the number of resident CTAs.  An
+// amax item publishes its max with atomicMax and then counts itself done
+// (fence + atomicAdd); the waiting side reads the count with acquire
+// semantics before it reads the amax.
+constexpr int kFlowThreads = 256;
+constexpr uint32_t kItemChunks = 2048;                        // 16384 elements
+constexpr int kItemChunksPerThread = kItemChunks / kFlowThreads;   // 8
+constexpr int kFlowMaxInst = 2048;                            // instances per launch
+constexpr uint64_t kFlowWaitNs = 2000000000ull;               // 2 s
+constexpr uint32_t kErrFlowTimeout = 2u;
+
+struct FlowMember {
+    const char* x;        // BF16, at this launch's first batch index
+    int64_t x_bs, x_rs;
+    char* out;            // packed codes (quant) or BF16 (fake)
+    int64_t o_bs, o_rs;
+    uint8_t* sb;          // quant: dense [B][M][N/16], at the first batch index
+    uint32_t chunks;      // chunks per batch slab (M * N / 8)
+    FastDiv cpr;          // chunks per row
+    int dense_x, dense_o;
+    uint32_t item_off;    // first item of this member inside an instance
+};
+
+struct FlowGroup {
+    int m_begin, m_count;
+    uint32_t inst_begin, batch;   // instances [inst_begin, inst_begin + batch)
+    uint32_t items;               // items per instance
+    uint32_t item_begin;          // items of all instances before inst_begin
+    float* gs_out;                // [batch] or null, at the first batch index
+    float* amax_out;              // [batch] or null
+};
+
+struct FlowArgs {
+    FlowMember m[kMaxLaunchTensors];
+    FlowGroup g[kMaxLaunchTensors];
+    int n_groups;
+    uint32_t n_inst;
+    uint32_t total_items;         // items per pass (A items = E items)
+    uint32_t* amax_bits;          // [n_inst]  (workspace, zeroed before launch)
+    uint32_t* done;               // [n_inst]  completed amax items
+    uint32_t* counter;            // [1]       queue head
+};
+
+__device__ uint32_t g_flow_error = 0u;
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ int flow_group_of(const FlowArgs& a, uint32_t inst) {
+    int g = 0;
+    for (int k = 1; k < a.n_groups; ++k)
+        if (inst >= a.g[k].inst_begin) g = k;
+    return g;
+}
+
+// Queue position q -> (encode?, instance, item within the instance's pass).
+// pa[i] = items before instance i (pa[I] = total).  Segment starts:
+// A(0) at 0, A(j) at pa[j] + pa[j-1]; E(j) at pa[min(j+2, I)] + pa[j].
+__device__ __forceinline__ void flow_decode(const uint32_t* pa, uint32_t I, uint32_t q, bool& is_e,
+                                            uint32_t& inst, uint32_t& k) {
+    uint32_t lo = 0, hi = I - 1;
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi + 1) >> 1;
+        if (pa[mid] + pa[mid - 1] <= q) lo = mid; else hi = mid - 1;
+    }
+    const uint32_t ja = lo;
+    const uint32_t sa = ja ? pa[ja] + pa[ja - 1] : 0u;
+    is_e = false;
+    inst = ja;
+    k = q - sa;
+    if (pa[min(2u, I)] + pa[0] > q) return;         // before E(0)
+    lo = 0;
+    hi = I - 1;
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi + 1) >> 1;
+        if (pa[min(mid + 2u, I)] + pa[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    const uint32_t se = pa[min(lo + 2u, I)] + pa[lo];
+    if (se > sa) {
+        is_e = true;
+        inst = lo;
+        k = q - se;
+    }
+}
+
+template <bool kFake>
+__global__ void __launch_bounds__(kFlowThreads) nvfp4_flow_kernel(const __grid_constant__ FlowArgs a) {
+    __shared__ uint32_t pa[kFlowMaxInst + 1];
+    __shared__ ScaleTable tab;
+    __shared__ uint32_t s_item, s_next, s_amax;
+    __shared__ uint32_t red[kFlowThreads / 32];
+    const uint32_t tid = threadIdx.x;
+    for (uint32_t i = tid; i <= a.n_inst; i += blockDim.x) {
+        uint32_t v = a.total_items;
+        if (i < a.n_inst) {
+            const FlowGroup& G = a.g[flow_group_of(a, i)];
+            v = G.item_begin + (i - G.inst_begin) * G.items;
+        }
+        pa[i] = v;
+    }
+    if (tid == 0) s_item = atomicAdd(a.counter, 1u);
+    __syncthreads();
+    const uint32_t total_q = 2u * a.total_items;
+    uint32_t item = s_item;
+    uint32_t cached = 0xffffffffu;
+    float gs = 0.0f, six_gs = 0.0f, r6 = 0.0f;
+    bool fast6 = false;
+    while (item < total_q) {
+        if (tid == 0) s_next = atomicAdd(a.counter, 1u);   // prefetch the next item
+        bool is_e;
+        uint32_t inst, k;
+        flow_decode(pa, a.n_inst, item, is_e, inst, k);
+        const FlowGroup& G = a.g[flow_group_of(a, inst)];
+        const uint32_t b = inst - G.inst_begin;
+        if (is_e) k = G.items - 1u - k;                    // encode walks the instance backwards
+        int mi = G.m_begin;
+        for (int t = 1; t < G.m_count; ++t)
+            if (k >= a.m[G.m_begin + t].item_off) mi = G.m_begin + t;
+        const FlowMember& M = a.m[mi];
+        const uint32_t c0 = (k - M.item_off) * kItemChunks;
+        const uint32_t c1 = min(c0 + kItemChunks, M.chunks);
+        const char* xb = M.x + (int64_t)b * M.x_bs;
+
+        uint4 v[kItemChunksPerThread];
+#pragma unroll
+        for (int j = 0; j < kItemChunksPerThread; ++j) {
+            const uint32_t c = c0 + (uint32_t)j * kFlowThreads + tid;
+            v[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (c < c1) {
+                int64_t off;
+                if (M.dense_x) {
+                    off = (int64_t)c * 16;
+                } else {
+                    const uint32_t r = fdiv(c, M.cpr);
+                    off = (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 16;
+                }
+                v[j] = ld_stream_v4(xb + off);
+            }
+        }
+
+        if (!is_e) {
+            // ---- amax item
+            uint32_t m = 0u;
+#pragma unroll
+            for (int j = 0; j < kItemChunksPerThread; ++j) m = max(m, amax_bits8(v[j]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if ((tid & 31u) == 0u) red[tid >> 5] = m;
+            __syncthreads();
+            if (tid == 0) {
+                for (int w = 1; w < kFlowThreads / 32; ++w) m = max(m, red[w]);
+                if (m != 0u) atomicMax(a.amax_bits + inst, m << 16);
+                __threadfence();
+                atomicAdd(a.done + inst, 1u);
+            }
+        } else {
+            // ---- encode item: wait for the instance's amax
+            if (tid == 0) {
+                if (ld_acquire_gpu(a.done + inst) < G.items) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_gpu(a.done + inst) < G.items) {
+                        if (globaltimer_ns() - t0 > kFlowWaitNs) {
+                            atomicOr(&g_flow_error, kErrFlowTimeout);
+                            break;
+                        }
+                        __nanosleep(200);
+                    }
+                }
+                s_amax = ld_relaxed_gpu(a.amax_bits + inst);
+            }
+            __syncthreads();
+            if (inst != cached) {   // CTA-uniform
+                const float A = __uint_as_float(s_amax);
+                gs = __fdiv_rn(A, 2688.0f);
+                six_gs = __fmul_rn(6.0f, gs);
+                r6 = __frcp_rn(six_gs);
+                fast6 = div_fast_ok(six_gs);
+                fill_scale_table(tab, gs);
+                if (tid == 0 && k == 0u) {
+                    if (G.gs_out) G.gs_out[b] = gs;
+                    if (G.amax_out) G.amax_out[b] = A;
+                }
+                __syncthreads();
+                cached = inst;
+            } else if (tid == 0 && k == 0u) {
+                if (G.gs_out) G.gs_out[b] = gs;
+                if (G.amax_out) G.amax_out[b] = __uint_as_float(s_amax);
+            }
+            char* ob = M.out + (int64_t)b * M.o_bs;
+            uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)b * (M.chunks >> 1);
+#pragma unroll
+            for (int j = 0; j < kItemChunksPerThread; ++j) {
+                const uint32_t c = c0 + (uint32_t)j * kFlowThreads + tid;
+                uint32_t m = amax_bits8(v[j]);
+                m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));   // lanes 2i, 2i+1: one block
+                const float amax_b = __uint_as_float(m << 16);
+                const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
+                const uint32_t sb = e4m3x2(ratio, 0.0f) & 0xffu;
+                const float4 e = tab.e[sb];
+                const uint32_t codes = codes_half(v[j], e.x, e.y);
+                if (c < c1) {
+                    int64_t oo;
+                    if (M.dense_o) {
+                        oo = (int64_t)c * (kFake ? 16 : 4);
+                    } else {
+                        const uint32_t r = fdiv(c, M.cpr);
+                        oo = (int64_t)r * M.o_rs + (int64_t)(c - r * M.cpr.d) * (kFake ? 16 : 4);
+                    }
+                    if (kFake) {
+                        st_v4(ob + oo, dequant_half(codes, e.z, gs));
+                    } else {
+                        st_u32(ob + oo, codes);
+                        if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)sb;
+                    }
+                }
+            }
+        }
+        __syncthreads();   // s_next is ready; red / s_amax / tab may be reused
+        item = s_next;
     }
 }
 
@@ -345,28 +606,141 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
     return cudaGetLastError();
 }
 
-cudaError_t launch_nvfp4_dequant(const View& q, const uint8_t* sb, const float* gs, const View& y,
-                                 cudaStream_t s) {
-    DequantArgs a;
-    a.q = q.ptr;
-    a.y = y.ptr;
-    a.sb = sb;
-    a.gs = gs;
-    a.q_bs = q.bstride;
-    a.q_rs = q.rstride;
-    a.y_bs = y.bstride;
-    a.y_rs = y.rstride;
-    const int64_t cpr = q.cols / 8;
-    a.cpr = make_fastdiv((uint32_t)cpr);
-    a.per_batch = make_fastdiv((uint32_t)(q.rows * cpr));
-    a.rows = make_fastdiv((uint32_t)q.rows);
-    a.total = (uint32_t)(q.batch * q.rows * cpr);
-    a.dense = q.rstride == q.cols / 2 && y.rstride == y.cols * 2 &&
-              (q.batch == 1 || (q.bstride == q.rows * q.rstride && y.bstride == y.rows * y.rstride));
-    const int64_t span = int64_t(kThreads) * kUnroll;
-    const int grid = persistent_grid((a.total + span - 1) / span, 8);
-    nvfp4_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
-    return cudaGetLastError();
+cudaError_t launch_nvfp4_dequant(const Job* jobs, int n, cudaStream_t s) {
+    const uint64_t kMaxSlots = uint64_t(1) << 31;   // chunk indices stay 32-bit
+    for (int j0 = 0; j0 < n;) {
+        DequantArgs a;
+        a.n = 0;
+        uint32_t slots = 0;
+        for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
+            const Job& j = jobs[j0 + a.n];
+            const View& q = j.in;
+            const View& y = j.out;
+            const uint64_t chunks = (uint64_t)(q.batch * q.rows * (q.cols / 8));
+            const uint64_t padded = (chunks + kSpan - 1) / kSpan * kSpan;
+            if (a.n > 0 && slots + padded > kMaxSlots) break;
+            DqTensor& T = a.t[a.n];
+            T.q = q.ptr;
+            T.y = y.ptr;
+            T.q_bs = q.bstride;
+            T.q_rs = q.rstride;
+            T.y_bs = y.bstride;
+            T.y_rs = y.rstride;
+            T.sb = static_cast<const uint8_t*>(j.scale);
+            T.gs = j.gs;
+            T.chunks = (uint32_t)chunks;
+            T.slot_begin = slots;
+            const int64_t cpr = std::max<int64_t>(1, q.cols / 8);
+            T.cpr = make_fastdiv((uint32_t)cpr);
+            T.per_batch = make_fastdiv((uint32_t)std::max<int64_t>(1, q.rows * cpr));
+            T.rows = make_fastdiv((uint32_t)std::max<int64_t>(1, q.rows));
+            T.dense = q.rstride == q.cols / 2 && y.rstride == y.cols * 2 &&
+                      (q.batch == 1 || (q.bstride == q.rows * q.rstride && y.bstride == y.rows * y.rstride));
+            slots += (uint32_t)padded;
+        }
+        j0 += a.n;
+        a.total_slots = slots;
+        if (slots == 0) continue;
+        const int grid = persistent_grid((slots + kThreads * kUnroll - 1) / (kThreads * kUnroll), 8);
+        nvfp4_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t read_and_clear_flow_error(uint32_t* code) {
+    uint32_t zero = 0u;
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_flow_error, sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbol(g_flow_error, &zero, sizeof(uint32_t));
+}
+
+size_t nvfp4_flow_workspace_bytes(int64_t instances) {
+    const int64_t per = std::max<int64_t>(1, std::min<int64_t>(instances, kFlowMaxInst));
+    return (size_t)((2 * per + 1) * 4 + 255) / 256 * 256;
+}
+
+cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, void* workspace, cudaStream_t s) {
+    uint32_t* words = static_cast<uint32_t*>(workspace);
+    const uint64_t kMaxItems = uint64_t(1) << 30;   // queue positions (2 per item) stay 32-bit
+    FlowArgs a;
+    int n_members = 0;
+    auto reset = [&]() {
+        a.n_groups = 0;
+        a.n_inst = 0;
+        a.total_items = 0;
+        n_members = 0;
+    };
+    auto flush = [&]() -> cudaError_t {
+        if (a.n_groups == 0) return cudaSuccess;
+        a.amax_bits = words;
+        a.done = words + a.n_inst;
+        a.counter = words + 2 * a.n_inst;
+        cudaError_t e = cudaMemsetAsync(words, 0, (size_t)(2 * a.n_inst + 1) * 4, s);
+        if (e != cudaSuccess) return e;
+        const int grid = (int)std::max<int64_t>(
+            1, std::min<int64_t>((int64_t)sm_count(current_device()) * 4, 2 * (int64_t)a.total_items));
+        if (fake)
+            nvfp4_flow_kernel<true><<<grid, kFlowThreads, 0, s>>>(a);
+        else
+            nvfp4_flow_kernel<false><<<grid, kFlowThreads, 0, s>>>(a);
+        e = cudaGetLastError();
+        reset();
+        return e;
+    };
+    reset();
+    for (int gi = 0; gi < n_groups; ++gi) {
+        const NvGroup& G = groups[gi];
+        const int64_t B = G.x[0].batch;
+        uint32_t items = 0;
+        for (int i = 0; i < G.n; ++i)
+            items += (uint32_t)((G.x[i].rows * (G.x[i].cols / 8) + kItemChunks - 1) / kItemChunks);
+        if (items == 0 || B == 0) continue;
+        for (int64_t b0 = 0; b0 < B;) {
+            const int64_t room_inst = kFlowMaxInst - (int64_t)a.n_inst;
+            const int64_t room_items = (int64_t)(kMaxItems - a.total_items) / items;
+            if (n_members + G.n > kMaxLaunchTensors || a.n_groups == kMaxLaunchTensors || room_inst < 1 ||
+                room_items < 1) {
+                cudaError_t e = flush();
+                if (e != cudaSuccess) return e;
+                continue;
+            }
+            const int64_t take = std::min<int64_t>({B - b0, room_inst, room_items});
+            FlowGroup& F = a.g[a.n_groups++];
+            F.m_begin = n_members;
+            F.m_count = G.n;
+            F.inst_begin = a.n_inst;
+            F.batch = (uint32_t)take;
+            F.items = items;
+            F.item_begin = a.total_items;
+            F.gs_out = G.gs_out ? G.gs_out + b0 : nullptr;
+            F.amax_out = G.amax_out ? G.amax_out + b0 : nullptr;
+            uint32_t off = 0;
+            for (int i = 0; i < G.n; ++i) {
+                const View& x = G.x[i];
+                const View& o = G.out[i];
+                FlowMember& M = a.m[n_members++];
+                M.x = x.ptr + b0 * x.bstride;
+                M.x_bs = x.bstride;
+                M.x_rs = x.rstride;
+                M.out = o.ptr + b0 * o.bstride;
+                M.o_bs = o.bstride;
+                M.o_rs = o.rstride;
+                M.chunks = (uint32_t)(x.rows * (x.cols / 8));
+                M.sb = fake ? nullptr : G.sb[i] + b0 * (int64_t)(M.chunks / 2);
+                M.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
+                M.dense_x = dense_rows(x, x.cols * 2);
+                M.dense_o = dense_rows(o, fake ? o.cols * 2 : o.cols / 2);
+                M.item_off = off;
+                off += (M.chunks + kItemChunks - 1) / kItemChunks;
+            }
+            a.n_inst += (uint32_t)take;
+            a.total_items += (uint32_t)take * items;
+            b0 += take;
+        }
+    }
+    return flush();
 }
 
 // ---------------------------------------------------------------- scratch for callers that cannot allocate

@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <vector>
 
 #include "pwq.h"
 #include "pwq_internal.h"
@@ -39,6 +40,7 @@ int persistent_grid(int64_t work_ctas, int per_sm) {
 
 namespace {
 
+using pwq::Job;
 using pwq::View;
 
 thread_local char g_detail[256] = "";
@@ -73,6 +75,8 @@ Extent extent_of(const void* p, size_t bytes) {
 bool empty(const pwq_tensor* t) { return t->batch == 0 || t->rows == 0 || t->cols == 0; }
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+// chunk (8-element) and tile counts of one tensor stay below 2^31
+constexpr int64_t kMaxChunks = (int64_t(1) << 31) - 1024;
 
 // Validates one tensor descriptor; fills a byte-stride view and its extent.
 pwq_status check_tensor(const pwq_tensor* t, Kind k, View* v, Extent* ext, const char* name) {
@@ -93,6 +97,8 @@ pwq_status check_tensor(const pwq_tensor* t, Kind k, View* v, Extent* ext, const
         return PWQ_OK;
     }
     if (!t->ptr) return fail(PWQ_ERR_NULL, name);
+    if ((t->batch * t->rows) > kMaxDim || t->batch * t->rows * ((t->cols + 7) / 8) > kMaxChunks)
+        return fail(PWQ_ERR_SHAPE, "tensor too large (more than 2^31 8-element chunks)");
     // BF16 rows are moved in 16-byte vectors (and by TMA); code rows in
     // 8-byte (E4M3) or 4-byte (packed E2M1) pieces
     const int64_t align = (k == Kind::kBF16) ? 16 : 8;
@@ -128,7 +134,96 @@ pwq_status check_overlaps(const Extent* in, int n_in, const Extent* out, int n_o
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-constexpr int64_t kMaxU32 = (int64_t(1) << 32) - 1;
+// ------------------------------------------------------------------ elementwise ops over tensor lists
+
+enum class Op { kFp8Quant, kFp8Dequant, kMxQuant, kMxDequant, kNvDequant };
+
+// in / out kinds and the scale array size (bytes) of one tensor
+struct OpSpec {
+    Kind in, out;
+    const char* name;
+};
+
+OpSpec spec(Op op) {
+    switch (op) {
+        case Op::kFp8Quant: return {Kind::kBF16, Kind::kByte, "fp8_block_quant"};
+        case Op::kFp8Dequant: return {Kind::kByte, Kind::kBF16, "fp8_block_dequant"};
+        case Op::kMxQuant: return {Kind::kBF16, Kind::kByte, "mxfp8_quant"};
+        case Op::kMxDequant: return {Kind::kByte, Kind::kBF16, "mxfp8_dequant"};
+        case Op::kNvDequant: return {Kind::kPacked4, Kind::kBF16, "nvfp4_dequant"};
+    }
+    return {Kind::kBF16, Kind::kBF16, "?"};
+}
+
+size_t scale_bytes(Op op, const pwq_tensor* t) {
+    switch (op) {
+        case Op::kFp8Quant:
+        case Op::kFp8Dequant: return (size_t)(t->batch * ceil_div(t->rows, 128) * ceil_div(t->cols, 128)) * 4;
+        case Op::kMxQuant:
+        case Op::kMxDequant: return (size_t)(t->batch * t->rows * (t->cols / 32));
+        case Op::kNvDequant: return (size_t)(t->batch * t->rows * (t->cols / 16));
+    }
+    return 0;
+}
+
+// Validates n (in, out, scale[, gs]) tensors and launches them as one
+// grouped call.  scale[i] is an input for dequantise ops and an output for
+// quantise ops; gs (NVFP4 dequant only) an input.
+pwq_status run_list(Op op, int n, const pwq_tensor* in, const pwq_tensor* out, void* const* scale,
+                    const float* const* gs, pwq_stream_t stream) {
+    if (n < 0 || n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "tensor count out of range");
+    if (n == 0) return PWQ_OK;
+    if (!in || !out || !scale) return fail(PWQ_ERR_NULL, "tensor or scale array");
+    if (op == Op::kNvDequant && !gs) return fail(PWQ_ERR_NULL, "global_scale array");
+    const OpSpec sp = spec(op);
+    const bool quant = (op == Op::kFp8Quant || op == Op::kMxQuant);
+    std::vector<Job> jobs;
+    std::vector<Extent> ins, outs;
+    jobs.reserve(n);
+    for (int i = 0; i < n; ++i) {
+        const pwq_tensor* a = &in[i];
+        const pwq_tensor* b = &out[i];
+        if (!same_shape(a, b)) return fail(PWQ_ERR_SHAPE, "output shape != input shape");
+        Job j;
+        Extent ea, eb;
+        pwq_status st;
+        if ((st = check_tensor(a, sp.in, &j.in, &ea, "input")) != PWQ_OK) return st;
+        if ((st = check_tensor(b, sp.out, &j.out, &eb, "output")) != PWQ_OK) return st;
+        if ((op == Op::kMxQuant || op == Op::kMxDequant) && a->cols % 32 != 0)
+            return fail(PWQ_ERR_SHAPE, "cols % 32 != 0");
+        if (op == Op::kNvDequant && a->cols % 16 != 0) return fail(PWQ_ERR_SHAPE, "cols % 16 != 0");
+        if (empty(a)) continue;
+        if (!scale[i]) return fail(PWQ_ERR_NULL, "scale");
+        const bool fp8 = (op == Op::kFp8Quant || op == Op::kFp8Dequant);
+        if (fp8 && (uintptr_t)scale[i] % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale");
+        j.scale = scale[i];
+        j.gs = nullptr;
+        const Extent es = extent_of(scale[i], scale_bytes(op, a));
+        ins.push_back(ea);
+        outs.push_back(eb);
+        (quant ? outs : ins).push_back(es);
+        if (op == Op::kNvDequant) {
+            if (!gs[i]) return fail(PWQ_ERR_NULL, "global_scale");
+            if ((uintptr_t)gs[i] % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
+            j.gs = gs[i];
+            ins.push_back(extent_of(gs[i], (size_t)a->batch * 4));
+        }
+        jobs.push_back(j);
+    }
+    pwq_status st = check_overlaps(ins.data(), (int)ins.size(), outs.data(), (int)outs.size());
+    if (st != PWQ_OK) return st;
+    if (jobs.empty()) return PWQ_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int m = (int)jobs.size();
+    switch (op) {
+        case Op::kFp8Quant: return from_cuda(pwq::launch_fp8_block_quant(jobs.data(), m, s));
+        case Op::kFp8Dequant: return from_cuda(pwq::launch_fp8_block_dequant(jobs.data(), m, s));
+        case Op::kMxQuant: return from_cuda(pwq::launch_mxfp8_quant(jobs.data(), m, s));
+        case Op::kMxDequant: return from_cuda(pwq::launch_mxfp8_dequant(jobs.data(), m, s));
+        case Op::kNvDequant: return from_cuda(pwq::launch_nvfp4_dequant(jobs.data(), m, s));
+    }
+    return fail(PWQ_ERR_ARG, "op");
+}
 
 }  // namespace
 
@@ -155,93 +250,79 @@ const char* pwq_build_info(void) { return "libpwq sm_100a; " PWQ_BUILD_FLAGS; }
 
 pwq_status pwq_device_error(uint32_t* code) {
     if (!code) return fail(PWQ_ERR_NULL, "code");
-    return from_cuda(pwq::read_and_clear_device_error(code));
+    uint32_t a = 0, b = 0;
+    cudaError_t e = pwq::read_and_clear_device_error(&a);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = pwq::read_and_clear_flow_error(&b);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *code = a | b;
+    return PWQ_OK;
 }
 
-// ------------------------------------------------------------------ FP8 block
+// ------------------------------------------------------------------ FP8 block-wise, MXFP8, NVFP4 dequant
 
 pwq_status fp8_block_quant(const pwq_tensor* x, const pwq_tensor* q, float* scale, pwq_stream_t stream) {
     if (!x || !q) return fail(PWQ_ERR_NULL, "tensor descriptor");
-    if (!same_shape(x, q)) return fail(PWQ_ERR_SHAPE, "q shape != x shape");
-    View vx, vq;
-    Extent ex, eq;
-    pwq_status st;
-    if ((st = check_tensor(x, Kind::kBF16, &vx, &ex, "x")) != PWQ_OK) return st;
-    if ((st = check_tensor(q, Kind::kByte, &vq, &eq, "q")) != PWQ_OK) return st;
-    if (empty(x)) return PWQ_OK;
-    if (!scale) return fail(PWQ_ERR_NULL, "scale");
-    if ((uintptr_t)scale % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale");
-    const int64_t tiles = x->batch * ceil_div(x->rows, 128) * ceil_div(x->cols, 128);
-    if (tiles > kMaxU32) return fail(PWQ_ERR_SHAPE, "too many tiles");
-    const Extent es = extent_of(scale, (size_t)tiles * 4);
-    const Extent ins[1] = {ex};
-    const Extent outs[2] = {eq, es};
-    if ((st = check_overlaps(ins, 1, outs, 2)) != PWQ_OK) return st;
-    return from_cuda(pwq::launch_fp8_block_quant(vx, vq, scale, (cudaStream_t)stream));
+    void* sc[1] = {scale};
+    return run_list(Op::kFp8Quant, 1, x, q, sc, nullptr, stream);
 }
 
 pwq_status fp8_block_dequant(const pwq_tensor* q, const float* scale, const pwq_tensor* y,
                              pwq_stream_t stream) {
     if (!q || !y) return fail(PWQ_ERR_NULL, "tensor descriptor");
-    if (!same_shape(q, y)) return fail(PWQ_ERR_SHAPE, "y shape != q shape");
-    View vq, vy;
-    Extent eq, ey;
-    pwq_status st;
-    if ((st = check_tensor(q, Kind::kByte, &vq, &eq, "q")) != PWQ_OK) return st;
-    if ((st = check_tensor(y, Kind::kBF16, &vy, &ey, "y")) != PWQ_OK) return st;
-    if (empty(q)) return PWQ_OK;
-    if (!scale) return fail(PWQ_ERR_NULL, "scale");
-    if ((uintptr_t)scale % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale");
-    if (q->batch * q->rows * ceil_div(q->cols, 8) > kMaxU32) return fail(PWQ_ERR_SHAPE, "too large");
-    const int64_t tiles = q->batch * ceil_div(q->rows, 128) * ceil_div(q->cols, 128);
-    const Extent es = extent_of(scale, (size_t)tiles * 4);
-    const Extent ins[2] = {eq, es};
-    const Extent outs[1] = {ey};
-    if ((st = check_overlaps(ins, 2, outs, 1)) != PWQ_OK) return st;
-    return from_cuda(pwq::launch_fp8_block_dequant(vq, scale, vy, (cudaStream_t)stream));
+    void* sc[1] = {const_cast<float*>(scale)};
+    return run_list(Op::kFp8Dequant, 1, q, y, sc, nullptr, stream);
 }
-
-// ------------------------------------------------------------------ MXFP8
 
 pwq_status mxfp8_quant(const pwq_tensor* x, const pwq_tensor* q, uint8_t* scale, pwq_stream_t stream) {
     if (!x || !q) return fail(PWQ_ERR_NULL, "tensor descriptor");
-    if (!same_shape(x, q)) return fail(PWQ_ERR_SHAPE, "q shape != x shape");
-    View vx, vq;
-    Extent ex, eq;
-    pwq_status st;
-    if ((st = check_tensor(x, Kind::kBF16, &vx, &ex, "x")) != PWQ_OK) return st;
-    if ((st = check_tensor(q, Kind::kByte, &vq, &eq, "q")) != PWQ_OK) return st;
-    if (x->cols % 32 != 0) return fail(PWQ_ERR_SHAPE, "cols % 32 != 0");
-    if (empty(x)) return PWQ_OK;
-    if (!scale) return fail(PWQ_ERR_NULL, "scale");
-    if (x->rows * (x->cols / 8) > kMaxU32 / 2) return fail(PWQ_ERR_SHAPE, "matrix too large");
-    const Extent es = extent_of(scale, (size_t)(x->batch * x->rows * (x->cols / 32)));
-    const Extent ins[1] = {ex};
-    const Extent outs[2] = {eq, es};
-    if ((st = check_overlaps(ins, 1, outs, 2)) != PWQ_OK) return st;
-    return from_cuda(pwq::launch_mxfp8_quant(vx, vq, scale, (cudaStream_t)stream));
+    void* sc[1] = {scale};
+    return run_list(Op::kMxQuant, 1, x, q, sc, nullptr, stream);
 }
 
 pwq_status mxfp8_dequant(const pwq_tensor* q, const uint8_t* scale, const pwq_tensor* y, pwq_stream_t stream) {
     if (!q || !y) return fail(PWQ_ERR_NULL, "tensor descriptor");
-    if (!same_shape(q, y)) return fail(PWQ_ERR_SHAPE, "y shape != q shape");
-    View vq, vy;
-    Extent eq, ey;
-    pwq_status st;
-    if ((st = check_tensor(q, Kind::kByte, &vq, &eq, "q")) != PWQ_OK) return st;
-    if ((st = check_tensor(y, Kind::kBF16, &vy, &ey, "y")) != PWQ_OK) return st;
-    if (q->cols % 32 != 0) return fail(PWQ_ERR_SHAPE, "cols % 32 != 0");
-    if (empty(q)) return PWQ_OK;
-    if (!scale) return fail(PWQ_ERR_NULL, "scale");
-    if (q->rows * (q->cols / 8) > kMaxU32 / 2) return fail(PWQ_ERR_SHAPE, "matrix too large");
-    const Extent es = extent_of(scale, (size_t)(q->batch * q->rows * (q->cols / 32)));
-    const Extent ins[2] = {eq, es};
-    const Extent outs[1] = {ey};
-    if ((st = check_overlaps(ins, 2, outs, 1)) != PWQ_OK) return st;
-    return from_cuda(pwq::launch_mxfp8_dequant(vq, scale, vy, (cudaStream_t)stream));
+    void* sc[1] = {const_cast<uint8_t*>(scale)};
+    return run_list(Op::kMxDequant, 1, q, y, sc, nullptr, stream);
 }
 
-// ------------------------------------------------------------------ NVFP4
+pwq_status nvfp4_dequant(const pwq_tensor* q_packed, const uint8_t* sb, const float* global_scale,
+                         const pwq_tensor* y, pwq_stream_t stream) {
+    if (!q_packed || !y) return fail(PWQ_ERR_NULL, "tensor descriptor");
+    void* sc[1] = {const_cast<uint8_t*>(sb)};
+    const float* g[1] = {global_scale};
+    return run_list(Op::kNvDequant, 1, q_packed, y, sc, g, stream);
+}
+
+pwq_status fp8_block_quant_grouped(int n, const pwq_tensor* x, const pwq_tensor* q, float* const* scale,
+                                   pwq_stream_t stream) {
+    return run_list(Op::kFp8Quant, n, x, q, reinterpret_cast<void* const*>(scale), nullptr, stream);
+}
+
+pwq_status fp8_block_dequant_grouped(int n, const pwq_tensor* q, const float* const* scale, const pwq_tensor* y,
+                                     pwq_stream_t stream) {
+    return run_list(Op::kFp8Dequant, n, q, y, reinterpret_cast<void* const*>(const_cast<float**>(scale)),
+                    nullptr, stream);
+}
+
+pwq_status mxfp8_quant_grouped(int n, const pwq_tensor* x, const pwq_tensor* q, uint8_t* const* scale,
+                               pwq_stream_t stream) {
+    return run_list(Op::kMxQuant, n, x, q, reinterpret_cast<void* const*>(scale), nullptr, stream);
+}
+
+pwq_status mxfp8_dequant_grouped(int n, const pwq_tensor* q, const uint8_t* const* scale, const pwq_tensor* y,
+                                 pwq_stream_t stream) {
+    return run_list(Op::kMxDequant, n, q, y, reinterpret_cast<void* const*>(const_cast<uint8_t**>(scale)),
+                    nullptr, stream);
+}
+
+pwq_status nvfp4_dequant_grouped(int n, const pwq_tensor* q_packed, const uint8_t* const* sb,
+                                 const float* const* global_scale, const pwq_tensor* y, pwq_stream_t stream) {
+    return run_list(Op::kNvDequant, n, q_packed, y, reinterpret_cast<void* const*>(const_cast<uint8_t**>(sb)),
+                    global_scale, stream);
+}
+
+// ------------------------------------------------------------------ NVFP4 quantise / fake-quantise
 
 namespace {
 
@@ -256,10 +337,76 @@ pwq_status check_siblings(const pwq_tensor* x, int n, View* vx, Extent* ex, bool
         if (st != PWQ_OK) return st;
         if (x[i].batch != x[0].batch) return fail(PWQ_ERR_ARG, "siblings differ in batch");
         if (x[i].cols % 16 != 0) return fail(PWQ_ERR_SHAPE, "cols % 16 != 0");
-        if (x[i].rows * (x[i].cols / 8) > kMaxU32) return fail(PWQ_ERR_SHAPE, "matrix too large");
         if (!empty(&x[i])) *all_empty = false;
     }
     if (x[0].batch > 65535) return fail(PWQ_ERR_SHAPE, "batch > 65535");
+    return PWQ_OK;
+}
+
+// One validated NVFP4 sibling group of a (possibly grouped) call.
+struct GroupCheck {
+    View x[PWQ_MAX_SIBLINGS], out[PWQ_MAX_SIBLINGS];
+    uint8_t* sb[PWQ_MAX_SIBLINGS];
+    int n;
+    bool all_empty;
+};
+
+// Validates group g (x, out of n members; sb for quantise) and appends the
+// extents of its inputs and outputs.  y[i] == x[i] exactly is allowed for
+// fake-quantise.
+pwq_status check_nv_group(const pwq_tensor* x, const pwq_tensor* out, uint8_t* const* sb, int n, bool fake,
+                          GroupCheck* G, std::vector<Extent>& ins, std::vector<Extent>& outs,
+                          std::vector<std::pair<Extent, Extent>>& aliases) {
+    Extent ex[PWQ_MAX_SIBLINGS];
+    pwq_status st = check_siblings(x, n, G->x, ex, &G->all_empty);
+    if (st != PWQ_OK) return st;
+    if (!out) return fail(PWQ_ERR_NULL, fake ? "y" : "q_packed");
+    if (!fake && !sb) return fail(PWQ_ERR_NULL, "sb");
+    G->n = n;
+    const int64_t B = x[0].batch;
+    for (int i = 0; i < n; ++i) {
+        if (!same_shape(&x[i], &out[i])) return fail(PWQ_ERR_SHAPE, "output shape != input shape");
+        Extent eo;
+        if ((st = check_tensor(&out[i], fake ? Kind::kBF16 : Kind::kPacked4, &G->out[i], &eo, "output")) !=
+            PWQ_OK)
+            return st;
+        G->sb[i] = nullptr;
+        if (empty(&x[i])) continue;
+        if (fake && exact_alias(&x[i], &out[i])) {
+            aliases.push_back({ex[i], eo});   // in place: checked against everything else
+        } else {
+            ins.push_back(ex[i]);
+            outs.push_back(eo);
+        }
+        if (!fake) {
+            if (!sb[i]) return fail(PWQ_ERR_NULL, "sb[i]");
+            G->sb[i] = sb[i];
+            outs.push_back(extent_of(sb[i], (size_t)(B * x[i].rows * (x[i].cols / 16))));
+        }
+    }
+    return PWQ_OK;
+}
+
+// Overlap rules with in-place members: an aliased pair counts as an output
+// that may coincide with exactly its own input.
+pwq_status check_nv_overlaps(const std::vector<Extent>& ins, const std::vector<Extent>& outs,
+                             const std::vector<std::pair<Extent, Extent>>& aliases) {
+    pwq_status st = check_overlaps(ins.data(), (int)ins.size(), outs.data(), (int)outs.size());
+    if (st != PWQ_OK) return st;
+    for (size_t i = 0; i < aliases.size(); ++i) {
+        for (const Extent& e : ins)
+            if (overlaps(aliases[i].second, e)) return fail(PWQ_ERR_OVERLAP, "y[i] overlaps an input");
+        for (const Extent& e : outs)
+            if (overlaps(aliases[i].second, e)) return fail(PWQ_ERR_OVERLAP, "two outputs overlap");
+        for (size_t j = i + 1; j < aliases.size(); ++j)
+            if (overlaps(aliases[i].second, aliases[j].second)) return fail(PWQ_ERR_OVERLAP, "two outputs overlap");
+    }
+    return PWQ_OK;
+}
+
+pwq_status check_workspace(void* ws, size_t bytes, int64_t instances) {
+    if (!ws || (uintptr_t)ws % 4 != 0 || bytes < pwq::nvfp4_flow_workspace_bytes(instances))
+        return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
     return PWQ_OK;
 }
 
@@ -267,8 +414,19 @@ pwq_status check_siblings(const pwq_tensor* x, int n, View* vx, Extent* ex, bool
 
 size_t nvfp4_workspace_size(int n_siblings, const pwq_tensor* x) {
     if (!x || n_siblings < 1 || n_siblings > PWQ_MAX_SIBLINGS || x[0].batch < 0) return 0;
-    const size_t b = (size_t)std::max<int64_t>(1, x[0].batch);
-    return (b * 4 + 255) / 256 * 256;
+    return pwq::nvfp4_flow_workspace_bytes(std::max<int64_t>(1, x[0].batch));
+}
+
+size_t nvfp4_workspace_size_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x) {
+    if (!x || !group_sizes || n_groups < 1) return 0;
+    int64_t inst = 0;
+    int m = 0;
+    for (int g = 0; g < n_groups; ++g) {
+        if (group_sizes[g] < 1 || group_sizes[g] > PWQ_MAX_SIBLINGS) return 0;
+        inst += std::max<int64_t>(0, x[m].batch);
+        m += group_sizes[g];
+    }
+    return pwq::nvfp4_flow_workspace_bytes(std::max<int64_t>(1, inst));
 }
 
 pwq_status nvfp4_group_amax(const pwq_tensor* x, int n_siblings, float* amax_out, pwq_stream_t stream) {
@@ -286,129 +444,103 @@ pwq_status nvfp4_group_amax(const pwq_tensor* x, int n_siblings, float* amax_out
                                             (cudaStream_t)stream));
 }
 
+namespace {
+
+// Shared body of nvfp4_quant / nvfp4_fake_quant and their grouped forms.
+pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq_tensor* out,
+                  uint8_t* const* sb, float* const* gs_out, const float* amax_in, float* const* amax_out,
+                  void* ws, size_t ws_bytes, bool fake, pwq_stream_t stream) {
+    if (n_groups < 1 || n_groups > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group count out of range");
+    if (!sizes || !x || !out) return fail(PWQ_ERR_NULL, "group sizes / tensors");
+    std::vector<GroupCheck> groups(n_groups);
+    std::vector<Extent> ins, outs;
+    std::vector<std::pair<Extent, Extent>> aliases;
+    std::vector<pwq::NvGroup> launch;
+    int m = 0;
+    int64_t instances = 0;
+    for (int g = 0; g < n_groups; ++g) {
+        const int n = sizes[g];
+        if (n < 1 || n > PWQ_MAX_SIBLINGS || m + n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group size");
+        GroupCheck& G = groups[g];
+        pwq_status st = check_nv_group(x + m, out + m, fake ? nullptr : sb + m, n, fake, &G, ins, outs, aliases);
+        if (st != PWQ_OK) return st;
+        const int64_t B = x[m].batch;
+        if (!G.all_empty && B > 0) {
+            pwq::NvGroup ng;
+            ng.x = G.x;
+            ng.out = G.out;
+            ng.sb = fake ? nullptr : G.sb;
+            ng.n = n;
+            ng.amax_in = amax_in;
+            ng.gs_out = nullptr;
+            ng.amax_out = nullptr;
+            if (!fake) {
+                if (!gs_out || !gs_out[g]) return fail(PWQ_ERR_NULL, "global_scale");
+                if ((uintptr_t)gs_out[g] % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
+                ng.gs_out = gs_out[g];
+                outs.push_back(extent_of(gs_out[g], (size_t)B * 4));
+            }
+            if (amax_out && amax_out[g]) {
+                if ((uintptr_t)amax_out[g] % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_out");
+                ng.amax_out = amax_out[g];
+                outs.push_back(extent_of(amax_out[g], (size_t)B * 4));
+            }
+            launch.push_back(ng);
+            instances += B;
+        }
+        m += n;
+    }
+    if (amax_in) {
+        if (n_groups != 1) return fail(PWQ_ERR_ARG, "amax_in needs a single group");
+        if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
+        ins.push_back(extent_of(amax_in, (size_t)x[0].batch * 4));
+    }
+    if (launch.empty()) return PWQ_OK;
+    if (!amax_in) {
+        pwq_status st = check_workspace(ws, ws_bytes, instances);
+        if (st != PWQ_OK) return st;
+        outs.push_back(extent_of(ws, pwq::nvfp4_flow_workspace_bytes(instances)));
+    }
+    pwq_status st = check_nv_overlaps(ins, outs, aliases);
+    if (st != PWQ_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (amax_in) {
+        const pwq::NvGroup& G = launch[0];
+        return from_cuda(pwq::launch_nvfp4_encode(G.x, G.n, G.out, G.sb, fake, nullptr, amax_in, G.gs_out,
+                                                  G.amax_out, s));
+    }
+    return from_cuda(pwq::launch_nvfp4_flow(launch.data(), (int)launch.size(), fake, ws, s));
+}
+
+}  // namespace
+
 pwq_status nvfp4_quant(const pwq_tensor* x, int n_siblings, const pwq_tensor* q_packed, uint8_t* const* sb,
                        float* global_scale, const float* amax_in, void* workspace, size_t workspace_bytes,
                        pwq_stream_t stream) {
-    View vx[PWQ_MAX_SIBLINGS], vq[PWQ_MAX_SIBLINGS];
-    Extent ex[PWQ_MAX_SIBLINGS + 1], eo[3 * PWQ_MAX_SIBLINGS + 2];
-    bool all_empty;
-    pwq_status st = check_siblings(x, n_siblings, vx, ex, &all_empty);
-    if (st != PWQ_OK) return st;
-    if (!q_packed || !sb) return fail(PWQ_ERR_NULL, "q_packed / sb");
-    int n_out = 0;
-    for (int i = 0; i < n_siblings; ++i) {
-        if (!same_shape(&x[i], &q_packed[i])) return fail(PWQ_ERR_SHAPE, "q_packed[i] shape != x[i] shape");
-        if ((st = check_tensor(&q_packed[i], Kind::kPacked4, &vq[i], &eo[n_out++], "q_packed[i]")) != PWQ_OK)
-            return st;
-    }
-    if (all_empty || x[0].batch == 0) return PWQ_OK;
-    const int64_t B = x[0].batch;
-    for (int i = 0; i < n_siblings; ++i) {
-        if (empty(&x[i])) continue;
-        if (!sb[i]) return fail(PWQ_ERR_NULL, "sb[i]");
-        eo[n_out++] = extent_of(sb[i], (size_t)(B * x[i].rows * (x[i].cols / 16)));
-    }
-    if (!global_scale) return fail(PWQ_ERR_NULL, "global_scale");
-    if ((uintptr_t)global_scale % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
-    eo[n_out++] = extent_of(global_scale, (size_t)B * 4);
-    int n_in = n_siblings;
-    if (amax_in) {
-        if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
-        ex[n_in++] = extent_of(amax_in, (size_t)B * 4);
-    } else {
-        if (!workspace || (uintptr_t)workspace % 4 != 0 || workspace_bytes < (size_t)B * 4)
-            return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
-        eo[n_out++] = extent_of(workspace, (size_t)B * 4);
-    }
-    if ((st = check_overlaps(ex, n_in, eo, n_out)) != PWQ_OK) return st;
-    cudaStream_t s = (cudaStream_t)stream;
-    uint32_t* amax_bits = static_cast<uint32_t*>(workspace);
-    if (!amax_in) {
-        cudaError_t e = pwq::launch_nvfp4_amax(vx, n_siblings, amax_bits, s);
-        if (e != cudaSuccess) return cuda_fail(e);
-    }
-    return from_cuda(pwq::launch_nvfp4_encode(vx, n_siblings, vq, sb, false, amax_in ? nullptr : amax_bits,
-                                              amax_in, global_scale, nullptr, s));
-}
-
-pwq_status nvfp4_dequant(const pwq_tensor* q_packed, const uint8_t* sb, const float* global_scale,
-                         const pwq_tensor* y, pwq_stream_t stream) {
-    if (!q_packed || !y) return fail(PWQ_ERR_NULL, "tensor descriptor");
-    if (!same_shape(q_packed, y)) return fail(PWQ_ERR_SHAPE, "y shape != q_packed shape");
-    View vq, vy;
-    Extent eq, ey;
-    pwq_status st;
-    if ((st = check_tensor(q_packed, Kind::kPacked4, &vq, &eq, "q_packed")) != PWQ_OK) return st;
-    if ((st = check_tensor(y, Kind::kBF16, &vy, &ey, "y")) != PWQ_OK) return st;
-    if (q_packed->cols % 16 != 0) return fail(PWQ_ERR_SHAPE, "cols % 16 != 0");
-    if (empty(q_packed)) return PWQ_OK;
-    if (!sb || !global_scale) return fail(PWQ_ERR_NULL, "sb / global_scale");
-    if ((uintptr_t)global_scale % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
-    if (q_packed->batch * q_packed->rows * (q_packed->cols / 8) > kMaxU32)
-        return fail(PWQ_ERR_SHAPE, "too large");
-    const int64_t B = q_packed->batch;
-    const Extent ins[3] = {eq, extent_of(sb, (size_t)(B * q_packed->rows * (q_packed->cols / 16))),
-                           extent_of(global_scale, (size_t)B * 4)};
-    const Extent outs[1] = {ey};
-    if ((st = check_overlaps(ins, 3, outs, 1)) != PWQ_OK) return st;
-    return from_cuda(pwq::launch_nvfp4_dequant(vq, sb, global_scale, vy, (cudaStream_t)stream));
+    const int sizes[1] = {n_siblings};
+    float* gs[1] = {global_scale};
+    return nv_run(1, sizes, x, q_packed, sb, gs, amax_in, nullptr, workspace, workspace_bytes, false, stream);
 }
 
 pwq_status nvfp4_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_siblings, const float* amax_in,
                             float* amax_out, void* workspace, size_t workspace_bytes, pwq_stream_t stream) {
-    View vx[PWQ_MAX_SIBLINGS], vy[PWQ_MAX_SIBLINGS];
-    Extent ex[PWQ_MAX_SIBLINGS + 1], ey[PWQ_MAX_SIBLINGS + 2];
-    bool all_empty;
-    pwq_status st = check_siblings(x, n_siblings, vx, ex, &all_empty);
-    if (st != PWQ_OK) return st;
-    if (!y) return fail(PWQ_ERR_NULL, "y");
-    for (int i = 0; i < n_siblings; ++i) {
-        if (!same_shape(&x[i], &y[i])) return fail(PWQ_ERR_SHAPE, "y[i] shape != x[i] shape");
-        if ((st = check_tensor(&y[i], Kind::kBF16, &vy[i], &ey[i], "y[i]")) != PWQ_OK) return st;
-    }
-    if (all_empty || x[0].batch == 0) return PWQ_OK;
-    const int64_t B = x[0].batch;
-    // y[i] may alias x[i] exactly; any other intersection is an error
-    for (int i = 0; i < n_siblings; ++i) {
-        for (int j = 0; j < n_siblings; ++j) {
-            if (i == j && exact_alias(&x[i], &y[i])) continue;
-            if (overlaps(ey[i], ex[j])) return fail(PWQ_ERR_OVERLAP, "y[i] overlaps an input");
-        }
-        for (int j = i + 1; j < n_siblings; ++j)
-            if (overlaps(ey[i], ey[j])) return fail(PWQ_ERR_OVERLAP, "two outputs overlap");
-    }
-    int n_in = n_siblings, n_out = 0;
-    Extent extra_out[2];
-    if (amax_in) {
-        if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
-        ex[n_in++] = extent_of(amax_in, (size_t)B * 4);
-    } else {
-        if (!workspace || (uintptr_t)workspace % 4 != 0 || workspace_bytes < (size_t)B * 4)
-            return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
-        extra_out[n_out++] = extent_of(workspace, (size_t)B * 4);
-    }
-    if (amax_out) {
-        if ((uintptr_t)amax_out % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_out");
-        extra_out[n_out++] = extent_of(amax_out, (size_t)B * 4);
-    }
-    for (int k = 0; k < n_out; ++k) {
-        for (int j = 0; j < n_in; ++j)
-            if (overlaps(extra_out[k], ex[j])) return fail(PWQ_ERR_OVERLAP, "amax/workspace overlaps an input");
-        for (int i = 0; i < n_siblings; ++i)
-            if (overlaps(extra_out[k], ey[i])) return fail(PWQ_ERR_OVERLAP, "amax/workspace overlaps y");
-        for (int j = k + 1; j < n_out; ++j)
-            if (overlaps(extra_out[k], extra_out[j])) return fail(PWQ_ERR_OVERLAP, "amax_out overlaps workspace");
-    }
-    for (int i = 0; i < n_siblings; ++i)
-        if (amax_in && overlaps(ey[i], ex[n_siblings])) return fail(PWQ_ERR_OVERLAP, "y overlaps amax_in");
-    cudaStream_t s = (cudaStream_t)stream;
-    uint32_t* amax_bits = static_cast<uint32_t*>(workspace);
-    if (!amax_in) {
-        cudaError_t e = pwq::launch_nvfp4_amax(vx, n_siblings, amax_bits, s);
-        if (e != cudaSuccess) return cuda_fail(e);
-    }
-    return from_cuda(pwq::launch_nvfp4_encode(vx, n_siblings, vy, nullptr, true, amax_in ? nullptr : amax_bits,
-                                              amax_in, nullptr, amax_out, s));
+    const int sizes[1] = {n_siblings};
+    float* ao[1] = {amax_out};
+    return nv_run(1, sizes, x, y, nullptr, nullptr, amax_in, ao, workspace, workspace_bytes, true, stream);
+}
+
+pwq_status nvfp4_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                               const pwq_tensor* q_packed, uint8_t* const* sb, float* const* global_scale,
+                               void* workspace, size_t workspace_bytes, pwq_stream_t stream) {
+    return nv_run(n_groups, group_sizes, x, q_packed, sb, global_scale, nullptr, nullptr, workspace,
+                  workspace_bytes, false, stream);
+}
+
+pwq_status nvfp4_fake_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                                    const pwq_tensor* y, float* const* amax_out, void* workspace,
+                                    size_t workspace_bytes, pwq_stream_t stream) {
+    return nv_run(n_groups, group_sizes, x, y, nullptr, nullptr, nullptr, amax_out, workspace, workspace_bytes,
+                  true, stream);
 }
 
 // ------------------------------------------------------------------ no-allocation variant
@@ -471,7 +603,7 @@ pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, in
 
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream) {
     if (!counts) return fail(PWQ_ERR_NULL, "counts");
-    if (which < 0 || which > 2) return fail(PWQ_ERR_ARG, "which");
+    if (which < 0 || which > 3) return fail(PWQ_ERR_ARG, "which");
     return from_cuda(pwq::launch_selftest_division(which, counts, (cudaStream_t)stream));
 }
 

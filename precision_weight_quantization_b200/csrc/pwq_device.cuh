@@ -49,7 +49,13 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 
 // Four binary32 -> four E4M3 codes in a 32-bit word (element 0 in byte 0).
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
-    return e4m3x2(a, b) | (e4m3x2(c, d) << 16);
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r) : "f"(a), "f"(b), "f"(c), "f"(d));
+    return r;
 }
 
 // Two E4M3 codes (lo in bits 0..7) -> exact binary32 values.
@@ -72,6 +78,21 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
     uint32_t r;
     asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
         : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Eight binary32 -> eight E2M1 codes in a 32-bit word (element 0 in bits
+// 0..3, element 2j in the low nibble of byte j).
+__device__ __forceinline__ uint32_t e2m1x8(const float (&q)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
     return r;
 }
 
@@ -165,6 +186,16 @@ __device__ __forceinline__ float div_slow(float x, float s) {
 template <bool kFast>
 __device__ __forceinline__ float quotient(float x, float s, float r) {
     return kFast ? div_fast(x, s, r) : div_slow(x, s);
+}
+
+// FP8 block-wise tile scale s = fl(amax / 448).  The divisor is the
+// constant 448, so its reciprocal RN(1/448) = 0x3b124925 is exact input to
+// the reciprocal path, which gives the IEEE quotient for amax >= 2^-100;
+// smaller (BF16-subnormal-range) amax use IEEE division.  s is stored, so
+// pwq_selftest_division checks it bit for bit for every BF16 amax.
+__device__ __forceinline__ float fp8_tile_scale(float amax) {
+    return amax >= 0x1p-100f ? div_fast(amax, 448.0f, __uint_as_float(0x3b124925u))
+                             : __fdiv_rn(amax, 448.0f);
 }
 
 // The quotients of the two BF16 values of a packed word.

@@ -24,26 +24,58 @@ int current_device();
 // `work_ctas`, at most `per_sm` resident CTAs per SM.
 int persistent_grid(int64_t work_ctas, int per_sm);
 
-cudaError_t launch_fp8_block_quant(const View& x, const View& q, float* scale, cudaStream_t s);
-cudaError_t launch_fp8_block_dequant(const View& q, const float* scale, const View& y, cudaStream_t s);
-cudaError_t launch_mxfp8_quant(const View& x, const View& q, uint8_t* scale, cudaStream_t s);
-cudaError_t launch_mxfp8_dequant(const View& q, const uint8_t* scale, const View& y, cudaStream_t s);
+// Tensors per kernel launch of a grouped call (their descriptors, TMA maps
+// included, travel as kernel parameters); longer lists are split.
+constexpr int kMaxLaunchTensors = 16;
 
-// NVFP4.  amax_bits: B words holding max |x| of each group as binary32 bits.
+// One independent tensor of a grouped elementwise call.
+struct Job {
+    View in, out;
+    void* scale;       // FP8: float [B][TM][TN]; MXFP8: uint8 [B][M][N/32]; NVFP4 dequant: uint8 sb [B][M][N/16]
+    const float* gs;   // NVFP4 dequant: [B]
+};
+
+cudaError_t launch_fp8_block_quant(const Job* jobs, int n, cudaStream_t s);
+cudaError_t launch_fp8_block_dequant(const Job* jobs, int n, cudaStream_t s);
+cudaError_t launch_mxfp8_quant(const Job* jobs, int n, cudaStream_t s);
+cudaError_t launch_mxfp8_dequant(const Job* jobs, int n, cudaStream_t s);
+cudaError_t launch_nvfp4_dequant(const Job* jobs, int n, cudaStream_t s);
+
+// NVFP4 sibling group: members share the per-batch-index group amax.
+struct NvGroup {
+    const View* x;          // n members
+    const View* out;        // packed codes (quant) or BF16 (fake-quant)
+    uint8_t* const* sb;     // quant: n block-scale arrays [B][M][N/16]; fake: null
+    int n;
+    const float* amax_in;   // [B] or null
+    float* gs_out;          // [B] or null
+    float* amax_out;        // [B] or null
+};
+
+// NVFP4 single-pass quantise / fake-quantise of groups whose amax is reduced
+// on the device (amax_in null for every group): one dataflow launch per
+// piece.  Workspace: nvfp4_flow_workspace_bytes(total batch over groups).
+size_t nvfp4_flow_workspace_bytes(int64_t instances);
+cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, void* workspace,
+                              cudaStream_t s);
+
+// Two-launch NVFP4 path for one group set (used with a precomputed amax and
+// by the no-allocation entry point).  amax_bits: B words holding max |x| of
+// each group as binary32 bits.
 cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStream_t s);
 cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* const* sb,
                                 bool fake, const uint32_t* amax_bits, const float* amax_in,
                                 float* gs_out, float* amax_out, cudaStream_t s);
-cudaError_t launch_nvfp4_dequant(const View& q, const uint8_t* sb, const float* gs, const View& y,
-                                 cudaStream_t s);
 
 // Device address (on the current device) of the file-scope group-amax
 // scratch used by nvfp4_fake_quant_noalloc; kStaticScratchGroups words.
 constexpr int64_t kStaticScratchGroups = 4096;
 cudaError_t static_amax_scratch(uint32_t** ptr);
 
-// Reads and clears the device error word (synchronous).
+// Read and clear the device error words (synchronous): TMA waits (FP8
+// block-wise quantise) and the NVFP4 single-pass amax waits.
 cudaError_t read_and_clear_device_error(uint32_t* code);
+cudaError_t read_and_clear_flow_error(uint32_t* code);
 
 cudaError_t launch_selftest_division(int which, unsigned long long* counts, cudaStream_t s);
 cudaError_t launch_selftest_codecs(uint32_t first, uint32_t count, uint8_t* e4m3, uint8_t* e2m1,

@@ -4,7 +4,8 @@
 // correctly rounded reciprocal per tile/block and an FMA residual correction
 // (pwq_device.cuh).  The numerators are BF16 values and the divisors come
 // from small finite sets (FP8 block-wise: fl(a / 448); NVFP4:
-// fl(dec(sb) * fl(a / 2688)), a a positive BF16, sb a non-zero E4M3 code), so
+// fl(dec(sb) * fl(a / 2688)) and fl(6 * fl(a / 2688)), a a positive BF16,
+// sb a non-zero E4M3 code), so
 // every (numerator, divisor) pair can be enumerated and compared with CUDA's
 // IEEE division __fdiv_rn in well under a second.
 //
@@ -94,6 +95,30 @@ __global__ void __launch_bounds__(kThreads) selftest_division_kernel(unsigned lo
     }
 }
 
+// FP8 tile scale: fp8_tile_scale(a) against fl(a / 448) for every finite
+// non-negative BF16 a.
+__global__ void __launch_bounds__(kThreads) selftest_tile_scale_kernel(unsigned long long* counts) {
+    unsigned long long n = 0, bad = 0, slow = 0;
+    for (uint32_t ab = blockIdx.x * blockDim.x + threadIdx.x; ab < 0x7f80u; ab += gridDim.x * blockDim.x) {
+        const float a = __uint_as_float(ab << 16);
+        ++n;
+        bad += __float_as_uint(fp8_tile_scale(a)) != __float_as_uint(__fdiv_rn(a, 448.0f));
+        slow += !(a >= 0x1p-100f);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n += __shfl_xor_sync(0xffffffffu, n, o);
+        bad += __shfl_xor_sync(0xffffffffu, bad, o);
+        slow += __shfl_xor_sync(0xffffffffu, slow, o);
+    }
+    if ((threadIdx.x & 31u) == 0u) {
+        atomicAdd(counts + 0, n);
+        atomicAdd(counts + 1, bad);
+        atomicAdd(counts + 2, bad);
+        atomicAdd(counts + 3, slow);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads)
 selftest_codecs_kernel(uint32_t first, uint32_t count, uint8_t* e4m3, uint8_t* e2m1, uint16_t* bf16) {
     const uint32_t stride = gridDim.x * blockDim.x;
@@ -114,8 +139,10 @@ cudaError_t launch_selftest_division(int which, unsigned long long* counts, cuda
         selftest_division_kernel<0><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
     else if (which == 1)
         selftest_division_kernel<1><<<dim3(0x7f7f, 0x7e), kThreads, 0, s>>>(counts);
-    else
+    else if (which == 2)
         selftest_division_kernel<2><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
+    else
+        selftest_tile_scale_kernel<<<dim3(64), kThreads, 0, s>>>(counts);
     return cudaGetLastError();
 }
 
