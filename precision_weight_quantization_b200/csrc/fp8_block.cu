@@ -48,7 +48,6 @@ struct TileTensor {
     uint32_t tile_begin;  // first tile of this tensor in the launch
     FastDiv tiles_n;      // tiles per tile row (TN)
     FastDiv tiles_mn;     // tiles per batch matrix (TM * TN)
-    int vec16;            // dequant: code rows 16-byte aligned
 };
 
 struct TileLoc {
@@ -212,17 +211,18 @@ fp8_block_quant_kernel(const __grid_constant__ QuantArgs a) {
 }
 
 // Dequantise: a persistent grid walks the tiles of the list; the tile scale
-// is one load per tile.  Thread t owns 16-code chunks at column (t & 7) * 16
-// of rows (t >> 3) + 32 j, j = 0..3: a 16-byte code load becomes two 16-byte
-// BF16 stores.  Edge tiles take a masked element-wise path.
+// is one load per tile.  Thread t owns 8-code chunks at column (t & 15) * 8
+// of rows (t >> 4) + 16 j, j = 0..7 (the quantiser's mapping): an 8-byte
+// code load becomes one 16-byte BF16 store, and the 16 lanes of a row write
+// 256 contiguous bytes.  Edge tiles take a masked element-wise path.
 struct DequantArgs {
     TileTensor t[kMaxLaunchTensors];
     int n;
     uint32_t total_tiles;
 };
 
-constexpr int kDqRowsPerPass = kThreads / 8;         // 32
-constexpr int kDqChunks = kTile / kDqRowsPerPass;     // 4
+constexpr int kDqRowsPerPass = kThreads / 16;        // 16
+constexpr int kDqChunks = kTile / kDqRowsPerPass;     // 8
 
 __device__ __forceinline__ uint4 dequant8(uint2 codes, float s) {
     uint32_t w[4];
@@ -236,8 +236,8 @@ __device__ __forceinline__ uint4 dequant8(uint2 codes, float s) {
 }
 
 __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const __grid_constant__ DequantArgs a) {
-    const int ccol = (int)(threadIdx.x & 7u) * 16;
-    const int row0 = (int)(threadIdx.x >> 3);
+    const int ccol = (int)(threadIdx.x & 15u) * 8;
+    const int row0 = (int)(threadIdx.x >> 4);
     for (uint32_t t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
         const TileLoc L = locate(a, t);
         const TileTensor& T = a.t[L.i];
@@ -247,30 +247,20 @@ __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const __gri
         const int rows_here = min(kTile, T.rows - L.tm * kTile);
         const int cols_here = min(kTile, T.cols - L.tn * kTile);
         if (rows_here == kTile && cols_here == kTile) {
-            uint4 v[kDqChunks];
+            uint2 v[kDqChunks];
 #pragma unroll
-            for (int j = 0; j < kDqChunks; ++j) {
-                const char* src = qt + (int64_t)(row0 + kDqRowsPerPass * j) * T.q_rs + ccol;
-                if (T.vec16) {
-                    v[j] = ld_stream_v4(src);
-                } else {
-                    const uint2 lo = ld_stream_v2(src), hi = ld_stream_v2(src + 8);
-                    v[j] = make_uint4(lo.x, lo.y, hi.x, hi.y);
-                }
-            }
+            for (int j = 0; j < kDqChunks; ++j)
+                v[j] = ld_stream_v2(qt + (int64_t)(row0 + kDqRowsPerPass * j) * T.q_rs + ccol);
 #pragma unroll
-            for (int j = 0; j < kDqChunks; ++j) {
-                char* dst = yt + (int64_t)(row0 + kDqRowsPerPass * j) * T.y_rs + ccol * 2;
-                st_v4(dst, dequant8(make_uint2(v[j].x, v[j].y), sc));
-                st_v4(dst + 16, dequant8(make_uint2(v[j].z, v[j].w), sc));
-            }
+            for (int j = 0; j < kDqChunks; ++j)
+                st_v4(yt + (int64_t)(row0 + kDqRowsPerPass * j) * T.y_rs + ccol * 2, dequant8(v[j], sc));
         } else {
             for (int j = 0; j < kDqChunks; ++j) {
                 const int r = row0 + kDqRowsPerPass * j;
                 if (r >= rows_here) break;
                 const unsigned char* src = reinterpret_cast<const unsigned char*>(qt + (int64_t)r * T.q_rs);
                 unsigned short* dst = reinterpret_cast<unsigned short*>(yt + (int64_t)r * T.y_rs);
-                for (int c = ccol; c < min(ccol + 16, cols_here); ++c) {
+                for (int c = ccol; c < min(ccol + 8, cols_here); ++c) {
                     const float f = __fmul_rn(e4m3_decode(src[c]), sc);
                     dst[c] = (unsigned short)(pack_bf16x2(f, 0.0f) & 0xffffu);
                 }
@@ -316,7 +306,6 @@ uint32_t fill_tile_tensor(TileTensor& T, const Job& j, bool quant, uint32_t tile
     T.tile_begin = tile_begin;
     T.tiles_n = make_fastdiv(tn);
     T.tiles_mn = make_fastdiv(tm * tn);
-    T.vec16 = ((uintptr_t)q.ptr % 16 == 0) && (q.rstride % 16 == 0) && (q.batch == 1 || q.bstride % 16 == 0);
     return (uint32_t)q.batch * tm * tn;
 }
 

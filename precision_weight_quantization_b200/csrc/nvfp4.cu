@@ -398,12 +398,48 @@ __device__ __forceinline__ void flow_decode(const uint32_t* pa, uint32_t I, uint
     }
 }
 
+// A decoded queue item.  Thread 0 decodes the next item while the CTA works
+// on the current one and publishes it in a double-buffered shared slot, so
+// each item costs one CTA barrier.
+struct FlowItem {
+    uint32_t valid, is_e, inst, k;   // k: item within its instance's pass (encode: reversed)
+    int g, m;                        // group, member
+    uint32_t b, c0, c1;              // batch index in the group; chunk range of the member slab
+};
+
+__device__ __forceinline__ FlowItem flow_item(const FlowArgs& a, const uint32_t* pa, uint32_t q) {
+    FlowItem it{};
+    it.valid = q < 2u * a.total_items;
+    if (!it.valid) return it;
+    bool is_e;
+    uint32_t inst, k;
+    flow_decode(pa, a.n_inst, q, is_e, inst, k);
+    const int g = flow_group_of(a, inst);
+    const FlowGroup& G = a.g[g];
+    if (is_e) k = G.items - 1u - k;                    // encode walks the instance backwards
+    int mi = G.m_begin;
+    for (int t = 1; t < G.m_count; ++t)
+        if (k >= a.m[G.m_begin + t].item_off) mi = G.m_begin + t;
+    const FlowMember& M = a.m[mi];
+    it.is_e = is_e;
+    it.inst = inst;
+    it.k = k;
+    it.g = g;
+    it.m = mi;
+    it.b = inst - G.inst_begin;
+    it.c0 = (k - M.item_off) * kItemChunks;
+    it.c1 = min(it.c0 + kItemChunks, M.chunks);
+    return it;
+}
+
 template <bool kFake>
-__global__ void __launch_bounds__(kFlowThreads) nvfp4_flow_kernel(const __grid_constant__ FlowArgs a) {
+__global__ void __launch_bounds__(kFlowThreads, 4) nvfp4_flow_kernel(const __grid_constant__ FlowArgs a) {
     __shared__ uint32_t pa[kFlowMaxInst + 1];
     __shared__ ScaleTable tab;
-    __shared__ uint32_t s_item, s_next, s_amax;
-    __shared__ uint32_t red[kFlowThreads / 32];
+    __shared__ FlowItem items[2];
+    __shared__ uint32_t s_amax[2];
+    __shared__ uint32_t red[2][kFlowThreads / 32];
+    __shared__ uint32_t s_q0;
     const uint32_t tid = threadIdx.x;
     for (uint32_t i = tid; i <= a.n_inst; i += blockDim.x) {
         uint32_t v = a.total_items;
@@ -413,35 +449,36 @@ __global__ void __launch_bounds__(kFlowThreads) nvfp4_flow_kernel(const __grid_c
         }
         pa[i] = v;
     }
-    if (tid == 0) s_item = atomicAdd(a.counter, 1u);
+    uint32_t pending = 0u;   // thread 0: queue position of the item after the next
+    if (tid == 0) {
+        s_q0 = atomicAdd(a.counter, 1u);
+        pending = atomicAdd(a.counter, 1u);
+    }
     __syncthreads();
-    const uint32_t total_q = 2u * a.total_items;
-    uint32_t item = s_item;
+    if (tid == 0) items[0] = flow_item(a, pa, s_q0);
+    __syncthreads();
+
+    // the amax pass keeps its data in L2 for the encode pass; the encode
+    // pass and every store stream through
+    const uint64_t keep = l2_policy_evict_last();
+    const uint64_t stream = l2_policy_evict_first();
     uint32_t cached = 0xffffffffu;
     float gs = 0.0f, six_gs = 0.0f, r6 = 0.0f;
     bool fast6 = false;
-    while (item < total_q) {
-        if (tid == 0) s_next = atomicAdd(a.counter, 1u);   // prefetch the next item
-        bool is_e;
-        uint32_t inst, k;
-        flow_decode(pa, a.n_inst, item, is_e, inst, k);
-        const FlowGroup& G = a.g[flow_group_of(a, inst)];
-        const uint32_t b = inst - G.inst_begin;
-        if (is_e) k = G.items - 1u - k;                    // encode walks the instance backwards
-        int mi = G.m_begin;
-        for (int t = 1; t < G.m_count; ++t)
-            if (k >= a.m[G.m_begin + t].item_off) mi = G.m_begin + t;
-        const FlowMember& M = a.m[mi];
-        const uint32_t c0 = (k - M.item_off) * kItemChunks;
-        const uint32_t c1 = min(c0 + kItemChunks, M.chunks);
-        const char* xb = M.x + (int64_t)b * M.x_bs;
-
+    for (uint32_t p = 0;; p ^= 1u) {
+        const FlowItem it = items[p];
+        if (!it.valid) break;
+        uint32_t next_q = 0u;
+        if (tid == 0) next_q = atomicAdd(a.counter, 1u);   // needed one item later
+        const FlowMember& M = a.m[it.m];
+        const char* xb = M.x + (int64_t)it.b * M.x_bs;
+        const uint64_t pol = it.is_e ? stream : keep;
         uint4 v[kItemChunksPerThread];
 #pragma unroll
         for (int j = 0; j < kItemChunksPerThread; ++j) {
-            const uint32_t c = c0 + (uint32_t)j * kFlowThreads + tid;
+            const uint32_t c = it.c0 + (uint32_t)j * kFlowThreads + tid;
             v[j] = make_uint4(0u, 0u, 0u, 0u);
-            if (c < c1) {
+            if (c < it.c1) {
                 int64_t off;
                 if (M.dense_x) {
                     off = (int64_t)c * 16;
@@ -449,91 +486,94 @@ __global__ void __launch_bounds__(kFlowThreads) nvfp4_flow_kernel(const __grid_c
                     const uint32_t r = fdiv(c, M.cpr);
                     off = (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 16;
                 }
-                v[j] = ld_stream_v4(xb + off);
+                v[j] = ld_hint_v4(xb + off, pol);
             }
         }
 
-        if (!is_e) {
+        if (!it.is_e) {
             // ---- amax item
             uint32_t m = 0u;
 #pragma unroll
             for (int j = 0; j < kItemChunksPerThread; ++j) m = max(m, amax_bits8(v[j]));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if ((tid & 31u) == 0u) red[tid >> 5] = m;
+            if ((tid & 31u) == 0u) red[p][tid >> 5] = m;
+            if (tid == 0) {
+                items[p ^ 1u] = flow_item(a, pa, pending);
+                pending = next_q;
+            }
             __syncthreads();
             if (tid == 0) {
-                for (int w = 1; w < kFlowThreads / 32; ++w) m = max(m, red[w]);
-                if (m != 0u) atomicMax(a.amax_bits + inst, m << 16);
+                for (int w = 1; w < kFlowThreads / 32; ++w) m = max(m, red[p][w]);
+                if (m != 0u) atomicMax(a.amax_bits + it.inst, m << 16);
                 __threadfence();
-                atomicAdd(a.done + inst, 1u);
+                atomicAdd(a.done + it.inst, 1u);
             }
-        } else {
-            // ---- encode item: wait for the instance's amax
-            if (tid == 0) {
-                if (ld_acquire_gpu(a.done + inst) < G.items) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(a.done + inst) < G.items) {
-                        if (globaltimer_ns() - t0 > kFlowWaitNs) {
-                            atomicOr(&g_flow_error, kErrFlowTimeout);
-                            break;
-                        }
-                        __nanosleep(200);
+            continue;
+        }
+
+        // ---- encode item: wait (bounded) for the instance's amax
+        const FlowGroup& G = a.g[it.g];
+        if (tid == 0) {
+            items[p ^ 1u] = flow_item(a, pa, pending);
+            pending = next_q;
+            if (ld_acquire_gpu(a.done + it.inst) < G.items) {
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_acquire_gpu(a.done + it.inst) < G.items) {
+                    if (globaltimer_ns() - t0 > kFlowWaitNs) {
+                        atomicOr(&g_flow_error, kErrFlowTimeout);
+                        break;
                     }
+                    __nanosleep(200);
                 }
-                s_amax = ld_relaxed_gpu(a.amax_bits + inst);
             }
+            s_amax[p] = ld_relaxed_gpu(a.amax_bits + it.inst);
+        }
+        __syncthreads();
+        if (it.inst != cached) {   // CTA-uniform
+            gs = __fdiv_rn(__uint_as_float(s_amax[p]), 2688.0f);
+            six_gs = __fmul_rn(6.0f, gs);
+            r6 = __frcp_rn(six_gs);
+            fast6 = div_fast_ok(six_gs);
+            fill_scale_table(tab, gs);
             __syncthreads();
-            if (inst != cached) {   // CTA-uniform
-                const float A = __uint_as_float(s_amax);
-                gs = __fdiv_rn(A, 2688.0f);
-                six_gs = __fmul_rn(6.0f, gs);
-                r6 = __frcp_rn(six_gs);
-                fast6 = div_fast_ok(six_gs);
-                fill_scale_table(tab, gs);
-                if (tid == 0 && k == 0u) {
-                    if (G.gs_out) G.gs_out[b] = gs;
-                    if (G.amax_out) G.amax_out[b] = A;
-                }
-                __syncthreads();
-                cached = inst;
-            } else if (tid == 0 && k == 0u) {
-                if (G.gs_out) G.gs_out[b] = gs;
-                if (G.amax_out) G.amax_out[b] = __uint_as_float(s_amax);
-            }
-            char* ob = M.out + (int64_t)b * M.o_bs;
-            uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)b * (M.chunks >> 1);
+            cached = it.inst;
+        }
+        if (tid == 0 && it.k == 0u) {
+            if (G.gs_out) G.gs_out[it.b] = gs;
+            if (G.amax_out) G.amax_out[it.b] = __uint_as_float(s_amax[p]);
+        }
+        char* ob = M.out + (int64_t)it.b * M.o_bs;
+        uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.chunks >> 1);
 #pragma unroll
-            for (int j = 0; j < kItemChunksPerThread; ++j) {
-                const uint32_t c = c0 + (uint32_t)j * kFlowThreads + tid;
-                uint32_t m = amax_bits8(v[j]);
-                m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));   // lanes 2i, 2i+1: one block
-                const float amax_b = __uint_as_float(m << 16);
-                const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
-                const uint32_t sb = e4m3x2(ratio, 0.0f) & 0xffu;
-                const float4 e = tab.e[sb];
-                const uint32_t codes = codes_half(v[j], e.x, e.y);
-                if (c < c1) {
-                    int64_t oo;
-                    if (M.dense_o) {
-                        oo = (int64_t)c * (kFake ? 16 : 4);
-                    } else {
-                        const uint32_t r = fdiv(c, M.cpr);
-                        oo = (int64_t)r * M.o_rs + (int64_t)(c - r * M.cpr.d) * (kFake ? 16 : 4);
-                    }
-                    if (kFake) {
-                        st_v4(ob + oo, dequant_half(codes, e.z, gs));
-                    } else {
-                        st_u32(ob + oo, codes);
-                        if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)sb;
-                    }
+        for (int j = 0; j < kItemChunksPerThread; ++j) {
+            const uint32_t c = it.c0 + (uint32_t)j * kFlowThreads + tid;
+            uint32_t m = amax_bits8(v[j]);
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));   // lanes 2i, 2i+1: one block
+            const float amax_b = __uint_as_float(m << 16);
+            const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
+            const uint32_t sb = e4m3x2(ratio, 0.0f) & 0xffu;
+            const float4 e = tab.e[sb];
+            const uint32_t codes = codes_half(v[j], e.x, e.y);
+            if (c < it.c1) {
+                int64_t oo;
+                if (M.dense_o) {
+                    oo = (int64_t)c * (kFake ? 16 : 4);
+                } else {
+                    const uint32_t r = fdiv(c, M.cpr);
+                    oo = (int64_t)r * M.o_rs + (int64_t)(c - r * M.cpr.d) * (kFake ? 16 : 4);
+                }
+                if (kFake) {
+                    st_hint_v4(ob + oo, dequant_half(codes, e.z, gs), stream);
+                } else {
+                    st_hint_u32(ob + oo, codes, stream);
+                    if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)sb;
                 }
             }
         }
-        __syncthreads();   // s_next is ready; red / s_amax / tab may be reused
-        item = s_next;
     }
 }
+
 
 bool dense_rows(const View& v, int64_t row_bytes) {
     return v.rstride == row_bytes;
