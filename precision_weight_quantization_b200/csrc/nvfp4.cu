@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_dequant_kernel(const __grid_co
 constexpr int kFlowThreads = 256;
 constexpr uint32_t kItemChunks = 2048;                        // 16384 elements
 constexpr int kItemChunksPerThread = kItemChunks / kFlowThreads;   // 8
-constexpr int kFlowMaxInst = 2048;                            // instances per launch
+constexpr int kFlowMaxInst = 512;                             // instances per launch
 constexpr uint64_t kFlowWaitNs = 2000000000ull;               // 2 s
 constexpr uint32_t kErrFlowTimeout = 2u;
 
@@ -398,9 +398,8 @@ __device__ __forceinline__ void flow_decode(const uint32_t* pa, uint32_t I, uint
     }
 }
 
-// A decoded queue item.  Thread 0 decodes the next item while the CTA works
-// on the current one and publishes it in a double-buffered shared slot, so
-// each item costs one CTA barrier.
+// A decoded queue item.  Thread 0 decodes items two ahead of the CTA and
+// publishes them in a three-slot ring in shared memory.
 struct FlowItem {
     uint32_t valid, is_e, inst, k;   // k: item within its instance's pass (encode: reversed)
     int g, m;                        // group, member
@@ -432,15 +431,98 @@ __device__ __forceinline__ FlowItem flow_item(const FlowArgs& a, const uint32_t*
     return it;
 }
 
+// Starts the data of item `it` into stage buffer `dst` (thread 0): one bulk
+// copy of the item's contiguous bytes when the member slab is dense,
+// otherwise a plain arrival (the item is then read straight from global
+// memory), so that every stage completes one barrier phase per item.
+__device__ __forceinline__ void flow_stage(const FlowArgs& a, const FlowItem& it, uint32_t dst, uint32_t bar,
+                                           uint64_t pol) {
+    const FlowMember& M = a.m[it.m];
+    if (M.dense_x) {
+        const uint32_t bytes = (it.c1 - it.c0) * 16u;
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load(dst, M.x + (int64_t)it.b * M.x_bs + (int64_t)it.c0 * 16, bytes, bar, pol);
+    } else {
+        mbar_arrive(bar);
+    }
+}
+
+constexpr int kFlowStages = 2;
+constexpr uint32_t kFlowStageBytes = kItemChunks * 16u;   // 32 KB
+
+// Encodes the chunks of one item held in registers.  kFast: every block
+// divisor of the instance lies in the reciprocal path's range (checked per
+// instance), so no per-block branch; a zero block scale then has d = 0 and a
+// zero table reciprocal, for which the reciprocal formula yields the signed
+// zero the zero-scale reading asks for.  kFull: all kItemChunks chunks of the
+// item exist and both operands are dense.
+template <bool kFake, bool kFast, bool kFull>
+__device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThread], const FlowItem& it,
+                                            const FlowMember& M, const ScaleTable& tab, float gs, float six_gs,
+                                            float r6, bool fast6, uint64_t pol) {
+    const uint32_t tid = threadIdx.x;
+    char* ob = M.out + (int64_t)it.b * M.o_bs;
+    uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.chunks >> 1);
+#pragma unroll
+    for (int j = 0; j < kItemChunksPerThread; ++j) {
+        const uint32_t c = it.c0 + (uint32_t)j * kFlowThreads + tid;
+        uint32_t m = amax_bits8(v[j]);
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));   // lanes 2i, 2i+1: one block
+        const float amax_b = __uint_as_float(m << 16);
+        float ratio;
+        if (kFast)
+            ratio = div_fast(amax_b, six_gs, r6);
+        else
+            ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
+        const uint32_t sb = e4m3x2(ratio, 0.0f) & 0xffu;
+        const float4 e = tab.e[sb];
+        uint32_t codes;
+        if (kFast) {
+            float q[8];
+            quotients8<true>(v[j], e.x, e.y, q);
+            codes = e2m1x8(q);
+        } else {
+            codes = codes_half(v[j], e.x, e.y);
+        }
+        if (kFull || c < it.c1) {
+            int64_t oo;
+            if (kFull || M.dense_o) {
+                oo = (int64_t)c * (kFake ? 16 : 4);
+            } else {
+                const uint32_t r = fdiv(c, M.cpr);
+                oo = (int64_t)r * M.o_rs + (int64_t)(c - r * M.cpr.d) * (kFake ? 16 : 4);
+            }
+            if (kFake) {
+                st_hint_v4(ob + oo, dequant_half(codes, e.z, gs), pol);
+            } else {
+                st_hint_u32(ob + oo, codes, pol);
+                if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
 template <bool kFake>
-__global__ void __launch_bounds__(kFlowThreads, 4) nvfp4_flow_kernel(const __grid_constant__ FlowArgs a) {
+__global__ void __launch_bounds__(kFlowThreads, 3) nvfp4_flow_kernel(const __grid_constant__ FlowArgs a) {
+    extern __shared__ __align__(128) unsigned char flow_smem[];
     __shared__ uint32_t pa[kFlowMaxInst + 1];
     __shared__ ScaleTable tab;
-    __shared__ FlowItem items[2];
+    __shared__ FlowItem items[3];
+    __shared__ __align__(8) uint64_t bars[kFlowStages];
     __shared__ uint32_t s_amax[2];
     __shared__ uint32_t red[2][kFlowThreads / 32];
-    __shared__ uint32_t s_q0;
+    __shared__ uint32_t s_q[2];
+    // thread 0: queue position of the item two ahead of the next one; stored
+    // at the end of an item so the atomic's latency overlaps warp 0's work
+    __shared__ volatile uint32_t s_pend;
     const uint32_t tid = threadIdx.x;
+    const uint32_t stage0 = smem_addr(flow_smem);
+
+    // the amax pass keeps its data in L2 for the encode pass; the encode
+    // pass and every store stream through
+    const uint64_t keep = l2_policy_evict_last();
+    const uint64_t stream = l2_policy_evict_first();
+
     for (uint32_t i = tid; i <= a.n_inst; i += blockDim.x) {
         uint32_t v = a.total_items;
         if (i < a.n_inst) {
@@ -449,44 +531,60 @@ __global__ void __launch_bounds__(kFlowThreads, 4) nvfp4_flow_kernel(const __gri
         }
         pa[i] = v;
     }
-    uint32_t pending = 0u;   // thread 0: queue position of the item after the next
     if (tid == 0) {
-        s_q0 = atomicAdd(a.counter, 1u);
-        pending = atomicAdd(a.counter, 1u);
+        for (int s = 0; s < kFlowStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+        fence_mbar_init();
+        s_q[0] = atomicAdd(a.counter, 1u);
+        s_q[1] = atomicAdd(a.counter, 1u);
+        s_pend = atomicAdd(a.counter, 1u);
     }
     __syncthreads();
-    if (tid == 0) items[0] = flow_item(a, pa, s_q0);
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            items[s] = flow_item(a, pa, s_q[s]);
+            if (items[s].valid)
+                flow_stage(a, items[s], stage0 + s * kFlowStageBytes, smem_addr(&bars[s]),
+                           items[s].is_e ? stream : keep);
+        }
+    }
     __syncthreads();
 
-    // the amax pass keeps its data in L2 for the encode pass; the encode
-    // pass and every store stream through
-    const uint64_t keep = l2_policy_evict_last();
-    const uint64_t stream = l2_policy_evict_first();
     uint32_t cached = 0xffffffffu;
     float gs = 0.0f, six_gs = 0.0f, r6 = 0.0f;
-    bool fast6 = false;
-    for (uint32_t p = 0;; p ^= 1u) {
-        const FlowItem it = items[p];
+    bool fast6 = false, all_fast = false;
+    for (uint32_t k = 0;; ++k) {
+        const uint32_t slot = k % 3u, st = k & 1u, par = (k >> 1) & 1u;
+        const FlowItem it = items[slot];
         if (!it.valid) break;
         uint32_t next_q = 0u;
-        if (tid == 0) next_q = atomicAdd(a.counter, 1u);   // needed one item later
+        if (tid == 0) next_q = atomicAdd(a.counter, 1u);   // decoded two items later
         const FlowMember& M = a.m[it.m];
-        const char* xb = M.x + (int64_t)it.b * M.x_bs;
-        const uint64_t pol = it.is_e ? stream : keep;
+
+        // ---- the item's data, into registers
+        if (!mbar_wait_bounded(smem_addr(&bars[st]), par, kFlowWaitNs)) atomicOr(&g_flow_error, kErrFlowTimeout);
         uint4 v[kItemChunksPerThread];
+        const unsigned char* buf = flow_smem + st * kFlowStageBytes;
+        const bool full = (it.c1 - it.c0 == kItemChunks) && M.dense_x && M.dense_o;
+        if (full) {
 #pragma unroll
-        for (int j = 0; j < kItemChunksPerThread; ++j) {
-            const uint32_t c = it.c0 + (uint32_t)j * kFlowThreads + tid;
-            v[j] = make_uint4(0u, 0u, 0u, 0u);
-            if (c < it.c1) {
-                int64_t off;
-                if (M.dense_x) {
-                    off = (int64_t)c * 16;
-                } else {
-                    const uint32_t r = fdiv(c, M.cpr);
-                    off = (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 16;
+            for (int j = 0; j < kItemChunksPerThread; ++j)
+                v[j] = *reinterpret_cast<const uint4*>(buf + ((uint32_t)j * kFlowThreads + tid) * 16u);
+        } else {
+            const char* xb = M.x + (int64_t)it.b * M.x_bs;
+#pragma unroll
+            for (int j = 0; j < kItemChunksPerThread; ++j) {
+                const uint32_t lc = (uint32_t)j * kFlowThreads + tid;   // chunk within the item
+                const uint32_t c = it.c0 + lc;
+                v[j] = make_uint4(0u, 0u, 0u, 0u);
+                if (c < it.c1) {
+                    if (M.dense_x) {
+                        v[j] = *reinterpret_cast<const uint4*>(buf + lc * 16u);
+                    } else {
+                        const uint32_t r = fdiv(c, M.cpr);
+                        v[j] = ld_hint_v4(xb + (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 16,
+                                          it.is_e ? stream : keep);
+                    }
                 }
-                v[j] = ld_hint_v4(xb + off, pol);
             }
         }
 
@@ -497,17 +595,18 @@ __global__ void __launch_bounds__(kFlowThreads, 4) nvfp4_flow_kernel(const __gri
             for (int j = 0; j < kItemChunksPerThread; ++j) m = max(m, amax_bits8(v[j]));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if ((tid & 31u) == 0u) red[p][tid >> 5] = m;
+            if ((tid & 31u) == 0u) red[k & 1u][tid >> 5] = m;
+            if (tid == 0) items[(k + 2u) % 3u] = flow_item(a, pa, s_pend);
+            __syncthreads();   // stage st is free; red and the new item are published
             if (tid == 0) {
-                items[p ^ 1u] = flow_item(a, pa, pending);
-                pending = next_q;
-            }
-            __syncthreads();
-            if (tid == 0) {
-                for (int w = 1; w < kFlowThreads / 32; ++w) m = max(m, red[p][w]);
+                const FlowItem& nx = items[(k + 2u) % 3u];
+                if (nx.valid)
+                    flow_stage(a, nx, stage0 + st * kFlowStageBytes, smem_addr(&bars[st]), nx.is_e ? stream : keep);
+                for (int w = 1; w < kFlowThreads / 32; ++w) m = max(m, red[k & 1u][w]);
                 if (m != 0u) atomicMax(a.amax_bits + it.inst, m << 16);
                 __threadfence();
                 atomicAdd(a.done + it.inst, 1u);
+                s_pend = next_q;
             }
             continue;
         }
@@ -515,8 +614,7 @@ __global__ void __launch_bounds__(kFlowThreads, 4) nvfp4_flow_kernel(const __gri
         // ---- encode item: wait (bounded) for the instance's amax
         const FlowGroup& G = a.g[it.g];
         if (tid == 0) {
-            items[p ^ 1u] = flow_item(a, pa, pending);
-            pending = next_q;
+            items[(k + 2u) % 3u] = flow_item(a, pa, s_pend);
             if (ld_acquire_gpu(a.done + it.inst) < G.items) {
                 const uint64_t t0 = globaltimer_ns();
                 while (ld_acquire_gpu(a.done + it.inst) < G.items) {
@@ -527,50 +625,34 @@ __global__ void __launch_bounds__(kFlowThreads, 4) nvfp4_flow_kernel(const __gri
                     __nanosleep(200);
                 }
             }
-            s_amax[p] = ld_relaxed_gpu(a.amax_bits + it.inst);
+            s_amax[k & 1u] = ld_relaxed_gpu(a.amax_bits + it.inst);
         }
-        __syncthreads();
+        __syncthreads();   // stage st is free; the amax and the new item are published
+        if (tid == 0) {
+            const FlowItem& nx = items[(k + 2u) % 3u];
+            if (nx.valid)
+                flow_stage(a, nx, stage0 + st * kFlowStageBytes, smem_addr(&bars[st]), nx.is_e ? stream : keep);
+        }
         if (it.inst != cached) {   // CTA-uniform
-            gs = __fdiv_rn(__uint_as_float(s_amax[p]), 2688.0f);
+            gs = __fdiv_rn(__uint_as_float(s_amax[k & 1u]), 2688.0f);
             six_gs = __fmul_rn(6.0f, gs);
             r6 = __frcp_rn(six_gs);
             fast6 = div_fast_ok(six_gs);
+            // every non-zero block scale gives dec(sb) * gs in [2^-9 gs, 448 gs]
+            all_fast = fast6 && __fmul_rn(0x1p-9f, gs) >= 0x1p-64f && __fmul_rn(448.0f, gs) <= 0x1p126f;
             fill_scale_table(tab, gs);
             __syncthreads();
             cached = it.inst;
         }
         if (tid == 0 && it.k == 0u) {
             if (G.gs_out) G.gs_out[it.b] = gs;
-            if (G.amax_out) G.amax_out[it.b] = __uint_as_float(s_amax[p]);
+            if (G.amax_out) G.amax_out[it.b] = __uint_as_float(s_amax[k & 1u]);
         }
-        char* ob = M.out + (int64_t)it.b * M.o_bs;
-        uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.chunks >> 1);
-#pragma unroll
-        for (int j = 0; j < kItemChunksPerThread; ++j) {
-            const uint32_t c = it.c0 + (uint32_t)j * kFlowThreads + tid;
-            uint32_t m = amax_bits8(v[j]);
-            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));   // lanes 2i, 2i+1: one block
-            const float amax_b = __uint_as_float(m << 16);
-            const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
-            const uint32_t sb = e4m3x2(ratio, 0.0f) & 0xffu;
-            const float4 e = tab.e[sb];
-            const uint32_t codes = codes_half(v[j], e.x, e.y);
-            if (c < it.c1) {
-                int64_t oo;
-                if (M.dense_o) {
-                    oo = (int64_t)c * (kFake ? 16 : 4);
-                } else {
-                    const uint32_t r = fdiv(c, M.cpr);
-                    oo = (int64_t)r * M.o_rs + (int64_t)(c - r * M.cpr.d) * (kFake ? 16 : 4);
-                }
-                if (kFake) {
-                    st_hint_v4(ob + oo, dequant_half(codes, e.z, gs), stream);
-                } else {
-                    st_hint_u32(ob + oo, codes, stream);
-                    if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)sb;
-                }
-            }
-        }
+        if (all_fast && full)
+            flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
+        else
+            flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
+        if (tid == 0) s_pend = next_q;
     }
 }
 
@@ -719,12 +801,23 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
         a.counter = words + 2 * a.n_inst;
         cudaError_t e = cudaMemsetAsync(words, 0, (size_t)(2 * a.n_inst + 1) * 4, s);
         if (e != cudaSuccess) return e;
+        const int dev = current_device();
+        const size_t smem = (size_t)kFlowStages * kFlowStageBytes;
+        static int configured[64] = {0};
+        if (dev >= 0 && dev < 64 && !configured[dev]) {
+            e = cudaFuncSetAttribute(nvfp4_flow_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(nvfp4_flow_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+            if (e != cudaSuccess) return e;
+            configured[dev] = 1;
+        }
         const int grid = (int)std::max<int64_t>(
-            1, std::min<int64_t>((int64_t)sm_count(current_device()) * 4, 2 * (int64_t)a.total_items));
+            1, std::min<int64_t>((int64_t)sm_count(dev) * 3, 2 * (int64_t)a.total_items));
         if (fake)
-            nvfp4_flow_kernel<true><<<grid, kFlowThreads, 0, s>>>(a);
+            nvfp4_flow_kernel<true><<<grid, kFlowThreads, smem, s>>>(a);
         else
-            nvfp4_flow_kernel<false><<<grid, kFlowThreads, 0, s>>>(a);
+            nvfp4_flow_kernel<false><<<grid, kFlowThreads, smem, s>>>(a);
         e = cudaGetLastError();
         reset();
         return e;
