@@ -298,10 +298,10 @@ __global__ void __launch_bounds__(kThreads) nvfp4_dequant_kernel(const __grid_co
 // groups, every batch index of a group being one "instance" with its own
 // amax.  The work is a queue of items of kItemChunks chunks of one member's
 // batch slab: amax items A(i, k) and encode items E(i, k) of instance i.  The
-// queue order is
-//     A(0) A(1) E(0) A(2) E(1) ... A(I-1) E(I-2) E(I-1)
-// so while the encode items of instance i run (ALU-heavy, reading data that
-// is still in L2), the amax items of instance i+1 keep HBM busy.  CTAs take
+// encode items of instance i follow its amax items after a lead of L amax
+// items of instance i+1 (the order is set out at flow_decode), so that they
+// re-read the instance while it is still in L2, and a CTA that takes one
+// seldom waits: the lead covers the amax items still in flight.  CTAs take
 // items from a global atomic counter.  An encode item waits (bounded) until
 // all amax items of its instance are done; those items all sit earlier in
 // the queue, were taken by running CTAs that never wait on later items, and
@@ -314,6 +314,10 @@ constexpr uint32_t kItemChunks = 2048;                        // 16384 elements
 constexpr int kItemChunksPerThread = kItemChunks / kFlowThreads;   // 8
 constexpr int kFlowMaxInst = 512;                             // instances per launch
 constexpr uint64_t kFlowWaitNs = 2000000000ull;               // 2 s
+constexpr uint32_t kFlowLeadPerCta = 4;                       // L = kFlowLeadPerCta * grid
+constexpr int kFlowStages = 2;
+constexpr int kFlowCtasPerSm = 3;
+constexpr uint32_t kFlowStageBytes = kItemChunks * 16u;   // 32 KB
 constexpr uint32_t kErrFlowTimeout = 2u;
 
 struct FlowMember {
@@ -343,9 +347,20 @@ struct FlowArgs {
     int n_groups;
     uint32_t n_inst;
     uint32_t total_items;         // items per pass (A items = E items)
+    uint32_t lead;                // amax items of the next instance between A(i) and E(i)
     uint32_t* amax_bits;          // [n_inst]  (workspace, zeroed before launch)
     uint32_t* done;               // [n_inst]  completed amax items
     uint32_t* counter;            // [1]       queue head
+};
+
+// The launch description in shared memory, so that the per-item decode and
+// the member fields cost shared-memory loads only.
+struct FlowTables {
+    FlowMember m[kMaxLaunchTensors];
+    FlowGroup g[kMaxLaunchTensors];
+    uint32_t pa[kFlowMaxInst + 1];   // items before instance i; pa[I] = total
+    uint32_t se[kFlowMaxInst];       // queue position of the first encode item of instance i
+    uint8_t ig[kFlowMaxInst];        // group of instance i
 };
 
 __device__ uint32_t g_flow_error = 0u;
@@ -368,58 +383,73 @@ __device__ __forceinline__ int flow_group_of(const FlowArgs& a, uint32_t inst) {
     return g;
 }
 
+// The queue order.  pa[i] = items before instance i (pa[I] = total), n_i =
+// pa[i+1] - pa[i].  The amax items of instance j >= 1 are split into a head
+// H(j) of lead(j) = min(n_j, L) items and the tail T(j); the queue is
+//     A(0) H(1) E(0) T(1) H(2) E(1) T(2) ... H(I-1) E(I-2) T(I-1) E(I-1)
+// so E(i) starts at se(i) = pa[i+1] + pa[i] + lead(i+1), at least L items
+// after the last amax item of instance i.
+__device__ __forceinline__ uint32_t flow_lead(const uint32_t* pa, uint32_t I, uint32_t L, uint32_t j) {
+    return j < I ? min(pa[j + 1] - pa[j], L) : 0u;
+}
+
 // Queue position q -> (encode?, instance, item within the instance's pass).
-// pa[i] = items before instance i (pa[I] = total).  Segment starts:
-// A(0) at 0, A(j) at pa[j] + pa[j-1]; E(j) at pa[min(j+2, I)] + pa[j].
-__device__ __forceinline__ void flow_decode(const uint32_t* pa, uint32_t I, uint32_t q, bool& is_e,
+__device__ __forceinline__ void flow_decode(const FlowTables& t, uint32_t I, uint32_t L, uint32_t q, bool& is_e,
                                             uint32_t& inst, uint32_t& k) {
+    is_e = false;
+    if (q < t.se[0]) {
+        inst = q < t.pa[1] ? 0u : 1u;
+        k = q - t.pa[inst];
+        return;
+    }
     uint32_t lo = 0, hi = I - 1;
     while (lo < hi) {
         const uint32_t mid = (lo + hi + 1) >> 1;
-        if (pa[mid] + pa[mid - 1] <= q) lo = mid; else hi = mid - 1;
+        if (t.se[mid] <= q) lo = mid; else hi = mid - 1;
     }
-    const uint32_t ja = lo;
-    const uint32_t sa = ja ? pa[ja] + pa[ja - 1] : 0u;
-    is_e = false;
-    inst = ja;
-    k = q - sa;
-    if (pa[min(2u, I)] + pa[0] > q) return;         // before E(0)
-    lo = 0;
-    hi = I - 1;
-    while (lo < hi) {
-        const uint32_t mid = (lo + hi + 1) >> 1;
-        if (pa[min(mid + 2u, I)] + pa[mid] <= q) lo = mid; else hi = mid - 1;
-    }
-    const uint32_t se = pa[min(lo + 2u, I)] + pa[lo];
-    if (se > sa) {
+    const uint32_t s = t.se[lo], n = t.pa[lo + 1] - t.pa[lo];
+    if (q < s + n) {
         is_e = true;
         inst = lo;
-        k = q - se;
+        k = q - s;
+        return;
+    }
+    // T(lo + 1), then H(lo + 2)
+    const uint32_t r = q - s - n, j = lo + 1;
+    const uint32_t lj = flow_lead(t.pa, I, L, j);
+    const uint32_t tail = t.pa[j + 1] - t.pa[j] - lj;
+    if (r < tail) {
+        inst = j;
+        k = lj + r;
+    } else {
+        inst = j + 1;
+        k = r - tail;
     }
 }
 
-// A decoded queue item.  Thread 0 decodes items two ahead of the CTA and
-// publishes them in a three-slot ring in shared memory.
+// A decoded queue item.  Thread 0 decodes items kFlowStages ahead of the CTA
+// and publishes them in a ring of kFlowStages + 1 slots in shared memory.
 struct FlowItem {
     uint32_t valid, is_e, inst, k;   // k: item within its instance's pass (encode: reversed)
     int g, m;                        // group, member
     uint32_t b, c0, c1;              // batch index in the group; chunk range of the member slab
 };
 
-__device__ __forceinline__ FlowItem flow_item(const FlowArgs& a, const uint32_t* pa, uint32_t q) {
+__device__ __forceinline__ FlowItem flow_item(const FlowTables& t, uint32_t I, uint32_t total, uint32_t L,
+                                              uint32_t q) {
     FlowItem it{};
-    it.valid = q < 2u * a.total_items;
+    it.valid = q < 2u * total;
     if (!it.valid) return it;
     bool is_e;
     uint32_t inst, k;
-    flow_decode(pa, a.n_inst, q, is_e, inst, k);
-    const int g = flow_group_of(a, inst);
-    const FlowGroup& G = a.g[g];
+    flow_decode(t, I, L, q, is_e, inst, k);
+    const int g = t.ig[inst];
+    const FlowGroup& G = t.g[g];
     if (is_e) k = G.items - 1u - k;                    // encode walks the instance backwards
     int mi = G.m_begin;
-    for (int t = 1; t < G.m_count; ++t)
-        if (k >= a.m[G.m_begin + t].item_off) mi = G.m_begin + t;
-    const FlowMember& M = a.m[mi];
+    for (int u = 1; u < G.m_count; ++u)
+        if (k >= t.m[G.m_begin + u].item_off) mi = G.m_begin + u;
+    const FlowMember& M = t.m[mi];
     it.is_e = is_e;
     it.inst = inst;
     it.k = k;
@@ -435,9 +465,8 @@ __device__ __forceinline__ FlowItem flow_item(const FlowArgs& a, const uint32_t*
 // copy of the item's contiguous bytes when the member slab is dense,
 // otherwise a plain arrival (the item is then read straight from global
 // memory), so that every stage completes one barrier phase per item.
-__device__ __forceinline__ void flow_stage(const FlowArgs& a, const FlowItem& it, uint32_t dst, uint32_t bar,
+__device__ __forceinline__ void flow_stage(const FlowMember& M, const FlowItem& it, uint32_t dst, uint32_t bar,
                                            uint64_t pol) {
-    const FlowMember& M = a.m[it.m];
     if (M.dense_x) {
         const uint32_t bytes = (it.c1 - it.c0) * 16u;
         mbar_arrive_expect_tx(bar, bytes);
@@ -446,9 +475,6 @@ __device__ __forceinline__ void flow_stage(const FlowArgs& a, const FlowItem& it
         mbar_arrive(bar);
     }
 }
-
-constexpr int kFlowStages = 2;
-constexpr uint32_t kFlowStageBytes = kItemChunks * 16u;   // 32 KB
 
 // Encodes the chunks of one item held in registers.  kFast: every block
 // divisor of the instance lies in the reciprocal path's range (checked per
@@ -503,47 +529,56 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
 }
 
 template <bool kFake>
-__global__ void __launch_bounds__(kFlowThreads, 3) nvfp4_flow_kernel(const __grid_constant__ FlowArgs a) {
+__global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kernel(const __grid_constant__ FlowArgs a) {
     extern __shared__ __align__(128) unsigned char flow_smem[];
-    __shared__ uint32_t pa[kFlowMaxInst + 1];
+    __shared__ FlowTables t;
     __shared__ ScaleTable tab;
-    __shared__ FlowItem items[3];
+    __shared__ FlowItem items[kFlowStages + 1];   // item n in slot n % (kFlowStages + 1)
     __shared__ __align__(8) uint64_t bars[kFlowStages];
     __shared__ uint32_t s_amax[2];
     __shared__ uint32_t red[2][kFlowThreads / 32];
-    __shared__ uint32_t s_q[2];
-    // thread 0: queue position of the item two ahead of the next one; stored
-    // at the end of an item so the atomic's latency overlaps warp 0's work
+    __shared__ uint32_t s_q[kFlowStages];
+    // thread 0: queue position of the item kFlowStages after the next one;
+    // stored at the end of an item so the atomic's latency overlaps warp 0's
+    // work
     __shared__ volatile uint32_t s_pend;
     const uint32_t tid = threadIdx.x;
     const uint32_t stage0 = smem_addr(flow_smem);
+    const uint32_t I = a.n_inst, L = a.lead, total = a.total_items;
 
     // the amax pass keeps its data in L2 for the encode pass; the encode
     // pass and every store stream through
     const uint64_t keep = l2_policy_evict_last();
     const uint64_t stream = l2_policy_evict_first();
 
-    for (uint32_t i = tid; i <= a.n_inst; i += blockDim.x) {
-        uint32_t v = a.total_items;
-        if (i < a.n_inst) {
-            const FlowGroup& G = a.g[flow_group_of(a, i)];
+    for (uint32_t i = tid; i < (uint32_t)kMaxLaunchTensors; i += blockDim.x) {
+        t.m[i] = a.m[i];
+        t.g[i] = a.g[i];
+    }
+    for (uint32_t i = tid; i <= I; i += blockDim.x) {
+        uint32_t v = total;
+        if (i < I) {
+            const int g = flow_group_of(a, i);
+            const FlowGroup& G = a.g[g];
             v = G.item_begin + (i - G.inst_begin) * G.items;
+            t.ig[i] = (uint8_t)g;
         }
-        pa[i] = v;
+        t.pa[i] = v;
     }
     if (tid == 0) {
         for (int s = 0; s < kFlowStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
         fence_mbar_init();
-        s_q[0] = atomicAdd(a.counter, 1u);
-        s_q[1] = atomicAdd(a.counter, 1u);
+        for (int s = 0; s < kFlowStages; ++s) s_q[s] = atomicAdd(a.counter, 1u);
         s_pend = atomicAdd(a.counter, 1u);
     }
     __syncthreads();
+    for (uint32_t i = tid; i < I; i += blockDim.x) t.se[i] = t.pa[i + 1] + t.pa[i] + flow_lead(t.pa, I, L, i + 1);
+    __syncthreads();
     if (tid == 0) {
-        for (int s = 0; s < 2; ++s) {
-            items[s] = flow_item(a, pa, s_q[s]);
+        for (int s = 0; s < kFlowStages; ++s) {
+            items[s] = flow_item(t, I, total, L, s_q[s]);
             if (items[s].valid)
-                flow_stage(a, items[s], stage0 + s * kFlowStageBytes, smem_addr(&bars[s]),
+                flow_stage(t.m[items[s].m], items[s], stage0 + s * kFlowStageBytes, smem_addr(&bars[s]),
                            items[s].is_e ? stream : keep);
         }
     }
@@ -552,13 +587,20 @@ __global__ void __launch_bounds__(kFlowThreads, 3) nvfp4_flow_kernel(const __gri
     uint32_t cached = 0xffffffffu;
     float gs = 0.0f, six_gs = 0.0f, r6 = 0.0f;
     bool fast6 = false, all_fast = false;
+    // thread 0: the current run of consecutive amax items of one instance;
+    // its max and count are published when the run ends, before the CTA
+    // takes any encode item, so no CTA waits while it holds unpublished work
+    uint32_t run_max = 0u, run_count = 0u;
+    // thread 0: the last instance whose amax this CTA has seen final
+    uint32_t known_inst = 0xffffffffu, known_amax = 0u;
     for (uint32_t k = 0;; ++k) {
-        const uint32_t slot = k % 3u, st = k & 1u, par = (k >> 1) & 1u;
+        const uint32_t slot = k % (kFlowStages + 1u), st = k % kFlowStages, par = (k / kFlowStages) & 1u;
+        const uint32_t ahead = (k + kFlowStages) % (kFlowStages + 1u);   // slot of item k + kFlowStages
         const FlowItem it = items[slot];
         if (!it.valid) break;
         uint32_t next_q = 0u;
-        if (tid == 0) next_q = atomicAdd(a.counter, 1u);   // decoded two items later
-        const FlowMember& M = a.m[it.m];
+        if (tid == 0) next_q = atomicAdd(a.counter, 1u);   // decoded at the next item
+        const FlowMember& M = t.m[it.m];
 
         // ---- the item's data, into registers
         if (!mbar_wait_bounded(smem_addr(&bars[st]), par, kFlowWaitNs)) atomicOr(&g_flow_error, kErrFlowTimeout);
@@ -596,42 +638,55 @@ __global__ void __launch_bounds__(kFlowThreads, 3) nvfp4_flow_kernel(const __gri
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((tid & 31u) == 0u) red[k & 1u][tid >> 5] = m;
-            if (tid == 0) items[(k + 2u) % 3u] = flow_item(a, pa, s_pend);
+            if (tid == 0) items[ahead] = flow_item(t, I, total, L, s_pend);
             __syncthreads();   // stage st is free; red and the new item are published
             if (tid == 0) {
-                const FlowItem& nx = items[(k + 2u) % 3u];
+                const FlowItem& nx = items[ahead];
                 if (nx.valid)
-                    flow_stage(a, nx, stage0 + st * kFlowStageBytes, smem_addr(&bars[st]), nx.is_e ? stream : keep);
+                    flow_stage(t.m[nx.m], nx, stage0 + st * kFlowStageBytes, smem_addr(&bars[st]),
+                               nx.is_e ? stream : keep);
                 for (int w = 1; w < kFlowThreads / 32; ++w) m = max(m, red[k & 1u][w]);
-                if (m != 0u) atomicMax(a.amax_bits + it.inst, m << 16);
-                __threadfence();
-                atomicAdd(a.done + it.inst, 1u);
+                run_max = max(run_max, m);
+                ++run_count;
+                const FlowItem& nn = items[(k + 1u) % (kFlowStages + 1u)];   // decoded earlier
+                if (!nn.valid || nn.is_e || nn.inst != it.inst) {
+                    if (run_max != 0u) atomicMax(a.amax_bits + it.inst, run_max << 16);
+                    __threadfence();
+                    atomicAdd(a.done + it.inst, run_count);
+                    run_max = 0u;
+                    run_count = 0u;
+                }
                 s_pend = next_q;
             }
             continue;
         }
 
         // ---- encode item: wait (bounded) for the instance's amax
-        const FlowGroup& G = a.g[it.g];
+        const FlowGroup& G = t.g[it.g];
         if (tid == 0) {
-            items[(k + 2u) % 3u] = flow_item(a, pa, s_pend);
-            if (ld_acquire_gpu(a.done + it.inst) < G.items) {
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_acquire_gpu(a.done + it.inst) < G.items) {
-                    if (globaltimer_ns() - t0 > kFlowWaitNs) {
-                        atomicOr(&g_flow_error, kErrFlowTimeout);
-                        break;
+            items[ahead] = flow_item(t, I, total, L, s_pend);
+            if (it.inst != known_inst) {
+                if (ld_acquire_gpu(a.done + it.inst) < G.items) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_gpu(a.done + it.inst) < G.items) {
+                        if (globaltimer_ns() - t0 > kFlowWaitNs) {
+                            atomicOr(&g_flow_error, kErrFlowTimeout);
+                            break;
+                        }
+                        __nanosleep(100);
                     }
-                    __nanosleep(200);
                 }
+                known_amax = ld_relaxed_gpu(a.amax_bits + it.inst);
+                known_inst = it.inst;
             }
-            s_amax[k & 1u] = ld_relaxed_gpu(a.amax_bits + it.inst);
+            s_amax[k & 1u] = known_amax;
         }
         __syncthreads();   // stage st is free; the amax and the new item are published
         if (tid == 0) {
-            const FlowItem& nx = items[(k + 2u) % 3u];
+            const FlowItem& nx = items[ahead];
             if (nx.valid)
-                flow_stage(a, nx, stage0 + st * kFlowStageBytes, smem_addr(&bars[st]), nx.is_e ? stream : keep);
+                flow_stage(t.m[nx.m], nx, stage0 + st * kFlowStageBytes, smem_addr(&bars[st]),
+                           nx.is_e ? stream : keep);
         }
         if (it.inst != cached) {   // CTA-uniform
             gs = __fdiv_rn(__uint_as_float(s_amax[k & 1u]), 2688.0f);
@@ -813,7 +868,8 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
             configured[dev] = 1;
         }
         const int grid = (int)std::max<int64_t>(
-            1, std::min<int64_t>((int64_t)sm_count(dev) * 3, 2 * (int64_t)a.total_items));
+            1, std::min<int64_t>((int64_t)sm_count(dev) * kFlowCtasPerSm, 2 * (int64_t)a.total_items));
+        a.lead = kFlowLeadPerCta * (uint32_t)grid;
         if (fake)
             nvfp4_flow_kernel<true><<<grid, kFlowThreads, smem, s>>>(a);
         else
