@@ -370,6 +370,11 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// Adds v with release semantics at GPU scope: the thread's earlier writes
+// (the amax atomicMax) are visible to whoever reads the sum with acquire.
+__device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -537,11 +542,11 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
     __shared__ __align__(8) uint64_t bars[kFlowStages];
     __shared__ uint32_t s_amax[2];
     __shared__ uint32_t red[2][kFlowThreads / 32];
-    __shared__ uint32_t s_q[kFlowStages];
-    // thread 0: queue position of the item kFlowStages after the next one;
-    // stored at the end of an item so the atomic's latency overlaps warp 0's
-    // work
-    __shared__ volatile uint32_t s_pend;
+    __shared__ uint32_t s_q[kFlowStages + 1];
+    // Thread 0 waits for amax values, starts the stage copies and publishes
+    // amax runs; thread kQueueThread (another warp) takes queue positions and
+    // decodes items, so the two chains overlap within an item.
+    constexpr uint32_t kQueueThread = 32;
     const uint32_t tid = threadIdx.x;
     const uint32_t stage0 = smem_addr(flow_smem);
     const uint32_t I = a.n_inst, L = a.lead, total = a.total_items;
@@ -568,8 +573,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
     if (tid == 0) {
         for (int s = 0; s < kFlowStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
         fence_mbar_init();
-        for (int s = 0; s < kFlowStages; ++s) s_q[s] = atomicAdd(a.counter, 1u);
-        s_pend = atomicAdd(a.counter, 1u);
+        for (int s = 0; s <= kFlowStages; ++s) s_q[s] = atomicAdd(a.counter, 1u);
     }
     __syncthreads();
     for (uint32_t i = tid; i < I; i += blockDim.x) t.se[i] = t.pa[i + 1] + t.pa[i] + flow_lead(t.pa, I, L, i + 1);
@@ -583,6 +587,8 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         }
     }
     __syncthreads();
+    // thread kQueueThread: queue position of the item kFlowStages ahead
+    uint32_t pend = s_q[kFlowStages];
 
     uint32_t cached = 0xffffffffu;
     float gs = 0.0f, six_gs = 0.0f, r6 = 0.0f;
@@ -599,7 +605,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         const FlowItem it = items[slot];
         if (!it.valid) break;
         uint32_t next_q = 0u;
-        if (tid == 0) next_q = atomicAdd(a.counter, 1u);   // decoded at the next item
+        if (tid == kQueueThread) next_q = atomicAdd(a.counter, 1u);   // decoded at the next item
         const FlowMember& M = t.m[it.m];
 
         // ---- the item's data, into registers
@@ -638,7 +644,10 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((tid & 31u) == 0u) red[k & 1u][tid >> 5] = m;
-            if (tid == 0) items[ahead] = flow_item(t, I, total, L, s_pend);
+            if (tid == kQueueThread) {
+                items[ahead] = flow_item(t, I, total, L, pend);
+                pend = next_q;
+            }
             __syncthreads();   // stage st is free; red and the new item are published
             if (tid == 0) {
                 const FlowItem& nx = items[ahead];
@@ -651,20 +660,21 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
                 const FlowItem& nn = items[(k + 1u) % (kFlowStages + 1u)];   // decoded earlier
                 if (!nn.valid || nn.is_e || nn.inst != it.inst) {
                     if (run_max != 0u) atomicMax(a.amax_bits + it.inst, run_max << 16);
-                    __threadfence();
-                    atomicAdd(a.done + it.inst, run_count);
+                    red_add_release_gpu(a.done + it.inst, run_count);   // ordered after the max
                     run_max = 0u;
                     run_count = 0u;
                 }
-                s_pend = next_q;
             }
             continue;
         }
 
         // ---- encode item: wait (bounded) for the instance's amax
         const FlowGroup& G = t.g[it.g];
+        if (tid == kQueueThread) {
+            items[ahead] = flow_item(t, I, total, L, pend);
+            pend = next_q;
+        }
         if (tid == 0) {
-            items[ahead] = flow_item(t, I, total, L, s_pend);
             if (it.inst != known_inst) {
                 if (ld_acquire_gpu(a.done + it.inst) < G.items) {
                     const uint64_t t0 = globaltimer_ns();
@@ -707,7 +717,6 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
             flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
         else
             flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
-        if (tid == 0) s_pend = next_q;
     }
 }
 
