@@ -54,6 +54,53 @@ KERNELS_PER_CALL = {"fp8_block_quant": 1, "fp8_block_dequant": 1, "mxfp8_quant":
                     "nvfp4_quant": 1, "nvfp4_dequant": 1, "nvfp4_fake_quant": 1}
 OPS = list(BYTES_PER_ELEM)
 
+# ncu DRAM traffic of one launch (one layer) for the kernels with a committed
+# summary under profiles/: the summary records the bytes and the sha256 of
+# the sources the capture ran on; once a source has changed the figure is
+# stale and `traffic` is reported as null.
+CSRC = "precision_weight_quantization_b200/csrc/"
+PROFILES = {
+    "nvfp4_fake_quant": ("profiles/nvfp4_flow_fake_quant_qwen3_4b_layer.md", "nvfp4.cu"),
+    "nvfp4_quant": ("profiles/nvfp4_flow_quant_qwen3_4b_layer.md", "nvfp4.cu"),
+    "fp8_block_quant": ("profiles/fp8_block_quant_qwen3_4b_layer.md", "fp8_block.cu"),
+    "fp8_block_dequant": ("profiles/fp8_block_dequant_qwen3_4b_layer.md", "fp8_block.cu"),
+    "mxfp8_quant": ("profiles/mxfp8_quant_qwen3_4b_layer.md", "mxfp8.cu"),
+    "mxfp8_dequant": ("profiles/mxfp8_dequant_qwen3_4b_layer.md", "mxfp8.cu"),
+    "nvfp4_dequant": ("profiles/nvfp4_dequant_qwen3_4b_layer.md", "nvfp4.cu"),
+}
+
+
+def source_sha256(kernel_file):
+    import hashlib
+    h = hashlib.sha256()
+    for f in (kernel_file, "pwq_device.cuh"):
+        with open(os.path.join(ROOT, CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(op):
+    """(bytes per launch, note) from the op's committed ncu summary."""
+    if op not in PROFILES:
+        return None, "no committed ncu summary for this kernel"
+    md, src = PROFILES[op]
+    try:
+        text = open(os.path.join(ROOT, md)).read()
+    except OSError:
+        return None, "summary %s missing" % md
+    import re
+    vals = {}
+    for key, pat in (("traffic_bytes_per_launch", r"^traffic_bytes_per_launch:\s*(\d+)"),
+                     ("source_sha256", r"^source_sha256:\s*`?([0-9a-f]{64})")):
+        m = re.search(pat, text, re.M)
+        if m:
+            vals[key] = m.group(1)
+    if "traffic_bytes_per_launch" not in vals or "source_sha256" not in vals:
+        return None, "summary %s records no traffic" % md
+    if vals["source_sha256"] != source_sha256(src):
+        return None, "kernel source changed since the capture in %s" % md
+    return int(vals["traffic_bytes_per_launch"]), "ncu dram read+write of one launch, %s" % md
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -132,6 +179,17 @@ class Clocks:
 
 
 # ------------------------------------------------------------------ workload
+
+def bench_config(args, grouped, world):
+    return {"workload": WORKLOAD, "layers": args.layers, "elements_per_rank": layer_elems() * args.layers,
+            "tensors": "q 4096x2560, k/v 1024x2560, o 2560x4096, gate/up 9728x2560, down 2560x9728",
+            "path": "fp8_block q+dq, mxfp8 q+dq, nvfp4 q (qkv, gate/up siblings)+dq, "
+                    "nvfp4 fake-quant (siblings)",
+            "l2": "inputs larger than L2 (7.3 GB per rank), no flush",
+            "launch": ("one grouped call per op per layer" if grouped else "one call per tensor") +
+                      "; one CUDA graph per op kind, replayed back to back",
+            "parallelism": "dp%d (independent sweeps)" % world}
+
 
 def make_layers(n_layers, device, rank):
     import workloads as W
@@ -389,22 +447,19 @@ def main():
                       "bytes_per_elem": round(BYTES_PER_ELEM[op], 5)}
     dom = max(OPS, key=lambda o: per_op_ms[o])
     dom_gbs = per_op[dom]["alg_gbs"]
+    traffic, traffic_note = recorded_traffic(dom) if grouped else (None, "per-tensor launches")
     roofline = {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(dom_gbs / hbm_peak, 4), "traffic": None, "peak_kind": peak_kind,
-                "note": "achieved = algorithmic bytes of all %d calls / their total device time per step "
-                        "(launch gaps included)" % ncalls[dom]}
+                "frac": round(dom_gbs / hbm_peak, 4), "traffic": traffic, "peak_kind": peak_kind,
+                "alg_bytes_per_launch": int(round(layer_elems() * BYTES_PER_ELEM[dom])),
+                "avg_launch_us": round(per_op_ms[dom] * 1e3 / ncalls[dom], 2),
+                "note": "achieved = algorithmic bytes of one launch (one layer) / the average launch "
+                        "duration (CUDA events around the graph of all %d launches of the step); traffic: %s"
+                        % (ncalls[dom], traffic_note)}
 
     line = {"metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "layers": args.layers, "elements_per_rank": elems_per_step,
-                       "tensors": "q 4096x2560, k/v 1024x2560, o 2560x4096, gate/up 9728x2560, down 2560x9728",
-                       "path": "fp8_block q+dq, mxfp8 q+dq, nvfp4 q (qkv, gate/up siblings)+dq, "
-                               "nvfp4 fake-quant (siblings)",
-                       "l2": "inputs larger than L2 (7.3 GB per rank), no flush",
-                       "launch": ("one grouped call per op per layer" if grouped else "one call per tensor") +
-                                 "; one CUDA graph per op kind, replayed back to back",
-                       "parallelism": "dp%d (independent sweeps)" % world},
+            "config": bench_config(args, grouped, world),
             "per_op": per_op, "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary() if rank == 0 else None}
 
@@ -446,20 +501,24 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
     def one_layer():
         for n in dx:
             dx[n].copy_(host_in[n], non_blocking=True)
-        res = {}
-        for n, x in dx.items():
-            q, s = P.fp8_block_quant(x)
-            P.fp8_block_dequant(q, s)
-            mq, me = P.mxfp8_quant(x)
-            P.mxfp8_dequant(mq, me)
-            res[n] = [q, s, mq, me]
-        for g in W.QWEN3_4B_GROUPS:
-            xs = [dx[n] for n in g]
-            pk, sb, gs = P.nvfp4_quant(xs)
+        names = list(dx)
+        xs = [dx[n] for n in names]
+        q, s = P.fp8_block_quant_grouped(xs)
+        P.fp8_block_dequant_grouped(q, s)
+        mq, me = P.mxfp8_quant_grouped(xs)
+        P.mxfp8_dequant_grouped(mq, me)
+        groups = [[dx[n] for n in g] for g in W.QWEN3_4B_GROUPS]
+        pk, sb, gs = P.nvfp4_quant_grouped(groups)
+        res = {n: [q[i], s[i], mq[i], me[i]] for i, n in enumerate(names)}
+        fpk, fsb, fgs = [], [], []
+        for gi, g in enumerate(W.QWEN3_4B_GROUPS):
             for k, n in enumerate(g):
-                P.nvfp4_dequant(pk[k], sb[k], gs)
-                res[n] += [pk[k], sb[k]]
-            P.nvfp4_fake_quant(xs)
+                fpk.append(pk[gi][k])
+                fsb.append(sb[gi][k])
+                fgs.append(gs[gi])
+                res[n] += [pk[gi][k], sb[gi][k]]
+        P.nvfp4_dequant_grouped(fpk, fsb, fgs)
+        P.nvfp4_fake_quant_grouped(groups)
         for n, ts in res.items():
             for h, d in zip(host_out[n], ts):
                 h.copy_(d.view(h.dtype) if d.dtype != h.dtype and d.element_size() == h.element_size() else d,
@@ -488,8 +547,9 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
     return {"value": elems_per_step * world / (ms / 1e3), "unit": "elem/s",
             "h2d_bytes_per_step": in_bytes * args.layers, "d2h_bytes_per_step": out_bytes * args.layers,
             "ms_per_step": ms, "steps": steps,
-            "note": "public Python API, one layer at a time from pinned host memory (the same host "
-                    "buffer feeds every layer), codes+scales of the three formats read back"}
+            "note": "public Python API (one grouped call per op per layer), one layer at a time from "
+                    "pinned host memory (the same host buffer feeds every layer), codes+scales of the "
+                    "three formats read back"}
 
 
 def main_reference(args, rank, world, torch, dist):
@@ -515,8 +575,8 @@ def main_reference(args, rank, world, torch, dist):
     line = {"metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "layers": args.layers,
-                       "sample_per_step": "256 rows of q/k/v of layer 0 (%d elements)" % n},
+            "config": dict(bench_config(args, not args.per_tensor, world),
+                           sample_per_step="256 rows of q/k/v of layer 0 (%d elements)" % n),
             "cpu_baseline": {"value": value, "unit": "elem/s", "cores": 1, "kind": "oracle",
                              "sample": "256-row slices of q/k/v (one sibling group) through every op, "
                                        "single-threaded scalar C oracle"},

@@ -1,0 +1,61 @@
+"""bench.py pieces that need no GPU: the reference arm's JSON line and the
+staleness rule of the recorded ncu traffic."""
+import hashlib
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_reference_arm_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["metric"] == bench.METRIC and line["unit"] == "elem/s" and line["higher_is_better"] is True
+    assert line["config"]["workload"] == bench.WORKLOAD
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def _fake_tree(tmp_path, kernel_src=b"kernel v1", traffic=123456789):
+    csrc = tmp_path / bench.CSRC
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_bytes(kernel_src)
+    (csrc / "pwq_device.cuh").write_bytes(b"helpers")
+    sha = hashlib.sha256(b"kernel v1" + b"helpers").hexdigest()
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "k.md").write_text(
+        "# k\n\n| metric | value |\n\ntraffic_bytes_per_launch: %d\nsource_sha256: `%s` (note)\n" % (traffic, sha))
+
+
+def test_recorded_traffic_fresh_and_stale(tmp_path, monkeypatch):
+    _fake_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "PROFILES", {"op": ("profiles/k.md", "k.cu")})
+    t, note = bench.recorded_traffic("op")
+    assert t == 123456789, note
+    (tmp_path / bench.CSRC / "k.cu").write_bytes(b"kernel v2")
+    t, note = bench.recorded_traffic("op")
+    assert t is None and "changed" in note
+    assert bench.recorded_traffic("other")[0] is None
+
+
+def test_every_profile_summary_parses():
+    # each committed summary names its traffic and the source hash it was taken on
+    for op, (md, src) in bench.PROFILES.items():
+        text = open(os.path.join(ROOT, md)).read()
+        assert "traffic_bytes_per_launch:" in text and "source_sha256:" in text, md
+        assert os.path.exists(os.path.join(ROOT, bench.CSRC, src)), src
