@@ -184,7 +184,7 @@ pwq_status mxfp8_dequant(const pwq_tensor* q, const uint8_t* scale, const pwq_te
  */
 
 /* Bytes of workspace an NVFP4 quantise / fake-quantise call over these
- * siblings needs: 4 * (2 * min(B, 2048) + 1), rounded up to 256.  x points
+ * siblings needs: 4 * (2 * min(B, 512) + 1), rounded up to 256.  x points
  * to n_siblings descriptors; returns 0 on bad input. */
 size_t nvfp4_workspace_size(int n_siblings, const pwq_tensor* x);
 

@@ -2,9 +2,9 @@
 single-pass NVFP4 path, against the CPU oracle, bit for bit.
 
 Lists mix ragged, batched and strided tensors; lists longer than one launch
-(16 tensors) and NVFP4 calls with more than 2048 group instances exercise the
-host-side splitting; members larger than one work item (16384 elements)
-exercise the item queue.
+(16 tensors) and NVFP4 calls with more than 512 group instances (one launch's
+worth) exercise the host-side splitting; members larger than one work item
+(16384 elements) exercise the item queue.
 """
 import numpy as np
 import pytest
