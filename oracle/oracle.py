@@ -243,3 +243,45 @@ def unpack_e2m1(packed):
     out[..., 0::2] = packed & 0xF
     out[..., 1::2] = packed >> 4
     return out
+
+
+# ---------------------------------------------------------------- FP8 block -> rollout formats
+#
+# "低精度训练与 Rollout", "FP8 训练 + FP8 Rollout" / "实现说明" item 3: on a
+# weight update the FP8 training weights are dequantised to BF16 and the BF16
+# weights are quantised into the rollout format.  The re-quantisation is
+# defined as exactly that composition; the functions below are the plain
+# composition of the pinned per-format functions above, with no shortcut.
+
+def fp8_block_requant(q, s):
+    """FP8 block codes + tile scales -> the FP8 block codes and scales of the
+    dequantised BF16 tensor: fp8_block_quant(fp8_block_dequant(q, s))."""
+    return fp8_block_quant(fp8_block_dequant(q, s))
+
+
+def fp8_block_requant_mxfp8(q, s):
+    """mxfp8_quant(fp8_block_dequant(q, s)); N % 32 == 0."""
+    return mxfp8_quant(fp8_block_dequant(q, s))
+
+
+def fp8_block_requant_nvfp4(qs, ss):
+    """A sibling group given as FP8 block members (codes [M][N] or
+    [B][M][N], tile scales): dequantise every member, then NVFP4-quantise
+    the group with the amax of the dequantised members, per batch index.
+    Returns (A [B], [(packed, sb)] per member, gs [B])."""
+    ys = [fp8_block_dequant(q, s) for q, s in zip(qs, ss)]
+    batched = ys[0].ndim == 3
+    y3 = [y if batched else y[None] for y in ys]
+    B = y3[0].shape[0]
+    A = np.array([nvfp4_group_amax([y[b] for y in y3]) for b in range(B)], np.float32)
+    gs = np.array([nvfp4_global_scale(a) for a in A], np.float32)
+    out = []
+    for y in y3:
+        pk, sb = [], []
+        for b in range(B):
+            p, s_, _ = nvfp4_quant(y[b], A[b])
+            pk.append(p)
+            sb.append(s_)
+        pk, sb = np.stack(pk), np.stack(sb)
+        out.append((pk if batched else pk[0], sb if batched else sb[0]))
+    return A, out, gs
