@@ -307,6 +307,53 @@ pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, in
                                     const float* amax_in, float* amax_out, pwq_stream_t stream);
 
 /* ===================================================================== */
+/* FP8 block-wise weights into a rollout format                           */
+/* ===================================================================== */
+
+/* "低精度训练与 Rollout", "FP8 训练 + FP8 Rollout" / "实现说明" item 3: on a
+ * weight update the FP8 training weights are dequantised to BF16 and the
+ * BF16 weights quantised into the rollout format.  These calls compute
+ * exactly that composition in one pass, without the BF16 tensor in memory:
+ * the input is FP8 block-wise (E4M3 codes q [B][M][N], FP32 tile scales
+ * s [B][ceil(M/128)][ceil(N/128)], as fp8_block_quant writes them), the
+ * values are y = bf16(fl(dec(q) * s)) as fp8_block_dequant computes them,
+ * and the outputs are bit for bit those of the named quantiser applied to
+ * y.  Code tensors: 8-byte aligned base and row stride (bytes = elements).
+ * Same error codes as the quantisers; no call allocates. */
+
+/* fp8_block_requant: FP8 block-wise -> FP8 block-wise with fresh tile
+ * scales, fp8_block_quant(fp8_block_dequant(q, s)).  q_out may be q exactly
+ * and scale_out may be scale_in (in place); other overlaps are
+ * PWQ_ERR_OVERLAP.  Any N. */
+pwq_status fp8_block_requant(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out,
+                             float* scale_out, pwq_stream_t stream);
+
+/* fp8_block_requant_mxfp8: FP8 block-wise -> MXFP8,
+ * mxfp8_quant(fp8_block_dequant(q, s)): codes into q_out (same shape; may
+ * be q_in exactly), UE8M0 bytes into scale_ue8m0 [B][M][N/32].  N % 32 == 0
+ * (a 1x32 block then never leaves its 128-wide tile). */
+pwq_status fp8_block_requant_mxfp8(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out,
+                                   uint8_t* scale_ue8m0, pwq_stream_t stream);
+
+/* Bytes of workspace fp8_block_requant_nvfp4 needs: 4 * B rounded up to 256
+ * (one amax word per group); 0 on bad input. */
+size_t fp8_block_requant_nvfp4_workspace_size(int n_siblings, const pwq_tensor* q_in);
+
+/* fp8_block_requant_nvfp4: a sibling group of FP8 block-wise members ->
+ * NVFP4, nvfp4_quant(fp8_block_dequant(q_i, s_i) for every member i): the
+ * group amax is taken over the dequantised members (per batch index), then
+ * every member is encoded with it.  q_in: n_siblings code tensors (N % 16
+ * == 0, same batch), scale_in: their tile scales; outputs as nvfp4_quant
+ * (q_packed, sb [B][M][N/16] per member, global_scale [B]).  amax_in
+ * (device, [B], nullable) replaces the reduction, e.g. after an all-reduce
+ * of a sharded group; otherwise workspace of
+ * fp8_block_requant_nvfp4_workspace_size() bytes is required. */
+pwq_status fp8_block_requant_nvfp4(const pwq_tensor* q_in, const float* const* scale_in, int n_siblings,
+                                   const pwq_tensor* q_packed, uint8_t* const* sb, float* global_scale,
+                                   const float* amax_in, void* workspace, size_t workspace_bytes,
+                                   pwq_stream_t stream);
+
+/* ===================================================================== */
 /* Diagnostics                                                            */
 /* ===================================================================== */
 

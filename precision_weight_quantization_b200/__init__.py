@@ -26,7 +26,7 @@ __all__ = [
     "nvfp4_workspace_size", "NVFP4FakeQuantSTE", "nvfp4_fake_quant_ste", "build_info",
     "device_error", "PwqError", "LIB_PATH", "fp8_block_quant_grouped", "fp8_block_dequant_grouped",
     "mxfp8_quant_grouped", "mxfp8_dequant_grouped", "nvfp4_dequant_grouped", "nvfp4_quant_grouped",
-    "nvfp4_fake_quant_grouped",
+    "nvfp4_fake_quant_grouped", "fp8_block_requant", "fp8_block_requant_mxfp8", "fp8_block_requant_nvfp4",
 ]
 
 _CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
@@ -390,6 +390,88 @@ def nvfp4_fake_quant_grouped(groups: Sequence[Sequence[torch.Tensor]], out=None,
 
 
 # ---------------------------------------------------------------- diagnostics
+
+# ---------------------------------------------------------------- FP8 block-wise -> rollout formats
+
+def _fp8_input(q, scale, name="q"):
+    _check_dtype(q, _CODE_DTYPES, name)
+    if not scale.is_contiguous() or scale.dtype != torch.float32:
+        raise ValueError("scale must be a contiguous float32 tensor")
+
+
+def fp8_block_requant(q: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor] = None,
+                      scale_out: Optional[torch.Tensor] = None, inplace: bool = False):
+    """FP8 block-wise codes + tile scales -> the FP8 block-wise codes and
+    scales of their dequantised BF16 values, in one pass (no BF16 tensor):
+    fp8_block_quant(fp8_block_dequant(q, scale)).  inplace=True overwrites
+    q and scale."""
+    _fp8_input(q, scale)
+    if out is None:
+        out = q if inplace else torch.empty(q.shape, dtype=torch.float8_e4m3fn, device=q.device)
+    if scale_out is None:
+        scale_out = scale if inplace else torch.empty_like(scale)
+    _check_dtype(out, _CODE_DTYPES, "out")
+    dq, do = _desc(q, "q"), _desc(out, "out")
+    check(lib.fp8_block_requant(ctypes.byref(dq), scale.data_ptr(), ctypes.byref(do), scale_out.data_ptr(),
+                                _stream(q)), "fp8_block_requant")
+    return out, scale_out
+
+
+def fp8_block_requant_mxfp8(q: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor] = None,
+                            scale_out: Optional[torch.Tensor] = None, inplace: bool = False):
+    """FP8 block-wise -> MXFP8 in one pass: mxfp8_quant(fp8_block_dequant(q,
+    scale)).  Returns (codes, UE8M0 bytes [.., M, N/32]); inplace=True
+    writes the codes over q."""
+    _fp8_input(q, scale)
+    if out is None:
+        out = q if inplace else torch.empty(q.shape, dtype=torch.float8_e4m3fn, device=q.device)
+    if scale_out is None:
+        scale_out = torch.empty(q.shape[:-1] + (q.shape[-1] // 32,), dtype=torch.uint8, device=q.device)
+    _check_dtype(out, _CODE_DTYPES, "out")
+    dq, do = _desc(q, "q"), _desc(out, "out")
+    check(lib.fp8_block_requant_mxfp8(ctypes.byref(dq), scale.data_ptr(), ctypes.byref(do),
+                                      scale_out.data_ptr(), _stream(q)), "fp8_block_requant_mxfp8")
+    return out, scale_out
+
+
+def fp8_block_requant_nvfp4(qs, scales, amax: Optional[torch.Tensor] = None, out=None, sb=None,
+                            global_scale: Optional[torch.Tensor] = None):
+    """A sibling group of FP8 block-wise members -> NVFP4 in one pass (amax
+    over the dequantised members, then encode): nvfp4_quant of the
+    dequantised group.  Returns (packed codes list, block scales list,
+    global scales [B]) like nvfp4_quant; ``amax`` replaces the reduction."""
+    single = isinstance(qs, torch.Tensor)
+    qs = [qs] if single else list(qs)
+    scales = [scales] if isinstance(scales, torch.Tensor) else list(scales)
+    if not 1 <= len(qs) <= PWQ_MAX_SIBLINGS or len(scales) != len(qs):
+        raise ValueError("1..%d members, one scale tensor each" % PWQ_MAX_SIBLINGS)
+    for i, (q, s_) in enumerate(zip(qs, scales)):
+        _fp8_input(q, s_, "q[%d]" % i)
+    dev = qs[0].device
+    B = _batch(qs[0])
+    if out is None:
+        out = [torch.empty(q.shape[:-1] + (q.shape[-1] // 2,), dtype=torch.uint8, device=dev) for q in qs]
+    if sb is None:
+        sb = [torch.empty(q.shape[:-1] + (q.shape[-1] // 16,), dtype=torch.float8_e4m3fn, device=dev) for q in qs]
+    if global_scale is None:
+        global_scale = torch.empty(B, dtype=torch.float32, device=dev)
+    aq = _desc_array(qs, "q")
+    ao = _desc_array(out, "out", packed=True)
+    sp = (ctypes.c_void_p * len(qs))(*[t.data_ptr() for t in scales])
+    sbp = (ctypes.c_void_p * len(qs))(*[t.data_ptr() for t in sb])
+    ws = None
+    if amax is None:
+        n = int(lib.fp8_block_requant_nvfp4_workspace_size(len(qs), aq))
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+    check(lib.fp8_block_requant_nvfp4(aq, sp, len(qs), ao, sbp, global_scale.data_ptr(),
+                                      amax.data_ptr() if amax is not None else None,
+                                      ws.data_ptr() if ws is not None else None,
+                                      ws.numel() if ws is not None else 0, _stream(qs[0])),
+          "fp8_block_requant_nvfp4")
+    if single:
+        return out[0], sb[0], global_scale
+    return out, sb, global_scale
+
 
 def build_info() -> str:
     return lib.pwq_build_info().decode()

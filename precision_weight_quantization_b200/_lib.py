@@ -60,6 +60,10 @@ _SIG = {
     "nvfp4_workspace_size_grouped": (ctypes.c_size_t, [ctypes.c_int, _IP, _T]),
     "nvfp4_quant_grouped": (_S, [ctypes.c_int, _IP, _T, _T, _PP, _PP, _P, ctypes.c_size_t, _P]),
     "nvfp4_fake_quant_grouped": (_S, [ctypes.c_int, _IP, _T, _T, _PP, _P, ctypes.c_size_t, _P]),
+    "fp8_block_requant": (_S, [_T, _P, _T, _P, _P]),
+    "fp8_block_requant_mxfp8": (_S, [_T, _P, _T, _P, _P]),
+    "fp8_block_requant_nvfp4_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _T]),
+    "fp8_block_requant_nvfp4": (_S, [_T, _PP, ctypes.c_int, _T, _PP, _P, _P, _P, ctypes.c_size_t, _P]),
     "pwq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "pwq_last_error_detail": (ctypes.c_char_p, []),
     "pwq_build_info": (ctypes.c_char_p, []),
@@ -71,8 +75,8 @@ _SIG = {
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libpwq.so is not built (%s); run `python -m "
-                          "precision_weight_quantization_b200.build`" % LIB_PATH)
+        raise ImportError("libpwq.so is not built (%s); run `python "
+                          "precision_weight_quantization_b200/build.py`" % LIB_PATH)
     L = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIG.items():
         f = getattr(L, name)

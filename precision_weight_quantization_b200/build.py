@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpwq.so")
-SOURCES = ["pwq_api.cu", "fp8_block.cu", "mxfp8.cu", "nvfp4.cu", "selftest.cu"]
+SOURCES = ["pwq_api.cu", "fp8_block.cu", "mxfp8.cu", "nvfp4.cu", "requant.cu", "selftest.cu"]
 HEADERS = ["pwq_device.cuh", "pwq_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -61,7 +61,7 @@ def build(force=False, verbose=False):
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
     if force or jobs or _stale(LIB, objs):
         tmp = LIB + ".tmp%d" % os.getpid()
-        cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
+        cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-Xlinker", "--no-undefined", "-o", tmp, *objs]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             sys.stderr.write(res.stdout + res.stderr)

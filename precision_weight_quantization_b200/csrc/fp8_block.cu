@@ -224,17 +224,6 @@ struct DequantArgs {
 constexpr int kDqRowsPerPass = kThreads / 16;        // 16
 constexpr int kDqChunks = kTile / kDqRowsPerPass;     // 8
 
-__device__ __forceinline__ uint4 dequant8(uint2 codes, float s) {
-    uint32_t w[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const uint32_t pair = ((h < 2 ? codes.x : codes.y) >> (16 * (h & 1))) & 0xffffu;
-        const float2 f = e4m3x2_decode(pair);
-        w[h] = pack_bf16x2(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const __grid_constant__ DequantArgs a) {
     const int ccol = (int)(threadIdx.x & 15u) * 8;
     const int row0 = (int)(threadIdx.x >> 4);
@@ -253,7 +242,7 @@ __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const __gri
                 v[j] = ld_stream_v2(qt + (int64_t)(row0 + kDqRowsPerPass * j) * T.q_rs + ccol);
 #pragma unroll
             for (int j = 0; j < kDqChunks; ++j)
-                st_v4(yt + (int64_t)(row0 + kDqRowsPerPass * j) * T.y_rs + ccol * 2, dequant8(v[j], sc));
+                st_v4(yt + (int64_t)(row0 + kDqRowsPerPass * j) * T.y_rs + ccol * 2, fp8_dequant8(v[j], sc));
         } else {
             for (int j = 0; j < kDqChunks; ++j) {
                 const int r = row0 + kDqRowsPerPass * j;

@@ -34,10 +34,15 @@ constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
 constexpr int kMaxSib = 8;
 
-// One sibling of a group set, addressed per batch slab.
+// One sibling of a group set, addressed per batch slab.  The source is BF16
+// or, for the FP8 block re-quantisation, E4M3 codes with one FP32 scale per
+// 128x128 tile (the kernels then see y = bf16(fl(dec(q) * s))).
 struct Sib {
-    const char* x;        // BF16
+    const char* x;        // BF16, or E4M3 codes
     int64_t x_bs, x_rs;   // bytes
+    const float* ts;      // FP8 source: tile scales [B][TM][TN]
+    int64_t ts_bs;        // FP8 source: TM * TN
+    uint32_t tn;          // FP8 source: TN
     char* out;            // packed codes (quant) or BF16 (fake); unused by amax
     int64_t o_bs, o_rs;   // bytes
     uint8_t* sb;          // dense [B][M][N/16] (quant only)
@@ -66,6 +71,17 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t m) {
     return m;
 }
 
+// Chunk c of an FP8-source slab: its 8 codes and its tile scale.
+__device__ __forceinline__ uint2 fp8_chunk(const Sib& S, const char* base, const float* tsb, uint32_t c,
+                                           float& s) {
+    const uint32_t r = fdiv(c, S.cpr);
+    const uint32_t k = c - r * S.cpr.d;
+    const int64_t off = S.dense_x ? (int64_t)c * 8 : (int64_t)r * S.x_rs + (int64_t)k * 8;
+    s = __ldg(tsb + (r >> 7) * S.tn + (k >> 4));
+    return ld_stream_v2(base + off);
+}
+
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads) nvfp4_amax_kernel(const AmaxArgs a) {
     const uint32_t b = blockIdx.y;
     const uint32_t stride = gridDim.x * blockDim.x;
@@ -74,25 +90,42 @@ __global__ void __launch_bounds__(kThreads) nvfp4_amax_kernel(const AmaxArgs a) 
     for (int i = 0; i < a.n; ++i) {
         const Sib& S = a.s[i];
         const char* base = S.x + (int64_t)b * S.x_bs;
-        for (uint32_t c0 = t0; c0 < S.chunks; c0 += stride * kUnroll) {
-            uint4 v[kUnroll];
+        if constexpr (kFp8) {
+            const float* tsb = S.ts + (int64_t)b * S.ts_bs;
+            for (uint32_t c0 = t0; c0 < S.chunks; c0 += stride * kUnroll) {
+                uint2 v[kUnroll];
+                float sc[kUnroll];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const uint32_t c = c0 + u * stride;
-                v[u] = make_uint4(0u, 0u, 0u, 0u);
-                if (c < S.chunks) {
-                    int64_t off;
-                    if (S.dense_x) {
-                        off = (int64_t)c * 16;
-                    } else {
-                        const uint32_t r = fdiv(c, S.cpr);
-                        off = (int64_t)r * S.x_rs + (int64_t)(c - r * S.cpr.d) * 16;
-                    }
-                    v[u] = ld_stream_v4(base + off);
+                for (int u = 0; u < kUnroll; ++u) {
+                    const uint32_t c = c0 + u * stride;
+                    v[u] = make_uint2(0u, 0u);
+                    sc[u] = 0.0f;
+                    if (c < S.chunks) v[u] = fp8_chunk(S, base, tsb, c, sc[u]);
                 }
-            }
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) m = max(m, amax_bits8(v[u]));
+                for (int u = 0; u < kUnroll; ++u) m = max(m, fp8_amax_bits16(e4m3_maxmag8(v[u]), sc[u]));
+            }
+        } else {
+            for (uint32_t c0 = t0; c0 < S.chunks; c0 += stride * kUnroll) {
+                uint4 v[kUnroll];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const uint32_t c = c0 + u * stride;
+                    v[u] = make_uint4(0u, 0u, 0u, 0u);
+                    if (c < S.chunks) {
+                        int64_t off;
+                        if (S.dense_x) {
+                            off = (int64_t)c * 16;
+                        } else {
+                            const uint32_t r = fdiv(c, S.cpr);
+                            off = (int64_t)r * S.x_rs + (int64_t)(c - r * S.cpr.d) * 16;
+                        }
+                        v[u] = ld_stream_v4(base + off);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) m = max(m, amax_bits8(v[u]));
+            }
         }
     }
     m = block_max_u32(m);
@@ -145,7 +178,7 @@ __device__ __forceinline__ uint4 dequant_half(uint32_t codes, float sbv, float g
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-template <bool kFake>
+template <bool kFake, bool kFp8>
 __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs a) {
     __shared__ ScaleTable tab;
     const uint32_t b = blockIdx.y;
@@ -167,6 +200,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
     for (int i = a.n - 1; i >= 0; --i) {
         const Sib& S = a.s[i];
         const char* xb = S.x + (int64_t)b * S.x_bs;
+        const float* tsb = kFp8 ? S.ts + (int64_t)b * S.ts_bs : nullptr;
         char* ob = S.out + (int64_t)b * S.o_bs;
         uint8_t* sbb = kFake ? nullptr : S.sb + (int64_t)b * (S.chunks >> 1);
         for (uint32_t base = gwarp * 32u * kUnroll; base < S.chunks; base += nwarps * 32u * kUnroll) {
@@ -178,7 +212,13 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
                 // lanes 2k and 2k+1 take the high and low halves of one block
                 cc[u] = S.chunks - 1u - j;
                 v[u] = make_uint4(0u, 0u, 0u, 0u);
-                if (j < S.chunks) {
+                if (kFp8) {
+                    if (j < S.chunks) {
+                        float sc;
+                        const uint2 codes = fp8_chunk(S, xb, tsb, cc[u], sc);
+                        v[u] = fp8_dequant8(codes, sc);
+                    }
+                } else if (j < S.chunks) {
                     int64_t off;
                     if (S.dense_x) {
                         off = (int64_t)cc[u] * 16;
@@ -725,9 +765,17 @@ bool dense_rows(const View& v, int64_t row_bytes) {
     return v.rstride == row_bytes;
 }
 
+// BF16 source (ts null) or E4M3 codes with tile scales ts [B][TM][TN].
+void set_source(Sib& S, const View& x, const float* ts) {
+    S.ts = ts;
+    S.tn = (uint32_t)((x.cols + 127) / 128);
+    S.ts_bs = (int64_t)((x.rows + 127) / 128) * S.tn;
+    S.dense_x = dense_rows(x, ts ? x.cols : x.cols * 2);
+}
+
 }  // namespace
 
-cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStream_t s) {
+cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStream_t s, const float* const* ts) {
     const int64_t B = x[0].batch;
     cudaError_t err = cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t) * B, s);
     if (err != cudaSuccess) return err;
@@ -742,7 +790,7 @@ cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStr
         S.x_rs = x[i].rstride;
         S.chunks = (uint32_t)(x[i].rows * (x[i].cols / 8));
         S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x[i].cols / 8));
-        S.dense_x = dense_rows(x[i], x[i].cols * 2);
+        set_source(S, x[i], ts ? ts[i] : nullptr);
         max_chunks = std::max<int64_t>(max_chunks, S.chunks);
     }
     const int64_t total_ctas = (max_chunks + int64_t(kThreads) * kUnroll - 1) / (int64_t(kThreads) * kUnroll);
@@ -750,13 +798,16 @@ cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStr
     const int64_t budget = (int64_t)sm_count(current_device()) * 4;
     int gx = (int)std::max<int64_t>(1, std::min<int64_t>(total_ctas, (budget + B - 1) / B));
     dim3 grid(gx, (unsigned)B);
-    nvfp4_amax_kernel<<<grid, kThreads, 0, s>>>(a);
+    if (ts)
+        nvfp4_amax_kernel<true><<<grid, kThreads, 0, s>>>(a);
+    else
+        nvfp4_amax_kernel<false><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* const* sb,
                                 bool fake, const uint32_t* amax_bits, const float* amax_in,
-                                float* gs_out, float* amax_out, cudaStream_t s) {
+                                float* gs_out, float* amax_out, cudaStream_t s, const float* const* ts) {
     const int64_t B = x[0].batch;
     EncodeArgs a{};
     a.n = n;
@@ -776,7 +827,7 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
         S.sb = fake ? nullptr : sb[i];
         S.chunks = (uint32_t)(x[i].rows * (x[i].cols / 8));
         S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x[i].cols / 8));
-        S.dense_x = dense_rows(x[i], x[i].cols * 2);
+        set_source(S, x[i], ts ? ts[i] : nullptr);
         S.dense_o = dense_rows(out[i], fake ? out[i].cols * 2 : out[i].cols / 2);
         max_chunks = std::max<int64_t>(max_chunks, S.chunks);
     }
@@ -785,10 +836,16 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
     const int64_t budget = (int64_t)sm_count(current_device()) * 8;
     int gx = (int)std::max<int64_t>(1, std::min<int64_t>(total_ctas, (budget + B - 1) / B));
     dim3 grid(gx, (unsigned)B);
-    if (fake)
-        nvfp4_encode_kernel<true><<<grid, kThreads, 0, s>>>(a);
-    else
-        nvfp4_encode_kernel<false><<<grid, kThreads, 0, s>>>(a);
+    if (ts) {
+        if (fake)
+            nvfp4_encode_kernel<true, true><<<grid, kThreads, 0, s>>>(a);
+        else
+            nvfp4_encode_kernel<false, true><<<grid, kThreads, 0, s>>>(a);
+    } else if (fake) {
+        nvfp4_encode_kernel<true, false><<<grid, kThreads, 0, s>>>(a);
+    } else {
+        nvfp4_encode_kernel<false, false><<<grid, kThreads, 0, s>>>(a);
+    }
     return cudaGetLastError();
 }
 

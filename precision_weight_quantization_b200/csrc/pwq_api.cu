@@ -599,6 +599,139 @@ pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, in
                                               amax_out, s));
 }
 
+// ------------------------------------------------------------------ FP8 block-wise -> rollout formats
+
+namespace {
+
+// Overlap rule of the re-quantisation calls: no output may touch an input or
+// another output, except the pairs listed in `allowed` (exact in-place use).
+pwq_status check_requant_overlaps(const std::vector<Extent>& ins, const std::vector<Extent>& outs,
+                                  const std::vector<std::pair<int, int>>& allowed) {
+    for (size_t i = 0; i < outs.size(); ++i) {
+        for (size_t j = 0; j < ins.size(); ++j) {
+            bool ok = false;
+            for (const auto& p : allowed) ok |= (p.first == (int)i && p.second == (int)j);
+            if (!ok && overlaps(outs[i], ins[j])) return fail(PWQ_ERR_OVERLAP, "output overlaps an input");
+        }
+        for (size_t j = i + 1; j < outs.size(); ++j)
+            if (overlaps(outs[i], outs[j])) return fail(PWQ_ERR_OVERLAP, "two outputs overlap");
+    }
+    return PWQ_OK;
+}
+
+size_t tile_scale_bytes(const pwq_tensor* t) {
+    return (size_t)(t->batch * ceil_div(t->rows, 128) * ceil_div(t->cols, 128)) * 4;
+}
+
+// The FP8 block-wise input (codes + tile scales) and a same-shaped code
+// output of the FP8 / MXFP8 re-quantisation.
+pwq_status check_requant_io(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out, View* vq,
+                            View* vo, Extent* eq, Extent* eo, Extent* esi) {
+    pwq_status st;
+    if ((st = check_tensor(q_in, Kind::kByte, vq, eq, "q_in")) != PWQ_OK) return st;
+    if (!q_out) return fail(PWQ_ERR_NULL, "q_out");
+    if (!same_shape(q_in, q_out)) return fail(PWQ_ERR_SHAPE, "q_out shape != q_in shape");
+    if ((st = check_tensor(q_out, Kind::kByte, vo, eo, "q_out")) != PWQ_OK) return st;
+    if (empty(q_in)) return PWQ_OK;
+    if (!scale_in) return fail(PWQ_ERR_NULL, "scale_in");
+    if ((uintptr_t)scale_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale_in");
+    *esi = extent_of(scale_in, tile_scale_bytes(q_in));
+    return PWQ_OK;
+}
+
+}  // namespace
+
+pwq_status fp8_block_requant(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out,
+                             float* scale_out, pwq_stream_t stream) {
+    View vq, vo;
+    Extent eq, eo, esi;
+    pwq_status st = check_requant_io(q_in, scale_in, q_out, &vq, &vo, &eq, &eo, &esi);
+    if (st != PWQ_OK || empty(q_in)) return st;
+    if (!scale_out) return fail(PWQ_ERR_NULL, "scale_out");
+    if ((uintptr_t)scale_out % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale_out");
+    const Extent eso = extent_of(scale_out, tile_scale_bytes(q_in));
+    std::vector<std::pair<int, int>> allowed;
+    if (exact_alias(q_in, q_out)) allowed.push_back({0, 0});
+    if (scale_out == scale_in) allowed.push_back({1, 1});
+    if ((st = check_requant_overlaps({eq, esi}, {eo, eso}, allowed)) != PWQ_OK) return st;
+    return from_cuda(pwq::launch_fp8_requant_fp8(vq, scale_in, vo, scale_out, (cudaStream_t)stream));
+}
+
+pwq_status fp8_block_requant_mxfp8(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out,
+                                   uint8_t* scale_ue8m0, pwq_stream_t stream) {
+    View vq, vo;
+    Extent eq, eo, esi;
+    pwq_status st = check_requant_io(q_in, scale_in, q_out, &vq, &vo, &eq, &eo, &esi);
+    if (st != PWQ_OK) return st;
+    if (q_in->cols % 32 != 0) return fail(PWQ_ERR_SHAPE, "cols % 32 != 0");
+    if (empty(q_in)) return PWQ_OK;
+    if (!scale_ue8m0) return fail(PWQ_ERR_NULL, "scale_ue8m0");
+    const Extent ee = extent_of(scale_ue8m0, (size_t)(q_in->batch * q_in->rows * (q_in->cols / 32)));
+    std::vector<std::pair<int, int>> allowed;
+    if (exact_alias(q_in, q_out)) allowed.push_back({0, 0});
+    if ((st = check_requant_overlaps({eq, esi}, {eo, ee}, allowed)) != PWQ_OK) return st;
+    return from_cuda(pwq::launch_fp8_requant_mxfp8(vq, scale_in, vo, scale_ue8m0, (cudaStream_t)stream));
+}
+
+size_t fp8_block_requant_nvfp4_workspace_size(int n_siblings, const pwq_tensor* q_in) {
+    if (!q_in || n_siblings < 1 || n_siblings > PWQ_MAX_SIBLINGS || q_in[0].batch < 0) return 0;
+    return (size_t)((std::max<int64_t>(1, q_in[0].batch) * 4 + 255) / 256 * 256);
+}
+
+pwq_status fp8_block_requant_nvfp4(const pwq_tensor* q_in, const float* const* scale_in, int n_siblings,
+                                   const pwq_tensor* q_packed, uint8_t* const* sb, float* global_scale,
+                                   const float* amax_in, void* workspace, size_t workspace_bytes,
+                                   pwq_stream_t stream) {
+    if (n_siblings < 1 || n_siblings > PWQ_MAX_SIBLINGS) return fail(PWQ_ERR_ARG, "n_siblings out of range");
+    if (!q_in || !q_packed) return fail(PWQ_ERR_NULL, "q_in / q_packed");
+    View vq[PWQ_MAX_SIBLINGS], vo[PWQ_MAX_SIBLINGS];
+    std::vector<Extent> ins, outs;
+    bool all_empty = true;
+    const int64_t B = q_in[0].batch;
+    pwq_status st;
+    for (int i = 0; i < n_siblings; ++i) {
+        Extent eq, eo;
+        if ((st = check_tensor(&q_in[i], Kind::kByte, &vq[i], &eq, "q_in[i]")) != PWQ_OK) return st;
+        if (q_in[i].batch != B) return fail(PWQ_ERR_ARG, "siblings differ in batch");
+        if (q_in[i].cols % 16 != 0) return fail(PWQ_ERR_SHAPE, "cols % 16 != 0");
+        if (!same_shape(&q_in[i], &q_packed[i])) return fail(PWQ_ERR_SHAPE, "q_packed shape != q_in shape");
+        if ((st = check_tensor(&q_packed[i], Kind::kPacked4, &vo[i], &eo, "q_packed[i]")) != PWQ_OK) return st;
+        if (empty(&q_in[i])) continue;
+        all_empty = false;
+        if (!scale_in || !scale_in[i]) return fail(PWQ_ERR_NULL, "scale_in[i]");
+        if ((uintptr_t)scale_in[i] % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale_in[i]");
+        if (!sb || !sb[i]) return fail(PWQ_ERR_NULL, "sb[i]");
+        ins.push_back(eq);
+        ins.push_back(extent_of(scale_in[i], tile_scale_bytes(&q_in[i])));
+        outs.push_back(eo);
+        outs.push_back(extent_of(sb[i], (size_t)(B * q_in[i].rows * (q_in[i].cols / 16))));
+    }
+    if (B > 65535) return fail(PWQ_ERR_SHAPE, "batch > 65535");
+    if (all_empty || B == 0) return PWQ_OK;
+    if (!global_scale) return fail(PWQ_ERR_NULL, "global_scale");
+    if ((uintptr_t)global_scale % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
+    outs.push_back(extent_of(global_scale, (size_t)B * 4));
+    if (amax_in) {
+        if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
+        ins.push_back(extent_of(amax_in, (size_t)B * 4));
+    } else {
+        const size_t need = fp8_block_requant_nvfp4_workspace_size(n_siblings, q_in);
+        if (!workspace || (uintptr_t)workspace % 4 != 0 || workspace_bytes < need)
+            return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
+        outs.push_back(extent_of(workspace, need));
+    }
+    if ((st = check_requant_overlaps(ins, outs, {})) != PWQ_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t* amax_bits = nullptr;
+    if (!amax_in) {
+        amax_bits = static_cast<uint32_t*>(workspace);
+        cudaError_t e = pwq::launch_nvfp4_amax(vq, n_siblings, amax_bits, s, scale_in);   // clears the words first
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return from_cuda(pwq::launch_nvfp4_encode(vq, n_siblings, vo, sb, false, amax_bits, amax_in, global_scale,
+                                              nullptr, s, scale_in));
+}
+
 // ------------------------------------------------------------------ self-tests
 
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream) {

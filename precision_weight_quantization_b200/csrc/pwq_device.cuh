@@ -71,6 +71,35 @@ __device__ __forceinline__ float2 e4m3x2_decode(uint32_t codes16) {
 // One E4M3 code -> exact binary32 value.
 __device__ __forceinline__ float e4m3_decode(uint32_t code) { return e4m3x2_decode(code & 0xffu).x; }
 
+// FP8 block-wise dequantisation of 8 codes (code 0 in bits 0..7 of c.x):
+// BF16 bits of y = bf16(fl(dec(q) * s)), element 0 in the low half of .x.
+__device__ __forceinline__ uint4 fp8_dequant8(uint2 c, float s) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const uint32_t pair = ((h < 2 ? c.x : c.y) >> (16 * (h & 1))) & 0xffffu;
+        const float2 f = e4m3x2_decode(pair);
+        w[h] = pack_bf16x2(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Largest magnitude byte (bits 0..6) among 8 E4M3 codes; positive E4M3
+// codes order like their values.
+__device__ __forceinline__ uint32_t e4m3_maxmag8(uint2 c) {
+    uint32_t m = __vmaxu4(c.x & 0x7f7f7f7fu, c.y & 0x7f7f7f7fu);
+    m = __vmaxu4(m, m >> 16);
+    m = __vmaxu4(m, m >> 8);
+    return m & 0xffu;
+}
+
+// BF16 magnitude bits of max |y| over FP8 codes of one scale s whose largest
+// magnitude byte is mc: rounding is monotone and symmetric in sign, so the
+// max of bf16(fl(dec(q) * s)) in magnitude is bf16(fl(dec(mc) * |s|)).
+__device__ __forceinline__ uint32_t fp8_amax_bits16(uint32_t mc, float s) {
+    return pack_bf16x2(__fmul_rn(e4m3_decode(mc), fabsf(s)), 0.0f) & 0xffffu;
+}
+
 // ---------------------------------------------------------------- E2M1
 
 // Two binary32 -> one byte of two E2M1 codes (lo element in bits 0..3).

@@ -59,13 +59,23 @@ size_t nvfp4_flow_workspace_bytes(int64_t instances);
 cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, void* workspace,
                               cudaStream_t s);
 
-// Two-launch NVFP4 path for one group set (used with a precomputed amax and
-// by the no-allocation entry point).  amax_bits: B words holding max |x| of
-// each group as binary32 bits.
-cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStream_t s);
+// Two-launch NVFP4 path for one group set (used with a precomputed amax, by
+// the no-allocation entry point and by the FP8 block re-quantisation).
+// amax_bits: B words holding max |x| of each group as binary32 bits.  With
+// ts non-null the members are E4M3 code views (FP8 block-wise, ts[i] the
+// member's tile scales [B][TM][TN]) and the source values are their
+// dequantised BF16 values.
+cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStream_t s,
+                              const float* const* ts = nullptr);
 cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* const* sb,
                                 bool fake, const uint32_t* amax_bits, const float* amax_in,
-                                float* gs_out, float* amax_out, cudaStream_t s);
+                                float* gs_out, float* amax_out, cudaStream_t s,
+                                const float* const* ts = nullptr);
+
+// FP8 block-wise codes + tile scales re-quantised (dequantise, quantise) into
+// FP8 block-wise (new scales) or MXFP8; q2 may be q, s2 may be s.
+cudaError_t launch_fp8_requant_fp8(const View& q, const float* s, const View& q2, float* s2, cudaStream_t st);
+cudaError_t launch_fp8_requant_mxfp8(const View& q, const float* s, const View& q2, uint8_t* e, cudaStream_t st);
 
 // Device address (on the current device) of the file-scope group-amax
 // scratch used by nvfp4_fake_quant_noalloc; kStaticScratchGroups words.

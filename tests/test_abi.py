@@ -12,8 +12,8 @@ HEADER = os.path.join(ROOT, "include", "pwq.h")
 
 
 def _lib():
-    from precision_weight_quantization_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._load_build_script().build()
     import precision_weight_quantization_b200._lib as L
     return L
 
@@ -147,3 +147,50 @@ def test_python_binding_names_match_the_abi():
     with pytest.raises(ValueError):
         import torch
         P.fp8_block_quant(torch.zeros(4, 4, dtype=torch.bfloat16))    # CPU tensor refused
+
+
+def test_requant_validation_without_gpu():
+    L = _lib()
+    lib = L.lib
+    by = ctypes.byref
+    base = 1 << 40
+    q = T(L, base, 1, 256, 512, 256 * 512, 512)
+    qo = T(L, base + (1 << 30), 1, 256, 512, 256 * 512, 512)
+    s = base + (2 << 30)
+    so = base + (3 << 30)
+    # nulls, alignment, shape
+    assert lib.fp8_block_requant(by(q), None, by(qo), so, None) == L.PWQ_ERR_NULL
+    assert lib.fp8_block_requant(by(q), s, by(qo), None, None) == L.PWQ_ERR_NULL
+    assert lib.fp8_block_requant(by(q), s + 2, by(qo), so, None) == L.PWQ_ERR_ALIGN
+    qa = T(L, base + 4, 1, 256, 512, 256 * 512, 512)                  # codes: 8-byte aligned base
+    assert lib.fp8_block_requant(by(qa), s, by(qo), so, None) == L.PWQ_ERR_ALIGN
+    q2 = T(L, base + (1 << 30), 1, 128, 512, 128 * 512, 512)
+    assert lib.fp8_block_requant(by(q), s, by(q2), so, None) == L.PWQ_ERR_SHAPE
+    # overlap: partial overlap of the output codes, new scales over the input codes
+    qp = T(L, base + 64, 1, 256, 512, 256 * 512, 512)
+    assert lib.fp8_block_requant(by(q), s, by(qp), so, None) == L.PWQ_ERR_OVERLAP
+    assert lib.fp8_block_requant(by(q), s, by(qo), base + 128, None) == L.PWQ_ERR_OVERLAP
+    # MXFP8 target: N % 32, scale bytes must not overlap
+    q48 = T(L, base, 1, 4, 48, 4 * 48, 48)
+    assert lib.fp8_block_requant_mxfp8(by(q48), s, by(q48), so, None) == L.PWQ_ERR_SHAPE
+    assert lib.fp8_block_requant_mxfp8(by(q), s, by(qo), base + 8, None) == L.PWQ_ERR_OVERLAP
+    # NVFP4 target
+    qs = (L.PwqTensor * 2)(q, T(L, base + (1 << 24), 1, 64, 512, 64 * 512, 512))
+    pk = (L.PwqTensor * 2)(T(L, base + (4 << 30), 1, 256, 512, 256 * 256, 256),
+                           T(L, base + (4 << 30) + (1 << 24), 1, 64, 512, 64 * 256, 256))
+    ss = (ctypes.c_void_p * 2)(s, s + 4096)
+    sb = (ctypes.c_void_p * 2)(base + (5 << 30), base + (5 << 30) + (1 << 24))
+    gs = base + (6 << 30)
+    ws = base + (7 << 30)
+    assert lib.fp8_block_requant_nvfp4_workspace_size(2, qs) == 256
+    assert lib.fp8_block_requant_nvfp4(qs, ss, 0, pk, sb, gs, None, ws, 256, None) == L.PWQ_ERR_ARG
+    assert lib.fp8_block_requant_nvfp4(qs, ss, 2, pk, sb, gs, None, None, 0, None) == L.PWQ_ERR_WORKSPACE
+    ss_null = (ctypes.c_void_p * 2)(s, None)
+    assert lib.fp8_block_requant_nvfp4(qs, ss_null, 2, pk, sb, gs, None, ws, 256, None) == L.PWQ_ERR_NULL
+    sbo = (ctypes.c_void_p * 2)(base + 256, base + (5 << 30) + (1 << 24))   # block scales over the codes
+    assert lib.fp8_block_requant_nvfp4(qs, ss, 2, pk, sbo, gs, None, ws, 256, None) == L.PWQ_ERR_OVERLAP
+    q24 = (L.PwqTensor * 1)(T(L, base, 1, 4, 24, 4 * 24, 24))
+    assert lib.fp8_block_requant_nvfp4(q24, ss, 1, q24, sb, gs, None, ws, 256, None) == L.PWQ_ERR_SHAPE
+    # empty input: a no-op that succeeds
+    qe = T(L, None, 1, 0, 512, 0, 512)
+    assert lib.fp8_block_requant(by(qe), None, by(qe), None, None) == L.PWQ_OK

@@ -35,8 +35,6 @@ def _rank(rank, world, port, out_dir):
     import torch.distributed as dist
     from oracle import oracle as O
     import workloads as W
-    from precision_weight_quantization_b200 import build
-    build.build()
     from precision_weight_quantization_b200.dist import allreduce_group_amax, row_shard
 
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
@@ -68,6 +66,9 @@ def _rank(rank, world, port, out_dir):
 
 
 def test_sharded_group_amax_two_ranks(tmp_path):
+    sys.path.insert(0, ROOT)
+    import __graft_entry__
+    __graft_entry__._load_build_script().build()   # once, before the ranks import the package
     ctx = mp.get_context("spawn")
     port = _port()
     procs = [ctx.Process(target=_rank, args=(r, 2, port, str(tmp_path))) for r in range(2)]

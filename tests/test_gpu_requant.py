@@ -1,0 +1,147 @@
+"""GPU parity of the FP8 block-wise -> {FP8 block-wise, MXFP8, NVFP4}
+re-quantisation against the oracle's dequantise-then-quantise, bit for bit.
+
+Inputs are FP8 block-wise codes and tile scales: the library's own
+quantisation of seeded BF16 tensors with the scales perturbed (so new scales
+differ from the old), and raw random codes with scales that include zero,
+BF16-subnormal and power-of-two values.  Ragged, batched, strided, in-place
+and sibling cases; a full Qwen3-4B gate_proj compared on sampled row blocks.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+import workloads as W
+
+from test_gpu_parity import DEV, f32bits, gpu, rand_bits, u8
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def P():
+    import precision_weight_quantization_b200 as P
+    assert torch.cuda.is_available()
+    return P
+
+
+def codes_and_scales(shape, seed, raw=False):
+    """(codes uint8 numpy, scales float32 numpy) of an FP8 block-wise tensor."""
+    rng = np.random.default_rng(seed)
+    B, M, N = (1,) + tuple(shape) if len(shape) == 2 else tuple(shape)
+    TM, TN = -(-M // 128), -(-N // 128)
+    if raw:
+        q = rng.integers(0, 0x7F, size=(B, M, N), dtype=np.uint8) | (rng.integers(0, 2, size=(B, M, N),
+                                                                                   dtype=np.uint8) << 7)
+        s = rng.uniform(1e-5, 1e-1, size=(B, TM, TN)).astype(np.float32)
+        flat = s.reshape(-1)
+        flat[0] = 0.0
+        if flat.size > 1:
+            flat[1] = np.float32(3e-40)          # subnormal binary32 scale
+        if flat.size > 2:
+            flat[2] = np.float32(2.0 ** -9)
+    else:
+        q, s = O.fp8_block_quant(rand_bits((B, M, N), seed))
+        s = (s * rng.uniform(0.5, 2.0, size=s.shape)).astype(np.float32)
+    if len(shape) == 2:
+        q, s = q[0], s[0]
+    return q, s
+
+
+def to_gpu_codes(q, pad=0):
+    if pad == 0:
+        return torch.from_numpy(np.ascontiguousarray(q)).to(DEV)
+    big = torch.zeros(q.shape[:-1] + (q.shape[-1] + pad,), dtype=torch.uint8, device=DEV)
+    big[..., :q.shape[-1]] = torch.from_numpy(q).to(DEV)
+    return big[..., :q.shape[-1]]
+
+
+FP8_SHAPES = [((130, 200), False, 0), ((3, 129, 136), True, 8), ((1, 8), True, 0), ((256, 512), False, 0),
+              ((2, 300, 1000), True, 24), ((128, 128), True, 0)]
+
+
+@pytest.mark.parametrize("shape,raw,pad", FP8_SHAPES)
+def test_fp8_to_fp8(P, shape, raw, pad):
+    q, s = codes_and_scales(shape, seed=hash(shape) % 1000, raw=raw)
+    oq, os_ = O.fp8_block_requant(q, s)
+    gq, gs = P.fp8_block_requant(to_gpu_codes(q, pad), torch.from_numpy(s).to(DEV))
+    assert np.array_equal(u8(gq), oq)
+    assert np.array_equal(f32bits(gs), os_.view(np.uint32))
+
+
+def test_fp8_to_fp8_in_place(P):
+    q, s = codes_and_scales((2, 260, 384), seed=5)
+    tq, ts = to_gpu_codes(q), torch.from_numpy(s).to(DEV)
+    P.fp8_block_requant(tq, ts, inplace=True)
+    oq, os_ = O.fp8_block_requant(q, s)
+    assert np.array_equal(u8(tq), oq) and np.array_equal(f32bits(ts), os_.view(np.uint32))
+
+
+MX_SHAPES = [((130, 256), False, 0), ((3, 129, 160), True, 16), ((1, 32), True, 0), ((2, 300, 1024), False, 32)]
+
+
+@pytest.mark.parametrize("shape,raw,pad", MX_SHAPES)
+def test_fp8_to_mxfp8(P, shape, raw, pad):
+    q, s = codes_and_scales(shape, seed=7 + len(shape), raw=raw)
+    oq, oe = O.fp8_block_requant_mxfp8(q, s)
+    gq, ge = P.fp8_block_requant_mxfp8(to_gpu_codes(q, pad), torch.from_numpy(s).to(DEV))
+    assert np.array_equal(u8(gq), oq) and np.array_equal(u8(ge), oe)
+    # in place over the codes
+    tq = to_gpu_codes(q, pad)
+    P.fp8_block_requant_mxfp8(tq, torch.from_numpy(s).to(DEV), inplace=True)
+    assert np.array_equal(u8(tq), oq)
+
+
+@pytest.mark.parametrize("shapes,raw", [([(96, 256), (32, 256), (32, 256)], False),
+                                        ([(3, 40, 160), (3, 24, 160)], True),
+                                        ([(130, 64)], True)])
+def test_fp8_to_nvfp4_siblings(P, shapes, raw):
+    members = [codes_and_scales(sh, seed=20 + i, raw=raw) for i, sh in enumerate(shapes)]
+    A, out, gs = O.fp8_block_requant_nvfp4([m[0] for m in members], [m[1] for m in members])
+    qs = [to_gpu_codes(m[0]) for m in members]
+    ss = [torch.from_numpy(m[1]).to(DEV) for m in members]
+    pk, sb, g = P.fp8_block_requant_nvfp4(qs, ss)
+    assert np.array_equal(f32bits(g), gs.view(np.uint32))
+    for i in range(len(shapes)):
+        assert np.array_equal(u8(pk[i]), out[i][0]), i
+        assert np.array_equal(u8(sb[i]), out[i][1]), i
+    # the same with the amax given (e.g. after an all-reduce)
+    pk2, sb2, g2 = P.fp8_block_requant_nvfp4(qs, ss, amax=torch.from_numpy(A).to(DEV))
+    assert torch.equal(g2, g)
+    for i in range(len(shapes)):
+        assert torch.equal(pk2[i], pk[i]) and torch.equal(sb2[i].view(torch.uint8), sb[i].view(torch.uint8))
+
+
+def test_fp8_to_nvfp4_equals_quant_of_dequant_on_gpu(P):
+    q, s = codes_and_scales((4, 200, 512), seed=31)
+    tq, ts = to_gpu_codes(q), torch.from_numpy(s).to(DEV)
+    y = P.fp8_block_dequant(tq, ts)
+    pk_ref, sb_ref, gs_ref = P.nvfp4_quant(y)
+    pk, sb, gs = P.fp8_block_requant_nvfp4(tq, ts)
+    assert torch.equal(gs, gs_ref) and torch.equal(pk, pk_ref)
+    assert torch.equal(sb.view(torch.uint8), sb_ref.view(torch.uint8))
+
+
+def test_full_size_gate_proj_sampled(P):
+    # Qwen3-4B gate_proj (9728 x 2560) quantised to FP8 block-wise on the GPU,
+    # then re-quantised; the oracle recomputes sampled 128-row blocks
+    x = W.qwen3_4b_layer(0, device=DEV)["gate_proj"]
+    q, s = P.fp8_block_quant(x)
+    s = s * 1.5
+    rq, rs = P.fp8_block_requant(q, s)
+    mq, me = P.fp8_block_requant_mxfp8(q, s)
+    pk, sb, gs = P.fp8_block_requant_nvfp4(q, s)
+    qn, sn = u8(q), s.cpu().numpy()
+    y = O.fp8_block_dequant(qn, sn)
+    A = np.float32(O.nvfp4_group_amax([y]))
+    assert f32bits(gs)[0] == np.float32(O.nvfp4_global_scale(A)).view(np.uint32)
+    rqn, rsn, mqn, men, pkn, sbn = u8(rq), f32bits(rs), u8(mq), u8(me), u8(pk), u8(sb)
+    for tm in [0, 1, 37, 75]:
+        r0, r1 = tm * 128, (tm + 1) * 128
+        oq, os_ = O.fp8_block_requant(qn[r0:r1], sn[tm:tm + 1])
+        assert np.array_equal(rqn[r0:r1], oq) and np.array_equal(rsn[tm:tm + 1], os_.view(np.uint32))
+        oq, oe = O.fp8_block_requant_mxfp8(qn[r0:r1], sn[tm:tm + 1])
+        assert np.array_equal(mqn[r0:r1], oq) and np.array_equal(men[r0:r1], oe)
+        opk, osb, _ = O.nvfp4_quant(y[r0:r1], A)
+        assert np.array_equal(pkn[r0:r1], opk) and np.array_equal(sbn[r0:r1], osb)
