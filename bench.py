@@ -19,6 +19,11 @@ API with the BF16 weights in pinned host memory, one layer at a time: H2D
 copy, every op, and a D2H read of the quantised artefacts (codes + scales of
 the three formats) inside the timed region.
 
+`next_rows` times the FP8 block-wise re-quantisation ops (FP8 block-wise
+codes + scales -> FP8 block-wise / MXFP8 / NVFP4 in one pass) on the step's
+FP8 outputs over the same sweep, each in its own graph after the timed
+steps; they are not part of `value`.
+
 `--impl reference` times the CPU oracle (single thread, as it stands) on a
 bounded sample of the same workload.
 """
@@ -111,6 +116,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=36)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip timing the FP8 block-wise re-quantisation ops (reported under next_rows)")
     ap.add_argument("--per-tensor", action="store_true",
                     help="one call per tensor / sibling group instead of one grouped call per layer")
     return ap.parse_args()
@@ -332,6 +339,85 @@ def capture(calls, torch):
     return g
 
 
+# ------------------------------------------------------------------ the FP8 block-wise re-quantisation row
+
+# FP8 block-wise codes + tile scales (the step's fp8_block_quant outputs)
+# straight into a rollout format; algorithmic bytes: one read of the codes
+# and scales, one write of each output
+NEXT_BYTES_PER_ELEM = {
+    "fp8_block_requant": 1 + 4 / 16384 + 1 + 4 / 16384,
+    "fp8_block_requant_mxfp8": 1 + 4 / 16384 + 1 + 1 / 32,
+    "fp8_block_requant_nvfp4": 1 + 4 / 16384 + 0.5 + 1 / 16,
+}
+
+
+def next_calls(op, layers, buf, P, torch):
+    """One call per tensor (one grouped call per layer for NVFP4, all four
+    sibling groups in one single-pass launch), reading the FP8 codes and
+    scales the step wrote; outputs shared by all layers."""
+    import workloads as W
+    lay0 = layers[0]
+    dev = lay0["q_proj"].device
+    out_q = {n: torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev) for n, x in lay0.items()}
+    calls = []
+    if op == "fp8_block_requant":
+        out_s = {n: torch.empty_like(buf.fp8[0][n][1]) for n in lay0}
+        for i in range(len(layers)):
+            for n in lay0:
+                q, sc = buf.fp8[i][n]
+                calls.append(lambda q=q, sc=sc, n=n: P.fp8_block_requant(q, sc, out=out_q[n], scale_out=out_s[n]))
+    elif op == "fp8_block_requant_mxfp8":
+        out_e = {n: torch.empty((x.shape[0], x.shape[1] // 32), dtype=torch.uint8, device=dev)
+                 for n, x in lay0.items()}
+        for i in range(len(layers)):
+            for n in lay0:
+                q, sc = buf.fp8[i][n]
+                calls.append(lambda q=q, sc=sc, n=n: P.fp8_block_requant_mxfp8(q, sc, out=out_q[n],
+                                                                               scale_out=out_e[n]))
+    else:
+        pk = {n: torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for n, x in lay0.items()}
+        sb = {n: torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev)
+              for n, x in lay0.items()}
+        G = W.QWEN3_4B_GROUPS
+        gsc = [torch.empty(1, dtype=torch.float32, device=dev) for _ in G]
+        for i in range(len(layers)):
+            qs = [[buf.fp8[i][n][0] for n in g] for g in G]
+            ss = [[buf.fp8[i][n][1] for n in g] for g in G]
+            calls.append(lambda qs=qs, ss=ss: P.fp8_block_requant_nvfp4_grouped(
+                qs, ss, out=[[pk[n] for n in g] for g in G], sb=[[sb[n] for n in g] for g in G],
+                global_scale=gsc))
+    return calls
+
+
+def time_next_rows(args, layers, buf, P, torch, hbm_peak, peak_kind):
+    """Device time of each re-quantisation op over the sweep (its own CUDA
+    graph, replayed after the step's timing; not part of `value`)."""
+    elems = layer_elems() * args.layers
+    stream = torch.cuda.current_stream()
+    out = {}
+    for op, bpe in NEXT_BYTES_PER_ELEM.items():
+        calls = next_calls(op, layers, buf, P, torch)
+        g = capture(calls, torch)
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.steps
+        gbs = elems * bpe / (ms / 1e3) / 1e9
+        out[op] = {"ms": round(ms, 4), "elem_per_s": elems / (ms / 1e3), "alg_gbs": round(gbs, 1),
+                   "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "calls": len(calls),
+                   "kernels_per_call": 1,
+                   "bytes_per_elem": round(bpe, 5)}
+        del g
+    return out
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 
 def cpu_sample_elems():
@@ -463,9 +549,11 @@ def main():
             "per_op": per_op, "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary() if rank == 0 else None}
 
+    del graphs
+    if not args.no_next:
+        line["next_rows"] = time_next_rows(args, layers, buf, P, torch, hbm_peak, peak_kind)
     if not args.no_e2e:
         line["e2e"] = e2e(args, layers, P, torch, dev, world, dist, elems_per_step)
-    del graphs
     if rank == 0 and not args.no_cpu_baseline:
         import workloads as W
         lay0 = {n: W.bits(x) for n, x in layers[0].items() if n in ("q_proj", "k_proj", "v_proj", "o_proj")}

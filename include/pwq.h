@@ -335,9 +335,12 @@ pwq_status fp8_block_requant(const pwq_tensor* q_in, const float* scale_in, cons
 pwq_status fp8_block_requant_mxfp8(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out,
                                    uint8_t* scale_ue8m0, pwq_stream_t stream);
 
-/* Bytes of workspace fp8_block_requant_nvfp4 needs: 4 * B rounded up to 256
- * (one amax word per group); 0 on bad input. */
+/* Bytes of workspace fp8_block_requant_nvfp4 / _grouped need: as
+ * nvfp4_workspace_size / nvfp4_workspace_size_grouped for the same shapes;
+ * 0 on bad input. */
 size_t fp8_block_requant_nvfp4_workspace_size(int n_siblings, const pwq_tensor* q_in);
+size_t fp8_block_requant_nvfp4_workspace_size_grouped(int n_groups, const int* group_sizes,
+                                                      const pwq_tensor* q_in);
 
 /* fp8_block_requant_nvfp4: a sibling group of FP8 block-wise members ->
  * NVFP4, nvfp4_quant(fp8_block_dequant(q_i, s_i) for every member i): the
@@ -352,6 +355,18 @@ pwq_status fp8_block_requant_nvfp4(const pwq_tensor* q_in, const float* const* s
                                    const pwq_tensor* q_packed, uint8_t* const* sb, float* global_scale,
                                    const float* amax_in, void* workspace, size_t workspace_bytes,
                                    pwq_stream_t stream);
+
+/* fp8_block_requant_nvfp4_grouped: several sibling groups in one call (e.g.
+ * a decoder layer's {q,k,v}, {o}, {gate,up}, {down}), laid out as in
+ * nvfp4_quant_grouped: group g has group_sizes[g] members, consecutive in
+ * q_in / scale_in / q_packed / sb, and writes global_scale[g] ([B_g]).
+ * Without amax_in the group amax is reduced on the device in the same
+ * single-pass launch that encodes (the codes are read once for the amax and
+ * once more, mostly from L2, for the encode pass). */
+pwq_status fp8_block_requant_nvfp4_grouped(int n_groups, const int* group_sizes, const pwq_tensor* q_in,
+                                           const float* const* scale_in, const pwq_tensor* q_packed,
+                                           uint8_t* const* sb, float* const* global_scale, void* workspace,
+                                           size_t workspace_bytes, pwq_stream_t stream);
 
 /* ===================================================================== */
 /* Diagnostics                                                            */

@@ -27,6 +27,7 @@ __all__ = [
     "device_error", "PwqError", "LIB_PATH", "fp8_block_quant_grouped", "fp8_block_dequant_grouped",
     "mxfp8_quant_grouped", "mxfp8_dequant_grouped", "nvfp4_dequant_grouped", "nvfp4_quant_grouped",
     "nvfp4_fake_quant_grouped", "fp8_block_requant", "fp8_block_requant_mxfp8", "fp8_block_requant_nvfp4",
+    "fp8_block_requant_nvfp4_grouped",
 ]
 
 _CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
@@ -470,6 +471,42 @@ def fp8_block_requant_nvfp4(qs, scales, amax: Optional[torch.Tensor] = None, out
           "fp8_block_requant_nvfp4")
     if single:
         return out[0], sb[0], global_scale
+    return out, sb, global_scale
+
+
+def fp8_block_requant_nvfp4_grouped(groups, scales, out=None, sb=None, global_scale=None):
+    """Several sibling groups of FP8 block-wise members (codes; `scales`
+    mirrors `groups` with their tile scales) -> NVFP4 in one single-pass
+    launch.  Returns (packed codes per group, block scales per group, global
+    scales per group)."""
+    groups = [list(g) for g in groups]
+    scales = [list(g) for g in scales]
+    if [len(g) for g in groups] != [len(g) for g in scales]:
+        raise ValueError("scales must mirror groups")
+    for gi, g in enumerate(groups):
+        if not 1 <= len(g) <= PWQ_MAX_SIBLINGS:
+            raise ValueError("1..%d members per group" % PWQ_MAX_SIBLINGS)
+        for i, (q, s_) in enumerate(zip(g, scales[gi])):
+            _fp8_input(q, s_, "groups[%d][%d]" % (gi, i))
+    flat = [q for g in groups for q in g]
+    sizes = (ctypes.c_int * len(groups))(*[len(g) for g in groups])
+    dev = flat[0].device
+    if out is None:
+        out = [[torch.empty(q.shape[:-1] + (q.shape[-1] // 2,), dtype=torch.uint8, device=dev) for q in g]
+               for g in groups]
+    if sb is None:
+        sb = [[torch.empty(q.shape[:-1] + (q.shape[-1] // 16,), dtype=torch.float8_e4m3fn, device=dev) for q in g]
+              for g in groups]
+    if global_scale is None:
+        global_scale = [torch.empty(_batch(g[0]), dtype=torch.float32, device=dev) for g in groups]
+    aq = _desc_array(flat, "q")
+    ws_bytes = int(lib.fp8_block_requant_nvfp4_workspace_size_grouped(len(groups), sizes, aq))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    check(lib.fp8_block_requant_nvfp4_grouped(len(groups), sizes, aq, _ptrs([t for g in scales for t in g]),
+                                              _desc_array([p_ for g in out for p_ in g], "out", packed=True),
+                                              _ptrs([t for g in sb for t in g]), _ptrs(global_scale),
+                                              ws.data_ptr(), ws.numel(), _stream(flat[0])),
+          "fp8_block_requant_nvfp4_grouped")
     return out, sb, global_scale
 
 

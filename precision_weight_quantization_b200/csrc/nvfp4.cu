@@ -370,6 +370,9 @@ struct FlowMember {
     FastDiv cpr;          // chunks per row
     int dense_x, dense_o;
     uint32_t item_off;    // first item of this member inside an instance
+    const float* ts;      // FP8 block-wise source: tile scales [B][TM][TN] at the first batch index
+    int64_t ts_bs;        // FP8 source: TM * TN
+    uint32_t tn;          // FP8 source: TN
 };
 
 struct FlowGroup {
@@ -513,9 +516,10 @@ __device__ __forceinline__ FlowItem flow_item(const FlowTables& t, uint32_t I, u
 __device__ __forceinline__ void flow_stage(const FlowMember& M, const FlowItem& it, uint32_t dst, uint32_t bar,
                                            uint64_t pol) {
     if (M.dense_x) {
-        const uint32_t bytes = (it.c1 - it.c0) * 16u;
+        const uint32_t cb = M.ts ? 8u : 16u;   // bytes per 8-element chunk: E4M3 codes or BF16
+        const uint32_t bytes = (it.c1 - it.c0) * cb;
         mbar_arrive_expect_tx(bar, bytes);
-        bulk_load(dst, M.x + (int64_t)it.b * M.x_bs + (int64_t)it.c0 * 16, bytes, bar, pol);
+        bulk_load(dst, M.x + (int64_t)it.b * M.x_bs + (int64_t)it.c0 * cb, bytes, bar, pol);
     } else {
         mbar_arrive(bar);
     }
@@ -573,7 +577,17 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
     }
 }
 
-template <bool kFake>
+// Chunk c of an FP8 block-wise member: the BF16 values of its 8 codes.
+__device__ __forceinline__ uint4 flow_fp8_chunk(const FlowMember& M, const FlowItem& it, uint2 codes, uint32_t c) {
+    const uint32_t r = fdiv(c, M.cpr);
+    const uint32_t k = c - r * M.cpr.d;
+    const float s = __ldg(M.ts + (int64_t)it.b * M.ts_bs + (r >> 7) * M.tn + (k >> 4));
+    return fp8_dequant8(codes, s);
+}
+
+// kFp8: the members are FP8 block-wise (E4M3 codes + tile scales) and the
+// values quantised are their dequantised BF16 values.
+template <bool kFake, bool kFp8>
 __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kernel(const __grid_constant__ FlowArgs a) {
     extern __shared__ __align__(128) unsigned char flow_smem[];
     __shared__ FlowTables t;
@@ -655,8 +669,13 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         const bool full = (it.c1 - it.c0 == kItemChunks) && M.dense_x && M.dense_o;
         if (full) {
 #pragma unroll
-            for (int j = 0; j < kItemChunksPerThread; ++j)
-                v[j] = *reinterpret_cast<const uint4*>(buf + ((uint32_t)j * kFlowThreads + tid) * 16u);
+            for (int j = 0; j < kItemChunksPerThread; ++j) {
+                const uint32_t lc = (uint32_t)j * kFlowThreads + tid;
+                if (kFp8)
+                    v[j] = flow_fp8_chunk(M, it, *reinterpret_cast<const uint2*>(buf + lc * 8u), it.c0 + lc);
+                else
+                    v[j] = *reinterpret_cast<const uint4*>(buf + lc * 16u);
+            }
         } else {
             const char* xb = M.x + (int64_t)it.b * M.x_bs;
 #pragma unroll
@@ -665,7 +684,16 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
                 const uint32_t c = it.c0 + lc;
                 v[j] = make_uint4(0u, 0u, 0u, 0u);
                 if (c < it.c1) {
-                    if (M.dense_x) {
+                    if (kFp8) {
+                        uint2 codes;
+                        if (M.dense_x) {
+                            codes = *reinterpret_cast<const uint2*>(buf + lc * 8u);
+                        } else {
+                            const uint32_t r = fdiv(c, M.cpr);
+                            codes = ld_stream_v2(xb + (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 8);
+                        }
+                        v[j] = flow_fp8_chunk(M, it, codes, c);
+                    } else if (M.dense_x) {
                         v[j] = *reinterpret_cast<const uint4*>(buf + lc * 16u);
                     } else {
                         const uint32_t r = fdiv(c, M.cpr);
@@ -905,6 +933,7 @@ size_t nvfp4_flow_workspace_bytes(int64_t instances) {
 }
 
 cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, void* workspace, cudaStream_t s) {
+    const bool fp8 = n_groups > 0 && groups[0].ts != nullptr;   // every group of a call has the same source
     uint32_t* words = static_cast<uint32_t*>(workspace);
     const uint64_t kMaxItems = uint64_t(1) << 30;   // queue positions (2 per item) stay 32-bit
     FlowArgs a;
@@ -926,20 +955,24 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
         const size_t smem = (size_t)kFlowStages * kFlowStageBytes;
         static int configured[64] = {0};
         if (dev >= 0 && dev < 64 && !configured[dev]) {
-            e = cudaFuncSetAttribute(nvfp4_flow_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(nvfp4_flow_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+            const void* fns[4] = {(const void*)nvfp4_flow_kernel<true, false>,
+                                  (const void*)nvfp4_flow_kernel<false, false>,
+                                  (const void*)nvfp4_flow_kernel<true, true>,
+                                  (const void*)nvfp4_flow_kernel<false, true>};
+            for (int f = 0; f < 4 && e == cudaSuccess; ++f)
+                e = cudaFuncSetAttribute(fns[f], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             configured[dev] = 1;
         }
         const int grid = (int)std::max<int64_t>(
             1, std::min<int64_t>((int64_t)sm_count(dev) * kFlowCtasPerSm, 2 * (int64_t)a.total_items));
         a.lead = kFlowLeadPerCta * (uint32_t)grid;
-        if (fake)
-            nvfp4_flow_kernel<true><<<grid, kFlowThreads, smem, s>>>(a);
+        if (fp8)
+            fake ? nvfp4_flow_kernel<true, true><<<grid, kFlowThreads, smem, s>>>(a)
+                 : nvfp4_flow_kernel<false, true><<<grid, kFlowThreads, smem, s>>>(a);
         else
-            nvfp4_flow_kernel<false><<<grid, kFlowThreads, smem, s>>>(a);
+            fake ? nvfp4_flow_kernel<true, false><<<grid, kFlowThreads, smem, s>>>(a)
+                 : nvfp4_flow_kernel<false, false><<<grid, kFlowThreads, smem, s>>>(a);
         e = cudaGetLastError();
         reset();
         return e;
@@ -985,8 +1018,11 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
                 M.chunks = (uint32_t)(x.rows * (x.cols / 8));
                 M.sb = fake ? nullptr : G.sb[i] + b0 * (int64_t)(M.chunks / 2);
                 M.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
-                M.dense_x = dense_rows(x, x.cols * 2);
+                M.dense_x = dense_rows(x, fp8 ? x.cols : x.cols * 2);
                 M.dense_o = dense_rows(o, fake ? o.cols * 2 : o.cols / 2);
+                M.tn = (uint32_t)((x.cols + 127) / 128);
+                M.ts_bs = (int64_t)((x.rows + 127) / 128) * M.tn;
+                M.ts = fp8 ? G.ts[i] + b0 * M.ts_bs : nullptr;
                 M.item_off = off;
                 off += (M.chunks + kItemChunks - 1) / kItemChunks;
             }

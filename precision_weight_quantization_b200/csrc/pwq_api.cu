@@ -673,23 +673,19 @@ pwq_status fp8_block_requant_mxfp8(const pwq_tensor* q_in, const float* scale_in
     return from_cuda(pwq::launch_fp8_requant_mxfp8(vq, scale_in, vo, scale_ue8m0, (cudaStream_t)stream));
 }
 
-size_t fp8_block_requant_nvfp4_workspace_size(int n_siblings, const pwq_tensor* q_in) {
-    if (!q_in || n_siblings < 1 || n_siblings > PWQ_MAX_SIBLINGS || q_in[0].batch < 0) return 0;
-    return (size_t)((std::max<int64_t>(1, q_in[0].batch) * 4 + 255) / 256 * 256);
-}
+namespace {
 
-pwq_status fp8_block_requant_nvfp4(const pwq_tensor* q_in, const float* const* scale_in, int n_siblings,
-                                   const pwq_tensor* q_packed, uint8_t* const* sb, float* global_scale,
-                                   const float* amax_in, void* workspace, size_t workspace_bytes,
-                                   pwq_stream_t stream) {
-    if (n_siblings < 1 || n_siblings > PWQ_MAX_SIBLINGS) return fail(PWQ_ERR_ARG, "n_siblings out of range");
-    if (!q_in || !q_packed) return fail(PWQ_ERR_NULL, "q_in / q_packed");
-    View vq[PWQ_MAX_SIBLINGS], vo[PWQ_MAX_SIBLINGS];
-    std::vector<Extent> ins, outs;
-    bool all_empty = true;
+// One FP8 block-wise sibling group of a re-quantisation into NVFP4: codes
+// (N % 16 == 0, same batch), their tile scales, packed outputs and block
+// scales; appends extents.
+pwq_status check_requant_nv_group(const pwq_tensor* q_in, const float* const* scale_in, int n,
+                                  const pwq_tensor* q_packed, uint8_t* const* sb, View* vq, View* vo,
+                                  std::vector<Extent>& ins, std::vector<Extent>& outs, bool* all_empty) {
+    if (n < 1 || n > PWQ_MAX_SIBLINGS) return fail(PWQ_ERR_ARG, "n_siblings out of range");
     const int64_t B = q_in[0].batch;
+    *all_empty = true;
     pwq_status st;
-    for (int i = 0; i < n_siblings; ++i) {
+    for (int i = 0; i < n; ++i) {
         Extent eq, eo;
         if ((st = check_tensor(&q_in[i], Kind::kByte, &vq[i], &eq, "q_in[i]")) != PWQ_OK) return st;
         if (q_in[i].batch != B) return fail(PWQ_ERR_ARG, "siblings differ in batch");
@@ -697,7 +693,7 @@ pwq_status fp8_block_requant_nvfp4(const pwq_tensor* q_in, const float* const* s
         if (!same_shape(&q_in[i], &q_packed[i])) return fail(PWQ_ERR_SHAPE, "q_packed shape != q_in shape");
         if ((st = check_tensor(&q_packed[i], Kind::kPacked4, &vo[i], &eo, "q_packed[i]")) != PWQ_OK) return st;
         if (empty(&q_in[i])) continue;
-        all_empty = false;
+        *all_empty = false;
         if (!scale_in || !scale_in[i]) return fail(PWQ_ERR_NULL, "scale_in[i]");
         if ((uintptr_t)scale_in[i] % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale_in[i]");
         if (!sb || !sb[i]) return fail(PWQ_ERR_NULL, "sb[i]");
@@ -707,29 +703,99 @@ pwq_status fp8_block_requant_nvfp4(const pwq_tensor* q_in, const float* const* s
         outs.push_back(extent_of(sb[i], (size_t)(B * q_in[i].rows * (q_in[i].cols / 16))));
     }
     if (B > 65535) return fail(PWQ_ERR_SHAPE, "batch > 65535");
-    if (all_empty || B == 0) return PWQ_OK;
-    if (!global_scale) return fail(PWQ_ERR_NULL, "global_scale");
-    if ((uintptr_t)global_scale % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
-    outs.push_back(extent_of(global_scale, (size_t)B * 4));
+    return PWQ_OK;
+}
+
+// Shared body of fp8_block_requant_nvfp4 and its grouped form.
+pwq_status requant_nv_run(int n_groups, const int* sizes, const pwq_tensor* q_in, const float* const* scale_in,
+                          const pwq_tensor* q_packed, uint8_t* const* sb, float* const* global_scale,
+                          const float* amax_in, void* ws, size_t ws_bytes, pwq_stream_t stream) {
+    if (n_groups < 1 || n_groups > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group count out of range");
+    if (!sizes || !q_in || !q_packed) return fail(PWQ_ERR_NULL, "group sizes / tensors");
+    struct G {
+        View q[PWQ_MAX_SIBLINGS], o[PWQ_MAX_SIBLINGS];
+    };
+    std::vector<G> views(n_groups);
+    std::vector<Extent> ins, outs;
+    std::vector<pwq::NvGroup> launch;
+    int m = 0;
+    int64_t instances = 0;
+    for (int g = 0; g < n_groups; ++g) {
+        const int n = sizes[g];
+        if (n < 1 || n > PWQ_MAX_SIBLINGS || m + n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group size");
+        bool all_empty;
+        pwq_status st = check_requant_nv_group(q_in + m, scale_in ? scale_in + m : nullptr, n, q_packed + m,
+                                               sb ? sb + m : nullptr, views[g].q, views[g].o, ins, outs,
+                                               &all_empty);
+        if (st != PWQ_OK) return st;
+        const int64_t B = q_in[m].batch;
+        if (!all_empty && B > 0) {
+            if (!global_scale || !global_scale[g]) return fail(PWQ_ERR_NULL, "global_scale");
+            if ((uintptr_t)global_scale[g] % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
+            outs.push_back(extent_of(global_scale[g], (size_t)B * 4));
+            pwq::NvGroup ng;
+            ng.x = views[g].q;
+            ng.out = views[g].o;
+            ng.sb = sb + m;
+            ng.n = n;
+            ng.amax_in = amax_in;
+            ng.gs_out = global_scale[g];
+            ng.amax_out = nullptr;
+            ng.ts = scale_in + m;
+            launch.push_back(ng);
+            instances += B;
+        }
+        m += n;
+    }
     if (amax_in) {
+        if (n_groups != 1) return fail(PWQ_ERR_ARG, "amax_in needs a single group");
         if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
-        ins.push_back(extent_of(amax_in, (size_t)B * 4));
-    } else {
-        const size_t need = fp8_block_requant_nvfp4_workspace_size(n_siblings, q_in);
-        if (!workspace || (uintptr_t)workspace % 4 != 0 || workspace_bytes < need)
-            return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
-        outs.push_back(extent_of(workspace, need));
+        ins.push_back(extent_of(amax_in, (size_t)q_in[0].batch * 4));
     }
-    if ((st = check_requant_overlaps(ins, outs, {})) != PWQ_OK) return st;
-    cudaStream_t s = (cudaStream_t)stream;
-    uint32_t* amax_bits = nullptr;
+    if (launch.empty()) return PWQ_OK;
     if (!amax_in) {
-        amax_bits = static_cast<uint32_t*>(workspace);
-        cudaError_t e = pwq::launch_nvfp4_amax(vq, n_siblings, amax_bits, s, scale_in);   // clears the words first
-        if (e != cudaSuccess) return cuda_fail(e);
+        pwq_status st = check_workspace(ws, ws_bytes, instances);
+        if (st != PWQ_OK) return st;
+        outs.push_back(extent_of(ws, pwq::nvfp4_flow_workspace_bytes(instances)));
     }
-    return from_cuda(pwq::launch_nvfp4_encode(vq, n_siblings, vo, sb, false, amax_bits, amax_in, global_scale,
-                                              nullptr, s, scale_in));
+    pwq_status st = check_requant_overlaps(ins, outs, {});
+    if (st != PWQ_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (amax_in) {
+        const pwq::NvGroup& G0 = launch[0];
+        return from_cuda(pwq::launch_nvfp4_encode(G0.x, G0.n, G0.out, G0.sb, false, nullptr, amax_in, G0.gs_out,
+                                                  nullptr, s, G0.ts));
+    }
+    return from_cuda(pwq::launch_nvfp4_flow(launch.data(), (int)launch.size(), false, ws, s));
+}
+
+}  // namespace
+
+size_t fp8_block_requant_nvfp4_workspace_size(int n_siblings, const pwq_tensor* q_in) {
+    return nvfp4_workspace_size(n_siblings, q_in);
+}
+
+size_t fp8_block_requant_nvfp4_workspace_size_grouped(int n_groups, const int* group_sizes,
+                                                      const pwq_tensor* q_in) {
+    return nvfp4_workspace_size_grouped(n_groups, group_sizes, q_in);
+}
+
+pwq_status fp8_block_requant_nvfp4(const pwq_tensor* q_in, const float* const* scale_in, int n_siblings,
+                                   const pwq_tensor* q_packed, uint8_t* const* sb, float* global_scale,
+                                   const float* amax_in, void* workspace, size_t workspace_bytes,
+                                   pwq_stream_t stream) {
+    const int sizes[1] = {n_siblings};
+    float* gs[1] = {global_scale};
+    if (n_siblings < 1 || n_siblings > PWQ_MAX_SIBLINGS) return fail(PWQ_ERR_ARG, "n_siblings out of range");
+    return requant_nv_run(1, sizes, q_in, scale_in, q_packed, sb, gs, amax_in, workspace, workspace_bytes, stream);
+}
+
+pwq_status fp8_block_requant_nvfp4_grouped(int n_groups, const int* group_sizes, const pwq_tensor* q_in,
+                                           const float* const* scale_in, const pwq_tensor* q_packed,
+                                           uint8_t* const* sb, float* const* global_scale, void* workspace,
+                                           size_t workspace_bytes, pwq_stream_t stream) {
+    return requant_nv_run(n_groups, group_sizes, q_in, scale_in, q_packed, sb, global_scale, nullptr, workspace,
+                          workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------------ self-tests

@@ -50,6 +50,7 @@ struct NvGroup {
     const float* amax_in;   // [B] or null
     float* gs_out;          // [B] or null
     float* amax_out;        // [B] or null
+    const float* const* ts = nullptr;   // FP8 block-wise source: n tile-scale arrays (x are E4M3 code views)
 };
 
 // NVFP4 single-pass quantise / fake-quantise of groups whose amax is reduced

@@ -182,7 +182,7 @@ def test_requant_validation_without_gpu():
     sb = (ctypes.c_void_p * 2)(base + (5 << 30), base + (5 << 30) + (1 << 24))
     gs = base + (6 << 30)
     ws = base + (7 << 30)
-    assert lib.fp8_block_requant_nvfp4_workspace_size(2, qs) == 256
+    assert lib.fp8_block_requant_nvfp4_workspace_size(2, qs) == lib.nvfp4_workspace_size(2, qs) == 256
     assert lib.fp8_block_requant_nvfp4(qs, ss, 0, pk, sb, gs, None, ws, 256, None) == L.PWQ_ERR_ARG
     assert lib.fp8_block_requant_nvfp4(qs, ss, 2, pk, sb, gs, None, None, 0, None) == L.PWQ_ERR_WORKSPACE
     ss_null = (ctypes.c_void_p * 2)(s, None)

@@ -145,3 +145,25 @@ def test_full_size_gate_proj_sampled(P):
         assert np.array_equal(mqn[r0:r1], oq) and np.array_equal(men[r0:r1], oe)
         opk, osb, _ = O.nvfp4_quant(y[r0:r1], A)
         assert np.array_equal(pkn[r0:r1], opk) and np.array_equal(sbn[r0:r1], osb)
+
+
+def test_fp8_to_nvfp4_grouped_single_pass(P):
+    # a layer-like list of sibling groups in one launch: ragged rows, a batched
+    # group, a strided member (read without the bulk copy) and a member larger
+    # than one 16384-element work item
+    specs = [[((96, 256), 0), ((32, 256), 16), ((32, 256), 0)], [((1024, 512), 0)],
+             [((3, 40, 160), 0), ((3, 24, 160), 8)], [((130, 64), 0)]]
+    groups, scales, oracle = [], [], []
+    for g, grp in enumerate(specs):
+        ms = [codes_and_scales(sh, seed=40 + 5 * g + i, raw=(g % 2 == 1)) for i, (sh, _) in enumerate(grp)]
+        groups.append([to_gpu_codes(m[0], pad) for m, (_, pad) in zip(ms, grp)])
+        scales.append([torch.from_numpy(m[1]).to(DEV) for m in ms])
+        oracle.append(O.fp8_block_requant_nvfp4([m[0] for m in ms], [m[1] for m in ms]))
+    pk, sb, gs = P.fp8_block_requant_nvfp4_grouped(groups, scales)
+    for g, (A, out, ogs) in enumerate(oracle):
+        assert np.array_equal(f32bits(gs[g]), ogs.view(np.uint32)), g
+        for i in range(len(out)):
+            assert np.array_equal(u8(pk[g][i]), out[i][0]), (g, i)
+            assert np.array_equal(u8(sb[g][i]), out[i][1]), (g, i)
+    torch.cuda.synchronize()
+    assert P.device_error() == 0
