@@ -352,28 +352,30 @@ NEXT_BYTES_PER_ELEM = {
 
 
 def next_calls(op, layers, buf, P, torch):
-    """One call per tensor (one grouped call per layer for NVFP4, all four
-    sibling groups in one single-pass launch), reading the FP8 codes and
-    scales the step wrote; outputs shared by all layers."""
+    """One grouped call per layer (the 7 tensors; for NVFP4 the four sibling
+    groups in one single-pass launch), reading the FP8 codes and scales the
+    step wrote; outputs shared by all layers."""
     import workloads as W
     lay0 = layers[0]
     dev = lay0["q_proj"].device
     out_q = {n: torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev) for n, x in lay0.items()}
     calls = []
+    names = list(lay0)
     if op == "fp8_block_requant":
-        out_s = {n: torch.empty_like(buf.fp8[0][n][1]) for n in lay0}
+        out_s = [torch.empty_like(buf.fp8[0][n][1]) for n in names]
         for i in range(len(layers)):
-            for n in lay0:
-                q, sc = buf.fp8[i][n]
-                calls.append(lambda q=q, sc=sc, n=n: P.fp8_block_requant(q, sc, out=out_q[n], scale_out=out_s[n]))
+            qs = [buf.fp8[i][n][0] for n in names]
+            ss = [buf.fp8[i][n][1] for n in names]
+            calls.append(lambda qs=qs, ss=ss: P.fp8_block_requant_grouped(
+                qs, ss, out=[out_q[n] for n in names], scale_out=out_s))
     elif op == "fp8_block_requant_mxfp8":
-        out_e = {n: torch.empty((x.shape[0], x.shape[1] // 32), dtype=torch.uint8, device=dev)
-                 for n, x in lay0.items()}
+        out_e = [torch.empty((lay0[n].shape[0], lay0[n].shape[1] // 32), dtype=torch.uint8, device=dev)
+                 for n in names]
         for i in range(len(layers)):
-            for n in lay0:
-                q, sc = buf.fp8[i][n]
-                calls.append(lambda q=q, sc=sc, n=n: P.fp8_block_requant_mxfp8(q, sc, out=out_q[n],
-                                                                               scale_out=out_e[n]))
+            qs = [buf.fp8[i][n][0] for n in names]
+            ss = [buf.fp8[i][n][1] for n in names]
+            calls.append(lambda qs=qs, ss=ss: P.fp8_block_requant_mxfp8_grouped(
+                qs, ss, out=[out_q[n] for n in names], scale_out=out_e))
     else:
         pk = {n: torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for n, x in lay0.items()}
         sb = {n: torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev)

@@ -335,6 +335,18 @@ pwq_status fp8_block_requant(const pwq_tensor* q_in, const float* scale_in, cons
 pwq_status fp8_block_requant_mxfp8(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out,
                                    uint8_t* scale_ue8m0, pwq_stream_t stream);
 
+/* Grouped forms: n tensors (at most 256; one launch per 16), e.g. the seven
+ * weights of a decoder layer; q_in / q_out / scale arrays indexed alike,
+ * each tensor under the rules of the single call.  The MXFP8 form reads 16
+ * codes per 16-byte load when every code tensor of the call has 16-byte
+ * aligned base and strides, and falls back to one launch per tensor with
+ * 8-byte loads otherwise. */
+pwq_status fp8_block_requant_grouped(int n, const pwq_tensor* q_in, const float* const* scale_in,
+                                     const pwq_tensor* q_out, float* const* scale_out, pwq_stream_t stream);
+pwq_status fp8_block_requant_mxfp8_grouped(int n, const pwq_tensor* q_in, const float* const* scale_in,
+                                           const pwq_tensor* q_out, uint8_t* const* scale_ue8m0,
+                                           pwq_stream_t stream);
+
 /* Bytes of workspace fp8_block_requant_nvfp4 / _grouped need: as
  * nvfp4_workspace_size / nvfp4_workspace_size_grouped for the same shapes;
  * 0 on bad input. */

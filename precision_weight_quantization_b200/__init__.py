@@ -27,7 +27,7 @@ __all__ = [
     "device_error", "PwqError", "LIB_PATH", "fp8_block_quant_grouped", "fp8_block_dequant_grouped",
     "mxfp8_quant_grouped", "mxfp8_dequant_grouped", "nvfp4_dequant_grouped", "nvfp4_quant_grouped",
     "nvfp4_fake_quant_grouped", "fp8_block_requant", "fp8_block_requant_mxfp8", "fp8_block_requant_nvfp4",
-    "fp8_block_requant_nvfp4_grouped",
+    "fp8_block_requant_nvfp4_grouped", "fp8_block_requant_grouped", "fp8_block_requant_mxfp8_grouped",
 ]
 
 _CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
@@ -472,6 +472,38 @@ def fp8_block_requant_nvfp4(qs, scales, amax: Optional[torch.Tensor] = None, out
     if single:
         return out[0], sb[0], global_scale
     return out, sb, global_scale
+
+
+def fp8_block_requant_grouped(qs: Sequence[torch.Tensor], scales: Sequence[torch.Tensor], out=None,
+                              scale_out=None, inplace: bool = False):
+    """fp8_block_requant over a list of tensors in one launch per 16."""
+    qs, scales = list(qs), list(scales)
+    for i, (q, s_) in enumerate(zip(qs, scales)):
+        _fp8_input(q, s_, "q[%d]" % i)
+    if out is None:
+        out = qs if inplace else [torch.empty(q.shape, dtype=torch.float8_e4m3fn, device=q.device) for q in qs]
+    if scale_out is None:
+        scale_out = scales if inplace else [torch.empty_like(s_) for s_ in scales]
+    check(lib.fp8_block_requant_grouped(len(qs), _desc_array(qs, "q"), _ptrs(scales), _desc_array(out, "out"),
+                                        _ptrs(scale_out), _stream(qs[0])), "fp8_block_requant_grouped")
+    return out, scale_out
+
+
+def fp8_block_requant_mxfp8_grouped(qs: Sequence[torch.Tensor], scales: Sequence[torch.Tensor], out=None,
+                                    scale_out=None, inplace: bool = False):
+    """fp8_block_requant_mxfp8 over a list of tensors in one launch per 16."""
+    qs, scales = list(qs), list(scales)
+    for i, (q, s_) in enumerate(zip(qs, scales)):
+        _fp8_input(q, s_, "q[%d]" % i)
+    if out is None:
+        out = qs if inplace else [torch.empty(q.shape, dtype=torch.float8_e4m3fn, device=q.device) for q in qs]
+    if scale_out is None:
+        scale_out = [torch.empty(q.shape[:-1] + (q.shape[-1] // 32,), dtype=torch.uint8, device=q.device)
+                     for q in qs]
+    check(lib.fp8_block_requant_mxfp8_grouped(len(qs), _desc_array(qs, "q"), _ptrs(scales),
+                                              _desc_array(out, "out"), _ptrs(scale_out), _stream(qs[0])),
+          "fp8_block_requant_mxfp8_grouped")
+    return out, scale_out
 
 
 def fp8_block_requant_nvfp4_grouped(groups, scales, out=None, sb=None, global_scale=None):

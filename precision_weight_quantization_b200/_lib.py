@@ -62,6 +62,8 @@ _SIG = {
     "nvfp4_fake_quant_grouped": (_S, [ctypes.c_int, _IP, _T, _T, _PP, _P, ctypes.c_size_t, _P]),
     "fp8_block_requant": (_S, [_T, _P, _T, _P, _P]),
     "fp8_block_requant_mxfp8": (_S, [_T, _P, _T, _P, _P]),
+    "fp8_block_requant_grouped": (_S, [ctypes.c_int, _T, _PP, _T, _PP, _P]),
+    "fp8_block_requant_mxfp8_grouped": (_S, [ctypes.c_int, _T, _PP, _T, _PP, _P]),
     "fp8_block_requant_nvfp4_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _T]),
     "fp8_block_requant_nvfp4": (_S, [_T, _PP, ctypes.c_int, _T, _PP, _P, _P, _P, ctypes.c_size_t, _P]),
     "fp8_block_requant_nvfp4_workspace_size_grouped": (ctypes.c_size_t, [ctypes.c_int, _IP, _T]),

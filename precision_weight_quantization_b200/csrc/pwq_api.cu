@@ -641,36 +641,74 @@ pwq_status check_requant_io(const pwq_tensor* q_in, const float* scale_in, const
 
 }  // namespace
 
+namespace {
+
+// Shared body of the FP8 -> FP8 / MXFP8 re-quantisation calls over a list of
+// n tensors.  In place: q_out[i] == q_in[i] exactly, and for FP8 scale_out[i]
+// == scale_in[i].
+pwq_status requant_list(bool mx, int n, const pwq_tensor* q_in, const float* const* scale_in,
+                        const pwq_tensor* q_out, void* const* scale_out, pwq_stream_t stream) {
+    if (n < 0 || n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "tensor count out of range");
+    if (n == 0) return PWQ_OK;
+    if (!q_in || !q_out || !scale_in || !scale_out) return fail(PWQ_ERR_NULL, "tensor or scale array");
+    std::vector<pwq::RequantJob> jobs;
+    std::vector<Extent> ins, outs;
+    std::vector<std::pair<int, int>> allowed;
+    for (int i = 0; i < n; ++i) {
+        pwq::RequantJob J;
+        Extent eq, eo, esi;
+        pwq_status st = check_requant_io(&q_in[i], scale_in[i], &q_out[i], &J.in, &J.out, &eq, &eo, &esi);
+        if (st != PWQ_OK) return st;
+        if (mx && q_in[i].cols % 32 != 0) return fail(PWQ_ERR_SHAPE, "cols % 32 != 0");
+        if (empty(&q_in[i])) continue;
+        if (!scale_out[i]) return fail(PWQ_ERR_NULL, "scale_out");
+        if (!mx && (uintptr_t)scale_out[i] % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale_out");
+        const Extent eso = extent_of(scale_out[i], mx ? (size_t)(q_in[i].batch * q_in[i].rows * (q_in[i].cols / 32))
+                                                      : tile_scale_bytes(&q_in[i]));
+        const int in0 = (int)ins.size(), out0 = (int)outs.size();
+        ins.push_back(eq);
+        ins.push_back(esi);
+        outs.push_back(eo);
+        outs.push_back(eso);
+        if (exact_alias(&q_in[i], &q_out[i])) allowed.push_back({out0, in0});
+        if (!mx && scale_out[i] == (const void*)scale_in[i]) allowed.push_back({out0 + 1, in0 + 1});
+        J.scale_in = scale_in[i];
+        J.scale_out = scale_out[i];
+        jobs.push_back(J);
+    }
+    pwq_status st = check_requant_overlaps(ins, outs, allowed);
+    if (st != PWQ_OK) return st;
+    if (jobs.empty()) return PWQ_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    return from_cuda(mx ? pwq::launch_fp8_requant_mxfp8(jobs.data(), (int)jobs.size(), s)
+                        : pwq::launch_fp8_requant_fp8(jobs.data(), (int)jobs.size(), s));
+}
+
+}  // namespace
+
 pwq_status fp8_block_requant(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out,
                              float* scale_out, pwq_stream_t stream) {
-    View vq, vo;
-    Extent eq, eo, esi;
-    pwq_status st = check_requant_io(q_in, scale_in, q_out, &vq, &vo, &eq, &eo, &esi);
-    if (st != PWQ_OK || empty(q_in)) return st;
-    if (!scale_out) return fail(PWQ_ERR_NULL, "scale_out");
-    if ((uintptr_t)scale_out % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale_out");
-    const Extent eso = extent_of(scale_out, tile_scale_bytes(q_in));
-    std::vector<std::pair<int, int>> allowed;
-    if (exact_alias(q_in, q_out)) allowed.push_back({0, 0});
-    if (scale_out == scale_in) allowed.push_back({1, 1});
-    if ((st = check_requant_overlaps({eq, esi}, {eo, eso}, allowed)) != PWQ_OK) return st;
-    return from_cuda(pwq::launch_fp8_requant_fp8(vq, scale_in, vo, scale_out, (cudaStream_t)stream));
+    const float* si[1] = {scale_in};
+    void* so[1] = {scale_out};
+    return requant_list(false, 1, q_in, si, q_out, so, stream);
 }
 
 pwq_status fp8_block_requant_mxfp8(const pwq_tensor* q_in, const float* scale_in, const pwq_tensor* q_out,
                                    uint8_t* scale_ue8m0, pwq_stream_t stream) {
-    View vq, vo;
-    Extent eq, eo, esi;
-    pwq_status st = check_requant_io(q_in, scale_in, q_out, &vq, &vo, &eq, &eo, &esi);
-    if (st != PWQ_OK) return st;
-    if (q_in->cols % 32 != 0) return fail(PWQ_ERR_SHAPE, "cols % 32 != 0");
-    if (empty(q_in)) return PWQ_OK;
-    if (!scale_ue8m0) return fail(PWQ_ERR_NULL, "scale_ue8m0");
-    const Extent ee = extent_of(scale_ue8m0, (size_t)(q_in->batch * q_in->rows * (q_in->cols / 32)));
-    std::vector<std::pair<int, int>> allowed;
-    if (exact_alias(q_in, q_out)) allowed.push_back({0, 0});
-    if ((st = check_requant_overlaps({eq, esi}, {eo, ee}, allowed)) != PWQ_OK) return st;
-    return from_cuda(pwq::launch_fp8_requant_mxfp8(vq, scale_in, vo, scale_ue8m0, (cudaStream_t)stream));
+    const float* si[1] = {scale_in};
+    void* so[1] = {scale_ue8m0};
+    return requant_list(true, 1, q_in, si, q_out, so, stream);
+}
+
+pwq_status fp8_block_requant_grouped(int n, const pwq_tensor* q_in, const float* const* scale_in,
+                                     const pwq_tensor* q_out, float* const* scale_out, pwq_stream_t stream) {
+    return requant_list(false, n, q_in, scale_in, q_out, reinterpret_cast<void* const*>(scale_out), stream);
+}
+
+pwq_status fp8_block_requant_mxfp8_grouped(int n, const pwq_tensor* q_in, const float* const* scale_in,
+                                           const pwq_tensor* q_out, uint8_t* const* scale_ue8m0,
+                                           pwq_stream_t stream) {
+    return requant_list(true, n, q_in, scale_in, q_out, reinterpret_cast<void* const*>(scale_ue8m0), stream);
 }
 
 namespace {

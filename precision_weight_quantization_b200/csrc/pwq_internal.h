@@ -74,9 +74,15 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
                                 const float* const* ts = nullptr);
 
 // FP8 block-wise codes + tile scales re-quantised (dequantise, quantise) into
-// FP8 block-wise (new scales) or MXFP8; q2 may be q, s2 may be s.
-cudaError_t launch_fp8_requant_fp8(const View& q, const float* s, const View& q2, float* s2, cudaStream_t st);
-cudaError_t launch_fp8_requant_mxfp8(const View& q, const float* s, const View& q2, uint8_t* e, cudaStream_t st);
+// FP8 block-wise (new FP32 tile scales) or MXFP8 (UE8M0 bytes), a list of
+// tensors per call; out may be in exactly, scale_out may be scale_in (FP8).
+struct RequantJob {
+    View in, out;           // E4M3 codes
+    const void* scale_in;   // FP32 [B][TM][TN]
+    void* scale_out;        // FP8: FP32 [B][TM][TN]; MXFP8: uint8 [B][M][N/32]
+};
+cudaError_t launch_fp8_requant_fp8(const RequantJob* jobs, int n, cudaStream_t st);
+cudaError_t launch_fp8_requant_mxfp8(const RequantJob* jobs, int n, cudaStream_t st);
 
 // Device address (on the current device) of the file-scope group-amax
 // scratch used by nvfp4_fake_quant_noalloc; kStaticScratchGroups words.

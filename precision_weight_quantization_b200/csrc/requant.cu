@@ -35,16 +35,73 @@ constexpr int kTile = 128;
 constexpr int kRowsPerPass = kThreads / 16;    // 16 rows of 16 threads x 8 codes
 constexpr int kChunks = kTile / kRowsPerPass;  // 8 chunks of 8 codes per thread
 
-struct TileArgs {
+// One tensor of a grouped FP8 -> FP8 launch.
+struct RqTensor {
     const char* q;            // E4M3 codes in
     char* q2;                 // E4M3 codes out (may be q)
     int64_t q_bs, q_rs, o_bs, o_rs;   // bytes
     const float* s;           // [B][TM][TN] in
     float* s2;                // [B][TM][TN] out (may be s)
     int rows, cols;
-    uint32_t tiles;           // B * TM * TN
+    uint32_t tile_begin;      // first tile of this tensor in the launch
     FastDiv tiles_n, tiles_mn;
 };
+
+struct TileArgs {
+    RqTensor t[kMaxLaunchTensors];
+    int n;
+    uint32_t total_tiles;
+};
+
+// Where tile `tile` of the launch lives, and its old scale.
+struct TileWork {
+    const char* qt;
+    char* ot;
+    int64_t q_rs, o_rs;
+    float* s2;                // address of the new scale
+    float s;
+    int rows_here, cols_here;
+};
+
+__device__ __forceinline__ TileWork tile_work(const TileArgs& a, uint32_t tile) {
+    int i = 0;
+    for (int k = 1; k < a.n; ++k)
+        if (tile >= a.t[k].tile_begin) i = k;
+    const RqTensor& T = a.t[i];
+    const uint32_t lt = tile - T.tile_begin;
+    const uint32_t b = fdiv(lt, T.tiles_mn);
+    const uint32_t rem = lt - b * T.tiles_mn.d;
+    const uint32_t tm = fdiv(rem, T.tiles_n);
+    const uint32_t tn = rem - tm * T.tiles_n.d;
+    TileWork w;
+    w.qt = T.q + (int64_t)b * T.q_bs + (int64_t)tm * kTile * T.q_rs + (int64_t)tn * kTile;
+    w.ot = T.q2 + (int64_t)b * T.o_bs + (int64_t)tm * kTile * T.o_rs + (int64_t)tn * kTile;
+    w.q_rs = T.q_rs;
+    w.o_rs = T.o_rs;
+    w.s2 = T.s2 + lt;
+    w.s = T.s[lt];
+    w.rows_here = min(kTile, T.rows - (int)tm * kTile);
+    w.cols_here = min(kTile, T.cols - (int)tn * kTile);
+    return w;
+}
+
+__device__ __forceinline__ void load_tile(const TileWork& w, int row0, int ccol, uint2 (&v)[kChunks]) {
+    if (w.rows_here == kTile && w.cols_here == kTile) {
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j) v[j] = ld_stream_v2(w.qt + (int64_t)(row0 + kRowsPerPass * j) * w.q_rs + ccol);
+    } else {
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j) {
+            const int r = row0 + kRowsPerPass * j;
+            uint64_t x = 0u;
+            if (r < w.rows_here) {
+                const unsigned char* src = reinterpret_cast<const unsigned char*>(w.qt + (int64_t)r * w.q_rs);
+                for (int c = ccol; c < min(ccol + 8, w.cols_here); ++c) x |= (uint64_t)src[c] << (8 * (c - ccol));
+            }
+            v[j] = make_uint2((uint32_t)x, (uint32_t)(x >> 32));
+        }
+    }
+}
 
 template <bool kFast>
 __device__ __forceinline__ uint2 requant8(uint2 c, float s, float s2, float r2) {
@@ -54,38 +111,26 @@ __device__ __forceinline__ uint2 requant8(uint2 c, float s, float s2, float r2) 
     return make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
 }
 
-__global__ void __launch_bounds__(kThreads, 4) fp8_requant_fp8_kernel(const __grid_constant__ TileArgs a) {
+// Persistent CTAs over the tiles of all tensors of the launch; each thread
+// holds the codes of the next tile (loads in flight) while it re-encodes the
+// current one.
+__global__ void __launch_bounds__(kThreads, 3) fp8_requant_fp8_kernel(const __grid_constant__ TileArgs a) {
     __shared__ uint32_t red[2][kThreads / 32];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     const int ccol = (int)(tid & 15u) * 8;
     const int row0 = (int)(tid >> 4);
-    uint32_t par = 0;
-    for (uint32_t t = blockIdx.x; t < a.tiles; t += gridDim.x, par ^= 1u) {
-        const uint32_t b = fdiv(t, a.tiles_mn);
-        const uint32_t rem = t - b * a.tiles_mn.d;
-        const uint32_t tm = fdiv(rem, a.tiles_n);
-        const uint32_t tn = rem - tm * a.tiles_n.d;
-        const float s = a.s[t];
-        const char* qt = a.q + (int64_t)b * a.q_bs + (int64_t)tm * kTile * a.q_rs + (int64_t)tn * kTile;
-        char* ot = a.q2 + (int64_t)b * a.o_bs + (int64_t)tm * kTile * a.o_rs + (int64_t)tn * kTile;
-        const int rows_here = min(kTile, a.rows - (int)tm * kTile);
-        const int cols_here = min(kTile, a.cols - (int)tn * kTile);
-        const bool full = rows_here == kTile && cols_here == kTile;
-        uint2 v[kChunks];
-        if (full) {
-#pragma unroll
-            for (int j = 0; j < kChunks; ++j) v[j] = ld_stream_v2(qt + (int64_t)(row0 + kRowsPerPass * j) * a.q_rs + ccol);
-        } else {
-#pragma unroll
-            for (int j = 0; j < kChunks; ++j) {
-                const int r = row0 + kRowsPerPass * j;
-                uint64_t w = 0u;
-                if (r < rows_here) {
-                    const unsigned char* src = reinterpret_cast<const unsigned char*>(qt + (int64_t)r * a.q_rs);
-                    for (int c = ccol; c < min(ccol + 8, cols_here); ++c) w |= (uint64_t)src[c] << (8 * (c - ccol));
-                }
-                v[j] = make_uint2((uint32_t)w, (uint32_t)(w >> 32));
-            }
+    uint32_t t = blockIdx.x;
+    if (t >= a.total_tiles) return;
+    TileWork w = tile_work(a, t);
+    uint2 v[kChunks];
+    load_tile(w, row0, ccol, v);
+    for (uint32_t par = 0;; par ^= 1u) {
+        const uint32_t tn = t + gridDim.x;
+        TileWork nw;
+        uint2 nv[kChunks];
+        if (tn < a.total_tiles) {
+            nw = tile_work(a, tn);
+            load_tile(nw, row0, ccol, nv);
         }
         uint32_t m = 0u;
 #pragma unroll
@@ -95,28 +140,33 @@ __global__ void __launch_bounds__(kThreads, 4) fp8_requant_fp8_kernel(const __gr
         if (lane == 0u) red[par][warp] = m;
         __syncthreads();   // codes of the tile all read (in place is safe from here on)
 #pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) m = max(m, red[par][w]);
-        const float amax = __uint_as_float(fp8_amax_bits16(m, s) << 16);
+        for (int k = 0; k < kThreads / 32; ++k) m = max(m, red[par][k]);
+        const float amax = __uint_as_float(fp8_amax_bits16(m, w.s) << 16);
         const float s2 = fp8_tile_scale(amax);
-        if (tid == 0) a.s2[t] = s2;
+        if (tid == 0) *w.s2 = s2;
         const bool fast = div_fast_ok(s2);   // CTA-uniform
         const float r2 = fast ? __frcp_rn(s2) : 0.0f;
         uint2 o[kChunks];
 #pragma unroll
-        for (int j = 0; j < kChunks; ++j) o[j] = fast ? requant8<true>(v[j], s, s2, r2) : requant8<false>(v[j], s, s2, r2);
-        if (full) {
+        for (int j = 0; j < kChunks; ++j) o[j] = fast ? requant8<true>(v[j], w.s, s2, r2) : requant8<false>(v[j], w.s, s2, r2);
+        if (w.rows_here == kTile && w.cols_here == kTile) {
 #pragma unroll
-            for (int j = 0; j < kChunks; ++j) st_v2(ot + (int64_t)(row0 + kRowsPerPass * j) * a.o_rs + ccol, o[j]);
+            for (int j = 0; j < kChunks; ++j) st_v2(w.ot + (int64_t)(row0 + kRowsPerPass * j) * w.o_rs + ccol, o[j]);
         } else {
 #pragma unroll
             for (int j = 0; j < kChunks; ++j) {
                 const int r = row0 + kRowsPerPass * j;
-                if (r >= rows_here) continue;
-                unsigned char* dst = reinterpret_cast<unsigned char*>(ot + (int64_t)r * a.o_rs);
-                const uint64_t w = (uint64_t)o[j].x | ((uint64_t)o[j].y << 32);
-                for (int c = ccol; c < min(ccol + 8, cols_here); ++c) dst[c] = (unsigned char)(w >> (8 * (c - ccol)));
+                if (r >= w.rows_here) continue;
+                unsigned char* dst = reinterpret_cast<unsigned char*>(w.ot + (int64_t)r * w.o_rs);
+                const uint64_t x = (uint64_t)o[j].x | ((uint64_t)o[j].y << 32);
+                for (int c = ccol; c < min(ccol + 8, w.cols_here); ++c) dst[c] = (unsigned char)(x >> (8 * (c - ccol)));
             }
         }
+        if (tn >= a.total_tiles) break;
+        t = tn;
+        w = nw;
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j) v[j] = nv[j];
     }
 }
 
@@ -188,32 +238,135 @@ __global__ void __launch_bounds__(kThreads) fp8_requant_mxfp8_kernel(const __gri
     }
 }
 
-}  // namespace
+// Grouped FP8 -> MXFP8 with 16-code chunks (one 16-byte load per lane; two
+// lanes per 1x32 block, one shuffle); needs 16-byte aligned code rows.
+struct Mx16Tensor {
+    const char* q;
+    char* q2;
+    int64_t q_bs, q_rs, o_bs, o_rs;   // bytes
+    const float* s;           // [B][TM][TN]
+    uint8_t* e;               // dense [B][M][N/32]
+    uint32_t chunks;          // B * M * N / 16
+    uint32_t slot_begin;      // multiple of kSpan
+    uint32_t tm, tn;
+    FastDiv cpr, rows;        // 16-code chunks per row (N / 16), M
+    int dense;
+};
 
-cudaError_t launch_fp8_requant_fp8(const View& q, const float* s, const View& q2, float* s2, cudaStream_t st) {
-    TileArgs a;
-    a.q = q.ptr;
-    a.q2 = q2.ptr;
-    a.q_bs = q.bstride;
-    a.q_rs = q.rstride;
-    a.o_bs = q2.bstride;
-    a.o_rs = q2.rstride;
-    a.s = s;
-    a.s2 = s2;
-    a.rows = (int)q.rows;
-    a.cols = (int)q.cols;
-    const uint32_t tm = (uint32_t)((q.rows + kTile - 1) / kTile);
-    const uint32_t tn = (uint32_t)((q.cols + kTile - 1) / kTile);
-    a.tiles = (uint32_t)q.batch * tm * tn;
-    a.tiles_n = make_fastdiv(tn);
-    a.tiles_mn = make_fastdiv(tm * tn);
-    if (a.tiles == 0) return cudaSuccess;
-    const int grid = persistent_grid(a.tiles, 4);
-    fp8_requant_fp8_kernel<<<grid, kThreads, 0, st>>>(a);
-    return cudaGetLastError();
+struct Mx16Args {
+    Mx16Tensor t[kMaxLaunchTensors];
+    int n;
+    uint32_t total_slots;
+};
+
+__device__ __forceinline__ uint2 mx_encode8(uint4 y, float inv) {
+    return make_uint2(e4m3x4(__fmul_rn(bf16_lo(y.x), inv), __fmul_rn(bf16_hi(y.x), inv),
+                             __fmul_rn(bf16_lo(y.y), inv), __fmul_rn(bf16_hi(y.y), inv)),
+                      e4m3x4(__fmul_rn(bf16_lo(y.z), inv), __fmul_rn(bf16_hi(y.z), inv),
+                             __fmul_rn(bf16_lo(y.w), inv), __fmul_rn(bf16_hi(y.w), inv)));
 }
 
-cudaError_t launch_fp8_requant_mxfp8(const View& q, const float* s, const View& q2, uint8_t* e, cudaStream_t st) {
+__global__ void __launch_bounds__(kThreads) fp8_requant_mxfp8_16_kernel(const __grid_constant__ Mx16Args a) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t slot = gwarp * kSpan; slot < a.total_slots; slot += nwarps * kSpan) {
+        int ti = 0;
+        for (int k = 1; k < a.n; ++k)
+            if (slot >= a.t[k].slot_begin) ti = k;
+        const Mx16Tensor& T = a.t[ti];
+        const uint32_t base = slot - T.slot_begin;
+        uint4 v[kUnroll];
+        float s[kUnroll];
+        int64_t oo[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint32_t c = base + u * 32u + lane;
+            const uint32_t R = fdiv(c, T.cpr);           // row over all batches
+            const uint32_t k = c - R * T.cpr.d;          // chunk within the row
+            const uint32_t b = fdiv(R, T.rows);
+            const uint32_t m = R - b * T.rows.d;
+            int64_t io;
+            if (T.dense) {
+                io = (int64_t)c * 16;
+                oo[u] = io;
+            } else {
+                io = (int64_t)b * T.q_bs + (int64_t)m * T.q_rs + (int64_t)k * 16;
+                oo[u] = (int64_t)b * T.o_bs + (int64_t)m * T.o_rs + (int64_t)k * 16;
+            }
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            s[u] = 0.0f;
+            if (c < T.chunks) {
+                v[u] = ld_stream_v4(T.q + io);
+                s[u] = __ldg(T.s + ((int64_t)b * T.tm + (m >> 7)) * T.tn + (k >> 3));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint32_t c = base + u * 32u + lane;
+            const uint2 lo = make_uint2(v[u].x, v[u].y), hi = make_uint2(v[u].z, v[u].w);
+            uint32_t mc = max(e4m3_maxmag8(lo), e4m3_maxmag8(hi));
+            mc = max(mc, __shfl_xor_sync(0xffffffffu, mc, 1));   // lanes 2i, 2i+1: one block
+            const int e = ue8m0_exponent(fp8_amax_bits16(mc, s[u]));
+            const float inv = exp2i(-e);   // exact power of two
+            const uint2 o0 = mx_encode8(fp8_dequant8(lo, s[u]), inv);
+            const uint2 o1 = mx_encode8(fp8_dequant8(hi, s[u]), inv);
+            if (c < T.chunks) {
+                st_v4(T.q2 + oo[u], make_uint4(o0.x, o0.y, o1.x, o1.y));
+                if ((lane & 1u) == 0u) T.e[c >> 1] = (uint8_t)(e + 127);
+            }
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_fp8_requant_fp8(const RequantJob* jobs, int n, cudaStream_t st) {
+    for (int j0 = 0; j0 < n;) {
+        TileArgs a;
+        a.n = 0;
+        uint32_t tiles = 0;
+        for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
+            const RequantJob& J = jobs[j0 + a.n];
+            const uint32_t tm = (uint32_t)((J.in.rows + kTile - 1) / kTile);
+            const uint32_t tn = (uint32_t)((J.in.cols + kTile - 1) / kTile);
+            const uint64_t count = (uint64_t)J.in.batch * tm * tn;
+            if (a.n > 0 && tiles + count > (uint64_t(1) << 31)) break;
+            RqTensor& T = a.t[a.n];
+            T.q = J.in.ptr;
+            T.q2 = J.out.ptr;
+            T.q_bs = J.in.bstride;
+            T.q_rs = J.in.rstride;
+            T.o_bs = J.out.bstride;
+            T.o_rs = J.out.rstride;
+            T.s = static_cast<const float*>(J.scale_in);
+            T.s2 = static_cast<float*>(J.scale_out);
+            T.rows = (int)J.in.rows;
+            T.cols = (int)J.in.cols;
+            T.tile_begin = tiles;
+            T.tiles_n = make_fastdiv(tn);
+            T.tiles_mn = make_fastdiv(tm * tn);
+            tiles += (uint32_t)count;
+        }
+        j0 += a.n;
+        a.total_tiles = tiles;
+        if (tiles == 0) continue;
+        fp8_requant_fp8_kernel<<<persistent_grid(tiles, 3), kThreads, 0, st>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+namespace {
+
+bool aligned16(const View& v) {
+    return (uintptr_t)v.ptr % 16 == 0 && v.rstride % 16 == 0 && (v.batch <= 1 || v.bstride % 16 == 0);
+}
+
+cudaError_t launch_mx8(const RequantJob& J, cudaStream_t st) {
+    const View& q = J.in;
+    const View& q2 = J.out;
     MxArgs a;
     a.q = q.ptr;
     a.q2 = q2.ptr;
@@ -221,8 +374,8 @@ cudaError_t launch_fp8_requant_mxfp8(const View& q, const float* s, const View& 
     a.q_rs = q.rstride;
     a.o_bs = q2.bstride;
     a.o_rs = q2.rstride;
-    a.s = s;
-    a.e = e;
+    a.s = static_cast<const float*>(J.scale_in);
+    a.e = static_cast<uint8_t*>(J.scale_out);
     a.chunks = (uint32_t)(q.batch * q.rows * (q.cols / 8));
     a.tm = (uint32_t)((q.rows + kTile - 1) / kTile);
     a.tn = (uint32_t)((q.cols + kTile - 1) / kTile);
@@ -234,6 +387,60 @@ cudaError_t launch_fp8_requant_mxfp8(const View& q, const float* s, const View& 
     const int grid = persistent_grid((a.chunks + kThreads * kUnroll - 1) / (kThreads * kUnroll), 8);
     fp8_requant_mxfp8_kernel<<<grid, kThreads, 0, st>>>(a);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fp8_requant_mxfp8(const RequantJob* jobs, int n, cudaStream_t st) {
+    bool all16 = true;
+    for (int i = 0; i < n; ++i) all16 = all16 && aligned16(jobs[i].in) && aligned16(jobs[i].out);
+    if (!all16) {   // 8-byte code rows: one launch per tensor with 8-code chunks
+        for (int i = 0; i < n; ++i) {
+            cudaError_t e = launch_mx8(jobs[i], st);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
+    const uint64_t kMaxSlots = uint64_t(1) << 31;
+    for (int j0 = 0; j0 < n;) {
+        Mx16Args a;
+        a.n = 0;
+        uint32_t slots = 0;
+        for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
+            const RequantJob& J = jobs[j0 + a.n];
+            const View& q = J.in;
+            const View& q2 = J.out;
+            const uint64_t chunks = (uint64_t)(q.batch * q.rows * (q.cols / 16));
+            const uint64_t padded = (chunks + kSpan - 1) / kSpan * kSpan;
+            if (a.n > 0 && slots + padded > kMaxSlots) break;
+            Mx16Tensor& T = a.t[a.n];
+            T.q = q.ptr;
+            T.q2 = q2.ptr;
+            T.q_bs = q.bstride;
+            T.q_rs = q.rstride;
+            T.o_bs = q2.bstride;
+            T.o_rs = q2.rstride;
+            T.s = static_cast<const float*>(J.scale_in);
+            T.e = static_cast<uint8_t*>(J.scale_out);
+            T.chunks = (uint32_t)chunks;
+            T.slot_begin = slots;
+            T.tm = (uint32_t)((q.rows + kTile - 1) / kTile);
+            T.tn = (uint32_t)((q.cols + kTile - 1) / kTile);
+            T.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, q.cols / 16));
+            T.rows = make_fastdiv((uint32_t)std::max<int64_t>(1, q.rows));
+            T.dense = q.rstride == q.cols && q2.rstride == q2.cols &&
+                      (q.batch == 1 || (q.bstride == q.rows * q.cols && q2.bstride == q2.rows * q2.cols));
+            slots += (uint32_t)padded;
+        }
+        j0 += a.n;
+        a.total_slots = slots;
+        if (slots == 0) continue;
+        const int grid = persistent_grid((slots + kThreads * kUnroll - 1) / (kThreads * kUnroll), 8);
+        fp8_requant_mxfp8_16_kernel<<<grid, kThreads, 0, st>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace pwq

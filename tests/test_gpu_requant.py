@@ -167,3 +167,31 @@ def test_fp8_to_nvfp4_grouped_single_pass(P):
             assert np.array_equal(u8(sb[g][i]), out[i][1]), (g, i)
     torch.cuda.synchronize()
     assert P.device_error() == 0
+
+
+def test_fp8_to_fp8_and_mxfp8_grouped(P):
+    # 20 tensors (two launches of 16), ragged and batched; the MXFP8 list is
+    # run twice: 16-byte aligned rows (grouped 16-code kernel) and with one
+    # member on 8-byte row strides (per-tensor fallback)
+    shapes = [(1 + 37 * i, 32 * (1 + i % 5)) for i in range(18)] + [(2, 130, 256), (129, 160)]
+    ms = [codes_and_scales(sh, seed=60 + i, raw=(i % 3 == 0)) for i, sh in enumerate(shapes)]
+    qs = [to_gpu_codes(m[0]) for m in ms]
+    ss = [torch.from_numpy(m[1]).to(DEV) for m in ms]
+    rq, rs = P.fp8_block_requant_grouped(qs, ss)
+    mq, me = P.fp8_block_requant_mxfp8_grouped(qs, ss)
+    for i, (q, s) in enumerate(ms):
+        oq, os_ = O.fp8_block_requant(q, s)
+        assert np.array_equal(u8(rq[i]), oq) and np.array_equal(f32bits(rs[i]), os_.view(np.uint32)), i
+        oq, oe = O.fp8_block_requant_mxfp8(q, s)
+        assert np.array_equal(u8(mq[i]), oq) and np.array_equal(u8(me[i]), oe), i
+    qs8 = list(qs)
+    qs8[5] = to_gpu_codes(ms[5][0], pad=8)
+    mq8, me8 = P.fp8_block_requant_mxfp8_grouped(qs8, ss)
+    for i in range(len(ms)):
+        assert torch.equal(mq8[i].view(torch.uint8), mq[i].view(torch.uint8)) and torch.equal(me8[i], me[i]), i
+    # in place, grouped
+    qi = [q.clone() for q in qs]
+    si = [s.clone() for s in ss]
+    P.fp8_block_requant_grouped(qi, si, inplace=True)
+    for i in range(len(ms)):
+        assert torch.equal(qi[i].view(torch.uint8), rq[i].view(torch.uint8)) and torch.equal(si[i], rs[i]), i
