@@ -285,3 +285,77 @@ def fp8_block_requant_nvfp4(qs, ss):
         pk, sb = np.stack(pk), np.stack(sb)
         out.append((pk if batched else pk[0], sb if batched else sb[0]))
     return A, out, gs
+
+
+# ---------------------------------------------------------------- W4A4 activation observers
+#
+# verl NVFP4 QAT article, 2.2 and 3.1: in W4A4 mode the activation has its own
+# global scale (input_global_scale), kept by an activation observer named
+# static_minmax (default), memoryless_minmax or minmax.  The names are all
+# the pages give; the readings (stated with the library's C ABI) are:
+#   state (lo, hi): binary32 minimum and maximum of the values observed,
+#     empty = (+inf, -inf); the order on values is the numeric one with
+#     -0 < +0, so the extremes of a tensor are unique;
+#   memoryless_minmax: (lo, hi) = (min x, max x) of this tensor;
+#   static_minmax:     (lo, hi) = (min(lo, min x), max(hi, max x));
+#   minmax:            moving average with constant c: an empty state takes
+#     (min x, max x); otherwise lo = fl(fl(fl(1 - c) * lo) + fl(c * min x)),
+#     hi likewise;
+# then A = max(|lo|, |hi|) and input_global_scale = fl(A / 2688) (as the
+# weight global scale).  The state is updated before the tensor is
+# quantised with A.
+
+MEMORYLESS_MINMAX, STATIC_MINMAX, MINMAX = 0, 1, 2
+
+
+def _bf16_key(bits):
+    """BF16 bits -> unsigned keys in the order of the values (-0 < +0)."""
+    b = np.asarray(bits, np.uint32)
+    return np.where(b & 0x8000, (~b) & 0xFFFF, b | 0x8000)
+
+
+def _key_bf16(key):
+    k = int(key)
+    return (k & 0x7FFF) if k & 0x8000 else ((~k) & 0xFFFF)
+
+
+def activation_minmax(x_bits):
+    """(min, max) of a BF16 tensor in the value order with -0 < +0."""
+    k = _bf16_key(np.asarray(x_bits, np.uint16).ravel())
+    lo = np.float32(bf16_to_f32(np.array([_key_bf16(k.min())], np.uint16))[0])
+    hi = np.float32(bf16_to_f32(np.array([_key_bf16(k.max())], np.uint16))[0])
+    return lo, hi
+
+
+def _minf(a, b):
+    # value order with -0 < +0 on binary32
+    if a == b:
+        return a if np.signbit(a) else b
+    return a if a < b else b
+
+
+def _maxf(a, b):
+    if a == b:
+        return b if np.signbit(a) else a
+    return a if a > b else b
+
+
+def observe(state, x_bits, kind, c=np.float32(0.01)):
+    """One observer step.  state: float32 [2] (lo, hi).  Returns (new state,
+    A, input_global_scale)."""
+    lo, hi = np.float32(state[0]), np.float32(state[1])
+    mn, mx = activation_minmax(x_bits)
+    empty = lo > hi
+    if kind == MEMORYLESS_MINMAX or (kind == MINMAX and empty):
+        lo, hi = mn, mx
+    elif kind == STATIC_MINMAX:
+        lo, hi = _minf(lo, mn), _maxf(hi, mx)
+    elif kind == MINMAX:
+        c = np.float32(c)
+        w = np.float32(np.float32(1) - c)
+        lo = np.float32(np.float32(w * lo) + np.float32(c * mn))
+        hi = np.float32(np.float32(w * hi) + np.float32(c * mx))
+    else:
+        raise ValueError("observer kind")
+    A = np.float32(max(abs(lo), abs(hi)))
+    return np.array([lo, hi], np.float32), A, np.float32(nvfp4_global_scale(A))
