@@ -381,6 +381,44 @@ pwq_status fp8_block_requant_nvfp4_grouped(int n_groups, const int* group_sizes,
                                            size_t workspace_bytes, pwq_stream_t stream);
 
 /* ===================================================================== */
+/* W4A4 activation observers                                              */
+/* ===================================================================== */
+
+/* verl NVFP4 QAT article, 2.2 and 3.1: in W4A4 mode each activation has its
+ * own NVFP4 global scale (input_global_scale), kept by an activation observer
+ * named static_minmax (the default), memoryless_minmax or minmax.  The pages
+ * give only the names; this library reads them as follows.  The observer
+ * state is two binary32 values (lo, hi), the minimum and maximum of the
+ * values observed so far, numerically ordered with -0 < +0; an empty state
+ * is (+inf, -inf) (any lo > hi), which the caller writes once.  One step on
+ * a tensor x with extremes (mn, mx):
+ *   PWQ_OBSERVER_MEMORYLESS_MINMAX  (lo, hi) = (mn, mx);
+ *   PWQ_OBSERVER_STATIC_MINMAX      (lo, hi) = (min(lo, mn), max(hi, mx));
+ *   PWQ_OBSERVER_MINMAX             moving average with constant c in [0, 1]:
+ *       an empty state takes (mn, mx), otherwise
+ *       lo = fl(fl(fl(1 - c) * lo) + fl(c * mn)) and hi alike;
+ * then A = max(|lo|, |hi|) and input_global_scale = fl(A / 2688), as the
+ * weight global scale.  Quantising the activation is then nvfp4_fake_quant
+ * (or nvfp4_quant) with amax_in = A: the step observes, then quantises. */
+#define PWQ_OBSERVER_MEMORYLESS_MINMAX 0
+#define PWQ_OBSERVER_STATIC_MINMAX 1
+#define PWQ_OBSERVER_MINMAX 2
+
+/* Bytes of workspace nvfp4_activation_observe needs (256). */
+size_t nvfp4_observe_workspace_size(void);
+
+/* nvfp4_activation_observe: one observer step over every element of x
+ * (BF16 [B][M][N], N % 16 == 0; the whole tensor is one observation).
+ * state: device float[2], read and written.  amax_out, input_global_scale:
+ * device float[1] each, nullable.  averaging_constant is used by
+ * PWQ_OBSERVER_MINMAX only (PWQ_ERR_ARG outside [0, 1]).  An empty x leaves
+ * everything unchanged.  Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _STRIDE,
+ * _OVERLAP, _WORKSPACE, _ARG, _CUDA. */
+pwq_status nvfp4_activation_observe(const pwq_tensor* x, int observer, float averaging_constant, float* state,
+                                    float* amax_out, float* input_global_scale, void* workspace,
+                                    size_t workspace_bytes, pwq_stream_t stream);
+
+/* ===================================================================== */
 /* Diagnostics                                                            */
 /* ===================================================================== */
 

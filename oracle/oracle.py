@@ -359,3 +359,5 @@ def observe(state, x_bits, kind, c=np.float32(0.01)):
         raise ValueError("observer kind")
     A = np.float32(max(abs(lo), abs(hi)))
     return np.array([lo, hi], np.float32), A, np.float32(nvfp4_global_scale(A))
+
+OBSERVERS_BY_NAME = {"memoryless_minmax": MEMORYLESS_MINMAX, "static_minmax": STATIC_MINMAX, "minmax": MINMAX}

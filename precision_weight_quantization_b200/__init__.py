@@ -28,6 +28,7 @@ __all__ = [
     "mxfp8_quant_grouped", "mxfp8_dequant_grouped", "nvfp4_dequant_grouped", "nvfp4_quant_grouped",
     "nvfp4_fake_quant_grouped", "fp8_block_requant", "fp8_block_requant_mxfp8", "fp8_block_requant_nvfp4",
     "fp8_block_requant_nvfp4_grouped", "fp8_block_requant_grouped", "fp8_block_requant_mxfp8_grouped",
+    "NVFP4ActivationObserver", "nvfp4_w4a4_fake_quant_ste", "OBSERVERS",
 ]
 
 _CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
@@ -540,6 +541,70 @@ def fp8_block_requant_nvfp4_grouped(groups, scales, out=None, sb=None, global_sc
                                               ws.data_ptr(), ws.numel(), _stream(flat[0])),
           "fp8_block_requant_nvfp4_grouped")
     return out, sb, global_scale
+
+
+# ---------------------------------------------------------------- W4A4 activation observers
+
+OBSERVERS = {"memoryless_minmax": 0, "static_minmax": 1, "minmax": 2}
+
+
+class NVFP4ActivationObserver:
+    """An activation observer of W4A4 NVFP4 fake-quantisation (verl NVFP4 QAT
+    article 2.2 / 3.1): keeps the running extremes (lo, hi) of the activations
+    it sees on the device and gives the activation's amax and
+    input_global_scale = fl(amax / 2688).  kind: "static_minmax" (default),
+    "memoryless_minmax" or "minmax" (moving average with constant
+    `averaging_constant`); the exact rules are those of nvfp4_activation_observe
+    in include/pwq.h.  No host synchronisation."""
+
+    def __init__(self, kind: str = "static_minmax", averaging_constant: float = 0.01, device="cuda"):
+        if kind not in OBSERVERS:
+            raise ValueError("observer kind must be one of %s" % sorted(OBSERVERS))
+        self.kind = kind
+        self.averaging_constant = float(averaging_constant)
+        self.state = torch.tensor([float("inf"), float("-inf")], dtype=torch.float32, device=device)
+        self.amax = torch.zeros(1, dtype=torch.float32, device=device)
+        self.input_global_scale = torch.zeros(1, dtype=torch.float32, device=device)
+        self._ws = torch.empty(int(lib.nvfp4_observe_workspace_size()), dtype=torch.uint8, device=device)
+
+    def reset(self):
+        self.state.copy_(torch.tensor([float("inf"), float("-inf")], dtype=torch.float32))
+
+    def observe(self, x: torch.Tensor) -> torch.Tensor:
+        """One observer step over x (BF16, last dim % 16 == 0); returns the
+        amax tensor (float32 [1], on the device)."""
+        _check_dtype(x, (torch.bfloat16,), "x")
+        dx = _desc(x, "x")
+        check(lib.nvfp4_activation_observe(ctypes.byref(dx), OBSERVERS[self.kind], self.averaging_constant,
+                                           self.state.data_ptr(), self.amax.data_ptr(),
+                                           self.input_global_scale.data_ptr(), self._ws.data_ptr(),
+                                           self._ws.numel(), _stream(x)), "nvfp4_activation_observe")
+        return self.amax
+
+    def fake_quant(self, x: torch.Tensor, out=None) -> torch.Tensor:
+        """Observe x, then NVFP4 fake-quantise it with the observed amax (one
+        global scale for the whole tensor: a 3-D x gets the amax once per
+        batch index, as nvfp4_fake_quant expects amax[B])."""
+        amax = self.observe(x)
+        if x.dim() == 3 and x.shape[0] != 1:
+            amax = amax.expand(x.shape[0]).contiguous()
+        return nvfp4_fake_quant(x, amax=amax, out=out)
+
+
+class _W4A4STE(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, observer):
+        return observer.fake_quant(x)
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        return grad_out, None
+
+
+def nvfp4_w4a4_fake_quant_ste(x: torch.Tensor, observer: NVFP4ActivationObserver) -> torch.Tensor:
+    """W4A4 activation fake-quantisation with the straight-through backward
+    (the gradient passes unchanged, verl NVFP4 QAT article 2.3)."""
+    return _W4A4STE.apply(x, observer)
 
 
 def build_info() -> str:

@@ -68,6 +68,8 @@ _SIG = {
     "fp8_block_requant_nvfp4": (_S, [_T, _PP, ctypes.c_int, _T, _PP, _P, _P, _P, ctypes.c_size_t, _P]),
     "fp8_block_requant_nvfp4_workspace_size_grouped": (ctypes.c_size_t, [ctypes.c_int, _IP, _T]),
     "fp8_block_requant_nvfp4_grouped": (_S, [ctypes.c_int, _IP, _T, _PP, _T, _PP, _PP, _P, ctypes.c_size_t, _P]),
+    "nvfp4_observe_workspace_size": (ctypes.c_size_t, []),
+    "nvfp4_activation_observe": (_S, [_T, ctypes.c_int, ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "pwq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "pwq_last_error_detail": (ctypes.c_char_p, []),
     "pwq_build_info": (ctypes.c_char_p, []),

@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
                 // block scale sb = e4m3(fl(amax_b / fl(6 gs)))
                 const float amax_b = __uint_as_float(m << 16);
                 const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
-                const uint32_t sb = e4m3x2(ratio, 0.0f) & 0xffu;
+                const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0 (a NaN ratio, outside the contract, stays in the table)
                 const float4 e = tab.e[sb];
                 const uint32_t codes = codes_half(v[u], e.x, e.y);
                 if (j < S.chunks) {
@@ -549,7 +549,7 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
             ratio = div_fast(amax_b, six_gs, r6);
         else
             ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
-        const uint32_t sb = e4m3x2(ratio, 0.0f) & 0xffu;
+        const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0 (a NaN ratio, outside the contract, stays in the table)
         const float4 e = tab.e[sb];
         uint32_t codes;
         if (kFast) {

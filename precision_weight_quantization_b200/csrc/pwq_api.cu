@@ -836,6 +836,37 @@ pwq_status fp8_block_requant_nvfp4_grouped(int n_groups, const int* group_sizes,
                           workspace_bytes, stream);
 }
 
+// ------------------------------------------------------------------ W4A4 activation observers
+
+size_t nvfp4_observe_workspace_size(void) { return 256; }
+
+pwq_status nvfp4_activation_observe(const pwq_tensor* x, int observer, float averaging_constant, float* state,
+                                    float* amax_out, float* input_global_scale, void* workspace,
+                                    size_t workspace_bytes, pwq_stream_t stream) {
+    View vx;
+    Extent ex;
+    pwq_status st = check_tensor(x, Kind::kBF16, &vx, &ex, "x");
+    if (st != PWQ_OK) return st;
+    if (x->cols % 16 != 0) return fail(PWQ_ERR_SHAPE, "cols % 16 != 0");
+    if (observer < PWQ_OBSERVER_MEMORYLESS_MINMAX || observer > PWQ_OBSERVER_MINMAX)
+        return fail(PWQ_ERR_ARG, "observer kind");
+    if (observer == PWQ_OBSERVER_MINMAX && !(averaging_constant >= 0.0f && averaging_constant <= 1.0f))
+        return fail(PWQ_ERR_ARG, "averaging_constant outside [0, 1]");
+    if (!state) return fail(PWQ_ERR_NULL, "state");
+    if ((uintptr_t)state % 4 != 0 || ((uintptr_t)amax_out % 4) != 0 || ((uintptr_t)input_global_scale % 4) != 0)
+        return fail(PWQ_ERR_ALIGN, "state / amax_out / input_global_scale");
+    if (empty(x)) return PWQ_OK;
+    if (!workspace || (uintptr_t)workspace % 4 != 0 || workspace_bytes < nvfp4_observe_workspace_size())
+        return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
+    std::vector<Extent> outs = {extent_of(state, 8), extent_of(workspace, nvfp4_observe_workspace_size())};
+    if (amax_out) outs.push_back(extent_of(amax_out, 4));
+    if (input_global_scale) outs.push_back(extent_of(input_global_scale, 4));
+    if ((st = check_overlaps(&ex, 1, outs.data(), (int)outs.size())) != PWQ_OK) return st;
+    return from_cuda(pwq::launch_activation_observe(vx, observer, averaging_constant, state, amax_out,
+                                                    input_global_scale, static_cast<uint32_t*>(workspace),
+                                                    (cudaStream_t)stream));
+}
+
 // ------------------------------------------------------------------ self-tests
 
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream) {

@@ -94,6 +94,12 @@ cudaError_t static_amax_scratch(uint32_t** ptr);
 cudaError_t read_and_clear_device_error(uint32_t* code);
 cudaError_t read_and_clear_flow_error(uint32_t* code);
 
+// W4A4 activation observer step over x (BF16): state (lo, hi) updated per
+// `kind` (0 memoryless, 1 static, 2 moving average with constant c),
+// amax_out / gs_out (nullable) = A and fl(A / 2688).  words: 2 scratch words.
+cudaError_t launch_activation_observe(const View& x, int kind, float c, float* state, float* amax_out,
+                                      float* gs_out, uint32_t* words, cudaStream_t s);
+
 cudaError_t launch_selftest_division(int which, unsigned long long* counts, cudaStream_t s);
 cudaError_t launch_selftest_codecs(uint32_t first, uint32_t count, uint8_t* e4m3, uint8_t* e2m1,
                                    uint16_t* bf16, cudaStream_t s);

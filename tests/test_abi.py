@@ -194,3 +194,23 @@ def test_requant_validation_without_gpu():
     # empty input: a no-op that succeeds
     qe = T(L, None, 1, 0, 512, 0, 512)
     assert lib.fp8_block_requant(by(qe), None, by(qe), None, None) == L.PWQ_OK
+
+
+def test_observer_validation_without_gpu():
+    L = _lib()
+    lib = L.lib
+    by = ctypes.byref
+    base = 1 << 40
+    x = T(L, base, 1, 64, 256, 64 * 256, 256)
+    st = base + (1 << 30)
+    ws = base + (2 << 30)
+    assert lib.nvfp4_observe_workspace_size() == 256
+    assert lib.nvfp4_activation_observe(by(x), 3, 0.0, st, None, None, ws, 256, None) == L.PWQ_ERR_ARG
+    assert lib.nvfp4_activation_observe(by(x), 2, 1.5, st, None, None, ws, 256, None) == L.PWQ_ERR_ARG
+    assert lib.nvfp4_activation_observe(by(x), 2, float("nan"), st, None, None, ws, 256, None) == L.PWQ_ERR_ARG
+    assert lib.nvfp4_activation_observe(by(x), 1, 0.0, None, None, None, ws, 256, None) == L.PWQ_ERR_NULL
+    assert lib.nvfp4_activation_observe(by(x), 1, 0.0, st + 2, None, None, ws, 256, None) == L.PWQ_ERR_ALIGN
+    assert lib.nvfp4_activation_observe(by(x), 1, 0.0, st, None, None, None, 0, None) == L.PWQ_ERR_WORKSPACE
+    assert lib.nvfp4_activation_observe(by(x), 1, 0.0, base + 64, None, None, ws, 256, None) == L.PWQ_ERR_OVERLAP
+    x24 = T(L, base, 1, 4, 24, 4 * 32, 32)
+    assert lib.nvfp4_activation_observe(by(x24), 1, 0.0, st, None, None, ws, 256, None) == L.PWQ_ERR_SHAPE
