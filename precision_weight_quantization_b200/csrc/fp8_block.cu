@@ -258,6 +258,130 @@ __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const __gri
     }
 }
 
+// FP8 block-wise -> FP8 block-wise re-quantisation (the composition
+// fp8_block_quant(fp8_block_dequant(q, s)), see requant.cu) with the code
+// tiles staged by TMA like the quantiser's BF16 tiles: 16 KB per tile, a
+// ring of kRqStages buffers, 3 CTAs per SM.  Used when every input code
+// tensor has 16-byte aligned rows (a TMA stride rule); the tile of old
+// scales is read before the CTA's barrier and the new scale written after
+// it, so in-place use is safe.
+constexpr int kRqStages = 4;
+constexpr int kRqTileBytes = kTile * kTile;   // E4M3
+
+struct RequantTmaArgs {
+    CUtensorMap tmap[kMaxLaunchTensors];   // input codes
+    TileTensor t[kMaxLaunchTensors];       // q = output codes, scale = new scales
+    const float* s_in[kMaxLaunchTensors];
+    int n;
+    uint32_t total_tiles;
+};
+
+__global__ void __launch_bounds__(kThreads, 3)
+fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
+    extern __shared__ unsigned char smem[];
+    __shared__ __align__(8) uint64_t bars[kRqStages];
+    __shared__ TileLoc meta[kRqStages];
+    __shared__ uint32_t red[2][kThreads / 32];
+
+    const uint32_t tid = threadIdx.x;
+    const uint32_t pad = (1024u - (smem_addr(smem) & 1023u)) & 1023u;
+    unsigned char* ring = smem + pad;
+    const uint32_t smem0 = smem_addr(ring);
+    if (tid == 0) {
+        for (int s = 0; s < kRqStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto issue = [&](uint32_t t, uint32_t s) {
+        const TileLoc L = locate(a, t);
+        meta[s] = L;
+        const uint32_t bar = smem_addr(&bars[s]);
+        mbar_arrive_expect_tx(bar, kRqTileBytes);
+        tma_load_3d(smem0 + s * kRqTileBytes, &a.tmap[L.i], bar, L.tn * kTile, L.tm * kTile, L.b);
+    };
+
+    const uint32_t first = blockIdx.x, step = gridDim.x;
+    if (tid == 0) {
+        for (int s = 0; s < kRqStages; ++s) {
+            const uint32_t t = first + (uint32_t)s * step;
+            if (t < a.total_tiles) issue(t, (uint32_t)s);
+        }
+    }
+    const int ccol = (int)(tid & 15u) * 8;
+    const int row0 = (int)(tid >> 4);
+
+    uint32_t it = 0;
+    for (uint32_t t = first; t < a.total_tiles; t += step, ++it) {
+        const uint32_t s = it % kRqStages;
+        const uint32_t parity = (it / kRqStages) & 1u;
+        const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity, kWaitLimitNs);
+        const unsigned char* buf = ring + s * kRqTileBytes;
+        const TileLoc L = meta[s];
+        const float sc = a.s_in[L.i][L.lt];
+        uint2 v[kChunksPerThread];
+        uint32_t m = 0u;
+#pragma unroll
+        for (int j = 0; j < kChunksPerThread; ++j) {
+            v[j] = make_uint2(0u, 0u);
+            if (ok) v[j] = *reinterpret_cast<const uint2*>(buf + (row0 + 16 * j) * kTile + ccol);
+            m = max(m, e4m3_maxmag8(v[j]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((tid & 31u) == 0u) red[it & 1u][tid >> 5] = m;
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_device_error, kErrTmaTimeout);
+                for (uint32_t k = 0; k < (uint32_t)kRqStages; ++k) {
+                    if (t + k * step < a.total_tiles)
+                        (void)mbar_wait_bounded(smem_addr(&bars[(it + k) % kRqStages]),
+                                                ((it + k) / kRqStages) & 1u, kWaitLimitNs);
+                }
+            }
+            return;
+        }
+        if (tid == 0) {
+            const uint32_t tn = t + (uint32_t)kRqStages * step;
+            if (tn < a.total_tiles) issue(tn, s);
+        }
+        uint32_t mc = red[it & 1u][0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) mc = max(mc, red[it & 1u][w]);
+        const float s2 = fp8_tile_scale(__uint_as_float(fp8_amax_bits16(mc, sc) << 16));
+        const bool fast = div_fast_ok(s2);   // CTA-uniform
+        const float r2 = fast ? __frcp_rn(s2) : 0.0f;
+        uint2 out[kChunksPerThread];
+#pragma unroll
+        for (int j = 0; j < kChunksPerThread; ++j)
+            out[j] = fast ? fp8_requant8<true>(v[j], sc, s2, r2) : fp8_requant8<false>(v[j], sc, s2, r2);
+
+        const TileTensor& T = a.t[L.i];
+        if (tid == 0) T.scale[L.lt] = s2;
+        const int rows_here = min(kTile, T.rows - L.tm * kTile);
+        const int cols_here = min(kTile, T.cols - L.tn * kTile);
+        char* qtile = T.q + (int64_t)L.b * T.q_bs + (int64_t)L.tm * kTile * T.q_rs + (int64_t)L.tn * kTile;
+        if (rows_here == kTile && cols_here == kTile) {
+#pragma unroll
+            for (int j = 0; j < kChunksPerThread; ++j)
+                st_v2(qtile + (int64_t)(row0 + 16 * j) * T.q_rs + ccol, out[j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < kChunksPerThread; ++j) {
+                const int r = row0 + 16 * j;
+                if (r >= rows_here || ccol >= cols_here) continue;
+                char* dst = qtile + (int64_t)r * T.q_rs + ccol;
+                if (ccol + 8 <= cols_here) {
+                    st_v2(dst, out[j]);
+                } else {
+                    for (int e = 0; e < cols_here - ccol; ++e)
+                        dst[e] = (char)((e < 4 ? out[j].x >> (8 * e) : out[j].y >> (8 * (e - 4))) & 0xffu);
+                }
+            }
+        }
+    }
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
 // link-time dependency on libcuda).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -357,6 +481,74 @@ cudaError_t launch_fp8_block_dequant(const Job* jobs, int n, cudaStream_t s) {
         if (tiles == 0) continue;
         const int grid = persistent_grid(tiles, 8);
         fp8_block_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+// FP8 -> FP8 re-quantisation through TMA-staged tiles; false (nothing
+// launched) when a tensor's code rows are not 16-byte aligned.
+bool fp8_requant_tma_ok(const RequantJob* jobs, int n) {
+    for (int i = 0; i < n; ++i) {
+        const View& q = jobs[i].in;
+        if ((uintptr_t)q.ptr % 16 != 0 || q.rstride % 16 != 0 || (q.batch > 1 && q.bstride % 16 != 0)) return false;
+    }
+    return encode_tiled_fn() != nullptr;
+}
+
+cudaError_t launch_fp8_requant_tma(const RequantJob* jobs, int n, cudaStream_t s) {
+    EncodeTiledFn encode = encode_tiled_fn();
+    if (!encode) return cudaErrorNotSupported;
+    const size_t smem = (size_t)kRqStages * kRqTileBytes + 1024;
+    static int configured[64] = {0};
+    const int dev = current_device();
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(fp8_requant_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        configured[dev] = 1;
+    }
+    for (int j0 = 0; j0 < n;) {
+        RequantTmaArgs a;
+        a.n = 0;
+        uint32_t tiles = 0;
+        for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
+            const RequantJob& J = jobs[j0 + a.n];
+            const View& q = J.in;
+            const uint32_t tm = (uint32_t)((q.rows + kTile - 1) / kTile);
+            const uint32_t tn = (uint32_t)((q.cols + kTile - 1) / kTile);
+            const uint64_t count = (uint64_t)q.batch * tm * tn;
+            if (a.n > 0 && tiles + count > (uint64_t(1) << 31)) break;
+            const cuuint64_t dims[3] = {(cuuint64_t)q.cols, (cuuint64_t)q.rows, (cuuint64_t)q.batch};
+            const cuuint64_t strides[2] = {(cuuint64_t)q.rstride,
+                                           (cuuint64_t)(q.batch > 1 ? q.bstride : q.rows * q.rstride)};
+            const cuuint32_t box[3] = {kTile, kTile, 1};
+            const cuuint32_t estr[3] = {1, 1, 1};
+            CUresult cr = encode(&a.tmap[a.n], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q.ptr, dims, strides, box, estr,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+            TileTensor& T = a.t[a.n];
+            T.q = J.out.ptr;
+            T.y = nullptr;
+            T.q_bs = J.out.bstride;
+            T.q_rs = J.out.rstride;
+            T.y_bs = T.y_rs = 0;
+            T.scale = static_cast<float*>(J.scale_out);
+            T.rows = (int)q.rows;
+            T.cols = (int)q.cols;
+            T.tile_begin = tiles;
+            T.tiles_n = make_fastdiv(tn);
+            T.tiles_mn = make_fastdiv(tm * tn);
+            a.s_in[a.n] = static_cast<const float*>(J.scale_in);
+            tiles += (uint32_t)count;
+        }
+        j0 += a.n;
+        a.total_tiles = tiles;
+        if (tiles == 0) continue;
+        const int grid = (int)std::min<int64_t>(tiles, (int64_t)sm_count(dev) * 3);
+        fp8_requant_tma_kernel<<<grid, kThreads, smem, s>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -246,6 +246,17 @@ __device__ __forceinline__ void quotients8(uint4 v, float s, float r, float q[8]
     }
 }
 
+// FP8 block-wise re-quantisation of 8 codes: the codes of the dequantised
+// values y = bf16(fl(dec(q) * s)) against the new tile scale s2 (r2 =
+// RN(1/s2) on the reciprocal path, kFast).
+template <bool kFast>
+__device__ __forceinline__ uint2 fp8_requant8(uint2 c, float s, float s2, float r2) {
+    const uint4 y = fp8_dequant8(c, s);
+    float q[8];
+    quotients8<kFast>(y, s2, r2, q);
+    return make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
+}
+
 // ---------------------------------------------------------------- UE8M0
 
 // e = min{k : amax <= 448 * 2^k} from the BF16 magnitude bits of amax,

@@ -82,6 +82,10 @@ struct RequantJob {
     void* scale_out;        // FP8: FP32 [B][TM][TN]; MXFP8: uint8 [B][M][N/32]
 };
 cudaError_t launch_fp8_requant_fp8(const RequantJob* jobs, int n, cudaStream_t st);
+// The TMA-staged form of the FP8 -> FP8 re-quantisation (fp8_block.cu),
+// usable when every input code tensor has 16-byte aligned rows.
+bool fp8_requant_tma_ok(const RequantJob* jobs, int n);
+cudaError_t launch_fp8_requant_tma(const RequantJob* jobs, int n, cudaStream_t st);
 cudaError_t launch_fp8_requant_mxfp8(const RequantJob* jobs, int n, cudaStream_t st);
 
 // Device address (on the current device) of the file-scope group-amax

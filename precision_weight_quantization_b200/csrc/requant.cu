@@ -103,14 +103,6 @@ __device__ __forceinline__ void load_tile(const TileWork& w, int row0, int ccol,
     }
 }
 
-template <bool kFast>
-__device__ __forceinline__ uint2 requant8(uint2 c, float s, float s2, float r2) {
-    const uint4 y = fp8_dequant8(c, s);
-    float q[8];
-    quotients8<kFast>(y, s2, r2, q);
-    return make_uint2(e4m3x4(q[0], q[1], q[2], q[3]), e4m3x4(q[4], q[5], q[6], q[7]));
-}
-
 // Persistent CTAs over the tiles of all tensors of the launch; each thread
 // holds the codes of the next tile (loads in flight) while it re-encodes the
 // current one.
@@ -148,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 3) fp8_requant_fp8_kernel(const __gr
         const float r2 = fast ? __frcp_rn(s2) : 0.0f;
         uint2 o[kChunks];
 #pragma unroll
-        for (int j = 0; j < kChunks; ++j) o[j] = fast ? requant8<true>(v[j], w.s, s2, r2) : requant8<false>(v[j], w.s, s2, r2);
+        for (int j = 0; j < kChunks; ++j) o[j] = fast ? fp8_requant8<true>(v[j], w.s, s2, r2) : fp8_requant8<false>(v[j], w.s, s2, r2);
         if (w.rows_here == kTile && w.cols_here == kTile) {
 #pragma unroll
             for (int j = 0; j < kChunks; ++j) st_v2(w.ot + (int64_t)(row0 + kRowsPerPass * j) * w.o_rs + ccol, o[j]);
@@ -322,6 +314,7 @@ __global__ void __launch_bounds__(kThreads) fp8_requant_mxfp8_16_kernel(const __
 }  // namespace
 
 cudaError_t launch_fp8_requant_fp8(const RequantJob* jobs, int n, cudaStream_t st) {
+    if (fp8_requant_tma_ok(jobs, n)) return launch_fp8_requant_tma(jobs, n, st);
     for (int j0 = 0; j0 < n;) {
         TileArgs a;
         a.n = 0;
