@@ -71,19 +71,6 @@ __device__ __forceinline__ float2 e4m3x2_decode(uint32_t codes16) {
 // One E4M3 code -> exact binary32 value.
 __device__ __forceinline__ float e4m3_decode(uint32_t code) { return e4m3x2_decode(code & 0xffu).x; }
 
-// FP8 block-wise dequantisation of 8 codes (code 0 in bits 0..7 of c.x):
-// BF16 bits of y = bf16(fl(dec(q) * s)), element 0 in the low half of .x.
-__device__ __forceinline__ uint4 fp8_dequant8(uint2 c, float s) {
-    uint32_t w[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const uint32_t pair = ((h < 2 ? c.x : c.y) >> (16 * (h & 1))) & 0xffffu;
-        const float2 f = e4m3x2_decode(pair);
-        w[h] = pack_bf16x2(__fmul_rn(f.x, s), __fmul_rn(f.y, s));
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 // Largest magnitude byte (bits 0..6) among 8 E4M3 codes; positive E4M3
 // codes order like their values.
 __device__ __forceinline__ uint32_t e4m3_maxmag8(uint2 c) {
@@ -193,6 +180,22 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
     uint64_t d;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
+}
+
+// FP8 block-wise dequantisation of 8 codes (code 0 in bits 0..7 of c.x):
+// BF16 bits of y = bf16(fl(dec(q) * s)), element 0 in the low half of .x.
+// The products are taken two at a time (f32x2).
+__device__ __forceinline__ uint4 fp8_dequant8(uint2 c, float s) {
+    const uint64_t s2 = f32x2(s, s);
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const uint32_t pair = ((h < 2 ? c.x : c.y) >> (16 * (h & 1))) & 0xffffu;
+        const float2 f = e4m3x2_decode(pair);
+        const float2 p = f32x2_split(mul_f32x2(f32x2(f.x, f.y), s2));
+        w[h] = pack_bf16x2(p.x, p.y);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // div_fast on the two BF16 values of a packed word w (low half first):
