@@ -20,7 +20,7 @@ namespace pwq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 2;
 constexpr uint32_t kSpan = 32u * kUnroll;   // chunks per warp span
 
 struct ChunkTensor {

@@ -31,7 +31,7 @@ namespace pwq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;
 constexpr int kMaxSib = 8;
 
 // One sibling of a group set, addressed per batch slab.  The source is BF16
