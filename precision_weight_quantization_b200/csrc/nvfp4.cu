@@ -6,7 +6,12 @@
 // siblings share the group's maximum amax), 3.3 (weight_scale_2 =
 // amax / (6.0 * 448.0)); "Low Precision RL", "Choose a precision" table.
 //
-// Two stream-ordered passes, no device-side waiting:
+// Quantise and fake-quantise run as one single-pass launch per call
+// (nvfp4_flow_kernel, described at its queue below): amax items and encode
+// items of every group of the call share one work queue, and an encode
+// item re-reads its data while it is still in L2.  Two stream-ordered
+// launches serve the calls whose amax is given (amax_in), the entry point
+// without allocation, and nvfp4_group_amax:
 //   1. amax: every CTA reduces a slice of one group to a max and publishes
 //      it with one atomicMax on the group's word (the float bit patterns of
 //      non-negative values order like unsigned integers);
@@ -15,6 +20,8 @@
 //      128-bit load each, amax combined with one shuffle).  It walks the
 //      tensor in the reverse order of pass 1 so that the most recently read
 //      data -- still in the 126 MB L2 -- is consumed first.
+// Every kernel also takes an FP8 block-wise source (E4M3 codes with tile
+// scales, dequantised in registers) for the re-quantisation calls.
 // Division: a group has at most 127 distinct code divisors d = fl(dec(sb) *
 // gs), so each CTA tabulates d and RN(1/d) for every block-scale code in
 // shared memory once; the block scale itself divides by fl(6 gs), whose
