@@ -76,11 +76,17 @@ PROFILES = {
 
 
 def source_sha256(kernel_file):
+    """sha256 of the code of a kernel file and the shared device header, with
+    comments and blank space left out (a comment edit is no kernel change)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in (kernel_file, "pwq_device.cuh"):
-        with open(os.path.join(ROOT, CSRC, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, CSRC, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("\n".join(line.strip() for line in text.splitlines() if line.strip()).encode())
     return h.hexdigest()
 
 

@@ -1,6 +1,5 @@
 """bench.py pieces that need no GPU: the reference arm's JSON line and the
 staleness rule of the recorded ncu traffic."""
-import hashlib
 import json
 import os
 import subprocess
@@ -30,24 +29,27 @@ def test_reference_arm_line():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
 
 
-def _fake_tree(tmp_path, kernel_src=b"kernel v1", traffic=123456789):
+def _fake_tree(tmp_path, monkeypatch, traffic=123456789):
     csrc = tmp_path / bench.CSRC
     csrc.mkdir(parents=True)
-    (csrc / "k.cu").write_bytes(kernel_src)
-    (csrc / "pwq_device.cuh").write_bytes(b"helpers")
-    sha = hashlib.sha256(b"kernel v1" + b"helpers").hexdigest()
+    (csrc / "k.cu").write_text("int kernel_v1;  // a comment\n")
+    (csrc / "pwq_device.cuh").write_text("/* helpers */ int helpers;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.source_sha256("k.cu")
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "k.md").write_text(
         "# k\n\n| metric | value |\n\ntraffic_bytes_per_launch: %d\nsource_sha256: `%s` (note)\n" % (traffic, sha))
 
 
 def test_recorded_traffic_fresh_and_stale(tmp_path, monkeypatch):
-    _fake_tree(tmp_path)
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    _fake_tree(tmp_path, monkeypatch)
     monkeypatch.setattr(bench, "PROFILES", {"op": ("profiles/k.md", "k.cu")})
     t, note = bench.recorded_traffic("op")
     assert t == 123456789, note
-    (tmp_path / bench.CSRC / "k.cu").write_bytes(b"kernel v2")
+    # a comment edit leaves the figure valid, a code edit makes it stale
+    (tmp_path / bench.CSRC / "k.cu").write_text("int kernel_v1;  // another comment\n\n")
+    assert bench.recorded_traffic("op")[0] == 123456789
+    (tmp_path / bench.CSRC / "k.cu").write_text("int kernel_v2;\n")
     t, note = bench.recorded_traffic("op")
     assert t is None and "changed" in note
     assert bench.recorded_traffic("other")[0] is None
