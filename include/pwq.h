@@ -453,6 +453,14 @@ pwq_status pwq_device_error(uint32_t* code);
  *              every BF16 amax a >= 0: [0] = values checked, [1] = [2] =
  *              binary32 mismatches against __fdiv_rn (s is stored, so it
  *              must be exact), [3] = values taking the IEEE path.
+ *   which = 4  BF16 magnitude max (bf16x2 abs-max form) against the
+ *              integer max of the magnitude bits, for every ordered pair of
+ *              finite BF16 values: [0] = pairs, [1] = mismatches.
+ *   which = 5  NVFP4 dequantisation through an exact binary16 product
+ *              against the binary32 form bf16(fl(fl(dec(c) dec(sb)) gs)),
+ *              for every E2M1 code pair, block scale code 0..126 and global
+ *              scale fl(a / 2688) (a = 0 or a positive finite BF16):
+ *              [0] = code pairs, [1] = mismatching BF16 pairs.
  * counts (device, 4 x uint64, zeroed by the call): [0] pairs checked,
  * [1] code mismatches, [2] binary32 quotient mismatches where |x| >= 2^-100
  * and the IEEE quotient is normal, [3] pairs whose divisor takes the

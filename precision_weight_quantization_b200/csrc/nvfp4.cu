@@ -174,17 +174,6 @@ __device__ __forceinline__ uint32_t codes_half(uint4 v, float d, float r) {
            (e2m1x2(q[6], q[7]) << 24);
 }
 
-// y = bf16(fl((dec(c) * dec(sb)) * gs)) for the 8 codes of a half block.
-__device__ __forceinline__ uint4 dequant_half(uint32_t codes, float sbv, float gs) {
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float2 c = e2m1x2_decode((codes >> (8 * j)) & 0xffu);
-        w[j] = pack_bf16x2(__fmul_rn(__fmul_rn(c.x, sbv), gs), __fmul_rn(__fmul_rn(c.y, sbv), gs));
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 template <bool kFake, bool kFp8>
 __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs a) {
     __shared__ ScaleTable tab;
@@ -380,6 +369,7 @@ struct FlowMember {
     const float* ts;      // FP8 block-wise source: tile scales [B][TM][TN] at the first batch index
     int64_t ts_bs;        // FP8 source: TM * TN
     uint32_t tn;          // FP8 source: TN
+    int vec32_o;          // fake-quant output slab and rows 32-byte aligned
 };
 
 struct FlowGroup {
@@ -532,7 +522,14 @@ __device__ __forceinline__ void flow_stage(const FlowMember& M, const FlowItem& 
     }
 }
 
-// Encodes the chunks of one item held in registers.  kFast: every block
+// Chunk of an item taken by thread tid at step j: steps 2i and 2i+1 give
+// the two chunks of one 16-element block, so a thread holds whole blocks
+// (no exchange for the block amax, one block scale per 16 elements).
+__device__ __forceinline__ uint32_t flow_lc(int j, uint32_t tid) {
+    return (uint32_t)(j >> 1) * (2u * kFlowThreads) + 2u * tid + (uint32_t)(j & 1);
+}
+
+// Encodes the blocks of one item held in registers.  kFast: every block
 // divisor of the instance lies in the reciprocal path's range (checked per
 // instance), so no per-block branch; a zero block scale then has d = 0 and a
 // zero table reciprocal, for which the reciprocal formula yields the signed
@@ -546,11 +543,13 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
     char* ob = M.out + (int64_t)it.b * M.o_bs;
     uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.chunks >> 1);
 #pragma unroll
-    for (int j = 0; j < kItemChunksPerThread; ++j) {
-        const uint32_t c = it.c0 + (uint32_t)j * kFlowThreads + tid;
-        uint32_t m = amax_bits8(v[j]);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));   // lanes 2i, 2i+1: one block
-        const float amax_b = __uint_as_float(m << 16);
+    for (int i = 0; i < kItemChunksPerThread / 2; ++i) {
+        const uint4 lo = v[2 * i], hi = v[2 * i + 1];
+        // c is even (the block's first chunk); rows hold an even number of
+        // chunks, so c + 1 is in the same row and c < c1 implies c + 1 < c1
+        const uint32_t c = it.c0 + flow_lc(2 * i, tid);
+        const uint32_t mw = hmax_abs(amax_word8(lo), amax_word8(hi)) & 0x7fff7fffu;
+        const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
         float ratio;
         if (kFast)
             ratio = div_fast(amax_b, six_gs, r6);
@@ -558,13 +557,16 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
             ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
         const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0 (a NaN ratio, outside the contract, stays in the table)
         const float4 e = tab.e[sb];
-        uint32_t codes;
+        uint32_t c0, c1;
         if (kFast) {
             float q[8];
-            quotients8<true>(v[j], e.x, e.y, q);
-            codes = e2m1x8(q);
+            quotients8<true>(lo, e.x, e.y, q);
+            c0 = e2m1x8(q);
+            quotients8<true>(hi, e.x, e.y, q);
+            c1 = e2m1x8(q);
         } else {
-            codes = codes_half(v[j], e.x, e.y);
+            c0 = codes_half(lo, e.x, e.y);
+            c1 = codes_half(hi, e.x, e.y);
         }
         if (kFull || c < it.c1) {
             int64_t oo;
@@ -575,10 +577,18 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
                 oo = (int64_t)r * M.o_rs + (int64_t)(c - r * M.cpr.d) * (kFake ? 16 : 4);
             }
             if (kFake) {
-                st_hint_v4(ob + oo, dequant_half(codes, e.z, gs), pol);
+                const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
+                const uint64_t gs2 = f32x2(gs, gs);
+                const uint4 y0 = dequant_half_h(c0, sb2, gs2), y1 = dequant_half_h(c1, sb2, gs2);
+                if (M.vec32_o) {
+                    st_hint_v8(ob + oo, y0, y1, pol);
+                } else {
+                    st_hint_v4(ob + oo, y0, pol);
+                    st_hint_v4(ob + oo + 16, y1, pol);
+                }
             } else {
-                st_hint_u32(ob + oo, codes, pol);
-                if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)sb;
+                st_hint_v2(ob + oo, c0, c1, pol);   // 8-byte aligned: c even, packed rows 8-byte aligned
+                sbb[c >> 1] = (uint8_t)sb;
             }
         }
     }
@@ -677,7 +687,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         if (full) {
 #pragma unroll
             for (int j = 0; j < kItemChunksPerThread; ++j) {
-                const uint32_t lc = (uint32_t)j * kFlowThreads + tid;
+                const uint32_t lc = flow_lc(j, tid);
                 if (kFp8)
                     v[j] = flow_fp8_chunk(M, it, *reinterpret_cast<const uint2*>(buf + lc * 8u), it.c0 + lc);
                 else
@@ -687,7 +697,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
             const char* xb = M.x + (int64_t)it.b * M.x_bs;
 #pragma unroll
             for (int j = 0; j < kItemChunksPerThread; ++j) {
-                const uint32_t lc = (uint32_t)j * kFlowThreads + tid;   // chunk within the item
+                const uint32_t lc = flow_lc(j, tid);   // chunk within the item
                 const uint32_t c = it.c0 + lc;
                 v[j] = make_uint4(0u, 0u, 0u, 0u);
                 if (c < it.c1) {
@@ -713,9 +723,11 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
 
         if (!it.is_e) {
             // ---- amax item
-            uint32_t m = 0u;
+            uint32_t mw = 0u;
 #pragma unroll
-            for (int j = 0; j < kItemChunksPerThread; ++j) m = max(m, amax_bits8(v[j]));
+            for (int j = 0; j < kItemChunksPerThread; ++j) mw = hmax_abs(mw, amax_word8(v[j]));
+            mw &= 0x7fff7fffu;
+            uint32_t m = max(mw & 0xffffu, mw >> 16);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((tid & 31u) == 0u) red[k & 1u][tid >> 5] = m;
@@ -1032,6 +1044,8 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
                 M.ts = fp8 ? G.ts[i] + b0 * M.ts_bs : nullptr;
                 M.item_off = off;
                 off += (M.chunks + kItemChunks - 1) / kItemChunks;
+                M.vec32_o = (uintptr_t)M.out % 32 == 0 && o.rstride % 32 == 0 &&
+                            (take == 1 || o.bstride % 32 == 0);
             }
             a.n_inst += (uint32_t)take;
             a.total_items += (uint32_t)take * items;

@@ -871,7 +871,7 @@ pwq_status nvfp4_activation_observe(const pwq_tensor* x, int observer, float ave
 
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream) {
     if (!counts) return fail(PWQ_ERR_NULL, "counts");
-    if (which < 0 || which > 3) return fail(PWQ_ERR_ARG, "which");
+    if (which < 0 || which > 5) return fail(PWQ_ERR_ARG, "which");
     return from_cuda(pwq::launch_selftest_division(which, counts, (cudaStream_t)stream));
 }
 

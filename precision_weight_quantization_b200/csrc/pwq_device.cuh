@@ -20,14 +20,27 @@ namespace pwq {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Per half of two BF16 pairs: the larger magnitude, exactly (finite values,
+// subnormals kept), with the sign bit set to the XOR of the inputs' signs.
+// One instruction per pair instead of a mask and an integer max; callers
+// clear the sign bits once at the end.  pwq_selftest_division(4) checks it
+// against the integer magnitude max for every pair of finite BF16 values.
+__device__ __forceinline__ uint32_t hmax_abs(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// Per half: the largest magnitude of the four BF16 values of that half of
+// a 16-byte chunk (sign bits not meaningful).
+__device__ __forceinline__ uint32_t amax_word8(uint4 v) {
+    return hmax_abs(hmax_abs(v.x, v.y), hmax_abs(v.z, v.w));
+}
+
 // Max of |x| over the 8 BF16 values of a 16-byte chunk, as BF16 magnitude
-// bits.  For finite values the magnitude order equals the unsigned order of
-// the low 15 bits, so the max is two SIMD halfword maxes.
+// bits (for finite values the magnitude order is the unsigned order of the
+// low 15 bits).
 __device__ __forceinline__ uint32_t amax_bits8(uint4 v) {
-    const uint32_t m = 0x7fff7fffu;
-    uint32_t a = __vmaxu2(v.x & m, v.y & m);
-    uint32_t b = __vmaxu2(v.z & m, v.w & m);
-    uint32_t c = __vmaxu2(a, b);
+    const uint32_t c = amax_word8(v) & 0x7fff7fffu;
     return max(c & 0xffffu, c >> 16);
 }
 
@@ -182,6 +195,53 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
     return d;
 }
 
+// y = bf16(fl((dec(c) * dec(sb)) * gs)) for the 8 codes of a half block.
+__device__ __forceinline__ uint4 dequant_half(uint32_t codes, float sbv, float gs) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 c = e2m1x2_decode((codes >> (8 * j)) & 0xffu);
+        w[j] = pack_bf16x2(__fmul_rn(__fmul_rn(c.x, sbv), gs), __fmul_rn(__fmul_rn(c.y, sbv), gs));
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Two E4M3 codes (16 bits, code 0 low) -> their exact binary16 values.
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t codes16) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)codes16));
+    return h2;
+}
+
+// dequant_half with dec(c) * dec(sb) taken as binary16 pairs, then times
+// gs as binary32 pairs.  The binary16 product is exact: dec(c) has at most
+// 2 significant bits and dec(sb) at most 4, and every non-zero product lies
+// in [2^-10, 2688], inside binary16's normal range; so the one rounding is
+// still fl(. * gs), then bf16.  sb2 = {dec(sb), dec(sb)} in binary16, gs2 =
+// {gs, gs}.  Each byte is shifted out before its decode (decoding straight
+// from a packed byte lane gave wrong results on the fast path).
+// pwq_selftest_division(5) compares it with dequant_half for every code
+// byte, every block scale and every global scale fl(a / 2688).
+__device__ __forceinline__ uint4 dequant_half_h(uint32_t codes, uint32_t sb2, uint64_t gs2) {
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}" : "=r"(h[j]) : "r"((codes >> (8 * j)) & 0xffu));
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t p2;
+        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p2) : "r"(h[j]), "r"(sb2));
+        float lo, hi;
+        asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"((uint16_t)(p2 & 0xffffu)));
+        asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"((uint16_t)(p2 >> 16)));
+        const float2 y = f32x2_split(mul_f32x2(f32x2(lo, hi), gs2));
+        w[j] = pack_bf16x2(y.x, y.y);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // FP8 block-wise dequantisation of 8 codes (code 0 in bits 0..7 of c.x):
 // BF16 bits of y = bf16(fl(dec(q) * s)), element 0 in the low half of .x.
 // The products are taken two at a time (f32x2).
@@ -200,9 +260,13 @@ __device__ __forceinline__ uint4 fp8_dequant8(uint2 c, float s) {
 
 // div_fast on the two BF16 values of a packed word w (low half first):
 // s2 = {s, s}, nr2 = {-r, -r}.  The negated numerators come straight from
-// the BF16 bits (widening and sign flip in one integer operation each).
+// the BF16 bits (widening and sign flip in one integer operation each; the
+// low one as a multiply-add, w * 2^16 + 2^31, which issues on the FMA pipe
+// and leaves the busier integer pipe to the rest).
 __device__ __forceinline__ float2 div_fast_bf16x2(uint32_t w, uint64_t s2, uint64_t nr2) {
-    const uint64_t nx = f32x2_bits((w << 16) + 0x80000000u, (w & 0xffff0000u) ^ 0x80000000u);
+    uint32_t lo;
+    asm("mad.lo.u32 %0, %1, 0x10000, 0x80000000;" : "=r"(lo) : "r"(w));
+    const uint64_t nx = f32x2_bits(lo, (w & 0xffff0000u) ^ 0x80000000u);
     const uint64_t q0 = mul_f32x2(nx, nr2);
     const uint64_t e = fma_f32x2(q0, s2, nx);
     return f32x2_split(fma_f32x2(e, nr2, q0));
@@ -323,6 +387,16 @@ __device__ __forceinline__ void st_hint_v4(void* p, uint4 v, uint64_t pol) {
 }
 __device__ __forceinline__ void st_hint_u32(void* p, uint32_t v, uint64_t pol) {
     asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" :: "l"(p), "r"(v), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_hint_v2(void* p, uint32_t a, uint32_t b, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" :: "l"(p), "r"(a), "r"(b), "l"(pol) : "memory");
+}
+// 32-byte store (sm_100 256-bit vector): p must be 32-byte aligned.
+__device__ __forceinline__ void st_hint_v8(void* p, uint4 a, uint4 b, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8}, %9;"
+                 :: "l"(p), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "l"(pol)
+                 : "memory");
 }
 
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {

@@ -11,6 +11,10 @@
 //
 // Codecs: writes the hardware conversions of a range of binary32 inputs so
 // the host can compare them with the CPU oracle.
+//
+// Rewrites: the BF16 magnitude max by the bf16x2 abs-max instruction and
+// the NVFP4 dequantisation through an exact binary16 product are compared
+// with their plain forms over every input they can see.
 #include "pwq_internal.h"
 
 namespace pwq {
@@ -119,6 +123,59 @@ __global__ void __launch_bounds__(kThreads) selftest_tile_scale_kernel(unsigned 
     }
 }
 
+// BF16 magnitude max: hmax_abs against the integer max of the magnitude
+// bits, for every ordered pair (a, b) of finite BF16 values, in both halves
+// of the word (a low in one operand, high in the other).  One CTA per a.
+__global__ void __launch_bounds__(kThreads) selftest_absmax_kernel(unsigned long long* counts) {
+    const uint32_t a = blockIdx.x;
+    unsigned long long n = 0, bad = 0;
+    if (bf16_is_finite(a)) {
+        for (uint32_t b = threadIdx.x; b < 0x10000u; b += blockDim.x) {
+            if (!bf16_is_finite(b)) continue;
+            const uint32_t want = max(a & 0x7fffu, b & 0x7fffu);
+            const uint32_t got = hmax_abs(a | (b << 16), b | (a << 16)) & 0x7fff7fffu;
+            ++n;
+            bad += (got & 0xffffu) != want || (got >> 16) != want;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n += __shfl_xor_sync(0xffffffffu, n, o);
+        bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    }
+    if ((threadIdx.x & 31u) == 0u && n != 0) {
+        atomicAdd(counts + 0, n);
+        atomicAdd(counts + 1, bad);
+    }
+}
+
+// NVFP4 dequantisation, binary16-product form (dequant_half_h) against the
+// binary32 form (dequant_half): every byte of two E2M1 codes, every block
+// scale code 0..126, every global scale gs = fl(a / 2688) with a = 0 or a
+// positive finite BF16 (one CTA per a).  Counts code pairs.
+__global__ void __launch_bounds__(kThreads) selftest_fp4_dequant_kernel(unsigned long long* counts) {
+    const float gs = __fdiv_rn(__uint_as_float(blockIdx.x << 16), 2688.0f);
+    const uint64_t gs2 = f32x2(gs, gs);
+    unsigned long long n = 0, bad = 0;
+    for (uint32_t i = threadIdx.x; i < 127u * 64u; i += blockDim.x) {
+        const uint32_t sb = i >> 6, w = (i & 63u) * 4u;
+        const uint32_t codes = w | ((w + 1u) << 8) | ((w + 2u) << 16) | ((w + 3u) << 24);
+        const uint4 want = dequant_half(codes, e4m3_decode(sb), gs);
+        const uint4 got = dequant_half_h(codes, e4m3x2_f16x2(sb * 0x101u), gs2);
+        n += 4;
+        bad += (got.x != want.x) + (got.y != want.y) + (got.z != want.z) + (got.w != want.w);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n += __shfl_xor_sync(0xffffffffu, n, o);
+        bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    }
+    if ((threadIdx.x & 31u) == 0u) {
+        atomicAdd(counts + 0, n);
+        atomicAdd(counts + 1, bad);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads)
 selftest_codecs_kernel(uint32_t first, uint32_t count, uint8_t* e4m3, uint8_t* e2m1, uint16_t* bf16) {
     const uint32_t stride = gridDim.x * blockDim.x;
@@ -141,8 +198,12 @@ cudaError_t launch_selftest_division(int which, unsigned long long* counts, cuda
         selftest_division_kernel<1><<<dim3(0x7f7f, 0x7e), kThreads, 0, s>>>(counts);
     else if (which == 2)
         selftest_division_kernel<2><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
-    else
+    else if (which == 3)
         selftest_tile_scale_kernel<<<dim3(64), kThreads, 0, s>>>(counts);
+    else if (which == 4)
+        selftest_absmax_kernel<<<dim3(0x10000), kThreads, 0, s>>>(counts);
+    else
+        selftest_fp4_dequant_kernel<<<dim3(0x7f80), kThreads, 0, s>>>(counts);
     return cudaGetLastError();
 }
 

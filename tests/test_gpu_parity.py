@@ -385,6 +385,29 @@ def test_division_exhaustive(P, which):
     assert quot_bad == 0
 
 
+def test_absmax_rewrite_exhaustive(P):
+    """The bf16x2 abs-max form of the block / tile amax equals the integer
+    max of the BF16 magnitude bits for every ordered pair of finite BF16
+    values (both halves of the word)."""
+    counts = torch.zeros(4, dtype=torch.int64, device=DEV)
+    P.check(P.lib.pwq_selftest_division(4, counts.data_ptr(), None), "pwq_selftest_division")
+    torch.cuda.synchronize()
+    n, bad = counts.tolist()[:2]
+    finite = 0x10000 - 2 * 0x80    # BF16 patterns with exponent 0xff excluded
+    assert n == finite * finite and bad == 0
+
+
+def test_fp4_dequant_rewrite_exhaustive(P):
+    """NVFP4 dequantisation through an exact binary16 product equals the
+    binary32 form for every E2M1 code pair, every block scale code and every
+    global scale fl(a / 2688) a BF16 group amax can give."""
+    counts = torch.zeros(4, dtype=torch.int64, device=DEV)
+    P.check(P.lib.pwq_selftest_division(5, counts.data_ptr(), None), "pwq_selftest_division")
+    torch.cuda.synchronize()
+    n, bad = counts.tolist()[:2]
+    assert n == 0x7F80 * 127 * 256 and bad == 0
+
+
 def test_device_codecs_match_oracle(P):
     """Hardware E4M3 / E2M1 / BF16 conversions against the oracle on every
     FP32 input of the active binades (both signs) and a strided sweep of the
