@@ -127,6 +127,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="pwq", choices=["pwq", "reference"])
     ap.add_argument("--layers", type=int, default=36)
+    ap.add_argument("--layers-per-call", type=int, default=2,
+                    help="layers per grouped call (2: 14 tensors, the most one launch takes)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next", action="store_true",
@@ -206,7 +208,8 @@ def bench_config(args, grouped, world):
             "path": "fp8_block q+dq, mxfp8 q+dq, nvfp4 q (qkv, gate/up siblings)+dq, "
                     "nvfp4 fake-quant (siblings)",
             "l2": "inputs larger than L2 (7.3 GB per rank), no flush",
-            "launch": ("one grouped call per op per layer" if grouped else "one call per tensor") +
+            "launch": ("one grouped call (one launch) per op per %d layers (%d tensors)"
+                       % (args.layers_per_call, 7 * args.layers_per_call) if grouped else "one call per tensor") +
                       "; one CUDA graph per op kind, replayed back to back",
             "parallelism": "dp%d (independent sweeps)" % world}
 
@@ -228,7 +231,7 @@ def layer_elems():
 class Buffers:
     """Pre-allocated outputs for every op of every layer."""
 
-    def __init__(self, layers, P, torch):
+    def __init__(self, layers, P, torch, per_call=1):
         import workloads as W
         self.fp8 = []
         self.mx = []
@@ -251,49 +254,55 @@ class Buffers:
                                       device=dev) for n in g],
                          torch.empty(1, dtype=torch.float32, device=dev))
             self.nv.append(nv)
-        # one BF16 output set shared by every dequant / fake-quant (largest layer)
-        self.y = {n: torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for n, x in layers[0].items()}
+        # BF16 output sets shared by every dequant / fake-quant, one per layer
+        # position within a call (the layers of one call need distinct outputs)
+        self.y = [{n: torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for n, x in layers[0].items()}
+                  for _ in range(min(per_call, len(layers)))]
 
 
-def op_calls(op, layers, buf, P, grouped=True):
+def op_calls(op, layers, buf, P, grouped=True, per_call=1):
     """Closures for every call of one op kind over all layers: one grouped
-    call per layer (all 7 tensors / all 4 sibling groups in one launch), or
-    with grouped=False one call per tensor / per group."""
+    call per `per_call` consecutive layers (all their tensors / sibling
+    groups in one launch), or with grouped=False one call per tensor / per
+    group."""
     import workloads as W
     if not grouped:
         return op_calls_per_tensor(op, layers, buf, P)
+    G = W.QWEN3_4B_GROUPS
     calls = []
-    for i, lay in enumerate(layers):
-        names = list(lay)
+    for i0 in range(0, len(layers), per_call):
+        idx = list(range(i0, min(i0 + per_call, len(layers))))
+        ts = [(i, k, n) for k, i in enumerate(idx) for n in layers[i]]       # (layer, position, name)
+        gts = [(i, k, g) for k, i in enumerate(idx) for g in G]
         if op == "fp8_block_quant":
-            calls.append(lambda xs=[lay[n] for n in names], q=[buf.fp8[i][n][0] for n in names],
-                         s=[buf.fp8[i][n][1] for n in names]: P.fp8_block_quant_grouped(xs, out=q, scale=s))
+            calls.append(lambda xs=[layers[i][n] for i, k, n in ts], q=[buf.fp8[i][n][0] for i, k, n in ts],
+                         s=[buf.fp8[i][n][1] for i, k, n in ts]: P.fp8_block_quant_grouped(xs, out=q, scale=s))
         elif op == "fp8_block_dequant":
-            calls.append(lambda q=[buf.fp8[i][n][0] for n in names], s=[buf.fp8[i][n][1] for n in names],
-                         y=[buf.y[n] for n in names]: P.fp8_block_dequant_grouped(q, s, out=y))
+            calls.append(lambda q=[buf.fp8[i][n][0] for i, k, n in ts], s=[buf.fp8[i][n][1] for i, k, n in ts],
+                         y=[buf.y[k][n] for i, k, n in ts]: P.fp8_block_dequant_grouped(q, s, out=y))
         elif op == "mxfp8_quant":
-            calls.append(lambda xs=[lay[n] for n in names], q=[buf.mx[i][n][0] for n in names],
-                         e=[buf.mx[i][n][1] for n in names]: P.mxfp8_quant_grouped(xs, out=q, scale=e))
+            calls.append(lambda xs=[layers[i][n] for i, k, n in ts], q=[buf.mx[i][n][0] for i, k, n in ts],
+                         e=[buf.mx[i][n][1] for i, k, n in ts]: P.mxfp8_quant_grouped(xs, out=q, scale=e))
         elif op == "mxfp8_dequant":
-            calls.append(lambda q=[buf.mx[i][n][0] for n in names], e=[buf.mx[i][n][1] for n in names],
-                         y=[buf.y[n] for n in names]: P.mxfp8_dequant_grouped(q, e, out=y))
+            calls.append(lambda q=[buf.mx[i][n][0] for i, k, n in ts], e=[buf.mx[i][n][1] for i, k, n in ts],
+                         y=[buf.y[k][n] for i, k, n in ts]: P.mxfp8_dequant_grouped(q, e, out=y))
         elif op == "nvfp4_quant":
-            gs_ = W.QWEN3_4B_GROUPS
-            calls.append(lambda xs=[[lay[n] for n in g] for g in gs_], pk=[buf.nv[i][g][0] for g in gs_],
-                         sb=[buf.nv[i][g][1] for g in gs_], gsc=[buf.nv[i][g][2] for g in gs_]:
+            calls.append(lambda xs=[[layers[i][n] for n in g] for i, k, g in gts],
+                         pk=[buf.nv[i][g][0] for i, k, g in gts], sb=[buf.nv[i][g][1] for i, k, g in gts],
+                         gsc=[buf.nv[i][g][2] for i, k, g in gts]:
                          P.nvfp4_quant_grouped(xs, out=pk, sb=sb, global_scale=gsc))
         elif op == "nvfp4_dequant":
             pk, sb, gs, ys = [], [], [], []
-            for g in W.QWEN3_4B_GROUPS:
-                for k, n in enumerate(g):
-                    pk.append(buf.nv[i][g][0][k])
-                    sb.append(buf.nv[i][g][1][k])
+            for i, k, g in gts:
+                for j, n in enumerate(g):
+                    pk.append(buf.nv[i][g][0][j])
+                    sb.append(buf.nv[i][g][1][j])
                     gs.append(buf.nv[i][g][2])
-                    ys.append(buf.y[n])
+                    ys.append(buf.y[k][n])
             calls.append(lambda pk=pk, sb=sb, gs=gs, ys=ys: P.nvfp4_dequant_grouped(pk, sb, gs, out=ys))
         elif op == "nvfp4_fake_quant":
-            gs_ = W.QWEN3_4B_GROUPS
-            calls.append(lambda xs=[[lay[n] for n in g] for g in gs_], ys=[[buf.y[n] for n in g] for g in gs_]:
+            calls.append(lambda xs=[[layers[i][n] for n in g] for i, k, g in gts],
+                         ys=[[buf.y[k][n] for n in g] for i, k, g in gts]:
                          P.nvfp4_fake_quant_grouped(xs, out=ys))
     return calls
 
@@ -309,7 +318,7 @@ def op_calls_per_tensor(op, layers, buf, P):
         elif op == "fp8_block_dequant":
             for n in lay:
                 q, s = buf.fp8[i][n]
-                calls.append(lambda q=q, s=s, y=buf.y[n]: P.fp8_block_dequant(q, s, out=y))
+                calls.append(lambda q=q, s=s, y=buf.y[0][n]: P.fp8_block_dequant(q, s, out=y))
         elif op == "mxfp8_quant":
             for n, x in lay.items():
                 q, e = buf.mx[i][n]
@@ -317,7 +326,7 @@ def op_calls_per_tensor(op, layers, buf, P):
         elif op == "mxfp8_dequant":
             for n in lay:
                 q, e = buf.mx[i][n]
-                calls.append(lambda q=q, e=e, y=buf.y[n]: P.mxfp8_dequant(q, e, out=y))
+                calls.append(lambda q=q, e=e, y=buf.y[0][n]: P.mxfp8_dequant(q, e, out=y))
         elif op == "nvfp4_quant":
             for g in W.QWEN3_4B_GROUPS:
                 pk, sb, gs = buf.nv[i][g]
@@ -327,11 +336,11 @@ def op_calls_per_tensor(op, layers, buf, P):
             for g in W.QWEN3_4B_GROUPS:
                 pk, sb, gs = buf.nv[i][g]
                 for k, n in enumerate(g):
-                    calls.append(lambda p=pk[k], s=sb[k], gs=gs, y=buf.y[n]: P.nvfp4_dequant(p, s, gs, out=y))
+                    calls.append(lambda p=pk[k], s=sb[k], gs=gs, y=buf.y[0][n]: P.nvfp4_dequant(p, s, gs, out=y))
         elif op == "nvfp4_fake_quant":
             for g in W.QWEN3_4B_GROUPS:
                 xs = [lay[n] for n in g]
-                ys = [buf.y[n] for n in g]
+                ys = [buf.y[0][n] for n in g]
                 calls.append(lambda xs=xs, ys=ys: P.nvfp4_fake_quant(xs, out=ys))
     return calls
 
@@ -366,43 +375,46 @@ NEXT_BYTES_PER_ELEM = {
 NEXT_ONE_PASS_BYTES_PER_ELEM = {"fp8_block_requant_nvfp4": 1 + 4 / 16384 + 0.5 + 1 / 16}
 
 
-def next_calls(op, layers, buf, P, torch):
-    """One grouped call per layer (the 7 tensors; for NVFP4 the four sibling
-    groups in one single-pass launch), reading the FP8 codes and scales the
-    step wrote; outputs shared by all layers."""
+def next_calls(op, layers, buf, P, torch, per_call=1):
+    """One grouped call per `per_call` layers (their tensors; for NVFP4 their
+    sibling groups in one single-pass launch), reading the FP8 codes and
+    scales the step wrote; one output set per layer position of a call."""
     import workloads as W
     lay0 = layers[0]
     dev = lay0["q_proj"].device
-    out_q = {n: torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev) for n, x in lay0.items()}
-    calls = []
     names = list(lay0)
-    if op == "fp8_block_requant":
-        out_s = [torch.empty_like(buf.fp8[0][n][1]) for n in names]
-        for i in range(len(layers)):
-            qs = [buf.fp8[i][n][0] for n in names]
-            ss = [buf.fp8[i][n][1] for n in names]
-            calls.append(lambda qs=qs, ss=ss: P.fp8_block_requant_grouped(
-                qs, ss, out=[out_q[n] for n in names], scale_out=out_s))
-    elif op == "fp8_block_requant_mxfp8":
-        out_e = [torch.empty((lay0[n].shape[0], lay0[n].shape[1] // 32), dtype=torch.uint8, device=dev)
-                 for n in names]
-        for i in range(len(layers)):
-            qs = [buf.fp8[i][n][0] for n in names]
-            ss = [buf.fp8[i][n][1] for n in names]
-            calls.append(lambda qs=qs, ss=ss: P.fp8_block_requant_mxfp8_grouped(
-                qs, ss, out=[out_q[n] for n in names], scale_out=out_e))
-    else:
-        pk = {n: torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for n, x in lay0.items()}
-        sb = {n: torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev)
-              for n, x in lay0.items()}
-        G = W.QWEN3_4B_GROUPS
-        gsc = [torch.empty(1, dtype=torch.float32, device=dev) for _ in G]
-        for i in range(len(layers)):
-            qs = [[buf.fp8[i][n][0] for n in g] for g in G]
-            ss = [[buf.fp8[i][n][1] for n in g] for g in G]
-            calls.append(lambda qs=qs, ss=ss: P.fp8_block_requant_nvfp4_grouped(
-                qs, ss, out=[[pk[n] for n in g] for g in G], sb=[[sb[n] for n in g] for g in G],
-                global_scale=gsc))
+    G = W.QWEN3_4B_GROUPS
+    npos = min(per_call, len(layers))
+    out_q = [{n: torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev) for n, x in lay0.items()}
+             for _ in range(npos)]
+    out_s = [{n: torch.empty_like(buf.fp8[0][n][1]) for n in names} for _ in range(npos)]
+    out_e = [{n: torch.empty((x.shape[0], x.shape[1] // 32), dtype=torch.uint8, device=dev) for n, x in lay0.items()}
+             for _ in range(npos)]
+    pk = [{n: torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for n, x in lay0.items()}
+          for _ in range(npos)]
+    sb = [{n: torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev)
+           for n, x in lay0.items()} for _ in range(npos)]
+    gsc = [[torch.empty(1, dtype=torch.float32, device=dev) for _ in G] for _ in range(npos)]
+    calls = []
+    for i0 in range(0, len(layers), per_call):
+        idx = list(range(i0, min(i0 + per_call, len(layers))))
+        ts = [(i, k, n) for k, i in enumerate(idx) for n in names]
+        gts = [(i, k, j) for k, i in enumerate(idx) for j in range(len(G))]
+        qs = [buf.fp8[i][n][0] for i, k, n in ts]
+        ss = [buf.fp8[i][n][1] for i, k, n in ts]
+        if op == "fp8_block_requant":
+            calls.append(lambda qs=qs, ss=ss, o=[out_q[k][n] for i, k, n in ts], so=[out_s[k][n] for i, k, n in ts]:
+                         P.fp8_block_requant_grouped(qs, ss, out=o, scale_out=so))
+        elif op == "fp8_block_requant_mxfp8":
+            calls.append(lambda qs=qs, ss=ss, o=[out_q[k][n] for i, k, n in ts], eo=[out_e[k][n] for i, k, n in ts]:
+                         P.fp8_block_requant_mxfp8_grouped(qs, ss, out=o, scale_out=eo))
+        else:
+            calls.append(lambda gq=[[buf.fp8[i][n][0] for n in G[j]] for i, k, j in gts],
+                         gs=[[buf.fp8[i][n][1] for n in G[j]] for i, k, j in gts],
+                         o=[[pk[k][n] for n in G[j]] for i, k, j in gts],
+                         so=[[sb[k][n] for n in G[j]] for i, k, j in gts],
+                         gso=[gsc[k][j] for i, k, j in gts]:
+                         P.fp8_block_requant_nvfp4_grouped(gq, gs, out=o, sb=so, global_scale=gso))
     return calls
 
 
@@ -422,7 +434,7 @@ def time_next_rows(args, layers, buf, P, torch, hbm_peak, peak_kind):
     stream = torch.cuda.current_stream()
     out = {}
     for op, bpe in NEXT_BYTES_PER_ELEM.items():
-        calls = next_calls(op, layers, buf, P, torch)
+        calls = next_calls(op, layers, buf, P, torch, max(1, args.layers_per_call))
         g = capture(calls, torch)
         for _ in range(args.warmup):
             g.replay()
@@ -505,11 +517,12 @@ def main():
     hbm_peak, peak_kind = peaks()
 
     layers = make_layers(args.layers, dev, rank)
-    buf = Buffers(layers, P, torch)
+    lpc = max(1, args.layers_per_call)
+    buf = Buffers(layers, P, torch, lpc)
     elems_per_step = layer_elems() * args.layers
     grouped = not args.per_tensor
-    graphs = {op: capture(op_calls(op, layers, buf, P, grouped), torch) for op in OPS}
-    ncalls = {op: len(op_calls(op, layers[:1], buf, P, grouped)) * args.layers for op in OPS}
+    graphs = {op: capture(op_calls(op, layers, buf, P, grouped, lpc), torch) for op in OPS}
+    ncalls = {op: len(op_calls(op, layers, buf, P, grouped, lpc)) for op in OPS}
     launches_per_step = sum(ncalls[op] * KERNELS_PER_CALL[op] for op in OPS)
 
     stream = torch.cuda.current_stream()
@@ -564,15 +577,16 @@ def main():
     traffic, traffic_note = recorded_traffic(dom) if grouped else (None, "per-tensor launches")
     roofline = {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(dom_gbs / hbm_peak, 4), "traffic": traffic, "peak_kind": peak_kind,
-                "alg_bytes_per_launch": int(round(layer_elems() * BYTES_PER_ELEM[dom])),
+                "alg_bytes_per_launch": int(round(elems_per_step / ncalls[dom] * BYTES_PER_ELEM[dom])),
                 "avg_launch_us": round(per_op_ms[dom] * 1e3 / ncalls[dom], 2),
-                "note": "achieved = algorithmic bytes of one launch (one layer) / the average launch "
+                "note": "achieved = algorithmic bytes of one launch / the average launch "
                         "duration (CUDA events around the graph of all %d launches of the step); traffic: %s"
                         % (ncalls[dom], traffic_note)}
     if dom in ONE_PASS_BYTES_PER_ELEM:
         one = per_op[dom]["alg_gbs_one_pass"]
         roofline.update({"achieved_one_pass": one, "frac_one_pass": round(one / hbm_peak, 4),
-                         "alg_bytes_per_launch_one_pass": int(round(layer_elems() * ONE_PASS_BYTES_PER_ELEM[dom]))})
+                         "alg_bytes_per_launch_one_pass":
+                             int(round(elems_per_step / ncalls[dom] * ONE_PASS_BYTES_PER_ELEM[dom]))})
         roofline["note"] += ("; achieved counts the amax pass's read of the input (two reads, as the method "
                              "is defined); *_one_pass counts a single read, the stricter ideal")
 

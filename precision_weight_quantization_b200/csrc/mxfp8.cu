@@ -84,16 +84,25 @@ __global__ void __launch_bounds__(kThreads) mxfp8_quant_kernel(const __grid_cons
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const uint32_t c = base + u * 32u + lane;
-            uint32_t m = amax_bits8(v[u]);
+            uint32_t m = amax_bits8_int(v[u]);
             m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
             m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
             const int e = ue8m0_exponent(m);
             const float inv = exp2i(-e);  // exact power of two
             uint2 out;
-            out.x = e4m3x4(__fmul_rn(bf16_lo(v[u].x), inv), __fmul_rn(bf16_hi(v[u].x), inv),
-                           __fmul_rn(bf16_lo(v[u].y), inv), __fmul_rn(bf16_hi(v[u].y), inv));
-            out.y = e4m3x4(__fmul_rn(bf16_lo(v[u].z), inv), __fmul_rn(bf16_hi(v[u].z), inv),
-                           __fmul_rn(bf16_lo(v[u].w), inv), __fmul_rn(bf16_hi(v[u].w), inv));
+            // x * 2^-e two at a time (f32x2); the low BF16 widened by a
+            // multiply (FMA pipe), the high one by a mask
+            const uint64_t inv2 = f32x2(inv, inv);
+            const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            float2 p[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                uint32_t lo;
+                asm("mul.lo.u32 %0, %1, 0x10000;" : "=r"(lo) : "r"(wv[h]));
+                p[h] = f32x2_split(mul_f32x2(f32x2_bits(lo, wv[h] & 0xffff0000u), inv2));
+            }
+            out.x = e4m3x4(p[0].x, p[0].y, p[1].x, p[1].y);
+            out.y = e4m3x4(p[2].x, p[2].y, p[3].x, p[3].y);
             if (c < T.chunks) {
                 st_v2(T.out + qo[u], out);
                 if ((lane & 3u) == 0u) T.e[c >> 2] = (uint8_t)(e + 127);

@@ -61,3 +61,52 @@ def test_every_profile_summary_parses():
         text = open(os.path.join(ROOT, md)).read()
         assert "traffic_bytes_per_launch:" in text and "source_sha256:" in text, md
         assert os.path.exists(os.path.join(ROOT, bench.CSRC, src)), src
+
+
+class _Recorder:
+    """Stands in for the binding: records the tensor lists of every call."""
+
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def f(*args, **kw):
+            self.calls.append((name, args, kw))
+        return f
+
+
+def _flat(x):
+    if isinstance(x, (list, tuple)):
+        for y in x:
+            yield from _flat(y)
+    else:
+        yield x
+
+
+@pytest.mark.parametrize("per_call", [1, 2])
+def test_grouped_calls_cover_every_layer_once(per_call):
+    # small stand-in layers with the workload's tensor names
+    import torch
+    import workloads as W
+    names = [n for g in W.QWEN3_4B_GROUPS for n in g]
+    layers = [{n: torch.zeros(32, 64, dtype=torch.bfloat16) for n in names} for _ in range(3)]
+    rec = _Recorder()
+    buf = bench.Buffers(layers, rec, torch, per_call)
+    for op in bench.OPS:
+        rec.calls.clear()
+        calls = bench.op_calls(op, layers, buf, rec, True, per_call)
+        assert len(calls) == -(-3 // per_call)
+        for c in calls:
+            c()
+        inputs, outputs = [], []
+        for name, args, kw in rec.calls:
+            inputs += [id(t) for t in _flat(args[:1])]
+            outputs += [id(t) for t in _flat(kw.get("out"))]
+        if op in ("fp8_block_quant", "mxfp8_quant", "nvfp4_quant", "nvfp4_fake_quant"):
+            # every tensor of every layer is an input exactly once
+            assert sorted(inputs) == sorted(id(t) for lay in layers for t in lay.values()), op
+        # no output appears twice within one call (the API rejects overlaps)
+        for j, (name, args, kw) in enumerate(rec.calls):
+            outs = [id(t) for t in _flat(kw.get("out"))]
+            assert len(outs) == len(set(outs)), op
+            assert len(outs) == 7 * min(per_call, 3 - j * per_call), op
