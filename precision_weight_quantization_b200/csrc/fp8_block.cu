@@ -282,6 +282,7 @@ fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
     __shared__ __align__(8) uint64_t bars[kRqStages];
     __shared__ TileLoc meta[kRqStages];
     __shared__ uint32_t red[2][kThreads / 32];
+    __shared__ __align__(16) uint8_t lut[256];   // per tile: input code -> output code
 
     const uint32_t tid = threadIdx.x;
     const uint32_t pad = (1024u - (smem_addr(smem) & 1023u)) & 1023u;
@@ -325,8 +326,9 @@ fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
         for (int j = 0; j < kChunksPerThread; ++j) {
             v[j] = make_uint2(0u, 0u);
             if (ok) v[j] = *reinterpret_cast<const uint2*>(buf + (row0 + 16 * j) * kTile + ccol);
-            m = max(m, e4m3_maxmag8(v[j]));
+            m = __vmaxu2(m, e4m3_maxmag_lanes(v[j]));
         }
+        m = e4m3_maxmag_fin(m);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((tid & 31u) == 0u) red[it & 1u][tid >> 5] = m;
@@ -349,12 +351,35 @@ fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
 #pragma unroll
         for (int w = 1; w < kThreads / 32; ++w) mc = max(mc, red[it & 1u][w]);
         const float s2 = fp8_tile_scale(__uint_as_float(fp8_amax_bits16(mc, sc) << 16));
-        const bool fast = div_fast_ok(s2);   // CTA-uniform
-        const float r2 = fast ? __frcp_rn(s2) : 0.0f;
+        // Within a tile every output code is a function of the input code
+        // alone (y = bf16(fl(dec(q) * s)), q' = e4m3(fl(y / s2))), so each
+        // thread encodes one of the 256 codes into a table and every element
+        // is mapped through it: the per-element arithmetic of the kernel
+        // becomes a byte lookup.  The table entry uses the same quotient
+        // path (reciprocal or IEEE, chosen by s2) as the per-element form.
+        {
+            const bool fast = div_fast_ok(s2);   // CTA-uniform
+            const float r2 = fast ? __frcp_rn(s2) : 0.0f;
+            const float y = __uint_as_float((pack_bf16x2(__fmul_rn(e4m3_decode(tid), sc), 0.0f) & 0xffffu) << 16);
+            const float q = fast ? div_fast(y, s2, r2) : div_slow(y, s2);
+            // one table: every thread finished mapping the previous tile
+            // before the barrier above
+            lut[tid] = (uint8_t)(e4m3x2(q, 0.0f) & 0xffu);
+        }
+        __syncthreads();   // the table is complete
         uint2 out[kChunksPerThread];
 #pragma unroll
-        for (int j = 0; j < kChunksPerThread; ++j)
-            out[j] = fast ? fp8_requant8<true>(v[j], sc, s2, r2) : fp8_requant8<false>(v[j], sc, s2, r2);
+        for (int j = 0; j < kChunksPerThread; ++j) {
+            const uint32_t w[2] = {v[j].x, v[j].y};
+            uint32_t o[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t b0 = lut[__byte_perm(w[h], 0u, 0x4440u)], b1 = lut[__byte_perm(w[h], 0u, 0x4441u)];
+                const uint32_t b2 = lut[__byte_perm(w[h], 0u, 0x4442u)], b3 = lut[__byte_perm(w[h], 0u, 0x4443u)];
+                o[h] = __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u);
+            }
+            out[j] = make_uint2(o[0], o[1]);
+        }
 
         const TileTensor& T = a.t[L.i];
         if (tid == 0) T.scale[L.lt] = s2;

@@ -93,14 +93,21 @@ __device__ __forceinline__ float2 e4m3x2_decode(uint32_t codes16) {
 // One E4M3 code -> exact binary32 value.
 __device__ __forceinline__ float e4m3_decode(uint32_t code) { return e4m3x2_decode(code & 0xffu).x; }
 
-// Largest magnitude byte (bits 0..6) among 8 E4M3 codes; positive E4M3
-// codes order like their values.
-__device__ __forceinline__ uint32_t e4m3_maxmag8(uint2 c) {
-    uint32_t m = __vmaxu4(c.x & 0x7f7f7f7fu, c.y & 0x7f7f7f7fu);
-    m = __vmaxu4(m, m >> 16);
-    m = __vmaxu4(m, m >> 8);
-    return m & 0xffu;
+// Largest magnitude byte (bits 0..6) among E4M3 codes; positive E4M3 codes
+// order like their values.  A per-byte SIMD max has no single instruction
+// on this target (it is emulated with several), so the bytes are compared
+// as the high bytes of 16-bit lanes: the masked words themselves (bytes 1
+// and 3 high) and the words shifted up by 8 (bytes 0 and 2 high).  The lane
+// form accumulates over chunks with __vmaxu2; e4m3_maxmag_fin reads the
+// maximum out once.
+__device__ __forceinline__ uint32_t e4m3_maxmag_lanes(uint2 c) {
+    const uint32_t a = c.x & 0x7f7f7f7fu, b = c.y & 0x7f7f7f7fu;
+    return __vmaxu2(__vmaxu2(a, b), __vmaxu2(a << 8, b << 8));
 }
+__device__ __forceinline__ uint32_t e4m3_maxmag_fin(uint32_t lanes) {
+    return max(lanes >> 24, (lanes >> 8) & 0xffu);
+}
+__device__ __forceinline__ uint32_t e4m3_maxmag8(uint2 c) { return e4m3_maxmag_fin(e4m3_maxmag_lanes(c)); }
 
 // BF16 magnitude bits of max |y| over FP8 codes of one scale s whose largest
 // magnitude byte is mc: rounding is monotone and symmetric in sign, so the

@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(kThreads, 3) fp8_requant_fp8_kernel(const __gr
         }
         uint32_t m = 0u;
 #pragma unroll
-        for (int j = 0; j < kChunks; ++j) m = max(m, e4m3_maxmag8(v[j]));
+        for (int j = 0; j < kChunks; ++j) m = __vmaxu2(m, e4m3_maxmag_lanes(v[j]));
+        m = e4m3_maxmag_fin(m);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0u) red[par][warp] = m;
