@@ -685,13 +685,24 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         const unsigned char* buf = flow_smem + st * kFlowStageBytes;
         const bool full = (it.c1 - it.c0 == kItemChunks) && M.dense_x && M.dense_o;
         if (full) {
+            if (kFp8) {
 #pragma unroll
-            for (int j = 0; j < kItemChunksPerThread; ++j) {
-                const uint32_t lc = flow_lc(j, tid);
-                if (kFp8)
-                    v[j] = flow_fp8_chunk(M, it, *reinterpret_cast<const uint2*>(buf + lc * 8u), it.c0 + lc);
-                else
-                    v[j] = *reinterpret_cast<const uint4*>(buf + lc * 16u);
+                for (int j = 0; j < kItemChunksPerThread; j += 2) {
+                    // lc even: the block's two chunks lie in one row and one
+                    // tile, so one row / column step and one tile-scale load
+                    const uint32_t lc = flow_lc(j, tid);
+                    const uint4 cc = *reinterpret_cast<const uint4*>(buf + lc * 8u);
+                    const uint32_t c = it.c0 + lc;
+                    const uint32_t r = fdiv(c, M.cpr);
+                    const uint32_t k = c - r * M.cpr.d;
+                    const float sc = __ldg(M.ts + (int64_t)it.b * M.ts_bs + (r >> 7) * M.tn + (k >> 4));
+                    v[j] = fp8_dequant8(make_uint2(cc.x, cc.y), sc);
+                    v[j + 1] = fp8_dequant8(make_uint2(cc.z, cc.w), sc);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < kItemChunksPerThread; ++j)
+                    v[j] = *reinterpret_cast<const uint4*>(buf + flow_lc(j, tid) * 16u);
             }
         } else {
             const char* xb = M.x + (int64_t)it.b * M.x_bs;
