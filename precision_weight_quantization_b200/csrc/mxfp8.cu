@@ -4,14 +4,16 @@
 // float8_e4m3fn weights).
 //
 // HBM-bound elementwise kernels over a list of up to kMaxLaunchTensors
-// tensors per launch.  Each thread owns 8-element chunks (16 B of BF16, one
-// 128-bit load); four consecutive lanes form one 32-element block and
-// combine their amax with two butterfly shuffles.  The scale is a power of
-// two, so x * 2^-e is an exact multiply and no division is needed.  A
-// persistent grid walks the concatenated chunk ranges in warp-sized spans of
-// kUnroll * 32 chunks (kUnroll independent 128-bit loads in flight per
-// thread); every tensor's range is padded to a whole number of spans so a
-// span never straddles two tensors.
+// tensors per launch, walked by a persistent grid in warp-sized spans; every
+// tensor's range is padded to a whole number of spans so a span never
+// straddles two tensors.  The scale is a power of two, so x * 2^-e is an
+// exact multiply and no division is needed.
+//
+// Quantise: one thread per 32-element block (64 bytes of BF16 in, 32 codes
+// and one scale byte out), so the block amax needs no lane exchange and the
+// exponent is found once per block.  Dequantise: 8-element chunks per thread
+// (8 code bytes in, 16 bytes of BF16 out), kUnroll chunks in flight; each
+// chunk reads its block's scale byte.
 #include <algorithm>
 
 #include "pwq_internal.h"
@@ -64,53 +66,6 @@ __device__ __forceinline__ void chunk_offsets(const ChunkTensor& T, uint32_t c, 
     }
 }
 
-__global__ void __launch_bounds__(kThreads) mxfp8_quant_kernel(const __grid_constant__ ChunkArgs a) {
-    const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-    for (uint32_t slot = gwarp * kSpan; slot < a.total_slots; slot += nwarps * kSpan) {
-        const ChunkTensor& T = a.t[span_tensor(a, slot)];
-        const uint32_t base = slot - T.slot_begin;
-        uint4 v[kUnroll];
-        int64_t qo[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * 32u + lane;
-            int64_t xo;
-            chunk_offsets(T, c, 16, 8, xo, qo[u]);
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
-            if (c < T.chunks) v[u] = ld_stream_v4(T.in + xo);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * 32u + lane;
-            uint32_t m = amax_bits8_int(v[u]);
-            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            const int e = ue8m0_exponent(m);
-            const float inv = exp2i(-e);  // exact power of two
-            uint2 out;
-            // x * 2^-e two at a time (f32x2); the low BF16 widened by a
-            // multiply (FMA pipe), the high one by a mask
-            const uint64_t inv2 = f32x2(inv, inv);
-            const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-            float2 p[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                uint32_t lo;
-                asm("mul.lo.u32 %0, %1, 0x10000;" : "=r"(lo) : "r"(wv[h]));
-                p[h] = f32x2_split(mul_f32x2(f32x2_bits(lo, wv[h] & 0xffff0000u), inv2));
-            }
-            out.x = e4m3x4(p[0].x, p[0].y, p[1].x, p[1].y);
-            out.y = e4m3x4(p[2].x, p[2].y, p[3].x, p[3].y);
-            if (c < T.chunks) {
-                st_v2(T.out + qo[u], out);
-                if ((lane & 3u) == 0u) T.e[c >> 2] = (uint8_t)(e + 127);
-            }
-        }
-    }
-}
-
 __global__ void __launch_bounds__(kThreads) mxfp8_dequant_kernel(const __grid_constant__ ChunkArgs a) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -156,9 +111,147 @@ bool dense_view(const View& v, int64_t row_bytes) {
     return v.rstride == row_bytes && (v.batch == 1 || v.bstride == v.rows * v.rstride);
 }
 
-// quant: in = BF16 x, out = codes; dequant: in = codes, out = BF16 y
-template <bool kQuant>
-cudaError_t launch_mx(const Job* jobs, int n, cudaStream_t s) {
+// ---------------------------------------------------------------- quantise: one thread per block
+//
+// Each thread owns whole 32-element blocks: 64 bytes of BF16 in (two
+// 256-bit loads when the rows are 32-byte aligned, else four 128-bit ones),
+// one block amax, one scale exponent, 32 codes and one scale byte out.  No
+// lane exchange, and the per-block work is paid once per 32 elements.
+constexpr uint32_t kBSpan = 32u;   // blocks per warp span (one per lane)
+
+struct BlockTensor {
+    const char* in;
+    char* out;
+    int64_t in_bs, in_rs, out_bs, out_rs;   // bytes
+    uint8_t* e;            // dense [B][M][N/32] scale bytes
+    uint32_t blocks;       // B * M * N / 32
+    uint32_t slot_begin;   // first block slot of this tensor (multiple of kBSpan)
+    FastDiv bpr;           // blocks per row (N / 32)
+    FastDiv rows;          // M
+    int dense;             // both operands dense
+    int in32, out32;       // BF16 rows / code rows (and slabs) 32-byte aligned
+};
+
+struct BlockArgs {
+    BlockTensor t[kMaxLaunchTensors];
+    int n;
+    uint32_t total_slots;
+};
+
+__device__ __forceinline__ int block_span_tensor(const BlockArgs& a, uint32_t slot) {
+    int i = 0;
+    for (int k = 1; k < a.n; ++k)
+        if (slot >= a.t[k].slot_begin) i = k;
+    return i;
+}
+
+__global__ void __launch_bounds__(kThreads) mxfp8_quant_block_kernel(const __grid_constant__ BlockArgs a) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t slot = gwarp * kBSpan; slot < a.total_slots; slot += nwarps * kBSpan) {
+        const BlockTensor& T = a.t[block_span_tensor(a, slot)];
+        const uint32_t bi = slot - T.slot_begin + lane;
+        if (bi >= T.blocks) continue;
+        int64_t io, oo;
+        if (T.dense) {
+            io = (int64_t)bi * 64;
+            oo = (int64_t)bi * 32;
+        } else {
+            const uint32_t r = fdiv(bi, T.bpr);          // row over all batches
+            const uint32_t k = bi - r * T.bpr.d;
+            const uint32_t b = fdiv(r, T.rows);
+            const uint32_t m = r - b * T.rows.d;
+            io = (int64_t)b * T.in_bs + (int64_t)m * T.in_rs + (int64_t)k * 64;
+            oo = (int64_t)b * T.out_bs + (int64_t)m * T.out_rs + (int64_t)k * 32;
+        }
+        uint4 v[4];
+        if (T.in32) {
+            ld_nc_v8(T.in + io, v[0], v[1]);
+            ld_nc_v8(T.in + io + 32, v[2], v[3]);
+        } else {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) v[h] = ld_stream_v4(T.in + io + 16 * h);
+        }
+        const uint32_t mw = hmax_abs(hmax_abs(amax_word8(v[0]), amax_word8(v[1])),
+                                     hmax_abs(amax_word8(v[2]), amax_word8(v[3]))) & 0x7fff7fffu;
+        const int e = ue8m0_exponent(max(mw & 0xffffu, mw >> 16));
+        const uint64_t inv2 = f32x2(exp2i(-e), exp2i(-e));   // exact power of two
+        uint32_t q[8];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            // x * 2^-e two at a time (f32x2); the low BF16 widened by a
+            // multiply (FMA pipe), the high one by a mask
+            const uint32_t wv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+            float2 p[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                uint32_t lo;
+                asm("mul.lo.u32 %0, %1, 0x10000;" : "=r"(lo) : "r"(wv[k]));
+                p[k] = f32x2_split(mul_f32x2(f32x2_bits(lo, wv[k] & 0xffff0000u), inv2));
+            }
+            q[2 * h] = e4m3x4(p[0].x, p[0].y, p[1].x, p[1].y);
+            q[2 * h + 1] = e4m3x4(p[2].x, p[2].y, p[3].x, p[3].y);
+        }
+        char* dst = T.out + oo;
+        if (T.out32) {
+            st_v8(dst, make_uint4(q[0], q[1], q[2], q[3]), make_uint4(q[4], q[5], q[6], q[7]));
+        } else {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) st_v2(dst + 8 * h, make_uint2(q[2 * h], q[2 * h + 1]));
+        }
+        T.e[bi] = (uint8_t)(e + 127);
+    }
+}
+
+// Base, row and slab strides all multiples of 32 bytes (256-bit accesses).
+bool aligned32(const View& v) {
+    return (uintptr_t)v.ptr % 32 == 0 && v.rstride % 32 == 0 && (v.batch == 1 || v.bstride % 32 == 0);
+}
+
+cudaError_t launch_mx_quant_blocks(const Job* jobs, int n, cudaStream_t s) {
+    const uint64_t kMaxSlots = uint64_t(1) << 31;   // block indices stay 32-bit
+    for (int j0 = 0; j0 < n;) {
+        BlockArgs a;
+        a.n = 0;
+        uint32_t slots = 0;
+        for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
+            const Job& j = jobs[j0 + a.n];
+            const View& x = j.in;    // BF16
+            const View& q = j.out;   // codes
+            const uint64_t padded = ((uint64_t)(x.batch * x.rows * (x.cols / 32)) + kBSpan - 1) / kBSpan * kBSpan;
+            if (a.n > 0 && slots + padded > kMaxSlots) break;
+            BlockTensor& T = a.t[a.n];
+            T.in = j.in.ptr;
+            T.out = j.out.ptr;
+            T.in_bs = j.in.bstride;
+            T.in_rs = j.in.rstride;
+            T.out_bs = j.out.bstride;
+            T.out_rs = j.out.rstride;
+            T.e = static_cast<uint8_t*>(j.scale);
+            T.blocks = (uint32_t)(x.batch * x.rows * (x.cols / 32));
+            T.slot_begin = slots;
+            T.bpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 32));
+            T.rows = make_fastdiv((uint32_t)std::max<int64_t>(1, x.rows));
+            T.dense = dense_view(x, x.cols * 2) && dense_view(q, q.cols);
+            T.in32 = aligned32(j.in);
+            T.out32 = aligned32(j.out);
+            slots += (uint32_t)padded;
+        }
+        j0 += a.n;
+        a.total_slots = slots;
+        if (slots == 0) continue;
+        const int grid = persistent_grid((slots + kThreads - 1) / kThreads, 8);
+        mxfp8_quant_block_kernel<<<grid, kThreads, 0, s>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+
+// in = codes, out = BF16 y
+cudaError_t launch_mx_dequant(const Job* jobs, int n, cudaStream_t s) {
     const uint64_t kMaxSlots = uint64_t(1) << 31;   // chunk indices stay 32-bit
     for (int j0 = 0; j0 < n;) {
         ChunkArgs a;
@@ -166,12 +259,12 @@ cudaError_t launch_mx(const Job* jobs, int n, cudaStream_t s) {
         uint32_t slots = 0;
         for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
             const Job& j = jobs[j0 + a.n];
-            const View& xv = kQuant ? j.in : j.out;
+            const View& xv = j.out;
             const uint64_t padded = ((uint64_t)(xv.batch * xv.rows * (xv.cols / 8)) + kSpan - 1) / kSpan * kSpan;
             if (a.n > 0 && slots + padded > kMaxSlots) break;
             ChunkTensor& T = a.t[a.n];
-            const View& x = kQuant ? j.in : j.out;   // the BF16 side
-            const View& q = kQuant ? j.out : j.in;   // the code side
+            const View& x = j.out;   // the BF16 side
+            const View& q = j.in;    // the code side
             T.in = j.in.ptr;
             T.out = j.out.ptr;
             T.in_bs = j.in.bstride;
@@ -190,10 +283,7 @@ cudaError_t launch_mx(const Job* jobs, int n, cudaStream_t s) {
         a.total_slots = slots;
         if (slots == 0) continue;
         const int grid = persistent_grid((slots + kThreads * kUnroll - 1) / (kThreads * kUnroll), 8);
-        if (kQuant)
-            mxfp8_quant_kernel<<<grid, kThreads, 0, s>>>(a);
-        else
-            mxfp8_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
+        mxfp8_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -202,8 +292,8 @@ cudaError_t launch_mx(const Job* jobs, int n, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_mxfp8_quant(const Job* jobs, int n, cudaStream_t s) { return launch_mx<true>(jobs, n, s); }
+cudaError_t launch_mxfp8_quant(const Job* jobs, int n, cudaStream_t s) { return launch_mx_quant_blocks(jobs, n, s); }
 
-cudaError_t launch_mxfp8_dequant(const Job* jobs, int n, cudaStream_t s) { return launch_mx<false>(jobs, n, s); }
+cudaError_t launch_mxfp8_dequant(const Job* jobs, int n, cudaStream_t s) { return launch_mx_dequant(jobs, n, s); }
 
 }  // namespace pwq

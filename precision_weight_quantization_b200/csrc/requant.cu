@@ -13,15 +13,20 @@
 // bf16(fl(dec(mc) * |s|)) for the set's largest code magnitude mc, because
 // the rounding is monotone and symmetric in sign.
 //
-//   FP8 block -> FP8 block: one CTA per 128x128 tile (persistent grid); each
-//     thread holds 64 codes (8-byte loads, 16 threads per tile row), one
-//     barrier combines the warp maxima, then codes are re-encoded against
-//     the new tile scale by the verified reciprocal path.  2 B per element.
-//   FP8 block -> MXFP8: a chunk walk like mxfp8_quant's; four lanes hold one
-//     1x32 block (which never leaves its 128-wide tile), the block amax comes
-//     from the largest code magnitude and the tile scale.  2 + 1/32 B per
-//     element.
-//   FP8 block -> NVFP4: the NVFP4 amax and encode kernels with an FP8 source
+//   FP8 block -> FP8 block: one CTA per 128x128 tile (persistent grid);
+//     the TMA path (fp8_block.cu, 16-byte aligned code rows) stages tiles in
+//     a ring and maps every code through a per-tile 256-entry table (within
+//     a tile the output code is a function of the input code alone); the
+//     fallback here holds 64 codes per thread (8-byte loads, 16 threads per
+//     tile row), one barrier combines the warp maxima, then codes are
+//     re-encoded against the new tile scale by the verified reciprocal path.
+//     2 B per element.
+//   FP8 block -> MXFP8: a block walk like mxfp8_quant's; with 16-byte
+//     aligned code rows one lane holds one 1x32 block (which never leaves
+//     its 128-wide tile), whose amax comes from the largest code magnitude
+//     and the tile scale; 8-byte aligned rows take a per-tensor kernel of
+//     8-code chunks, four lanes per block.  2 + 1/32 B per element.
+//   FP8 block -> NVFP4: the NVFP4 single-pass kernel with an FP8 source
 //     (nvfp4.cu).
 #include <algorithm>
 
@@ -231,84 +236,76 @@ __global__ void __launch_bounds__(kThreads) fp8_requant_mxfp8_kernel(const __gri
     }
 }
 
-// Grouped FP8 -> MXFP8 with 16-code chunks (one 16-byte load per lane; two
-// lanes per 1x32 block, one shuffle); needs 16-byte aligned code rows.
-struct Mx16Tensor {
+// Grouped FP8 -> MXFP8 (16-byte aligned code rows): one lane per 1x32
+// block, two 16-byte loads and two 16-byte stores.
+struct MxBlkTensor {
     const char* q;
     char* q2;
     int64_t q_bs, q_rs, o_bs, o_rs;   // bytes
     const float* s;           // [B][TM][TN]
     uint8_t* e;               // dense [B][M][N/32]
-    uint32_t chunks;          // B * M * N / 16
-    uint32_t slot_begin;      // multiple of kSpan
+    uint32_t chunks;          // 32-code blocks: B * M * N / 32
+    uint32_t slot_begin;      // multiple of 32 (one warp span)
     uint32_t tm, tn;
-    FastDiv cpr, rows;        // 16-code chunks per row (N / 16), M
+    FastDiv cpr, rows;        // blocks per row (N / 32), M
     int dense;
 };
 
-struct Mx16Args {
-    Mx16Tensor t[kMaxLaunchTensors];
+struct MxBlkArgs {
+    MxBlkTensor t[kMaxLaunchTensors];
     int n;
     uint32_t total_slots;
 };
 
 __device__ __forceinline__ uint2 mx_encode8(uint4 y, float inv) {
-    return make_uint2(e4m3x4(__fmul_rn(bf16_lo(y.x), inv), __fmul_rn(bf16_hi(y.x), inv),
-                             __fmul_rn(bf16_lo(y.y), inv), __fmul_rn(bf16_hi(y.y), inv)),
-                      e4m3x4(__fmul_rn(bf16_lo(y.z), inv), __fmul_rn(bf16_hi(y.z), inv),
-                             __fmul_rn(bf16_lo(y.w), inv), __fmul_rn(bf16_hi(y.w), inv)));
+    const uint64_t inv2 = f32x2(inv, inv);
+    const uint32_t wv[4] = {y.x, y.y, y.z, y.w};
+    float2 p[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t lo;
+        asm("mul.lo.u32 %0, %1, 0x10000;" : "=r"(lo) : "r"(wv[k]));
+        p[k] = f32x2_split(mul_f32x2(f32x2_bits(lo, wv[k] & 0xffff0000u), inv2));
+    }
+    return make_uint2(e4m3x4(p[0].x, p[0].y, p[1].x, p[1].y), e4m3x4(p[2].x, p[2].y, p[3].x, p[3].y));
 }
 
-__global__ void __launch_bounds__(kThreads) fp8_requant_mxfp8_16_kernel(const __grid_constant__ Mx16Args a) {
+__global__ void __launch_bounds__(kThreads) fp8_requant_mxfp8_block_kernel(const __grid_constant__ MxBlkArgs a) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-    for (uint32_t slot = gwarp * kSpan; slot < a.total_slots; slot += nwarps * kSpan) {
+    for (uint32_t slot = gwarp * 32u; slot < a.total_slots; slot += nwarps * 32u) {
         int ti = 0;
         for (int k = 1; k < a.n; ++k)
             if (slot >= a.t[k].slot_begin) ti = k;
-        const Mx16Tensor& T = a.t[ti];
-        const uint32_t base = slot - T.slot_begin;
-        uint4 v[kUnroll];
-        float s[kUnroll];
-        int64_t oo[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * 32u + lane;
-            const uint32_t R = fdiv(c, T.cpr);           // row over all batches
-            const uint32_t k = c - R * T.cpr.d;          // chunk within the row
-            const uint32_t b = fdiv(R, T.rows);
-            const uint32_t m = R - b * T.rows.d;
-            int64_t io;
-            if (T.dense) {
-                io = (int64_t)c * 16;
-                oo[u] = io;
-            } else {
-                io = (int64_t)b * T.q_bs + (int64_t)m * T.q_rs + (int64_t)k * 16;
-                oo[u] = (int64_t)b * T.o_bs + (int64_t)m * T.o_rs + (int64_t)k * 16;
-            }
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
-            s[u] = 0.0f;
-            if (c < T.chunks) {
-                v[u] = ld_stream_v4(T.q + io);
-                s[u] = __ldg(T.s + ((int64_t)b * T.tm + (m >> 7)) * T.tn + (k >> 3));
-            }
+        const MxBlkTensor& T = a.t[ti];
+        const uint32_t bi = slot - T.slot_begin + lane;   // 32-code block
+        if (bi >= T.chunks) continue;
+        const uint32_t R = fdiv(bi, T.cpr);           // row over all batches
+        const uint32_t k = bi - R * T.cpr.d;          // block within the row
+        const uint32_t b = fdiv(R, T.rows);
+        const uint32_t m = R - b * T.rows.d;
+        int64_t io, oo;
+        if (T.dense) {
+            io = (int64_t)bi * 32;
+            oo = io;
+        } else {
+            io = (int64_t)b * T.q_bs + (int64_t)m * T.q_rs + (int64_t)k * 32;
+            oo = (int64_t)b * T.o_bs + (int64_t)m * T.o_rs + (int64_t)k * 32;
         }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * 32u + lane;
-            const uint2 lo = make_uint2(v[u].x, v[u].y), hi = make_uint2(v[u].z, v[u].w);
-            uint32_t mc = max(e4m3_maxmag8(lo), e4m3_maxmag8(hi));
-            mc = max(mc, __shfl_xor_sync(0xffffffffu, mc, 1));   // lanes 2i, 2i+1: one block
-            const int e = ue8m0_exponent(fp8_amax_bits16(mc, s[u]));
-            const float inv = exp2i(-e);   // exact power of two
-            const uint2 o0 = mx_encode8(fp8_dequant8(lo, s[u]), inv);
-            const uint2 o1 = mx_encode8(fp8_dequant8(hi, s[u]), inv);
-            if (c < T.chunks) {
-                st_v4(T.q2 + oo[u], make_uint4(o0.x, o0.y, o1.x, o1.y));
-                if ((lane & 1u) == 0u) T.e[c >> 1] = (uint8_t)(e + 127);
-            }
-        }
+        uint4 v0 = ld_stream_v4(T.q + io), v1 = ld_stream_v4(T.q + io + 16);
+        const float sc = __ldg(T.s + ((int64_t)b * T.tm + (m >> 7)) * T.tn + (k >> 2));
+        uint32_t lanes = __vmaxu2(e4m3_maxmag_lanes(make_uint2(v0.x, v0.y)), e4m3_maxmag_lanes(make_uint2(v0.z, v0.w)));
+        lanes = __vmaxu2(lanes, __vmaxu2(e4m3_maxmag_lanes(make_uint2(v1.x, v1.y)), e4m3_maxmag_lanes(make_uint2(v1.z, v1.w))));
+        const int e = ue8m0_exponent(fp8_amax_bits16(e4m3_maxmag_fin(lanes), sc));
+        const float inv = exp2i(-e);   // exact power of two
+        const uint2 o0 = mx_encode8(fp8_dequant8(make_uint2(v0.x, v0.y), sc), inv);
+        const uint2 o1 = mx_encode8(fp8_dequant8(make_uint2(v0.z, v0.w), sc), inv);
+        const uint2 o2 = mx_encode8(fp8_dequant8(make_uint2(v1.x, v1.y), sc), inv);
+        const uint2 o3 = mx_encode8(fp8_dequant8(make_uint2(v1.z, v1.w), sc), inv);
+        st_v4(T.q2 + oo, make_uint4(o0.x, o0.y, o1.x, o1.y));
+        st_v4(T.q2 + oo + 16, make_uint4(o2.x, o2.y, o3.x, o3.y));
+        T.e[bi] = (uint8_t)(e + 127);
     }
 }
 
@@ -397,17 +394,17 @@ cudaError_t launch_fp8_requant_mxfp8(const RequantJob* jobs, int n, cudaStream_t
     }
     const uint64_t kMaxSlots = uint64_t(1) << 31;
     for (int j0 = 0; j0 < n;) {
-        Mx16Args a;
+        MxBlkArgs a;
         a.n = 0;
         uint32_t slots = 0;
         for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
             const RequantJob& J = jobs[j0 + a.n];
             const View& q = J.in;
             const View& q2 = J.out;
-            const uint64_t chunks = (uint64_t)(q.batch * q.rows * (q.cols / 16));
-            const uint64_t padded = (chunks + kSpan - 1) / kSpan * kSpan;
+            const uint64_t chunks = (uint64_t)(q.batch * q.rows * (q.cols / 32));
+            const uint64_t padded = (chunks + 31) / 32 * 32;
             if (a.n > 0 && slots + padded > kMaxSlots) break;
-            Mx16Tensor& T = a.t[a.n];
+            MxBlkTensor& T = a.t[a.n];
             T.q = q.ptr;
             T.q2 = q2.ptr;
             T.q_bs = q.bstride;
@@ -420,7 +417,7 @@ cudaError_t launch_fp8_requant_mxfp8(const RequantJob* jobs, int n, cudaStream_t
             T.slot_begin = slots;
             T.tm = (uint32_t)((q.rows + kTile - 1) / kTile);
             T.tn = (uint32_t)((q.cols + kTile - 1) / kTile);
-            T.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, q.cols / 16));
+            T.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, q.cols / 32));
             T.rows = make_fastdiv((uint32_t)std::max<int64_t>(1, q.rows));
             T.dense = q.rstride == q.cols && q2.rstride == q2.cols &&
                       (q.batch == 1 || (q.bstride == q.rows * q.cols && q2.bstride == q2.rows * q2.cols));
@@ -429,8 +426,8 @@ cudaError_t launch_fp8_requant_mxfp8(const RequantJob* jobs, int n, cudaStream_t
         j0 += a.n;
         a.total_slots = slots;
         if (slots == 0) continue;
-        const int grid = persistent_grid((slots + kThreads * kUnroll - 1) / (kThreads * kUnroll), 8);
-        fp8_requant_mxfp8_16_kernel<<<grid, kThreads, 0, st>>>(a);
+        const int grid = persistent_grid((slots + kThreads - 1) / kThreads, 8);
+        fp8_requant_mxfp8_block_kernel<<<grid, kThreads, 0, st>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
