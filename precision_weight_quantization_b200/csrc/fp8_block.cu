@@ -48,6 +48,7 @@ struct TileTensor {
     uint32_t tile_begin;  // first tile of this tensor in the launch
     FastDiv tiles_n;      // tiles per tile row (TN)
     FastDiv tiles_mn;     // tiles per batch matrix (TM * TN)
+    int q16, y32;         // dequant: code rows 16-byte, BF16 rows 32-byte aligned
 };
 
 struct TileLoc {
@@ -235,7 +236,26 @@ __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const __gri
         char* yt = T.y + (int64_t)L.b * T.y_bs + (int64_t)L.tm * kTile * T.y_rs + (int64_t)L.tn * kTile * 2;
         const int rows_here = min(kTile, T.rows - L.tm * kTile);
         const int cols_here = min(kTile, T.cols - L.tn * kTile);
-        if (rows_here == kTile && cols_here == kTile) {
+        if (rows_here == kTile && cols_here == kTile && T.q16) {
+            // 16 codes per thread per row pass: 8 threads per 128-code row
+            const int c16 = (int)(threadIdx.x & 7u) * 16;
+            const int r16 = (int)(threadIdx.x >> 3);
+            uint4 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = ld_stream_v4(qt + (int64_t)(r16 + 32 * j) * T.q_rs + c16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 y0 = fp8_dequant8(make_uint2(v[j].x, v[j].y), sc);
+                const uint4 y1 = fp8_dequant8(make_uint2(v[j].z, v[j].w), sc);
+                char* dst = yt + (int64_t)(r16 + 32 * j) * T.y_rs + c16 * 2;
+                if (T.y32) {
+                    st_v8(dst, y0, y1);
+                } else {
+                    st_v4(dst, y0);
+                    st_v4(dst + 16, y1);
+                }
+            }
+        } else if (rows_here == kTile && cols_here == kTile) {
             uint2 v[kDqChunks];
 #pragma unroll
             for (int j = 0; j < kDqChunks; ++j)
@@ -444,6 +464,9 @@ uint32_t fill_tile_tensor(TileTensor& T, const Job& j, bool quant, uint32_t tile
     T.tile_begin = tile_begin;
     T.tiles_n = make_fastdiv(tn);
     T.tiles_mn = make_fastdiv(tm * tn);
+    T.q16 = (uintptr_t)q.ptr % 16 == 0 && q.rstride % 16 == 0 && (q.batch == 1 || q.bstride % 16 == 0);
+    T.y32 = !quant && (uintptr_t)j.out.ptr % 32 == 0 && j.out.rstride % 32 == 0 &&
+            (j.out.batch == 1 || j.out.bstride % 32 == 0);
     return (uint32_t)q.batch * tm * tn;
 }
 
