@@ -22,7 +22,11 @@ the three formats) inside the timed region.
 `next_rows` times the FP8 block-wise re-quantisation ops (FP8 block-wise
 codes + scales -> FP8 block-wise / MXFP8 / NVFP4 in one pass) on the step's
 FP8 outputs over the same sweep, each in its own graph after the timed
-steps; they are not part of `value`.
+steps; they are not part of `value`.  FP8 -> FP8 is timed twice: on the
+quantiser's codes (every tile holds a +-448 code, so its code map is the
+identity and the kernel copies the codes) and, as
+`fp8_block_requant_general`, on seeded random codes whose magnitudes stop
+below 448 with the same scales (every tile's codes change).
 
 `--impl reference` times the CPU oracle (single thread, as it stands) on a
 bounded sample of the same workload.
@@ -369,6 +373,7 @@ def capture(calls, torch):
 # of each output
 NEXT_BYTES_PER_ELEM = {
     "fp8_block_requant": 1 + 4 / 16384 + 1 + 4 / 16384,
+    "fp8_block_requant_general": 1 + 4 / 16384 + 1 + 4 / 16384,
     "fp8_block_requant_mxfp8": 1 + 4 / 16384 + 1 + 1 / 32,
     "fp8_block_requant_nvfp4": 1 + 4 / 16384 + 1 + 4 / 16384 + 0.5 + 1 / 16,
 }
@@ -395,6 +400,10 @@ def next_calls(op, layers, buf, P, torch, per_call=1):
     sb = [{n: torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev)
            for n, x in lay0.items()} for _ in range(npos)]
     gsc = [[torch.empty(1, dtype=torch.float32, device=dev) for _ in G] for _ in range(npos)]
+    general = None
+    if op == "fp8_block_requant_general":
+        general = [{n: W.random_code_bytes(tuple(x.shape), seed=9000 + 16 * i + t, max_mag=0x7D, device=dev)
+                    for t, (n, x) in enumerate(layers[i].items())} for i in range(len(layers))]
     calls = []
     for i0 in range(0, len(layers), per_call):
         idx = list(range(i0, min(i0 + per_call, len(layers))))
@@ -402,7 +411,9 @@ def next_calls(op, layers, buf, P, torch, per_call=1):
         gts = [(i, k, j) for k, i in enumerate(idx) for j in range(len(G))]
         qs = [buf.fp8[i][n][0] for i, k, n in ts]
         ss = [buf.fp8[i][n][1] for i, k, n in ts]
-        if op == "fp8_block_requant":
+        if op == "fp8_block_requant_general":
+            qs = [general[i][n] for i, k, n in ts]
+        if op in ("fp8_block_requant", "fp8_block_requant_general"):
             calls.append(lambda qs=qs, ss=ss, o=[out_q[k][n] for i, k, n in ts], so=[out_s[k][n] for i, k, n in ts]:
                          P.fp8_block_requant_grouped(qs, ss, out=o, scale_out=so))
         elif op == "fp8_block_requant_mxfp8":

@@ -302,7 +302,7 @@ fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
     __shared__ __align__(8) uint64_t bars[kRqStages];
     __shared__ TileLoc meta[kRqStages];
     __shared__ uint32_t red[2][kThreads / 32];
-    __shared__ __align__(16) uint8_t lut[256];   // per tile: input code -> output code
+    __shared__ __align__(16) uint8_t lut[128];   // per tile: input magnitude -> output code
 
     const uint32_t tid = threadIdx.x;
     const uint32_t pad = (1024u - (smem_addr(smem) & 1023u)) & 1023u;
@@ -372,33 +372,65 @@ fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
         for (int w = 1; w < kThreads / 32; ++w) mc = max(mc, red[it & 1u][w]);
         const float s2 = fp8_tile_scale(__uint_as_float(fp8_amax_bits16(mc, sc) << 16));
         // Within a tile every output code is a function of the input code
-        // alone (y = bf16(fl(dec(q) * s)), q' = e4m3(fl(y / s2))), so each
-        // thread encodes one of the 256 codes into a table and every element
-        // is mapped through it: the per-element arithmetic of the kernel
-        // becomes a byte lookup.  The table entry uses the same quotient
-        // path (reciprocal or IEEE, chosen by s2) as the per-element form.
+        // alone (y = bf16(fl(dec(q) * s)), q' = e4m3(fl(y / s2))), so the
+        // codes are mapped through a per-tile table and the per-element
+        // arithmetic becomes a byte lookup.  Every step is symmetric in sign
+        // (a product, RNE to BF16, a quotient whose zero-divisor case keeps
+        // the sign of zero, RNE to E4M3), so the map of code q ^ 0x80 is the
+        // map of q with the sign bit flipped: the table holds the 128
+        // magnitudes (thread m encodes magnitude m, with the same quotient
+        // path, reciprocal or IEEE chosen by s2, as the per-element form),
+        // one byte per shared-memory bank word position, so a warp's lookups
+        // never conflict, and the input sign bit is xor-ed into the result.
+        //
+        // When the table is the identity on every non-NaN magnitude the
+        // tile's codes are copied unchanged.  That is the usual case, not a
+        // special one: if the tile's largest magnitude code is 448 (every
+        // tile a quantiser writes) then s2 = fl(bf16(fl(448 s)) / 448) and
+        // each quotient is dec(q) times a factor within about 2^-8 of 1, far
+        // inside the half-step of E4M3 (2^-5 relative, 2^-10 absolute for
+        // subnormal codes), so every code maps to itself.  The decision is
+        // taken from the computed table, not from that argument.  The NaN
+        // magnitude 0x7F is left out of the test: a tile holding a NaN code
+        // has a NaN s2 and a table that is not the identity anywhere else.
+        bool ident;
         {
-            const bool fast = div_fast_ok(s2);   // CTA-uniform
-            const float r2 = fast ? __frcp_rn(s2) : 0.0f;
-            const float y = __uint_as_float((pack_bf16x2(__fmul_rn(e4m3_decode(tid), sc), 0.0f) & 0xffffu) << 16);
-            const float q = fast ? div_fast(y, s2, r2) : div_slow(y, s2);
-            // one table: every thread finished mapping the previous tile
-            // before the barrier above
-            lut[tid] = (uint8_t)(e4m3x2(q, 0.0f) & 0xffu);
-        }
-        __syncthreads();   // the table is complete
-        uint2 out[kChunksPerThread];
-#pragma unroll
-        for (int j = 0; j < kChunksPerThread; ++j) {
-            const uint32_t w[2] = {v[j].x, v[j].y};
-            uint32_t o[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t b0 = lut[__byte_perm(w[h], 0u, 0x4440u)], b1 = lut[__byte_perm(w[h], 0u, 0x4441u)];
-                const uint32_t b2 = lut[__byte_perm(w[h], 0u, 0x4442u)], b3 = lut[__byte_perm(w[h], 0u, 0x4443u)];
-                o[h] = __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u);
+            uint32_t code = 0u;
+            if (tid < 128u) {
+                const bool fast = div_fast_ok(s2);   // CTA-uniform
+                const float r2 = fast ? __frcp_rn(s2) : 0.0f;
+                const float y =
+                    __uint_as_float((pack_bf16x2(__fmul_rn(e4m3_decode(tid), sc), 0.0f) & 0xffffu) << 16);
+                const float q = fast ? div_fast(y, s2, r2) : div_slow(y, s2);
+                code = e4m3x2(q, 0.0f) & 0xffu;
+                // one table: every thread finished mapping the previous tile
+                // before the barrier above
+                lut[tid] = (uint8_t)code;
             }
-            out[j] = make_uint2(o[0], o[1]);
+            // the table is complete, and whether it is the identity is known
+            ident = __syncthreads_and(tid >= 127u || code == tid) != 0;
+        }
+        uint2 out[kChunksPerThread];
+        if (ident) {
+#pragma unroll
+            for (int j = 0; j < kChunksPerThread; ++j) out[j] = v[j];
+        } else {
+#pragma unroll
+            for (int j = 0; j < kChunksPerThread; ++j) {
+                const uint32_t w[2] = {v[j].x, v[j].y};
+                uint32_t o[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t mag = w[h] & 0x7f7f7f7fu;
+                    const uint32_t b0 = lut[__byte_perm(mag, 0u, 0x4440u)];
+                    const uint32_t b1 = lut[__byte_perm(mag, 0u, 0x4441u)];
+                    const uint32_t b2 = lut[__byte_perm(mag, 0u, 0x4442u)];
+                    const uint32_t b3 = lut[__byte_perm(mag, 0u, 0x4443u)];
+                    o[h] = __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u) ^
+                           (w[h] & 0x80808080u);
+                }
+                out[j] = make_uint2(o[0], o[1]);
+            }
         }
 
         const TileTensor& T = a.t[L.i];

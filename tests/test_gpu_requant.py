@@ -26,13 +26,14 @@ def P():
     return P
 
 
-def codes_and_scales(shape, seed, raw=False):
-    """(codes uint8 numpy, scales float32 numpy) of an FP8 block-wise tensor."""
+def codes_and_scales(shape, seed, raw=False, max_mag=0x7E):
+    """(codes uint8 numpy, scales float32 numpy) of an FP8 block-wise tensor;
+    raw codes have magnitudes 0..max_mag."""
     rng = np.random.default_rng(seed)
     B, M, N = (1,) + tuple(shape) if len(shape) == 2 else tuple(shape)
     TM, TN = -(-M // 128), -(-N // 128)
     if raw:
-        q = rng.integers(0, 0x7F, size=(B, M, N), dtype=np.uint8) | (rng.integers(0, 2, size=(B, M, N),
+        q = rng.integers(0, max_mag + 1, size=(B, M, N), dtype=np.uint8) | (rng.integers(0, 2, size=(B, M, N),
                                                                                    dtype=np.uint8) << 7)
         s = rng.uniform(1e-5, 1e-1, size=(B, TM, TN)).astype(np.float32)
         flat = s.reshape(-1)
@@ -76,6 +77,24 @@ def test_fp8_to_fp8_in_place(P):
     P.fp8_block_requant(tq, ts, inplace=True)
     oq, os_ = O.fp8_block_requant(q, s)
     assert np.array_equal(u8(tq), oq) and np.array_equal(f32bits(ts), os_.view(np.uint32))
+
+
+@pytest.mark.parametrize("max_mag", [0x7D, 0x70, 0x38, 0x06])
+def test_fp8_to_fp8_tiles_below_448(P, max_mag):
+    """Tiles whose largest code is below 448 change their codes (the per-tile
+    code map is not the identity: normal, subnormal-only and mixed tiles),
+    side by side in one launch with tiles that hold 448 (whose codes come
+    back unchanged)."""
+    q, s = codes_and_scales((3, 256, 384), seed=40 + max_mag, raw=True, max_mag=max_mag)
+    qf, sf = codes_and_scales((3, 256, 384), seed=41, raw=False)
+    q[:, :128, :] = qf[:, :128, :]
+    s[:, 0, :] = sf[:, 0, :]
+    s[1] = -s[1]                                   # negative scales flip signs
+    oq, os_ = O.fp8_block_requant(q, s)
+    assert not np.array_equal(oq[:, 128:, :], q[:, 128:, :])
+    gq, gs = P.fp8_block_requant(to_gpu_codes(q), torch.from_numpy(s).to(DEV))
+    assert np.array_equal(u8(gq), oq)
+    assert np.array_equal(f32bits(gs), os_.view(np.uint32))
 
 
 MX_SHAPES = [((130, 256), False, 0), ((3, 129, 160), True, 16), ((1, 32), True, 0), ((2, 300, 1024), False, 32)]

@@ -54,6 +54,30 @@ def test_fp8_power_of_two_scales_round_trip(shape):
     assert np.array_equal(s2.view(np.uint32), s.view(np.uint32))
 
 
+@pytest.mark.parametrize("shape", [(1, 256, 384), (3, 130, 200)])
+def test_fp8_tiles_holding_448_map_codes_to_themselves(shape):
+    """Any scale with normal products, not only powers of two: when a tile
+    holds a +-448 code, y = dec(q) * s * (1 + d) with |d| <= 2^-8 (one BF16
+    rounding), the new scale is fl(bf16(fl(448 s)) / 448), and each quotient
+    is dec(q) times a factor within about 2^-7 of 1, inside the half-step of
+    E4M3 (at least 2^-5 relative for normal codes, 2^-10 absolute for
+    subnormal ones): every code comes back unchanged.  The expected scale is
+    formed with numpy binary32 and torch's BF16 rounding."""
+    import torch
+    q = random_codes(shape, seed=21)
+    rng = np.random.default_rng(22)
+    s = np.exp2(rng.uniform(-100.0, 100.0, size=tile_shape(q))).astype(np.float32)
+    s *= np.where(rng.integers(0, 2, size=s.shape) == 1, np.float32(-1.0), np.float32(1.0))
+    q2, s2 = O.fp8_block_requant(q, s)
+    assert np.array_equal(q2 & 0x7F, q & 0x7F)
+    # a negative scale flips every sign (the sign of zero included)
+    flip = np.repeat(np.repeat(s < 0, 128, axis=1), 128, axis=2)[:, :q.shape[1], :q.shape[2]]
+    assert np.array_equal(q2, np.where(flip, q ^ 0x80, q))
+    top = np.float32(448.0) * np.abs(s)
+    top_bf16 = torch.from_numpy(top).to(torch.bfloat16).to(torch.float32).numpy()
+    assert np.array_equal(s2.view(np.uint32), (top_bf16 / np.float32(448.0)).astype(np.float32).view(np.uint32))
+
+
 def test_mxfp8_power_of_two_scales_keep_codes_of_full_blocks():
     q = random_codes((1, 128, 256), seed=13, with_max=False)
     q[:, :, ::32] = 0x7E                                             # every 1x32 block holds 448

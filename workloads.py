@@ -149,6 +149,15 @@ def random_bf16(shape, seed: int, std: float = 1.0, device="cpu") -> torch.Tenso
     return normal_bf16(shape, std, seed=seed, device=device)
 
 
+def random_code_bytes(shape, seed: int, max_mag: int, device="cpu") -> torch.Tensor:
+    """Uniform random 8-bit code bytes: low seven bits 0..max_mag, random top
+    (sign) bit; uint8."""
+    g = _gen(seed, device)
+    mag = torch.randint(0, max_mag + 1, shape, generator=g, device=device, dtype=torch.uint8)
+    sign = torch.randint(0, 2, shape, generator=g, device=device, dtype=torch.uint8)
+    return mag | (sign << 7)
+
+
 def bits(x: torch.Tensor):
     """BF16 tensor -> numpy uint16 bit patterns (host copy)."""
     return x.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")
