@@ -383,22 +383,25 @@ NEXT_ONE_PASS_BYTES_PER_ELEM = {"fp8_block_requant_nvfp4": 1 + 4 / 16384 + 0.5 +
 def next_calls(op, layers, buf, P, torch, per_call=1):
     """One grouped call per `per_call` layers (their tensors; for NVFP4 their
     sibling groups in one single-pass launch), reading the FP8 codes and
-    scales the step wrote; one output set per layer position of a call."""
+    scales the step wrote; every layer writes its own outputs (no call
+    writes over lines a previous call left in L2)."""
     import workloads as W
     lay0 = layers[0]
     dev = lay0["q_proj"].device
     names = list(lay0)
     G = W.QWEN3_4B_GROUPS
-    npos = min(per_call, len(layers))
-    out_q = [{n: torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev) for n, x in lay0.items()}
-             for _ in range(npos)]
+    npos = len(layers)
+    nv = op == "fp8_block_requant_nvfp4"
+
+    def per_layer(make, want):
+        return [{n: make(x) for n, x in lay0.items()} for _ in range(npos)] if want else None
+
+    out_q = per_layer(lambda x: torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev), not nv)
     out_s = [{n: torch.empty_like(buf.fp8[0][n][1]) for n in names} for _ in range(npos)]
-    out_e = [{n: torch.empty((x.shape[0], x.shape[1] // 32), dtype=torch.uint8, device=dev) for n, x in lay0.items()}
-             for _ in range(npos)]
-    pk = [{n: torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for n, x in lay0.items()}
-          for _ in range(npos)]
-    sb = [{n: torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev)
-           for n, x in lay0.items()} for _ in range(npos)]
+    out_e = per_layer(lambda x: torch.empty((x.shape[0], x.shape[1] // 32), dtype=torch.uint8, device=dev),
+                      op == "fp8_block_requant_mxfp8")
+    pk = per_layer(lambda x: torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev), nv)
+    sb = per_layer(lambda x: torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev), nv)
     gsc = [[torch.empty(1, dtype=torch.float32, device=dev) for _ in G] for _ in range(npos)]
     general = None
     if op == "fp8_block_requant_general":
@@ -414,17 +417,17 @@ def next_calls(op, layers, buf, P, torch, per_call=1):
         if op == "fp8_block_requant_general":
             qs = [general[i][n] for i, k, n in ts]
         if op in ("fp8_block_requant", "fp8_block_requant_general"):
-            calls.append(lambda qs=qs, ss=ss, o=[out_q[k][n] for i, k, n in ts], so=[out_s[k][n] for i, k, n in ts]:
+            calls.append(lambda qs=qs, ss=ss, o=[out_q[i][n] for i, k, n in ts], so=[out_s[i][n] for i, k, n in ts]:
                          P.fp8_block_requant_grouped(qs, ss, out=o, scale_out=so))
         elif op == "fp8_block_requant_mxfp8":
-            calls.append(lambda qs=qs, ss=ss, o=[out_q[k][n] for i, k, n in ts], eo=[out_e[k][n] for i, k, n in ts]:
+            calls.append(lambda qs=qs, ss=ss, o=[out_q[i][n] for i, k, n in ts], eo=[out_e[i][n] for i, k, n in ts]:
                          P.fp8_block_requant_mxfp8_grouped(qs, ss, out=o, scale_out=eo))
         else:
             calls.append(lambda gq=[[buf.fp8[i][n][0] for n in G[j]] for i, k, j in gts],
                          gs=[[buf.fp8[i][n][1] for n in G[j]] for i, k, j in gts],
-                         o=[[pk[k][n] for n in G[j]] for i, k, j in gts],
-                         so=[[sb[k][n] for n in G[j]] for i, k, j in gts],
-                         gso=[gsc[k][j] for i, k, j in gts]:
+                         o=[[pk[i][n] for n in G[j]] for i, k, j in gts],
+                         so=[[sb[i][n] for n in G[j]] for i, k, j in gts],
+                         gso=[gsc[i][j] for i, k, j in gts]:
                          P.fp8_block_requant_nvfp4_grouped(gq, gs, out=o, sb=so, global_scale=gso))
     return calls
 
