@@ -9,16 +9,18 @@
 // (one decoder layer's weights, say) and walk the concatenation of their
 // tiles with a persistent grid, so a whole list costs one launch.
 //
-// Quantise: 2 CTAs per SM.  Each tile is brought into shared memory by one
-// 3-D TMA box load (cp.async.bulk.tensor, no multicast) from its tensor's
-// map; the out-of-range part of an edge tile is zero-filled, and zeros never
-// raise the amax, so the load side needs no masking.  A ring of kStages tile
-// buffers keeps the next tiles in flight while the current one is reduced:
-// every thread copies its 64 elements to registers, one barrier publishes
-// the warp maxima and frees the buffer, which is refilled at once, and the
-// codes are computed from registers with one correctly rounded reciprocal
-// per tile plus an FMA residual correction per element (proved to give the
-// IEEE-division codes by the exhaustive self-test).
+// Quantise: one 512-thread CTA per SM over pairs of horizontally adjacent
+// tiles.  Each pair is brought into shared memory by one 3-D TMA box load
+// (cp.async.bulk.tensor, no multicast, 128 rows x 256 columns) from its
+// tensor's map; the out-of-range part of an edge box is zero-filled, and
+// zeros never raise the amax, so the load side needs no masking.  A ring of
+// kPairStages box buffers keeps the next pairs in flight while the current
+// one is reduced: every thread copies its 64 elements to registers, one
+// barrier publishes the warp maxima and frees the buffer, which is refilled
+// at once, and each half of the CTA computes its tile's codes from
+// registers with one correctly rounded reciprocal per tile plus an FMA
+// residual correction per element (proved to give the IEEE-division codes
+// by the exhaustive self-test).
 #include <algorithm>
 #include <cuda.h>
 
@@ -29,7 +31,6 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kThreads = 256;
-constexpr int kStages = 3;
 constexpr int kTileBytes = kTile * kTile * 2;  // BF16
 constexpr int kChunksPerThread = kTile * kTile / 8 / kThreads;  // 8
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
@@ -49,6 +50,9 @@ struct TileTensor {
     FastDiv tiles_n;      // tiles per tile row (TN)
     FastDiv tiles_mn;     // tiles per batch matrix (TM * TN)
     int q16, y32;         // dequant: code rows 16-byte, BF16 rows 32-byte aligned
+    uint32_t pair_begin;  // quantise: first tile pair of this tensor in the launch
+    FastDiv pairs_n;      // quantise: tile pairs per tile row (ceil(TN / 2))
+    FastDiv pairs_mn;     // quantise: tile pairs per batch matrix (TM * ceil(TN / 2))
 };
 
 struct TileLoc {
@@ -96,12 +100,46 @@ __device__ __forceinline__ void encode_chunks(const uint4 (&v)[kChunksPerThread]
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+// Quantise kernel: one CTA per SM takes pairs of horizontally adjacent tiles
+// (one 3-D TMA box of 128 rows x 256 columns, 512 contiguous bytes per row;
+// the tile walk reads memory in longer contiguous pieces than a box per
+// tile, which the DRAM serves more efficiently).  Threads 0..255 own the
+// left tile, 256..511 the right one, each half exactly as one tile's worth
+// of work: 64 elements per thread.  A right tile beyond the tensor's last
+// tile column (an odd tile count) is zero-filled by the load and skipped.
+constexpr int kPairThreads = 2 * kThreads;
+constexpr int kPairStages = 3;
+constexpr int kPairCols = 2 * kTile;
+constexpr int kPairBytes = kTile * kPairCols * 2;  // BF16
+
+struct PairLoc {
+    int i;                // tensor
+    int b, tm, tp;        // batch, tile row, tile pair (tiles 2 tp, 2 tp + 1)
+};
+
+__device__ __forceinline__ PairLoc locate_pair(const QuantArgs& a, uint32_t pair) {
+    int i = 0;
+    for (int k = 1; k < a.n; ++k)
+        if (pair >= a.t[k].pair_begin) i = k;
+    const TileTensor& T = a.t[i];
+    PairLoc L;
+    L.i = i;
+    const uint32_t lp = pair - T.pair_begin;
+    const uint32_t b = fdiv(lp, T.pairs_mn);
+    const uint32_t rem = lp - b * T.pairs_mn.d;
+    const uint32_t tm = fdiv(rem, T.pairs_n);
+    L.b = (int)b;
+    L.tm = (int)tm;
+    L.tp = (int)(rem - tm * T.pairs_n.d);
+    return L;
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1)
 fp8_block_quant_kernel(const __grid_constant__ QuantArgs a) {
     extern __shared__ unsigned char smem[];
-    __shared__ __align__(8) uint64_t bars[kStages];
-    __shared__ TileLoc meta[kStages];
-    __shared__ uint32_t red[2][kThreads / 32];
+    __shared__ __align__(8) uint64_t bars[kPairStages];
+    __shared__ PairLoc meta[kPairStages];
+    __shared__ uint32_t red[2][kPairThreads / 32];
 
     const uint32_t tid = threadIdx.x;
     // the ring starts at the first 1024-byte boundary of dynamic shared memory
@@ -109,47 +147,49 @@ fp8_block_quant_kernel(const __grid_constant__ QuantArgs a) {
     unsigned char* ring = smem + pad;
     const uint32_t smem0 = smem_addr(ring);
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+        for (int s = 0; s < kPairStages; ++s) mbar_init(smem_addr(&bars[s]), 1);
         fence_mbar_init();
     }
     __syncthreads();
 
-    // thread 0 locates a tile, records it for the consumers (visible to them
-    // once they observe the barrier phase) and starts its TMA load
-    auto issue = [&](uint32_t t, uint32_t s) {
-        const TileLoc L = locate(a, t);
+    // thread 0 locates a tile pair, records it for the consumers (visible to
+    // them once they observe the barrier phase) and starts its TMA load
+    auto issue = [&](uint32_t p, uint32_t s) {
+        const PairLoc L = locate_pair(a, p);
         meta[s] = L;
         const uint32_t bar = smem_addr(&bars[s]);
-        mbar_arrive_expect_tx(bar, kTileBytes);
-        tma_load_3d(smem0 + s * kTileBytes, &a.tmap[L.i], bar, L.tn * kTile, L.tm * kTile, L.b);
+        mbar_arrive_expect_tx(bar, kPairBytes);
+        tma_load_3d(smem0 + s * kPairBytes, &a.tmap[L.i], bar, L.tp * kPairCols, L.tm * kTile, L.b);
     };
 
     const uint32_t first = blockIdx.x, step = gridDim.x;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            const uint32_t t = first + (uint32_t)s * step;
-            if (t < a.total_tiles) issue(t, (uint32_t)s);
+        for (int s = 0; s < kPairStages; ++s) {
+            const uint32_t p = first + (uint32_t)s * step;
+            if (p < a.total_tiles) issue(p, (uint32_t)s);
         }
     }
 
-    // thread -> (row, 16-byte column chunk) pairs: chunk j covers row
-    // (tid >> 4) + 16 j, columns (tid & 15) * 8 .. + 7
-    const int ccol = (int)(tid & 15u) * 8;
-    const int row0 = (int)(tid >> 4);
+    // half h of the CTA owns tile 2 tp + h; within it, thread -> (row,
+    // 16-byte column chunk) pairs: chunk j covers row (lt >> 4) + 16 j,
+    // columns (lt & 15) * 8 .. + 7 of the tile
+    const uint32_t h = tid >> 8, lt = tid & 255u;
+    const int ccol = (int)(lt & 15u) * 8;
+    const int row0 = (int)(lt >> 4);
 
     uint32_t it = 0;
-    for (uint32_t t = first; t < a.total_tiles; t += step, ++it) {
-        const uint32_t s = it % kStages;
-        const uint32_t parity = (it / kStages) & 1u;
+    for (uint32_t p = first; p < a.total_tiles; p += step, ++it) {
+        const uint32_t s = it % kPairStages;
+        const uint32_t parity = (it / kPairStages) & 1u;
         const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), parity, kWaitLimitNs);
-        const unsigned char* buf = ring + s * kTileBytes;
-        const TileLoc L = meta[s];
+        const unsigned char* buf = ring + s * kPairBytes + h * (kTile * 2);
+        const PairLoc L = meta[s];
         uint4 v[kChunksPerThread];
         uint32_t m = 0u;
 #pragma unroll
         for (int j = 0; j < kChunksPerThread; ++j) {
             v[j] = make_uint4(0u, 0u, 0u, 0u);
-            if (ok) v[j] = *reinterpret_cast<const uint4*>(buf + (row0 + 16 * j) * (kTile * 2) + ccol * 2);
+            if (ok) v[j] = *reinterpret_cast<const uint4*>(buf + (row0 + 16 * j) * (kPairCols * 2) + ccol * 2);
             m = max(m, amax_bits8(v[j]));
         }
 #pragma unroll
@@ -161,35 +201,37 @@ fp8_block_quant_kernel(const __grid_constant__ QuantArgs a) {
             if (tid == 0) {
                 atomicOr(&g_device_error, kErrTmaTimeout);
                 // let every issued copy land before shared memory is released
-                for (uint32_t k = 0; k < (uint32_t)kStages; ++k) {
-                    if (t + k * step < a.total_tiles)
-                        (void)mbar_wait_bounded(smem_addr(&bars[(it + k) % kStages]),
-                                                ((it + k) / kStages) & 1u, kWaitLimitNs);
+                for (uint32_t k = 0; k < (uint32_t)kPairStages; ++k) {
+                    if (p + k * step < a.total_tiles)
+                        (void)mbar_wait_bounded(smem_addr(&bars[(it + k) % kPairStages]),
+                                                ((it + k) / kPairStages) & 1u, kWaitLimitNs);
                 }
             }
             return;
         }
         if (tid == 0) {
-            const uint32_t tn = t + (uint32_t)kStages * step;
-            if (tn < a.total_tiles) issue(tn, s);
+            const uint32_t pn = p + (uint32_t)kPairStages * step;
+            if (pn < a.total_tiles) issue(pn, s);
         }
-        uint32_t am = red[it & 1u][0];
+        const TileTensor& T = a.t[L.i];
+        const int tn = 2 * L.tp + (int)h;
+        if (tn >= (int)T.tiles_n.d) continue;   // uniform over the half: no right tile
+        uint32_t am = red[it & 1u][h * 8u];
 #pragma unroll
-        for (int w = 1; w < kThreads / 32; ++w) am = max(am, red[it & 1u][w]);
+        for (int w = 1; w < kThreads / 32; ++w) am = max(am, red[it & 1u][h * 8u + w]);
 
         const float sc = fp8_tile_scale(__uint_as_float(am << 16));
         const float rc = __frcp_rn(sc);
         uint2 out[kChunksPerThread];
-        if (div_fast_ok(sc))   // CTA-uniform
+        if (div_fast_ok(sc))   // uniform over the half
             encode_chunks<true>(v, sc, rc, out);
         else
             encode_chunks<false>(v, sc, rc, out);
 
-        const TileTensor& T = a.t[L.i];
-        if (tid == 0) T.scale[L.lt] = sc;
+        if (lt == 0) T.scale[(uint32_t)L.b * T.tiles_mn.d + (uint32_t)L.tm * T.tiles_n.d + (uint32_t)tn] = sc;
         const int rows_here = min(kTile, T.rows - L.tm * kTile);
-        const int cols_here = min(kTile, T.cols - L.tn * kTile);
-        char* qtile = T.q + (int64_t)L.b * T.q_bs + (int64_t)L.tm * kTile * T.q_rs + (int64_t)L.tn * kTile;
+        const int cols_here = min(kTile, T.cols - tn * kTile);
+        char* qtile = T.q + (int64_t)L.b * T.q_bs + (int64_t)L.tm * kTile * T.q_rs + (int64_t)tn * kTile;
         if (rows_here == kTile && cols_here == kTile) {
 #pragma unroll
             for (int j = 0; j < kChunksPerThread; ++j)
@@ -496,6 +538,10 @@ uint32_t fill_tile_tensor(TileTensor& T, const Job& j, bool quant, uint32_t tile
     T.tile_begin = tile_begin;
     T.tiles_n = make_fastdiv(tn);
     T.tiles_mn = make_fastdiv(tm * tn);
+    const uint32_t tp = (tn + 1) / 2;
+    T.pair_begin = 0;
+    T.pairs_n = make_fastdiv(tp);
+    T.pairs_mn = make_fastdiv(tm * tp);
     T.q16 = (uintptr_t)q.ptr % 16 == 0 && q.rstride % 16 == 0 && (q.batch == 1 || q.bstride % 16 == 0);
     T.y32 = !quant && (uintptr_t)j.out.ptr % 32 == 0 && j.out.rstride % 32 == 0 &&
             (j.out.batch == 1 || j.out.bstride % 32 == 0);
@@ -514,7 +560,7 @@ cudaError_t read_and_clear_device_error(uint32_t* code) {
 cudaError_t launch_fp8_block_quant(const Job* jobs, int n, cudaStream_t s) {
     EncodeTiledFn encode = encode_tiled_fn();
     if (!encode) return cudaErrorNotSupported;
-    const size_t smem = (size_t)kStages * kTileBytes + 1024;
+    const size_t smem = (size_t)kPairStages * kPairBytes + 1024;
     static int configured[64] = {0};
     const int dev = current_device();
     if (dev >= 0 && dev < 64 && !configured[dev]) {
@@ -526,25 +572,28 @@ cudaError_t launch_fp8_block_quant(const Job* jobs, int n, cudaStream_t s) {
     for (int j0 = 0; j0 < n; j0 += kMaxLaunchTensors) {
         QuantArgs a;
         a.n = std::min(n - j0, kMaxLaunchTensors);
-        uint32_t tiles = 0;
+        uint32_t pairs = 0;
         for (int k = 0; k < a.n; ++k) {
             const Job& j = jobs[j0 + k];
             const View& x = j.in;
             const cuuint64_t dims[3] = {(cuuint64_t)x.cols, (cuuint64_t)x.rows, (cuuint64_t)x.batch};
             const cuuint64_t strides[2] = {(cuuint64_t)x.rstride,
                                            (cuuint64_t)(x.batch > 1 ? x.bstride : x.rows * x.rstride)};
-            const cuuint32_t box[3] = {kTile, kTile, 1};
+            const cuuint32_t box[3] = {kPairCols, kTile, 1};
             const cuuint32_t estr[3] = {1, 1, 1};
             CUresult cr = encode(&a.tmap[k], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x.ptr, dims, strides, box, estr,
                                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
             if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-            tiles += fill_tile_tensor(a.t[k], j, true, tiles);
+            TileTensor& T = a.t[k];
+            fill_tile_tensor(T, j, true, 0);
+            T.pair_begin = pairs;
+            pairs += (uint32_t)x.batch * T.pairs_mn.d;
         }
-        a.total_tiles = tiles;
-        if (tiles == 0) continue;
-        const int grid = (int)std::min<int64_t>(tiles, (int64_t)sm_count(dev) * 2);
-        fp8_block_quant_kernel<<<grid, kThreads, smem, s>>>(a);
+        a.total_tiles = pairs;   // work units of this kernel: tile pairs
+        if (pairs == 0) continue;
+        const int grid = (int)std::min<int64_t>(pairs, (int64_t)sm_count(dev));
+        fp8_block_quant_kernel<<<grid, kPairThreads, smem, s>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
