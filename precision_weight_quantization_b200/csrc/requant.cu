@@ -236,8 +236,12 @@ __global__ void __launch_bounds__(kThreads) fp8_requant_mxfp8_kernel(const __gri
     }
 }
 
-// Grouped FP8 -> MXFP8 (16-byte aligned code rows): one lane per 1x32
-// block, two 16-byte loads and two 16-byte stores.
+// Grouped FP8 -> MXFP8 (16-byte aligned code rows): each lane takes
+// kMxBlocksPerLane 1x32 blocks a warp span apart, loading all their codes
+// (two 16-byte loads each) and tile scales before encoding any, then two
+// 16-byte stores and a scale byte per block.  One block per lane measured
+// 1.43 ms per 36-layer sweep, two 1.32, four 1.27, eight (126 registers)
+// 1.49.
 struct MxBlkTensor {
     const char* q;
     char* q2;
@@ -245,11 +249,19 @@ struct MxBlkTensor {
     const float* s;           // [B][TM][TN]
     uint8_t* e;               // dense [B][M][N/32]
     uint32_t chunks;          // 32-code blocks: B * M * N / 32
-    uint32_t slot_begin;      // multiple of 32 (one warp span)
+    uint32_t slot_begin;      // multiple of one warp span (32 kMxBlocksPerLane)
     uint32_t tm, tn;
     FastDiv cpr, rows;        // blocks per row (N / 32), M
     int dense;
 };
+
+// 32-code blocks per lane per step of the block walk (their loads in
+// flight together)
+constexpr uint32_t kMxBlocksPerLane = 4;
+// CTAs launched per SM: about 4 are resident at the 64 registers a lane
+// takes, and the rest start as those finish; measured faster (1.27 against
+// 1.30 ms per 36-layer sweep) than a grid of resident CTAs only
+constexpr int kMxGridPerSm = 8;
 
 struct MxBlkArgs {
     MxBlkTensor t[kMaxLaunchTensors];
@@ -274,38 +286,60 @@ __global__ void __launch_bounds__(kThreads) fp8_requant_mxfp8_block_kernel(const
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-    for (uint32_t slot = gwarp * 32u; slot < a.total_slots; slot += nwarps * 32u) {
+    constexpr uint32_t kSpan = 32u * kMxBlocksPerLane;
+    for (uint32_t slot = gwarp * kSpan; slot < a.total_slots; slot += nwarps * kSpan) {
         int ti = 0;
         for (int k = 1; k < a.n; ++k)
             if (slot >= a.t[k].slot_begin) ti = k;
         const MxBlkTensor& T = a.t[ti];
-        const uint32_t bi = slot - T.slot_begin + lane;   // 32-code block
-        if (bi >= T.chunks) continue;
-        const uint32_t R = fdiv(bi, T.cpr);           // row over all batches
-        const uint32_t k = bi - R * T.cpr.d;          // block within the row
-        const uint32_t b = fdiv(R, T.rows);
-        const uint32_t m = R - b * T.rows.d;
-        int64_t io, oo;
-        if (T.dense) {
-            io = (int64_t)bi * 32;
-            oo = io;
-        } else {
-            io = (int64_t)b * T.q_bs + (int64_t)m * T.q_rs + (int64_t)k * 32;
-            oo = (int64_t)b * T.o_bs + (int64_t)m * T.o_rs + (int64_t)k * 32;
+        // every block's codes and tile scale are loaded before any is used:
+        // kMxBlocksPerLane x 32 bytes in flight per lane
+        uint4 v[kMxBlocksPerLane][2];
+        float sc[kMxBlocksPerLane];
+        uint32_t bis[kMxBlocksPerLane];
+        int64_t oos[kMxBlocksPerLane];
+#pragma unroll
+        for (int u = 0; u < (int)kMxBlocksPerLane; ++u) {
+            const uint32_t bi = slot - T.slot_begin + lane + 32u * u;   // 32-code block
+            bis[u] = bi;
+            v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
+            sc[u] = 0.0f;
+            oos[u] = 0;
+            if (bi >= T.chunks) continue;
+            const uint32_t R = fdiv(bi, T.cpr);           // row over all batches
+            const uint32_t k = bi - R * T.cpr.d;          // block within the row
+            const uint32_t b = fdiv(R, T.rows);
+            const uint32_t m = R - b * T.rows.d;
+            int64_t io;
+            if (T.dense) {
+                io = (int64_t)bi * 32;
+                oos[u] = io;
+            } else {
+                io = (int64_t)b * T.q_bs + (int64_t)m * T.q_rs + (int64_t)k * 32;
+                oos[u] = (int64_t)b * T.o_bs + (int64_t)m * T.o_rs + (int64_t)k * 32;
+            }
+            v[u][0] = ld_stream_v4(T.q + io);
+            v[u][1] = ld_stream_v4(T.q + io + 16);
+            sc[u] = __ldg(T.s + ((int64_t)b * T.tm + (m >> 7)) * T.tn + (k >> 2));
         }
-        uint4 v0 = ld_stream_v4(T.q + io), v1 = ld_stream_v4(T.q + io + 16);
-        const float sc = __ldg(T.s + ((int64_t)b * T.tm + (m >> 7)) * T.tn + (k >> 2));
-        uint32_t lanes = __vmaxu2(e4m3_maxmag_lanes(make_uint2(v0.x, v0.y)), e4m3_maxmag_lanes(make_uint2(v0.z, v0.w)));
-        lanes = __vmaxu2(lanes, __vmaxu2(e4m3_maxmag_lanes(make_uint2(v1.x, v1.y)), e4m3_maxmag_lanes(make_uint2(v1.z, v1.w))));
-        const int e = ue8m0_exponent(fp8_amax_bits16(e4m3_maxmag_fin(lanes), sc));
-        const float inv = exp2i(-e);   // exact power of two
-        const uint2 o0 = mx_encode8(fp8_dequant8(make_uint2(v0.x, v0.y), sc), inv);
-        const uint2 o1 = mx_encode8(fp8_dequant8(make_uint2(v0.z, v0.w), sc), inv);
-        const uint2 o2 = mx_encode8(fp8_dequant8(make_uint2(v1.x, v1.y), sc), inv);
-        const uint2 o3 = mx_encode8(fp8_dequant8(make_uint2(v1.z, v1.w), sc), inv);
-        st_v4(T.q2 + oo, make_uint4(o0.x, o0.y, o1.x, o1.y));
-        st_v4(T.q2 + oo + 16, make_uint4(o2.x, o2.y, o3.x, o3.y));
-        T.e[bi] = (uint8_t)(e + 127);
+#pragma unroll
+        for (int u = 0; u < (int)kMxBlocksPerLane; ++u) {
+            if (bis[u] >= T.chunks) continue;
+            const uint4 v0 = v[u][0], v1 = v[u][1];
+            uint32_t lanes = __vmaxu2(e4m3_maxmag_lanes(make_uint2(v0.x, v0.y)),
+                                      e4m3_maxmag_lanes(make_uint2(v0.z, v0.w)));
+            lanes = __vmaxu2(lanes, __vmaxu2(e4m3_maxmag_lanes(make_uint2(v1.x, v1.y)),
+                                             e4m3_maxmag_lanes(make_uint2(v1.z, v1.w))));
+            const int e = ue8m0_exponent(fp8_amax_bits16(e4m3_maxmag_fin(lanes), sc[u]));
+            const float inv = exp2i(-e);   // exact power of two
+            const uint2 o0 = mx_encode8(fp8_dequant8(make_uint2(v0.x, v0.y), sc[u]), inv);
+            const uint2 o1 = mx_encode8(fp8_dequant8(make_uint2(v0.z, v0.w), sc[u]), inv);
+            const uint2 o2 = mx_encode8(fp8_dequant8(make_uint2(v1.x, v1.y), sc[u]), inv);
+            const uint2 o3 = mx_encode8(fp8_dequant8(make_uint2(v1.z, v1.w), sc[u]), inv);
+            st_v4(T.q2 + oos[u], make_uint4(o0.x, o0.y, o1.x, o1.y));
+            st_v4(T.q2 + oos[u] + 16, make_uint4(o2.x, o2.y, o3.x, o3.y));
+            T.e[bis[u]] = (uint8_t)(e + 127);
+        }
     }
 }
 
@@ -402,7 +436,8 @@ cudaError_t launch_fp8_requant_mxfp8(const RequantJob* jobs, int n, cudaStream_t
             const View& q = J.in;
             const View& q2 = J.out;
             const uint64_t chunks = (uint64_t)(q.batch * q.rows * (q.cols / 32));
-            const uint64_t padded = (chunks + 31) / 32 * 32;
+            const uint64_t span = 32u * kMxBlocksPerLane;
+            const uint64_t padded = (chunks + span - 1) / span * span;
             if (a.n > 0 && slots + padded > kMaxSlots) break;
             MxBlkTensor& T = a.t[a.n];
             T.q = q.ptr;
@@ -426,7 +461,7 @@ cudaError_t launch_fp8_requant_mxfp8(const RequantJob* jobs, int n, cudaStream_t
         j0 += a.n;
         a.total_slots = slots;
         if (slots == 0) continue;
-        const int grid = persistent_grid((slots + kThreads - 1) / kThreads, 8);
+        const int grid = persistent_grid((slots + kThreads * kMxBlocksPerLane - 1) / (kThreads * kMxBlocksPerLane), kMxGridPerSm);
         fp8_requant_mxfp8_block_kernel<<<grid, kThreads, 0, st>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
