@@ -69,7 +69,7 @@ def strided(xbits, pad_cols, dtype_bytes=2):
 # ------------------------------------------------------------------ FP8 block-wise
 
 FP8_SHAPES = [(1, 16), (2, 48), (1, 1), (7, 3), (128, 128), (130, 260), (257, 300), (3, 129, 131),
-              (2, 256, 512), (1000, 8), (64, 1000)]
+              (2, 256, 512), (1000, 8), (64, 1000), (2, 256, 640)]
 
 
 @pytest.mark.parametrize("shape", FP8_SHAPES, ids=str)
