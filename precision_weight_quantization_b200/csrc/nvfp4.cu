@@ -257,10 +257,15 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
     }
 }
 
-// Dequantise: a grouped chunk walk like MXFP8's.  Per 8-element chunk: 4
-// packed bytes in, 16 bytes of BF16 out; the chunk's block scale and its
-// batch index's global scale are cached loads.
-constexpr uint32_t kSpan = 32u * kUnroll;   // chunks per warp span
+// Dequantise: a grouped walk over 16-element blocks like MXFP8's.  Per
+// block: 8 packed bytes in, 32 bytes of BF16 out (one 256-bit store when the
+// BF16 rows are 32-byte aligned); the block scale and the batch index's
+// global scale are cached loads.  A lane loads kDqUnroll blocks, a warp span
+// apart, before storing any: streams that write twice what they read run
+// far below the copy rate with 16-byte stores, and 32-byte stores with more
+// loads in flight close the gap.
+constexpr int kDqUnroll = 8;
+constexpr uint32_t kSpan = 32u * kDqUnroll;   // blocks per warp span
 
 struct DqTensor {
     const char* q;        // packed codes
@@ -268,12 +273,13 @@ struct DqTensor {
     int64_t q_bs, q_rs, y_bs, y_rs;
     const uint8_t* sb;    // dense [B][M][N/16]
     const float* gs;      // [B]
-    uint32_t chunks;      // B * M * N / 8
+    uint32_t blocks;      // B * M * N / 16
     uint32_t slot_begin;  // multiple of kSpan
-    FastDiv cpr;          // chunks per row (N / 8)
-    FastDiv per_batch;    // chunks per batch matrix (M * N / 8)
+    FastDiv bpr;          // blocks per row (N / 16)
+    FastDiv per_batch;    // blocks per batch matrix (M * N / 16)
     FastDiv rows;         // M
     int dense;
+    int y32;              // BF16 base, row and slab strides multiples of 32 bytes
 };
 
 struct DequantArgs {
@@ -292,37 +298,44 @@ __global__ void __launch_bounds__(kThreads) nvfp4_dequant_kernel(const __grid_co
             if (slot >= a.t[k].slot_begin) ti = k;
         const DqTensor& T = a.t[ti];
         const uint32_t base = slot - T.slot_begin;
-        uint32_t codes[kUnroll], sbyte[kUnroll], bidx[kUnroll];
-        int64_t yo[kUnroll];
+        uint2 codes[kDqUnroll];
+        uint32_t sbyte[kDqUnroll], bidx[kDqUnroll];
+        int64_t yo[kDqUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t c = base + u * 32u + lane;
+        for (int u = 0; u < kDqUnroll; ++u) {
+            const uint32_t c = base + u * 32u + lane;   // block
             const uint32_t b = fdiv(c, T.per_batch);
             int64_t qo;
             if (T.dense) {
-                qo = (int64_t)c * 4;
-                yo[u] = (int64_t)c * 16;
+                qo = (int64_t)c * 8;
+                yo[u] = (int64_t)c * 32;
             } else {
-                const uint32_t r = fdiv(c, T.cpr);          // row over all batches
-                const uint32_t k = c - r * T.cpr.d;
+                const uint32_t r = fdiv(c, T.bpr);          // row over all batches
+                const uint32_t k = c - r * T.bpr.d;
                 const uint32_t mrow = r - b * T.rows.d;
-                qo = (int64_t)b * T.q_bs + (int64_t)mrow * T.q_rs + (int64_t)k * 4;
-                yo[u] = (int64_t)b * T.y_bs + (int64_t)mrow * T.y_rs + (int64_t)k * 16;
+                qo = (int64_t)b * T.q_bs + (int64_t)mrow * T.q_rs + (int64_t)k * 8;
+                yo[u] = (int64_t)b * T.y_bs + (int64_t)mrow * T.y_rs + (int64_t)k * 32;
             }
             bidx[u] = b;
-            codes[u] = 0u;
+            codes[u] = make_uint2(0u, 0u);
             sbyte[u] = 0u;
-            if (c < T.chunks) {
-                codes[u] = ld_stream_u32(T.q + qo);
-                sbyte[u] = __ldg(T.sb + (c >> 1));
+            if (c < T.blocks) {
+                codes[u] = ld_stream_v2(T.q + qo);
+                sbyte[u] = __ldg(T.sb + c);
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < kDqUnroll; ++u) {
             const uint32_t c = base + u * 32u + lane;
-            if (c < T.chunks) {
-                const float gs = __ldg(T.gs + bidx[u]);
-                st_v4(T.y + yo[u], dequant_half(codes[u], e4m3_decode(sbyte[u]), gs));
+            if (c >= T.blocks) continue;
+            const float gs = __ldg(T.gs + bidx[u]);
+            const float sbv = e4m3_decode(sbyte[u]);
+            const uint4 y0 = dequant_half(codes[u].x, sbv, gs), y1 = dequant_half(codes[u].y, sbv, gs);
+            if (T.y32) {
+                st_v8(T.y + yo[u], y0, y1);
+            } else {
+                st_v4(T.y + yo[u], y0);
+                st_v4(T.y + yo[u] + 16, y1);
             }
         }
     }
@@ -917,8 +930,8 @@ cudaError_t launch_nvfp4_dequant(const Job* jobs, int n, cudaStream_t s) {
             const Job& j = jobs[j0 + a.n];
             const View& q = j.in;
             const View& y = j.out;
-            const uint64_t chunks = (uint64_t)(q.batch * q.rows * (q.cols / 8));
-            const uint64_t padded = (chunks + kSpan - 1) / kSpan * kSpan;
+            const uint64_t blocks = (uint64_t)(q.batch * q.rows * (q.cols / 16));
+            const uint64_t padded = (blocks + kSpan - 1) / kSpan * kSpan;
             if (a.n > 0 && slots + padded > kMaxSlots) break;
             DqTensor& T = a.t[a.n];
             T.q = q.ptr;
@@ -929,20 +942,21 @@ cudaError_t launch_nvfp4_dequant(const Job* jobs, int n, cudaStream_t s) {
             T.y_rs = y.rstride;
             T.sb = static_cast<const uint8_t*>(j.scale);
             T.gs = j.gs;
-            T.chunks = (uint32_t)chunks;
+            T.blocks = (uint32_t)blocks;
             T.slot_begin = slots;
-            const int64_t cpr = std::max<int64_t>(1, q.cols / 8);
-            T.cpr = make_fastdiv((uint32_t)cpr);
-            T.per_batch = make_fastdiv((uint32_t)std::max<int64_t>(1, q.rows * cpr));
+            const int64_t bpr = std::max<int64_t>(1, q.cols / 16);
+            T.bpr = make_fastdiv((uint32_t)bpr);
+            T.per_batch = make_fastdiv((uint32_t)std::max<int64_t>(1, q.rows * bpr));
             T.rows = make_fastdiv((uint32_t)std::max<int64_t>(1, q.rows));
             T.dense = q.rstride == q.cols / 2 && y.rstride == y.cols * 2 &&
                       (q.batch == 1 || (q.bstride == q.rows * q.rstride && y.bstride == y.rows * y.rstride));
+            T.y32 = (uintptr_t)y.ptr % 32 == 0 && y.rstride % 32 == 0 && (y.batch == 1 || y.bstride % 32 == 0);
             slots += (uint32_t)padded;
         }
         j0 += a.n;
         a.total_slots = slots;
         if (slots == 0) continue;
-        const int grid = persistent_grid((slots + kThreads * kUnroll - 1) / (kThreads * kUnroll), 8);
+        const int grid = persistent_grid((slots + kThreads * kDqUnroll - 1) / (kThreads * kDqUnroll), 8);
         nvfp4_dequant_kernel<<<grid, kThreads, 0, s>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
