@@ -170,12 +170,14 @@ fp8_block_quant_kernel(const __grid_constant__ QuantArgs a) {
         }
     }
 
-    // half h of the CTA owns tile 2 tp + h; within it, thread -> (row,
-    // 16-byte column chunk) pairs: chunk j covers row (lt >> 4) + 16 j,
-    // columns (lt & 15) * 8 .. + 7 of the tile
+    // half h of the CTA owns tile 2 tp + h; within it, thread lt owns 16
+    // consecutive elements of rows (lt >> 3) + 32 i, i = 0..3, at columns
+    // (lt & 7) * 16: chunk j (8 elements) is row (lt >> 3) + 32 (j >> 1),
+    // columns (lt & 7) * 16 + 8 (j & 1), so a row's 16 codes leave in one
+    // 16-byte store
     const uint32_t h = tid >> 8, lt = tid & 255u;
-    const int ccol = (int)(lt & 15u) * 8;
-    const int row0 = (int)(lt >> 4);
+    const int c16 = (int)(lt & 7u) * 16;
+    const int r16 = (int)(lt >> 3);
 
     uint32_t it = 0;
     for (uint32_t p = first; p < a.total_tiles; p += step, ++it) {
@@ -189,7 +191,7 @@ fp8_block_quant_kernel(const __grid_constant__ QuantArgs a) {
 #pragma unroll
         for (int j = 0; j < kChunksPerThread; ++j) {
             v[j] = make_uint4(0u, 0u, 0u, 0u);
-            if (ok) v[j] = *reinterpret_cast<const uint4*>(buf + (row0 + 16 * j) * (kPairCols * 2) + ccol * 2);
+            if (ok) v[j] = *reinterpret_cast<const uint4*>(buf + (r16 + 32 * (j >> 1)) * (kPairCols * 2) + (c16 + 8 * (j & 1)) * 2);
             m = max(m, amax_bits8(v[j]));
         }
 #pragma unroll
@@ -232,14 +234,15 @@ fp8_block_quant_kernel(const __grid_constant__ QuantArgs a) {
         const int rows_here = min(kTile, T.rows - L.tm * kTile);
         const int cols_here = min(kTile, T.cols - tn * kTile);
         char* qtile = T.q + (int64_t)L.b * T.q_bs + (int64_t)L.tm * kTile * T.q_rs + (int64_t)tn * kTile;
-        if (rows_here == kTile && cols_here == kTile) {
+        if (rows_here == kTile && cols_here == kTile && T.q16) {
 #pragma unroll
-            for (int j = 0; j < kChunksPerThread; ++j)
-                st_v2(qtile + (int64_t)(row0 + 16 * j) * T.q_rs + ccol, out[j]);
+            for (int i = 0; i < kChunksPerThread / 2; ++i)
+                st_v4(qtile + (int64_t)(r16 + 32 * i) * T.q_rs + c16,
+                      make_uint4(out[2 * i].x, out[2 * i].y, out[2 * i + 1].x, out[2 * i + 1].y));
         } else {
 #pragma unroll
             for (int j = 0; j < kChunksPerThread; ++j) {
-                const int r = row0 + 16 * j;
+                const int r = r16 + 32 * (j >> 1), ccol = c16 + 8 * (j & 1);
                 if (r >= rows_here || ccol >= cols_here) continue;
                 char* dst = qtile + (int64_t)r * T.q_rs + ccol;
                 if (ccol + 8 <= cols_here) {
