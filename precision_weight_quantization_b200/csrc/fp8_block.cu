@@ -374,8 +374,11 @@ fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
             if (t < a.total_tiles) issue(t, (uint32_t)s);
         }
     }
-    const int ccol = (int)(tid & 15u) * 8;
-    const int row0 = (int)(tid >> 4);
+    // thread -> 16 consecutive codes of rows (tid >> 3) + 32 i, i = 0..3, at
+    // column (tid & 7) * 16; chunk j (8 codes) is row (tid >> 3) + 32 (j >> 1),
+    // columns (tid & 7) * 16 + 8 (j & 1)
+    const int c16 = (int)(tid & 7u) * 16;
+    const int r16 = (int)(tid >> 3);
 
     uint32_t it = 0;
     for (uint32_t t = first; t < a.total_tiles; t += step, ++it) {
@@ -388,10 +391,12 @@ fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
         uint2 v[kChunksPerThread];
         uint32_t m = 0u;
 #pragma unroll
-        for (int j = 0; j < kChunksPerThread; ++j) {
-            v[j] = make_uint2(0u, 0u);
-            if (ok) v[j] = *reinterpret_cast<const uint2*>(buf + (row0 + 16 * j) * kTile + ccol);
-            m = __vmaxu2(m, e4m3_maxmag_lanes(v[j]));
+        for (int i = 0; i < kChunksPerThread / 2; ++i) {
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (ok) w = *reinterpret_cast<const uint4*>(buf + (r16 + 32 * i) * kTile + c16);
+            v[2 * i] = make_uint2(w.x, w.y);
+            v[2 * i + 1] = make_uint2(w.z, w.w);
+            m = __vmaxu2(m, __vmaxu2(e4m3_maxmag_lanes(v[2 * i]), e4m3_maxmag_lanes(v[2 * i + 1])));
         }
         m = e4m3_maxmag_fin(m);
 #pragma unroll
@@ -483,14 +488,15 @@ fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
         const int rows_here = min(kTile, T.rows - L.tm * kTile);
         const int cols_here = min(kTile, T.cols - L.tn * kTile);
         char* qtile = T.q + (int64_t)L.b * T.q_bs + (int64_t)L.tm * kTile * T.q_rs + (int64_t)L.tn * kTile;
-        if (rows_here == kTile && cols_here == kTile) {
+        if (rows_here == kTile && cols_here == kTile && T.q16) {
 #pragma unroll
-            for (int j = 0; j < kChunksPerThread; ++j)
-                st_v2(qtile + (int64_t)(row0 + 16 * j) * T.q_rs + ccol, out[j]);
+            for (int i = 0; i < kChunksPerThread / 2; ++i)
+                st_v4(qtile + (int64_t)(r16 + 32 * i) * T.q_rs + c16,
+                      make_uint4(out[2 * i].x, out[2 * i].y, out[2 * i + 1].x, out[2 * i + 1].y));
         } else {
 #pragma unroll
             for (int j = 0; j < kChunksPerThread; ++j) {
-                const int r = row0 + 16 * j;
+                const int r = r16 + 32 * (j >> 1), ccol = c16 + 8 * (j & 1);
                 if (r >= rows_here || ccol >= cols_here) continue;
                 char* dst = qtile + (int64_t)r * T.q_rs + ccol;
                 if (ccol + 8 <= cols_here) {
@@ -667,6 +673,8 @@ cudaError_t launch_fp8_requant_tma(const RequantJob* jobs, int n, cudaStream_t s
             T.q_bs = J.out.bstride;
             T.q_rs = J.out.rstride;
             T.y_bs = T.y_rs = 0;
+            T.q16 = (uintptr_t)J.out.ptr % 16 == 0 && J.out.rstride % 16 == 0 &&
+                    (J.out.batch == 1 || J.out.bstride % 16 == 0);
             T.scale = static_cast<float*>(J.scale_out);
             T.rows = (int)q.rows;
             T.cols = (int)q.cols;
