@@ -323,6 +323,88 @@ __global__ void __launch_bounds__(kThreads) fp8_block_dequant_kernel(const __gri
     }
 }
 
+// Dequantise by rows: the dequantiser needs no reduction over a tile, so
+// when every tensor of a launch has N % 16 == 0 and 16-byte aligned code
+// rows it streams the rows like the MXFP8 dequantiser instead of walking
+// tiles: 16-code chunks in row-major order (a chunk never leaves its tile:
+// 128 is a multiple of 16), a warp span of 32 consecutive chunks per step,
+// kRowDqUnroll chunks per lane loaded before any is stored, one cached
+// tile-scale load per chunk, 32 bytes of BF16 out per chunk (one 256-bit
+// store when the BF16 rows are 32-byte aligned).
+struct RowDqTensor {
+    const char* q;
+    char* y;
+    int64_t q_bs, q_rs, y_bs, y_rs;   // bytes
+    const float* scale;               // dense [B][TM][TN]
+    uint32_t chunks;                  // B * M * N / 16
+    uint32_t slot_begin;              // multiple of kRowDqSpan
+    FastDiv cpr;                      // chunks per row (N / 16)
+    FastDiv rows;                     // M
+    uint32_t tm, tn;                  // tiles per column / per row
+    int dense;
+    int y32;
+};
+
+struct RowDqArgs {
+    RowDqTensor t[kMaxLaunchTensors];
+    int n;
+    uint32_t total_slots;
+};
+
+constexpr int kRowDqUnroll = 8;
+constexpr uint32_t kRowDqSpan = 32u * kRowDqUnroll;
+
+__global__ void __launch_bounds__(kThreads) fp8_block_dequant_rows_kernel(const __grid_constant__ RowDqArgs a) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t slot = gwarp * kRowDqSpan; slot < a.total_slots; slot += nwarps * kRowDqSpan) {
+        int ti = 0;
+        for (int k = 1; k < a.n; ++k)
+            if (slot >= a.t[k].slot_begin) ti = k;
+        const RowDqTensor& T = a.t[ti];
+        const uint32_t base = slot - T.slot_begin;
+        uint4 v[kRowDqUnroll];
+        float sc[kRowDqUnroll];
+        int64_t yo[kRowDqUnroll];
+#pragma unroll
+        for (int u = 0; u < kRowDqUnroll; ++u) {
+            const uint32_t c = base + u * 32u + lane;
+            const uint32_t r = fdiv(c, T.cpr);            // row over all batches
+            const uint32_t k = c - r * T.cpr.d;           // chunk within the row
+            const uint32_t b = fdiv(r, T.rows);
+            const uint32_t m = r - b * T.rows.d;
+            int64_t qo;
+            if (T.dense) {
+                qo = (int64_t)c * 16;
+                yo[u] = (int64_t)c * 32;
+            } else {
+                qo = (int64_t)b * T.q_bs + (int64_t)m * T.q_rs + (int64_t)k * 16;
+                yo[u] = (int64_t)b * T.y_bs + (int64_t)m * T.y_rs + (int64_t)k * 32;
+            }
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            sc[u] = 0.0f;
+            if (c < T.chunks) {
+                v[u] = ld_stream_v4(T.q + qo);
+                sc[u] = __ldg(T.scale + ((int64_t)b * T.tm + (m >> 7)) * T.tn + (k >> 3));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kRowDqUnroll; ++u) {
+            const uint32_t c = base + u * 32u + lane;
+            if (c >= T.chunks) continue;
+            const uint4 y0 = fp8_dequant8(make_uint2(v[u].x, v[u].y), sc[u]);
+            const uint4 y1 = fp8_dequant8(make_uint2(v[u].z, v[u].w), sc[u]);
+            if (T.y32) {
+                st_v8(T.y + yo[u], y0, y1);
+            } else {
+                st_v4(T.y + yo[u], y0);
+                st_v4(T.y + yo[u] + 16, y1);
+            }
+        }
+    }
+}
+
 // FP8 block-wise -> FP8 block-wise re-quantisation (the composition
 // fp8_block_quant(fp8_block_dequant(q, s)), see requant.cu) with the code
 // tiles staged by TMA like the quantiser's BF16 tiles: 16 KB per tile, a
@@ -609,7 +691,59 @@ cudaError_t launch_fp8_block_quant(const Job* jobs, int n, cudaStream_t s) {
     return cudaSuccess;
 }
 
+// Row-streaming dequantise of a list whose tensors all have N % 16 == 0 and
+// 16-byte aligned code rows.
+cudaError_t launch_fp8_block_dequant_rows(const Job* jobs, int n, cudaStream_t s) {
+    const uint64_t kMaxSlots = uint64_t(1) << 31;   // chunk indices stay 32-bit
+    for (int j0 = 0; j0 < n;) {
+        RowDqArgs a;
+        a.n = 0;
+        uint32_t slots = 0;
+        for (; j0 + a.n < n && a.n < kMaxLaunchTensors; ++a.n) {
+            const Job& j = jobs[j0 + a.n];
+            const View& q = j.in;
+            const View& y = j.out;
+            const uint64_t chunks = (uint64_t)(q.batch * q.rows * (q.cols / 16));
+            const uint64_t padded = (chunks + kRowDqSpan - 1) / kRowDqSpan * kRowDqSpan;
+            if (a.n > 0 && slots + padded > kMaxSlots) break;
+            RowDqTensor& T = a.t[a.n];
+            T.q = q.ptr;
+            T.y = y.ptr;
+            T.q_bs = q.bstride;
+            T.q_rs = q.rstride;
+            T.y_bs = y.bstride;
+            T.y_rs = y.rstride;
+            T.scale = static_cast<const float*>(j.scale);
+            T.chunks = (uint32_t)chunks;
+            T.slot_begin = slots;
+            T.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, q.cols / 16));
+            T.rows = make_fastdiv((uint32_t)std::max<int64_t>(1, q.rows));
+            T.tm = (uint32_t)((q.rows + kTile - 1) / kTile);
+            T.tn = (uint32_t)((q.cols + kTile - 1) / kTile);
+            T.dense = q.rstride == q.cols && y.rstride == y.cols * 2 &&
+                      (q.batch == 1 || (q.bstride == q.rows * q.cols && y.bstride == y.rows * y.cols * 2));
+            T.y32 = (uintptr_t)y.ptr % 32 == 0 && y.rstride % 32 == 0 && (y.batch == 1 || y.bstride % 32 == 0);
+            slots += (uint32_t)padded;
+        }
+        j0 += a.n;
+        a.total_slots = slots;
+        if (slots == 0) continue;
+        const int grid = persistent_grid((slots + kThreads * kRowDqUnroll - 1) / (kThreads * kRowDqUnroll), 8);
+        fp8_block_dequant_rows_kernel<<<grid, kThreads, 0, s>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t launch_fp8_block_dequant(const Job* jobs, int n, cudaStream_t s) {
+    bool rows = true;
+    for (int i = 0; i < n; ++i) {
+        const View& q = jobs[i].in;
+        rows = rows && q.cols % 16 == 0 && (uintptr_t)q.ptr % 16 == 0 && q.rstride % 16 == 0 &&
+               (q.batch == 1 || q.bstride % 16 == 0);
+    }
+    if (rows) return launch_fp8_block_dequant_rows(jobs, n, s);
     for (int j0 = 0; j0 < n; j0 += kMaxLaunchTensors) {
         DequantArgs a;
         a.n = std::min(n - j0, kMaxLaunchTensors);
