@@ -408,11 +408,15 @@ __global__ void __launch_bounds__(kThreads) fp8_block_dequant_rows_kernel(const 
 // FP8 block-wise -> FP8 block-wise re-quantisation (the composition
 // fp8_block_quant(fp8_block_dequant(q, s)), see requant.cu) with the code
 // tiles staged by TMA like the quantiser's BF16 tiles: 16 KB per tile, a
-// ring of kRqStages buffers, 3 CTAs per SM.  Used when every input code
+// ring of kRqStages buffers, 2 CTAs per SM.  The ring depth trades the two
+// per-tile paths against each other (ms per 36-layer sweep, identity tiles /
+// table lookups): 2 CTAs x 6 stages 1.24 / 1.56, 3 x 4 1.41 / 1.42, 4 x 3
+// 1.43 / 1.33; the copy of identity tiles (every tile a quantiser wrote)
+// wants the deep ring, the lookups want warps.  Used when every input code
 // tensor has 16-byte aligned rows (a TMA stride rule); the tile of old
 // scales is read before the CTA's barrier and the new scale written after
 // it, so in-place use is safe.
-constexpr int kRqStages = 4;
+constexpr int kRqStages = 6;
 constexpr int kRqTileBytes = kTile * kTile;   // E4M3
 
 struct RequantTmaArgs {
@@ -423,7 +427,7 @@ struct RequantTmaArgs {
     uint32_t total_tiles;
 };
 
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 2)
 fp8_requant_tma_kernel(const __grid_constant__ RequantTmaArgs a) {
     extern __shared__ unsigned char smem[];
     __shared__ __align__(8) uint64_t bars[kRqStages];
@@ -821,7 +825,7 @@ cudaError_t launch_fp8_requant_tma(const RequantJob* jobs, int n, cudaStream_t s
         j0 += a.n;
         a.total_tiles = tiles;
         if (tiles == 0) continue;
-        const int grid = (int)std::min<int64_t>(tiles, (int64_t)sm_count(dev) * 3);
+        const int grid = (int)std::min<int64_t>(tiles, (int64_t)sm_count(dev) * 2);
         fp8_requant_tma_kernel<<<grid, kThreads, smem, s>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
