@@ -5,9 +5,12 @@
 // "低精度训练与 Rollout", "FP8 训练 + FP8 Rollout" (FP32 block scales; FP8
 // weights dequantised to BF16 on weight update).
 //
-// Both kernels take a list of up to kMaxLaunchTensors independent tensors
-// (one decoder layer's weights, say) and walk the concatenation of their
-// tiles with a persistent grid, so a whole list costs one launch.
+// Every kernel takes a list of up to kMaxLaunchTensors independent tensors
+// (one decoder layer's weights, say) and walks the concatenation of their
+// work units with a persistent grid, so a whole list costs one launch: tile
+// pairs for the quantiser, rows of 16-code chunks for the dequantiser when
+// every tensor has N % 16 == 0 and 16-byte aligned code rows (tiles
+// otherwise), tiles for the FP8 -> FP8 re-quantiser.
 //
 // Quantise: one 512-thread CTA per SM over pairs of horizontally adjacent
 // tiles.  Each pair is brought into shared memory by one 3-D TMA box load
