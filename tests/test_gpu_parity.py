@@ -459,3 +459,45 @@ def test_empty_tensors_are_noops(P):
     q, e = P.mxfp8_quant(x)
     assert q.numel() == 0
     assert P.nvfp4_fake_quant(x).numel() == 0
+
+
+# ------------------------------------------------------------------ strided rows through the streaming dequantisers
+
+def padded_codes(codes, pad):
+    """GPU uint8 view of code bytes [.., M, N] whose rows are padded by pad bytes."""
+    *lead, M, N = codes.shape
+    big = torch.zeros(tuple(lead) + (M, N + pad), dtype=torch.uint8, device=DEV)
+    v = big[..., :N]
+    v.copy_(torch.from_numpy(np.ascontiguousarray(codes)).to(DEV))
+    return v
+
+
+def padded_bf16_out(shape, pad):
+    *lead, M, N = shape
+    big = torch.full(tuple(lead) + (M, N + pad), float("nan"), dtype=torch.bfloat16, device=DEV)
+    return big[..., :N]
+
+
+@pytest.mark.parametrize("shape,pad_q,pad_y", [((3, 130, 256), 16, 8), ((2, 256, 384), 32, 16),
+                                               ((1, 96, 128), 16, 0)], ids=str)
+def test_dequantisers_on_padded_rows(P, shape, pad_q, pad_y):
+    """The row-streaming dequantisers on batched slabs whose code rows are
+    16-byte aligned but not dense, writing BF16 rows that are 16-byte (pad
+    of 8 elements) or 32-byte aligned: bit for bit the oracle's values."""
+    x = rand_bits(shape, seed=sum(shape) + pad_q)
+    oq, os_ = O.fp8_block_quant(x)
+    y = padded_bf16_out(shape, pad_y)
+    P.fp8_block_dequant(padded_codes(oq, pad_q), torch.from_numpy(os_).to(DEV), out=y)
+    assert np.array_equal(u16(y), O.fp8_block_dequant(oq, os_))
+    mq, me = O.mxfp8_quant(x)
+    y = padded_bf16_out(shape, pad_y)
+    P.mxfp8_dequant(padded_codes(mq, pad_q), torch.from_numpy(np.ascontiguousarray(me)).to(DEV), out=y)
+    assert np.array_equal(u16(y), O.mxfp8_dequant(mq, me))
+    per = [O.nvfp4_quant(x[b], O.nvfp4_group_amax([x[b]])) for b in range(shape[0])]
+    pk = np.stack([p[0] for p in per])
+    sb = np.stack([p[1] for p in per])
+    gs = torch.tensor([p[2] for p in per], dtype=torch.float32, device=DEV)
+    y = padded_bf16_out(shape, pad_y)
+    P.nvfp4_dequant(padded_codes(pk, pad_q // 2), torch.from_numpy(sb).to(DEV), gs, out=y)
+    expect = np.stack([O.nvfp4_dequant(per[b][0], per[b][1], per[b][2], shape[-1]) for b in range(shape[0])])
+    assert np.array_equal(u16(y), expect)
