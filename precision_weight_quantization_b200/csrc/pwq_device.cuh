@@ -44,15 +44,6 @@ __device__ __forceinline__ uint32_t amax_bits8(uint4 v) {
     return max(c & 0xffffu, c >> 16);
 }
 
-// The same value by integer SIMD maxes of the masked magnitude bits (more
-// instructions, shorter dependent chain; the MXFP8 quantiser, whose block
-// amax sits on the path of two shuffles, measured faster with it).
-__device__ __forceinline__ uint32_t amax_bits8_int(uint4 v) {
-    const uint32_t m = 0x7fff7fffu;
-    const uint32_t c = __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
-    return max(c & 0xffffu, c >> 16);
-}
-
 // Pack two binary32 into a BF16x2 word (lo in bits 0..15), RNE.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
@@ -375,11 +366,6 @@ __device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
                  : "=r"(v.x), "=r"(v.y) : "l"(p));
     return v;
 }
-__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
 // L2 eviction-priority policies for loads and stores that carry a cache hint.
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     uint64_t p;
@@ -400,9 +386,6 @@ __device__ __forceinline__ uint4 ld_hint_v4(const void* p, uint64_t pol) {
 __device__ __forceinline__ void st_hint_v4(void* p, uint4 v, uint64_t pol) {
     asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;"
                  :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol) : "memory");
-}
-__device__ __forceinline__ void st_hint_u32(void* p, uint32_t v, uint64_t pol) {
-    asm volatile("st.global.L2::cache_hint.u32 [%0], %1, %2;" :: "l"(p), "r"(v), "l"(pol) : "memory");
 }
 
 __device__ __forceinline__ void st_hint_v2(void* p, uint32_t a, uint32_t b, uint64_t pol) {
