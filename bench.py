@@ -516,14 +516,17 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    import datetime
+    if args.impl == "reference":
+        # the reference arm runs on the host alone: its ranks meet over gloo
+        # (no GPU or NCCL involved), rank 0 times the oracle
+        if world > 1:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=900))
+        return main_reference(args, rank, world, torch, dist)
     if world > 1:
-        import datetime
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-
-    if args.impl == "reference":
-        return main_reference(args, rank, world, torch, dist)
 
     import precision_weight_quantization_b200 as P
     dev = torch.device("cuda", local)

@@ -1,5 +1,6 @@
-"""bench.py pieces that need no GPU: the reference arm's JSON line and the
-staleness rule of the recorded ncu traffic."""
+"""bench.py pieces that need no GPU: the reference arm's JSON line (alone and
+under a two-rank torchrun launch) and the staleness rule of the recorded ncu
+traffic."""
 import json
 import os
 import subprocess
@@ -27,6 +28,25 @@ def test_reference_arm_line():
     assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """Launched as the driver launches N > 1 (torchrun, one process per
+    rank): the ranks meet over gloo, rank 0 alone prints one line, every
+    rank exits 0."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
 
 
 def _fake_tree(tmp_path, monkeypatch, traffic=123456789):
