@@ -14,9 +14,11 @@
 // exponent is found once per block; each lane loads kQBlocksPerLane blocks
 // (a warp span apart) before encoding any, 256 bytes in flight per lane
 // (one block per lane measured 1.88 ms per 36-layer sweep, two 1.79, four
-// 1.70).  Dequantise: 8-element chunks per thread
-// (8 code bytes in, 16 bytes of BF16 out), kUnroll chunks in flight; each
-// chunk reads its block's scale byte.
+// 1.70).  Dequantise: when every code tensor of the call has 16-byte
+// aligned rows, 16-element chunks (16 code bytes in, 32 bytes of BF16 out
+// in one 256-bit store), eight per lane in flight; otherwise 8-element
+// chunks (8 code bytes in, 16 bytes out), kUnroll in flight.  Each chunk
+// reads its block's scale byte.
 #include <algorithm>
 
 #include "pwq_internal.h"
