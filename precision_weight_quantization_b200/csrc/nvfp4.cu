@@ -22,6 +22,9 @@
 //      data -- still in the 126 MB L2 -- is consumed first.
 // Every kernel also takes an FP8 block-wise source (E4M3 codes with tile
 // scales, dequantised in registers) for the re-quantisation calls.
+// Dequantise is a grouped walk over 16-element blocks (8 packed bytes and a
+// block-scale byte in, 32 bytes of BF16 out), eight blocks per lane in
+// flight.
 // Division: a group has at most 127 distinct code divisors d = fl(dec(sb) *
 // gs), so each CTA tabulates d and RN(1/d) for every block-scale code in
 // shared memory once; the block scale itself divides by fl(6 gs), whose
