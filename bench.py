@@ -635,39 +635,56 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
     H2D copy from pinned memory, every op (one grouped call each), and a D2H
     read of the codes and scales of the three formats.  Three streams
     (copy in, compute, copy out) and two device buffer sets pipeline the
-    layers, so the two copy directions and the kernels overlap."""
+    layers, so the two copy directions and the kernels overlap.  A layer's
+    tensors of one kind sit in one contiguous slab on both sides, so a
+    layer moves in one H2D copy and six D2H copies."""
     import workloads as W
     names = list(layers[0])
-    host_in = {n: layers[0][n].cpu().pin_memory() for n in names}
     shapes = {n: tuple(layers[0][n].shape) for n in names}
     G = W.QWEN3_4B_GROUPS
 
+    def slab(kind_shapes, dtype, device=None, pinned=False):
+        """One contiguous buffer holding a tensor per name (row-major, in
+        order), so a layer's tensors of one kind move in one copy."""
+        numel = [int(torch.Size(sh).numel()) for sh in kind_shapes.values()]
+        if device is None:
+            flat = torch.empty(sum(numel), dtype=dtype)
+            if pinned:
+                flat = flat.pin_memory()
+        else:
+            flat = torch.empty(sum(numel), dtype=dtype, device=device)
+        views, o = {}, 0
+        for (n, sh), k in zip(kind_shapes.items(), numel):
+            views[n] = flat[o:o + k].view(sh)
+            o += k
+        return flat, views
+
+    tile_sh = {n: (-(-shapes[n][0] // 128), -(-shapes[n][1] // 128)) for n in names}
+    mxs_sh = {n: (shapes[n][0], shapes[n][1] // 32) for n in names}
+    pk_sh = {n: (shapes[n][0], shapes[n][1] // 2) for n in names}
+    sb_sh = {n: (shapes[n][0], shapes[n][1] // 16) for n in names}
+    host_x, hx = slab(shapes, torch.bfloat16, pinned=True)
+    for n in names:
+        hx[n].copy_(layers[0][n].cpu())
+    # host images of a layer's outputs, one pinned slab per kind
+    kinds = (("q", shapes, torch.uint8), ("s", tile_sh, torch.float32), ("mq", shapes, torch.uint8),
+             ("me", mxs_sh, torch.uint8), ("pk", pk_sh, torch.uint8), ("sb", sb_sh, torch.uint8))
+    host_out = {k: slab(sh, dt, pinned=True)[0] for k, sh, dt in kinds}
+
     def device_set():
-        d = {"x": {n: torch.empty(shapes[n], dtype=torch.bfloat16, device=dev) for n in names}}
-        d["q"] = [torch.empty(shapes[n], dtype=torch.float8_e4m3fn, device=dev) for n in names]
-        d["s"] = [torch.empty((-(-shapes[n][0] // 128), -(-shapes[n][1] // 128)), dtype=torch.float32, device=dev)
-                  for n in names]
-        d["mq"] = [torch.empty(shapes[n], dtype=torch.float8_e4m3fn, device=dev) for n in names]
-        d["me"] = [torch.empty((shapes[n][0], shapes[n][1] // 32), dtype=torch.uint8, device=dev) for n in names]
-        d["pk"] = [[torch.empty((shapes[n][0], shapes[n][1] // 2), dtype=torch.uint8, device=dev) for n in g]
-                   for g in G]
-        d["sb"] = [[torch.empty((shapes[n][0], shapes[n][1] // 16), dtype=torch.float8_e4m3fn, device=dev)
-                    for n in g] for g in G]
+        d = {}
+        d["x_flat"], d["x"] = slab(shapes, torch.bfloat16, device=dev)
+        for k, sh, dt in kinds:
+            d[k + "_flat"], views = slab(sh, dt, device=dev)
+            d[k] = views
         d["gs"] = [torch.empty(1, dtype=torch.float32, device=dev) for _ in G]
         return d
 
     sets = [device_set(), device_set()]
     y = [torch.empty(shapes[n], dtype=torch.bfloat16, device=dev) for n in names]   # dequant / QDQ outputs
     yg = [[y[names.index(n)] for n in g] for g in G]
-    host_out = {n: [torch.empty(shapes[n], dtype=torch.uint8).pin_memory(),
-                    torch.empty((-(-shapes[n][0] // 128), -(-shapes[n][1] // 128)), dtype=torch.float32).pin_memory(),
-                    torch.empty(shapes[n], dtype=torch.uint8).pin_memory(),
-                    torch.empty((shapes[n][0], shapes[n][1] // 32), dtype=torch.uint8).pin_memory(),
-                    torch.empty((shapes[n][0], shapes[n][1] // 2), dtype=torch.uint8).pin_memory(),
-                    torch.empty((shapes[n][0], shapes[n][1] // 16), dtype=torch.uint8).pin_memory()]
-                for n in names}
-    out_bytes = sum(t.numel() * t.element_size() for v in host_out.values() for t in v)
-    in_bytes = sum(t.numel() * 2 for t in host_in.values())
+    out_bytes = sum(t.numel() * t.element_size() for t in host_out.values())
+    in_bytes = host_x.numel() * 2
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "comp", "out")}
     started = {k: [False, False] for k in ("comp", "out")}
@@ -678,34 +695,34 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
         with torch.cuda.stream(s_in):
             if started["comp"][b]:
                 s_in.wait_event(ev["comp"][b])        # the layer that last read this input set is done
-            for n in names:
-                d["x"][n].copy_(host_in[n], non_blocking=True)
+            d["x_flat"].copy_(host_x, non_blocking=True)
             ev["in"][b].record(s_in)
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(ev["in"][b])
             if started["out"][b]:
                 s_comp.wait_event(ev["out"][b])       # this output set has been read back
             xs = [d["x"][n] for n in names]
-            P.fp8_block_quant_grouped(xs, out=d["q"], scale=d["s"])
-            P.fp8_block_dequant_grouped(d["q"], d["s"], out=y)
-            P.mxfp8_quant_grouped(xs, out=d["mq"], scale=d["me"])
-            P.mxfp8_dequant_grouped(d["mq"], d["me"], out=y)
+            q = [d["q"][n].view(torch.float8_e4m3fn) for n in names]
+            sc = [d["s"][n] for n in names]
+            mq = [d["mq"][n].view(torch.float8_e4m3fn) for n in names]
+            me = [d["me"][n] for n in names]
+            P.fp8_block_quant_grouped(xs, out=q, scale=sc)
+            P.fp8_block_dequant_grouped(q, sc, out=y)
+            P.mxfp8_quant_grouped(xs, out=mq, scale=me)
+            P.mxfp8_dequant_grouped(mq, me, out=y)
             groups = [[d["x"][n] for n in g] for g in G]
-            P.nvfp4_quant_grouped(groups, out=d["pk"], sb=d["sb"], global_scale=d["gs"])
-            P.nvfp4_dequant_grouped([p_ for g in d["pk"] for p_ in g], [t for g in d["sb"] for t in g],
+            pk = [[d["pk"][n] for n in g] for g in G]
+            sbg = [[d["sb"][n].view(torch.float8_e4m3fn) for n in g] for g in G]
+            P.nvfp4_quant_grouped(groups, out=pk, sb=sbg, global_scale=d["gs"])
+            P.nvfp4_dequant_grouped([p_ for g in pk for p_ in g], [t for g in sbg for t in g],
                                     [d["gs"][gi] for gi, g in enumerate(G) for _ in g], out=y)
             P.nvfp4_fake_quant_grouped(groups, out=yg)
             ev["comp"][b].record(s_comp)
             started["comp"][b] = True
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev["comp"][b])
-            for k, n in enumerate(names):
-                gi = next(j for j, g in enumerate(G) if n in g)
-                pos = G[gi].index(n)
-                srcs = [d["q"][k], d["s"][k], d["mq"][k], d["me"][k], d["pk"][gi][pos], d["sb"][gi][pos]]
-                for h, t in zip(host_out[n], srcs):
-                    h.copy_(t.view(h.dtype) if t.dtype != h.dtype and t.element_size() == h.element_size() else t,
-                            non_blocking=True)
+            for k, _, _ in kinds:
+                host_out[k].copy_(d[k + "_flat"], non_blocking=True)
             ev["out"][b].record(s_out)
             started["out"][b] = True
 
@@ -744,7 +761,8 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
             "note": "public Python API (one grouped call per op per layer), one layer at a time from "
                     "pinned host memory (the same host buffer feeds every layer), codes+scales of the "
                     "three formats read back; copy-in, compute and copy-out on three streams with two "
-                    "device buffer sets, so layers overlap"}
+                    "device buffer sets, so layers overlap; a layer's tensors of one kind sit in one "
+                    "contiguous slab on both sides (one H2D copy and six D2H copies per layer)"}
 
 
 def main_reference(args, rank, world, torch, dist):
