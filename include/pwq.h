@@ -37,7 +37,10 @@
  * default stream) and returns; the status covers host-side validation and
  * the launch itself (cudaGetLastError right after each launch).  Device code
  * never traps; a bounded wait that gives up records a code readable with
- * pwq_device_error().
+ * pwq_device_error().  The outputs of a call that records such a code are
+ * unspecified (an encode step that gave up waiting for its group amax goes
+ * on with a partial one): a caller that needs to know reads
+ * pwq_device_error() after the stream has finished the call.
  *
  * Empty tensors (batch, rows or cols equal to 0) return PWQ_OK and launch
  * nothing.  Outputs may not overlap inputs or each other (PWQ_ERR_OVERLAP),
@@ -435,8 +438,9 @@ const char* pwq_build_info(void);
 
 /* Reads and clears the device-side error word of the current device
  * (synchronous; 0 = no error; bit 0 = a TMA load wait gave up, bit 1 = an
- * NVFP4 single-pass encode item gave up waiting for its group amax).  Returns
- * PWQ_ERR_NULL or PWQ_ERR_CUDA on failure. */
+ * NVFP4 single-pass encode item gave up waiting for its group amax).  When
+ * a bit is set, the outputs of the calls since the previous read are
+ * unspecified.  Returns PWQ_ERR_NULL or PWQ_ERR_CUDA on failure. */
 pwq_status pwq_device_error(uint32_t* code);
 
 /* Exhaustive self-check of the device arithmetic against CUDA's IEEE

@@ -31,7 +31,7 @@
  *   [PR503] vime pull request #503, review thread on the NVFP4 QDQ config
  *          (exact round-to-nearest numerics, fast math refused).
  *
- * Readings where the pages are silent (each one also listed in the design doc):
+ * Readings where the pages are silent:
  *   R1 FP8 tile scale s = fl(amax / 448) is the dequantisation multiplier.
  *   R2 Codes are e4m3(fl(x / s)): IEEE division, then RNE onto E4M3.
  *   R3 A zero scale (all-zero tile/block/group) gives signed-zero codes.

@@ -659,13 +659,12 @@ cudaError_t launch_fp8_block_quant(const Job* jobs, int n, cudaStream_t s) {
     EncodeTiledFn encode = encode_tiled_fn();
     if (!encode) return cudaErrorNotSupported;
     const size_t smem = (size_t)kPairStages * kPairBytes + 1024;
-    static int configured[64] = {0};
+    static int configured[kMaxDevices] = {0};
     const int dev = current_device();
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(fp8_block_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const void* fn = (const void*)fp8_block_quant_kernel;
+        const cudaError_t e = set_smem_limit_once(configured, &fn, 1, (int)smem);
         if (e != cudaSuccess) return e;
-        configured[dev] = 1;
     }
     for (int j0 = 0; j0 < n; j0 += kMaxLaunchTensors) {
         QuantArgs a;
@@ -780,13 +779,12 @@ cudaError_t launch_fp8_requant_tma(const RequantJob* jobs, int n, cudaStream_t s
     EncodeTiledFn encode = encode_tiled_fn();
     if (!encode) return cudaErrorNotSupported;
     const size_t smem = (size_t)kRqStages * kRqTileBytes + 1024;
-    static int configured[64] = {0};
+    static int configured[kMaxDevices] = {0};
     const int dev = current_device();
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(fp8_requant_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const void* fn = (const void*)fp8_requant_tma_kernel;
+        const cudaError_t e = set_smem_limit_once(configured, &fn, 1, (int)smem);
         if (e != cudaSuccess) return e;
-        configured[dev] = 1;
     }
     for (int j0 = 0; j0 < n;) {
         RequantTmaArgs a;

@@ -1018,17 +1018,11 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
         if (e != cudaSuccess) return e;
         const int dev = current_device();
         const size_t smem = (size_t)kFlowStages * kFlowStageBytes;
-        static int configured[64] = {0};
-        if (dev >= 0 && dev < 64 && !configured[dev]) {
-            const void* fns[4] = {(const void*)nvfp4_flow_kernel<true, false>,
-                                  (const void*)nvfp4_flow_kernel<false, false>,
-                                  (const void*)nvfp4_flow_kernel<true, true>,
-                                  (const void*)nvfp4_flow_kernel<false, true>};
-            for (int f = 0; f < 4 && e == cudaSuccess; ++f)
-                e = cudaFuncSetAttribute(fns[f], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            configured[dev] = 1;
-        }
+        static int configured[kMaxDevices] = {0};
+        const void* fns[4] = {(const void*)nvfp4_flow_kernel<true, false>, (const void*)nvfp4_flow_kernel<false, false>,
+                              (const void*)nvfp4_flow_kernel<true, true>, (const void*)nvfp4_flow_kernel<false, true>};
+        e = set_smem_limit_once(configured, fns, 4, (int)smem);
+        if (e != cudaSuccess) return e;
         const int grid = (int)std::max<int64_t>(
             1, std::min<int64_t>((int64_t)sm_count(dev) * kFlowCtasPerSm, 2 * (int64_t)a.total_items));
         a.lead = kFlowLeadPerCta * (uint32_t)grid;
@@ -1112,7 +1106,6 @@ cudaError_t static_amax_scratch(uint32_t** ptr) {
     // In host code g_static_amax names a host-side stand-in, not the device
     // array: the device address is looked up once per device, with that
     // device current, and cached.
-    constexpr int kMaxDevices = 64;
     static uint32_t* addr[kMaxDevices] = {};
     static std::mutex mu;
     int dev = 0;

@@ -3,8 +3,10 @@
 // conversion to byte-stride views and dispatch to the kernel launchers.
 // Nothing here allocates device memory or synchronises.
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "pwq.h"
@@ -23,12 +25,29 @@ int current_device() {
 }
 
 int sm_count(int device) {
-    static int cache[64] = {0};
-    if (device >= 0 && device < 64 && cache[device] > 0) return cache[device];
+    static std::atomic<int> cache[kMaxDevices] = {};
+    const bool cacheable = device >= 0 && device < kMaxDevices;
+    if (cacheable) {
+        const int c = cache[device].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) n = 148;
-    if (device >= 0 && device < 64) cache[device] = n;
+    if (cacheable) cache[device].store(n, std::memory_order_relaxed);
     return n;
+}
+
+cudaError_t set_smem_limit_once(int* done, const void* const* fns, int n, int bytes) {
+    static std::mutex mu;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < kMaxDevices && done[dev]) return cudaSuccess;
+    for (int f = 0; f < n; ++f) {
+        const cudaError_t e = cudaFuncSetAttribute(fns[f], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+    }
+    if (dev >= 0 && dev < kMaxDevices) done[dev] = 1;
+    return cudaSuccess;
 }
 
 int persistent_grid(int64_t work_ctas, int per_sm) {

@@ -20,6 +20,13 @@ struct View {
 int sm_count(int device);
 int current_device();
 
+// Raises the dynamic shared-memory limit of the n kernels `fns` to `bytes`
+// on the current device, once per device for each call site (`done` is that
+// site's per-device flag array of kMaxDevices entries).  Thread-safe: the
+// flags are read and written under one lock.
+constexpr int kMaxDevices = 64;
+cudaError_t set_smem_limit_once(int* done, const void* const* fns, int n, int bytes);
+
 // Grid size for a persistent elementwise kernel: enough CTAs to cover
 // `work_ctas`, at most `per_sm` resident CTAs per SM.
 int persistent_grid(int64_t work_ctas, int per_sm);
