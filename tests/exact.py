@@ -136,3 +136,29 @@ def f32(v):
 
 def is_zero(v):
     return v[1] == 0
+
+
+def to_rational(v) -> Fraction:
+    """(neg, finite magnitude) -> signed Fraction."""
+    assert v[1] != INF
+    return -v[1] if v[0] else v[1]
+
+
+def add(a, b):
+    """Exact sum of two finite signed values.  A zero sum of operands with
+    different signs is +0, as IEEE addition gives under round-to-nearest;
+    -0 + -0 = -0."""
+    s = to_rational(a) + to_rational(b)
+    if s == 0:
+        return (a[0] and b[0], Fraction(0))
+    return (s < 0, abs(s))
+
+
+def neg(a):
+    return (not a[0], a[1])
+
+
+def f32_value_to_exact(x) -> tuple:
+    """A Python / numpy binary32 value -> (neg, magnitude)."""
+    u = struct.unpack("<I", struct.pack("<f", float(x)))[0]
+    return f32_bits_to_exact(u)
