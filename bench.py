@@ -1,35 +1,42 @@
-"""Benchmark: the whole block-scaled quantisation path on the Qwen3-4B-shaped
-weight sweep (36 decoder layers x 7 BF16 weight tensors, 3.633 G elements,
-seeded synthetic N(0, 0.02) weights), on N GPUs of one node.
+"""Benchmark of the block-scaled quantisation path on N GPUs of one node.
 
-One step takes every element of the sweep through every row of the path:
-  fp8_block_quant -> fp8_block_dequant         (128x128 tiles, FP32 scales)
-  mxfp8_quant     -> mxfp8_dequant             (1x32, UE8M0)
-  nvfp4_quant (q/k/v and gate/up siblings share the global amax) -> nvfp4_dequant
-  nvfp4_fake_quant (siblings; the straight-through backward needs no kernel)
-Each op kind is captured once in a CUDA graph (one node per call, 36 layers)
-and the step replays the graphs back to back on one stream; CUDA events
-between them give the per-op device times.  Inputs (7.3 GB) are larger than
-the 126 MB L2, so no flush is needed between steps.
+Headline step (the largest workload that fits one GPU): a DeepSeek-V3-shaped
+MoE layer -- 256 routed experts, gate/up [256][2048][7168] and down
+[256][7168][2048], BF16 N(0, 0.01), 11.27 G elements -- quantised and
+dequantised in the three formats, plus the W4A4 NVFP4 fake-quantisation of
+a 16384 x 7168 BF16 activation (N(0, 1), 8 outlier channels x 20):
+  fp8_block_quant -> fp8_block_dequant        (128x128 tiles, FP32 scales)
+  mxfp8_quant     -> mxfp8_dequant            (1x32, UE8M0)
+  nvfp4_quant (gate/up of each expert share one global amax, down alone)
+                  -> nvfp4_dequant
+  nvfp4_fake_quant of the activation (its own dynamic amax; the
+                  straight-through backward needs no kernel)
+Every op is one grouped call over the three batched expert tensors (one
+kernel launch); the pages quantise these experts in FP8 block-wise and
+NVFP4, and MXFP8 is added so that one step takes the experts through every
+row of the path.  Each op is captured once in a CUDA graph and a step
+replays the seven graphs back to back on one stream; CUDA events between
+them give the per-op device times.  Inputs (22.5 GB) are larger than the
+126 MB L2, so no flush is needed between steps.
 
-`value` = elements of the sweep taken through the whole path per second,
-summed over ranks (weak scaling: every rank sweeps its own seeded layers; the
-path needs no collective).  `e2e` = the same metric through the public Python
-API with the BF16 weights in pinned host memory, one layer at a time: H2D
-copy, every op, and a D2H read of the quantised artefacts (codes + scales of
-the three formats) inside the timed region.
+`value` = elements taken through the step (experts + activation) per
+second, summed over ranks (weak scaling: every rank draws its own seeded
+experts; the path needs no collective).  `e2e` = the same metric through
+the public Python API from pinned host memory, 16 experts at a time (plus
+the activation): the H2D copy of the BF16 inputs, every op, and the D2H
+read of every result -- codes and scales of the three formats and the BF16
+outputs of the three dequantisers and of the fake-quantisation.
 
-`next_rows` times the FP8 block-wise re-quantisation ops (FP8 block-wise
-codes + scales -> FP8 block-wise / MXFP8 / NVFP4 in one pass) on the step's
-FP8 outputs over the same sweep, each in its own graph after the timed
-steps; they are not part of `value`.  FP8 -> FP8 is timed twice: on the
-quantiser's codes (every tile holds a +-448 code, so its code map is the
-identity and the kernel copies the codes) and, as
-`fp8_block_requant_general`, on seeded random codes whose magnitudes stop
-below 448 with the same scales (every tile's codes change).
-
-`--impl reference` times the CPU oracle (single thread, as it stands) on a
-bounded sample of the same workload.
+`per_config` times every workload of the benchmark set with its own launch
+shape: the 256 x 512 matrix (all ops; alone and as a batch of 64), the
+Qwen3-4B weight sweep (36 layers, one grouped call per two layers), the
+Qwen3-30B-A3B expert layer (128 experts, MXFP8, one call per layer over 48
+layers), the 2048-hidden QAT block (NVFP4 fake-quant of its sibling groups
+in one launch) and the two parts of the headline.  Workloads smaller than
+L2 are timed call by call with a 256 MB write between calls (L2 flushed).
+`next_rows` times the FP8 block-wise re-quantisation ops on the Qwen3-4B
+sweep.  `--impl reference` times the CPU oracle (all host threads) on a
+bounded sample of the headline workload.
 """
 import argparse
 import json
@@ -43,8 +50,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "quantized elements/s and achieved HBM GB/s (% of B200 peak) per format"
-WORKLOAD = "qwen3_4b_weight_sweep_36x7"
+WORKLOAD = "dsv3_moe_layer_256_experts_and_w4a4_activation"
 FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
 
 # algorithmic HBM bytes per element: one read of every input, one write of
 # every output, plus, for NVFP4 quantise / fake-quantise, the read of the
@@ -64,25 +72,23 @@ ONE_PASS_BYTES_PER_ELEM = {
     "nvfp4_quant": 2 + 0.5 + 1 / 16,
     "nvfp4_fake_quant": 2 + 2,
 }
-# our kernels launched per call (memsets are not counted)
-# (NVFP4 quantise / fake-quantise is one single-pass kernel after a memset)
-KERNELS_PER_CALL = {"fp8_block_quant": 1, "fp8_block_dequant": 1, "mxfp8_quant": 1, "mxfp8_dequant": 1,
-                    "nvfp4_quant": 1, "nvfp4_dequant": 1, "nvfp4_fake_quant": 1}
-OPS = list(BYTES_PER_ELEM)
+QWEN_OPS = list(BYTES_PER_ELEM)
+# the spec bar: every quantise / QDQ kernel at 70 % of the HBM roofline
+BAR_FRAC = 0.70
 
-# ncu DRAM traffic of one launch (one layer) for the kernels with a committed
-# summary under profiles/: the summary records the bytes and the sha256 of
-# the sources the capture ran on; once a source has changed the figure is
-# stale and `traffic` is reported as null.
+# ncu DRAM traffic of one launch of a kernel in the headline launch shape,
+# from its committed summary under profiles/ (the summary records the bytes
+# and the sha256 of the sources the capture ran on; once a source has
+# changed the figure is stale and `traffic` is reported as null)
 CSRC = "precision_weight_quantization_b200/csrc/"
 PROFILES = {
-    "nvfp4_fake_quant": ("profiles/nvfp4_flow_fake_quant_qwen3_4b_layer.md", "nvfp4.cu"),
-    "nvfp4_quant": ("profiles/nvfp4_flow_quant_qwen3_4b_layer.md", "nvfp4.cu"),
-    "fp8_block_quant": ("profiles/fp8_block_quant_qwen3_4b_layer.md", "fp8_block.cu"),
-    "fp8_block_dequant": ("profiles/fp8_block_dequant_qwen3_4b_layer.md", "fp8_block.cu"),
-    "mxfp8_quant": ("profiles/mxfp8_quant_qwen3_4b_layer.md", "mxfp8.cu"),
-    "mxfp8_dequant": ("profiles/mxfp8_dequant_qwen3_4b_layer.md", "mxfp8.cu"),
-    "nvfp4_dequant": ("profiles/nvfp4_dequant_qwen3_4b_layer.md", "nvfp4.cu"),
+    "nvfp4_quant": ("profiles/nvfp4_flow_quant_dsv3_experts.md", "nvfp4.cu"),
+    "nvfp4_fake_quant": ("profiles/nvfp4_flow_fake_quant_dsv3_activation.md", "nvfp4.cu"),
+    "fp8_block_quant": ("profiles/fp8_block_quant_dsv3_experts.md", "fp8_block.cu"),
+    "fp8_block_dequant": ("profiles/fp8_block_dequant_dsv3_experts.md", "fp8_block.cu"),
+    "mxfp8_quant": ("profiles/mxfp8_quant_dsv3_experts.md", "mxfp8.cu"),
+    "mxfp8_dequant": ("profiles/mxfp8_dequant_dsv3_experts.md", "mxfp8.cu"),
+    "nvfp4_dequant": ("profiles/nvfp4_dequant_dsv3_experts.md", "nvfp4.cu"),
 }
 
 
@@ -124,22 +130,27 @@ def recorded_traffic(op):
     return int(vals["traffic_bytes_per_launch"]), "ncu dram read+write of one launch, %s" % md
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="pwq", choices=["pwq", "reference"])
-    ap.add_argument("--layers", type=int, default=36)
+    ap.add_argument("--experts", type=int, default=256,
+                    help="routed experts of the headline layer (256 = the DeepSeek-V3 shape)")
+    ap.add_argument("--layers", type=int, default=36, help="layers of the Qwen3-4B sweep (per_config)")
+    ap.add_argument("--moe-layers", type=int, default=48, help="layers of the Qwen3-30B-A3B workload (per_config)")
     ap.add_argument("--layers-per-call", type=int, default=2,
-                    help="layers per grouped call (2: 14 tensors, the most one launch takes)")
+                    help="Qwen3-4B layers per grouped call (2: 14 tensors, the most one launch takes)")
+    ap.add_argument("--e2e-experts", type=int, default=16, help="experts per host round trip in e2e")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--no-next", action="store_true",
                     help="skip timing the FP8 block-wise re-quantisation ops (reported under next_rows)")
     ap.add_argument("--per-tensor", action="store_true",
-                    help="one call per tensor / sibling group instead of one grouped call per layer")
-    return ap.parse_args()
+                    help="Qwen3-4B sweep: one call per tensor / sibling group instead of one grouped call")
+    return ap.parse_args(argv)
 
 
 def peaks():
@@ -204,27 +215,98 @@ class Clocks:
                 "reasons": reasons, "samples": len(rows)}
 
 
-# ------------------------------------------------------------------ workload
+# ------------------------------------------------------------------ ops and workloads
 
-def bench_config(args, grouped, world):
-    return {"workload": WORKLOAD, "layers": args.layers, "elements_per_rank": layer_elems() * args.layers,
-            "tensors": "q 4096x2560, k/v 1024x2560, o 2560x4096, gate/up 9728x2560, down 2560x9728",
-            "path": "fp8_block q+dq, mxfp8 q+dq, nvfp4 q (qkv, gate/up siblings)+dq, "
-                    "nvfp4 fake-quant (siblings)",
-            "l2": "inputs larger than L2 (7.3 GB per rank), no flush",
-            "launch": ("one grouped call (one launch) per op per %d layers (%d tensors)"
-                       % (args.layers_per_call, 7 * args.layers_per_call) if grouped else "one call per tensor") +
-                      "; one CUDA graph per op kind, replayed back to back",
-            "parallelism": "dp%d (independent sweeps)" % world}
+class Op:
+    """One op of a workload: its calls (closures over pre-allocated inputs
+    and outputs, one kernel launch each), the elements they process and the
+    algorithmic bytes per element of its kind."""
 
+    def __init__(self, name, kind, calls, elems, kernels_per_call=1):
+        self.name, self.kind, self.calls, self.elems = name, kind, calls, int(elems)
+        self.kernels_per_call = kernels_per_call
+        self.bpe = BYTES_PER_ELEM[kind]
+        self.one_pass = ONE_PASS_BYTES_PER_ELEM.get(kind)
+
+    @property
+    def launches(self):
+        return len(self.calls) * self.kernels_per_call
+
+    def run(self):
+        for c in self.calls:
+            c()
+
+
+class Workload:
+    def __init__(self, name, ops, elems, config, tensors=None):
+        self.name, self.ops, self.elems, self.config = name, ops, int(elems), config
+        self.tensors = tensors or {}
+
+
+def op_fields(op, ms, hbm_peak, peak_kind):
+    gbs = op.elems * op.bpe / (ms / 1e3) / 1e9
+    d = {"ms": round(ms, 5), "elements": op.elems, "elem_per_s": op.elems / (ms / 1e3),
+         "alg_gbs": round(gbs, 1), "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4),
+         "launches": op.launches, "bytes_per_elem": round(op.bpe, 5)}
+    if op.one_pass is not None:
+        g1 = op.elems * op.one_pass / (ms / 1e3) / 1e9
+        d.update({"alg_gbs_one_pass": round(g1, 1), "frac_of_%s_hbm_one_pass" % peak_kind: round(g1 / hbm_peak, 4),
+                  "bytes_per_elem_one_pass": round(op.one_pass, 5)})
+    return d
+
+
+def dsv3_workload(P, torch, dev, rank=0, experts=256):
+    """The headline: DeepSeek-V3 expert layer (three batched tensors) and
+    the W4A4 activation.  One grouped call (one launch) per op."""
+    import workloads as W
+    ex = W.dsv3_experts(device=dev, experts=experts, seed=5000 + 1000 * rank)
+    names = [n for n, _ in W.DSV3_EXPERT_SHAPES]
+    xs = [ex[n] for n in names]
+    f8 = torch.float8_e4m3fn
+    q = [torch.empty(x.shape, dtype=f8, device=dev) for x in xs]
+    s = [torch.empty((x.shape[0], -(-x.shape[1] // 128), -(-x.shape[2] // 128)), dtype=torch.float32, device=dev)
+         for x in xs]
+    mq = [torch.empty(x.shape, dtype=f8, device=dev) for x in xs]
+    me = [torch.empty(x.shape[:-1] + (x.shape[-1] // 32,), dtype=torch.uint8, device=dev) for x in xs]
+    pk = [torch.empty(x.shape[:-1] + (x.shape[-1] // 2,), dtype=torch.uint8, device=dev) for x in xs]
+    sb = [torch.empty(x.shape[:-1] + (x.shape[-1] // 16,), dtype=f8, device=dev) for x in xs]
+    gs = [torch.empty(experts, dtype=torch.float32, device=dev) for _ in range(2)]   # {gate, up}, {down}
+    y = [torch.empty_like(x) for x in xs]      # BF16 output shared by the three dequantisers
+    act = W.dsv3_activation(device=dev, seed=5100 + 1000 * rank)
+    yact = torch.empty_like(act)
+    act_amax = torch.empty(1, dtype=torch.float32, device=dev)
+    E = sum(x.numel() for x in xs)
+    groups = [[xs[0], xs[1]], [xs[2]]]
+    ops = [
+        Op("fp8_block_quant", "fp8_block_quant", [lambda: P.fp8_block_quant_grouped(xs, out=q, scale=s)], E),
+        Op("fp8_block_dequant", "fp8_block_dequant", [lambda: P.fp8_block_dequant_grouped(q, s, out=y)], E),
+        Op("mxfp8_quant", "mxfp8_quant", [lambda: P.mxfp8_quant_grouped(xs, out=mq, scale=me)], E),
+        Op("mxfp8_dequant", "mxfp8_dequant", [lambda: P.mxfp8_dequant_grouped(mq, me, out=y)], E),
+        Op("nvfp4_quant", "nvfp4_quant",
+           [lambda: P.nvfp4_quant_grouped(groups, out=[pk[:2], pk[2:]], sb=[sb[:2], sb[2:]], global_scale=gs)], E),
+        Op("nvfp4_dequant", "nvfp4_dequant",
+           [lambda: P.nvfp4_dequant_grouped(pk, sb, [gs[0], gs[0], gs[1]], out=y)], E),
+        Op("nvfp4_fake_quant", "nvfp4_fake_quant",
+           [lambda: P.nvfp4_fake_quant(act, out=yact, amax_out=act_amax)], act.numel()),
+    ]
+    config = {"workload": WORKLOAD, "experts": experts,
+              "tensors": "gate/up [%d][2048][7168], down [%d][7168][2048] BF16 N(0, 0.01); activation "
+                         "16384x7168 BF16 N(0, 1) with 8 channels x20" % (experts, experts),
+              "elements_per_rank": E + act.numel(),
+              "path": "experts: fp8_block q+dq, mxfp8 q+dq, nvfp4 q (gate/up siblings per expert)+dq; "
+                      "activation: nvfp4 fake-quant (W4A4, dynamic amax)",
+              "launch": "one grouped call (one launch) per op; one CUDA graph per op, replayed back to back",
+              "l2": "inputs larger than L2 (22.7 GB per rank), no flush"}
+    tensors = dict(xs=xs, q=q, s=s, mq=mq, me=me, pk=pk, sb=sb, gs=gs, y=y, act=act, yact=yact, act_amax=act_amax,
+                   names=names)
+    return Workload("5_dsv3_experts_and_w4a4_activation", ops, E + act.numel(), config, tensors)
+
+
+# ---- Qwen3-4B weight sweep (36 layers x 7 tensors)
 
 def make_layers(n_layers, device, rank):
     import workloads as W
-    layers = []
-    for L in range(n_layers):
-        # every rank sweeps its own seeded layers (weak scaling)
-        layers.append(W.qwen3_4b_layer(L + 1000 * rank, device=device))
-    return layers
+    return [W.qwen3_4b_layer(L + 1000 * rank, device=device) for L in range(n_layers)]
 
 
 def layer_elems():
@@ -233,15 +315,13 @@ def layer_elems():
 
 
 class Buffers:
-    """Pre-allocated outputs for every op of every layer."""
+    """Pre-allocated outputs for every op of every Qwen3-4B layer."""
 
     def __init__(self, layers, P, torch, per_call=1):
         import workloads as W
         self.fp8 = []
         self.mx = []
         self.nv = []
-        self.y = []
-        self.ws = []
         dev = layers[0]["q_proj"].device
         for lay in layers:
             self.fp8.append({n: (torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev),
@@ -349,6 +429,101 @@ def op_calls_per_tensor(op, layers, buf, P):
     return calls
 
 
+def qwen3_4b_workload(P, torch, dev, rank=0, layers=36, per_call=2, grouped=True):
+    lays = make_layers(layers, dev, rank)
+    buf = Buffers(lays, P, torch, per_call)
+    E = layer_elems() * layers
+    ops = [Op(op, op, op_calls(op, lays, buf, P, grouped, per_call), E) for op in QWEN_OPS]
+    config = {"workload": "qwen3_4b_weight_sweep_%dx7" % layers, "layers": layers,
+              "tensors": "q 4096x2560, k/v 1024x2560, o 2560x4096, gate/up 9728x2560, down 2560x9728",
+              "path": "fp8_block q+dq, mxfp8 q+dq, nvfp4 q (qkv, gate/up siblings)+dq, nvfp4 fake-quant (siblings)",
+              "launch": ("one grouped call (one launch) per op per %d layers (%d tensors)" % (per_call, 7 * per_call)
+                         if grouped else "one call per tensor"),
+              "l2": "inputs larger than L2 (%.1f GB per rank), no flush" % (2 * E / 1e9)}
+    return Workload("2_qwen3_4b_weight_sweep", ops, E, config, dict(layers=lays, buf=buf, per_call=per_call))
+
+
+def qwen3_30b_workload(P, torch, dev, rank=0, layers=48, layer_index=None):
+    """128 batched experts per tensor kind, MXFP8 quant and dequant of all
+    of them in one grouped call per layer; one layer's buffers serve all
+    layers (1.2 GB of BF16, larger than L2).  layer_index picks the seeded
+    layer drawn (default: one per rank)."""
+    import workloads as W
+    lay = W.qwen3_30b_moe_layer(1000 * rank if layer_index is None else layer_index, device=dev)
+    xs = [lay[n] for n, _ in W.QWEN3_30B_EXPERT_SHAPES]
+    q = [torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev) for x in xs]
+    e = [torch.empty(x.shape[:-1] + (x.shape[-1] // 32,), dtype=torch.uint8, device=dev) for x in xs]
+    y = [torch.empty_like(x) for x in xs]
+    E1 = sum(x.numel() for x in xs)
+    ops = [Op("mxfp8_quant", "mxfp8_quant", [lambda: P.mxfp8_quant_grouped(xs, out=q, scale=e)] * layers, E1 * layers),
+           Op("mxfp8_dequant", "mxfp8_dequant", [lambda: P.mxfp8_dequant_grouped(q, e, out=y)] * layers, E1 * layers)]
+    config = {"workload": "qwen3_30b_a3b_moe_mxfp8_%d_layers" % layers,
+              "tensors": "128 experts: gate/up [128][768][2048], down [128][2048][768] BF16 N(0, 0.02) x "
+                         "per-expert LogUniform(0.5, 2)",
+              "launch": "one grouped call (one launch) per layer and op, %d layers, one layer's buffers reused"
+                        % layers,
+              "l2": "inputs larger than L2 (1.2 GB per layer), no flush"}
+    return Workload("3_qwen3_30b_a3b_moe_mxfp8", ops, E1 * layers, config, dict(xs=xs, q=q, e=e, y=y))
+
+
+def block2048_workload(P, torch, dev):
+    """The 2048-hidden QAT block: its three sibling groups fake-quantised in
+    one single-pass launch (W4A16); the straight-through backward is the
+    identity and launches nothing."""
+    import workloads as W
+    blk = W.block2048(device=dev)
+    groups = [[blk[n] for n in g] for g in W.BLOCK2048_GROUPS]
+    ys = [[torch.empty_like(x) for x in g] for g in groups]
+    amax = [torch.empty(1, dtype=torch.float32, device=dev) for _ in groups]
+    E = sum(x.numel() for g in groups for x in g)
+    ops = [Op("nvfp4_fake_quant", "nvfp4_fake_quant",
+              [lambda: P.nvfp4_fake_quant_grouped(groups, out=ys, amax_out=amax)], E)]
+    config = {"workload": "block2048_nvfp4_qat_w4a16",
+              "tensors": "q 4096x2048, k/v 512x2048 (siblings), gate/up 6144x2048 (siblings), down 2048x6144; "
+                         "N(0, 0.02) + 0.05%% x100",
+              "launch": "one grouped call (one launch) over the three sibling groups; STE backward: identity, "
+                        "no kernel",
+              "l2": "flushed before every timed call (inputs 96 MB, smaller than L2)"}
+    return Workload("4_block2048_nvfp4_qat", ops, E, config, dict(blk=blk, groups=groups, ys=ys, amax=amax))
+
+
+def small_workload(P, torch, dev, batch=1):
+    """The 256 x 512 matrix through every op (batch > 1: that many copies as
+    one batched tensor, each copy its own NVFP4 group)."""
+    import workloads as W
+    x = W.small_matrix(device="cpu").to(dev)
+    if batch > 1:
+        x = x.unsqueeze(0).repeat(batch, 1, 1).contiguous()
+    f8 = torch.float8_e4m3fn
+    M, N = x.shape[-2:]
+    lead = tuple(x.shape[:-2])
+    q = torch.empty(x.shape, dtype=f8, device=dev)
+    s = torch.empty(lead + (-(-M // 128), -(-N // 128)), dtype=torch.float32, device=dev)
+    mq = torch.empty(x.shape, dtype=f8, device=dev)
+    me = torch.empty(x.shape[:-1] + (N // 32,), dtype=torch.uint8, device=dev)
+    pk = torch.empty(x.shape[:-1] + (N // 2,), dtype=torch.uint8, device=dev)
+    sb = torch.empty(x.shape[:-1] + (N // 16,), dtype=f8, device=dev)
+    gs = torch.empty(batch, dtype=torch.float32, device=dev)
+    y = torch.empty_like(x)
+    E = x.numel()
+    ops = [Op("fp8_block_quant", "fp8_block_quant", [lambda: P.fp8_block_quant(x, out=q, scale=s)], E),
+           Op("fp8_block_dequant", "fp8_block_dequant", [lambda: P.fp8_block_dequant(q, s, out=y)], E),
+           Op("mxfp8_quant", "mxfp8_quant", [lambda: P.mxfp8_quant(x, out=mq, scale=me)], E),
+           Op("mxfp8_dequant", "mxfp8_dequant", [lambda: P.mxfp8_dequant(mq, me, out=y)], E),
+           Op("nvfp4_quant", "nvfp4_quant", [lambda: P.nvfp4_quant(x, out=[pk], sb=[sb], global_scale=gs)], E),
+           Op("nvfp4_dequant", "nvfp4_dequant", [lambda: P.nvfp4_dequant(pk, sb, gs, out=y)], E),
+           Op("nvfp4_fake_quant", "nvfp4_fake_quant", [lambda: P.nvfp4_fake_quant(x, out=y)], E)]
+    config = {"workload": "small_256x512" + ("_batch%d" % batch if batch > 1 else ""),
+              "tensors": "256x512 BF16 N(0, 0.02), 131 entries x50" + (", %d copies as one batch" % batch
+                                                                        if batch > 1 else ""),
+              "launch": "one call (one launch) per op",
+              "l2": "flushed before every timed call"}
+    return Workload("1_small_256x512" + ("_batch%d" % batch if batch > 1 else ""), ops, E, config,
+                    dict(x=x, q=q, s=s, mq=mq, me=me, pk=pk, sb=sb, gs=gs, y=y))
+
+
+# ------------------------------------------------------------------ timing
+
 def capture(calls, torch):
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
@@ -365,9 +540,87 @@ def capture(calls, torch):
     return g
 
 
+def time_back_to_back(ops, torch, steps, warmup, barrier=None, clocks=None):
+    """Each op in its own graph, the graphs of a step replayed back to back;
+    returns (ms per step, {op name: ms per step}, clock summary)."""
+    graphs = [capture(op.calls, torch) for op in ops]
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        for k, g in enumerate(graphs):
+            if evs is not None:
+                evs[k].record(stream)
+            g.replay()
+        if evs is not None:
+            evs[len(graphs)].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)] for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    clk = Clocks(torch.cuda.current_device()) if clocks else None
+    if clk:
+        clk.__enter__()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        step(evsets[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if clk:
+        clk.__exit__()
+    if barrier:
+        barrier()
+    per = {op.name: sum(evs[k].elapsed_time(evs[k + 1]) for evs in evsets) / steps for k, op in enumerate(ops)}
+    del graphs
+    return start.elapsed_time(end) / steps, per, (clk.summary() if clk else None)
+
+
+def time_flushed(ops, torch, iters, warmup):
+    """Each op's graph replayed `iters` times, a write of L2_FLUSH_BYTES
+    before every replay; the replay alone is timed (median)."""
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    out = {}
+    for op in ops:
+        g = capture(op.calls, torch)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+        for i in range(warmup + iters):
+            flush.zero_()
+            if i >= warmup:
+                evs[i - warmup][0].record(stream)
+            g.replay()
+            if i >= warmup:
+                evs[i - warmup][1].record(stream)
+        torch.cuda.synchronize()
+        out[op.name] = statistics.median(a.elapsed_time(b) for a, b in evs)
+        del g
+    return out
+
+
+def bars(per_op, peak_kind):
+    """Which quantise / QDQ kernels meet the 70 % bar."""
+    key = "frac_of_%s_hbm" % peak_kind
+    return {op: d[key] >= BAR_FRAC for op, d in per_op.items() if key in d}
+
+
+def config_entry(w, per_ms, hbm_peak, peak_kind, extra=None):
+    per_op = {op.name: op_fields(op, per_ms[op.name], hbm_peak, peak_kind) for op in w.ops}
+    d = dict(w.config)
+    d["ops"] = per_op
+    d["meets_%d_pct_bar" % int(BAR_FRAC * 100)] = bars(per_op, peak_kind)
+    if extra:
+        d.update(extra)
+    return d
+
+
 # ------------------------------------------------------------------ the FP8 block-wise re-quantisation row
 
-# FP8 block-wise codes + tile scales (the step's fp8_block_quant outputs)
+# FP8 block-wise codes + tile scales (the sweep's fp8_block_quant outputs)
 # straight into a rollout format; algorithmic bytes: one read of the codes
 # and scales (two for NVFP4: the amax pass and the encode pass), one write
 # of each output
@@ -383,7 +636,7 @@ NEXT_ONE_PASS_BYTES_PER_ELEM = {"fp8_block_requant_nvfp4": 1 + 4 / 16384 + 0.5 +
 def next_calls(op, layers, buf, P, torch, per_call=1):
     """One grouped call per `per_call` layers (their tensors; for NVFP4 their
     sibling groups in one single-pass launch), reading the FP8 codes and
-    scales the step wrote; every layer writes its own outputs (no call
+    scales the sweep wrote; every layer writes its own outputs (no call
     writes over lines a previous call left in L2)."""
     import workloads as W
     lay0 = layers[0]
@@ -432,78 +685,75 @@ def next_calls(op, layers, buf, P, torch, per_call=1):
     return calls
 
 
-def one_pass_fields(op, table, elems, ms, hbm_peak, peak_kind):
-    """The one-pass figures of a two-pass op (empty for the others)."""
-    if op not in table:
-        return {}
-    gbs = elems * table[op] / (ms / 1e3) / 1e9
-    return {"alg_gbs_one_pass": round(gbs, 1), "frac_of_%s_hbm_one_pass" % peak_kind: round(gbs / hbm_peak, 4),
-            "bytes_per_elem_one_pass": round(table[op], 5)}
-
-
-def time_next_rows(args, layers, buf, P, torch, hbm_peak, peak_kind):
-    """Device time of each re-quantisation op over the sweep (its own CUDA
-    graph, replayed after the step's timing; not part of `value`)."""
-    elems = layer_elems() * args.layers
+def time_next_rows(args, w, P, torch, hbm_peak, peak_kind):
+    """Device time of each re-quantisation op over the Qwen3-4B sweep (its
+    own CUDA graph, replayed after the sweep's timing)."""
+    layers, buf = w.tensors["layers"], w.tensors["buf"]
+    elems = layer_elems() * len(layers)
     stream = torch.cuda.current_stream()
     out = {}
     for op, bpe in NEXT_BYTES_PER_ELEM.items():
-        calls = next_calls(op, layers, buf, P, torch, max(1, args.layers_per_call))
+        calls = next_calls(op, layers, buf, P, torch, w.tensors["per_call"])
         g = capture(calls, torch)
         for _ in range(args.warmup):
             g.replay()
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
+        n = max(1, min(args.steps, 10))
         a.record(stream)
-        for _ in range(args.steps):
+        for _ in range(n):
             g.replay()
         b.record(stream)
         torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / args.steps
+        ms = a.elapsed_time(b) / n
         gbs = elems * bpe / (ms / 1e3) / 1e9
         out[op] = {"ms": round(ms, 4), "elem_per_s": elems / (ms / 1e3), "alg_gbs": round(gbs, 1),
-                   "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "calls": len(calls),
-                   "kernels_per_call": 1,
+                   "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "launches": len(calls),
                    "bytes_per_elem": round(bpe, 5)}
-        out[op].update(one_pass_fields(op, NEXT_ONE_PASS_BYTES_PER_ELEM, elems, ms, hbm_peak, peak_kind))
+        if op in NEXT_ONE_PASS_BYTES_PER_ELEM:
+            g1 = elems * NEXT_ONE_PASS_BYTES_PER_ELEM[op] / (ms / 1e3) / 1e9
+            out[op].update({"alg_gbs_one_pass": round(g1, 1),
+                            "frac_of_%s_hbm_one_pass" % peak_kind: round(g1 / hbm_peak, 4)})
         del g
     return out
 
 
 # ------------------------------------------------------------------ CPU oracle timing
 
-def cpu_sample_elems():
-    import workloads as W
-    return sum(r * c for n, (r, c) in W.QWEN3_4B_LAYER if n in ("q_proj", "k_proj", "v_proj", "o_proj"))
-
-
-def run_oracle_path(xs_bits, O):
-    """The oracle over the same path for a list of member tensors (one
-    sibling group)."""
+def oracle_path(xs_bits, PO, threads):
+    """The oracle (threaded driver) through the headline path for one expert:
+    FP8 block-wise and MXFP8 quantise + dequantise of each tensor, NVFP4 of
+    the {gate, up} group and of down, quantise + dequantise."""
     for x in xs_bits:
-        q, s = O.fp8_block_quant(x)
-        O.fp8_block_dequant(q, s)
-        q, e = O.mxfp8_quant(x)
-        O.mxfp8_dequant(q, e)
-    A = O.nvfp4_group_amax(xs_bits)
-    for x in xs_bits:
-        pk, sb, gs = O.nvfp4_quant(x, A)
-        O.nvfp4_dequant(pk, sb, gs, x.shape[-1])
-        O.nvfp4_fake_quant(x, A)
+        q, s = PO.fp8_block_quant(x, threads)
+        PO.fp8_block_dequant(q, s, threads)
+        q, e = PO.mxfp8_quant(x, threads)
+        PO.mxfp8_dequant(q, e, threads)
+    for grp in (xs_bits[:2], xs_bits[2:]):
+        A = PO.nvfp4_group_amax(grp, threads)
+        for x in grp:
+            pk, sb, gs = PO.nvfp4_quant(x, A, threads)
+            PO.nvfp4_dequant(pk, sb, gs, x.shape[-1], threads)
 
 
-def cpu_baseline(layer_cpu_bits):
-    from oracle import oracle as O
-    groups = [["q_proj", "k_proj", "v_proj"], ["o_proj"]]
-    n = cpu_sample_elems()
-    t0 = time.perf_counter()
-    for g in groups:
-        run_oracle_path([layer_cpu_bits[k] for k in g], O)
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "elem/s", "cores": 1, "kind": "oracle",
-            "sample": "layer 0 q/k/v (one NVFP4 sibling group) + o_proj: %d elements through every op "
-                      "of the path, single-threaded scalar C oracle, %.1f s" % (n, dt)}
+def cpu_baseline(expert_bits):
+    """The oracle as it stands on expert 0 of the headline layer, once on
+    one thread and once on every host thread."""
+    from oracle import parallel as PO
+    n = sum(x.size for x in expert_bits)
+    nthreads = PO.host_threads()
+    rates = {}
+    for th in (1, nthreads):
+        t0 = time.perf_counter()
+        oracle_path(expert_bits, PO, th)
+        rates[th] = (n / (time.perf_counter() - t0), time.perf_counter() - t0)
+    return {"value": rates[nthreads][0], "unit": "elem/s", "cores": nthreads, "kind": "oracle",
+            "single_thread_value": rates[1][0], "host_threads": nthreads, "nproc": os.cpu_count(),
+            "sample": "expert 0 of the headline layer (gate/up 2048x7168 as one NVFP4 sibling group, down "
+                      "7168x2048): %d elements through fp8_block q+dq, mxfp8 q+dq, nvfp4 q+dq; scalar C oracle, "
+                      "%.1f s on 1 thread, %.1f s on %d threads (rows split evenly)"
+                      % (n, rates[1][1], rates[nthreads][1], nthreads)}
 
 
 # ------------------------------------------------------------------ main
@@ -532,97 +782,62 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     hbm_peak, peak_kind = peaks()
+    barrier = dist.barrier if world > 1 else None
 
-    layers = make_layers(args.layers, dev, rank)
-    lpc = max(1, args.layers_per_call)
-    buf = Buffers(layers, P, torch, lpc)
-    elems_per_step = layer_elems() * args.layers
-    grouped = not args.per_tensor
-    graphs = {op: capture(op_calls(op, layers, buf, P, grouped, lpc), torch) for op in OPS}
-    ncalls = {op: len(op_calls(op, layers, buf, P, grouped, lpc)) for op in OPS}
-    launches_per_step = sum(ncalls[op] * KERNELS_PER_CALL[op] for op in OPS)
-
-    stream = torch.cuda.current_stream()
-
-    def step(evs=None):
-        for k, op in enumerate(OPS):
-            if evs is not None:
-                evs[k].record(stream)
-            graphs[op].replay()
-        if evs is not None:
-            evs[len(OPS)].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    per_op_ms = {op: 0.0 for op in OPS}
-    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(len(OPS) + 1)] for _ in range(args.steps)]
-    with Clocks(local) as clk:
-        torch.cuda.synchronize()
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
-        start.record(stream)
-        for i in range(args.steps):
-            step(evsets[i])
-        end.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    total_ms = start.elapsed_time(end)
-    for evs in evsets:
-        for k, op in enumerate(OPS):
-            per_op_ms[op] += evs[k].elapsed_time(evs[k + 1]) / args.steps
-    ms_per_step = total_ms / args.steps
-    t = torch.tensor([ms_per_step], dtype=torch.float64, device=dev)
+    # ---- headline: DeepSeek-V3 expert layer + W4A4 activation
+    w5 = dsv3_workload(P, torch, dev, rank, args.experts)
+    ms_step, per_ms, clocks = time_back_to_back(w5.ops, torch, args.steps, args.warmup, barrier, clocks=True)
+    t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_max = float(t.item())
-    value = elems_per_step * world / (ms_max / 1e3)
-
-    per_op = {}
-    for op in OPS:
-        ms = per_op_ms[op]
-        gbs = elems_per_step * BYTES_PER_ELEM[op] / (ms / 1e3) / 1e9
-        per_op[op] = {"ms": round(ms, 4), "elem_per_s": elems_per_step / (ms / 1e3), "alg_gbs": round(gbs, 1),
-                      "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "calls": ncalls[op],
-                      "bytes_per_elem": round(BYTES_PER_ELEM[op], 5)}
-        per_op[op].update(one_pass_fields(op, ONE_PASS_BYTES_PER_ELEM, elems_per_step, ms, hbm_peak, peak_kind))
-    dom = max(OPS, key=lambda o: per_op_ms[o])
-    dom_gbs = per_op[dom]["alg_gbs"]
-    traffic, traffic_note = recorded_traffic(dom) if grouped else (None, "per-tensor launches")
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(dom_gbs / hbm_peak, 4), "traffic": traffic, "peak_kind": peak_kind,
-                "alg_bytes_per_launch": int(round(elems_per_step / ncalls[dom] * BYTES_PER_ELEM[dom])),
-                "avg_launch_us": round(per_op_ms[dom] * 1e3 / ncalls[dom], 2),
-                "note": "achieved = algorithmic bytes of one launch / the average launch "
-                        "duration (CUDA events around the graph of all %d launches of the step); traffic: %s"
-                        % (ncalls[dom], traffic_note)}
-    if dom in ONE_PASS_BYTES_PER_ELEM:
-        one = per_op[dom]["alg_gbs_one_pass"]
-        roofline.update({"achieved_one_pass": one, "frac_one_pass": round(one / hbm_peak, 4),
-                         "alg_bytes_per_launch_one_pass":
-                             int(round(elems_per_step / ncalls[dom] * ONE_PASS_BYTES_PER_ELEM[dom]))})
-        roofline["note"] += ("; achieved counts the amax pass's read of the input (two reads, as the method "
-                             "is defined); *_one_pass counts a single read, the stricter ideal")
-
+    value = w5.elems * world / (ms_max / 1e3)
+    per_op = {op.name: op_fields(op, per_ms[op.name], hbm_peak, peak_kind) for op in w5.ops}
+    dom = max(w5.ops, key=lambda o: per_ms[o.name])
+    avg_launch_ms = per_ms[dom.name] / dom.launches
+    alg_bytes = dom.elems * dom.bpe / dom.launches
+    achieved = alg_bytes / (avg_launch_ms / 1e3) / 1e9
+    traffic, traffic_note = recorded_traffic(dom.name)
+    roofline = {"bound": "hbm", "kernel": dom.name, "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": traffic, "peak_kind": peak_kind,
+                "alg_bytes_per_launch": int(round(alg_bytes)), "avg_launch_us": round(avg_launch_ms * 1e3, 2),
+                "note": "achieved = algorithmic bytes of one launch / its duration (CUDA events around the op's "
+                        "graph in every timed step); traffic: %s" % traffic_note}
+    if dom.one_pass is not None:
+        one = dom.elems * dom.one_pass / dom.launches / (avg_launch_ms / 1e3) / 1e9
+        roofline.update({"achieved_one_pass": round(one, 1), "frac_one_pass": round(one / hbm_peak, 4)})
+        roofline["note"] += ("; achieved counts the amax pass's read of the input (two reads, as the method is "
+                             "defined); *_one_pass counts a single read, the stricter ideal")
+    launches_per_step = sum(op.launches for op in w5.ops)
     line = {"metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": bench_config(args, grouped, world),
+            "config": dict(w5.config, parallelism="dp%d (independent experts per rank)" % world),
             "per_op": per_op, "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk.summary() if rank == 0 else None}
-
-    del graphs
-    if not args.no_next:
-        line["next_rows"] = time_next_rows(args, layers, buf, P, torch, hbm_peak, peak_kind)
-    if not args.no_e2e:
-        line["e2e"] = e2e(args, layers, P, torch, dev, world, dist, elems_per_step)
+            "clocks": clocks if rank == 0 else None}
+    per_config = {}
+    per_config["5a_dsv3_experts"] = config_entry(
+        Workload("5a", [o for o in w5.ops if o.name != "nvfp4_fake_quant"], 0,
+                 {"workload": "dsv3_experts_%d" % args.experts}), per_ms, hbm_peak, peak_kind,
+        {"source": "the headline step"})
+    per_config["5b_dsv3_w4a4_activation"] = config_entry(
+        Workload("5b", [o for o in w5.ops if o.name == "nvfp4_fake_quant"], 0,
+                 {"workload": "dsv3_w4a4_activation_16384x7168"}), per_ms, hbm_peak, peak_kind,
+        {"source": "the headline step"})
+    expert0 = None
     if rank == 0 and not args.no_cpu_baseline:
         import workloads as W
-        lay0 = {n: W.bits(x) for n, x in layers[0].items() if n in ("q_proj", "k_proj", "v_proj", "o_proj")}
-        line["cpu_baseline"] = cpu_baseline(lay0)
+        expert0 = [W.bits(w5.tensors["xs"][i][0]) for i in range(3)]
+    if not args.no_e2e:
+        line["e2e"] = e2e(args, w5, P, torch, dev, world, dist)
+    del w5
+    torch.cuda.empty_cache()
+
+    if not args.no_per_config:
+        per_config.update(time_per_config(args, P, torch, dev, rank, hbm_peak, peak_kind, line))
+    line["per_config"] = per_config
+    if expert0 is not None:
+        line["cpu_baseline"] = cpu_baseline(expert0)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -630,22 +845,61 @@ def main():
         dist.destroy_process_group()
 
 
-def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
-    """Same path through the public API, host-resident weights: per layer an
-    H2D copy from pinned memory, every op (one grouped call each), and a D2H
-    read of the codes and scales of the three formats.  Three streams
-    (copy in, compute, copy out) and two device buffer sets pipeline the
-    layers, so the two copy directions and the kernels overlap.  A layer's
-    tensors of one kind sit in one contiguous slab on both sides, so a
-    layer moves in one H2D copy and six D2H copies."""
+def time_per_config(args, P, torch, dev, rank, hbm_peak, peak_kind, line):
+    out = {}
+    steps = max(1, min(args.steps, 10))
+    # Qwen3-4B sweep (and the re-quantisation row on its FP8 outputs)
+    w2 = qwen3_4b_workload(P, torch, dev, rank, args.layers, max(1, args.layers_per_call), not args.per_tensor)
+    ms, per, _ = time_back_to_back(w2.ops, torch, steps, args.warmup)
+    out[w2.name] = config_entry(w2, per, hbm_peak, peak_kind,
+                                {"ms_per_step": round(ms, 4), "elem_per_s_whole_path": w2.elems / (ms / 1e3)})
+    if not args.no_next:
+        w2.ops[0].run()
+        line["next_rows"] = time_next_rows(args, w2, P, torch, hbm_peak, peak_kind)
+    del w2
+    torch.cuda.empty_cache()
+    # Qwen3-30B-A3B experts, MXFP8 per layer
+    w3 = qwen3_30b_workload(P, torch, dev, rank, args.moe_layers)
+    ms, per, _ = time_back_to_back(w3.ops, torch, steps, args.warmup)
+    e = config_entry(w3, per, hbm_peak, peak_kind)
+    for name, d in e["ops"].items():
+        d["us_per_layer"] = round(d["ms"] * 1e3 / args.moe_layers, 2)
+    out[w3.name] = e
+    del w3
+    torch.cuda.empty_cache()
+    # small workloads: L2 flushed before every timed call
+    for w in (block2048_workload(P, torch, dev), small_workload(P, torch, dev, 1), small_workload(P, torch, dev, 64)):
+        per = time_flushed(w.ops, torch, iters=max(5, steps), warmup=args.warmup)
+        e = config_entry(w, per, hbm_peak, peak_kind)
+        if w.name.startswith("4_"):
+            e["ste_backward"] = "grad_x = grad_y (identity): no kernel, 0 bytes"
+        out[w.name] = e
+        del w
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------------ end to end through the public API
+
+def e2e(args, w5, P, torch, dev, world, dist):
+    """The headline path through the public Python API from pinned host
+    memory: per chunk of experts an H2D copy of the BF16 inputs, every op
+    (one grouped call each) and a D2H read of every result (codes and scales
+    of the three formats, BF16 outputs of the three dequantisers); the
+    activation once per step (H2D, fake-quant, D2H).  Copy-in, compute and
+    copy-out run on three streams over two device buffer sets, so chunks
+    overlap; a chunk's tensors of one kind sit in one contiguous slab on
+    both sides (one copy per kind).  The same host input chunk feeds every
+    chunk of the layer, and every chunk's results land in the same host
+    slabs."""
     import workloads as W
-    names = list(layers[0])
-    shapes = {n: tuple(layers[0][n].shape) for n in names}
-    G = W.QWEN3_4B_GROUPS
+    E = args.experts
+    C = max(1, min(args.e2e_experts, E))
+    n_chunks = -(-E // C)
+    names = [n for n, _ in W.DSV3_EXPERT_SHAPES]
+    shp = {n: (C,) + tuple(s) for n, s in W.DSV3_EXPERT_SHAPES}
 
     def slab(kind_shapes, dtype, device=None, pinned=False):
-        """One contiguous buffer holding a tensor per name (row-major, in
-        order), so a layer's tensors of one kind move in one copy."""
         numel = [int(torch.Size(sh).numel()) for sh in kind_shapes.values()]
         if device is None:
             flat = torch.empty(sum(numel), dtype=dtype)
@@ -659,42 +913,45 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
             o += k
         return flat, views
 
-    tile_sh = {n: (-(-shapes[n][0] // 128), -(-shapes[n][1] // 128)) for n in names}
-    mxs_sh = {n: (shapes[n][0], shapes[n][1] // 32) for n in names}
-    pk_sh = {n: (shapes[n][0], shapes[n][1] // 2) for n in names}
-    sb_sh = {n: (shapes[n][0], shapes[n][1] // 16) for n in names}
-    host_x, hx = slab(shapes, torch.bfloat16, pinned=True)
+    tile = {n: (C, -(-s[1] // 128), -(-s[2] // 128)) for n, s in shp.items()}
+    mxs = {n: (C, s[1], s[2] // 32) for n, s in shp.items()}
+    pks = {n: (C, s[1], s[2] // 2) for n, s in shp.items()}
+    sbs = {n: (C, s[1], s[2] // 16) for n, s in shp.items()}
+    gss = {"gate_up": (C,), "down": (C,)}
+    kinds = (("q", shp, torch.uint8), ("s", tile, torch.float32), ("mq", shp, torch.uint8),
+             ("me", mxs, torch.uint8), ("pk", pks, torch.uint8), ("sb", sbs, torch.uint8),
+             ("gs", gss, torch.float32), ("y8", shp, torch.bfloat16), ("ymx", shp, torch.bfloat16),
+             ("ynv", shp, torch.bfloat16))
+    host_x, hx = slab(shp, torch.bfloat16, pinned=True)
     for n in names:
-        hx[n].copy_(layers[0][n].cpu())
-    # host images of a layer's outputs, one pinned slab per kind
-    kinds = (("q", shapes, torch.uint8), ("s", tile_sh, torch.float32), ("mq", shapes, torch.uint8),
-             ("me", mxs_sh, torch.uint8), ("pk", pk_sh, torch.uint8), ("sb", sb_sh, torch.uint8))
+        hx[n].copy_(w5.tensors["xs"][names.index(n)][:C].cpu())
     host_out = {k: slab(sh, dt, pinned=True)[0] for k, sh, dt in kinds}
+    act_h = w5.tensors["act"].cpu().pin_memory()
+    act_out_h = torch.empty_like(act_h).pin_memory()
+    act_d = torch.empty_like(w5.tensors["act"])
+    act_y = torch.empty_like(act_d)
 
     def device_set():
         d = {}
-        d["x_flat"], d["x"] = slab(shapes, torch.bfloat16, device=dev)
+        d["x_flat"], d["x"] = slab(shp, torch.bfloat16, device=dev)
         for k, sh, dt in kinds:
-            d[k + "_flat"], views = slab(sh, dt, device=dev)
-            d[k] = views
-        d["gs"] = [torch.empty(1, dtype=torch.float32, device=dev) for _ in G]
+            d[k + "_flat"], d[k] = slab(sh, dt, device=dev)
         return d
 
     sets = [device_set(), device_set()]
-    y = [torch.empty(shapes[n], dtype=torch.bfloat16, device=dev) for n in names]   # dequant / QDQ outputs
-    yg = [[y[names.index(n)] for n in g] for g in G]
     out_bytes = sum(t.numel() * t.element_size() for t in host_out.values())
     in_bytes = host_x.numel() * 2
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "comp", "out")}
     started = {k: [False, False] for k in ("comp", "out")}
+    f8 = torch.float8_e4m3fn
 
-    def one_layer(i):
+    def one_chunk(i):
         b = i % 2
         d = sets[b]
         with torch.cuda.stream(s_in):
             if started["comp"][b]:
-                s_in.wait_event(ev["comp"][b])        # the layer that last read this input set is done
+                s_in.wait_event(ev["comp"][b])        # the chunk that last read this input set is done
             d["x_flat"].copy_(host_x, non_blocking=True)
             ev["in"][b].record(s_in)
         with torch.cuda.stream(s_comp):
@@ -702,21 +959,19 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
             if started["out"][b]:
                 s_comp.wait_event(ev["out"][b])       # this output set has been read back
             xs = [d["x"][n] for n in names]
-            q = [d["q"][n].view(torch.float8_e4m3fn) for n in names]
+            q = [d["q"][n].view(f8) for n in names]
             sc = [d["s"][n] for n in names]
-            mq = [d["mq"][n].view(torch.float8_e4m3fn) for n in names]
+            mq = [d["mq"][n].view(f8) for n in names]
             me = [d["me"][n] for n in names]
+            pk = [d["pk"][n] for n in names]
+            sb = [d["sb"][n].view(f8) for n in names]
+            gs = [d["gs"]["gate_up"], d["gs"]["down"]]
             P.fp8_block_quant_grouped(xs, out=q, scale=sc)
-            P.fp8_block_dequant_grouped(q, sc, out=y)
+            P.fp8_block_dequant_grouped(q, sc, out=[d["y8"][n] for n in names])
             P.mxfp8_quant_grouped(xs, out=mq, scale=me)
-            P.mxfp8_dequant_grouped(mq, me, out=y)
-            groups = [[d["x"][n] for n in g] for g in G]
-            pk = [[d["pk"][n] for n in g] for g in G]
-            sbg = [[d["sb"][n].view(torch.float8_e4m3fn) for n in g] for g in G]
-            P.nvfp4_quant_grouped(groups, out=pk, sb=sbg, global_scale=d["gs"])
-            P.nvfp4_dequant_grouped([p_ for g in pk for p_ in g], [t for g in sbg for t in g],
-                                    [d["gs"][gi] for gi, g in enumerate(G) for _ in g], out=y)
-            P.nvfp4_fake_quant_grouped(groups, out=yg)
+            P.mxfp8_dequant_grouped(mq, me, out=[d["ymx"][n] for n in names])
+            P.nvfp4_quant_grouped([xs[:2], xs[2:]], out=[pk[:2], pk[2:]], sb=[sb[:2], sb[2:]], global_scale=gs)
+            P.nvfp4_dequant_grouped(pk, sb, [gs[0], gs[0], gs[1]], out=[d["ynv"][n] for n in names])
             ev["comp"][b].record(s_comp)
             started["comp"][b] = True
         with torch.cuda.stream(s_out):
@@ -726,16 +981,23 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
             ev["out"][b].record(s_out)
             started["out"][b] = True
 
-    def run(n_layers):
-        for i in range(n_layers):
-            one_layer(i)
+    def activation():
+        with torch.cuda.stream(s_comp):
+            act_d.copy_(act_h, non_blocking=True)
+            P.nvfp4_fake_quant(act_d, out=act_y)
+            act_out_h.copy_(act_y, non_blocking=True)
+
+    def run():
+        activation()
+        for i in range(n_chunks):
+            one_chunk(i)
         cur = torch.cuda.current_stream()
         cur.wait_stream(s_in)
         cur.wait_stream(s_comp)
         cur.wait_stream(s_out)
 
-    steps = max(1, min(args.steps, 3))
-    run(args.layers)                                  # warm-up pass
+    steps = max(1, args.steps)
+    run()                                             # warm-up pass
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -747,7 +1009,7 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
     s_comp.wait_stream(stream)
     s_out.wait_stream(stream)
     for _ in range(steps):
-        run(args.layers)
+        run()
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
@@ -755,44 +1017,64 @@ def e2e(args, layers, P, torch, dev, world, dist, elems_per_step):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
-    return {"value": elems_per_step * world / (ms / 1e3), "unit": "elem/s",
-            "h2d_bytes_per_step": in_bytes * args.layers, "d2h_bytes_per_step": out_bytes * args.layers,
+    act_bytes = act_h.numel() * 2
+    return {"value": w5.elems * world / (ms / 1e3), "unit": "elem/s",
+            "h2d_bytes_per_step": in_bytes * n_chunks + act_bytes,
+            "d2h_bytes_per_step": out_bytes * n_chunks + act_bytes,
             "ms_per_step": ms, "steps": steps,
-            "note": "public Python API (one grouped call per op per layer), one layer at a time from "
-                    "pinned host memory (the same host buffer feeds every layer), codes+scales of the "
-                    "three formats read back; copy-in, compute and copy-out on three streams with two "
-                    "device buffer sets, so layers overlap; a layer's tensors of one kind sit in one "
-                    "contiguous slab on both sides (one H2D copy and six D2H copies per layer)"}
+            "note": "public Python API (one grouped call per op per chunk of %d experts), from pinned host memory "
+                    "(the same host chunk feeds every chunk), every result read back: codes + scales of the "
+                    "three formats, NVFP4 global scales, the BF16 outputs of the three dequantisers and of the "
+                    "activation's fake-quant; copy-in, compute and copy-out on three streams with two device "
+                    "buffer sets" % C}
 
+
+# ------------------------------------------------------------------ reference arm
 
 def main_reference(args, rank, world, torch, dist):
-    """The CPU oracle, as it stands, on a bounded sample of the same workload."""
+    """The CPU oracle, as it stands, on every host thread, on a bounded sample
+    of the headline workload per step: 256-row slices of one expert's gate,
+    up and down and of the activation."""
     if rank != 0:
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
         return
+    import numpy as np
     import workloads as W
-    from oracle import oracle as O
-    lay = W.qwen3_4b_layer(0, device="cpu")
-    # per step: a 256-row slice of each q/k/v member (one sibling group) = 1.57 M elements
-    sample = [W.bits(lay[n][:256]) for n in ("q_proj", "k_proj", "v_proj")]
-    n = sum(x.size for x in sample)
-    for _ in range(args.warmup):
-        run_oracle_path(sample, O)
+    from oracle import parallel as PO
+    threads = PO.host_threads()
+    rows = 256
+    samples = []
+    for e in range(4):
+        xs = [W.bits(W.normal_bf16((rows,) + tuple(s)[1:], 0.01, seed=5000 + 10 * e + t))
+              for t, (n, s) in enumerate(W.DSV3_EXPERT_SHAPES)]
+        samples.append(xs)
+    act = W.bits(W.normal_bf16((rows, 7168), 1.0, seed=5100))
+    n = sum(x.size for x in samples[0]) + act.size
+
+    def step(i):
+        xs = samples[i % len(samples)]
+        oracle_path(xs, PO, threads)
+        PO.nvfp4_fake_quant(act, PO.nvfp4_group_amax([act], threads), threads)
+
+    for i in range(args.warmup):
+        step(i)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        run_oracle_path(sample, O)
-    dt = (time.perf_counter() - t0) / args.steps
+    for i in range(args.steps):
+        step(i)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
     value = n / dt
+    cfg = {"workload": WORKLOAD, "experts": args.experts,
+           "sample_per_step": "256 rows of one expert's gate, up, down and of the activation (%d elements)" % n}
     line = {"metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
-            "config": dict(bench_config(args, not args.per_tensor, world),
-                           sample_per_step="256 rows of q/k/v of layer 0 (%d elements)" % n),
-            "cpu_baseline": {"value": value, "unit": "elem/s", "cores": 1, "kind": "oracle",
-                             "sample": "256-row slices of q/k/v (one sibling group) through every op, "
-                                       "single-threaded scalar C oracle"},
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "elem/s", "cores": threads, "kind": "oracle",
+                             "nproc": os.cpu_count(),
+                             "sample": "256-row slices of one expert's gate/up/down (FP8 block-wise and MXFP8 "
+                                       "q+dq, NVFP4 q+dq with gate/up siblings) and of the activation (NVFP4 "
+                                       "fake-quant), scalar C oracle on %d host threads" % threads},
             "e2e": {"value": value, "unit": "elem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     if world > 1:

@@ -471,6 +471,22 @@ pwq_status pwq_device_error(uint32_t* code);
  * IEEE-division path instead of the reciprocal path.  Asynchronous. */
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream);
 
+/* Self-test of the bounded wait of the NVFP4 single-pass kernel (the wait
+ * of an encode item for its group's amax, which normal calls bound at 2 s).
+ * It runs nvfp4_fake_quant of one BF16 tensor x ([B][M][N], B <= 512,
+ * N % 16 == 0, non-empty) into y through the single-pass kernel with that
+ * limit set to wait_ns (1 us .. 2 s) and with every encode item waiting on
+ * a completion count that no amax item adds to, so every such wait runs
+ * out.  Expected: the kernel returns after about wait_ns per waiting CTA,
+ * pwq_device_error() then reports bit 1, and y is unspecified; nothing
+ * faults or hangs, and the next call runs normally.  workspace: device,
+ * at least pwq_selftest_flow_timeout_workspace_size(x) bytes (0 on bad x).
+ * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _STRIDE, _OVERLAP, _WORKSPACE,
+ * _ARG (wait_ns out of range), _CUDA. */
+size_t pwq_selftest_flow_timeout_workspace_size(const pwq_tensor* x);
+pwq_status pwq_selftest_flow_timeout(const pwq_tensor* x, const pwq_tensor* y, uint64_t wait_ns, void* workspace,
+                                     size_t workspace_bytes, pwq_stream_t stream);
+
 /* Runs the device codecs over `count` consecutive binary32 bit patterns
  * starting at `first`
  * and writes: e4m3 codes (count bytes), e2m1 codes (count bytes, one code

@@ -76,6 +76,9 @@ _SIG = {
     "pwq_device_error": (_S, [ctypes.POINTER(ctypes.c_uint32)]),
     "pwq_selftest_division": (_S, [ctypes.c_int, _P, _P]),
     "pwq_selftest_codecs": (_S, [ctypes.c_uint32, ctypes.c_uint32, _P, _P, _P, _P]),
+    "pwq_selftest_flow_timeout_workspace_size": (ctypes.c_size_t, [_T]),
+    "pwq_selftest_flow_timeout": (_S, [_T, _T, ctypes.c_uint64, _P, ctypes.c_size_t, _P]),
+    "nvfp4_fake_quant_noalloc": (_S, [_T, _T, ctypes.c_int, _P, _P, _P]),
 }
 
 

@@ -365,7 +365,7 @@ constexpr int kFlowThreads = 256;
 constexpr uint32_t kItemChunks = 2048;                        // 16384 elements
 constexpr int kItemChunksPerThread = kItemChunks / kFlowThreads;   // 8
 constexpr int kFlowMaxInst = 512;                             // instances per launch
-constexpr uint64_t kFlowWaitNs = 2000000000ull;               // 2 s
+constexpr uint64_t kFlowWaitNs = kFlowWaitLimitNs;             // 2 s
 constexpr uint32_t kFlowLeadPerCta = 4;                       // L = kFlowLeadPerCta * grid
 constexpr int kFlowStages = 2;
 constexpr int kFlowCtasPerSm = 3;
@@ -407,6 +407,9 @@ struct FlowArgs {
     uint32_t* amax_bits;          // [n_inst]  (workspace, zeroed before launch)
     uint32_t* done;               // [n_inst]  completed amax items
     uint32_t* counter;            // [1]       queue head
+    const uint32_t* wait_done;    // the counts an encode item waits on: done (the self-test
+                                  // of the bounded wait points it at counts nothing adds to)
+    uint64_t wait_ns;             // limit of that wait (kFlowWaitNs; shorter in the self-test)
 };
 
 // The launch description in shared memory, so that the per-item decode and
@@ -808,10 +811,10 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         }
         if (tid == 0) {
             if (it.inst != known_inst) {
-                if (ld_acquire_gpu(a.done + it.inst) < G.items) {
+                if (ld_acquire_gpu(a.wait_done + it.inst) < G.items) {
                     const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(a.done + it.inst) < G.items) {
-                        if (globaltimer_ns() - t0 > kFlowWaitNs) {
+                    while (ld_acquire_gpu(a.wait_done + it.inst) < G.items) {
+                        if (globaltimer_ns() - t0 > a.wait_ns) {
                             atomicOr(&g_flow_error, kErrFlowTimeout);
                             break;
                         }
@@ -997,7 +1000,13 @@ size_t nvfp4_flow_workspace_bytes(int64_t instances) {
     return (size_t)((2 * per + 1) * 4 + 255) / 256 * 256;
 }
 
-cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, void* workspace, cudaStream_t s) {
+size_t nvfp4_flow_timeout_selftest_bytes(int64_t instances) {
+    const int64_t per = std::max<int64_t>(1, std::min<int64_t>(instances, kFlowMaxInst));
+    return (size_t)((3 * per + 1) * 4 + 255) / 256 * 256;
+}
+
+cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, void* workspace, cudaStream_t s,
+                              uint64_t wait_ns, bool wait_on_idle_counts) {
     const bool fp8 = n_groups > 0 && groups[0].ts != nullptr;   // every group of a call has the same source
     uint32_t* words = static_cast<uint32_t*>(workspace);
     const uint64_t kMaxItems = uint64_t(1) << 30;   // queue positions (2 per item) stay 32-bit
@@ -1014,7 +1023,12 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
         a.amax_bits = words;
         a.done = words + a.n_inst;
         a.counter = words + 2 * a.n_inst;
-        cudaError_t e = cudaMemsetAsync(words, 0, (size_t)(2 * a.n_inst + 1) * 4, s);
+        // the self-test's encode items wait on n_inst zeroed words that no
+        // amax item adds to, so every such wait runs out after wait_ns
+        a.wait_done = wait_on_idle_counts ? words + 2 * a.n_inst + 1 : a.done;
+        a.wait_ns = wait_ns;
+        const size_t words_used = (size_t)((wait_on_idle_counts ? 3 : 2) * a.n_inst + 1);
+        cudaError_t e = cudaMemsetAsync(words, 0, words_used * 4, s);
         if (e != cudaSuccess) return e;
         const int dev = current_device();
         const size_t smem = (size_t)kFlowStages * kFlowStageBytes;

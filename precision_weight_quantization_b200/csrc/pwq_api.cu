@@ -888,6 +888,38 @@ pwq_status nvfp4_activation_observe(const pwq_tensor* x, int observer, float ave
 
 // ------------------------------------------------------------------ self-tests
 
+size_t pwq_selftest_flow_timeout_workspace_size(const pwq_tensor* x) {
+    if (!x || x->batch < 0 || x->batch > 512) return 0;
+    return pwq::nvfp4_flow_timeout_selftest_bytes(std::max<int64_t>(1, x->batch));
+}
+
+pwq_status pwq_selftest_flow_timeout(const pwq_tensor* x, const pwq_tensor* y, uint64_t wait_ns, void* workspace,
+                                     size_t workspace_bytes, pwq_stream_t stream) {
+    if (wait_ns < 1000ull || wait_ns > pwq::kFlowWaitLimitNs)
+        return fail(PWQ_ERR_ARG, "wait_ns outside [1 us, 2 s]");
+    View vx, vy;
+    Extent ex, ey;
+    pwq_status st = check_tensor(x, Kind::kBF16, &vx, &ex, "x");
+    if (st != PWQ_OK) return st;
+    if (!y) return fail(PWQ_ERR_NULL, "y");
+    if (!same_shape(x, y)) return fail(PWQ_ERR_SHAPE, "y shape != x shape");
+    if ((st = check_tensor(y, Kind::kBF16, &vy, &ey, "y")) != PWQ_OK) return st;
+    if (empty(x)) return fail(PWQ_ERR_SHAPE, "the self-test needs a non-empty x");
+    if (x->cols % 16 != 0) return fail(PWQ_ERR_SHAPE, "cols % 16 != 0");
+    if (x->batch > 512) return fail(PWQ_ERR_SHAPE, "the self-test takes at most 512 batch slabs");
+    const size_t need = pwq::nvfp4_flow_timeout_selftest_bytes(x->batch);
+    if (!workspace || (uintptr_t)workspace % 4 != 0 || workspace_bytes < need)
+        return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
+    const Extent ew = extent_of(workspace, need);
+    if (overlaps(ey, ex) || overlaps(ew, ex) || overlaps(ew, ey)) return fail(PWQ_ERR_OVERLAP, "operands overlap");
+    pwq::NvGroup g{};
+    g.x = &vx;
+    g.out = &vy;
+    g.sb = nullptr;
+    g.n = 1;
+    return from_cuda(pwq::launch_nvfp4_flow(&g, 1, true, workspace, (cudaStream_t)stream, wait_ns, true));
+}
+
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream) {
     if (!counts) return fail(PWQ_ERR_NULL, "counts");
     if (which < 0 || which > 5) return fail(PWQ_ERR_ARG, "which");

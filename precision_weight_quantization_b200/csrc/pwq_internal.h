@@ -63,9 +63,16 @@ struct NvGroup {
 // NVFP4 single-pass quantise / fake-quantise of groups whose amax is reduced
 // on the device (amax_in null for every group): one dataflow launch per
 // piece.  Workspace: nvfp4_flow_workspace_bytes(total batch over groups).
+// wait_ns bounds an encode item's wait for its instance's amax (2 s);
+// wait_on_idle_counts (the self-test of that bound only) makes the encode
+// items wait on counts that no amax item adds to, so every wait runs out;
+// its workspace is nvfp4_flow_timeout_selftest_bytes(instances).
+constexpr uint64_t kFlowWaitLimitNs = 2000000000ull;
 size_t nvfp4_flow_workspace_bytes(int64_t instances);
+size_t nvfp4_flow_timeout_selftest_bytes(int64_t instances);
 cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, void* workspace,
-                              cudaStream_t s);
+                              cudaStream_t s, uint64_t wait_ns = kFlowWaitLimitNs,
+                              bool wait_on_idle_counts = false);
 
 // Two-launch NVFP4 path for one group set (used with a precomputed amax, by
 // the no-allocation entry point and by the FP8 block re-quantisation).

@@ -214,3 +214,55 @@ def test_observer_validation_without_gpu():
     assert lib.nvfp4_activation_observe(by(x), 1, 0.0, base + 64, None, None, ws, 256, None) == L.PWQ_ERR_OVERLAP
     x24 = T(L, base, 1, 4, 24, 4 * 32, 32)
     assert lib.nvfp4_activation_observe(by(x24), 1, 0.0, st, None, None, ws, 256, None) == L.PWQ_ERR_SHAPE
+
+
+def test_noalloc_validation_without_gpu():
+    """nvfp4_fake_quant_noalloc: the 4096-group limit of its static scratch,
+    lifted when amax_in is given, and the overlap rules, all decided before
+    any CUDA call."""
+    L = _lib()
+    lib = L.lib
+    base = 1 << 40
+    by = ctypes.byref
+    big = T(L, base, 4097, 1, 16, 16, 16)
+    ybig = T(L, base + (1 << 30), 4097, 1, 16, 16, 16)
+    assert lib.nvfp4_fake_quant_noalloc(by(big), by(ybig), 1, None, None, None) == L.PWQ_ERR_SHAPE
+    assert "4096" in lib.pwq_last_error_detail().decode()
+    # y partly over x, amax_out over x, y over amax_in: overlaps
+    x = T(L, base, 3, 64, 512, 64 * 512, 512)
+    y_part = T(L, base + 1024, 3, 64, 512, 64 * 512, 512)
+    y = T(L, base + (1 << 30), 3, 64, 512, 64 * 512, 512)
+    assert lib.nvfp4_fake_quant_noalloc(by(x), by(y_part), 1, None, None, None) == L.PWQ_ERR_OVERLAP
+    assert lib.nvfp4_fake_quant_noalloc(by(x), by(y), 1, None, base + 64, None) == L.PWQ_ERR_OVERLAP
+    assert lib.nvfp4_fake_quant_noalloc(by(x), by(y), 1, base + (1 << 30) + 32, None, None) == L.PWQ_ERR_OVERLAP
+    # misaligned amax_out; shape mismatch between x and y; N % 16
+    assert lib.nvfp4_fake_quant_noalloc(by(x), by(y), 1, None, base + (2 << 30) + 2, None) == L.PWQ_ERR_ALIGN
+    y2 = T(L, base + (1 << 30), 3, 32, 512, 32 * 512, 512)
+    assert lib.nvfp4_fake_quant_noalloc(by(x), by(y2), 1, None, None, None) == L.PWQ_ERR_SHAPE
+    x24 = T(L, base, 1, 4, 24, 4 * 24, 24)
+    y24 = T(L, base + (1 << 30), 1, 4, 24, 4 * 24, 24)
+    assert lib.nvfp4_fake_quant_noalloc(by(x24), by(y24), 1, None, None, None) == L.PWQ_ERR_SHAPE
+
+
+def test_flow_timeout_selftest_validation_without_gpu():
+    L = _lib()
+    lib = L.lib
+    base = 1 << 40
+    by = ctypes.byref
+    x = T(L, base, 3, 64, 512, 64 * 512, 512)
+    y = T(L, base + (1 << 30), 3, 64, 512, 64 * 512, 512)
+    ws = base + (2 << 30)
+    n = lib.pwq_selftest_flow_timeout_workspace_size(by(x))
+    assert n == 256
+    assert lib.pwq_selftest_flow_timeout(by(x), by(y), 10, ws, n, None) == L.PWQ_ERR_ARG
+    assert lib.pwq_selftest_flow_timeout(by(x), by(y), 3 * 10 ** 9, ws, n, None) == L.PWQ_ERR_ARG
+    assert lib.pwq_selftest_flow_timeout(by(x), by(y), 10 ** 6, ws, n - 4, None) == L.PWQ_ERR_WORKSPACE
+    assert lib.pwq_selftest_flow_timeout(by(x), by(y), 10 ** 6, None, n, None) == L.PWQ_ERR_WORKSPACE
+    assert lib.pwq_selftest_flow_timeout(by(x), by(x), 10 ** 6, ws, n, None) == L.PWQ_ERR_OVERLAP
+    assert lib.pwq_selftest_flow_timeout(by(x), by(y), 10 ** 6, base + 64, n, None) == L.PWQ_ERR_OVERLAP
+    xb = T(L, base, 513, 1, 16, 16, 16)
+    yb = T(L, base + (1 << 30), 513, 1, 16, 16, 16)
+    assert lib.pwq_selftest_flow_timeout_workspace_size(by(xb)) == 0
+    assert lib.pwq_selftest_flow_timeout(by(xb), by(yb), 10 ** 6, ws, 1 << 20, None) == L.PWQ_ERR_SHAPE
+    xe = T(L, None, 1, 0, 512, 0, 512)
+    assert lib.pwq_selftest_flow_timeout(by(xe), by(xe), 10 ** 6, ws, n, None) == L.PWQ_ERR_SHAPE

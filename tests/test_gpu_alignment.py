@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import guard
 from oracle import oracle as O
 import workloads as W
 
@@ -50,26 +51,20 @@ def bf16_at(xbits, lead_elems=8, pad_elems=16):
     """GPU BF16 copy of xbits whose base sits lead_elems * 2 bytes into its
     buffer and whose rows are lead + pad elements longer (base and row
     stride 16-byte but not 32-byte aligned)."""
-    *lead, M, N = xbits.shape
-    big = torch.zeros(tuple(lead) + (M, lead_elems + N + pad_elems), dtype=torch.bfloat16, device=DEV)
-    v = big[..., lead_elems:lead_elems + N]
+    v = guard.empty(xbits.shape, torch.bfloat16, lead=lead_elems, pad=pad_elems)
     v.copy_(W.from_bits(xbits, DEV))
     assert v.data_ptr() % 32 == 16 and (v.stride(-2) * 2) % 32 == 16
     return v
 
 
 def bf16_out(shape, lead_elems=8, pad_elems=16):
-    *lead, M, N = shape
-    big = torch.empty(tuple(lead) + (M, lead_elems + N + pad_elems), dtype=torch.bfloat16, device=DEV)
-    v = big[..., lead_elems:lead_elems + N]
+    v = guard.empty(shape, torch.bfloat16, lead=lead_elems, pad=pad_elems)
     assert v.data_ptr() % 32 == 16 and (v.stride(-2) * 2) % 32 == 16
     return v
 
 
 def bytes_out(shape, lead=8, pad=8, dtype=torch.uint8):
-    *lead_dims, M, N = shape
-    big = torch.empty(tuple(lead_dims) + (M, lead + N + pad), dtype=dtype, device=DEV)
-    v = big[..., lead:lead + N]
+    v = guard.empty(shape, dtype, lead=lead, pad=pad)
     assert v.data_ptr() % 16 == 8
     return v
 

@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import guard
 from oracle import oracle as O
 import workloads as W
 
@@ -36,11 +37,9 @@ def test_fp8_block_grouped_matches_oracle(P):
         N = x.shape[-1]
         pad = (-N) % 8
         xg.append(strided(x, pad) if pad else gpu(x))
-        big = torch.empty(x.shape[:-1] + (N + (-N) % 8,), dtype=torch.uint8, device=DEV)
-        outs.append(big[..., :N])
+        outs.append(guard.empty(x.shape, torch.uint8, pad=(-N) % 8))
     q, s = P.fp8_block_quant_grouped(xg, out=outs)
-    ys = [torch.empty(x.shape[:-1] + (x.shape[-1] + (-x.shape[-1]) % 8,), dtype=torch.bfloat16,
-                      device=DEV)[..., :x.shape[-1]] for x in xs]
+    ys = [guard.empty(x.shape, torch.bfloat16, pad=(-x.shape[-1]) % 8) for x in xs]
     y = P.fp8_block_dequant_grouped(q, s, out=ys)
     for i, x in enumerate(xs):
         oq, os_ = O.fp8_block_quant(x)
@@ -93,7 +92,7 @@ def test_nvfp4_grouped_layer_single_pass(P):
               for g, grp in enumerate(LAYER_GROUPS)]
     gg = [[gpu(x) for x in grp] for grp in groups]
     packed, sb, gs = P.nvfp4_quant_grouped(gg)
-    amax = [torch.empty(grp[0].shape[0] if grp[0].dim() == 3 else 1, dtype=torch.float32, device=DEV)
+    amax = [guard.empty((grp[0].shape[0] if grp[0].dim() == 3 else 1,), torch.float32)
             for grp in gg]
     fq = P.nvfp4_fake_quant_grouped(gg, amax_out=amax)
     for g, grp in enumerate(groups):
@@ -145,7 +144,7 @@ def test_nvfp4_single_pass_more_than_2048_instances(P):
 
 
 def test_tile_scale_exhaustive(P):
-    counts = torch.zeros(4, dtype=torch.int64, device=DEV)
+    counts = guard.empty((4,), torch.int64)
     P.check(P.lib.pwq_selftest_division(3, counts.data_ptr(), None), "pwq_selftest_division")
     torch.cuda.synchronize()
     n, bad, _, slow = counts.tolist()

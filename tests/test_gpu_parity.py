@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import guard
 from oracle import oracle as O
 import workloads as W
 
@@ -58,10 +59,9 @@ def rand_bits(shape, seed, std=0.02, outliers=True):
 
 
 def strided(xbits, pad_cols, dtype_bytes=2):
-    """A GPU BF16 view of xbits whose rows are padded by pad_cols elements."""
-    *lead, M, N = xbits.shape
-    big = torch.zeros(tuple(lead) + (M, N + pad_cols), dtype=torch.bfloat16, device=DEV)
-    v = big[..., :N]
+    """A GPU BF16 view of xbits whose rows are padded by pad_cols elements
+    (guarded: the padding must stay untouched, in place calls included)."""
+    v = guard.empty(xbits.shape, torch.bfloat16, pad=pad_cols)
     v.copy_(gpu(xbits))
     return v
 
@@ -79,15 +79,13 @@ def test_fp8_block_quant_dequant_exact(P, shape):
     pad = (-N) % 8                       # BF16 rows must be 16-byte aligned
     xg = strided(x, pad) if pad else gpu(x)
     if pad:
-        qbig = torch.empty(shape[:-1] + (N + (-N) % 16,), dtype=torch.uint8, device=DEV)
-        q, s = P.fp8_block_quant(xg, out=qbig[..., :N])
+        q, s = P.fp8_block_quant(xg, out=guard.empty(shape, torch.uint8, pad=(-N) % 16))
     else:
         q, s = P.fp8_block_quant(xg)
     oq, os_ = O.fp8_block_quant(x)
     assert np.array_equal(f32bits(s), os_.view(np.uint32))
     assert np.array_equal(u8(q), oq)
-    ybig = torch.empty(shape[:-1] + (N + pad,), dtype=torch.bfloat16, device=DEV)
-    y = P.fp8_block_dequant(q, s, out=ybig[..., :N])
+    y = P.fp8_block_dequant(q, s, out=guard.empty(shape, torch.bfloat16, pad=pad))
     assert np.array_equal(u16(y), O.fp8_block_dequant(oq, os_))
 
 
@@ -128,12 +126,10 @@ def test_mxfp8_strided_and_extreme(P):
     x[0, 1, :32] = np.arange(1, 33)
     x[1, 2, :] = 0x8000
     xg = strided(x, 64)
-    qbig = torch.empty((3, 40, 256 + 48), dtype=torch.uint8, device=DEV)
-    q, e = P.mxfp8_quant(xg, out=qbig[..., :256])
+    q, e = P.mxfp8_quant(xg, out=guard.empty((3, 40, 256), torch.uint8, pad=48))
     oq, oe = O.mxfp8_quant(x)
     assert np.array_equal(u8(q), oq) and np.array_equal(u8(e), oe)
-    ybig = torch.empty((3, 40, 256 + 8), dtype=torch.bfloat16, device=DEV)
-    y = P.mxfp8_dequant(q, e, out=ybig[..., :256])
+    y = P.mxfp8_dequant(q, e, out=guard.empty((3, 40, 256), torch.bfloat16, pad=8))
     assert np.array_equal(u16(y), O.mxfp8_dequant(oq, oe))
 
 
@@ -308,7 +304,7 @@ def test_block2048_nvfp4_qat_full_size(P):
     for group in W.BLOCK2048_GROUPS:
         xs = [blk[n] for n in group]
         A = O.nvfp4_group_amax([u16(x) for x in xs])
-        amax_out = torch.empty(1, dtype=torch.float32, device=DEV)
+        amax_out = guard.empty((1,), torch.float32)
         fq = P.nvfp4_fake_quant(xs, amax_out=amax_out)
         assert np.float32(amax_out.item()) == np.float32(A)
         packed, sb, gs = P.nvfp4_quant(xs)
@@ -370,7 +366,7 @@ def test_dsv3_experts_and_activation_full_size(P):
 
 @pytest.mark.parametrize("which", [0, 1, 2], ids=["fp8_divisors", "nvfp4_divisors", "nvfp4_scale_divisors"])
 def test_division_exhaustive(P, which):
-    counts = torch.zeros(4, dtype=torch.int64, device=DEV)
+    counts = guard.empty((4,), torch.int64)
     P.check(P.lib.pwq_selftest_division(which, counts.data_ptr(), None), "pwq_selftest_division")
     torch.cuda.synchronize()
     n, code_bad, quot_bad, fallback = counts.tolist()
@@ -389,7 +385,7 @@ def test_absmax_rewrite_exhaustive(P):
     """The bf16x2 abs-max form of the block / tile amax equals the integer
     max of the BF16 magnitude bits for every ordered pair of finite BF16
     values (both halves of the word)."""
-    counts = torch.zeros(4, dtype=torch.int64, device=DEV)
+    counts = guard.empty((4,), torch.int64)
     P.check(P.lib.pwq_selftest_division(4, counts.data_ptr(), None), "pwq_selftest_division")
     torch.cuda.synchronize()
     n, bad = counts.tolist()[:2]
@@ -401,7 +397,7 @@ def test_fp4_dequant_rewrite_exhaustive(P):
     """NVFP4 dequantisation through an exact binary16 product equals the
     binary32 form for every E2M1 code pair, every block scale code and every
     global scale fl(a / 2688) a BF16 group amax can give."""
-    counts = torch.zeros(4, dtype=torch.int64, device=DEV)
+    counts = guard.empty((4,), torch.int64)
     P.check(P.lib.pwq_selftest_division(5, counts.data_ptr(), None), "pwq_selftest_division")
     torch.cuda.synchronize()
     n, bad = counts.tolist()[:2]
@@ -413,9 +409,9 @@ def test_device_codecs_match_oracle(P):
     FP32 input of the active binades (both signs) and a strided sweep of the
     rest of the FP32 range."""
     def run(first, count):
-        e4 = torch.empty(count, dtype=torch.uint8, device=DEV)
-        e2 = torch.empty(count, dtype=torch.uint8, device=DEV)
-        bf = torch.empty(count, dtype=torch.int16, device=DEV)
+        e4 = guard.empty((count,), torch.uint8)
+        e2 = guard.empty((count,), torch.uint8)
+        bf = guard.empty((count,), torch.int16)
         P.check(P.lib.pwq_selftest_codecs(first, count, e4.data_ptr(), e2.data_ptr(), bf.data_ptr(), None),
                 "pwq_selftest_codecs")
         return e4.cpu().numpy(), e2.cpu().numpy(), bf.cpu().numpy().view(np.uint16)
@@ -465,17 +461,13 @@ def test_empty_tensors_are_noops(P):
 
 def padded_codes(codes, pad):
     """GPU uint8 view of code bytes [.., M, N] whose rows are padded by pad bytes."""
-    *lead, M, N = codes.shape
-    big = torch.zeros(tuple(lead) + (M, N + pad), dtype=torch.uint8, device=DEV)
-    v = big[..., :N]
+    v = guard.empty(codes.shape, torch.uint8, pad=pad)
     v.copy_(torch.from_numpy(np.ascontiguousarray(codes)).to(DEV))
     return v
 
 
 def padded_bf16_out(shape, pad):
-    *lead, M, N = shape
-    big = torch.full(tuple(lead) + (M, N + pad), float("nan"), dtype=torch.bfloat16, device=DEV)
-    return big[..., :N]
+    return guard.empty(shape, torch.bfloat16, pad=pad)
 
 
 @pytest.mark.parametrize("shape,pad_q,pad_y", [((3, 130, 256), 16, 8), ((2, 256, 384), 32, 16),

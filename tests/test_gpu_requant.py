@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import guard
 from oracle import oracle as O
 import workloads as W
 
@@ -53,9 +54,9 @@ def codes_and_scales(shape, seed, raw=False, max_mag=0x7E):
 def to_gpu_codes(q, pad=0):
     if pad == 0:
         return torch.from_numpy(np.ascontiguousarray(q)).to(DEV)
-    big = torch.zeros(q.shape[:-1] + (q.shape[-1] + pad,), dtype=torch.uint8, device=DEV)
-    big[..., :q.shape[-1]] = torch.from_numpy(q).to(DEV)
-    return big[..., :q.shape[-1]]
+    v = guard.empty(q.shape, torch.uint8, pad=pad)
+    v.copy_(torch.from_numpy(np.ascontiguousarray(q)).to(DEV))
+    return v
 
 
 FP8_SHAPES = [((130, 200), False, 0), ((3, 129, 136), True, 8), ((1, 8), True, 0), ((256, 512), False, 0),

@@ -131,18 +131,18 @@ def block2048_grad(name: str, device="cpu") -> torch.Tensor:
                        device=device)
 
 
-def dsv3_experts(device="cpu", experts: int = DSV3_EXPERTS) -> dict:
+def dsv3_experts(device="cpu", experts: int = DSV3_EXPERTS, seed: int = 5000) -> dict:
     """DeepSeek-V3-shaped routed experts, batched [E][rows][cols], N(0, 0.01)."""
     out = {}
     for t, (name, (r, c)) in enumerate(DSV3_EXPERT_SHAPES):
-        out[name] = normal_bf16((experts, r, c), 0.01, seed=5000 + t, device=device)
+        out[name] = normal_bf16((experts, r, c), 0.01, seed=seed + t, device=device)
     return out
 
 
-def dsv3_activation(device="cpu") -> torch.Tensor:
+def dsv3_activation(device="cpu", seed: int = 5100) -> torch.Tensor:
     """16384 x 7168 activation, N(0, 1) with 8 seeded channels multiplied by 20."""
-    x = normal_bf16(DSV3_ACT_SHAPE, 1.0, seed=5100, device=device)
-    return outlier_channels(x, 8, 20.0, seed=5100)
+    x = normal_bf16(DSV3_ACT_SHAPE, 1.0, seed=seed, device=device)
+    return outlier_channels(x, 8, 20.0, seed=seed)
 
 
 def random_bf16(shape, seed: int, std: float = 1.0, device="cpu") -> torch.Tensor:
