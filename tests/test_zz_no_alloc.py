@@ -10,9 +10,12 @@ second call's output.  The file is named so that pytest collects it last.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import guard
+from oracle import oracle as O
 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -32,8 +35,8 @@ def test_noalloc_entry_point_matches_workspace_entry_point_twice():
         # a batched sibling pair: 3 groups, each {x0[b], x1[b]}
         xs = [W.random_bf16((3, 64, 512), seed=seed, std=std, device=dev),
               W.random_bf16((3, 32, 512), seed=seed + 100, std=std, device=dev)]
-        ys = [torch.full_like(x, float("nan")) for x in xs]
-        amax_out = torch.full((3,), -1.0, dtype=torch.float32, device=dev)
+        ys = [guard.empty(x.shape, torch.bfloat16) for x in xs]
+        amax_out = guard.empty((3,), torch.float32)
         ax = (PwqTensor * 2)(*[P._desc(x, "x") for x in xs])
         ay = (PwqTensor * 2)(*[P._desc(y, "y") for y in ys])
         st = f(ax, ay, 2, None, amax_out.data_ptr(), stream)
@@ -49,3 +52,33 @@ def test_noalloc_entry_point_matches_workspace_entry_point_twice():
         expect = torch.stack([torch.maximum(xs[0][b].float().abs().max(), xs[1][b].float().abs().max())
                               for b in range(3)])
         assert torch.equal(amax_out, expect), call
+        # and the oracle, group by group
+        for b in range(3):
+            bits = [W.bits(x[b]) for x in xs]
+            A = O.nvfp4_group_amax(bits)
+            for x_b, y in zip(bits, ys):
+                assert np.array_equal(W.bits(y[b]), O.nvfp4_fake_quant(x_b, A)), (call, b)
+
+
+def test_noalloc_with_amax_in_beyond_the_scratch_limit():
+    """With amax_in the static scratch is unused, so more than 4096 groups
+    are accepted; the result equals nvfp4_fake_quant's with the same amax."""
+    import precision_weight_quantization_b200 as P
+    from precision_weight_quantization_b200._lib import PwqTensor, lib
+
+    dev = torch.device("cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    B = 4097
+    x = W.random_bf16((B, 4, 32), seed=21, std=1.0, device=dev)
+    amax = x.float().abs().amax(dim=(1, 2)).contiguous()
+    amax[::7] *= 2.0                      # cached / all-reduced amax may exceed the slab's own
+    y = guard.empty(x.shape, torch.bfloat16)
+    ax, ay = P._desc(x, "x"), P._desc(y, "y")
+    st = lib.nvfp4_fake_quant_noalloc(ctypes.byref(ax), ctypes.byref(ay), 1, amax.data_ptr(), None, stream)
+    assert st == 0, (P.status_string(st), lib.pwq_last_error_detail().decode())
+    ref = P.nvfp4_fake_quant(x, amax=amax)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+    xb, yb, ab = W.bits(x), W.bits(y), amax.cpu().numpy()
+    for b in (0, 7, 2048, B - 1):
+        assert np.array_equal(yb[b], O.nvfp4_fake_quant(xb[b], ab[b])), b
