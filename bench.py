@@ -146,6 +146,8 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--configs", default="1,2,3,4",
+                    help="per_config workloads to time besides the headline (1 small, 2 Qwen3-4B, 3 Qwen3-30B, 4 QAT block)")
     ap.add_argument("--no-next", action="store_true",
                     help="skip timing the FP8 block-wise re-quantisation ops (reported under next_rows)")
     ap.add_argument("--per-tensor", action="store_true",
@@ -848,7 +850,30 @@ def main():
 def time_per_config(args, P, torch, dev, rank, hbm_peak, peak_kind, line):
     out = {}
     steps = max(1, min(args.steps, 10))
-    # Qwen3-4B sweep (and the re-quantisation row on its FP8 outputs)
+    want = set(args.configs.split(","))
+    if "2" in want:
+        time_qwen3_4b(args, P, torch, dev, rank, hbm_peak, peak_kind, line, out, steps)
+    if "3" in want:
+        time_qwen3_30b(args, P, torch, dev, rank, hbm_peak, peak_kind, out, steps)
+    small = []
+    if "4" in want:
+        small.append(block2048_workload(P, torch, dev))
+    if "1" in want:
+        small += [small_workload(P, torch, dev, 1), small_workload(P, torch, dev, 64)]
+    # small workloads: L2 flushed before every timed call
+    for w in small:
+        per = time_flushed(w.ops, torch, iters=max(5, steps), warmup=args.warmup)
+        e = config_entry(w, per, hbm_peak, peak_kind)
+        if w.name.startswith("4_"):
+            e["ste_backward"] = "grad_x = grad_y (identity): no kernel, 0 bytes"
+        out[w.name] = e
+    del small
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_qwen3_4b(args, P, torch, dev, rank, hbm_peak, peak_kind, line, out, steps):
+    """The Qwen3-4B sweep (and the re-quantisation row on its FP8 outputs)."""
     w2 = qwen3_4b_workload(P, torch, dev, rank, args.layers, max(1, args.layers_per_call), not args.per_tensor)
     ms, per, _ = time_back_to_back(w2.ops, torch, steps, args.warmup)
     out[w2.name] = config_entry(w2, per, hbm_peak, peak_kind,
@@ -858,7 +883,10 @@ def time_per_config(args, P, torch, dev, rank, hbm_peak, peak_kind, line):
         line["next_rows"] = time_next_rows(args, w2, P, torch, hbm_peak, peak_kind)
     del w2
     torch.cuda.empty_cache()
-    # Qwen3-30B-A3B experts, MXFP8 per layer
+
+
+def time_qwen3_30b(args, P, torch, dev, rank, hbm_peak, peak_kind, out, steps):
+    """Qwen3-30B-A3B experts, MXFP8 per layer."""
     w3 = qwen3_30b_workload(P, torch, dev, rank, args.moe_layers)
     ms, per, _ = time_back_to_back(w3.ops, torch, steps, args.warmup)
     e = config_entry(w3, per, hbm_peak, peak_kind)
@@ -867,16 +895,6 @@ def time_per_config(args, P, torch, dev, rank, hbm_peak, peak_kind, line):
     out[w3.name] = e
     del w3
     torch.cuda.empty_cache()
-    # small workloads: L2 flushed before every timed call
-    for w in (block2048_workload(P, torch, dev), small_workload(P, torch, dev, 1), small_workload(P, torch, dev, 64)):
-        per = time_flushed(w.ops, torch, iters=max(5, steps), warmup=args.warmup)
-        e = config_entry(w, per, hbm_peak, peak_kind)
-        if w.name.startswith("4_"):
-            e["ste_backward"] = "grad_x = grad_y (identity): no kernel, 0 bytes"
-        out[w.name] = e
-        del w
-    torch.cuda.empty_cache()
-    return out
 
 
 # ------------------------------------------------------------------ end to end through the public API

@@ -310,6 +310,49 @@ pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, in
                                     const float* amax_in, float* amax_out, pwq_stream_t stream);
 
 /* ===================================================================== */
+/* Block scales in the tensor-core (block-scaled MMA) layout              */
+/* ===================================================================== */
+/*
+ * The rollout GEMM consumes the quantised weights ("Low Precision RL",
+ * "Modes" 3; the NVFP4 exporter repacks the scales for the inference
+ * kernels, verl NVFP4 QAT article 2.5); the pages do not give the layout
+ * such a GEMM reads.  The one used here is the layout in which the sm_100
+ * block-scaled tensor-core MMA takes its scale factors (NVIDIA PTX ISA,
+ * tcgen05.mma with block scaling and tcgen05.cp's 32x128b.warpx4 shape;
+ * cuBLAS documentation, 1D block-scaling-factor layout).  For an [B][M][S]
+ * array of scale bytes (S = N / 32 for MXFP8, N / 16 for NVFP4), every
+ * batch slab is ceil(M/128) x ceil(S/4) tiles of 512 contiguous bytes;
+ * tiles follow each other along S within a 128-row band, then band after
+ * band; the scale of tile row r (0..127) and column c (0..3) is at byte
+ * (r % 32) * 16 + (r / 32) * 4 + c of its tile.  Rows past M and columns
+ * past S are zero bytes (the calls below write them).
+ */
+
+/* Bytes of one such array: B * ceil(M/128) * ceil(S/4) * 512 (0 on negative input). */
+size_t pwq_mma_scale_bytes(int64_t batch, int64_t rows, int64_t scale_cols);
+
+/* Dense [B][M][S] scale bytes -> the tile layout (padding written as zero),
+ * and back (padding ignored).  mma: 16-byte aligned device array of
+ * pwq_mma_scale_bytes() bytes; dense: device array of B*M*S bytes.  The two
+ * may not overlap.  Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _OVERLAP, _CUDA. */
+pwq_status pwq_scales_to_mma(const uint8_t* dense, int64_t batch, int64_t rows, int64_t scale_cols, uint8_t* mma,
+                             pwq_stream_t stream);
+pwq_status pwq_scales_from_mma(const uint8_t* mma, int64_t batch, int64_t rows, int64_t scale_cols, uint8_t* dense,
+                               pwq_stream_t stream);
+
+/* mxfp8_quant_grouped / nvfp4_quant_grouped writing every tensor's block
+ * scales straight into the tile layout (scale_mma[i] / sb_mma[i]: device
+ * arrays of pwq_mma_scale_bytes(B, M, N/32) / (B, M, N/16) bytes, any
+ * alignment); codes, global scales and every other rule as the dense
+ * calls.  When M % 128 or S % 4 is not zero the call first clears the
+ * array (one memset on the stream) so that the padding is zero. */
+pwq_status mxfp8_quant_grouped_mma(int n, const pwq_tensor* x, const pwq_tensor* q, uint8_t* const* scale_mma,
+                                   pwq_stream_t stream);
+pwq_status nvfp4_quant_grouped_mma(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                                   const pwq_tensor* q_packed, uint8_t* const* sb_mma, float* const* global_scale,
+                                   void* workspace, size_t workspace_bytes, pwq_stream_t stream);
+
+/* ===================================================================== */
 /* FP8 block-wise weights into a rollout format                           */
 /* ===================================================================== */
 

@@ -361,3 +361,49 @@ def observe(state, x_bits, kind, c=np.float32(0.01)):
     return np.array([lo, hi], np.float32), A, np.float32(nvfp4_global_scale(A))
 
 OBSERVERS_BY_NAME = {"memoryless_minmax": MEMORYLESS_MINMAX, "static_minmax": STATIC_MINMAX, "minmax": MINMAX}
+
+
+# ---------------------------------------------------------------- tensor-core block-scale layout
+#
+# The block-scaled tensor-core MMA of sm_100 (PTX ISA, tcgen05.mma with
+# block scaling; the scale factors reach tensor memory with tcgen05.cp's
+# 32x128b.warpx4 shape, i.e. 32 rows of 16 bytes fanned out to four warps)
+# and cuBLAS's 1D block-scaling-factor layout take the scale bytes of an
+# [M][S] scale matrix (S = K / 32 for MXFP8, K / 16 for NVFP4) in tiles of
+# 128 rows x 4 scale columns.  Each tile is 512 contiguous bytes, the tiles
+# of one 128-row band follow each other along S, the bands follow each
+# other along M, and inside a tile the scale of tile row r (0..127) and
+# column c (0..3) sits at byte (r % 32) * 16 + (r // 32) * 4 + c.  Rows
+# are padded to a multiple of 128 and columns to a multiple of 4 with zero
+# bytes.  A batch [B][M][S] is B such slabs one after the other.  (The
+# pages name the consumer -- the rollout GEMM takes the quantised weights,
+# "Low Precision RL", "Modes" 3; the exporter repacks NVFP4 scales for the
+# inference kernels, verl NVFP4 QAT article 2.5 -- but not the layout.)
+
+def mma_scale_bytes(B, M, S):
+    return B * (-(-M // 128)) * (-(-S // 4)) * 512
+
+
+def mma_scale_offset(M, S, b, r, c):
+    """Byte offset of the scale of (batch b, row r, scale column c)."""
+    ct = -(-S // 4)
+    slab = (-(-M // 128)) * ct * 512
+    return b * slab + ((r // 128) * ct + c // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + c % 4
+
+
+def mma_scale_layout(dense):
+    """Dense scale bytes [M][S] or [B][M][S] -> the tile layout (uint8, flat)."""
+    d = np.asarray(dense, np.uint8)
+    d3 = d if d.ndim == 3 else d[None]
+    B, M, S = d3.shape
+    out = np.zeros(mma_scale_bytes(B, M, S), np.uint8)
+    b, r, c = np.meshgrid(np.arange(B), np.arange(M), np.arange(S), indexing="ij")
+    out[mma_scale_offset(M, S, b, r, c)] = d3
+    return out
+
+
+def mma_scale_dense(mma, B, M, S):
+    """The tile layout back to dense [B][M][S] scale bytes."""
+    m = np.asarray(mma, np.uint8).reshape(-1)
+    b, r, c = np.meshgrid(np.arange(B), np.arange(M), np.arange(S), indexing="ij")
+    return m[mma_scale_offset(M, S, b, r, c)]

@@ -28,7 +28,8 @@ __all__ = [
     "mxfp8_quant_grouped", "mxfp8_dequant_grouped", "nvfp4_dequant_grouped", "nvfp4_quant_grouped",
     "nvfp4_fake_quant_grouped", "fp8_block_requant", "fp8_block_requant_mxfp8", "fp8_block_requant_nvfp4",
     "fp8_block_requant_nvfp4_grouped", "fp8_block_requant_grouped", "fp8_block_requant_mxfp8_grouped",
-    "NVFP4ActivationObserver", "nvfp4_w4a4_fake_quant_ste", "OBSERVERS",
+    "NVFP4ActivationObserver", "nvfp4_w4a4_fake_quant_ste", "OBSERVERS", "mma_scale_bytes", "scales_to_mma",
+    "scales_from_mma", "mxfp8_quant_grouped_mma", "nvfp4_quant_grouped_mma",
 ]
 
 _CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
@@ -389,6 +390,78 @@ def nvfp4_fake_quant_grouped(groups: Sequence[Sequence[torch.Tensor]], out=None,
     check(lib.nvfp4_fake_quant_grouped(len(groups), sizes, ax, _desc_array([y for g in out for y in g], "out"), ao,
                                        ws.data_ptr(), ws.numel(), _stream(flat[0])), "nvfp4_fake_quant_grouped")
     return out
+
+
+# ---------------------------------------------------------------- block scales in the tensor-core layout
+
+def mma_scale_bytes(batch: int, rows: int, scale_cols: int) -> int:
+    """Bytes of an [B][M][S] scale array in the tensor-core tile layout
+    (include/pwq.h: 128 x 4 tiles of 512 bytes, zero padding)."""
+    return int(lib.pwq_mma_scale_bytes(batch, rows, scale_cols))
+
+
+def _scale_shape(dense_or_shape):
+    shape = tuple(dense_or_shape.shape) if isinstance(dense_or_shape, torch.Tensor) else tuple(dense_or_shape)
+    return (1,) + shape if len(shape) == 2 else shape
+
+
+def scales_to_mma(dense: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Dense scale bytes [.., M, S] (uint8 or float8_e4m3fn) -> the tile
+    layout, a flat uint8 tensor of mma_scale_bytes(B, M, S) bytes."""
+    if not dense.is_contiguous():
+        raise ValueError("dense scales must be contiguous")
+    B, M, S = _scale_shape(dense)
+    if out is None:
+        out = torch.empty(mma_scale_bytes(B, M, S), dtype=torch.uint8, device=dense.device)
+    check(lib.pwq_scales_to_mma(dense.data_ptr(), B, M, S, out.data_ptr(), _stream(dense)), "pwq_scales_to_mma")
+    return out
+
+
+def scales_from_mma(mma: torch.Tensor, shape, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The tile layout back to dense uint8 scale bytes of `shape` ([M, S] or [B, M, S])."""
+    B, M, S = _scale_shape(shape)
+    if out is None:
+        out = torch.empty(tuple(shape), dtype=torch.uint8, device=mma.device)
+    check(lib.pwq_scales_from_mma(mma.data_ptr(), B, M, S, out.data_ptr(), _stream(mma)), "pwq_scales_from_mma")
+    return out
+
+
+def mxfp8_quant_grouped_mma(xs: Sequence[torch.Tensor], out=None, scale=None):
+    """mxfp8_quant_grouped with every tensor's UE8M0 scales written in the
+    tensor-core tile layout.  Returns (codes list, flat uint8 scale arrays)."""
+    xs = list(xs)
+    if out is None:
+        out = [torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device) for x in xs]
+    if scale is None:
+        scale = [torch.empty(mma_scale_bytes(*_scale_shape(x.shape[:-1] + (x.shape[-1] // 32,))), dtype=torch.uint8,
+                             device=x.device) for x in xs]
+    if xs:
+        check(lib.mxfp8_quant_grouped_mma(len(xs), _desc_array(xs, "x"), _desc_array(out, "out"), _ptrs(scale),
+                                          _stream(xs[0])), "mxfp8_quant_grouped_mma")
+    return out, scale
+
+
+def nvfp4_quant_grouped_mma(groups: Sequence[Sequence[torch.Tensor]], out=None, sb=None, global_scale=None):
+    """nvfp4_quant_grouped with the E4M3 block scales written in the
+    tensor-core tile layout (flat uint8 arrays, one per member)."""
+    groups, flat, sizes = _groups(groups)
+    dev = flat[0].device
+    if out is None:
+        out = [[torch.empty(x.shape[:-1] + (x.shape[-1] // 2,), dtype=torch.uint8, device=dev) for x in g]
+               for g in groups]
+    if sb is None:
+        sb = [[torch.empty(mma_scale_bytes(*_scale_shape(x.shape[:-1] + (x.shape[-1] // 16,))), dtype=torch.uint8,
+                           device=dev) for x in g] for g in groups]
+    if global_scale is None:
+        global_scale = [torch.empty(_batch(g[0]), dtype=torch.float32, device=dev) for g in groups]
+    ax = _desc_array(flat, "x")
+    ws_bytes = int(lib.nvfp4_workspace_size_grouped(len(groups), sizes, ax))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    check(lib.nvfp4_quant_grouped_mma(len(groups), sizes, ax,
+                                      _desc_array([p for g in out for p in g], "out", packed=True),
+                                      _ptrs([s for g in sb for s in g]), _ptrs(global_scale), ws.data_ptr(),
+                                      ws.numel(), _stream(flat[0])), "nvfp4_quant_grouped_mma")
+    return out, sb, global_scale
 
 
 # ---------------------------------------------------------------- diagnostics

@@ -79,6 +79,11 @@ _SIG = {
     "pwq_selftest_flow_timeout_workspace_size": (ctypes.c_size_t, [_T]),
     "pwq_selftest_flow_timeout": (_S, [_T, _T, ctypes.c_uint64, _P, ctypes.c_size_t, _P]),
     "nvfp4_fake_quant_noalloc": (_S, [_T, _T, ctypes.c_int, _P, _P, _P]),
+    "pwq_mma_scale_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]),
+    "pwq_scales_to_mma": (_S, [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _P, _P]),
+    "pwq_scales_from_mma": (_S, [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _P, _P]),
+    "mxfp8_quant_grouped_mma": (_S, [ctypes.c_int, _T, _T, _PP, _P]),
+    "nvfp4_quant_grouped_mma": (_S, [ctypes.c_int, _IP, _T, _T, _PP, _PP, _P, ctypes.c_size_t, _P]),
 }
 
 

@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpwq.so")
-SOURCES = ["pwq_api.cu", "fp8_block.cu", "mxfp8.cu", "nvfp4.cu", "requant.cu", "observer.cu", "selftest.cu"]
+SOURCES = ["pwq_api.cu", "fp8_block.cu", "mxfp8.cu", "nvfp4.cu", "requant.cu", "observer.cu", "selftest.cu",
+           "scale_layout.cu"]
 HEADERS = ["pwq_device.cuh", "pwq_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

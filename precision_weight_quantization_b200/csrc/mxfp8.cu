@@ -215,13 +215,16 @@ struct BlockTensor {
     const char* in;
     char* out;
     int64_t in_bs, in_rs, out_bs, out_rs;   // bytes
-    uint8_t* e;            // dense [B][M][N/32] scale bytes
+    uint8_t* e;            // scale bytes: dense [B][M][N/32], or the tensor-core tile layout
     uint32_t blocks;       // B * M * N / 32
     uint32_t slot_begin;   // first block slot of this tensor (multiple of kBSpan)
     FastDiv bpr;           // blocks per row (N / 32)
     FastDiv rows;          // M
     int dense;             // both operands dense
     int in32, out32;       // BF16 rows / code rows (and slabs) 32-byte aligned
+    int sf_mma;            // scales in the tile layout: sf_ct column tiles, sf_slab bytes per batch slab
+    uint32_t sf_ct;
+    int64_t sf_slab;
 };
 
 struct BlockArgs {
@@ -304,7 +307,14 @@ __global__ void __launch_bounds__(kThreads) mxfp8_quant_block_kernel(const __gri
 #pragma unroll
                 for (int h = 0; h < 4; ++h) st_v2(dst + 8 * h, make_uint2(q[2 * h], q[2 * h + 1]));
             }
-            T.e[bis[u]] = (uint8_t)(e + 127);
+            if (T.sf_mma) {
+                const uint32_t r = fdiv(bis[u], T.bpr);          // row over all batches
+                const uint32_t b = fdiv(r, T.rows);
+                const uint32_t m = r - b * T.rows.d;
+                T.e[(int64_t)b * T.sf_slab + mma_scale_offset(m, bis[u] - r * T.bpr.d, T.sf_ct)] = (uint8_t)(e + 127);
+            } else {
+                T.e[bis[u]] = (uint8_t)(e + 127);
+            }
         }
     }
 }
@@ -341,6 +351,9 @@ cudaError_t launch_mx_quant_blocks(const Job* jobs, int n, cudaStream_t s) {
             T.dense = dense_view(x, x.cols * 2) && dense_view(q, q.cols);
             T.in32 = aligned32(j.in);
             T.out32 = aligned32(j.out);
+            T.sf_mma = j.scale_mma;
+            T.sf_ct = (uint32_t)mma_scale_col_tiles(x.cols / 32);
+            T.sf_slab = mma_scale_slab_bytes(x.rows, x.cols / 32);
             slots += (uint32_t)padded;
         }
         j0 += a.n;

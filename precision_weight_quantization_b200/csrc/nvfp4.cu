@@ -386,6 +386,9 @@ struct FlowMember {
     int64_t ts_bs;        // FP8 source: TM * TN
     uint32_t tn;          // FP8 source: TN
     int vec32_o;          // fake-quant output slab and rows 32-byte aligned
+    int sf_mma;           // quant: block scales in the tensor-core tile layout (sf_ct column tiles,
+    uint32_t sf_ct;       // sf_slab bytes per batch slab) instead of dense [B][M][N/16]
+    int64_t sf_slab;
 };
 
 struct FlowGroup {
@@ -560,7 +563,7 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
                                             float r6, bool fast6, uint64_t pol) {
     const uint32_t tid = threadIdx.x;
     char* ob = M.out + (int64_t)it.b * M.o_bs;
-    uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.chunks >> 1);
+    uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.sf_mma ? M.sf_slab : (int64_t)(M.chunks >> 1));
 #pragma unroll
     for (int i = 0; i < kItemChunksPerThread / 2; ++i) {
         const uint4 lo = v[2 * i], hi = v[2 * i + 1];
@@ -607,7 +610,12 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
                 }
             } else {
                 st_hint_v2(ob + oo, c0, c1, pol);   // 8-byte aligned: c even, packed rows 8-byte aligned
-                sbb[c >> 1] = (uint8_t)sb;
+                if (M.sf_mma) {
+                    const uint32_t r = fdiv(c, M.cpr);
+                    sbb[mma_scale_offset(r, (c - r * M.cpr.d) >> 1, M.sf_ct)] = (uint8_t)sb;
+                } else {
+                    sbb[c >> 1] = (uint8_t)sb;
+                }
             }
         }
     }
@@ -1089,7 +1097,10 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
                 M.o_bs = o.bstride;
                 M.o_rs = o.rstride;
                 M.chunks = (uint32_t)(x.rows * (x.cols / 8));
-                M.sb = fake ? nullptr : G.sb[i] + b0 * (int64_t)(M.chunks / 2);
+                M.sf_mma = G.sb_mma;
+                M.sf_ct = (uint32_t)mma_scale_col_tiles(x.cols / 16);
+                M.sf_slab = mma_scale_slab_bytes(x.rows, x.cols / 16);
+                M.sb = fake ? nullptr : G.sb[i] + b0 * (G.sb_mma ? M.sf_slab : (int64_t)(M.chunks / 2));
                 M.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
                 M.dense_x = dense_rows(x, fp8 ? x.cols : x.cols * 2);
                 M.dense_o = dense_rows(o, fake ? o.cols * 2 : o.cols / 2);

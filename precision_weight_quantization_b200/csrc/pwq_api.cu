@@ -189,7 +189,7 @@ size_t scale_bytes(Op op, const pwq_tensor* t) {
 // grouped call.  scale[i] is an input for dequantise ops and an output for
 // quantise ops; gs (NVFP4 dequant only) an input.
 pwq_status run_list(Op op, int n, const pwq_tensor* in, const pwq_tensor* out, void* const* scale,
-                    const float* const* gs, pwq_stream_t stream) {
+                    const float* const* gs, pwq_stream_t stream, bool scale_mma = false) {
     if (n < 0 || n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "tensor count out of range");
     if (n == 0) return PWQ_OK;
     if (!in || !out || !scale) return fail(PWQ_ERR_NULL, "tensor or scale array");
@@ -217,7 +217,10 @@ pwq_status run_list(Op op, int n, const pwq_tensor* in, const pwq_tensor* out, v
         if (fp8 && (uintptr_t)scale[i] % 4 != 0) return fail(PWQ_ERR_ALIGN, "scale");
         j.scale = scale[i];
         j.gs = nullptr;
-        const Extent es = extent_of(scale[i], scale_bytes(op, a));
+        j.scale_mma = scale_mma ? 1 : 0;
+        const Extent es = extent_of(scale[i], scale_mma ? (size_t)(a->batch * pwq::mma_scale_slab_bytes(
+                                                              a->rows, a->cols / 32))
+                                                        : scale_bytes(op, a));
         ins.push_back(ea);
         outs.push_back(eb);
         (quant ? outs : ins).push_back(es);
@@ -234,6 +237,13 @@ pwq_status run_list(Op op, int n, const pwq_tensor* in, const pwq_tensor* out, v
     if (jobs.empty()) return PWQ_OK;
     cudaStream_t s = (cudaStream_t)stream;
     const int m = (int)jobs.size();
+    if (scale_mma)
+        for (const Job& j : jobs)
+            if (pwq::mma_scale_padded(j.in.rows, j.in.cols / 32)) {
+                cudaError_t e = cudaMemsetAsync(
+                    j.scale, 0, (size_t)(j.in.batch * pwq::mma_scale_slab_bytes(j.in.rows, j.in.cols / 32)), s);
+                if (e != cudaSuccess) return cuda_fail(e);
+            }
     switch (op) {
         case Op::kFp8Quant: return from_cuda(pwq::launch_fp8_block_quant(jobs.data(), m, s));
         case Op::kFp8Dequant: return from_cuda(pwq::launch_fp8_block_dequant(jobs.data(), m, s));
@@ -329,6 +339,45 @@ pwq_status mxfp8_quant_grouped(int n, const pwq_tensor* x, const pwq_tensor* q, 
     return run_list(Op::kMxQuant, n, x, q, reinterpret_cast<void* const*>(scale), nullptr, stream);
 }
 
+pwq_status mxfp8_quant_grouped_mma(int n, const pwq_tensor* x, const pwq_tensor* q, uint8_t* const* scale_mma,
+                                   pwq_stream_t stream) {
+    return run_list(Op::kMxQuant, n, x, q, reinterpret_cast<void* const*>(scale_mma), nullptr, stream, true);
+}
+
+size_t pwq_mma_scale_bytes(int64_t batch, int64_t rows, int64_t scale_cols) {
+    if (batch < 0 || rows < 0 || scale_cols < 0) return 0;
+    return (size_t)(batch * pwq::mma_scale_slab_bytes(rows, scale_cols));
+}
+
+namespace {
+pwq_status scale_layout_args(const void* dense, int64_t batch, int64_t rows, int64_t scale_cols, const void* mma) {
+    if (batch < 0 || rows < 0 || scale_cols < 0 || batch > kMaxDim || rows > kMaxDim || scale_cols > kMaxDim)
+        return fail(PWQ_ERR_SHAPE, "negative or too large extent");
+    if (batch * rows * scale_cols > ((int64_t)1 << 40)) return fail(PWQ_ERR_SHAPE, "scale array too large");
+    if (batch == 0 || rows == 0 || scale_cols == 0) return PWQ_OK;
+    if (!dense || !mma) return fail(PWQ_ERR_NULL, "scale array");
+    if ((uintptr_t)mma % 16 != 0) return fail(PWQ_ERR_ALIGN, "tile-layout array (16-byte aligned)");
+    const Extent ed = extent_of(dense, (size_t)(batch * rows * scale_cols));
+    const Extent em = extent_of(mma, (size_t)(batch * pwq::mma_scale_slab_bytes(rows, scale_cols)));
+    if (overlaps(ed, em)) return fail(PWQ_ERR_OVERLAP, "dense and tile-layout arrays overlap");
+    return PWQ_OK;
+}
+}  // namespace
+
+pwq_status pwq_scales_to_mma(const uint8_t* dense, int64_t batch, int64_t rows, int64_t scale_cols, uint8_t* mma,
+                             pwq_stream_t stream) {
+    pwq_status st = scale_layout_args(dense, batch, rows, scale_cols, mma);
+    if (st != PWQ_OK || batch == 0 || rows == 0 || scale_cols == 0) return st;
+    return from_cuda(pwq::launch_scales_to_mma(dense, batch, rows, scale_cols, mma, (cudaStream_t)stream));
+}
+
+pwq_status pwq_scales_from_mma(const uint8_t* mma, int64_t batch, int64_t rows, int64_t scale_cols, uint8_t* dense,
+                               pwq_stream_t stream) {
+    pwq_status st = scale_layout_args(dense, batch, rows, scale_cols, mma);
+    if (st != PWQ_OK || batch == 0 || rows == 0 || scale_cols == 0) return st;
+    return from_cuda(pwq::launch_scales_from_mma(mma, batch, rows, scale_cols, dense, (cudaStream_t)stream));
+}
+
 pwq_status mxfp8_dequant_grouped(int n, const pwq_tensor* q, const uint8_t* const* scale, const pwq_tensor* y,
                                  pwq_stream_t stream) {
     return run_list(Op::kMxDequant, n, q, y, reinterpret_cast<void* const*>(const_cast<uint8_t**>(scale)),
@@ -375,7 +424,7 @@ struct GroupCheck {
 // fake-quantise.
 pwq_status check_nv_group(const pwq_tensor* x, const pwq_tensor* out, uint8_t* const* sb, int n, bool fake,
                           GroupCheck* G, std::vector<Extent>& ins, std::vector<Extent>& outs,
-                          std::vector<std::pair<Extent, Extent>>& aliases) {
+                          std::vector<std::pair<Extent, Extent>>& aliases, bool sb_mma = false) {
     Extent ex[PWQ_MAX_SIBLINGS];
     pwq_status st = check_siblings(x, n, G->x, ex, &G->all_empty);
     if (st != PWQ_OK) return st;
@@ -400,7 +449,8 @@ pwq_status check_nv_group(const pwq_tensor* x, const pwq_tensor* out, uint8_t* c
         if (!fake) {
             if (!sb[i]) return fail(PWQ_ERR_NULL, "sb[i]");
             G->sb[i] = sb[i];
-            outs.push_back(extent_of(sb[i], (size_t)(B * x[i].rows * (x[i].cols / 16))));
+            outs.push_back(extent_of(sb[i], sb_mma ? (size_t)(B * pwq::mma_scale_slab_bytes(x[i].rows, x[i].cols / 16))
+                                                   : (size_t)(B * x[i].rows * (x[i].cols / 16))));
         }
     }
     return PWQ_OK;
@@ -468,7 +518,7 @@ namespace {
 // Shared body of nvfp4_quant / nvfp4_fake_quant and their grouped forms.
 pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq_tensor* out,
                   uint8_t* const* sb, float* const* gs_out, const float* amax_in, float* const* amax_out,
-                  void* ws, size_t ws_bytes, bool fake, pwq_stream_t stream) {
+                  void* ws, size_t ws_bytes, bool fake, pwq_stream_t stream, bool sb_mma = false) {
     if (n_groups < 1 || n_groups > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group count out of range");
     if (!sizes || !x || !out) return fail(PWQ_ERR_NULL, "group sizes / tensors");
     std::vector<GroupCheck> groups(n_groups);
@@ -481,11 +531,13 @@ pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq
         const int n = sizes[g];
         if (n < 1 || n > PWQ_MAX_SIBLINGS || m + n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group size");
         GroupCheck& G = groups[g];
-        pwq_status st = check_nv_group(x + m, out + m, fake ? nullptr : sb + m, n, fake, &G, ins, outs, aliases);
+        pwq_status st =
+            check_nv_group(x + m, out + m, fake ? nullptr : sb + m, n, fake, &G, ins, outs, aliases, sb_mma);
         if (st != PWQ_OK) return st;
         const int64_t B = x[m].batch;
         if (!G.all_empty && B > 0) {
             pwq::NvGroup ng;
+            ng.sb_mma = sb_mma ? 1 : 0;
             ng.x = G.x;
             ng.out = G.out;
             ng.sb = fake ? nullptr : G.sb;
@@ -523,6 +575,18 @@ pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq
     pwq_status st = check_nv_overlaps(ins, outs, aliases);
     if (st != PWQ_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
+    if (sb_mma) {
+        // the tile layout's padding (rows to 128, columns to 4) is zero bytes
+        for (const pwq::NvGroup& G : launch)
+            for (int i = 0; i < G.n; ++i) {
+                const pwq::View& v = G.x[i];
+                if (v.rows > 0 && pwq::mma_scale_padded(v.rows, v.cols / 16)) {
+                    cudaError_t e = cudaMemsetAsync(G.sb[i], 0, (size_t)(v.batch * pwq::mma_scale_slab_bytes(
+                                                                    v.rows, v.cols / 16)), s);
+                    if (e != cudaSuccess) return cuda_fail(e);
+                }
+            }
+    }
     if (amax_in) {
         const pwq::NvGroup& G = launch[0];
         return from_cuda(pwq::launch_nvfp4_encode(G.x, G.n, G.out, G.sb, fake, nullptr, amax_in, G.gs_out,
@@ -553,6 +617,13 @@ pwq_status nvfp4_quant_grouped(int n_groups, const int* group_sizes, const pwq_t
                                void* workspace, size_t workspace_bytes, pwq_stream_t stream) {
     return nv_run(n_groups, group_sizes, x, q_packed, sb, global_scale, nullptr, nullptr, workspace,
                   workspace_bytes, false, stream);
+}
+
+pwq_status nvfp4_quant_grouped_mma(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                                   const pwq_tensor* q_packed, uint8_t* const* sb_mma, float* const* global_scale,
+                                   void* workspace, size_t workspace_bytes, pwq_stream_t stream) {
+    return nv_run(n_groups, group_sizes, x, q_packed, sb_mma, global_scale, nullptr, nullptr, workspace,
+                  workspace_bytes, false, stream, true);
 }
 
 pwq_status nvfp4_fake_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,

@@ -40,7 +40,25 @@ struct Job {
     View in, out;
     void* scale;       // FP8: float [B][TM][TN]; MXFP8: uint8 [B][M][N/32]; NVFP4 dequant: uint8 sb [B][M][N/16]
     const float* gs;   // NVFP4 dequant: [B]
+    int scale_mma = 0; // MXFP8 quantise: scale bytes in the tensor-core tile layout instead of dense
 };
+
+// The tensor-core (block-scaled MMA) layout of an [B][M][S] array of scale
+// bytes: per batch slab, tiles of 128 rows x 4 scale columns, 512
+// contiguous bytes each, ordered along S within a 128-row band and band
+// after band; the scale of tile row r and column c at byte
+// (r % 32) * 16 + (r / 32) * 4 + c; rows padded to 128, columns to 4.
+inline int64_t mma_scale_col_tiles(int64_t S) { return (S + 3) / 4; }
+inline int64_t mma_scale_slab_bytes(int64_t M, int64_t S) { return (M + 127) / 128 * mma_scale_col_tiles(S) * 512; }
+inline bool mma_scale_padded(int64_t M, int64_t S) { return M % 128 != 0 || S % 4 != 0; }
+// Byte offset of (row r, scale column c) inside one slab (device and host).
+__host__ __device__ __forceinline__ uint32_t mma_scale_offset(uint32_t r, uint32_t c, uint32_t col_tiles) {
+    return ((r >> 7) * col_tiles + (c >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (c & 3u);
+}
+cudaError_t launch_scales_to_mma(const uint8_t* dense, int64_t B, int64_t M, int64_t S, uint8_t* mma,
+                                 cudaStream_t s);
+cudaError_t launch_scales_from_mma(const uint8_t* mma, int64_t B, int64_t M, int64_t S, uint8_t* dense,
+                                   cudaStream_t s);
 
 cudaError_t launch_fp8_block_quant(const Job* jobs, int n, cudaStream_t s);
 cudaError_t launch_fp8_block_dequant(const Job* jobs, int n, cudaStream_t s);
@@ -58,6 +76,7 @@ struct NvGroup {
     float* gs_out;          // [B] or null
     float* amax_out;        // [B] or null
     const float* const* ts = nullptr;   // FP8 block-wise source: n tile-scale arrays (x are E4M3 code views)
+    int sb_mma = 0;                     // quantise: block scales in the tensor-core tile layout
 };
 
 // NVFP4 single-pass quantise / fake-quantise of groups whose amax is reduced

@@ -266,3 +266,35 @@ def test_flow_timeout_selftest_validation_without_gpu():
     assert lib.pwq_selftest_flow_timeout(by(xb), by(yb), 10 ** 6, ws, 1 << 20, None) == L.PWQ_ERR_SHAPE
     xe = T(L, None, 1, 0, 512, 0, 512)
     assert lib.pwq_selftest_flow_timeout(by(xe), by(xe), 10 ** 6, ws, n, None) == L.PWQ_ERR_SHAPE
+
+
+def test_scale_layout_validation_without_gpu():
+    L = _lib()
+    lib = L.lib
+    base = 1 << 40
+    assert lib.pwq_mma_scale_bytes(2, 200, 10) == 2 * 2 * 3 * 512
+    assert lib.pwq_mma_scale_bytes(1, 128, 4) == 512
+    assert lib.pwq_mma_scale_bytes(-1, 1, 1) == 0
+    d, m = base, base + (1 << 30)
+    assert lib.pwq_scales_to_mma(None, 1, 128, 4, m, None) == L.PWQ_ERR_NULL
+    assert lib.pwq_scales_to_mma(d, 1, 128, 4, m + 8, None) == L.PWQ_ERR_ALIGN
+    assert lib.pwq_scales_to_mma(d, 1, -1, 4, m, None) == L.PWQ_ERR_SHAPE
+    assert lib.pwq_scales_to_mma(d, 1, 128, 4, d + 256, None) == L.PWQ_ERR_OVERLAP
+    assert lib.pwq_scales_from_mma(m, 1, 128, 4, m + 100, None) == L.PWQ_ERR_OVERLAP
+    assert lib.pwq_scales_to_mma(None, 0, 128, 4, None, None) == L.PWQ_OK           # empty: no-op
+    # the fused quantisers check the tile-layout extent against the other operands
+    by = ctypes.byref
+    x = (L.PwqTensor * 1)(T(L, base, 1, 256, 512, 256 * 512, 512))
+    q = (L.PwqTensor * 1)(T(L, base + (1 << 30), 1, 256, 512, 256 * 512, 512))
+    sc_over_q = (ctypes.c_void_p * 1)(base + (1 << 30) + 64)
+    assert lib.mxfp8_quant_grouped_mma(1, x, q, sc_over_q, None) == L.PWQ_ERR_OVERLAP
+    pk = (L.PwqTensor * 1)(T(L, base + (1 << 30), 1, 256, 512, 256 * 256, 256))
+    sb_over_x = (ctypes.c_void_p * 1)(base + 1024)
+    gs = (ctypes.c_void_p * 1)(base + (3 << 30))
+    sizes = (ctypes.c_int * 1)(1)
+    ws = base + (4 << 30)
+    assert lib.nvfp4_quant_grouped_mma(1, sizes, x, pk, sb_over_x, gs, ws, 256, None) == L.PWQ_ERR_OVERLAP
+    x24 = (L.PwqTensor * 1)(T(L, base, 1, 4, 48, 4 * 48, 48))
+    q24 = (L.PwqTensor * 1)(T(L, base + (1 << 30), 1, 4, 48, 4 * 48, 48))
+    sc = (ctypes.c_void_p * 1)(base + (2 << 30))
+    assert lib.mxfp8_quant_grouped_mma(1, x24, q24, sc, None) == L.PWQ_ERR_SHAPE
