@@ -729,7 +729,26 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         uint4 v[kItemChunksPerThread];
         const unsigned char* buf = flow_smem + st * kFlowStageBytes;
         const bool full = (it.c1 - it.c0 == kItemChunks) && M.dense_x && M.dense_o;
-        if (full) {
+        // FP8 source, amax item over whole chunk pairs: the block maxima come
+        // from the largest code magnitude of each pair (one tile scale each),
+        // bf16(fl(dec(mc) |s|)) -- rounding is monotone and symmetric in sign,
+        // so that is the largest |y| of the pair -- without dequantising
+        uint32_t fp8_m = 0u;
+        const bool fp8_amax = kFp8 && full && !it.is_e;
+        if (fp8_amax) {
+#pragma unroll
+            for (int j = 0; j < kItemChunksPerThread; j += 2) {
+                const uint32_t lc = flow_lc(j, tid);
+                const uint4 cc = *reinterpret_cast<const uint4*>(buf + lc * 8u);
+                const uint32_t c = it.c0 + lc;
+                const uint32_t r = fdiv(c, M.cpr);
+                const uint32_t k = c - r * M.cpr.d;
+                const float sc = __ldg(M.ts + (int64_t)it.b * M.ts_bs + (r >> 7) * M.tn + (k >> 4));
+                const uint32_t lanes = __vmaxu2(e4m3_maxmag_lanes(make_uint2(cc.x, cc.y)),
+                                                e4m3_maxmag_lanes(make_uint2(cc.z, cc.w)));
+                fp8_m = max(fp8_m, fp8_amax_bits16(e4m3_maxmag_fin(lanes), sc));
+            }
+        } else if (full) {
             if (kFp8) {
 #pragma unroll
                 for (int j = 0; j < kItemChunksPerThread; j += 2) {
@@ -779,11 +798,16 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
 
         if (!it.is_e) {
             // ---- amax item
-            uint32_t mw = 0u;
+            uint32_t m;
+            if (fp8_amax) {
+                m = fp8_m;
+            } else {
+                uint32_t mw = 0u;
 #pragma unroll
-            for (int j = 0; j < kItemChunksPerThread; ++j) mw = hmax_abs(mw, amax_word8(v[j]));
-            mw &= 0x7fff7fffu;
-            uint32_t m = max(mw & 0xffffu, mw >> 16);
+                for (int j = 0; j < kItemChunksPerThread; ++j) mw = hmax_abs(mw, amax_word8(v[j]));
+                mw &= 0x7fff7fffu;
+                m = max(mw & 0xffffu, mw >> 16);
+            }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((tid & 31u) == 0u) red[k & 1u][tid >> 5] = m;
