@@ -451,47 +451,76 @@ __device__ __forceinline__ int flow_group_of(const FlowArgs& a, uint32_t inst) {
 }
 
 // The queue order.  pa[i] = items before instance i (pa[I] = total), n_i =
-// pa[i+1] - pa[i].  The amax items of instance j >= 1 are split into a head
-// H(j) of lead(j) = min(n_j, L) items and the tail T(j); the queue is
-//     A(0) H(1) E(0) T(1) H(2) E(1) T(2) ... H(I-1) E(I-2) T(I-1) E(I-1)
-// so E(i) starts at se(i) = pa[i+1] + pa[i] + lead(i+1), at least L items
-// after the last amax item of instance i.
-__device__ __forceinline__ uint32_t flow_lead(const uint32_t* pa, uint32_t I, uint32_t L, uint32_t j) {
-    return j < I ? min(pa[j + 1] - pa[j], L) : 0u;
-}
-
-// Queue position q -> (encode?, instance, item within the instance's pass).
-__device__ __forceinline__ void flow_decode(const FlowTables& t, uint32_t I, uint32_t L, uint32_t q, bool& is_e,
-                                            uint32_t& inst, uint32_t& k) {
+// pa[i+1] - pa[i].  The amax items of all instances form one stream, in
+// instance order; the encode items of instance i form one block, released
+// once the amax stream has gone lead(i) = max(min(n_{i+1}, L), Lmin) items
+// past the last amax item of instance i (or reached its end):
+//     R(i) = min(pa[i+1] + lead(i), total),   se(i) = pa[i] + R(i)
+// is the queue position of E(i)'s first item, and an amax item with stream
+// index a sits at a + pa[m], m being the number of encode blocks released
+// before it.  With instances of at least Lmin items this reads
+//     A(0) H(1) E(0) T(1) H(2) E(1) T(2) ... E(I-1),
+// H(j) the first min(n_j, L) amax items of instance j: E(i) re-reads
+// instance i while the head of the next instance is read, and the data it
+// re-reads was read at most n_i + lead(i) items ago.  Lmin (one item per
+// CTA of the grid) matters for small instances: releasing E(i) after the
+// few items of a small next instance chained them -- a CTA that claimed an
+// encode item ahead of its own amax items of a later instance made that
+// instance's encode wait on its encode (64 instances of 8 items took 113
+// us against 27 with the minimum lead).
+//
+// A decoding thread takes positions in increasing order, so it keeps in
+// `hint` the last encode block it found (se[hint] <= every later q) and
+// steps forward from there; a CTA's consecutive positions are about a grid
+// apart, a fraction of an instance of the large workloads, so one or two
+// steps usually do, and the binary search runs only after four.
+__device__ __forceinline__ void flow_decode(const FlowTables& t, uint32_t I, uint32_t q, uint32_t& hint,
+                                            bool& is_e, uint32_t& inst, uint32_t& k) {
+    uint32_t a = q, lo = 0;
+    if (q >= t.se[0]) {
+        lo = hint;
+        int fwd = 0;
+        while (lo + 1 < I && t.se[lo + 1] <= q && fwd < 4) {
+            ++lo;
+            ++fwd;
+        }
+        if (fwd == 4) {
+            uint32_t hi = I - 1;
+            while (lo < hi) {
+                const uint32_t mid = (lo + hi + 1) >> 1;
+                if (t.se[mid] <= q) lo = mid; else hi = mid - 1;
+            }
+        }
+        hint = lo;
+        if (q < t.se[lo] + (t.pa[lo + 1] - t.pa[lo])) {
+            is_e = true;
+            inst = lo;
+            k = q - t.se[lo];
+            return;
+        }
+        a = q - t.pa[lo + 1];   // the encode items of instances 0..lo precede q
+        ++lo;                   // and a >= R(lo) >= pa[lo + 1]
+    }
     is_e = false;
-    if (q < t.se[0]) {
-        inst = q < t.pa[1] ? 0u : 1u;
-        k = q - t.pa[inst];
-        return;
+    // the instance of amax stream index a: with instances of Lmin items or
+    // more it is lo or one of the next two, so a few forward steps find it
+    // (a second binary search over hundreds of instances would sit on the
+    // decoding thread's path every item); smaller instances fall back to
+    // the search
+    int steps = 0;
+    while (lo + 1 < I && t.pa[lo + 1] <= a && steps < 4) {
+        ++lo;
+        ++steps;
     }
-    uint32_t lo = 0, hi = I - 1;
-    while (lo < hi) {
-        const uint32_t mid = (lo + hi + 1) >> 1;
-        if (t.se[mid] <= q) lo = mid; else hi = mid - 1;
+    if (steps == 4) {
+        uint32_t hi = I - 1;
+        while (lo < hi) {
+            const uint32_t mid = (lo + hi + 1) >> 1;
+            if (t.pa[mid] <= a) lo = mid; else hi = mid - 1;
+        }
     }
-    const uint32_t s = t.se[lo], n = t.pa[lo + 1] - t.pa[lo];
-    if (q < s + n) {
-        is_e = true;
-        inst = lo;
-        k = q - s;
-        return;
-    }
-    // T(lo + 1), then H(lo + 2)
-    const uint32_t r = q - s - n, j = lo + 1;
-    const uint32_t lj = flow_lead(t.pa, I, L, j);
-    const uint32_t tail = t.pa[j + 1] - t.pa[j] - lj;
-    if (r < tail) {
-        inst = j;
-        k = lj + r;
-    } else {
-        inst = j + 1;
-        k = r - tail;
-    }
+    inst = lo;
+    k = a - t.pa[lo];
 }
 
 // A decoded queue item.  Thread 0 decodes items kFlowStages ahead of the CTA
@@ -502,14 +531,14 @@ struct FlowItem {
     uint32_t b, c0, c1;              // batch index in the group; chunk range of the member slab
 };
 
-__device__ __forceinline__ FlowItem flow_item(const FlowTables& t, uint32_t I, uint32_t total, uint32_t L,
-                                              uint32_t q) {
+__device__ __forceinline__ FlowItem flow_item(const FlowTables& t, uint32_t I, uint32_t total, uint32_t q,
+                                              uint32_t& hint) {
     FlowItem it{};
     it.valid = q < 2u * total;
     if (!it.valid) return it;
     bool is_e;
     uint32_t inst, k;
-    flow_decode(t, I, L, q, is_e, inst, k);
+    flow_decode(t, I, q, hint, is_e, inst, k);
     const int g = t.ig[inst];
     const FlowGroup& G = t.g[g];
     if (is_e) k = G.items - 1u - k;                    // encode walks the instance backwards
@@ -692,11 +721,15 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         for (int s = 0; s <= kFlowStages; ++s) s_q[s] = atomicAdd(a.counter, 1u);
     }
     __syncthreads();
-    for (uint32_t i = tid; i < I; i += blockDim.x) t.se[i] = t.pa[i + 1] + t.pa[i] + flow_lead(t.pa, I, L, i + 1);
+    for (uint32_t i = tid; i < I; i += blockDim.x) {
+        const uint32_t next_n = i + 1 < I ? t.pa[i + 2] - t.pa[i + 1] : 0u;
+        t.se[i] = t.pa[i] + min(t.pa[i + 1] + max(min(next_n, L), gridDim.x), total);
+    }
     __syncthreads();
     if (tid == 0) {
+        uint32_t hint0 = 0u;
         for (int s = 0; s < kFlowStages; ++s) {
-            items[s] = flow_item(t, I, total, L, s_q[s]);
+            items[s] = flow_item(t, I, total, s_q[s], hint0);
             if (items[s].valid)
                 flow_stage(t.m[items[s].m], items[s], stage0 + s * kFlowStageBytes, smem_addr(&bars[s]),
                            flow_amax_policy(t, items[s], keep, stream));
@@ -705,6 +738,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
     __syncthreads();
     // thread kQueueThread: queue position of the item kFlowStages ahead
     uint32_t pend = s_q[kFlowStages];
+    uint32_t hint = 0u;   // thread kQueueThread: its last encode block (flow_decode)
 
     uint32_t cached = 0xffffffffu;
     float gs = 0.0f, six_gs = 0.0f, r6 = 0.0f;
@@ -812,7 +846,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((tid & 31u) == 0u) red[k & 1u][tid >> 5] = m;
             if (tid == kQueueThread) {
-                items[ahead] = flow_item(t, I, total, L, pend);
+                items[ahead] = flow_item(t, I, total, pend, hint);
                 pend = next_q;
             }
             __syncthreads();   // stage st is free; red and the new item are published
@@ -838,7 +872,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         // ---- encode item: wait (bounded) for the instance's amax
         const FlowGroup& G = t.g[it.g];
         if (tid == kQueueThread) {
-            items[ahead] = flow_item(t, I, total, L, pend);
+            items[ahead] = flow_item(t, I, total, pend, hint);
             pend = next_q;
         }
         if (tid == 0) {
