@@ -361,14 +361,14 @@ __global__ void __launch_bounds__(kThreads) nvfp4_dequant_kernel(const __grid_co
 // amax item publishes its max with atomicMax and then counts itself done
 // (fence + atomicAdd); the waiting side reads the count with acquire
 // semantics before it reads the amax.
-constexpr int kFlowThreads = 128;
-constexpr uint32_t kItemChunks = 1024;                        // 16384 elements
+constexpr int kFlowThreads = 256;
+constexpr uint32_t kItemChunks = 2048;                        // 16384 elements
 constexpr int kItemChunksPerThread = kItemChunks / kFlowThreads;   // 8
 constexpr int kFlowMaxInst = 512;                             // instances per launch
 constexpr uint64_t kFlowWaitNs = kFlowWaitLimitNs;             // 2 s
-constexpr uint32_t kFlowLeadPerCta = 5;                       // L = kFlowLeadPerCta * grid
+constexpr uint32_t kFlowLeadPerCta = 4;                       // L = kFlowLeadPerCta * grid
 constexpr int kFlowStages = 2;
-constexpr int kFlowCtasPerSm = 5;
+constexpr int kFlowCtasPerSm = 3;
 constexpr uint32_t kFlowStageBytes = kItemChunks * 16u;   // 32 KB
 constexpr uint32_t kErrFlowTimeout = 2u;
 
@@ -671,7 +671,7 @@ __device__ __forceinline__ uint4 flow_fp8_chunk(const FlowMember& M, const FlowI
 // quantise / fake-quantise): every amax item kept 2.86 / 3.39, the last
 // 3072 items 2.87 / 3.39, 2048 2.82 / 3.33, 1024 2.82 / 3.30, 512 2.82 /
 // 3.35, 256 2.82 / 3.46, none 2.95 / 3.50.
-constexpr uint32_t kKeepItems = 2048;
+constexpr uint32_t kKeepItems = 1024;
 __device__ __forceinline__ uint64_t flow_amax_policy(const FlowTables& t, const FlowItem& it, uint64_t keep,
                                                      uint64_t stream) {
     if (it.is_e) return stream;
