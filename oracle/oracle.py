@@ -55,9 +55,13 @@ def lib():
         L.or_nvfp4_quant.argtypes = [P, I64, I64, F, P, P]
         L.or_nvfp4_dequant.argtypes = [P, P, F, I64, I64, P]
         L.or_nvfp4_fake_quant.argtypes = [P, I64, I64, F, P]
+        L.or_nvfp4_4over6_global_scale.argtypes = [F, ctypes.c_int]
+        L.or_nvfp4_4over6_global_scale.restype = F
+        L.or_nvfp4_4over6_quant.argtypes = [P, I64, I64, F, ctypes.c_int, P, P, P, P]
+        L.or_nvfp4_4over6_fake_quant.argtypes = [P, I64, I64, F, ctypes.c_int, P]
         for name in ("or_fp8_block_quant", "or_fp8_block_dequant", "or_mxfp8_quant",
                      "or_mxfp8_dequant", "or_nvfp4_quant", "or_nvfp4_dequant",
-                     "or_nvfp4_fake_quant"):
+                     "or_nvfp4_fake_quant", "or_nvfp4_4over6_quant", "or_nvfp4_4over6_fake_quant"):
             getattr(L, name).restype = None
         _LIB = L
     return _LIB
@@ -243,6 +247,56 @@ def unpack_e2m1(packed):
     out[..., 0::2] = packed & 0xF
     out[..., 1::2] = packed >> 4
     return out
+
+
+# ---------------------------------------------------------------- NVFP4 "4over6"
+#
+# vime pull request #503, NVFP4 QDQ config thread: NVTE_NVFP4_4OVER6 and
+# NVTE_NVFP4_4OVER6_E4M3_USE_256 (E4M3 maximum 256 instead of 448).  Each
+# block is scaled so its amax maps to 6 or to 4 and keeps the candidate with
+# the smaller squared error (readings R19-R21 of pwq_oracle.c; parity
+# unpinned against the pages, which give no selection rule).  The result is
+# plain NVFP4: nvfp4_dequant reads it.
+
+def nvfp4_4over6_global_scale(group_amax, e4m3_max=256):
+    return float(np.float32(lib().or_nvfp4_4over6_global_scale(np.float32(group_amax), int(e4m3_max))))
+
+
+def nvfp4_4over6_quant(x_bits, group_amax, e4m3_max=256, details=False):
+    """One member tensor [..., M, N] with its group's amax.  Returns (packed,
+    sb, gs), plus (choice u8 [..., N/16] of 4 / 6, err f32 [..., N/16, 2]
+    with the t = 6 error first) when ``details``."""
+    x = _c(x_bits, np.uint16)
+    N = x.shape[-1]
+    assert N % 16 == 0
+    x2 = _as_2d(x)
+    packed = np.empty(x.shape[:-1] + (N // 2,), np.uint8)
+    sb = np.empty(x.shape[:-1] + (N // 16,), np.uint8)
+    choice = np.empty(x.shape[:-1] + (N // 16,), np.uint8)
+    err = np.empty(x.shape[:-1] + (N // 16, 2), np.float32)
+    if x.size:
+        lib().or_nvfp4_4over6_quant(_p(x2), x2.shape[0], N, np.float32(group_amax), int(e4m3_max),
+                                    _p(packed), _p(sb), _p(choice), _p(err))
+    gs = nvfp4_4over6_global_scale(group_amax, e4m3_max)
+    if details:
+        return packed, sb, gs, choice, err
+    return packed, sb, gs
+
+
+def nvfp4_4over6_fake_quant(x_bits, group_amax, e4m3_max=256):
+    x = _c(x_bits, np.uint16)
+    N = x.shape[-1]
+    x2 = _as_2d(x)
+    y = np.empty(x.shape, np.uint16)
+    if x.size:
+        lib().or_nvfp4_4over6_fake_quant(_p(x2), x2.shape[0], N, np.float32(group_amax), int(e4m3_max), _p(y))
+    return y
+
+
+def nvfp4_4over6_quant_group(members, e4m3_max=256):
+    """A sibling group under 4over6: (A, [(packed, sb, gs) per member])."""
+    A = nvfp4_group_amax(members)
+    return A, [nvfp4_4over6_quant(m, A, e4m3_max) for m in members]
 
 
 # ---------------------------------------------------------------- FP8 block -> rollout formats

@@ -42,6 +42,16 @@
  *   R7 NVFP4 dequant y = bf16(fl((dec(c) * dec(sb)) * gs)).
  *   R8 Packed nibbles: element 2j in the low nibble, 2j+1 in the high one.
  *   R9 Sign of zero is kept everywhere.
+ *   R19-R21 (NVFP4 "4over6", [PR503] NVFP4 QDQ config thread: the flags
+ *      NVTE_NVFP4_4OVER6 and NVTE_NVFP4_4OVER6_E4M3_USE_256, which sets the
+ *      E4M3 maximum of the global scale to 256 instead of 448; the pages
+ *      give no selection rule, so the rule below is a reading and this
+ *      part is PARITY UNPINNED against the pages):
+ *   R19 gs = fl(A / (6 * E)), E the E4M3 maximum (448 or 256).
+ *   R20 Per block, candidate t in {6, 4}: sb_t = e4m3(fl(amax_b /
+ *      fl(t * gs))), then codes and values as R6, R7 with sb_t.
+ *   R21 err_t = sum over the block's elements, left to right in binary32,
+ *      of fl(fl(x - y_t)^2); t = 4 is kept iff err_4 < err_6.
  */
 #include <stdint.h>
 #include <string.h>
@@ -384,8 +394,9 @@ float or_nvfp4_global_scale(float group_amax) {
     return gs;
 }
 
-/* One 1x16 block: the E4M3 scale byte and the 16 codes (unpacked). */
-static void nvfp4_block(const uint16_t* xb, float gs, uint8_t* sb_out, uint8_t codes[NV_BLOCK]) {
+/* One 1x16 block whose amax is scaled to t (6 for NVFP4): the E4M3 scale
+ * byte and the 16 codes (unpacked). */
+static void nvfp4_block_to(const uint16_t* xb, float gs, float t, uint8_t* sb_out, uint8_t codes[NV_BLOCK]) {
     float amax_b = 0.0f;
     for (int j = 0; j < NV_BLOCK; j++) {
         float a = fabsf(or_bf16_to_f32(xb[j]));
@@ -395,9 +406,9 @@ static void nvfp4_block(const uint16_t* xb, float gs, uint8_t* sb_out, uint8_t c
     if (gs == 0.0f) {
         sb = 0x00;                                      /* R3 */
     } else {
-        float six_gs = 6.0f * gs;                       /* fl(6*gs) */
-        float ratio = amax_b / six_gs;                  /* fl(amax_b/fl(6*gs)) */
-        sb = or_e4m3_encode((double)ratio);             /* R5 */
+        float t_gs = t * gs;                            /* fl(t*gs) */
+        float ratio = amax_b / t_gs;                    /* fl(amax_b/fl(t*gs)) */
+        sb = or_e4m3_encode((double)ratio);             /* R5 (R20 for t = 4) */
     }
     *sb_out = sb;
     float d = (float)or_e4m3_decode(sb) * gs;          /* fl(dec(sb)*gs) */
@@ -410,6 +421,10 @@ static void nvfp4_block(const uint16_t* xb, float gs, uint8_t* sb_out, uint8_t c
             codes[j] = or_e2m1_encode((double)quot);
         }
     }
+}
+
+static void nvfp4_block(const uint16_t* xb, float gs, uint8_t* sb_out, uint8_t codes[NV_BLOCK]) {
+    nvfp4_block_to(xb, gs, 6.0f, sb_out, codes);
 }
 
 /* y = bf16(fl((dec(c) * dec(sb)) * gs)); the inner product is exact. */
@@ -458,6 +473,89 @@ void or_nvfp4_fake_quant(const uint16_t* x, int64_t M, int64_t N, float group_am
     for (int64_t k = 0; k < nb; k++) {
         uint8_t codes[NV_BLOCK], sbk;
         nvfp4_block(x + r * N + k * NV_BLOCK, gs, &sbk, codes);
+        for (int j = 0; j < NV_BLOCK; j++)
+            y[r * N + k * NV_BLOCK + j] = nvfp4_value(codes[j], sbk, gs);
+    }
+    env_leave(env);
+}
+
+/* ------------------------------------------------------------------ */
+/* NVFP4 "4over6": each block is scaled so that its amax maps to 6 (the */
+/* NVFP4 rule) or to 4, and keeps the one whose dequantised values are   */
+/* closer to x; the global scale leaves room for the larger block scale  */
+/* by using E = 256 as the E4M3 maximum.                                 */
+/*   [PR503] NVFP4 QDQ config thread (NVTE_NVFP4_4OVER6,                  */
+/*   NVTE_NVFP4_4OVER6_E4M3_USE_256 -> e4m3_max 256).  Readings R19-R21;  */
+/*   PARITY UNPINNED against the pages (no selection rule there).         */
+/* The output format is plain NVFP4: or_nvfp4_dequant reads it.          */
+/* ------------------------------------------------------------------ */
+
+/* R19: gs = fl(A / (6 * E)); 6 * 448 = 2688 and 6 * 256 = 1536 exactly. */
+float or_nvfp4_4over6_global_scale(float group_amax, int e4m3_max) {
+    fpenv_save env = env_enter();
+    float gs = group_amax / (float)(6 * e4m3_max);
+    env_leave(env);
+    return gs;
+}
+
+/* R21: sum of squared differences of the block's values and its
+ * dequantised values, left to right, every step one binary32 operation. */
+static float nvfp4_block_err(const uint16_t* xb, const uint8_t codes[NV_BLOCK], uint8_t sb, float gs) {
+    float err = 0.0f;
+    for (int j = 0; j < NV_BLOCK; j++) {
+        float d = or_bf16_to_f32(xb[j]) - or_bf16_to_f32(nvfp4_value(codes[j], sb, gs));
+        float sq = d * d;
+        err = err + sq;
+    }
+    return err;
+}
+
+/* One block under 4over6: the kept scale byte and codes; *choice = 4 or 6,
+ * and the two errors when err6 / err4 are not NULL. */
+static void nvfp4_4over6_block(const uint16_t* xb, float gs, uint8_t* sb_out, uint8_t codes[NV_BLOCK],
+                               uint8_t* choice, float* err6, float* err4) {
+    uint8_t sb6, sb4, c6[NV_BLOCK], c4[NV_BLOCK];
+    nvfp4_block_to(xb, gs, 6.0f, &sb6, c6);                                 /* R20, t = 6 */
+    nvfp4_block_to(xb, gs, 4.0f, &sb4, c4);                                 /* R20, t = 4 */
+    float e6 = nvfp4_block_err(xb, c6, sb6, gs), e4 = nvfp4_block_err(xb, c4, sb4, gs);
+    int four = e4 < e6;                                                     /* R21 */
+    *sb_out = four ? sb4 : sb6;
+    memcpy(codes, four ? c4 : c6, NV_BLOCK);
+    if (choice) *choice = four ? 4 : 6;
+    if (err6) *err6 = e6;
+    if (err4) *err4 = e4;
+}
+
+/* x dense [M][N] (N % 16 == 0) with its group's amax A.  choice (optional,
+ * [M][N/16]) receives 4 or 6 per block, err (optional, [M][N/16][2]) the
+ * two errors (t = 6 first). */
+void or_nvfp4_4over6_quant(const uint16_t* x, int64_t M, int64_t N, float group_amax, int e4m3_max,
+                           uint8_t* packed, uint8_t* sb, uint8_t* choice, float* err) {
+    fpenv_save env = env_enter();
+    float gs = group_amax / (float)(6 * e4m3_max);
+    int64_t nb = N / NV_BLOCK;
+    for (int64_t r = 0; r < M; r++)
+    for (int64_t k = 0; k < nb; k++) {
+        uint8_t codes[NV_BLOCK];
+        int64_t i = r * nb + k;
+        nvfp4_4over6_block(x + r * N + k * NV_BLOCK, gs, &sb[i], codes, choice ? &choice[i] : NULL,
+                           err ? &err[2 * i] : NULL, err ? &err[2 * i + 1] : NULL);
+        for (int j = 0; j < NV_BLOCK; j += 2)          /* R8 */
+            packed[r * (N / 2) + (k * NV_BLOCK + j) / 2] =
+                (uint8_t)(codes[j] | (codes[j + 1] << 4));
+    }
+    env_leave(env);
+}
+
+void or_nvfp4_4over6_fake_quant(const uint16_t* x, int64_t M, int64_t N, float group_amax, int e4m3_max,
+                                uint16_t* y) {
+    fpenv_save env = env_enter();
+    float gs = group_amax / (float)(6 * e4m3_max);
+    int64_t nb = N / NV_BLOCK;
+    for (int64_t r = 0; r < M; r++)
+    for (int64_t k = 0; k < nb; k++) {
+        uint8_t codes[NV_BLOCK], sbk;
+        nvfp4_4over6_block(x + r * N + k * NV_BLOCK, gs, &sbk, codes, NULL, NULL, NULL);
         for (int j = 0; j < NV_BLOCK; j++)
             y[r * N + k * NV_BLOCK + j] = nvfp4_value(codes[j], sbk, gs);
     }
