@@ -34,8 +34,8 @@ Qwen3-30B-A3B expert layer (128 experts, MXFP8, one call per layer over 48
 layers), the 2048-hidden QAT block (NVFP4 fake-quant of its sibling groups
 in one launch) and the two parts of the headline.  Workloads smaller than
 L2 are timed call by call with a 256 MB write between calls (L2 flushed).
-`next_rows` times the FP8 block-wise re-quantisation ops on the Qwen3-4B
-sweep.  `--impl reference` times the CPU oracle (all host threads) on a
+`next_rows` times the FP8 block-wise re-quantisation ops and the NVFP4
+"4over6" variant on the Qwen3-4B sweep.  `--impl reference` times the CPU oracle (all host threads) on a
 bounded sample of the headline workload.
 """
 import argparse
@@ -687,15 +687,51 @@ def next_calls(op, layers, buf, P, torch, per_call=1):
     return calls
 
 
+# NVFP4 "4over6" (E4M3 maximum 256) of the BF16 sweep, one call per sibling
+# group: the group amax pass and the encode pass that evaluates both block
+# candidates; algorithmic bytes as for NVFP4 (two reads of the input)
+FOUR_SIX_BYTES_PER_ELEM = {"nvfp4_4over6_quant": 2 + 2 + 0.5 + 1 / 16, "nvfp4_4over6_fake_quant": 2 + 2 + 2}
+FOUR_SIX_ONE_PASS_BYTES_PER_ELEM = {"nvfp4_4over6_quant": 2 + 0.5 + 1 / 16, "nvfp4_4over6_fake_quant": 2 + 2}
+
+
+def four_six_calls(op, layers, P, torch):
+    """One call per sibling group of every layer, each writing its own outputs."""
+    import workloads as W
+    calls = []
+    for lay in layers:
+        for grp in W.QWEN3_4B_GROUPS:
+            xs = [lay[n] for n in grp]
+            dev = xs[0].device
+            ws = torch.empty(256, dtype=torch.uint8, device=dev)
+            if op == "nvfp4_4over6_quant":
+                pk = [torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for x in xs]
+                sb = [torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev) for x in xs]
+                gs = torch.empty(1, dtype=torch.float32, device=dev)
+                calls.append(lambda xs=xs, pk=pk, sb=sb, gs=gs: P.nvfp4_4over6_quant(xs, 256, out=pk, sb=sb,
+                                                                                    global_scale=gs))
+            else:
+                ys = [torch.empty_like(x) for x in xs]
+                calls.append(lambda xs=xs, ys=ys: P.nvfp4_4over6_fake_quant(xs, 256, out=ys))
+    return calls
+
+
 def time_next_rows(args, w, P, torch, hbm_peak, peak_kind):
-    """Device time of each re-quantisation op over the Qwen3-4B sweep (its
-    own CUDA graph, replayed after the sweep's timing)."""
+    """Device time of each re-quantisation op, and of the NVFP4 4over6
+    variant, over the Qwen3-4B sweep (each its own CUDA graph, replayed after
+    the sweep's timing)."""
     layers, buf = w.tensors["layers"], w.tensors["buf"]
     elems = layer_elems() * len(layers)
     stream = torch.cuda.current_stream()
     out = {}
-    for op, bpe in NEXT_BYTES_PER_ELEM.items():
-        calls = next_calls(op, layers, buf, P, torch, w.tensors["per_call"])
+    ops = dict(NEXT_BYTES_PER_ELEM)
+    ops.update(FOUR_SIX_BYTES_PER_ELEM)
+    one_pass = dict(NEXT_ONE_PASS_BYTES_PER_ELEM)
+    one_pass.update(FOUR_SIX_ONE_PASS_BYTES_PER_ELEM)
+    for op, bpe in ops.items():
+        if op in FOUR_SIX_BYTES_PER_ELEM:
+            calls = four_six_calls(op, layers, P, torch)
+        else:
+            calls = next_calls(op, layers, buf, P, torch, w.tensors["per_call"])
         g = capture(calls, torch)
         for _ in range(args.warmup):
             g.replay()
@@ -711,10 +747,10 @@ def time_next_rows(args, w, P, torch, hbm_peak, peak_kind):
         ms = a.elapsed_time(b) / n
         gbs = elems * bpe / (ms / 1e3) / 1e9
         out[op] = {"ms": round(ms, 4), "elem_per_s": elems / (ms / 1e3), "alg_gbs": round(gbs, 1),
-                   "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "launches": len(calls),
+                   "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "launches": len(calls) * (2 if op in FOUR_SIX_BYTES_PER_ELEM else 1),
                    "bytes_per_elem": round(bpe, 5)}
-        if op in NEXT_ONE_PASS_BYTES_PER_ELEM:
-            g1 = elems * NEXT_ONE_PASS_BYTES_PER_ELEM[op] / (ms / 1e3) / 1e9
+        if op in one_pass:
+            g1 = elems * one_pass[op] / (ms / 1e3) / 1e9
             out[op].update({"alg_gbs_one_pass": round(g1, 1),
                             "frac_of_%s_hbm_one_pass" % peak_kind: round(g1 / hbm_peak, 4)})
         del g

@@ -234,6 +234,40 @@ pwq_status nvfp4_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_sibl
                             size_t workspace_bytes, pwq_stream_t stream);
 
 /* ===================================================================== */
+/* NVFP4 "4over6"                                                         */
+/* ===================================================================== */
+/*
+ * Source: vime pull request #503, review thread on the NVFP4 QDQ config
+ * (NVTE_NVFP4_4OVER6 switches the variant on; NVTE_NVFP4_4OVER6_E4M3_USE_256
+ * makes the E4M3 maximum of the global scale 256 instead of 448, and
+ * defaults to on with the variant).  The pages name the variant and the
+ * constant only; the per-block rule below is this library's reading, taken
+ * from the variant's name (a block's amax maps to 4 or to 6):
+ *   gs_b = fl(A_b / (6 E)),                     E = e4m3_max (256 or 448),
+ * and for each block, for t = 6 and t = 4:
+ *   sb_t = e4m3(fl(a / fl(t * gs_b))),  codes and values y_t as in NVFP4,
+ *   err_t = fl(fl(x_0 - y_t,0)^2) + ... + fl(fl(x_15 - y_t,15)^2), added
+ *           left to right in binary32;
+ * the block keeps t = 4 when err_4 < err_6, else t = 6.  With E = 256 the
+ * block scale of t = 4 stays below 384, inside E4M3.  The result is plain
+ * NVFP4 (nvfp4_dequant reads it); siblings, layouts, amax_in and amax_out
+ * are those of nvfp4_quant / nvfp4_fake_quant.
+ *
+ * Two launches: the group amax (skipped when amax_in is given) into
+ * workspace of at least nvfp4_4over6_workspace_size() bytes (4-byte
+ * aligned; 4 bytes per batch index, rounded up to 256), then one encode
+ * launch that evaluates both candidates of every block.
+ * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _STRIDE, _OVERLAP, _WORKSPACE,
+ * _ARG (e4m3_max not 256 or 448, n_siblings), _CUDA. */
+size_t nvfp4_4over6_workspace_size(int n_siblings, const pwq_tensor* x);
+pwq_status nvfp4_4over6_quant(const pwq_tensor* x, int n_siblings, const pwq_tensor* q_packed,
+                              uint8_t* const* sb, float* global_scale, const float* amax_in, int e4m3_max,
+                              void* workspace, size_t workspace_bytes, pwq_stream_t stream);
+pwq_status nvfp4_4over6_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_siblings,
+                                   const float* amax_in, float* amax_out, int e4m3_max, void* workspace,
+                                   size_t workspace_bytes, pwq_stream_t stream);
+
+/* ===================================================================== */
 /* Grouped calls: a list of independent tensors in one launch             */
 /* ===================================================================== */
 /*
@@ -508,6 +542,11 @@ pwq_status pwq_device_error(uint32_t* code);
  *              for every E2M1 code pair, block scale code 0..126 and global
  *              scale fl(a / 2688) (a = 0 or a positive finite BF16):
  *              [0] = code pairs, [1] = mismatching BF16 pairs.
+ *   which = 6  as 1 with the 4over6 global scale fl(a / 1536) (E = 256).
+ *   which = 7  as 2 with fl(6 * fl(a / 1536)).
+ *   which = 8  the 4over6 block-scale divisor of the candidate 4,
+ *              fl(4 * fl(a / 1536)); numerators |x| <= a.
+ *   which = 9  as 8 with fl(4 * fl(a / 2688)) (E = 448).
  * counts (device, 4 x uint64, zeroed by the call): [0] pairs checked,
  * [1] code mismatches, [2] binary32 quotient mismatches where |x| >= 2^-100
  * and the IEEE quotient is normal, [3] pairs whose divisor takes the

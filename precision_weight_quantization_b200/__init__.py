@@ -275,6 +275,68 @@ def nvfp4_fake_quant_ste(xs: Sequence[torch.Tensor], amax: Optional[torch.Tensor
     return list(_SiblingSTE.apply(amax, *xs))
 
 
+# ---------------------------------------------------------------- NVFP4 4over6
+
+def nvfp4_4over6_quant(xs, e4m3_max: int = 256, amax: Optional[torch.Tensor] = None, out=None, sb=None,
+                       global_scale: Optional[torch.Tensor] = None):
+    """NVFP4 "4over6" quantisation of a sibling group (vime pull request
+    #503, NVFP4 QDQ config: NVTE_NVFP4_4OVER6, E4M3 maximum 256 by default).
+    Every block keeps the candidate -- its amax mapped to 6 or to 4 -- whose
+    dequantised values have the smaller squared error; gs = fl(A / (6 E)).
+    Returns what nvfp4_quant returns; nvfp4_dequant reads the result."""
+    single = isinstance(xs, torch.Tensor)
+    xs = _siblings(xs)
+    dev = xs[0].device
+    B = _batch(xs[0])
+    if out is None:
+        out = [torch.empty(x.shape[:-1] + (x.shape[-1] // 2,), dtype=torch.uint8, device=dev) for x in xs]
+    if sb is None:
+        sb = [torch.empty(x.shape[:-1] + (x.shape[-1] // 16,), dtype=torch.float8_e4m3fn, device=dev)
+              for x in xs]
+    if global_scale is None:
+        global_scale = torch.empty(B, dtype=torch.float32, device=dev)
+    for t in sb:
+        if not t.is_contiguous():
+            raise ValueError("block scale tensors must be contiguous")
+    ax = _desc_array(xs, "x")
+    aq = _desc_array(out, "out", packed=True)
+    sbp = (ctypes.c_void_p * len(xs))(*[t.data_ptr() for t in sb])
+    ws = None
+    if amax is None:
+        ws = torch.empty(max(int(lib.nvfp4_4over6_workspace_size(len(xs), ax)), 256), dtype=torch.uint8, device=dev)
+    check(lib.nvfp4_4over6_quant(ax, len(xs), aq, sbp, global_scale.data_ptr(),
+                                 amax.data_ptr() if amax is not None else None, int(e4m3_max),
+                                 ws.data_ptr() if ws is not None else None,
+                                 ws.numel() if ws is not None else 0, _stream(xs[0])), "nvfp4_4over6_quant")
+    if single:
+        return out[0], sb[0], global_scale
+    return out, sb, global_scale
+
+
+def nvfp4_4over6_fake_quant(xs, e4m3_max: int = 256, amax: Optional[torch.Tensor] = None, out=None,
+                            inplace: bool = False, amax_out: Optional[torch.Tensor] = None):
+    """BF16 outputs equal to nvfp4_dequant(nvfp4_4over6_quant(x)), without
+    materialising codes.  Returns the output tensor or list of outputs."""
+    single = isinstance(xs, torch.Tensor)
+    xs = _siblings(xs)
+    if out is None:
+        out = xs if inplace else [torch.empty_like(x) for x in xs]
+    elif isinstance(out, torch.Tensor):
+        out = [out]
+    ax = _desc_array(xs, "x")
+    ay = _desc_array(out, "out")
+    ws = None
+    if amax is None:
+        ws = torch.empty(max(int(lib.nvfp4_4over6_workspace_size(len(xs), ax)), 256), dtype=torch.uint8,
+                         device=xs[0].device)
+    check(lib.nvfp4_4over6_fake_quant(ax, ay, len(xs), amax.data_ptr() if amax is not None else None,
+                                      amax_out.data_ptr() if amax_out is not None else None, int(e4m3_max),
+                                      ws.data_ptr() if ws is not None else None,
+                                      ws.numel() if ws is not None else 0, _stream(xs[0])),
+          "nvfp4_4over6_fake_quant")
+    return out[0] if single else out
+
+
 # ---------------------------------------------------------------- grouped calls (one launch per list)
 
 def _ptrs(ts):

@@ -52,6 +52,10 @@ _SIG = {
                          ctypes.c_size_t, _P]),
     "nvfp4_dequant": (_S, [_T, _P, _P, _T, _P]),
     "nvfp4_fake_quant": (_S, [_T, _T, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
+    "nvfp4_4over6_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _T]),
+    "nvfp4_4over6_quant": (_S, [_T, ctypes.c_int, _T, ctypes.POINTER(ctypes.c_void_p), _P, _P, ctypes.c_int, _P,
+                                ctypes.c_size_t, _P]),
+    "nvfp4_4over6_fake_quant": (_S, [_T, _T, ctypes.c_int, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "fp8_block_quant_grouped": (_S, [ctypes.c_int, _T, _T, _PP, _P]),
     "fp8_block_dequant_grouped": (_S, [ctypes.c_int, _T, _PP, _T, _P]),
     "mxfp8_quant_grouped": (_S, [ctypes.c_int, _T, _T, _PP, _P]),

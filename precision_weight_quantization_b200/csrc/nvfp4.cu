@@ -260,6 +260,131 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
     }
 }
 
+// NVFP4 "4over6" (vime pull request #503, NVFP4 QDQ config thread:
+// NVTE_NVFP4_4OVER6 and NVTE_NVFP4_4OVER6_E4M3_USE_256).  The global scale
+// leaves room for a larger block scale, gs = fl(A / (6 E)) with E = 256 (or
+// 448); every block is encoded twice, its amax mapped to 6 (the NVFP4 rule)
+// and to 4, and keeps the candidate whose dequantised values have the
+// smaller sum of squared errors -- fl(fl(x - y)^2) added left to right in
+// binary32, ties keeping 6.  The output is plain NVFP4 (nvfp4_dequant reads
+// it).  The error sum is one chain over the block, so a thread owns whole
+// 16-element blocks (two 16-byte chunks); neighbouring threads take
+// neighbouring blocks, walking the siblings in the reverse order of the
+// amax pass so that the most recently read data, still in L2, goes first.
+struct FourSixArgs {
+    Sib s[kMaxSib];
+    int n;
+    const uint32_t* amax_bits;  // [B] or null
+    const float* amax_in;       // [B] or null (takes precedence)
+    float* gs_out;              // [B] or null
+    float* amax_out;            // [B] or null
+    float six_e;                // 6 E: 2688 or 1536
+};
+
+// The BF16 pairs of a chunk widened to binary32 pairs (element 0 first).
+__device__ __forceinline__ void widen8(uint4 v, uint64_t (&w)[4]) {
+    const uint32_t a[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = f32x2_bits(a[i] << 16, a[i] & 0xffff0000u);
+}
+
+// err + sum of fl(fl(x_j - y_j)^2) over the 8 elements of a chunk, one
+// rounding per operation, element 0 first.  fl(x - y) is taken as
+// fma(y, -1, x): the product is exact, so the one rounding is the
+// difference's.
+__device__ __forceinline__ float sse8(const uint64_t (&x)[4], uint4 y, float err) {
+    uint64_t yw[4];
+    widen8(y, yw);
+    const uint64_t m1 = f32x2(-1.0f, -1.0f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint64_t d = fma_f32x2(yw[i], m1, x[i]);
+        const float2 sq = f32x2_split(mul_f32x2(d, d));
+        err = __fadd_rn(err, sq.x);
+        err = __fadd_rn(err, sq.y);
+    }
+    return err;
+}
+
+// One candidate of a block: the block scale code for the amax divided by
+// t_gs = fl(t gs), the codes of its two chunks, and the error of their
+// dequantised values.
+__device__ __forceinline__ float four_six_candidate(uint4 lo, uint4 hi, const uint64_t (&xl)[4],
+                                                    const uint64_t (&xh)[4], float amax_b, float t_gs, float rt,
+                                                    bool fast_t, const ScaleTable& tab, uint64_t gs2,
+                                                    uint32_t& sb, uint32_t& c0, uint32_t& c1, uint4& y0,
+                                                    uint4& y1) {
+    const float ratio = fast_t ? div_fast(amax_b, t_gs, rt) : div_slow(amax_b, t_gs);
+    sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
+    const float4 e = tab.e[sb];
+    c0 = codes_half(lo, e.x, e.y);
+    c1 = codes_half(hi, e.x, e.y);
+    const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
+    y0 = dequant_half_h(c0, sb2, gs2);
+    y1 = dequant_half_h(c1, sb2, gs2);
+    return sse8(xh, y1, sse8(xl, y0, 0.0f));
+}
+
+template <bool kFake>
+__global__ void __launch_bounds__(kThreads) nvfp4_4over6_kernel(const FourSixArgs a) {
+    __shared__ ScaleTable tab;
+    const uint32_t b = blockIdx.y;
+    const float A = a.amax_in ? a.amax_in[b] : __uint_as_float(a.amax_bits[b]);
+    const float gs = __fdiv_rn(A, a.six_e);
+    const float g6 = __fmul_rn(6.0f, gs), g4 = __fmul_rn(4.0f, gs);
+    const float r6 = __frcp_rn(g6), r4 = __frcp_rn(g4);
+    const bool fast6 = div_fast_ok(g6), fast4 = div_fast_ok(g4);
+    const uint64_t gs2 = f32x2(gs, gs);
+    fill_scale_table(tab, gs);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (a.gs_out) a.gs_out[b] = gs;
+        if (a.amax_out) a.amax_out[b] = A;
+    }
+    __syncthreads();
+    const uint32_t gtid = blockIdx.x * blockDim.x + threadIdx.x;
+    const uint32_t nthreads = gridDim.x * blockDim.x;
+    for (int i = a.n - 1; i >= 0; --i) {
+        const Sib& S = a.s[i];
+        const char* xb = S.x + (int64_t)b * S.x_bs;
+        char* ob = S.out + (int64_t)b * S.o_bs;
+        uint8_t* sbb = kFake ? nullptr : S.sb + (int64_t)b * (S.chunks >> 1);
+        const uint32_t nblk = S.chunks >> 1;
+        for (uint32_t j = gtid; j < nblk; j += nthreads) {
+            const uint32_t c = 2u * (nblk - 1u - j);   // the block's first chunk; c + 1 is in the same row
+            int64_t xo, oo;
+            if (S.dense_x && S.dense_o) {
+                xo = (int64_t)c * 16;
+                oo = (int64_t)c * (kFake ? 16 : 4);
+            } else {
+                const uint32_t r = fdiv(c, S.cpr);
+                const uint32_t k = c - r * S.cpr.d;
+                xo = S.dense_x ? (int64_t)c * 16 : (int64_t)r * S.x_rs + (int64_t)k * 16;
+                oo = S.dense_o ? (int64_t)c * (kFake ? 16 : 4) : (int64_t)r * S.o_rs + (int64_t)k * (kFake ? 16 : 4);
+            }
+            const uint4 lo = ld_stream_v4(xb + xo), hi = ld_stream_v4(xb + xo + 16);
+            const uint32_t mw = hmax_abs(amax_word8(lo), amax_word8(hi)) & 0x7fff7fffu;
+            const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
+            uint64_t xl[4], xh[4];
+            widen8(lo, xl);
+            widen8(hi, xh);
+            uint32_t sb6, a0, a1, sb4, b0, b1;
+            uint4 ya0, ya1, yb0, yb1;
+            const float e6 = four_six_candidate(lo, hi, xl, xh, amax_b, g6, r6, fast6, tab, gs2, sb6, a0, a1,
+                                                ya0, ya1);
+            const float e4 = four_six_candidate(lo, hi, xl, xh, amax_b, g4, r4, fast4, tab, gs2, sb4, b0, b1,
+                                                yb0, yb1);
+            const bool four = e4 < e6;
+            if (kFake) {
+                st_v4(ob + oo, four ? yb0 : ya0);
+                st_v4(ob + oo + 16, four ? yb1 : ya1);
+            } else {
+                st_v2(ob + oo, make_uint2(four ? b0 : a0, four ? b1 : a1));   // 8-byte aligned: c even
+                sbb[c >> 1] = (uint8_t)(four ? sb4 : sb6);
+            }
+        }
+    }
+}
+
 // Dequantise: a grouped walk over 16-element blocks like MXFP8's.  Per
 // block: 8 packed bytes in, 32 bytes of BF16 out (one 256-bit store when the
 // BF16 rows are 32-byte aligned); the block scale and the batch index's
@@ -1007,6 +1132,44 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
     } else {
         nvfp4_encode_kernel<false, false><<<grid, kThreads, 0, s>>>(a);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_4over6(const View* x, int n, const View* out, uint8_t* const* sb, bool fake,
+                               const uint32_t* amax_bits, const float* amax_in, float* gs_out, float* amax_out,
+                               int e4m3_max, cudaStream_t s) {
+    const int64_t B = x[0].batch;
+    FourSixArgs a{};
+    a.n = n;
+    a.amax_bits = amax_bits;
+    a.amax_in = amax_in;
+    a.gs_out = gs_out;
+    a.amax_out = amax_out;
+    a.six_e = (float)(6 * e4m3_max);
+    int64_t max_blocks = 0;
+    for (int i = 0; i < n; ++i) {
+        Sib& S = a.s[i];
+        S.x = x[i].ptr;
+        S.x_bs = x[i].bstride;
+        S.x_rs = x[i].rstride;
+        S.out = out[i].ptr;
+        S.o_bs = out[i].bstride;
+        S.o_rs = out[i].rstride;
+        S.sb = fake ? nullptr : sb[i];
+        S.chunks = (uint32_t)(x[i].rows * (x[i].cols / 8));
+        S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x[i].cols / 8));
+        set_source(S, x[i], nullptr);
+        S.dense_o = dense_rows(out[i], fake ? out[i].cols * 2 : out[i].cols / 2);
+        max_blocks = std::max<int64_t>(max_blocks, S.chunks / 2);
+    }
+    const int64_t total_ctas = (max_blocks + kThreads - 1) / kThreads;
+    const int64_t budget = (int64_t)sm_count(current_device()) * 8;
+    int gx = (int)std::max<int64_t>(1, std::min<int64_t>(total_ctas, (budget + B - 1) / B));
+    dim3 grid(gx, (unsigned)B);
+    if (fake)
+        nvfp4_4over6_kernel<true><<<grid, kThreads, 0, s>>>(a);
+    else
+        nvfp4_4over6_kernel<false><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -633,6 +633,76 @@ pwq_status nvfp4_fake_quant_grouped(int n_groups, const int* group_sizes, const 
                   true, stream);
 }
 
+// ------------------------------------------------------------------ NVFP4 4over6
+
+namespace {
+
+size_t four_six_ws_bytes(int64_t B) { return (size_t)((std::max<int64_t>(1, B) * 4 + 255) / 256 * 256); }
+
+// Shared body of nvfp4_4over6_quant / nvfp4_4over6_fake_quant: the checks of
+// the NVFP4 calls, then the group amax (unless given) and the 4over6 encode.
+pwq_status four_six_run(const pwq_tensor* x, int n, const pwq_tensor* out, uint8_t* const* sb, float* gs_out,
+                        const float* amax_in, float* amax_out, int e4m3_max, void* ws, size_t ws_bytes, bool fake,
+                        pwq_stream_t stream) {
+    if (e4m3_max != 256 && e4m3_max != 448) return fail(PWQ_ERR_ARG, "e4m3_max must be 256 or 448");
+    if (!x || !out) return fail(PWQ_ERR_NULL, "tensors");
+    GroupCheck G;
+    std::vector<Extent> ins, outs;
+    std::vector<std::pair<Extent, Extent>> aliases;
+    pwq_status st = check_nv_group(x, out, fake ? nullptr : sb, n, fake, &G, ins, outs, aliases);
+    if (st != PWQ_OK) return st;
+    const int64_t B = x[0].batch;
+    if (G.all_empty || B == 0) return PWQ_OK;
+    if (!fake) {
+        if (!gs_out) return fail(PWQ_ERR_NULL, "global_scale");
+        if ((uintptr_t)gs_out % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
+        outs.push_back(extent_of(gs_out, (size_t)B * 4));
+    }
+    if (amax_out) {
+        if ((uintptr_t)amax_out % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_out");
+        outs.push_back(extent_of(amax_out, (size_t)B * 4));
+    }
+    if (amax_in) {
+        if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
+        ins.push_back(extent_of(amax_in, (size_t)B * 4));
+    } else {
+        if (!ws || (uintptr_t)ws % 4 != 0 || ws_bytes < four_six_ws_bytes(B))
+            return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
+        outs.push_back(extent_of(ws, four_six_ws_bytes(B)));
+    }
+    if ((st = check_nv_overlaps(ins, outs, aliases)) != PWQ_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t* amax_bits = nullptr;
+    if (!amax_in) {
+        amax_bits = static_cast<uint32_t*>(ws);
+        cudaError_t e = pwq::launch_nvfp4_amax(G.x, n, amax_bits, s);   // clears the words first
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return from_cuda(pwq::launch_nvfp4_4over6(G.x, n, G.out, fake ? nullptr : G.sb, fake, amax_bits, amax_in,
+                                              gs_out, amax_out, e4m3_max, s));
+}
+
+}  // namespace
+
+size_t nvfp4_4over6_workspace_size(int n_siblings, const pwq_tensor* x) {
+    if (!x || n_siblings < 1 || n_siblings > PWQ_MAX_SIBLINGS || x[0].batch < 0) return 0;
+    return four_six_ws_bytes(x[0].batch);
+}
+
+pwq_status nvfp4_4over6_quant(const pwq_tensor* x, int n_siblings, const pwq_tensor* q_packed, uint8_t* const* sb,
+                              float* global_scale, const float* amax_in, int e4m3_max, void* workspace,
+                              size_t workspace_bytes, pwq_stream_t stream) {
+    return four_six_run(x, n_siblings, q_packed, sb, global_scale, amax_in, nullptr, e4m3_max, workspace,
+                        workspace_bytes, false, stream);
+}
+
+pwq_status nvfp4_4over6_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_siblings, const float* amax_in,
+                                   float* amax_out, int e4m3_max, void* workspace, size_t workspace_bytes,
+                                   pwq_stream_t stream) {
+    return four_six_run(x, n_siblings, y, nullptr, nullptr, amax_in, amax_out, e4m3_max, workspace,
+                        workspace_bytes, true, stream);
+}
+
 // ------------------------------------------------------------------ no-allocation variant
 
 // nvfp4_fake_quant with the group-amax scratch in a file-scope device array
@@ -993,7 +1063,7 @@ pwq_status pwq_selftest_flow_timeout(const pwq_tensor* x, const pwq_tensor* y, u
 
 pwq_status pwq_selftest_division(int which, unsigned long long* counts, pwq_stream_t stream) {
     if (!counts) return fail(PWQ_ERR_NULL, "counts");
-    if (which < 0 || which > 5) return fail(PWQ_ERR_ARG, "which");
+    if (which < 0 || which > 9) return fail(PWQ_ERR_ARG, "which");
     return from_cuda(pwq::launch_selftest_division(which, counts, (cudaStream_t)stream));
 }
 

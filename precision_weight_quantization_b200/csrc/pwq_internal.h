@@ -106,6 +106,13 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
                                 float* gs_out, float* amax_out, cudaStream_t s,
                                 const float* const* ts = nullptr);
 
+// NVFP4 "4over6" encode of one group set (the amax from launch_nvfp4_amax's
+// words or from amax_in): every block keeps the candidate, amax mapped to 6
+// or to 4, with the smaller squared error; gs = fl(A / (6 e4m3_max)).
+cudaError_t launch_nvfp4_4over6(const View* x, int n, const View* out, uint8_t* const* sb, bool fake,
+                               const uint32_t* amax_bits, const float* amax_in, float* gs_out, float* amax_out,
+                               int e4m3_max, cudaStream_t s);
+
 // FP8 block-wise codes + tile scales re-quantised (dequantise, quantise) into
 // FP8 block-wise (new FP32 tile scales) or MXFP8 (UE8M0 bytes), a list of
 // tensors per call; out may be in exactly, scale_out may be scale_in (FP8).

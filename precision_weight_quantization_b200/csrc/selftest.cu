@@ -4,8 +4,9 @@
 // correctly rounded reciprocal per tile/block and an FMA residual correction
 // (pwq_device.cuh).  The numerators are BF16 values and the divisors come
 // from small finite sets (FP8 block-wise: fl(a / 448); NVFP4:
-// fl(dec(sb) * fl(a / 2688)) and fl(6 * fl(a / 2688)), a a positive BF16,
-// sb a non-zero E4M3 code), so
+// fl(dec(sb) * fl(a / 2688)) and fl(6 * fl(a / 2688)); the 4over6 variant
+// adds fl(a / 1536) for the global scale and 4 for the block-scale
+// multiplier; a a positive BF16, sb a non-zero E4M3 code), so
 // every (numerator, divisor) pair can be enumerated and compared with CUDA's
 // IEEE division __fdiv_rn in well under a second.
 //
@@ -26,30 +27,32 @@ __device__ __forceinline__ bool bf16_is_finite(uint32_t b) { return ((b >> 7) & 
 
 // One divisor per CTA; every finite BF16 numerator the format can pair with
 // it:
-//   kWhich 0  FP8 block-wise code divisor s = fl(a / 448), |x| <= a (x is in
-//             the tile whose amax is a);
-//   kWhich 1  NVFP4 code divisor d = fl(dec(sb) * fl(a / 2688)), |x| <= 16 d
-//             (x / d stays below 6 / (1 - 2^-4) for an E4M3-normal block
-//             scale and below 9.1 for a subnormal one);
-//   kWhich 2  NVFP4 block-scale divisor fl(6 * fl(a / 2688)), |x| <= a (the
-//             block amax never exceeds the group amax a).
-// The kernels' path (reciprocal or IEEE, chosen by the divisor) is compared
-// with __fdiv_rn: codes for every pair, binary32 quotients where |x| >=
-// 2^-100 and the IEEE quotient is normal.
-template <int kWhich>
+//   kKind 0  FP8 block-wise code divisor s = fl(a / 448), |x| <= a (x is in
+//            the tile whose amax is a);
+//   kKind 1  NVFP4 code divisor d = fl(dec(sb) * fl(a / kDen)), |x| <= 16 d
+//            (x / d stays below 6 / (1 - 2^-4) for an E4M3-normal block
+//            scale and below 9.1 for a subnormal one; the 4over6 candidate
+//            of 4 stays lower);
+//   kKind 2  NVFP4 block-scale divisor fl(kMul * fl(a / kDen)), |x| <= a
+//            (the block amax never exceeds the group amax a).
+// kDen = 6 E: 2688 for NVFP4, 1536 for 4over6 with E = 256; kMul = 6, or 4
+// for the 4over6 candidate.  The kernels' path (reciprocal or IEEE, chosen
+// by the divisor) is compared with __fdiv_rn: codes for every pair, binary32
+// quotients where |x| >= 2^-100 and the IEEE quotient is normal.
+template <int kKind, int kDen = 2688, int kMul = 6>
 __global__ void __launch_bounds__(kThreads) selftest_division_kernel(unsigned long long* counts) {
     const uint32_t a = blockIdx.x + 1u;                // positive finite BF16 0x0001..0x7f7f
     const float av = __uint_as_float(a << 16);
     float d, xmax;
-    if (kWhich == 0) {
+    if (kKind == 0) {
         d = __fdiv_rn(av, 448.0f);
         xmax = av;
-    } else if (kWhich == 1) {
+    } else if (kKind == 1) {
         const uint32_t sb = blockIdx.y + 1u;           // E4M3 0x01..0x7e
-        d = __fmul_rn(e4m3_decode(sb), __fdiv_rn(av, 2688.0f));
+        d = __fmul_rn(e4m3_decode(sb), __fdiv_rn(av, (float)kDen));
         xmax = __fmul_rn(16.0f, d);
     } else {
-        d = __fmul_rn(6.0f, __fdiv_rn(av, 2688.0f));
+        d = __fmul_rn((float)kMul, __fdiv_rn(av, (float)kDen));
         xmax = av;
     }
     const float r = __frcp_rn(d);
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(kThreads) selftest_division_kernel(unsigned lo
     for (uint32_t wi = threadIdx.x; wi < 32768u; wi += kThreads) {
         const uint32_t w = (2u * wi) | ((2u * wi + 1u) << 16);
         float2 qp;
-        if (kWhich == 2) {
+        if (kKind == 2) {
             qp.x = fast ? quotient<true>(bf16_lo(w), d, r) : quotient<false>(bf16_lo(w), d, r);
             qp.y = fast ? quotient<true>(bf16_hi(w), d, r) : quotient<false>(bf16_hi(w), d, r);
         } else {
@@ -76,7 +79,7 @@ __global__ void __launch_bounds__(kThreads) selftest_division_kernel(unsigned lo
             const float qr = (d == 0.0f) ? __uint_as_float((xb << 16) & 0x80000000u) : __fdiv_rn(x, d);
             ++n;
             slow += !fast;
-            if (kWhich == 1)
+            if (kKind == 1)
                 code_bad += (e2m1x2(qf, 0.0f) & 0xfu) != (e2m1x2(qr, 0.0f) & 0xfu);
             else
                 code_bad += (e4m3x2(qf, 0.0f) & 0xffu) != (e4m3x2(qr, 0.0f) & 0xffu);
@@ -202,8 +205,16 @@ cudaError_t launch_selftest_division(int which, unsigned long long* counts, cuda
         selftest_tile_scale_kernel<<<dim3(64), kThreads, 0, s>>>(counts);
     else if (which == 4)
         selftest_absmax_kernel<<<dim3(0x10000), kThreads, 0, s>>>(counts);
-    else
+    else if (which == 5)
         selftest_fp4_dequant_kernel<<<dim3(0x7f80), kThreads, 0, s>>>(counts);
+    else if (which == 6)
+        selftest_division_kernel<1, 1536><<<dim3(0x7f7f, 0x7e), kThreads, 0, s>>>(counts);
+    else if (which == 7)
+        selftest_division_kernel<2, 1536, 6><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
+    else if (which == 8)
+        selftest_division_kernel<2, 1536, 4><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
+    else
+        selftest_division_kernel<2, 2688, 4><<<dim3(0x7f7f), kThreads, 0, s>>>(counts);
     return cudaGetLastError();
 }
 

@@ -298,3 +298,51 @@ def test_scale_layout_validation_without_gpu():
     q24 = (L.PwqTensor * 1)(T(L, base + (1 << 30), 1, 4, 48, 4 * 48, 48))
     sc = (ctypes.c_void_p * 1)(base + (2 << 30))
     assert lib.mxfp8_quant_grouped_mma(1, x24, q24, sc, None) == L.PWQ_ERR_SHAPE
+
+
+def test_4over6_validation_without_gpu():
+    """nvfp4_4over6_quant / _fake_quant: e4m3_max, siblings, workspace and
+    overlap rules, all decided before any CUDA call."""
+    L = _lib()
+    lib = L.lib
+    base = 1 << 40
+    xs = (L.PwqTensor * 2)(T(L, base, 3, 64, 256, 64 * 256, 256),
+                           T(L, base + (1 << 24), 3, 32, 256, 32 * 256, 256))
+    qs = (L.PwqTensor * 2)(T(L, base + (1 << 30), 3, 64, 256, 64 * 128, 128),
+                           T(L, base + (1 << 30) + (1 << 24), 3, 32, 256, 32 * 128, 128))
+    sb = (ctypes.c_void_p * 2)(base + (2 << 30), base + (2 << 30) + (1 << 24))
+    gs = base + (3 << 30)
+    ws = base + (4 << 30)
+    assert lib.nvfp4_4over6_workspace_size(2, xs) == 256
+    big = T(L, base, 100, 16, 16, 256, 16)
+    assert lib.nvfp4_4over6_workspace_size(1, ctypes.byref(big)) == 512
+    assert lib.nvfp4_4over6_workspace_size(0, xs) == 0
+    for E in (0, 255, 257, 447, 449, 1000):
+        assert lib.nvfp4_4over6_quant(xs, 2, qs, sb, gs, None, E, ws, 256, None) == L.PWQ_ERR_ARG
+        assert lib.nvfp4_4over6_fake_quant(xs, xs, 2, None, None, E, ws, 256, None) == L.PWQ_ERR_ARG
+    assert "e4m3_max" in lib.pwq_last_error_detail().decode()
+    assert lib.nvfp4_4over6_quant(xs, 0, qs, sb, gs, None, 256, ws, 256, None) == L.PWQ_ERR_ARG
+    assert lib.nvfp4_4over6_quant(xs, 9, qs, sb, gs, None, 256, ws, 256, None) == L.PWQ_ERR_ARG
+    # workspace: required without amax_in, at least 4 bytes per batch index
+    assert lib.nvfp4_4over6_quant(xs, 2, qs, sb, gs, None, 256, None, 0, None) == L.PWQ_ERR_WORKSPACE
+    assert lib.nvfp4_4over6_quant(xs, 2, qs, sb, gs, None, 256, ws, 8, None) == L.PWQ_ERR_WORKSPACE
+    assert lib.nvfp4_4over6_quant(xs, 2, qs, sb, gs, None, 256, ws + 2, 256, None) == L.PWQ_ERR_WORKSPACE
+    # null global scale, misaligned amax_in
+    assert lib.nvfp4_4over6_quant(xs, 2, qs, sb, None, None, 256, ws, 256, None) == L.PWQ_ERR_NULL
+    assert lib.nvfp4_4over6_quant(xs, 2, qs, sb, gs, gs + 66, 448, None, 0, None) == L.PWQ_ERR_ALIGN
+    # overlaps: block scales over an input, workspace over an output, y over the other input
+    sbo = (ctypes.c_void_p * 2)(base + 64, base + (2 << 30) + (1 << 24))
+    assert lib.nvfp4_4over6_quant(xs, 2, qs, sbo, gs, None, 256, ws, 256, None) == L.PWQ_ERR_OVERLAP
+    assert lib.nvfp4_4over6_quant(xs, 2, qs, sb, gs, None, 256, gs, 256, None) == L.PWQ_ERR_OVERLAP
+    xe = (L.PwqTensor * 2)(T(L, base, 1, 64, 256, 64 * 256, 256), T(L, base + (1 << 24), 1, 64, 256, 64 * 256, 256))
+    ys = (L.PwqTensor * 2)(xe[1], xe[0])
+    assert lib.nvfp4_4over6_fake_quant(xe, ys, 2, None, None, 256, ws, 256, None) == L.PWQ_ERR_OVERLAP
+    # N % 16 and shape mismatch
+    x24 = T(L, base, 1, 4, 24, 4 * 32, 32)
+    y24 = T(L, base + (1 << 30), 1, 4, 24, 4 * 32, 32)
+    assert lib.nvfp4_4over6_fake_quant(ctypes.byref(x24), ctypes.byref(y24), 1, None, None, 256, ws, 256,
+                                       None) == L.PWQ_ERR_SHAPE
+    # empty tensors: a no-op that succeeds without a CUDA call
+    xz = T(L, None, 1, 0, 256, 0, 256)
+    assert lib.nvfp4_4over6_fake_quant(ctypes.byref(xz), ctypes.byref(xz), 1, None, None, 256, None, 0,
+                                       None) == L.PWQ_OK
