@@ -306,6 +306,26 @@ __device__ __forceinline__ float sse8(const uint64_t (&x)[4], uint4 y, float err
     return err;
 }
 
+// E2M1 codes of 8 values widened to binary32 pairs, divided by d on the
+// reciprocal path (nr2 = {-r, -r}, r = RN(1/d)).  The quotient is formed
+// negated -- q0 = x (-r), e = q0 d + x, q = e (-r) + q0, one rounding each
+// -- which is exactly the negation of div_fast's quotient (every step is
+// the same operation with all signs flipped, and rounding to nearest is
+// symmetric in sign), so flipping the sign bit of each code gives the codes
+// of the quotient itself, signed zeros included.
+__device__ __forceinline__ uint32_t codes_neg8(const uint64_t (&x)[4], uint64_t d2, uint64_t nr2) {
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint64_t q0 = mul_f32x2(x[i], nr2);
+        const uint64_t e = fma_f32x2(q0, d2, x[i]);
+        const float2 qn = f32x2_split(fma_f32x2(e, nr2, q0));
+        q[2 * i] = qn.x;
+        q[2 * i + 1] = qn.y;
+    }
+    return e2m1x8(q) ^ 0x88888888u;
+}
+
 // One candidate of a block: the block scale code for the amax divided by
 // t_gs = fl(t gs), the codes of its two chunks, and the error of their
 // dequantised values.
@@ -317,16 +337,24 @@ __device__ __forceinline__ float four_six_candidate(uint4 lo, uint4 hi, const ui
     const float ratio = fast_t ? div_fast(amax_b, t_gs, rt) : div_slow(amax_b, t_gs);
     sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
     const float4 e = tab.e[sb];
-    c0 = codes_half(lo, e.x, e.y);
-    c1 = codes_half(hi, e.x, e.y);
+    if (e.y != 0.0f) {
+        const uint64_t d2 = f32x2(e.x, e.x), nr2 = f32x2(-e.y, -e.y);
+        c0 = codes_neg8(xl, d2, nr2);
+        c1 = codes_neg8(xh, d2, nr2);
+    } else {
+        c0 = codes_half(lo, e.x, e.y);
+        c1 = codes_half(hi, e.x, e.y);
+    }
     const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
     y0 = dequant_half_h(c0, sb2, gs2);
     y1 = dequant_half_h(c1, sb2, gs2);
     return sse8(xh, y1, sse8(xl, y0, 0.0f));
 }
 
+constexpr int kFourSixCtasPerSm = 3;
+
 template <bool kFake>
-__global__ void __launch_bounds__(kThreads) nvfp4_4over6_kernel(const FourSixArgs a) {
+__global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kernel(const FourSixArgs a) {
     __shared__ ScaleTable tab;
     const uint32_t b = blockIdx.y;
     const float A = a.amax_in ? a.amax_in[b] : __uint_as_float(a.amax_bits[b]);
@@ -349,9 +377,10 @@ __global__ void __launch_bounds__(kThreads) nvfp4_4over6_kernel(const FourSixArg
         char* ob = S.out + (int64_t)b * S.o_bs;
         uint8_t* sbb = kFake ? nullptr : S.sb + (int64_t)b * (S.chunks >> 1);
         const uint32_t nblk = S.chunks >> 1;
-        for (uint32_t j = gtid; j < nblk; j += nthreads) {
-            const uint32_t c = 2u * (nblk - 1u - j);   // the block's first chunk; c + 1 is in the same row
-            int64_t xo, oo;
+        // block j: its first chunk c (c + 1 is in the same row) and the byte
+        // offsets of its input and output
+        auto offsets = [&](uint32_t j, uint32_t& c, int64_t& xo, int64_t& oo) {
+            c = 2u * (nblk - 1u - j);
             if (S.dense_x && S.dense_o) {
                 xo = (int64_t)c * 16;
                 oo = (int64_t)c * (kFake ? 16 : 4);
@@ -361,7 +390,25 @@ __global__ void __launch_bounds__(kThreads) nvfp4_4over6_kernel(const FourSixArg
                 xo = S.dense_x ? (int64_t)c * 16 : (int64_t)r * S.x_rs + (int64_t)k * 16;
                 oo = S.dense_o ? (int64_t)c * (kFake ? 16 : 4) : (int64_t)r * S.o_rs + (int64_t)k * (kFake ? 16 : 4);
             }
-            const uint4 lo = ld_stream_v4(xb + xo), hi = ld_stream_v4(xb + xo + 16);
+        };
+        uint32_t c = 0u;
+        int64_t xo = 0, oo = 0;
+        uint4 nlo = make_uint4(0u, 0u, 0u, 0u), nhi = nlo;
+        if (gtid < nblk) {
+            offsets(gtid, c, xo, oo);
+            nlo = ld_stream_v4(xb + xo);
+            nhi = ld_stream_v4(xb + xo + 16);
+        }
+        for (uint32_t j = gtid; j < nblk; j += nthreads) {
+            // this block's data was loaded one step ahead; start the next one's
+            const uint4 lo = nlo, hi = nhi;
+            const uint32_t cc = c;
+            const int64_t ooc = oo;
+            if (j + nthreads < nblk) {
+                offsets(j + nthreads, c, xo, oo);
+                nlo = ld_stream_v4(xb + xo);
+                nhi = ld_stream_v4(xb + xo + 16);
+            }
             const uint32_t mw = hmax_abs(amax_word8(lo), amax_word8(hi)) & 0x7fff7fffu;
             const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
             uint64_t xl[4], xh[4];
@@ -375,11 +422,11 @@ __global__ void __launch_bounds__(kThreads) nvfp4_4over6_kernel(const FourSixArg
                                                 yb0, yb1);
             const bool four = e4 < e6;
             if (kFake) {
-                st_v4(ob + oo, four ? yb0 : ya0);
-                st_v4(ob + oo + 16, four ? yb1 : ya1);
+                st_v4(ob + ooc, four ? yb0 : ya0);
+                st_v4(ob + ooc + 16, four ? yb1 : ya1);
             } else {
-                st_v2(ob + oo, make_uint2(four ? b0 : a0, four ? b1 : a1));   // 8-byte aligned: c even
-                sbb[c >> 1] = (uint8_t)(four ? sb4 : sb6);
+                st_v2(ob + ooc, make_uint2(four ? b0 : a0, four ? b1 : a1));   // 8-byte aligned: cc even
+                sbb[cc >> 1] = (uint8_t)(four ? sb4 : sb6);
             }
         }
     }
@@ -1162,9 +1209,10 @@ cudaError_t launch_nvfp4_4over6(const View* x, int n, const View* out, uint8_t* 
         S.dense_o = dense_rows(out[i], fake ? out[i].cols * 2 : out[i].cols / 2);
         max_blocks = std::max<int64_t>(max_blocks, S.chunks / 2);
     }
+    // every CTA resident at once, spread over the batch indices
     const int64_t total_ctas = (max_blocks + kThreads - 1) / kThreads;
-    const int64_t budget = (int64_t)sm_count(current_device()) * 8;
-    int gx = (int)std::max<int64_t>(1, std::min<int64_t>(total_ctas, (budget + B - 1) / B));
+    const int64_t budget = (int64_t)sm_count(current_device()) * kFourSixCtasPerSm;
+    int gx = (int)std::max<int64_t>(1, std::min<int64_t>(total_ctas, budget / B));
     dim3 grid(gx, (unsigned)B);
     if (fake)
         nvfp4_4over6_kernel<true><<<grid, kThreads, 0, s>>>(a);
