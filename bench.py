@@ -687,31 +687,31 @@ def next_calls(op, layers, buf, P, torch, per_call=1):
     return calls
 
 
-# NVFP4 "4over6" (E4M3 maximum 256) of the BF16 sweep, one call per sibling
-# group: the group amax pass and the encode pass that evaluates both block
-# candidates; algorithmic bytes as for NVFP4 (two reads of the input)
+# NVFP4 "4over6" (E4M3 maximum 256) of the BF16 sweep, one grouped call per
+# `per_call` layers (their sibling groups): the group amax launch and the
+# encode launch that evaluates both block candidates; algorithmic bytes as
+# for NVFP4 (two reads of the input)
 FOUR_SIX_BYTES_PER_ELEM = {"nvfp4_4over6_quant": 2 + 2 + 0.5 + 1 / 16, "nvfp4_4over6_fake_quant": 2 + 2 + 2}
 FOUR_SIX_ONE_PASS_BYTES_PER_ELEM = {"nvfp4_4over6_quant": 2 + 0.5 + 1 / 16, "nvfp4_4over6_fake_quant": 2 + 2}
 
 
-def four_six_calls(op, layers, P, torch):
-    """One call per sibling group of every layer, each writing its own outputs."""
+def four_six_calls(op, layers, P, torch, per_call=1):
+    """One grouped call per `per_call` layers, every layer writing its own outputs."""
     import workloads as W
     calls = []
-    for lay in layers:
-        for grp in W.QWEN3_4B_GROUPS:
-            xs = [lay[n] for n in grp]
-            dev = xs[0].device
-            ws = torch.empty(256, dtype=torch.uint8, device=dev)
-            if op == "nvfp4_4over6_quant":
-                pk = [torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for x in xs]
-                sb = [torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev) for x in xs]
-                gs = torch.empty(1, dtype=torch.float32, device=dev)
-                calls.append(lambda xs=xs, pk=pk, sb=sb, gs=gs: P.nvfp4_4over6_quant(xs, 256, out=pk, sb=sb,
-                                                                                    global_scale=gs))
-            else:
-                ys = [torch.empty_like(x) for x in xs]
-                calls.append(lambda xs=xs, ys=ys: P.nvfp4_4over6_fake_quant(xs, 256, out=ys))
+    for i0 in range(0, len(layers), per_call):
+        groups = [[lay[n] for n in grp] for lay in layers[i0:i0 + per_call] for grp in W.QWEN3_4B_GROUPS]
+        dev = groups[0][0].device
+        if op == "nvfp4_4over6_quant":
+            pk = [[torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for x in g] for g in groups]
+            sb = [[torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev) for x in g]
+                  for g in groups]
+            gs = [torch.empty(1, dtype=torch.float32, device=dev) for _ in groups]
+            calls.append(lambda groups=groups, pk=pk, sb=sb, gs=gs:
+                         P.nvfp4_4over6_quant_grouped(groups, 256, out=pk, sb=sb, global_scale=gs))
+        else:
+            ys = [[torch.empty_like(x) for x in g] for g in groups]
+            calls.append(lambda groups=groups, ys=ys: P.nvfp4_4over6_fake_quant_grouped(groups, 256, out=ys))
     return calls
 
 
@@ -729,7 +729,7 @@ def time_next_rows(args, w, P, torch, hbm_peak, peak_kind):
     one_pass.update(FOUR_SIX_ONE_PASS_BYTES_PER_ELEM)
     for op, bpe in ops.items():
         if op in FOUR_SIX_BYTES_PER_ELEM:
-            calls = four_six_calls(op, layers, P, torch)
+            calls = four_six_calls(op, layers, P, torch, w.tensors["per_call"])
         else:
             calls = next_calls(op, layers, buf, P, torch, w.tensors["per_call"])
         g = capture(calls, torch)

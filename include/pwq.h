@@ -253,12 +253,18 @@ pwq_status nvfp4_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_sibl
  * NVFP4 (nvfp4_dequant reads it); siblings, layouts, amax_in and amax_out
  * are those of nvfp4_quant / nvfp4_fake_quant.
  *
- * Two launches: the group amax (skipped when amax_in is given) into
- * workspace of at least nvfp4_4over6_workspace_size() bytes (4-byte
- * aligned; 4 bytes per batch index, rounded up to 256), then one encode
- * launch that evaluates both candidates of every block.
+ * The grouped forms take several sibling groups with the layout rules of
+ * nvfp4_quant_grouped / nvfp4_fake_quant_grouped (the amax is always
+ * reduced on the device).
+ *
+ * Two launches per PWQ_LAUNCH_TENSORS members: the group amaxes (skipped
+ * when amax_in is given) into workspace of at least
+ * nvfp4_4over6_workspace_size() / _grouped() bytes (4-byte aligned; 4 bytes
+ * per batch index of every group, rounded up to 256; its contents on entry
+ * do not matter), then one encode launch that evaluates both candidates of
+ * every block.
  * Errors: PWQ_ERR_NULL, _ALIGN, _SHAPE, _STRIDE, _OVERLAP, _WORKSPACE,
- * _ARG (e4m3_max not 256 or 448, n_siblings), _CUDA. */
+ * _ARG (e4m3_max not 256 or 448, n_siblings / group sizes), _CUDA. */
 size_t nvfp4_4over6_workspace_size(int n_siblings, const pwq_tensor* x);
 pwq_status nvfp4_4over6_quant(const pwq_tensor* x, int n_siblings, const pwq_tensor* q_packed,
                               uint8_t* const* sb, float* global_scale, const float* amax_in, int e4m3_max,
@@ -266,6 +272,14 @@ pwq_status nvfp4_4over6_quant(const pwq_tensor* x, int n_siblings, const pwq_ten
 pwq_status nvfp4_4over6_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_siblings,
                                    const float* amax_in, float* amax_out, int e4m3_max, void* workspace,
                                    size_t workspace_bytes, pwq_stream_t stream);
+size_t nvfp4_4over6_workspace_size_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x);
+pwq_status nvfp4_4over6_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                                      const pwq_tensor* q_packed, uint8_t* const* sb,
+                                      float* const* global_scale, int e4m3_max, void* workspace,
+                                      size_t workspace_bytes, pwq_stream_t stream);
+pwq_status nvfp4_4over6_fake_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                                           const pwq_tensor* y, float* const* amax_out, int e4m3_max,
+                                           void* workspace, size_t workspace_bytes, pwq_stream_t stream);
 
 /* ===================================================================== */
 /* Grouped calls: a list of independent tensors in one launch             */

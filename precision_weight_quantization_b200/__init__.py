@@ -454,6 +454,50 @@ def nvfp4_fake_quant_grouped(groups: Sequence[Sequence[torch.Tensor]], out=None,
     return out
 
 
+def nvfp4_4over6_quant_grouped(groups: Sequence[Sequence[torch.Tensor]], e4m3_max: int = 256, out=None, sb=None,
+                               global_scale=None):
+    """NVFP4 "4over6" quantisation of several sibling groups (two launches per
+    16 members).  Returns what nvfp4_quant_grouped returns."""
+    groups, flat, sizes = _groups(groups)
+    dev = flat[0].device
+    if out is None:
+        out = [[torch.empty(x.shape[:-1] + (x.shape[-1] // 2,), dtype=torch.uint8, device=dev) for x in g]
+               for g in groups]
+    if sb is None:
+        sb = [[torch.empty(x.shape[:-1] + (x.shape[-1] // 16,), dtype=torch.float8_e4m3fn, device=dev) for x in g]
+              for g in groups]
+    if global_scale is None:
+        global_scale = [torch.empty(_batch(g[0]), dtype=torch.float32, device=dev) for g in groups]
+    ax = _desc_array(flat, "x")
+    ws_bytes = int(lib.nvfp4_4over6_workspace_size_grouped(len(groups), sizes, ax))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    check(lib.nvfp4_4over6_quant_grouped(len(groups), sizes, ax,
+                                         _desc_array([p for g in out for p in g], "out", packed=True),
+                                         _ptrs([s for g in sb for s in g]), _ptrs(global_scale), int(e4m3_max),
+                                         ws.data_ptr(), ws.numel(), _stream(flat[0])), "nvfp4_4over6_quant_grouped")
+    return out, sb, global_scale
+
+
+def nvfp4_4over6_fake_quant_grouped(groups: Sequence[Sequence[torch.Tensor]], e4m3_max: int = 256, out=None,
+                                    inplace: bool = False, amax_out=None):
+    """NVFP4 "4over6" fake-quantisation of several sibling groups.  Returns
+    the BF16 outputs per group."""
+    groups, flat, sizes = _groups(groups)
+    dev = flat[0].device
+    if out is None:
+        out = groups if inplace else [[torch.empty_like(x) for x in g] for g in groups]
+    ax = _desc_array(flat, "x")
+    ws_bytes = int(lib.nvfp4_4over6_workspace_size_grouped(len(groups), sizes, ax))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    ao = None
+    if amax_out is not None:
+        ao = (ctypes.c_void_p * len(groups))(*[a.data_ptr() if a is not None else None for a in amax_out])
+    check(lib.nvfp4_4over6_fake_quant_grouped(len(groups), sizes, ax, _desc_array([y for g in out for y in g], "out"),
+                                              ao, int(e4m3_max), ws.data_ptr(), ws.numel(), _stream(flat[0])),
+          "nvfp4_4over6_fake_quant_grouped")
+    return out
+
+
 # ---------------------------------------------------------------- block scales in the tensor-core layout
 
 def mma_scale_bytes(batch: int, rows: int, scale_cols: int) -> int:

@@ -56,6 +56,11 @@ _SIG = {
     "nvfp4_4over6_quant": (_S, [_T, ctypes.c_int, _T, ctypes.POINTER(ctypes.c_void_p), _P, _P, ctypes.c_int, _P,
                                 ctypes.c_size_t, _P]),
     "nvfp4_4over6_fake_quant": (_S, [_T, _T, ctypes.c_int, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "nvfp4_4over6_workspace_size_grouped": (ctypes.c_size_t, [ctypes.c_int, _IP, _T]),
+    "nvfp4_4over6_quant_grouped": (_S, [ctypes.c_int, _IP, _T, _T, _PP, _PP, ctypes.c_int, _P, ctypes.c_size_t,
+                                        _P]),
+    "nvfp4_4over6_fake_quant_grouped": (_S, [ctypes.c_int, _IP, _T, _T, _PP, ctypes.c_int, _P, ctypes.c_size_t,
+                                             _P]),
     "fp8_block_quant_grouped": (_S, [ctypes.c_int, _T, _T, _PP, _P]),
     "fp8_block_dequant_grouped": (_S, [ctypes.c_int, _T, _PP, _T, _P]),
     "mxfp8_quant_grouped": (_S, [ctypes.c_int, _T, _T, _PP, _P]),

@@ -267,19 +267,81 @@ __global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs
 // and to 4, and keeps the candidate whose dequantised values have the
 // smaller sum of squared errors -- fl(fl(x - y)^2) added left to right in
 // binary32, ties keeping 6.  The output is plain NVFP4 (nvfp4_dequant reads
-// it).  The error sum is one chain over the block, so a thread owns whole
-// 16-element blocks (two 16-byte chunks); neighbouring threads take
-// neighbouring blocks, walking the siblings in the reverse order of the
-// amax pass so that the most recently read data, still in L2, goes first.
-struct FourSixArgs {
-    Sib s[kMaxSib];
-    int n;
-    const uint32_t* amax_bits;  // [B] or null
-    const float* amax_in;       // [B] or null (takes precedence)
-    float* gs_out;              // [B] or null
-    float* amax_out;            // [B] or null
-    float six_e;                // 6 E: 2688 or 1536
+// it).
+//
+// Work units are 16-element blocks.  The units of a launch (up to 16
+// members in up to 16 sibling groups) form one index space: group after
+// group, batch index (instance) after batch index, member after member, row
+// after row.  Each persistent CTA takes one contiguous range of it, so a
+// 256-expert batch fills every SM as well as one large tensor does.  Two
+// launches: the amax kernel reduces each instance piece of a range to one
+// atomicMax on the instance's word; the encode kernel walks its range
+// backwards, one instance piece at a time (the scale table depends on the
+// instance's gs), so that the data its own amax pass read last -- still in
+// L2 -- comes first.  The error sum is one chain over a block, so a thread
+// owns whole blocks (two 16-byte chunks); neighbouring threads take
+// neighbouring blocks.
+struct FourSixGroup {
+    uint64_t unit0;         // first unit of the group in the launch
+    uint32_t units;         // units per instance: sum of the members' blocks
+    uint32_t inst0;         // first amax word of the group
+    uint32_t batch;         // instances
+    int m0, nm;             // members m0 .. m0 + nm - 1
+    const float* amax_in;   // [batch] or null
+    float* gs_out;          // [batch] or null
+    float* amax_out;        // [batch] or null
 };
+
+struct FourSixArgs {
+    Sib m[kMaxLaunchTensors];
+    uint32_t mblk0[kMaxLaunchTensors];   // first unit of each member inside its instance
+    FourSixGroup g[kMaxLaunchTensors];
+    int n_groups;
+    uint64_t total;                      // units of the launch
+    uint32_t* amax_bits;                 // one word per instance
+    float six_e;                         // 6 E: 2688 or 1536
+};
+
+// The CTA's contiguous range of units.
+__device__ __forceinline__ void four_six_range(const FourSixArgs& a, uint64_t& lo, uint64_t& hi) {
+    const uint64_t per = (a.total + gridDim.x - 1) / gridDim.x;
+    lo = min(a.total, (uint64_t)blockIdx.x * per);
+    hi = min(a.total, lo + per);
+}
+
+// Group, instance and the instance's first unit of unit u.
+__device__ __forceinline__ void four_six_locate(const FourSixArgs& a, uint64_t u, int& gi, uint32_t& b,
+                                                uint64_t& inst_lo) {
+    gi = 0;
+    while (gi + 1 < a.n_groups && u >= a.g[gi + 1].unit0) ++gi;
+    const FourSixGroup& G = a.g[gi];
+    b = (uint32_t)((u - G.unit0) / G.units);
+    inst_lo = G.unit0 + (uint64_t)b * G.units;
+}
+
+// Member, and the byte offsets of a block's input and output (and its
+// block-scale index), for unit r of an instance of group G.
+__device__ __forceinline__ int four_six_member(const FourSixArgs& a, const FourSixGroup& G, uint32_t r) {
+    int i = G.m0 + G.nm - 1;
+    while (r < a.mblk0[i]) --i;
+    return i;
+}
+
+template <bool kFake>
+__device__ __forceinline__ void four_six_offsets(const Sib& S, uint32_t b, uint32_t j, int64_t& xo, int64_t& oo) {
+    const uint32_t c = 2u * j;   // the block's first chunk; c + 1 is in the same row
+    if (S.dense_x && S.dense_o) {
+        xo = (int64_t)c * 16;
+        oo = (int64_t)c * (kFake ? 16 : 4);
+    } else {
+        const uint32_t r = fdiv(c, S.cpr);
+        const uint32_t k = c - r * S.cpr.d;
+        xo = S.dense_x ? (int64_t)c * 16 : (int64_t)r * S.x_rs + (int64_t)k * 16;
+        oo = S.dense_o ? (int64_t)c * (kFake ? 16 : 4) : (int64_t)r * S.o_rs + (int64_t)k * (kFake ? 16 : 4);
+    }
+    xo += (int64_t)b * S.x_bs;
+    oo += (int64_t)b * S.o_bs;
+}
 
 // The BF16 pairs of a chunk widened to binary32 pairs (element 0 first).
 __device__ __forceinline__ void widen8(uint4 v, uint64_t (&w)[4]) {
@@ -352,83 +414,126 @@ __device__ __forceinline__ float four_six_candidate(uint4 lo, uint4 hi, const ui
 }
 
 constexpr int kFourSixCtasPerSm = 3;
+constexpr int kFourSixAmaxUnroll = 4;
+
+__global__ void __launch_bounds__(kThreads) nvfp4_4over6_amax_kernel(const FourSixArgs a) {
+    __shared__ uint32_t red[kThreads / 32];
+    uint64_t lo, hi;
+    four_six_range(a, lo, hi);
+    for (uint64_t u = lo; u < hi;) {
+        int gi;
+        uint32_t b;
+        uint64_t inst_lo;
+        four_six_locate(a, u, gi, b, inst_lo);
+        const FourSixGroup& G = a.g[gi];
+        const uint64_t end = min(hi, inst_lo + G.units);   // this instance's piece of the range
+        if (!G.amax_in) {
+            uint32_t m = 0u;
+            const uint32_t r0 = (uint32_t)(u - inst_lo), r1 = (uint32_t)(end - inst_lo);
+            for (uint32_t r = r0 + threadIdx.x; r < r1; r += kThreads * kFourSixAmaxUnroll) {
+                uint4 v[2 * kFourSixAmaxUnroll];
+#pragma unroll
+                for (int k = 0; k < kFourSixAmaxUnroll; ++k) {
+                    const uint32_t rk = r + (uint32_t)k * kThreads;
+                    v[2 * k] = v[2 * k + 1] = make_uint4(0u, 0u, 0u, 0u);
+                    if (rk < r1) {
+                        const int i = four_six_member(a, G, rk);
+                        int64_t xo, oo;
+                        four_six_offsets<true>(a.m[i], b, rk - a.mblk0[i], xo, oo);
+                        v[2 * k] = ld_stream_v4(a.m[i].x + xo);
+                        v[2 * k + 1] = ld_stream_v4(a.m[i].x + xo + 16);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 2 * kFourSixAmaxUnroll; ++k) m = max(m, amax_bits8(v[k]));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if ((threadIdx.x & 31u) == 0u) red[threadIdx.x >> 5] = m;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                for (int w = 1; w < kThreads / 32; ++w) m = max(m, red[w]);
+                if (m != 0u) atomicMax(a.amax_bits + G.inst0 + b, m << 16);
+            }
+            __syncthreads();   // red is reused by the next piece
+        }
+        u = end;
+    }
+}
 
 template <bool kFake>
 __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kernel(const FourSixArgs a) {
     __shared__ ScaleTable tab;
-    const uint32_t b = blockIdx.y;
-    const float A = a.amax_in ? a.amax_in[b] : __uint_as_float(a.amax_bits[b]);
-    const float gs = __fdiv_rn(A, a.six_e);
-    const float g6 = __fmul_rn(6.0f, gs), g4 = __fmul_rn(4.0f, gs);
-    const float r6 = __frcp_rn(g6), r4 = __frcp_rn(g4);
-    const bool fast6 = div_fast_ok(g6), fast4 = div_fast_ok(g4);
-    const uint64_t gs2 = f32x2(gs, gs);
-    fill_scale_table(tab, gs);
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        if (a.gs_out) a.gs_out[b] = gs;
-        if (a.amax_out) a.amax_out[b] = A;
-    }
-    __syncthreads();
-    const uint32_t gtid = blockIdx.x * blockDim.x + threadIdx.x;
-    const uint32_t nthreads = gridDim.x * blockDim.x;
-    for (int i = a.n - 1; i >= 0; --i) {
-        const Sib& S = a.s[i];
-        const char* xb = S.x + (int64_t)b * S.x_bs;
-        char* ob = S.out + (int64_t)b * S.o_bs;
-        uint8_t* sbb = kFake ? nullptr : S.sb + (int64_t)b * (S.chunks >> 1);
-        const uint32_t nblk = S.chunks >> 1;
-        // block j: its first chunk c (c + 1 is in the same row) and the byte
-        // offsets of its input and output
-        auto offsets = [&](uint32_t j, uint32_t& c, int64_t& xo, int64_t& oo) {
-            c = 2u * (nblk - 1u - j);
-            if (S.dense_x && S.dense_o) {
-                xo = (int64_t)c * 16;
-                oo = (int64_t)c * (kFake ? 16 : 4);
-            } else {
-                const uint32_t r = fdiv(c, S.cpr);
-                const uint32_t k = c - r * S.cpr.d;
-                xo = S.dense_x ? (int64_t)c * 16 : (int64_t)r * S.x_rs + (int64_t)k * 16;
-                oo = S.dense_o ? (int64_t)c * (kFake ? 16 : 4) : (int64_t)r * S.o_rs + (int64_t)k * (kFake ? 16 : 4);
-            }
-        };
-        uint32_t c = 0u;
+    uint64_t lo, hi;
+    four_six_range(a, lo, hi);
+    for (uint64_t u = hi; u > lo;) {
+        int gi;
+        uint32_t b;
+        uint64_t inst_lo;
+        four_six_locate(a, u - 1, gi, b, inst_lo);
+        const FourSixGroup& G = a.g[gi];
+        const uint64_t start = max(lo, inst_lo);   // this instance's piece of the range: [start, u)
+        const float A = G.amax_in ? G.amax_in[b] : __uint_as_float(a.amax_bits[G.inst0 + b]);
+        const float gs = __fdiv_rn(A, a.six_e);
+        const float g6 = __fmul_rn(6.0f, gs), g4 = __fmul_rn(4.0f, gs);
+        const float r6 = __frcp_rn(g6), r4 = __frcp_rn(g4);
+        const bool fast6 = div_fast_ok(g6), fast4 = div_fast_ok(g4);
+        const uint64_t gs2 = f32x2(gs, gs);
+        __syncthreads();   // the previous piece's table reads are done
+        fill_scale_table(tab, gs);
+        if (start == inst_lo && threadIdx.x == 0) {   // the one CTA that holds the instance's first unit
+            if (G.gs_out) G.gs_out[b] = gs;
+            if (G.amax_out) G.amax_out[b] = A;
+        }
+        __syncthreads();
+        // units u - 1 - t, u - 1 - t - kThreads, ... down to start; the next
+        // one's two loads are issued before the current one is encoded
+        const uint32_t rs = (uint32_t)(start - inst_lo), re = (uint32_t)(u - inst_lo);
+        const uint32_t n = re - rs;
+        int i = 0;
         int64_t xo = 0, oo = 0;
         uint4 nlo = make_uint4(0u, 0u, 0u, 0u), nhi = nlo;
-        if (gtid < nblk) {
-            offsets(gtid, c, xo, oo);
-            nlo = ld_stream_v4(xb + xo);
-            nhi = ld_stream_v4(xb + xo + 16);
+        if (threadIdx.x < n) {
+            const uint32_t r = re - 1u - threadIdx.x;
+            i = four_six_member(a, G, r);
+            four_six_offsets<kFake>(a.m[i], b, r - a.mblk0[i], xo, oo);
+            nlo = ld_stream_v4(a.m[i].x + xo);
+            nhi = ld_stream_v4(a.m[i].x + xo + 16);
         }
-        for (uint32_t j = gtid; j < nblk; j += nthreads) {
-            // this block's data was loaded one step ahead; start the next one's
-            const uint4 lo = nlo, hi = nhi;
-            const uint32_t cc = c;
+        for (uint32_t k = threadIdx.x; k < n; k += kThreads) {
+            const uint4 lo4 = nlo, hi4 = nhi;
+            const int ic = i;
             const int64_t ooc = oo;
-            if (j + nthreads < nblk) {
-                offsets(j + nthreads, c, xo, oo);
-                nlo = ld_stream_v4(xb + xo);
-                nhi = ld_stream_v4(xb + xo + 16);
+            const uint32_t jc = re - 1u - k - a.mblk0[ic];   // block within the member
+            if (k + kThreads < n) {
+                const uint32_t r = re - 1u - k - kThreads;
+                i = four_six_member(a, G, r);
+                four_six_offsets<kFake>(a.m[i], b, r - a.mblk0[i], xo, oo);
+                nlo = ld_stream_v4(a.m[i].x + xo);
+                nhi = ld_stream_v4(a.m[i].x + xo + 16);
             }
-            const uint32_t mw = hmax_abs(amax_word8(lo), amax_word8(hi)) & 0x7fff7fffu;
+            const Sib& S = a.m[ic];
+            const uint32_t mw = hmax_abs(amax_word8(lo4), amax_word8(hi4)) & 0x7fff7fffu;
             const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
             uint64_t xl[4], xh[4];
-            widen8(lo, xl);
-            widen8(hi, xh);
+            widen8(lo4, xl);
+            widen8(hi4, xh);
             uint32_t sb6, a0, a1, sb4, b0, b1;
             uint4 ya0, ya1, yb0, yb1;
-            const float e6 = four_six_candidate(lo, hi, xl, xh, amax_b, g6, r6, fast6, tab, gs2, sb6, a0, a1,
+            const float e6 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g6, r6, fast6, tab, gs2, sb6, a0, a1,
                                                 ya0, ya1);
-            const float e4 = four_six_candidate(lo, hi, xl, xh, amax_b, g4, r4, fast4, tab, gs2, sb4, b0, b1,
+            const float e4 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g4, r4, fast4, tab, gs2, sb4, b0, b1,
                                                 yb0, yb1);
             const bool four = e4 < e6;
             if (kFake) {
-                st_v4(ob + ooc, four ? yb0 : ya0);
-                st_v4(ob + ooc + 16, four ? yb1 : ya1);
+                st_v4(S.out + ooc, four ? yb0 : ya0);
+                st_v4(S.out + ooc + 16, four ? yb1 : ya1);
             } else {
-                st_v2(ob + ooc, make_uint2(four ? b0 : a0, four ? b1 : a1));   // 8-byte aligned: cc even
-                sbb[cc >> 1] = (uint8_t)(four ? sb4 : sb6);
+                st_v2(S.out + ooc, make_uint2(four ? b0 : a0, four ? b1 : a1));   // 8-byte aligned: 2 jc even
+                S.sb[(int64_t)b * (S.chunks >> 1) + jc] = (uint8_t)(four ? sb4 : sb6);
             }
         }
+        u = start;
     }
 }
 
@@ -1182,43 +1287,91 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
     return cudaGetLastError();
 }
 
-cudaError_t launch_nvfp4_4over6(const View* x, int n, const View* out, uint8_t* const* sb, bool fake,
-                               const uint32_t* amax_bits, const float* amax_in, float* gs_out, float* amax_out,
-                               int e4m3_max, cudaStream_t s) {
-    const int64_t B = x[0].batch;
+size_t nvfp4_4over6_workspace_bytes(int64_t instances) {
+    return (size_t)((std::max<int64_t>(1, instances) * 4 + 255) / 256 * 256);
+}
+
+cudaError_t launch_nvfp4_4over6(const NvGroup* groups, int n_groups, bool fake, int e4m3_max, void* workspace,
+                               cudaStream_t s) {
+    uint32_t* words = static_cast<uint32_t*>(workspace);
+    const int grid_cap = sm_count(current_device()) * kFourSixCtasPerSm;
     FourSixArgs a{};
-    a.n = n;
-    a.amax_bits = amax_bits;
-    a.amax_in = amax_in;
-    a.gs_out = gs_out;
-    a.amax_out = amax_out;
-    a.six_e = (float)(6 * e4m3_max);
-    int64_t max_blocks = 0;
-    for (int i = 0; i < n; ++i) {
-        Sib& S = a.s[i];
-        S.x = x[i].ptr;
-        S.x_bs = x[i].bstride;
-        S.x_rs = x[i].rstride;
-        S.out = out[i].ptr;
-        S.o_bs = out[i].bstride;
-        S.o_rs = out[i].rstride;
-        S.sb = fake ? nullptr : sb[i];
-        S.chunks = (uint32_t)(x[i].rows * (x[i].cols / 8));
-        S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x[i].cols / 8));
-        set_source(S, x[i], nullptr);
-        S.dense_o = dense_rows(out[i], fake ? out[i].cols * 2 : out[i].cols / 2);
-        max_blocks = std::max<int64_t>(max_blocks, S.chunks / 2);
+    uint32_t inst = 0;             // amax words used by earlier groups of the call
+    auto flush = [&]() -> cudaError_t {
+        if (a.n_groups == 0) return cudaSuccess;
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(grid_cap, (int64_t)((a.total + kThreads - 1) / kThreads)));
+        bool reduce = false;
+        uint32_t w0 = UINT32_MAX, w1 = 0;
+        for (int g = 0; g < a.n_groups; ++g)
+            if (!a.g[g].amax_in) {
+                reduce = true;
+                w0 = std::min(w0, a.g[g].inst0);
+                w1 = std::max(w1, a.g[g].inst0 + a.g[g].batch);
+            }
+        if (reduce) {
+            cudaError_t e = cudaMemsetAsync(words + w0, 0, sizeof(uint32_t) * (w1 - w0), s);
+            if (e != cudaSuccess) return e;
+            nvfp4_4over6_amax_kernel<<<grid, kThreads, 0, s>>>(a);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if (fake)
+            nvfp4_4over6_kernel<true><<<grid, kThreads, 0, s>>>(a);
+        else
+            nvfp4_4over6_kernel<false><<<grid, kThreads, 0, s>>>(a);
+        cudaError_t e = cudaGetLastError();
+        a = FourSixArgs{};
+        return e;
+    };
+    int n_members = 0;
+    for (int gi = 0; gi < n_groups; ++gi) {
+        const NvGroup& G = groups[gi];
+        if (n_members + G.n > kMaxLaunchTensors || a.n_groups == kMaxLaunchTensors) {
+            cudaError_t e = flush();
+            if (e != cudaSuccess) return e;
+            n_members = 0;
+        }
+        if (a.n_groups == 0) {
+            a.amax_bits = words;
+            a.six_e = (float)(6 * e4m3_max);
+        }
+        FourSixGroup& F = a.g[a.n_groups];
+        F.unit0 = a.total;
+        F.inst0 = inst;
+        F.batch = (uint32_t)G.x[0].batch;
+        F.m0 = n_members;
+        F.nm = G.n;
+        F.amax_in = G.amax_in;
+        F.gs_out = G.gs_out;
+        F.amax_out = G.amax_out;
+        uint64_t units = 0;
+        for (int i = 0; i < G.n; ++i) {
+            Sib& S = a.m[n_members + i];
+            const View& x = G.x[i];
+            S.x = x.ptr;
+            S.x_bs = x.bstride;
+            S.x_rs = x.rstride;
+            S.out = G.out[i].ptr;
+            S.o_bs = G.out[i].bstride;
+            S.o_rs = G.out[i].rstride;
+            S.sb = fake ? nullptr : G.sb[i];
+            S.chunks = (uint32_t)(x.rows * (x.cols / 8));
+            S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
+            set_source(S, x, nullptr);
+            S.dense_o = dense_rows(G.out[i], fake ? G.out[i].cols * 2 : G.out[i].cols / 2);
+            a.mblk0[n_members + i] = (uint32_t)units;
+            units += S.chunks / 2;
+        }
+        if (units == 0 || units > UINT32_MAX) {
+            if (units > UINT32_MAX) return cudaErrorInvalidValue;   // more than 2^32 blocks per instance
+            continue;                                               // an empty group: nothing to launch
+        }
+        F.units = (uint32_t)units;
+        a.total += units * F.batch;
+        inst += F.batch;
+        n_members += G.n;
+        ++a.n_groups;
     }
-    // every CTA resident at once, spread over the batch indices
-    const int64_t total_ctas = (max_blocks + kThreads - 1) / kThreads;
-    const int64_t budget = (int64_t)sm_count(current_device()) * kFourSixCtasPerSm;
-    int gx = (int)std::max<int64_t>(1, std::min<int64_t>(total_ctas, budget / B));
-    dim3 grid(gx, (unsigned)B);
-    if (fake)
-        nvfp4_4over6_kernel<true><<<grid, kThreads, 0, s>>>(a);
-    else
-        nvfp4_4over6_kernel<false><<<grid, kThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return flush();
 }
 
 cudaError_t launch_nvfp4_dequant(const Job* jobs, int n, cudaStream_t s) {

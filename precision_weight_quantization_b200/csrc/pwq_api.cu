@@ -637,69 +637,118 @@ pwq_status nvfp4_fake_quant_grouped(int n_groups, const int* group_sizes, const 
 
 namespace {
 
-size_t four_six_ws_bytes(int64_t B) { return (size_t)((std::max<int64_t>(1, B) * 4 + 255) / 256 * 256); }
-
-// Shared body of nvfp4_4over6_quant / nvfp4_4over6_fake_quant: the checks of
-// the NVFP4 calls, then the group amax (unless given) and the 4over6 encode.
-pwq_status four_six_run(const pwq_tensor* x, int n, const pwq_tensor* out, uint8_t* const* sb, float* gs_out,
-                        const float* amax_in, float* amax_out, int e4m3_max, void* ws, size_t ws_bytes, bool fake,
-                        pwq_stream_t stream) {
+// Shared body of the nvfp4_4over6_* calls: the checks of the NVFP4 calls
+// (per group), then the group amaxes (unless amax_in is given) and the
+// 4over6 encode.
+pwq_status four_six_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq_tensor* out,
+                        uint8_t* const* sb, float* const* gs_out, const float* amax_in, float* const* amax_out,
+                        int e4m3_max, void* ws, size_t ws_bytes, bool fake, pwq_stream_t stream) {
     if (e4m3_max != 256 && e4m3_max != 448) return fail(PWQ_ERR_ARG, "e4m3_max must be 256 or 448");
-    if (!x || !out) return fail(PWQ_ERR_NULL, "tensors");
-    GroupCheck G;
+    if (n_groups < 1 || n_groups > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group count out of range");
+    if (!sizes || !x || !out) return fail(PWQ_ERR_NULL, "group sizes / tensors");
+    std::vector<GroupCheck> groups(n_groups);
     std::vector<Extent> ins, outs;
     std::vector<std::pair<Extent, Extent>> aliases;
-    pwq_status st = check_nv_group(x, out, fake ? nullptr : sb, n, fake, &G, ins, outs, aliases);
-    if (st != PWQ_OK) return st;
-    const int64_t B = x[0].batch;
-    if (G.all_empty || B == 0) return PWQ_OK;
-    if (!fake) {
-        if (!gs_out) return fail(PWQ_ERR_NULL, "global_scale");
-        if ((uintptr_t)gs_out % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
-        outs.push_back(extent_of(gs_out, (size_t)B * 4));
-    }
-    if (amax_out) {
-        if ((uintptr_t)amax_out % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_out");
-        outs.push_back(extent_of(amax_out, (size_t)B * 4));
+    std::vector<pwq::NvGroup> launch;
+    int m = 0;
+    int64_t instances = 0;
+    for (int g = 0; g < n_groups; ++g) {
+        const int n = sizes[g];
+        if (n < 1 || n > PWQ_MAX_SIBLINGS || m + n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group size");
+        GroupCheck& G = groups[g];
+        pwq_status st = check_nv_group(x + m, out + m, fake ? nullptr : sb + m, n, fake, &G, ins, outs, aliases);
+        if (st != PWQ_OK) return st;
+        const int64_t B = x[m].batch;
+        if (!G.all_empty && B > 0) {
+            pwq::NvGroup ng;
+            ng.x = G.x;
+            ng.out = G.out;
+            ng.sb = fake ? nullptr : G.sb;
+            ng.n = n;
+            ng.amax_in = amax_in;
+            ng.gs_out = nullptr;
+            ng.amax_out = nullptr;
+            if (!fake) {
+                if (!gs_out || !gs_out[g]) return fail(PWQ_ERR_NULL, "global_scale");
+                if ((uintptr_t)gs_out[g] % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
+                ng.gs_out = gs_out[g];
+                outs.push_back(extent_of(gs_out[g], (size_t)B * 4));
+            }
+            if (amax_out && amax_out[g]) {
+                if ((uintptr_t)amax_out[g] % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_out");
+                ng.amax_out = amax_out[g];
+                outs.push_back(extent_of(amax_out[g], (size_t)B * 4));
+            }
+            launch.push_back(ng);
+            instances += B;
+        }
+        m += n;
     }
     if (amax_in) {
+        if (n_groups != 1) return fail(PWQ_ERR_ARG, "amax_in needs a single group");
         if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
-        ins.push_back(extent_of(amax_in, (size_t)B * 4));
-    } else {
-        if (!ws || (uintptr_t)ws % 4 != 0 || ws_bytes < four_six_ws_bytes(B))
-            return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
-        outs.push_back(extent_of(ws, four_six_ws_bytes(B)));
+        ins.push_back(extent_of(amax_in, (size_t)x[0].batch * 4));
     }
-    if ((st = check_nv_overlaps(ins, outs, aliases)) != PWQ_OK) return st;
-    cudaStream_t s = (cudaStream_t)stream;
-    uint32_t* amax_bits = nullptr;
+    if (launch.empty()) return PWQ_OK;
     if (!amax_in) {
-        amax_bits = static_cast<uint32_t*>(ws);
-        cudaError_t e = pwq::launch_nvfp4_amax(G.x, n, amax_bits, s);   // clears the words first
-        if (e != cudaSuccess) return cuda_fail(e);
+        if (!ws || (uintptr_t)ws % 4 != 0 || ws_bytes < pwq::nvfp4_4over6_workspace_bytes(instances))
+            return fail(PWQ_ERR_WORKSPACE, "workspace missing, misaligned or too small");
+        outs.push_back(extent_of(ws, pwq::nvfp4_4over6_workspace_bytes(instances)));
     }
-    return from_cuda(pwq::launch_nvfp4_4over6(G.x, n, G.out, fake ? nullptr : G.sb, fake, amax_bits, amax_in,
-                                              gs_out, amax_out, e4m3_max, s));
+    pwq_status st = check_nv_overlaps(ins, outs, aliases);
+    if (st != PWQ_OK) return st;
+    return from_cuda(pwq::launch_nvfp4_4over6(launch.data(), (int)launch.size(), fake, e4m3_max, ws,
+                                              (cudaStream_t)stream));
 }
 
 }  // namespace
 
 size_t nvfp4_4over6_workspace_size(int n_siblings, const pwq_tensor* x) {
     if (!x || n_siblings < 1 || n_siblings > PWQ_MAX_SIBLINGS || x[0].batch < 0) return 0;
-    return four_six_ws_bytes(x[0].batch);
+    return pwq::nvfp4_4over6_workspace_bytes(x[0].batch);
+}
+
+size_t nvfp4_4over6_workspace_size_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x) {
+    if (!x || !group_sizes || n_groups < 1 || n_groups > PWQ_MAX_GROUPED) return 0;
+    int64_t inst = 0;
+    int m = 0;
+    for (int g = 0; g < n_groups; ++g) {
+        if (group_sizes[g] < 1 || group_sizes[g] > PWQ_MAX_SIBLINGS || m + group_sizes[g] > PWQ_MAX_GROUPED) return 0;
+        inst += std::max<int64_t>(0, x[m].batch);
+        m += group_sizes[g];
+    }
+    return pwq::nvfp4_4over6_workspace_bytes(inst);
 }
 
 pwq_status nvfp4_4over6_quant(const pwq_tensor* x, int n_siblings, const pwq_tensor* q_packed, uint8_t* const* sb,
                               float* global_scale, const float* amax_in, int e4m3_max, void* workspace,
                               size_t workspace_bytes, pwq_stream_t stream) {
-    return four_six_run(x, n_siblings, q_packed, sb, global_scale, amax_in, nullptr, e4m3_max, workspace,
-                        workspace_bytes, false, stream);
+    const int sizes[1] = {n_siblings};
+    float* gs[1] = {global_scale};
+    return four_six_run(1, sizes, x, q_packed, sb, gs, amax_in, nullptr, e4m3_max, workspace, workspace_bytes,
+                        false, stream);
 }
 
 pwq_status nvfp4_4over6_fake_quant(const pwq_tensor* x, const pwq_tensor* y, int n_siblings, const float* amax_in,
                                    float* amax_out, int e4m3_max, void* workspace, size_t workspace_bytes,
                                    pwq_stream_t stream) {
-    return four_six_run(x, n_siblings, y, nullptr, nullptr, amax_in, amax_out, e4m3_max, workspace,
+    const int sizes[1] = {n_siblings};
+    float* ao[1] = {amax_out};
+    return four_six_run(1, sizes, x, y, nullptr, nullptr, amax_in, ao, e4m3_max, workspace, workspace_bytes, true,
+                        stream);
+}
+
+pwq_status nvfp4_4over6_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                                      const pwq_tensor* q_packed, uint8_t* const* sb, float* const* global_scale,
+                                      int e4m3_max, void* workspace, size_t workspace_bytes, pwq_stream_t stream) {
+    return four_six_run(n_groups, group_sizes, x, q_packed, sb, global_scale, nullptr, nullptr, e4m3_max,
+                        workspace, workspace_bytes, false, stream);
+}
+
+pwq_status nvfp4_4over6_fake_quant_grouped(int n_groups, const int* group_sizes, const pwq_tensor* x,
+                                           const pwq_tensor* y, float* const* amax_out, int e4m3_max,
+                                           void* workspace, size_t workspace_bytes, pwq_stream_t stream) {
+    return four_six_run(n_groups, group_sizes, x, y, nullptr, nullptr, nullptr, amax_out, e4m3_max, workspace,
                         workspace_bytes, true, stream);
 }
 

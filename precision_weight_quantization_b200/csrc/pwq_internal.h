@@ -106,12 +106,15 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
                                 float* gs_out, float* amax_out, cudaStream_t s,
                                 const float* const* ts = nullptr);
 
-// NVFP4 "4over6" encode of one group set (the amax from launch_nvfp4_amax's
-// words or from amax_in): every block keeps the candidate, amax mapped to 6
-// or to 4, with the smaller squared error; gs = fl(A / (6 e4m3_max)).
-cudaError_t launch_nvfp4_4over6(const View* x, int n, const View* out, uint8_t* const* sb, bool fake,
-                               const uint32_t* amax_bits, const float* amax_in, float* gs_out, float* amax_out,
-                               int e4m3_max, cudaStream_t s);
+// NVFP4 "4over6" quantise / fake-quantise of sibling groups (launches of up
+// to kMaxLaunchTensors members): the group amax (unless the group has
+// amax_in) and the encode that keeps, per block, the candidate -- amax
+// mapped to 6 or to 4 -- with the smaller squared error; gs = fl(A / (6
+// e4m3_max)).  Workspace: nvfp4_4over6_workspace_bytes(total batch over
+// groups), one amax word per instance.
+size_t nvfp4_4over6_workspace_bytes(int64_t instances);
+cudaError_t launch_nvfp4_4over6(const NvGroup* groups, int n_groups, bool fake, int e4m3_max, void* workspace,
+                               cudaStream_t s);
 
 // FP8 block-wise codes + tile scales re-quantised (dequantise, quantise) into
 // FP8 block-wise (new FP32 tile scales) or MXFP8 (UE8M0 bytes), a list of

@@ -346,3 +346,35 @@ def test_4over6_validation_without_gpu():
     xz = T(L, None, 1, 0, 256, 0, 256)
     assert lib.nvfp4_4over6_fake_quant(ctypes.byref(xz), ctypes.byref(xz), 1, None, None, 256, None, 0,
                                        None) == L.PWQ_OK
+
+
+def test_4over6_grouped_validation_without_gpu():
+    L = _lib()
+    lib = L.lib
+    base = 1 << 40
+    IP = ctypes.c_int * 2
+    xs = (L.PwqTensor * 3)(T(L, base, 4, 64, 256, 64 * 256, 256), T(L, base + (1 << 24), 4, 32, 256, 32 * 256, 256),
+                           T(L, base + (1 << 26), 2, 16, 512, 16 * 512, 512))
+    ys = (L.PwqTensor * 3)(T(L, base + (1 << 30), 4, 64, 256, 64 * 256, 256),
+                           T(L, base + (1 << 30) + (1 << 24), 4, 32, 256, 32 * 256, 256),
+                           T(L, base + (1 << 30) + (1 << 26), 2, 16, 512, 16 * 512, 512))
+    sizes = IP(2, 1)
+    # 4 + 2 instances: 24 bytes, rounded up to 256
+    assert lib.nvfp4_4over6_workspace_size_grouped(2, sizes, xs) == 256
+    assert lib.nvfp4_4over6_workspace_size_grouped(2, IP(2, 9), xs) == 0
+    ws = base + (4 << 30)
+    ao = (ctypes.c_void_p * 2)(None, None)
+    assert lib.nvfp4_4over6_fake_quant_grouped(2, sizes, xs, ys, ao, 300, ws, 256, None) == L.PWQ_ERR_ARG
+    assert lib.nvfp4_4over6_fake_quant_grouped(2, sizes, xs, ys, ao, 256, None, 0, None) == L.PWQ_ERR_WORKSPACE
+    assert lib.nvfp4_4over6_fake_quant_grouped(0, sizes, xs, ys, ao, 256, ws, 256, None) == L.PWQ_ERR_ARG
+    assert lib.nvfp4_4over6_fake_quant_grouped(2, IP(2, 0), xs, ys, ao, 256, ws, 256, None) == L.PWQ_ERR_ARG
+    # an output of group 1 over an input of group 0
+    ys2 = (L.PwqTensor * 3)(ys[0], ys[1], T(L, base + 512, 2, 16, 512, 16 * 512, 512))
+    assert lib.nvfp4_4over6_fake_quant_grouped(2, sizes, xs, ys2, ao, 256, ws, 256, None) == L.PWQ_ERR_OVERLAP
+    # quantise: a missing global scale of the second group
+    qs = (L.PwqTensor * 3)(T(L, base + (1 << 30), 4, 64, 256, 64 * 128, 128),
+                           T(L, base + (1 << 30) + (1 << 24), 4, 32, 256, 32 * 128, 128),
+                           T(L, base + (1 << 30) + (1 << 26), 2, 16, 512, 16 * 256, 256))
+    sb = (ctypes.c_void_p * 3)(base + (2 << 30), base + (2 << 30) + (1 << 24), base + (2 << 30) + (1 << 26))
+    gs = (ctypes.c_void_p * 2)(base + (3 << 30), None)
+    assert lib.nvfp4_4over6_quant_grouped(2, sizes, xs, qs, sb, gs, 256, ws, 256, None) == L.PWQ_ERR_NULL

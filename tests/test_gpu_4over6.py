@@ -191,3 +191,52 @@ def test_4over6_division_exhaustive(P, which):
     torch.cuda.synchronize()
     n, code_bad, quot_bad, slow = counts.tolist()
     assert n > 10 ** 9 and code_bad == 0 and quot_bad == 0, (which, n, code_bad, quot_bad, slow)
+
+
+@pytest.mark.parametrize("E", [256, 448])
+def test_4over6_grouped_call_exact(P, E):
+    """Several sibling groups in one grouped call: batched and plain groups,
+    ragged rows, more than 16 members (two launches of each kind)."""
+    shapes = [[(3, 40, 256), (3, 24, 256)], [(33, 272)], [(2, 64, 512), (2, 16, 512), (2, 16, 512)],
+              [(130, 1040)], [(7, 64), (5, 64), (9, 64), (1, 64), (2, 64), (3, 64), (4, 64), (6, 64)],
+              [(4, 48, 128), (4, 8, 128)]]
+    groups = [[rand_bits(s, seed=900 + 11 * g + 3 * i + E) for i, s in enumerate(grp)] for g, grp in enumerate(shapes)]
+    gg = [[gpu(x) for x in grp] for grp in groups]
+    packed, sb, gs = P.nvfp4_4over6_quant_grouped(gg, E)
+    amax_out = [guard.empty((grp[0].shape[0] if grp[0].ndim == 3 else 1,), torch.float32) for grp in groups]
+    fq = P.nvfp4_4over6_fake_quant_grouped(gg, E, amax_out=amax_out)
+    for g, grp in enumerate(groups):
+        ref = _oracle(grp, E)
+        B = len(ref)
+        for b, (A, gsb, outs) in enumerate(ref):
+            assert f32bits(gs[g])[b] == gsb, (g, b)
+            assert np.float32(amax_out[g][b].item()) == np.float32(A), (g, b)
+            for i, (opk, osb, oy) in enumerate(outs):
+                assert np.array_equal(u8(sb[g][i]).reshape(B, -1, osb.shape[-1])[b], osb), (g, b, i)
+                assert np.array_equal(u8(packed[g][i]).reshape(B, -1, opk.shape[-1])[b], opk), (g, b, i)
+                assert np.array_equal(u16(fq[g][i]).reshape(B, -1, oy.shape[-1])[b], oy), (g, b, i)
+
+
+def test_4over6_dsv3_experts_full_size(P):
+    """The DeepSeek-V3 expert layer (256 experts; gate/up one sibling group
+    per expert, down alone) through one grouped call: every expert's group
+    amax and global scale exactly, and sampled rows of 6 experts (first,
+    last, four random) against the oracle."""
+    xs = [t for t in W.dsv3_experts(device=DEV).values()]
+    packed, sb, gs = P.nvfp4_4over6_quant_grouped([xs[:2], xs[2:]], 256)
+    fq = P.nvfp4_4over6_fake_quant_grouped([xs[:2], xs[2:]], 256)
+    E = xs[0].shape[0]
+    rng = np.random.default_rng(17)
+    experts = sorted({0, E - 1} | set(int(e) for e in rng.integers(0, E, size=4)))
+    for g, members in enumerate((xs[:2], xs[2:])):
+        for e in experts:
+            mb = [u16(m[e]) for m in members]
+            A = max(O.amax_bf16(x) for x in mb)
+            assert f32bits(gs[g])[e] == np.float32(O.nvfp4_4over6_global_scale(A, 256)).view(np.uint32), (g, e)
+            for i, x in enumerate(mb):
+                M = x.shape[0]
+                rows = sorted({0, M - 1} | set(int(r) for r in rng.integers(0, M, size=6)))
+                opk, osb, _ = O.nvfp4_4over6_quant(x[rows], A, 256)
+                assert np.array_equal(u8(packed[g][i][e])[rows], opk), (g, e, i)
+                assert np.array_equal(u8(sb[g][i][e])[rows], osb), (g, e, i)
+                assert np.array_equal(u16(fq[g][i][e][rows]), O.nvfp4_4over6_fake_quant(x[rows], A, 256)), (g, e, i)
