@@ -55,6 +55,9 @@ def _desc(t: torch.Tensor, name: str, packed: bool = False) -> PwqTensor:
     if not t.is_cuda:
         raise ValueError("%s must be a CUDA tensor" % name)
     B, M, N, bs, rs = _bmn(t, name)
+    if t.numel() == 0:
+        # an empty tensor's strides are arbitrary; the library launches nothing for it
+        return PwqTensor(t.data_ptr(), B, M, 2 * N if packed else N, M * N, N)
     if N > 1 and t.stride(-1) != 1:
         raise ValueError("%s: last dimension must be contiguous" % name)
     return PwqTensor(t.data_ptr(), B, M, 2 * N if packed else N, bs, rs)

@@ -515,18 +515,20 @@ pwq_status nvfp4_group_amax(const pwq_tensor* x, int n_siblings, float* amax_out
 
 namespace {
 
-// Shared body of nvfp4_quant / nvfp4_fake_quant and their grouped forms.
-pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq_tensor* out,
-                  uint8_t* const* sb, float* const* gs_out, const float* amax_in, float* const* amax_out,
-                  void* ws, size_t ws_bytes, bool fake, pwq_stream_t stream, bool sb_mma = false) {
+// Validates the groups of an NVFP4 call (nvfp4_quant / nvfp4_fake_quant,
+// their grouped and 4over6 forms) and collects the non-empty ones for the
+// launcher, with the extents of every input and output and the call's
+// instance count.
+pwq_status collect_nv_groups(int n_groups, const int* sizes, const pwq_tensor* x, const pwq_tensor* out,
+                             uint8_t* const* sb, float* const* gs_out, const float* amax_in,
+                             float* const* amax_out, bool fake, bool sb_mma, std::vector<GroupCheck>& groups,
+                             std::vector<pwq::NvGroup>& launch, std::vector<Extent>& ins, std::vector<Extent>& outs,
+                             std::vector<std::pair<Extent, Extent>>& aliases, int64_t* instances) {
     if (n_groups < 1 || n_groups > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group count out of range");
     if (!sizes || !x || !out) return fail(PWQ_ERR_NULL, "group sizes / tensors");
-    std::vector<GroupCheck> groups(n_groups);
-    std::vector<Extent> ins, outs;
-    std::vector<std::pair<Extent, Extent>> aliases;
-    std::vector<pwq::NvGroup> launch;
+    groups.resize(n_groups);
     int m = 0;
-    int64_t instances = 0;
+    *instances = 0;
     for (int g = 0; g < n_groups; ++g) {
         const int n = sizes[g];
         if (n < 1 || n > PWQ_MAX_SIBLINGS || m + n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group size");
@@ -557,7 +559,7 @@ pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq
                 outs.push_back(extent_of(amax_out[g], (size_t)B * 4));
             }
             launch.push_back(ng);
-            instances += B;
+            *instances += B;
         }
         m += n;
     }
@@ -566,6 +568,21 @@ pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq
         if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
         ins.push_back(extent_of(amax_in, (size_t)x[0].batch * 4));
     }
+    return PWQ_OK;
+}
+
+// Shared body of nvfp4_quant / nvfp4_fake_quant and their grouped forms.
+pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq_tensor* out,
+                  uint8_t* const* sb, float* const* gs_out, const float* amax_in, float* const* amax_out,
+                  void* ws, size_t ws_bytes, bool fake, pwq_stream_t stream, bool sb_mma = false) {
+    std::vector<GroupCheck> groups;
+    std::vector<Extent> ins, outs;
+    std::vector<std::pair<Extent, Extent>> aliases;
+    std::vector<pwq::NvGroup> launch;
+    int64_t instances = 0;
+    pwq_status cst = collect_nv_groups(n_groups, sizes, x, out, sb, gs_out, amax_in, amax_out, fake, sb_mma, groups,
+                                       launch, ins, outs, aliases, &instances);
+    if (cst != PWQ_OK) return cst;
     if (launch.empty()) return PWQ_OK;
     if (!amax_in) {
         pwq_status st = check_workspace(ws, ws_bytes, instances);
@@ -644,51 +661,14 @@ pwq_status four_six_run(int n_groups, const int* sizes, const pwq_tensor* x, con
                         uint8_t* const* sb, float* const* gs_out, const float* amax_in, float* const* amax_out,
                         int e4m3_max, void* ws, size_t ws_bytes, bool fake, pwq_stream_t stream) {
     if (e4m3_max != 256 && e4m3_max != 448) return fail(PWQ_ERR_ARG, "e4m3_max must be 256 or 448");
-    if (n_groups < 1 || n_groups > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group count out of range");
-    if (!sizes || !x || !out) return fail(PWQ_ERR_NULL, "group sizes / tensors");
-    std::vector<GroupCheck> groups(n_groups);
+    std::vector<GroupCheck> groups;
     std::vector<Extent> ins, outs;
     std::vector<std::pair<Extent, Extent>> aliases;
     std::vector<pwq::NvGroup> launch;
-    int m = 0;
     int64_t instances = 0;
-    for (int g = 0; g < n_groups; ++g) {
-        const int n = sizes[g];
-        if (n < 1 || n > PWQ_MAX_SIBLINGS || m + n > PWQ_MAX_GROUPED) return fail(PWQ_ERR_ARG, "group size");
-        GroupCheck& G = groups[g];
-        pwq_status st = check_nv_group(x + m, out + m, fake ? nullptr : sb + m, n, fake, &G, ins, outs, aliases);
-        if (st != PWQ_OK) return st;
-        const int64_t B = x[m].batch;
-        if (!G.all_empty && B > 0) {
-            pwq::NvGroup ng;
-            ng.x = G.x;
-            ng.out = G.out;
-            ng.sb = fake ? nullptr : G.sb;
-            ng.n = n;
-            ng.amax_in = amax_in;
-            ng.gs_out = nullptr;
-            ng.amax_out = nullptr;
-            if (!fake) {
-                if (!gs_out || !gs_out[g]) return fail(PWQ_ERR_NULL, "global_scale");
-                if ((uintptr_t)gs_out[g] % 4 != 0) return fail(PWQ_ERR_ALIGN, "global_scale");
-                ng.gs_out = gs_out[g];
-                outs.push_back(extent_of(gs_out[g], (size_t)B * 4));
-            }
-            if (amax_out && amax_out[g]) {
-                if ((uintptr_t)amax_out[g] % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_out");
-                ng.amax_out = amax_out[g];
-                outs.push_back(extent_of(amax_out[g], (size_t)B * 4));
-            }
-            launch.push_back(ng);
-            instances += B;
-        }
-        m += n;
-    }
-    if (amax_in) {
-        if (n_groups != 1) return fail(PWQ_ERR_ARG, "amax_in needs a single group");
-        if ((uintptr_t)amax_in % 4 != 0) return fail(PWQ_ERR_ALIGN, "amax_in");
-        ins.push_back(extent_of(amax_in, (size_t)x[0].batch * 4));
-    }
+    pwq_status cst = collect_nv_groups(n_groups, sizes, x, out, sb, gs_out, amax_in, amax_out, fake, false, groups,
+                                       launch, ins, outs, aliases, &instances);
+    if (cst != PWQ_OK) return cst;
     if (launch.empty()) return PWQ_OK;
     if (!amax_in) {
         if (!ws || (uintptr_t)ws % 4 != 0 || ws_bytes < pwq::nvfp4_4over6_workspace_bytes(instances))

@@ -196,10 +196,11 @@ def test_4over6_division_exhaustive(P, which):
 @pytest.mark.parametrize("E", [256, 448])
 def test_4over6_grouped_call_exact(P, E):
     """Several sibling groups in one grouped call: batched and plain groups,
-    ragged rows, more than 16 members (two launches of each kind)."""
+    ragged rows, members with no rows, more than 16 members (two launches of
+    each kind)."""
     shapes = [[(3, 40, 256), (3, 24, 256)], [(33, 272)], [(2, 64, 512), (2, 16, 512), (2, 16, 512)],
               [(130, 1040)], [(7, 64), (5, 64), (9, 64), (1, 64), (2, 64), (3, 64), (4, 64), (6, 64)],
-              [(4, 48, 128), (4, 8, 128)]]
+              [(4, 48, 128), (4, 8, 128)], [(5, 64), (0, 64), (3, 64)], [(6, 32), (0, 32)]]
     groups = [[rand_bits(s, seed=900 + 11 * g + 3 * i + E) for i, s in enumerate(grp)] for g, grp in enumerate(shapes)]
     gg = [[gpu(x) for x in grp] for grp in groups]
     packed, sb, gs = P.nvfp4_4over6_quant_grouped(gg, E)
