@@ -35,6 +35,8 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cooperative_groups.h>
+
 #include "pwq_internal.h"
 
 namespace pwq {
@@ -535,6 +537,119 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kern
         }
         u = start;
     }
+}
+
+// ---------------------------------------------------------------- small instances, one cluster each
+//
+// When every instance (batch index of a sibling group) of a call has at most
+// kClusterUnits 16-element blocks, one thread-block cluster of up to
+// kMaxCluster CTAs owns each instance: every thread holds up to
+// kClusterUnitsPerThread blocks in registers, the CTA maxima meet across the
+// cluster in distributed shared memory (barrier.cluster orders them), and
+// the blocks are encoded from the registers.  One launch, one read of the
+// input, no workspace and no global atomics -- for the small tensors whose
+// time the single pass's queue, amax handshake and workspace clear would
+// dominate.  The units of an instance are numbered as for the 4over6 kernels
+// (member after member, row after row); CTA r of a cluster takes the r-th
+// contiguous share of them.
+namespace cg = cooperative_groups;
+
+constexpr int kClusterUnitsPerThread = 4;
+constexpr int kClusterCtaUnits = kThreads * kClusterUnitsPerThread;   // 1024 blocks per CTA
+constexpr int kMaxCluster = 8;                                         // portable cluster size
+constexpr uint32_t kClusterUnits = kMaxCluster * kClusterCtaUnits;     // 131072 elements
+
+template <bool kFake>
+__global__ void __launch_bounds__(kThreads) nvfp4_cluster_kernel(const FourSixArgs a) {
+    __shared__ ScaleTable tab;
+    __shared__ uint32_t red[kThreads / 32];
+    __shared__ uint32_t cta_max, s_amax;
+    const cg::cluster_group cluster = cg::this_cluster();
+    const uint32_t cs = cluster.num_blocks(), rank = cluster.block_rank();
+    const uint32_t inst = blockIdx.x / cs;
+    int gi = 0;
+    while (gi + 1 < a.n_groups && inst >= a.g[gi + 1].inst0) ++gi;
+    const FourSixGroup& G = a.g[gi];
+    const uint32_t b = inst - G.inst0;
+    const uint32_t per = (G.units + cs - 1) / cs;
+    const uint32_t u0 = min(G.units, rank * per), u1 = min(G.units, u0 + per);
+
+    // ---- the CTA's blocks into registers, and their maximum
+    uint4 lo[kClusterUnitsPerThread], hi[kClusterUnitsPerThread];
+    uint32_t m = 0u;
+#pragma unroll
+    for (int k = 0; k < kClusterUnitsPerThread; ++k) {
+        const uint32_t r = u0 + threadIdx.x + (uint32_t)k * kThreads;
+        lo[k] = hi[k] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < u1) {
+            const int i = four_six_member(a, G, r);
+            int64_t xo, oo;
+            four_six_offsets<kFake>(a.m[i], b, r - a.mblk0[i], xo, oo);
+            lo[k] = ld_stream_v4(a.m[i].x + xo);
+            hi[k] = ld_stream_v4(a.m[i].x + xo + 16);
+        }
+        m = max(m, max(amax_bits8(lo[k]), amax_bits8(hi[k])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31u) == 0u) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kThreads / 32; ++w) m = max(m, red[w]);
+        cta_max = m;
+    }
+    // ---- the group amax: every CTA reads every CTA's maximum of the cluster
+    cluster.sync();
+    if (threadIdx.x < 32u) {
+        uint32_t v = threadIdx.x < cs ? *cluster.map_shared_rank(&cta_max, threadIdx.x) : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (threadIdx.x == 0) s_amax = v;
+    }
+    // no CTA may leave while another still reads its cta_max: arrive now,
+    // wait before the end
+    cluster.barrier_arrive();
+    __syncthreads();
+    const float A = G.amax_in ? G.amax_in[b] : __uint_as_float(s_amax << 16);
+    const float gs = __fdiv_rn(A, 2688.0f);
+    const float six_gs = __fmul_rn(6.0f, gs);
+    const float r6 = __frcp_rn(six_gs);
+    const bool fast6 = div_fast_ok(six_gs);
+    const uint64_t gs2 = f32x2(gs, gs);
+    fill_scale_table(tab, gs);
+    if (rank == 0 && threadIdx.x == 0) {
+        if (G.gs_out) G.gs_out[b] = gs;
+        if (G.amax_out) G.amax_out[b] = A;
+    }
+    __syncthreads();
+
+    // ---- encode from the registers
+#pragma unroll
+    for (int k = 0; k < kClusterUnitsPerThread; ++k) {
+        const uint32_t r = u0 + threadIdx.x + (uint32_t)k * kThreads;
+        if (r < u1) {
+            const int i = four_six_member(a, G, r);
+            const Sib& S = a.m[i];
+            const uint32_t j = r - a.mblk0[i];
+            int64_t xo, oo;
+            four_six_offsets<kFake>(S, b, j, xo, oo);
+            const uint32_t mw = hmax_abs(amax_word8(lo[k]), amax_word8(hi[k])) & 0x7fff7fffu;
+            const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
+            const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
+            const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
+            const float4 e = tab.e[sb];
+            const uint32_t c0 = codes_half(lo[k], e.x, e.y), c1 = codes_half(hi[k], e.x, e.y);
+            if (kFake) {
+                const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
+                st_v4(S.out + oo, dequant_half_h(c0, sb2, gs2));
+                st_v4(S.out + oo + 16, dequant_half_h(c1, sb2, gs2));
+            } else {
+                st_v2(S.out + oo, make_uint2(c0, c1));   // 8-byte aligned: 2 j even
+                S.sb[(int64_t)b * (S.chunks >> 1) + j] = (uint8_t)sb;
+            }
+        }
+    }
+    cluster.barrier_wait();
 }
 
 // Dequantise: a grouped walk over 16-element blocks like MXFP8's.  Per
@@ -1370,6 +1485,96 @@ cudaError_t launch_nvfp4_4over6(const NvGroup* groups, int n_groups, bool fake, 
         inst += F.batch;
         n_members += G.n;
         ++a.n_groups;
+    }
+    return flush();
+}
+
+bool nvfp4_cluster_ok(const NvGroup* groups, int n_groups) {
+    for (int gi = 0; gi < n_groups; ++gi) {
+        const NvGroup& G = groups[gi];
+        if (G.sb_mma || G.ts) return false;
+        int64_t units = 0;
+        for (int i = 0; i < G.n; ++i) units += G.x[i].rows * (G.x[i].cols / 16);
+        if (units > (int64_t)kClusterUnits) return false;
+    }
+    return true;
+}
+
+cudaError_t launch_nvfp4_cluster(const NvGroup* groups, int n_groups, bool fake, cudaStream_t s) {
+    FourSixArgs a{};
+    uint32_t max_units = 0;
+    int n_members = 0;
+    auto flush = [&]() -> cudaError_t {
+        if (a.n_groups == 0) return cudaSuccess;
+        const uint32_t n_inst = a.g[a.n_groups - 1].inst0 + a.g[a.n_groups - 1].batch;
+        const uint32_t cs = std::max<uint32_t>(1, (max_units + kClusterCtaUnits - 1) / kClusterCtaUnits);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(n_inst * cs);
+        cfg.blockDim = dim3(kThreads);
+        cfg.stream = s;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = cs;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        cudaError_t e = fake ? cudaLaunchKernelEx(&cfg, nvfp4_cluster_kernel<true>, a)
+                             : cudaLaunchKernelEx(&cfg, nvfp4_cluster_kernel<false>, a);
+        a = FourSixArgs{};
+        max_units = 0;
+        n_members = 0;
+        return e;
+    };
+    for (int gi = 0; gi < n_groups; ++gi) {
+        const NvGroup& G = groups[gi];
+        for (int64_t b0 = 0; b0 < G.x[0].batch;) {
+            if (n_members + G.n > kMaxLaunchTensors || a.n_groups == kMaxLaunchTensors) {
+                cudaError_t e = flush();
+                if (e != cudaSuccess) return e;
+            }
+            // at most 2^16 instances per launch keep the grid within range
+            const uint32_t inst0 = a.n_groups ? a.g[a.n_groups - 1].inst0 + a.g[a.n_groups - 1].batch : 0u;
+            const uint32_t nb = (uint32_t)std::min<int64_t>(G.x[0].batch - b0, 65536 - (int64_t)inst0);
+            if (nb == 0) {
+                cudaError_t e = flush();
+                if (e != cudaSuccess) return e;
+                continue;
+            }
+            FourSixGroup& F = a.g[a.n_groups];
+            F.unit0 = 0;
+            F.inst0 = inst0;
+            F.batch = nb;
+            F.m0 = n_members;
+            F.nm = G.n;
+            F.amax_in = G.amax_in ? G.amax_in + b0 : nullptr;
+            F.gs_out = G.gs_out ? G.gs_out + b0 : nullptr;
+            F.amax_out = G.amax_out ? G.amax_out + b0 : nullptr;
+            uint32_t units = 0;
+            for (int i = 0; i < G.n; ++i) {
+                Sib& S = a.m[n_members + i];
+                const View& x = G.x[i];
+                const View& o = G.out[i];
+                S.x = x.ptr + b0 * x.bstride;
+                S.x_bs = x.bstride;
+                S.x_rs = x.rstride;
+                S.out = o.ptr + b0 * o.bstride;
+                S.o_bs = o.bstride;
+                S.o_rs = o.rstride;
+                S.chunks = (uint32_t)(x.rows * (x.cols / 8));
+                S.sb = fake ? nullptr : G.sb[i] + b0 * (int64_t)(S.chunks / 2);
+                S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
+                set_source(S, x, nullptr);
+                S.dense_o = dense_rows(o, fake ? o.cols * 2 : o.cols / 2);
+                a.mblk0[n_members + i] = units;
+                units += S.chunks / 2;
+            }
+            b0 += nb;
+            F.units = units;
+            max_units = std::max(max_units, units);
+            n_members += G.n;
+            ++a.n_groups;
+        }
     }
     return flush();
 }

@@ -604,6 +604,9 @@ pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq
                 }
             }
     }
+    // every instance small: one cluster each, one launch, the workspace unused
+    if (pwq::nvfp4_cluster_ok(launch.data(), (int)launch.size()))
+        return from_cuda(pwq::launch_nvfp4_cluster(launch.data(), (int)launch.size(), fake, s));
     if (amax_in) {
         const pwq::NvGroup& G = launch[0];
         return from_cuda(pwq::launch_nvfp4_encode(G.x, G.n, G.out, G.sb, fake, nullptr, amax_in, G.gs_out,

@@ -113,6 +113,13 @@ cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* 
 // e4m3_max)).  Workspace: nvfp4_4over6_workspace_bytes(total batch over
 // groups), one amax word per instance.
 size_t nvfp4_4over6_workspace_bytes(int64_t instances);
+
+// NVFP4 quantise / fake-quantise of groups whose every instance has at most
+// 131072 elements (BF16 source, dense block scales): one thread-block
+// cluster per instance, one launch, no workspace.  nvfp4_cluster_ok tells
+// whether a call qualifies.
+bool nvfp4_cluster_ok(const NvGroup* groups, int n_groups);
+cudaError_t launch_nvfp4_cluster(const NvGroup* groups, int n_groups, bool fake, cudaStream_t s);
 cudaError_t launch_nvfp4_4over6(const NvGroup* groups, int n_groups, bool fake, int e4m3_max, void* workspace,
                                cudaStream_t s);
 
