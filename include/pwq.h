@@ -183,7 +183,11 @@ pwq_status mxfp8_dequant(const pwq_tensor* q, const uint8_t* scale, const pwq_te
  * counters and queue head live in caller-provided workspace of at least
  * nvfp4_workspace_size() / nvfp4_workspace_size_grouped() bytes (4-byte
  * aligned; 256-byte aligned is best).  Its contents on entry do not matter.
- * When amax_in is given, workspace may be NULL.
+ * When amax_in is given, workspace may be NULL.  Calls whose every group
+ * instance has at most 131072 elements (and whose block scales are dense)
+ * run one thread-block cluster per instance instead, also one launch, with
+ * the group amax exchanged in distributed shared memory; the workspace is
+ * still validated but not used.
  */
 
 /* Bytes of workspace an NVFP4 quantise / fake-quantise call over these
