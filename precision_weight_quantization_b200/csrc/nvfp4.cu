@@ -1729,7 +1729,11 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
                 M.sf_slab = mma_scale_slab_bytes(x.rows, x.cols / 16);
                 M.sb = fake ? nullptr : G.sb[i] + b0 * (G.sb_mma ? M.sf_slab : (int64_t)(M.chunks / 2));
                 M.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
-                M.dense_x = dense_rows(x, fp8 ? x.cols : x.cols * 2);
+                // the stage copy of a dense slab needs 16-byte aligned addresses;
+                // E4M3 code tensors are only checked to 8 bytes, so such a
+                // member is read row by row with 8-byte loads instead
+                M.dense_x = dense_rows(x, fp8 ? x.cols : x.cols * 2) &&
+                            (!fp8 || ((uintptr_t)M.x % 16 == 0 && (take == 1 || x.bstride % 16 == 0)));
                 M.dense_o = dense_rows(o, fake ? o.cols * 2 : o.cols / 2);
                 M.tn = (uint32_t)((x.cols + 127) / 128);
                 M.ts_bs = (int64_t)((x.rows + 127) / 128) * M.tn;

@@ -133,6 +133,35 @@ def test_fp8_to_nvfp4_siblings(P, shapes, raw):
         assert torch.equal(pk2[i], pk[i]) and torch.equal(sb2[i].view(torch.uint8), sb[i].view(torch.uint8))
 
 
+def test_fp8_to_nvfp4_codes_only_8_byte_aligned(P):
+    """E4M3 code tensors need only 8-byte alignment: dense code rows whose
+    base, or whose batch stride, is 8 bytes off a 16-byte boundary are read
+    with 8-byte loads instead of the stage copy, with the same results."""
+    M, N = 256, 512
+    q, s = codes_and_scales((2, M, N), seed=41)
+    want = [O.fp8_block_requant_nvfp4([q[b]], [s[b]]) for b in range(2)]
+    # one matrix at base + 8
+    buf = torch.zeros(M * N + 8, dtype=torch.uint8, device=DEV)
+    q0 = buf[8:8 + M * N].view(M, N)
+    q0.copy_(torch.from_numpy(q[0]).to(DEV))
+    assert q0.data_ptr() % 16 == 8
+    pk, sb, g = P.fp8_block_requant_nvfp4(q0, torch.from_numpy(s[0]).to(DEV))
+    A, out, gs = want[0]
+    assert np.array_equal(f32bits(g), gs.view(np.uint32))
+    assert np.array_equal(u8(pk), out[0][0]) and np.array_equal(u8(sb), out[0][1])
+    # a batch of two with a batch stride of M * N + 8 bytes
+    bs = M * N + 8
+    buf2 = torch.zeros(2 * bs, dtype=torch.uint8, device=DEV)
+    q2 = buf2.as_strided((2, M, N), (bs, N, 1))
+    for b in range(2):
+        q2[b].copy_(torch.from_numpy(q[b]).to(DEV))
+    pk2, sb2, g2 = P.fp8_block_requant_nvfp4(q2, torch.from_numpy(s).to(DEV))
+    for b in range(2):
+        A, out, gs = want[b]
+        assert f32bits(g2)[b] == gs.view(np.uint32)[0], b
+        assert np.array_equal(u8(pk2[b]), out[0][0]) and np.array_equal(u8(sb2[b]), out[0][1]), b
+
+
 def test_fp8_to_nvfp4_equals_quant_of_dequant_on_gpu(P):
     q, s = codes_and_scales((4, 200, 512), seed=31)
     tq, ts = to_gpu_codes(q), torch.from_numpy(s).to(DEV)
