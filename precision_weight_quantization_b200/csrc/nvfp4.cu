@@ -755,6 +755,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_dequant_kernel(const __grid_co
 // semantics before it reads the amax.
 constexpr int kFlowThreads = 256;
 constexpr uint32_t kItemChunks = 2048;                        // 16384 elements
+constexpr uint32_t kItemChunksFp8 = 2 * kItemChunks;          // FP8 source: 32 KB of codes, two halves
 constexpr int kItemChunksPerThread = kItemChunks / kFlowThreads;   // 8
 constexpr int kFlowMaxInst = 512;                             // instances per launch
 constexpr uint64_t kFlowWaitNs = kFlowWaitLimitNs;             // 2 s
@@ -924,7 +925,7 @@ struct FlowItem {
 };
 
 __device__ __forceinline__ FlowItem flow_item(const FlowTables& t, uint32_t I, uint32_t total, uint32_t q,
-                                              uint32_t& hint) {
+                                              uint32_t& hint, uint32_t chunks) {
     FlowItem it{};
     it.valid = q < 2u * total;
     if (!it.valid) return it;
@@ -944,8 +945,8 @@ __device__ __forceinline__ FlowItem flow_item(const FlowTables& t, uint32_t I, u
     it.g = g;
     it.m = mi;
     it.b = inst - G.inst_begin;
-    it.c0 = (k - M.item_off) * kItemChunks;
-    it.c1 = min(it.c0 + kItemChunks, M.chunks);
+    it.c0 = (k - M.item_off) * chunks;
+    it.c1 = min(it.c0 + chunks, M.chunks);
     return it;
 }
 
@@ -981,7 +982,7 @@ __device__ __forceinline__ uint32_t flow_lc(int j, uint32_t tid) {
 template <bool kFake, bool kFast, bool kFull>
 __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThread], const FlowItem& it,
                                             const FlowMember& M, const ScaleTable& tab, float gs, float six_gs,
-                                            float r6, bool fast6, uint64_t pol) {
+                                            float r6, bool fast6, uint64_t pol, uint32_t c_off = 0u) {
     const uint32_t tid = threadIdx.x;
     char* ob = M.out + (int64_t)it.b * M.o_bs;
     uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.sf_mma ? M.sf_slab : (int64_t)(M.chunks >> 1));
@@ -990,7 +991,7 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
         const uint4 lo = v[2 * i], hi = v[2 * i + 1];
         // c is even (the block's first chunk); rows hold an even number of
         // chunks, so c + 1 is in the same row and c < c1 implies c + 1 < c1
-        const uint32_t c = it.c0 + flow_lc(2 * i, tid);
+        const uint32_t c = it.c0 + c_off + flow_lc(2 * i, tid);
         const uint32_t mw = hmax_abs(amax_word8(lo), amax_word8(hi)) & 0x7fff7fffu;
         const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
         float ratio;
@@ -1084,6 +1085,9 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
     // amax runs; thread kQueueThread (another warp) takes queue positions and
     // decodes items, so the two chains overlap within an item.
     constexpr uint32_t kQueueThread = 32;
+    // FP8 source: items of two halves of kItemChunks chunks (32 KB of codes)
+    constexpr uint32_t kChunks = kFp8 ? kItemChunksFp8 : kItemChunks;
+    constexpr int kHalves = kFp8 ? 2 : 1;
     const uint32_t tid = threadIdx.x;
     const uint32_t stage0 = smem_addr(flow_smem);
     const uint32_t I = a.n_inst, L = a.lead, total = a.total_items;
@@ -1121,7 +1125,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
     if (tid == 0) {
         uint32_t hint0 = 0u;
         for (int s = 0; s < kFlowStages; ++s) {
-            items[s] = flow_item(t, I, total, s_q[s], hint0);
+            items[s] = flow_item(t, I, total, s_q[s], hint0, kChunks);
             if (items[s].valid)
                 flow_stage(t.m[items[s].m], items[s], stage0 + s * kFlowStageBytes, smem_addr(&bars[s]),
                            flow_amax_policy(t, items[s], keep, stream));
@@ -1150,95 +1154,100 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         if (tid == kQueueThread) next_q = atomicAdd(a.counter, 1u);   // decoded at the next item
         const FlowMember& M = t.m[it.m];
 
-        // ---- the item's data, into registers
+        // ---- the item's data
         if (!mbar_wait_bounded(smem_addr(&bars[st]), par, kFlowWaitNs)) atomicOr(&g_flow_error, kErrFlowTimeout);
-        uint4 v[kItemChunksPerThread];
         const unsigned char* buf = flow_smem + st * kFlowStageBytes;
-        const bool full = (it.c1 - it.c0 == kItemChunks) && M.dense_x && M.dense_o;
-        // FP8 source, amax item over whole chunk pairs: the block maxima come
-        // from the largest code magnitude of each pair (one tile scale each),
-        // bf16(fl(dec(mc) |s|)) -- rounding is monotone and symmetric in sign,
-        // so that is the largest |y| of the pair -- without dequantising
-        uint32_t fp8_m = 0u;
-        const bool fp8_amax = kFp8 && full && !it.is_e;
-        if (fp8_amax) {
+        const bool full = (it.c1 - it.c0 == kChunks) && M.dense_x && M.dense_o;
+        // the chunks of half h into registers (BF16 values; FP8 codes dequantised)
+        auto load_half = [&](int h, uint4 (&v)[kItemChunksPerThread]) {
+            const uint32_t hoff = (uint32_t)h * kItemChunks;
+            if (full) {
+                if (kFp8) {
 #pragma unroll
-            for (int j = 0; j < kItemChunksPerThread; j += 2) {
-                const uint32_t lc = flow_lc(j, tid);
-                const uint4 cc = *reinterpret_cast<const uint4*>(buf + lc * 8u);
-                const uint32_t c = it.c0 + lc;
-                const uint32_t r = fdiv(c, M.cpr);
-                const uint32_t k = c - r * M.cpr.d;
-                const float sc = __ldg(M.ts + (int64_t)it.b * M.ts_bs + (r >> 7) * M.tn + (k >> 4));
-                const uint32_t lanes = __vmaxu2(e4m3_maxmag_lanes(make_uint2(cc.x, cc.y)),
-                                                e4m3_maxmag_lanes(make_uint2(cc.z, cc.w)));
-                fp8_m = max(fp8_m, fp8_amax_bits16(e4m3_maxmag_fin(lanes), sc));
-            }
-        } else if (full) {
-            if (kFp8) {
+                    for (int j = 0; j < kItemChunksPerThread; j += 2) {
+                        // lc even: the block's two chunks lie in one row and one
+                        // tile, so one row / column step and one tile-scale load
+                        const uint32_t lc = hoff + flow_lc(j, tid);
+                        const uint4 cc = *reinterpret_cast<const uint4*>(buf + lc * 8u);
+                        const uint32_t c = it.c0 + lc;
+                        const uint32_t r = fdiv(c, M.cpr);
+                        const uint32_t k = c - r * M.cpr.d;
+                        const float sc = __ldg(M.ts + (int64_t)it.b * M.ts_bs + (r >> 7) * M.tn + (k >> 4));
+                        v[j] = fp8_dequant8(make_uint2(cc.x, cc.y), sc);
+                        v[j + 1] = fp8_dequant8(make_uint2(cc.z, cc.w), sc);
+                    }
+                } else {
 #pragma unroll
-                for (int j = 0; j < kItemChunksPerThread; j += 2) {
-                    // lc even: the block's two chunks lie in one row and one
-                    // tile, so one row / column step and one tile-scale load
-                    const uint32_t lc = flow_lc(j, tid);
-                    const uint4 cc = *reinterpret_cast<const uint4*>(buf + lc * 8u);
-                    const uint32_t c = it.c0 + lc;
-                    const uint32_t r = fdiv(c, M.cpr);
-                    const uint32_t k = c - r * M.cpr.d;
-                    const float sc = __ldg(M.ts + (int64_t)it.b * M.ts_bs + (r >> 7) * M.tn + (k >> 4));
-                    v[j] = fp8_dequant8(make_uint2(cc.x, cc.y), sc);
-                    v[j + 1] = fp8_dequant8(make_uint2(cc.z, cc.w), sc);
+                    for (int j = 0; j < kItemChunksPerThread; ++j)
+                        v[j] = *reinterpret_cast<const uint4*>(buf + flow_lc(j, tid) * 16u);
                 }
             } else {
+                const char* xb = M.x + (int64_t)it.b * M.x_bs;
 #pragma unroll
-                for (int j = 0; j < kItemChunksPerThread; ++j)
-                    v[j] = *reinterpret_cast<const uint4*>(buf + flow_lc(j, tid) * 16u);
-            }
-        } else {
-            const char* xb = M.x + (int64_t)it.b * M.x_bs;
-#pragma unroll
-            for (int j = 0; j < kItemChunksPerThread; ++j) {
-                const uint32_t lc = flow_lc(j, tid);   // chunk within the item
-                const uint32_t c = it.c0 + lc;
-                v[j] = make_uint4(0u, 0u, 0u, 0u);
-                if (c < it.c1) {
-                    if (kFp8) {
-                        uint2 codes;
-                        if (M.dense_x) {
-                            codes = *reinterpret_cast<const uint2*>(buf + lc * 8u);
+                for (int j = 0; j < kItemChunksPerThread; ++j) {
+                    const uint32_t lc = hoff + flow_lc(j, tid);   // chunk within the item
+                    const uint32_t c = it.c0 + lc;
+                    v[j] = make_uint4(0u, 0u, 0u, 0u);
+                    if (c < it.c1) {
+                        if (kFp8) {
+                            uint2 codes;
+                            if (M.dense_x) {
+                                codes = *reinterpret_cast<const uint2*>(buf + lc * 8u);
+                            } else {
+                                const uint32_t r = fdiv(c, M.cpr);
+                                codes = ld_stream_v2(xb + (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 8);
+                            }
+                            v[j] = flow_fp8_chunk(M, it, codes, c);
+                        } else if (M.dense_x) {
+                            v[j] = *reinterpret_cast<const uint4*>(buf + lc * 16u);
                         } else {
                             const uint32_t r = fdiv(c, M.cpr);
-                            codes = ld_stream_v2(xb + (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 8);
+                            v[j] = ld_hint_v4(xb + (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 16,
+                                              it.is_e ? stream : keep);
                         }
-                        v[j] = flow_fp8_chunk(M, it, codes, c);
-                    } else if (M.dense_x) {
-                        v[j] = *reinterpret_cast<const uint4*>(buf + lc * 16u);
-                    } else {
-                        const uint32_t r = fdiv(c, M.cpr);
-                        v[j] = ld_hint_v4(xb + (int64_t)r * M.x_rs + (int64_t)(c - r * M.cpr.d) * 16,
-                                          it.is_e ? stream : keep);
                     }
                 }
             }
-        }
+        };
 
         if (!it.is_e) {
             // ---- amax item
-            uint32_t m;
-            if (fp8_amax) {
-                m = fp8_m;
-            } else {
-                uint32_t mw = 0u;
+            uint32_t m = 0u;
 #pragma unroll
-                for (int j = 0; j < kItemChunksPerThread; ++j) mw = hmax_abs(mw, amax_word8(v[j]));
-                mw &= 0x7fff7fffu;
-                m = max(mw & 0xffffu, mw >> 16);
+            for (int h = 0; h < kHalves; ++h) {
+                if (kFp8 && full) {
+                    // FP8 source over whole chunk pairs: the block maxima come
+                    // from the largest code magnitude of each pair (one tile
+                    // scale each), bf16(fl(dec(mc) |s|)) -- rounding is
+                    // monotone and symmetric in sign, so that is the largest
+                    // |y| of the pair -- without dequantising
+#pragma unroll
+                    for (int j = 0; j < kItemChunksPerThread; j += 2) {
+                        const uint32_t lc = (uint32_t)h * kItemChunks + flow_lc(j, tid);
+                        const uint4 cc = *reinterpret_cast<const uint4*>(buf + lc * 8u);
+                        const uint32_t c = it.c0 + lc;
+                        const uint32_t r = fdiv(c, M.cpr);
+                        const uint32_t k = c - r * M.cpr.d;
+                        const float sc = __ldg(M.ts + (int64_t)it.b * M.ts_bs + (r >> 7) * M.tn + (k >> 4));
+                        const uint32_t lanes = __vmaxu2(e4m3_maxmag_lanes(make_uint2(cc.x, cc.y)),
+                                                        e4m3_maxmag_lanes(make_uint2(cc.z, cc.w)));
+                        m = max(m, fp8_amax_bits16(e4m3_maxmag_fin(lanes), sc));
+                    }
+                } else {
+                    uint4 v[kItemChunksPerThread];
+                    load_half(h, v);
+                    uint32_t mw = 0u;
+#pragma unroll
+                    for (int j = 0; j < kItemChunksPerThread; ++j) mw = hmax_abs(mw, amax_word8(v[j]));
+                    mw &= 0x7fff7fffu;
+                    m = max(m, max(mw & 0xffffu, mw >> 16));
+                }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((tid & 31u) == 0u) red[k & 1u][tid >> 5] = m;
             if (tid == kQueueThread) {
-                items[ahead] = flow_item(t, I, total, pend, hint);
+                items[ahead] = flow_item(t, I, total, pend, hint, kChunks);
                 pend = next_q;
             }
             __syncthreads();   // stage st is free; red and the new item are published
@@ -1261,10 +1270,15 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
             continue;
         }
 
+        // BF16 source: the item goes to registers and frees its stage at the
+        // barrier below; an FP8 item is encoded from the stage, half by half
+        uint4 v[kItemChunksPerThread];
+        if (!kFp8) load_half(0, v);
+
         // ---- encode item: wait (bounded) for the instance's amax
         const FlowGroup& G = t.g[it.g];
         if (tid == kQueueThread) {
-            items[ahead] = flow_item(t, I, total, pend, hint);
+            items[ahead] = flow_item(t, I, total, pend, hint, kChunks);
             pend = next_q;
         }
         if (tid == 0) {
@@ -1284,8 +1298,8 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
             }
             s_amax[k & 1u] = known_amax;
         }
-        __syncthreads();   // stage st is free; the amax and the new item are published
-        if (tid == 0) {
+        __syncthreads();   // the amax and the new item are published (BF16: stage st is free)
+        if (!kFp8 && tid == 0) {
             const FlowItem& nx = items[ahead];
             if (nx.valid)
                 flow_stage(t.m[nx.m], nx, stage0 + st * kFlowStageBytes, smem_addr(&bars[st]),
@@ -1306,10 +1320,30 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
             if (G.gs_out) G.gs_out[it.b] = gs;
             if (G.amax_out) G.amax_out[it.b] = __uint_as_float(s_amax[k & 1u]);
         }
-        if (all_fast && full)
-            flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
-        else
-            flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
+        if (!kFp8) {
+            if (all_fast && full)
+                flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
+            else
+                flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
+        } else {
+#pragma unroll 1
+            for (int h = 0; h < kHalves; ++h) {
+                load_half(h, v);
+                if (all_fast && full)
+                    flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream,
+                                                   (uint32_t)h * kItemChunks);
+                else
+                    flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream,
+                                                     (uint32_t)h * kItemChunks);
+            }
+            __syncthreads();   // stage st is free
+            if (tid == 0) {
+                const FlowItem& nx = items[ahead];
+                if (nx.valid)
+                    flow_stage(t.m[nx.m], nx, stage0 + st * kFlowStageBytes, smem_addr(&bars[st]),
+                               flow_amax_policy(t, nx, keep, stream));
+            }
+        }
     }
 }
 
@@ -1643,6 +1677,7 @@ size_t nvfp4_flow_timeout_selftest_bytes(int64_t instances) {
 cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, void* workspace, cudaStream_t s,
                               uint64_t wait_ns, bool wait_on_idle_counts) {
     const bool fp8 = n_groups > 0 && groups[0].ts != nullptr;   // every group of a call has the same source
+    const uint32_t item_chunks = fp8 ? kItemChunksFp8 : kItemChunks;
     uint32_t* words = static_cast<uint32_t*>(workspace);
     const uint64_t kMaxItems = uint64_t(1) << 30;   // queue positions (2 per item) stay 32-bit
     FlowArgs a;
@@ -1691,7 +1726,7 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
         const int64_t B = G.x[0].batch;
         uint32_t items = 0;
         for (int i = 0; i < G.n; ++i)
-            items += (uint32_t)((G.x[i].rows * (G.x[i].cols / 8) + kItemChunks - 1) / kItemChunks);
+            items += (uint32_t)((G.x[i].rows * (G.x[i].cols / 8) + item_chunks - 1) / item_chunks);
         if (items == 0 || B == 0) continue;
         for (int64_t b0 = 0; b0 < B;) {
             const int64_t room_inst = kFlowMaxInst - (int64_t)a.n_inst;
@@ -1739,7 +1774,7 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
                 M.ts_bs = (int64_t)((x.rows + 127) / 128) * M.tn;
                 M.ts = fp8 ? G.ts[i] + b0 * M.ts_bs : nullptr;
                 M.item_off = off;
-                off += (M.chunks + kItemChunks - 1) / kItemChunks;
+                off += (M.chunks + item_chunks - 1) / item_chunks;
                 M.vec32_o = (uintptr_t)M.out % 32 == 0 && o.rstride % 32 == 0 &&
                             (take == 1 || o.bstride % 32 == 0);
             }
