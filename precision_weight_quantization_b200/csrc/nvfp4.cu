@@ -740,8 +740,10 @@ __global__ void __launch_bounds__(kThreads) nvfp4_dequant_kernel(const __grid_co
 //
 // One launch covers up to kMaxLaunchTensors members in up to as many sibling
 // groups, every batch index of a group being one "instance" with its own
-// amax.  The work is a queue of items of kItemChunks chunks of one member's
-// batch slab: amax items A(i, k) and encode items E(i, k) of instance i.  The
+// amax.  The work is a queue of items of one member's batch slab -- 32 KB of
+// data, one stage: kItemChunks chunks of BF16, or kItemChunksFp8 chunks of
+// E4M3 codes for an FP8 block-wise source, worked in two halves -- amax
+// items A(i, k) and encode items E(i, k) of instance i.  The
 // encode items of instance i follow its amax items after a lead of L amax
 // items of instance i+1 (the order is set out at flow_decode), so that they
 // re-read the instance while it is still in L2, and a CTA that takes one
