@@ -241,3 +241,15 @@ def test_4over6_dsv3_experts_full_size(P):
                 assert np.array_equal(u8(packed[g][i][e])[rows], opk), (g, e, i)
                 assert np.array_equal(u8(sb[g][i][e])[rows], osb), (g, e, i)
                 assert np.array_equal(u16(fq[g][i][e][rows]), O.nvfp4_4over6_fake_quant(x[rows], A, 256)), (g, e, i)
+
+
+def test_4over6_w4_worked_example_on_gpu(P):
+    from test_oracle_4over6 import read_w4, _bf16_bits
+    w = read_w4()
+    E = int(w["e4m3_max"][0])
+    x = np.array([_bf16_bits(v) for v in w["x"]], np.uint16)[None]
+    packed, sb, gs = P.nvfp4_4over6_quant(gpu(x), e4m3_max=E)
+    assert f32bits(gs)[0] == int(w["global_scale"][0], 16)
+    assert [int(v) for v in u8(sb)[0]] == [int(v, 16) for v in w["sb"]]
+    assert list(u8(packed)[0]) == [int(v, 16) for v in w["packed"]]
+    assert list(u16(P.nvfp4_4over6_fake_quant(gpu(x), e4m3_max=E))[0]) == [_bf16_bits(v) for v in w["y"]]

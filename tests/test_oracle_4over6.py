@@ -19,9 +19,12 @@ is pinned here:
     exactly and keeps 4 (6);
   * reductions: with E = 448, blocks that keep 6 are the plain NVFP4 blocks,
     and no block's error exceeds plain NVFP4's;
-  * symmetries: x -> -x and x, A -> 2^j x, 2^j A.
+  * symmetries: x -> -x and x, A -> 2^j x, 2^j A;
+  * the worked example W4 (tests/golden/w4_nvfp4_4over6.txt), derived by
+    hand from the reading.
 """
 from fractions import Fraction
+import os
 import struct
 
 import numpy as np
@@ -301,3 +304,40 @@ def test_4over6_sibling_group_shares_the_amax():
         assert gs == O.nvfp4_4over6_global_scale(512.0, 256) == np.float32(512.0) / np.float32(1536.0)
         p1, s1, _ = O.nvfp4_4over6_quant(x, A, 256)
         assert np.array_equal(packed, p1) and np.array_equal(sb, s1)
+
+
+# ------------------------------------------------------------------ worked example W4
+
+GOLDEN_W4 = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "w4_nvfp4_4over6.txt")
+
+
+def read_w4():
+    """The fields of tests/golden/w4_nvfp4_4over6.txt as a dict of token lists."""
+    out = {}
+    for line in open(GOLDEN_W4):
+        line = line.split("#")[0].strip()
+        if line:
+            key, *vals = line.split()
+            out[key] = vals
+    return out
+
+
+def test_4over6_w4_worked_example():
+    w = read_w4()
+    E = int(w["e4m3_max"][0])
+    x = np.array([_bf16_bits(v) for v in w["x"]], np.uint16)[None]
+    A = O.amax_bf16(x)
+    assert A == float(w["group_amax"][0])
+    packed, sb, gs, choice, err = O.nvfp4_4over6_quant(x, A, E, details=True)
+    assert int(np.float32(gs).view(np.uint32)) == int(w["global_scale"][0], 16)
+    assert list(choice[0]) == [int(v) for v in w["choice"]]
+    assert list(err[0, :, 0]) == [float(v) for v in w["err6"]]
+    assert list(err[0, :, 1]) == [float(v) for v in w["err4"]]
+    assert [int(v) for v in sb[0]] == [int(v, 16) for v in w["sb"]]
+    assert list(O.unpack_e2m1(packed)[0]) == [int(v, 16) for v in w["codes"]]
+    assert list(packed[0]) == [int(v, 16) for v in w["packed"]]
+    assert list(O.nvfp4_4over6_fake_quant(x, A, E)[0]) == [_bf16_bits(v) for v in w["y"]]
+    # and the exact-rational restatement agrees
+    egs, eouts = ex_4over6([x], E)
+    assert egs == int(w["global_scale"][0], 16)
+    assert list(eouts[0][2][0]) == [int(v) for v in w["choice"]]
