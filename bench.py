@@ -639,7 +639,8 @@ def next_calls(op, layers, buf, P, torch, per_call=1):
     """One grouped call per `per_call` layers (their tensors; for NVFP4 their
     sibling groups in one single-pass launch), reading the FP8 codes and
     scales the sweep wrote; every layer writes its own outputs (no call
-    writes over lines a previous call left in L2)."""
+    writes over lines a previous call left in L2).  Returns the calls and
+    their outputs per layer."""
     import workloads as W
     lay0 = layers[0]
     dev = lay0["q_proj"].device
@@ -684,7 +685,7 @@ def next_calls(op, layers, buf, P, torch, per_call=1):
                          so=[[sb[i][n] for n in G[j]] for i, k, j in gts],
                          gso=[gsc[i][j] for i, k, j in gts]:
                          P.fp8_block_requant_nvfp4_grouped(gq, gs, out=o, sb=so, global_scale=gso))
-    return calls
+    return calls, {"q": out_q, "s": out_s, "e": out_e, "pk": pk, "sb": sb, "gs": gsc, "codes": general}
 
 
 # NVFP4 "4over6" (E4M3 maximum 256) of the BF16 sweep, one grouped call per
@@ -696,9 +697,10 @@ FOUR_SIX_ONE_PASS_BYTES_PER_ELEM = {"nvfp4_4over6_quant": 2 + 0.5 + 1 / 16, "nvf
 
 
 def four_six_calls(op, layers, P, torch, per_call=1):
-    """One grouped call per `per_call` layers, every layer writing its own outputs."""
+    """One grouped call per `per_call` layers, every layer writing its own
+    outputs.  Returns the calls and, per call, its groups and outputs."""
     import workloads as W
-    calls = []
+    calls, outs = [], []
     for i0 in range(0, len(layers), per_call):
         groups = [[lay[n] for n in grp] for lay in layers[i0:i0 + per_call] for grp in W.QWEN3_4B_GROUPS]
         dev = groups[0][0].device
@@ -709,10 +711,12 @@ def four_six_calls(op, layers, P, torch, per_call=1):
             gs = [torch.empty(1, dtype=torch.float32, device=dev) for _ in groups]
             calls.append(lambda groups=groups, pk=pk, sb=sb, gs=gs:
                          P.nvfp4_4over6_quant_grouped(groups, 256, out=pk, sb=sb, global_scale=gs))
+            outs.append((groups, pk, sb, gs))
         else:
             ys = [[torch.empty_like(x) for x in g] for g in groups]
             calls.append(lambda groups=groups, ys=ys: P.nvfp4_4over6_fake_quant_grouped(groups, 256, out=ys))
-    return calls
+            outs.append((groups, ys))
+    return calls, outs
 
 
 def time_next_rows(args, w, P, torch, hbm_peak, peak_kind):
@@ -729,9 +733,9 @@ def time_next_rows(args, w, P, torch, hbm_peak, peak_kind):
     one_pass.update(FOUR_SIX_ONE_PASS_BYTES_PER_ELEM)
     for op, bpe in ops.items():
         if op in FOUR_SIX_BYTES_PER_ELEM:
-            calls = four_six_calls(op, layers, P, torch, w.tensors["per_call"])
+            calls, _ = four_six_calls(op, layers, P, torch, w.tensors["per_call"])
         else:
-            calls = next_calls(op, layers, buf, P, torch, w.tensors["per_call"])
+            calls, _ = next_calls(op, layers, buf, P, torch, w.tensors["per_call"])
         g = capture(calls, torch)
         for _ in range(args.warmup):
             g.replay()

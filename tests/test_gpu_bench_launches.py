@@ -6,7 +6,8 @@ groups, batch slabs, instances per single-pass launch -- is the timed one):
     grouped launch per op; NVFP4 with 512 instances in one single-pass
     launch) and the W4A4 activation, at full size, sampled;
   - the Qwen3-4B sweep's grouped calls over two layers (14 tensors, 8
-    sibling groups in one launch), sampled, group amax exact;
+    sibling groups in one launch), sampled, group amax exact, and the
+    next-row launches on them (FP8 block-wise -> NVFP4, NVFP4 4over6);
   - the Qwen3-30B-A3B expert layer's MXFP8 call on layers 0, 47 and 8
     random layers, sampled;
   - the 2048-hidden QAT block's single launch over three sibling groups,
@@ -177,6 +178,55 @@ def test_qwen3_4b_two_layer_grouped_launches(P):
                 rows = sample_rows(rng, lay[n].shape[0], 16)
                 assert np.array_equal(u16(buf.y[i][n][rows]), O.nvfp4_fake_quant(u16(lay[n][rows]), amax[i, g])), \
                     (i, n)
+    torch.cuda.synchronize()
+    assert P.device_error() == 0
+
+
+def test_qwen3_4b_next_rows_launches(P):
+    """bench.py's next-row launches over two Qwen3-4B layers: the FP8
+    block-wise -> NVFP4 single pass over the sweep's FP8 outputs (14 members,
+    8 sibling groups in one launch) and the NVFP4 4over6 grouped calls;
+    group amax and global scales exact, sampled rows against the oracle."""
+    w = bench.qwen3_4b_workload(P, T, DEV, rank=0, layers=2, per_call=2)
+    layers, buf = w.tensors["layers"], w.tensors["buf"]
+    ops = {op.name: op for op in w.ops}
+    ops["fp8_block_quant"].run()          # the FP8 codes and tile scales the rows read
+    rng = np.random.default_rng(77)
+    calls, out = bench.next_calls("fp8_block_requant_nvfp4", layers, buf, P, T, 2)
+    assert len(calls) == 1
+    calls[0]()
+    for i, lay in enumerate(layers):
+        for j, g in enumerate(W.QWEN3_4B_GROUPS):
+            # the dequantised members, from the oracle's threaded driver
+            ys = [PO.fp8_block_dequant(u8(buf.fp8[i][n][0]), buf.fp8[i][n][1].cpu().numpy()) for n in g]
+            A = PO.nvfp4_group_amax(ys)
+            assert f32bits(out["gs"][i][j])[0] == np.float32(O.nvfp4_global_scale(A)).view(np.uint32), (i, g)
+            for n, y in zip(g, ys):
+                rows = sample_rows(rng, y.shape[0], 12)
+                opk, osb, _ = O.nvfp4_quant(y[rows], A)
+                assert np.array_equal(u8(out["pk"][i][n][rows]), opk), (i, n)
+                assert np.array_equal(u8(out["sb"][i][n])[rows], osb), (i, n)
+    for op in ("nvfp4_4over6_quant", "nvfp4_4over6_fake_quant"):
+        calls, outs = bench.four_six_calls(op, layers, P, T, 2)
+        assert len(calls) == 1
+        calls[0]()
+        groups = outs[0][0]
+        assert len(groups) == 8 and sum(len(g) for g in groups) == 14
+        for gi, grp in enumerate(groups):
+            xb = [u16(x) for x in grp]
+            A = PO.nvfp4_group_amax(xb)
+            if op == "nvfp4_4over6_quant":
+                _, pk, sb, gs = outs[0]
+                assert f32bits(gs[gi])[0] == np.float32(O.nvfp4_4over6_global_scale(A, 256)).view(np.uint32), gi
+            for mi, x in enumerate(xb):
+                rows = sample_rows(rng, x.shape[0], 12)
+                if op == "nvfp4_4over6_quant":
+                    opk, osb, _ = O.nvfp4_4over6_quant(x[rows], A, 256)
+                    assert np.array_equal(u8(pk[gi][mi])[rows], opk), (gi, mi)
+                    assert np.array_equal(u8(sb[gi][mi])[rows], osb), (gi, mi)
+                else:
+                    ys = outs[0][1]
+                    assert np.array_equal(u16(ys[gi][mi][rows]), O.nvfp4_4over6_fake_quant(x[rows], A, 256)), (gi, mi)
     torch.cuda.synchronize()
     assert P.device_error() == 0
 
