@@ -356,6 +356,9 @@ pwq_status nvfp4_fake_quant_grouped(int n_groups, const int* group_sizes, const 
  *     (each call clears the words it needs before using them), so calls
  *     that may overlap on the GPU -- on different streams without ordering
  *     between them, or from several host threads -- race: order them;
+ *   - a call whose every group has at most 131072 elements runs one
+ *     thread-block cluster per group (the path nvfp4_fake_quant takes for
+ *     such calls) and does not touch the array, so such calls do not race;
  *   - it calls no cudaMalloc, cudaFree or other allocating routine.
  * Errors as nvfp4_fake_quant, except that there is no PWQ_ERR_WORKSPACE. */
 pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, int n_siblings,

@@ -780,6 +780,16 @@ pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, in
         for (int i = 0; i < n_siblings; ++i)
             if (overlaps(ey[i], ex[n_siblings])) return fail(PWQ_ERR_OVERLAP, "y overlaps amax_in");
     cudaStream_t s = (cudaStream_t)stream;
+    // every instance small: one cluster each, the static scratch untouched
+    pwq::NvGroup ng;
+    ng.x = vx;
+    ng.out = vy;
+    ng.sb = nullptr;
+    ng.n = n_siblings;
+    ng.amax_in = amax_in;
+    ng.gs_out = nullptr;
+    ng.amax_out = amax_out;
+    if (pwq::nvfp4_cluster_ok(&ng, 1)) return from_cuda(pwq::launch_nvfp4_cluster(&ng, 1, true, s));
     uint32_t* amax_bits = nullptr;
     if (!amax_in) {
         cudaError_t e = pwq::static_amax_scratch(&amax_bits);

@@ -21,7 +21,13 @@ import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def test_noalloc_entry_point_matches_workspace_entry_point_twice():
+# (rows of the two siblings): small groups run one cluster each and leave the
+# static scratch alone; larger ones (more than 131072 elements) use it
+SHAPES = {"cluster": (64, 32), "scratch": (300, 100)}
+
+
+@pytest.mark.parametrize("path", list(SHAPES))
+def test_noalloc_entry_point_matches_workspace_entry_point_twice(path):
     import precision_weight_quantization_b200 as P
     from precision_weight_quantization_b200._lib import PwqTensor, lib
 
@@ -33,8 +39,9 @@ def test_noalloc_entry_point_matches_workspace_entry_point_twice():
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     for call, (seed, std) in enumerate(((11, 40.0), (12, 0.003))):
         # a batched sibling pair: 3 groups, each {x0[b], x1[b]}
-        xs = [W.random_bf16((3, 64, 512), seed=seed, std=std, device=dev),
-              W.random_bf16((3, 32, 512), seed=seed + 100, std=std, device=dev)]
+        m0, m1 = SHAPES[path]
+        xs = [W.random_bf16((3, m0, 512), seed=seed, std=std, device=dev),
+              W.random_bf16((3, m1, 512), seed=seed + 100, std=std, device=dev)]
         ys = [guard.empty(x.shape, torch.bfloat16) for x in xs]
         amax_out = guard.empty((3,), torch.float32)
         ax = (PwqTensor * 2)(*[P._desc(x, "x") for x in xs])
