@@ -34,8 +34,9 @@ Qwen3-30B-A3B expert layer (128 experts, MXFP8, one call per layer over 48
 layers), the 2048-hidden QAT block (NVFP4 fake-quant of its sibling groups
 in one launch) and the two parts of the headline.  Workloads smaller than
 L2 are timed call by call with a 256 MB write between calls (L2 flushed).
-`next_rows` times the FP8 block-wise re-quantisation ops and the NVFP4
-"4over6" variant on the Qwen3-4B sweep.  `--impl reference` times the CPU oracle (all host threads) on a
+`next_rows` times the FP8 block-wise re-quantisation ops, the NVFP4
+"4over6" variant and NVFP4 with a given group amax on the Qwen3-4B sweep,
+and the W4A4 activation observer on the headline's activation shape.  `--impl reference` times the CPU oracle (all host threads) on a
 bounded sample of the headline workload.
 """
 import argparse
@@ -719,45 +720,98 @@ def four_six_calls(op, layers, P, torch, per_call=1):
     return calls, outs
 
 
+# NVFP4 with the group amax given (the path of a sibling group sharded over
+# data-parallel ranks, after the all-reduce of its amax): one call per
+# sibling group of the sweep, each with its amax computed before timing; one
+# read of the input.  The W4A4 activation observer: observe the activation
+# (one read), then fake-quantise it with the observed amax.
+AMAX_IN_BYTES_PER_ELEM = {"nvfp4_quant_amax_in": 2 + 0.5 + 1 / 16, "nvfp4_fake_quant_amax_in": 2 + 2}
+OBSERVER_BYTES_PER_ELEM = 2 + 2 + 2
+OBSERVER_ONE_PASS_BYTES_PER_ELEM = 2 + 2
+
+
+def amax_in_calls(op, layers, P, torch):
+    """One call per sibling group of every layer, with its precomputed amax."""
+    import workloads as W
+    calls = []
+    for lay in layers:
+        for grp in W.QWEN3_4B_GROUPS:
+            xs = [lay[n] for n in grp]
+            dev = xs[0].device
+            amax = P.nvfp4_group_amax(xs)
+            if op == "nvfp4_quant_amax_in":
+                pk = [torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=dev) for x in xs]
+                sb = [torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.float8_e4m3fn, device=dev) for x in xs]
+                gs = torch.empty(1, dtype=torch.float32, device=dev)
+                calls.append(lambda xs=xs, amax=amax, pk=pk, sb=sb, gs=gs:
+                             P.nvfp4_quant(xs, amax=amax, out=pk, sb=sb, global_scale=gs))
+            else:
+                ys = [torch.empty_like(x) for x in xs]
+                calls.append(lambda xs=xs, amax=amax, ys=ys: P.nvfp4_fake_quant(xs, amax=amax, out=ys))
+    return calls
+
+
+def time_graph(calls, args, torch):
+    """ms per replay of one CUDA graph of `calls` (warm-up replays first)."""
+    stream = torch.cuda.current_stream()
+    g = capture(calls, torch)
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    n = max(1, min(args.steps, 10))
+    a.record(stream)
+    for _ in range(n):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / n
+
+
+def row_entry(ms, elems, bpe, one_pass, launches, hbm_peak, peak_kind):
+    gbs = elems * bpe / (ms / 1e3) / 1e9
+    e = {"ms": round(ms, 4), "elem_per_s": elems / (ms / 1e3), "alg_gbs": round(gbs, 1),
+         "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "launches": launches,
+         "bytes_per_elem": round(bpe, 5)}
+    if one_pass is not None:
+        g1 = elems * one_pass / (ms / 1e3) / 1e9
+        e.update({"alg_gbs_one_pass": round(g1, 1), "frac_of_%s_hbm_one_pass" % peak_kind: round(g1 / hbm_peak, 4)})
+    return e
+
+
 def time_next_rows(args, w, P, torch, hbm_peak, peak_kind):
-    """Device time of each re-quantisation op, and of the NVFP4 4over6
-    variant, over the Qwen3-4B sweep (each its own CUDA graph, replayed after
-    the sweep's timing)."""
+    """Device time of each re-quantisation op, of the NVFP4 4over6 variant
+    and of NVFP4 with a given amax over the Qwen3-4B sweep, and of the W4A4
+    activation observer (each its own CUDA graph, replayed after the sweep's
+    timing)."""
+    import workloads as W
     layers, buf = w.tensors["layers"], w.tensors["buf"]
     elems = layer_elems() * len(layers)
-    stream = torch.cuda.current_stream()
     out = {}
-    ops = dict(NEXT_BYTES_PER_ELEM)
-    ops.update(FOUR_SIX_BYTES_PER_ELEM)
     one_pass = dict(NEXT_ONE_PASS_BYTES_PER_ELEM)
     one_pass.update(FOUR_SIX_ONE_PASS_BYTES_PER_ELEM)
-    for op, bpe in ops.items():
-        if op in FOUR_SIX_BYTES_PER_ELEM:
-            calls, _ = four_six_calls(op, layers, P, torch, w.tensors["per_call"])
-        else:
-            calls, _ = next_calls(op, layers, buf, P, torch, w.tensors["per_call"])
-        g = capture(calls, torch)
-        for _ in range(args.warmup):
-            g.replay()
-        torch.cuda.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        n = max(1, min(args.steps, 10))
-        a.record(stream)
-        for _ in range(n):
-            g.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / n
-        gbs = elems * bpe / (ms / 1e3) / 1e9
-        out[op] = {"ms": round(ms, 4), "elem_per_s": elems / (ms / 1e3), "alg_gbs": round(gbs, 1),
-                   "frac_of_%s_hbm" % peak_kind: round(gbs / hbm_peak, 4), "launches": len(calls) * (2 if op in FOUR_SIX_BYTES_PER_ELEM else 1),
-                   "bytes_per_elem": round(bpe, 5)}
-        if op in one_pass:
-            g1 = elems * one_pass[op] / (ms / 1e3) / 1e9
-            out[op].update({"alg_gbs_one_pass": round(g1, 1),
-                            "frac_of_%s_hbm_one_pass" % peak_kind: round(g1 / hbm_peak, 4)})
-        del g
+    for op, bpe in NEXT_BYTES_PER_ELEM.items():
+        calls, _ = next_calls(op, layers, buf, P, torch, w.tensors["per_call"])
+        out[op] = row_entry(time_graph(calls, args, torch), elems, bpe, one_pass.get(op), len(calls), hbm_peak,
+                            peak_kind)
+    for op, bpe in FOUR_SIX_BYTES_PER_ELEM.items():
+        calls, _ = four_six_calls(op, layers, P, torch, w.tensors["per_call"])
+        out[op] = row_entry(time_graph(calls, args, torch), elems, bpe, one_pass.get(op), 2 * len(calls), hbm_peak,
+                            peak_kind)
+    for op, bpe in AMAX_IN_BYTES_PER_ELEM.items():
+        calls = amax_in_calls(op, layers, P, torch)
+        out[op] = row_entry(time_graph(calls, args, torch), elems, bpe, None, len(calls), hbm_peak, peak_kind)
+    # the W4A4 activation observer (static_minmax) on the 16384 x 7168 activation
+    x = W.dsv3_activation(device=layers[0]["q_proj"].device)
+    y = torch.empty_like(x)
+    obs = P.NVFP4ActivationObserver("static_minmax", device=x.device)
+    ms = time_graph([lambda: obs.fake_quant(x, out=y)], args, torch)
+    out["nvfp4_w4a4_observer_fake_quant"] = row_entry(ms, x.numel(), OBSERVER_BYTES_PER_ELEM,
+                                                      OBSERVER_ONE_PASS_BYTES_PER_ELEM, 3, hbm_peak, peak_kind)
+    out["nvfp4_w4a4_observer_fake_quant"]["workload"] = "16384x7168 activation, observe (2 launches) + fake-quantise"
+    del x, y
     return out
 
 

@@ -9,18 +9,17 @@
 // Quantise and fake-quantise run as one single-pass launch per call
 // (nvfp4_flow_kernel, described at its queue below): amax items and encode
 // items of every group of the call share one work queue, and an encode
-// item re-reads its data while it is still in L2.  Two stream-ordered
-// launches serve the calls whose amax is given (amax_in), the entry point
-// without allocation, and nvfp4_group_amax:
-//   1. amax: every CTA reduces a slice of one group to a max and publishes
-//      it with one atomicMax on the group's word (the float bit patterns of
-//      non-negative values order like unsigned integers);
-//   2. encode: every CTA reads its group's amax, forms the global scale and
-//      quantises 16-element blocks held by lane pairs (8 elements, one
-//      128-bit load each, amax combined with one shuffle).  It walks the
-//      tensor in the reverse order of pass 1 so that the most recently read
-//      data -- still in the 126 MB L2 -- is consumed first.
-// Every kernel also takes an FP8 block-wise source (E4M3 codes with tile
+// item re-reads its data while it is still in L2.  Calls whose every
+// instance is small run one thread-block cluster per instance instead
+// (nvfp4_cluster_kernel).  Calls whose amax is given (amax_in, or the words
+// of an amax launch: the entry point without allocation) run one streaming
+// encode over the blocks of all their instances (nvfp4_units_kernel); the
+// group amax alone (nvfp4_group_amax) is nvfp4_amax_kernel: every CTA
+// reduces a slice of one group to a max and publishes it with one atomicMax
+// on the group's word (the float bit patterns of non-negative values order
+// like unsigned integers).  The NVFP4 "4over6" variant has its own pair of
+// kernels over the same block space.
+// The kernels also take an FP8 block-wise source (E4M3 codes with tile
 // scales, dequantised in registers) for the re-quantisation calls.
 // Dequantise is a grouped walk over 16-element blocks (8 packed bytes and a
 // block-scale byte in, 32 bytes of BF16 out), eight blocks per lane in
@@ -61,6 +60,7 @@ struct Sib {
     uint32_t chunks;      // 8-element chunks per batch slab (M * N / 8)
     FastDiv cpr;          // chunks per row (N / 8)
     int dense_x, dense_o; // slab rows are contiguous
+    int vec16_x;          // FP8 source: every block's 16 codes start on a 16-byte boundary
 };
 
 struct AmaxArgs {
@@ -144,15 +144,6 @@ __global__ void __launch_bounds__(kThreads) nvfp4_amax_kernel(const AmaxArgs a) 
     if (threadIdx.x == 0 && m != 0u) atomicMax(a.amax_bits + b, m << 16);
 }
 
-struct EncodeArgs {
-    Sib s[kMaxSib];
-    int n;
-    const uint32_t* amax_bits;  // [B] or null
-    const float* amax_in;       // [B] or null (takes precedence)
-    float* gs_out;              // [B] or null
-    float* amax_out;            // [B] or null
-};
-
 // Per-group constants of the encode pass, for every E4M3 block-scale code
 // k: d_k = fl(dec(k) * gs) (the code divisor), r_k = RN(1/d_k) when d_k is
 // in the reciprocal path's range (else 0: IEEE division), and dec(k).
@@ -177,89 +168,6 @@ __device__ __forceinline__ uint32_t codes_half(uint4 v, float d, float r) {
         quotients8<false>(v, d, r, q);
     return e2m1x2(q[0], q[1]) | (e2m1x2(q[2], q[3]) << 8) | (e2m1x2(q[4], q[5]) << 16) |
            (e2m1x2(q[6], q[7]) << 24);
-}
-
-template <bool kFake, bool kFp8>
-__global__ void __launch_bounds__(kThreads) nvfp4_encode_kernel(const EncodeArgs a) {
-    __shared__ ScaleTable tab;
-    const uint32_t b = blockIdx.y;
-    const float A = a.amax_in ? a.amax_in[b] : __uint_as_float(a.amax_bits[b]);
-    const float gs = __fdiv_rn(A, 2688.0f);
-    const float six_gs = __fmul_rn(6.0f, gs);
-    const float r6 = __frcp_rn(six_gs);
-    const bool fast6 = div_fast_ok(six_gs);
-    fill_scale_table(tab, gs);
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        if (a.gs_out) a.gs_out[b] = gs;
-        if (a.amax_out) a.amax_out[b] = A;
-    }
-    __syncthreads();
-    const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-    // Reverse order: last sibling first, each walked from its end.
-    for (int i = a.n - 1; i >= 0; --i) {
-        const Sib& S = a.s[i];
-        const char* xb = S.x + (int64_t)b * S.x_bs;
-        const float* tsb = kFp8 ? S.ts + (int64_t)b * S.ts_bs : nullptr;
-        char* ob = S.out + (int64_t)b * S.o_bs;
-        uint8_t* sbb = kFake ? nullptr : S.sb + (int64_t)b * (S.chunks >> 1);
-        for (uint32_t base = gwarp * 32u * kUnroll; base < S.chunks; base += nwarps * 32u * kUnroll) {
-            uint4 v[kUnroll];
-            uint32_t cc[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const uint32_t j = base + u * 32u + lane;
-                // lanes 2k and 2k+1 take the high and low halves of one block
-                cc[u] = S.chunks - 1u - j;
-                v[u] = make_uint4(0u, 0u, 0u, 0u);
-                if (kFp8) {
-                    if (j < S.chunks) {
-                        float sc;
-                        const uint2 codes = fp8_chunk(S, xb, tsb, cc[u], sc);
-                        v[u] = fp8_dequant8(codes, sc);
-                    }
-                } else if (j < S.chunks) {
-                    int64_t off;
-                    if (S.dense_x) {
-                        off = (int64_t)cc[u] * 16;
-                    } else {
-                        const uint32_t r = fdiv(cc[u], S.cpr);
-                        off = (int64_t)r * S.x_rs + (int64_t)(cc[u] - r * S.cpr.d) * 16;
-                    }
-                    v[u] = ld_stream_v4(xb + off);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const uint32_t j = base + u * 32u + lane;
-                uint32_t m = amax_bits8(v[u]);
-                m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-                // block scale sb = e4m3(fl(amax_b / fl(6 gs)))
-                const float amax_b = __uint_as_float(m << 16);
-                const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
-                const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0 (a NaN ratio, outside the contract, stays in the table)
-                const float4 e = tab.e[sb];
-                const uint32_t codes = codes_half(v[u], e.x, e.y);
-                if (j < S.chunks) {
-                    const uint32_t c = cc[u];
-                    int64_t oo;
-                    if (S.dense_o) {
-                        oo = (int64_t)c * (kFake ? 16 : 4);
-                    } else {
-                        const uint32_t r = fdiv(c, S.cpr);
-                        oo = (int64_t)r * S.o_rs + (int64_t)(c - r * S.cpr.d) * (kFake ? 16 : 4);
-                    }
-                    if (kFake) {
-                        st_v4(ob + oo, dequant_half(codes, e.z, gs));
-                    } else {
-                        st_u32(ob + oo, codes);
-                        if ((c & 1u) == 0u) sbb[c >> 1] = (uint8_t)sb;
-                    }
-                }
-            }
-        }
-    }
 }
 
 // NVFP4 "4over6" (vime pull request #503, NVFP4 QDQ config thread:
@@ -533,6 +441,117 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kern
             } else {
                 st_v2(S.out + ooc, make_uint2(four ? b0 : a0, four ? b1 : a1));   // 8-byte aligned: 2 jc even
                 S.sb[(int64_t)b * (S.chunks >> 1) + jc] = (uint8_t)(four ? sb4 : sb6);
+            }
+        }
+        u = start;
+    }
+}
+
+// ---------------------------------------------------------------- plain NVFP4 with a given amax
+//
+// Quantise / fake-quantise when every instance's amax is known before the
+// launch (amax_in: a cached or all-reduced value; or the words an amax
+// launch has just written): one streaming pass over the unit space of the
+// 4over6 kernels, each persistent CTA walking its contiguous range
+// backwards one instance piece at a time (the scale table belongs to the
+// instance's gs), one thread per 16-element block, the next block's loads
+// issued before the current one is encoded.  kFp8: an FP8 block-wise source
+// whose codes are dequantised in registers, y = bf16(fl(dec(q) s)).
+
+// Block j of member S at batch index b, FP8 block-wise source: its 16 codes
+// (one 16-byte load, or two 8-byte loads for code rows that are only 8-byte
+// aligned) and its tile scale (both chunks of a block lie in one tile).
+__device__ __forceinline__ uint4 unit_fp8_codes(const Sib& S, uint32_t b, uint32_t j, float& s) {
+    const uint32_t c = 2u * j;
+    const uint32_t r = fdiv(c, S.cpr);
+    const uint32_t k = c - r * S.cpr.d;
+    const char* p = S.x + (int64_t)b * S.x_bs + (S.dense_x ? (int64_t)c * 8 : (int64_t)r * S.x_rs + (int64_t)k * 8);
+    s = __ldg(S.ts + (int64_t)b * S.ts_bs + (r >> 7) * S.tn + (k >> 4));
+    if (S.vec16_x) return ld_stream_v4(p);
+    const uint2 c0 = ld_stream_v2(p), c1 = ld_stream_v2(p + 8);
+    return make_uint4(c0.x, c0.y, c1.x, c1.y);
+}
+
+template <bool kFake, bool kFp8>
+__global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_units_kernel(const FourSixArgs a) {
+    __shared__ ScaleTable tab;
+    uint64_t lo, hi;
+    four_six_range(a, lo, hi);
+    for (uint64_t u = hi; u > lo;) {
+        int gi;
+        uint32_t b;
+        uint64_t inst_lo;
+        four_six_locate(a, u - 1, gi, b, inst_lo);
+        const FourSixGroup& G = a.g[gi];
+        const uint64_t start = max(lo, inst_lo);   // this instance's piece of the range: [start, u)
+        const float A = G.amax_in ? G.amax_in[b] : __uint_as_float(a.amax_bits[G.inst0 + b]);
+        const float gs = __fdiv_rn(A, 2688.0f);
+        const float six_gs = __fmul_rn(6.0f, gs);
+        const float r6 = __frcp_rn(six_gs);
+        const bool fast6 = div_fast_ok(six_gs);
+        // every non-zero block scale gives dec(sb) * gs in [2^-9 gs, 448 gs]
+        const bool all_fast = fast6 && __fmul_rn(0x1p-9f, gs) >= 0x1p-64f && __fmul_rn(448.0f, gs) <= 0x1p126f;
+        const uint64_t gs2 = f32x2(gs, gs);
+        __syncthreads();   // the previous piece's table reads are done
+        fill_scale_table(tab, gs);
+        if (start == inst_lo && threadIdx.x == 0) {   // the one CTA that holds the instance's first unit
+            if (G.gs_out) G.gs_out[b] = gs;
+            if (G.amax_out) G.amax_out[b] = A;
+        }
+        __syncthreads();
+        const uint32_t rs = (uint32_t)(start - inst_lo), re = (uint32_t)(u - inst_lo);
+        const uint32_t n = re - rs;
+        int i = 0;
+        int64_t xo = 0, oo = 0;
+        uint4 nlo = make_uint4(0u, 0u, 0u, 0u), nhi = nlo;
+        float nsc = 0.0f;
+        auto fetch = [&](uint32_t r) {
+            i = four_six_member(a, G, r);
+            const uint32_t j = r - a.mblk0[i];
+            four_six_offsets<kFake>(a.m[i], b, j, xo, oo);
+            if (kFp8) {
+                nlo = unit_fp8_codes(a.m[i], b, j, nsc);
+            } else {
+                nlo = ld_stream_v4(a.m[i].x + xo);
+                nhi = ld_stream_v4(a.m[i].x + xo + 16);
+            }
+        };
+        if (threadIdx.x < n) fetch(re - 1u - threadIdx.x);
+        for (uint32_t k = threadIdx.x; k < n; k += kThreads) {
+            uint4 lo4 = nlo, hi4 = nhi;
+            const float sc = nsc;
+            const int ic = i;
+            const int64_t ooc = oo;
+            const uint32_t jc = re - 1u - k - a.mblk0[ic];
+            if (k + kThreads < n) fetch(re - 1u - k - kThreads);
+            if (kFp8) {
+                hi4 = fp8_dequant8(make_uint2(lo4.z, lo4.w), sc);
+                lo4 = fp8_dequant8(make_uint2(lo4.x, lo4.y), sc);
+            }
+            const Sib& S = a.m[ic];
+            const uint32_t mw = hmax_abs(amax_word8(lo4), amax_word8(hi4)) & 0x7fff7fffu;
+            const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
+            const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
+            const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
+            const float4 e = tab.e[sb];
+            uint32_t c0, c1;
+            if (all_fast) {
+                float q[8];
+                quotients8<true>(lo4, e.x, e.y, q);
+                c0 = e2m1x8(q);
+                quotients8<true>(hi4, e.x, e.y, q);
+                c1 = e2m1x8(q);
+            } else {
+                c0 = codes_half(lo4, e.x, e.y);
+                c1 = codes_half(hi4, e.x, e.y);
+            }
+            if (kFake) {
+                const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
+                st_v4(S.out + ooc, dequant_half_h(c0, sb2, gs2));
+                st_v4(S.out + ooc + 16, dequant_half_h(c1, sb2, gs2));
+            } else {
+                st_v2(S.out + ooc, make_uint2(c0, c1));   // 8-byte aligned: 2 jc even
+                S.sb[(int64_t)b * (S.chunks >> 1) + jc] = (uint8_t)sb;
             }
         }
         u = start;
@@ -1394,63 +1413,84 @@ cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStr
     return cudaGetLastError();
 }
 
-cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* const* sb,
-                                bool fake, const uint32_t* amax_bits, const float* amax_in,
-                                float* gs_out, float* amax_out, cudaStream_t s, const float* const* ts) {
-    const int64_t B = x[0].batch;
-    EncodeArgs a{};
-    a.n = n;
-    a.amax_bits = amax_bits;
-    a.amax_in = amax_in;
-    a.gs_out = gs_out;
-    a.amax_out = amax_out;
-    int64_t max_chunks = 0;
-    for (int i = 0; i < n; ++i) {
-        Sib& S = a.s[i];
-        S.x = x[i].ptr;
-        S.x_bs = x[i].bstride;
-        S.x_rs = x[i].rstride;
-        S.out = out[i].ptr;
-        S.o_bs = out[i].bstride;
-        S.o_rs = out[i].rstride;
-        S.sb = fake ? nullptr : sb[i];
-        S.chunks = (uint32_t)(x[i].rows * (x[i].cols / 8));
-        S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x[i].cols / 8));
-        set_source(S, x[i], ts ? ts[i] : nullptr);
-        S.dense_o = dense_rows(out[i], fake ? out[i].cols * 2 : out[i].cols / 2);
-        max_chunks = std::max<int64_t>(max_chunks, S.chunks);
-    }
-    const int64_t span = int64_t(kThreads) * kUnroll;
-    const int64_t total_ctas = (max_chunks + span - 1) / span;
-    const int64_t budget = (int64_t)sm_count(current_device()) * 8;
-    int gx = (int)std::max<int64_t>(1, std::min<int64_t>(total_ctas, (budget + B - 1) / B));
-    dim3 grid(gx, (unsigned)B);
-    if (ts) {
-        if (fake)
-            nvfp4_encode_kernel<true, true><<<grid, kThreads, 0, s>>>(a);
-        else
-            nvfp4_encode_kernel<false, true><<<grid, kThreads, 0, s>>>(a);
-    } else if (fake) {
-        nvfp4_encode_kernel<true, false><<<grid, kThreads, 0, s>>>(a);
-    } else {
-        nvfp4_encode_kernel<false, false><<<grid, kThreads, 0, s>>>(a);
-    }
-    return cudaGetLastError();
-}
-
 size_t nvfp4_4over6_workspace_bytes(int64_t instances) {
     return (size_t)((std::max<int64_t>(1, instances) * 4 + 255) / 256 * 256);
 }
 
+namespace {
+
+// Cuts a list of NVFP4 groups into launches over the unit space (at most
+// kMaxLaunchTensors members and groups each) and calls run(args) for each.
+// Instance words (amax_bits) are numbered across the whole call.
+template <typename Run>
+cudaError_t for_unit_launches(const NvGroup* groups, int n_groups, bool fake, uint32_t* words, float six_e,
+                              Run run) {
+    FourSixArgs a{};
+    uint32_t inst = 0;   // amax words used by earlier groups of the call
+    int n_members = 0;
+    for (int gi = 0; gi < n_groups; ++gi) {
+        const NvGroup& G = groups[gi];
+        if (n_members + G.n > kMaxLaunchTensors || a.n_groups == kMaxLaunchTensors) {
+            cudaError_t e = run(a);
+            if (e != cudaSuccess) return e;
+            a = FourSixArgs{};
+            n_members = 0;
+        }
+        a.amax_bits = words;
+        a.six_e = six_e;
+        FourSixGroup& F = a.g[a.n_groups];
+        F.unit0 = a.total;
+        F.inst0 = inst;
+        F.batch = (uint32_t)G.x[0].batch;
+        F.m0 = n_members;
+        F.nm = G.n;
+        F.amax_in = G.amax_in;
+        F.gs_out = G.gs_out;
+        F.amax_out = G.amax_out;
+        uint64_t units = 0;
+        for (int i = 0; i < G.n; ++i) {
+            Sib& S = a.m[n_members + i];
+            const View& x = G.x[i];
+            const View& o = G.out[i];
+            S.x = x.ptr;
+            S.x_bs = x.bstride;
+            S.x_rs = x.rstride;
+            S.out = o.ptr;
+            S.o_bs = o.bstride;
+            S.o_rs = o.rstride;
+            S.sb = fake ? nullptr : G.sb[i];
+            S.chunks = (uint32_t)(x.rows * (x.cols / 8));
+            S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
+            set_source(S, x, G.ts ? G.ts[i] : nullptr);
+            S.dense_o = dense_rows(o, fake ? o.cols * 2 : o.cols / 2);
+            S.vec16_x = (uintptr_t)x.ptr % 16 == 0 && (x.rows <= 1 || x.rstride % 16 == 0) &&
+                        (x.batch <= 1 || x.bstride % 16 == 0);
+            a.mblk0[n_members + i] = (uint32_t)units;
+            units += S.chunks / 2;
+        }
+        if (units == 0) continue;                               // an empty group: nothing to launch
+        if (units > UINT32_MAX) return cudaErrorInvalidValue;   // more than 2^32 blocks per instance
+        F.units = (uint32_t)units;
+        a.total += units * F.batch;
+        inst += F.batch;
+        n_members += G.n;
+        ++a.n_groups;
+    }
+    return a.n_groups ? run(a) : cudaSuccess;
+}
+
+int unit_grid(const FourSixArgs& a) {
+    const int cap = sm_count(current_device()) * kFourSixCtasPerSm;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(cap, (int64_t)((a.total + kThreads - 1) / kThreads)));
+}
+
+}  // namespace
+
 cudaError_t launch_nvfp4_4over6(const NvGroup* groups, int n_groups, bool fake, int e4m3_max, void* workspace,
                                cudaStream_t s) {
     uint32_t* words = static_cast<uint32_t*>(workspace);
-    const int grid_cap = sm_count(current_device()) * kFourSixCtasPerSm;
-    FourSixArgs a{};
-    uint32_t inst = 0;             // amax words used by earlier groups of the call
-    auto flush = [&]() -> cudaError_t {
-        if (a.n_groups == 0) return cudaSuccess;
-        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(grid_cap, (int64_t)((a.total + kThreads - 1) / kThreads)));
+    return for_unit_launches(groups, n_groups, fake, words, (float)(6 * e4m3_max), [&](const FourSixArgs& a) {
+        const int grid = unit_grid(a);
         bool reduce = false;
         uint32_t w0 = UINT32_MAX, w1 = 0;
         for (int g = 0; g < a.n_groups; ++g)
@@ -1469,60 +1509,24 @@ cudaError_t launch_nvfp4_4over6(const NvGroup* groups, int n_groups, bool fake, 
             nvfp4_4over6_kernel<true><<<grid, kThreads, 0, s>>>(a);
         else
             nvfp4_4over6_kernel<false><<<grid, kThreads, 0, s>>>(a);
-        cudaError_t e = cudaGetLastError();
-        a = FourSixArgs{};
-        return e;
-    };
-    int n_members = 0;
-    for (int gi = 0; gi < n_groups; ++gi) {
-        const NvGroup& G = groups[gi];
-        if (n_members + G.n > kMaxLaunchTensors || a.n_groups == kMaxLaunchTensors) {
-            cudaError_t e = flush();
-            if (e != cudaSuccess) return e;
-            n_members = 0;
-        }
-        if (a.n_groups == 0) {
-            a.amax_bits = words;
-            a.six_e = (float)(6 * e4m3_max);
-        }
-        FourSixGroup& F = a.g[a.n_groups];
-        F.unit0 = a.total;
-        F.inst0 = inst;
-        F.batch = (uint32_t)G.x[0].batch;
-        F.m0 = n_members;
-        F.nm = G.n;
-        F.amax_in = G.amax_in;
-        F.gs_out = G.gs_out;
-        F.amax_out = G.amax_out;
-        uint64_t units = 0;
-        for (int i = 0; i < G.n; ++i) {
-            Sib& S = a.m[n_members + i];
-            const View& x = G.x[i];
-            S.x = x.ptr;
-            S.x_bs = x.bstride;
-            S.x_rs = x.rstride;
-            S.out = G.out[i].ptr;
-            S.o_bs = G.out[i].bstride;
-            S.o_rs = G.out[i].rstride;
-            S.sb = fake ? nullptr : G.sb[i];
-            S.chunks = (uint32_t)(x.rows * (x.cols / 8));
-            S.cpr = make_fastdiv((uint32_t)std::max<int64_t>(1, x.cols / 8));
-            set_source(S, x, nullptr);
-            S.dense_o = dense_rows(G.out[i], fake ? G.out[i].cols * 2 : G.out[i].cols / 2);
-            a.mblk0[n_members + i] = (uint32_t)units;
-            units += S.chunks / 2;
-        }
-        if (units == 0 || units > UINT32_MAX) {
-            if (units > UINT32_MAX) return cudaErrorInvalidValue;   // more than 2^32 blocks per instance
-            continue;                                               // an empty group: nothing to launch
-        }
-        F.units = (uint32_t)units;
-        a.total += units * F.batch;
-        inst += F.batch;
-        n_members += G.n;
-        ++a.n_groups;
-    }
-    return flush();
+        return cudaGetLastError();
+    });
+}
+
+cudaError_t launch_nvfp4_units_encode(const NvGroup* groups, int n_groups, bool fake, const uint32_t* amax_bits,
+                                      cudaStream_t s) {
+    const bool fp8 = n_groups > 0 && groups[0].ts != nullptr;   // every group of a call has the same source
+    return for_unit_launches(groups, n_groups, fake, const_cast<uint32_t*>(amax_bits), 2688.0f,
+                             [&](const FourSixArgs& a) {
+                                 const int grid = unit_grid(a);
+                                 if (fp8)
+                                     nvfp4_units_kernel<false, true><<<grid, kThreads, 0, s>>>(a);
+                                 else if (fake)
+                                     nvfp4_units_kernel<true, false><<<grid, kThreads, 0, s>>>(a);
+                                 else
+                                     nvfp4_units_kernel<false, false><<<grid, kThreads, 0, s>>>(a);
+                                 return cudaGetLastError();
+                             });
 }
 
 bool nvfp4_cluster_ok(const NvGroup* groups, int n_groups) {

@@ -607,11 +607,7 @@ pwq_status nv_run(int n_groups, const int* sizes, const pwq_tensor* x, const pwq
     // every instance small: one cluster each, one launch, the workspace unused
     if (pwq::nvfp4_cluster_ok(launch.data(), (int)launch.size()))
         return from_cuda(pwq::launch_nvfp4_cluster(launch.data(), (int)launch.size(), fake, s));
-    if (amax_in) {
-        const pwq::NvGroup& G = launch[0];
-        return from_cuda(pwq::launch_nvfp4_encode(G.x, G.n, G.out, G.sb, fake, nullptr, amax_in, G.gs_out,
-                                                  G.amax_out, s));
-    }
+    if (amax_in) return from_cuda(pwq::launch_nvfp4_units_encode(launch.data(), 1, fake, nullptr, s));
     return from_cuda(pwq::launch_nvfp4_flow(launch.data(), (int)launch.size(), fake, ws, s));
 }
 
@@ -797,8 +793,7 @@ pwq_status nvfp4_fake_quant_noalloc(const pwq_tensor* x, const pwq_tensor* y, in
         e = pwq::launch_nvfp4_amax(vx, n_siblings, amax_bits, s);  // clears the words first
         if (e != cudaSuccess) return cuda_fail(e);
     }
-    return from_cuda(pwq::launch_nvfp4_encode(vx, n_siblings, vy, nullptr, true, amax_bits, amax_in, nullptr,
-                                              amax_out, s));
+    return from_cuda(pwq::launch_nvfp4_units_encode(&ng, 1, true, amax_bits, s));
 }
 
 // ------------------------------------------------------------------ FP8 block-wise -> rollout formats
@@ -1001,11 +996,7 @@ pwq_status requant_nv_run(int n_groups, const int* sizes, const pwq_tensor* q_in
     pwq_status st = check_requant_overlaps(ins, outs, {});
     if (st != PWQ_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    if (amax_in) {
-        const pwq::NvGroup& G0 = launch[0];
-        return from_cuda(pwq::launch_nvfp4_encode(G0.x, G0.n, G0.out, G0.sb, false, nullptr, amax_in, G0.gs_out,
-                                                  nullptr, s, G0.ts));
-    }
+    if (amax_in) return from_cuda(pwq::launch_nvfp4_units_encode(launch.data(), 1, false, nullptr, s));
     return from_cuda(pwq::launch_nvfp4_flow(launch.data(), (int)launch.size(), false, ws, s));
 }
 

@@ -93,19 +93,13 @@ cudaError_t launch_nvfp4_flow(const NvGroup* groups, int n_groups, bool fake, vo
                               cudaStream_t s, uint64_t wait_ns = kFlowWaitLimitNs,
                               bool wait_on_idle_counts = false);
 
-// Two-launch NVFP4 path for one group set (used with a precomputed amax, by
-// the no-allocation entry point and by the FP8 block re-quantisation).
-// amax_bits: B words holding max |x| of each group as binary32 bits.  With
-// ts non-null the members are E4M3 code views (FP8 block-wise, ts[i] the
-// member's tile scales [B][TM][TN]) and the source values are their
-// dequantised BF16 values.
+// NVFP4 group amax of one group set (nvfp4_group_amax, and the amax launch
+// of the no-allocation entry point): amax_bits receives B words holding
+// max |x| of each group as binary32 bits (cleared first).  With ts non-null
+// the members are E4M3 code views (FP8 block-wise, ts[i] the member's tile
+// scales [B][TM][TN]) and the values are their dequantised BF16 values.
 cudaError_t launch_nvfp4_amax(const View* x, int n, uint32_t* amax_bits, cudaStream_t s,
                               const float* const* ts = nullptr);
-cudaError_t launch_nvfp4_encode(const View* x, int n, const View* out, uint8_t* const* sb,
-                                bool fake, const uint32_t* amax_bits, const float* amax_in,
-                                float* gs_out, float* amax_out, cudaStream_t s,
-                                const float* const* ts = nullptr);
-
 // NVFP4 "4over6" quantise / fake-quantise of sibling groups (launches of up
 // to kMaxLaunchTensors members): the group amax (unless the group has
 // amax_in) and the encode that keeps, per block, the candidate -- amax
@@ -119,6 +113,13 @@ size_t nvfp4_4over6_workspace_bytes(int64_t instances);
 // cluster per instance, one launch, no workspace.  nvfp4_cluster_ok tells
 // whether a call qualifies.
 bool nvfp4_cluster_ok(const NvGroup* groups, int n_groups);
+
+// NVFP4 quantise / fake-quantise of sibling groups whose amax is known before
+// the launch: G.amax_in per group, else amax_bits (one word per instance,
+// numbered across the call).  One streaming launch per kMaxLaunchTensors
+// members; with G.ts set the source is FP8 block-wise (quantise only).
+cudaError_t launch_nvfp4_units_encode(const NvGroup* groups, int n_groups, bool fake, const uint32_t* amax_bits,
+                                      cudaStream_t s);
 cudaError_t launch_nvfp4_cluster(const NvGroup* groups, int n_groups, bool fake, cudaStream_t s);
 cudaError_t launch_nvfp4_4over6(const NvGroup* groups, int n_groups, bool fake, int e4m3_max, void* workspace,
                                cudaStream_t s);
