@@ -61,7 +61,29 @@ struct Sib {
     FastDiv cpr;          // chunks per row (N / 8)
     int dense_x, dense_o; // slab rows are contiguous
     int vec16_x;          // FP8 source: every block's 16 codes start on a 16-byte boundary
+    int vec32_x, vec32_o; // BF16 source / fake-quant output: every block's 32 bytes on a 32-byte boundary
 };
+
+// The 32 bytes of a 16-element BF16 block at byte offset xo of a member's
+// source: one 256-bit load when the member's blocks are 32-byte aligned
+// (the two halves then leave L2 as one request), else two 128-bit loads.
+__device__ __forceinline__ void ld_block32(const Sib& S, int64_t xo, uint4& lo, uint4& hi) {
+    if (S.vec32_x) {
+        ld_nc_v8(S.x + xo, lo, hi);
+    } else {
+        lo = ld_stream_v4(S.x + xo);
+        hi = ld_stream_v4(S.x + xo + 16);
+    }
+}
+// The 32 bytes of a fake-quantised block at byte offset oo of the output.
+__device__ __forceinline__ void st_block32(const Sib& S, int64_t oo, uint4 y0, uint4 y1) {
+    if (S.vec32_o) {
+        st_v8(S.out + oo, y0, y1);
+    } else {
+        st_v4(S.out + oo, y0);
+        st_v4(S.out + oo + 16, y1);
+    }
+}
 
 struct AmaxArgs {
     Sib s[kMaxSib];
@@ -148,14 +170,14 @@ __global__ void __launch_bounds__(kThreads) nvfp4_amax_kernel(const AmaxArgs a) 
 // k: d_k = fl(dec(k) * gs) (the code divisor), r_k = RN(1/d_k) when d_k is
 // in the reciprocal path's range (else 0: IEEE division), and dec(k).
 struct ScaleTable {
-    float4 e[128];
+    float2 e[128];   // {d_k, RN(1 / d_k)}, or {d_k, 0} off the reciprocal path
 };
 
 __device__ __forceinline__ void fill_scale_table(ScaleTable& t, float gs) {
     for (uint32_t k = threadIdx.x; k < 128u; k += blockDim.x) {
         const float dec = e4m3_decode(k);  // k = 0x7f (NaN) is never produced
         const float d = __fmul_rn(dec, gs);
-        t.e[k] = make_float4(d, div_fast_ok(d) ? __frcp_rn(d) : 0.0f, dec, 0.0f);
+        t.e[k] = make_float2(d, div_fast_ok(d) ? __frcp_rn(d) : 0.0f);
     }
 }
 
@@ -308,7 +330,7 @@ __device__ __forceinline__ float four_six_candidate(uint4 lo, uint4 hi, const ui
                                                     uint4& y1) {
     const float ratio = fast_t ? div_fast(amax_b, t_gs, rt) : div_slow(amax_b, t_gs);
     sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
-    const float4 e = tab.e[sb];
+    const float2 e = tab.e[sb];
     if (e.y != 0.0f) {
         const uint64_t d2 = f32x2(e.x, e.x), nr2 = f32x2(-e.y, -e.y);
         c0 = codes_neg8(xl, d2, nr2);
@@ -472,8 +494,9 @@ __device__ __forceinline__ uint4 unit_fp8_codes(const Sib& S, uint32_t b, uint32
     return make_uint4(c0.x, c0.y, c1.x, c1.y);
 }
 
+constexpr int kUnitCtasPerSm = 4;
 template <bool kFake, bool kFp8>
-__global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_units_kernel(const FourSixArgs a) {
+__global__ void __launch_bounds__(kThreads, kUnitCtasPerSm) nvfp4_units_kernel(const FourSixArgs a) {
     __shared__ ScaleTable tab;
     uint64_t lo, hi;
     four_six_range(a, lo, hi);
@@ -512,8 +535,7 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_units_kerne
             if (kFp8) {
                 nlo = unit_fp8_codes(a.m[i], b, j, nsc);
             } else {
-                nlo = ld_stream_v4(a.m[i].x + xo);
-                nhi = ld_stream_v4(a.m[i].x + xo + 16);
+                ld_block32(a.m[i], xo, nlo, nhi);
             }
         };
         if (threadIdx.x < n) fetch(re - 1u - threadIdx.x);
@@ -533,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_units_kerne
             const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
             const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
             const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
-            const float4 e = tab.e[sb];
+            const float2 e = tab.e[sb];
             uint32_t c0, c1;
             if (all_fast) {
                 float q[8];
@@ -547,8 +569,7 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_units_kerne
             }
             if (kFake) {
                 const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
-                st_v4(S.out + ooc, dequant_half_h(c0, sb2, gs2));
-                st_v4(S.out + ooc + 16, dequant_half_h(c1, sb2, gs2));
+                st_block32(S, ooc, dequant_half_h(c0, sb2, gs2), dequant_half_h(c1, sb2, gs2));
             } else {
                 st_v2(S.out + ooc, make_uint2(c0, c1));   // 8-byte aligned: 2 jc even
                 S.sb[(int64_t)b * (S.chunks >> 1) + jc] = (uint8_t)sb;
@@ -604,8 +625,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_cluster_kernel(const FourSixAr
             const int i = four_six_member(a, G, r);
             int64_t xo, oo;
             four_six_offsets<kFake>(a.m[i], b, r - a.mblk0[i], xo, oo);
-            lo[k] = ld_stream_v4(a.m[i].x + xo);
-            hi[k] = ld_stream_v4(a.m[i].x + xo + 16);
+            ld_block32(a.m[i], xo, lo[k], hi[k]);
         }
         m = max(m, max(amax_bits8(lo[k]), amax_bits8(hi[k])));
     }
@@ -656,12 +676,11 @@ __global__ void __launch_bounds__(kThreads) nvfp4_cluster_kernel(const FourSixAr
             const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
             const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
             const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
-            const float4 e = tab.e[sb];
+            const float2 e = tab.e[sb];
             const uint32_t c0 = codes_half(lo[k], e.x, e.y), c1 = codes_half(hi[k], e.x, e.y);
             if (kFake) {
                 const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
-                st_v4(S.out + oo, dequant_half_h(c0, sb2, gs2));
-                st_v4(S.out + oo + 16, dequant_half_h(c1, sb2, gs2));
+                st_block32(S, oo, dequant_half_h(c0, sb2, gs2), dequant_half_h(c1, sb2, gs2));
             } else {
                 st_v2(S.out + oo, make_uint2(c0, c1));   // 8-byte aligned: 2 j even
                 S.sb[(int64_t)b * (S.chunks >> 1) + j] = (uint8_t)sb;
@@ -987,11 +1006,18 @@ __device__ __forceinline__ void flow_stage(const FlowMember& M, const FlowItem& 
     }
 }
 
-// Chunk of an item taken by thread tid at step j: steps 2i and 2i+1 give
-// the two chunks of one 16-element block, so a thread holds whole blocks
-// (no exchange for the block amax, one block scale per 16 elements).
-__device__ __forceinline__ uint32_t flow_lc(int j, uint32_t tid) {
-    return (uint32_t)(j >> 1) * (2u * kFlowThreads) + 2u * tid + (uint32_t)(j & 1);
+// Chunks of an item taken by thread tid: steps 2i and 2i+1 give the two
+// chunks of one 16-element block (first chunk flow_blk(i, tid)), so a thread
+// holds whole blocks (no exchange for the block amax, one block scale per 16
+// elements).  sw = 1 takes the block's second chunk first: a BF16 stage is
+// read with sw = bit 2 of the lane, so that the 8 lanes of each quarter-warp
+// (one shared-memory wavefront of 16-byte loads) cover the 32 banks once --
+// chunks 32 bytes apart in lane order would put two lanes on every bank.
+__device__ __forceinline__ uint32_t flow_blk(int i, uint32_t tid) {
+    return (uint32_t)i * (2u * kFlowThreads) + 2u * tid;
+}
+__device__ __forceinline__ uint32_t flow_lc(int j, uint32_t tid, uint32_t sw) {
+    return flow_blk(j >> 1, tid) + ((uint32_t)(j & 1) ^ sw);
 }
 
 // Encodes the blocks of one item held in registers.  kFast: every block
@@ -1003,7 +1029,7 @@ __device__ __forceinline__ uint32_t flow_lc(int j, uint32_t tid) {
 template <bool kFake, bool kFast, bool kFull>
 __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThread], const FlowItem& it,
                                             const FlowMember& M, const ScaleTable& tab, float gs, float six_gs,
-                                            float r6, bool fast6, uint64_t pol, uint32_t c_off = 0u) {
+                                            float r6, bool fast6, uint64_t pol, uint32_t sw, uint32_t c_off = 0u) {
     const uint32_t tid = threadIdx.x;
     char* ob = M.out + (int64_t)it.b * M.o_bs;
     uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.sf_mma ? M.sf_slab : (int64_t)(M.chunks >> 1));
@@ -1012,7 +1038,7 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
         const uint4 lo = v[2 * i], hi = v[2 * i + 1];
         // c is even (the block's first chunk); rows hold an even number of
         // chunks, so c + 1 is in the same row and c < c1 implies c + 1 < c1
-        const uint32_t c = it.c0 + c_off + flow_lc(2 * i, tid);
+        const uint32_t c = it.c0 + c_off + flow_blk(i, tid);
         const uint32_t mw = hmax_abs(amax_word8(lo), amax_word8(hi)) & 0x7fff7fffu;
         const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
         float ratio;
@@ -1021,7 +1047,7 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
         else
             ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
         const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0 (a NaN ratio, outside the contract, stays in the table)
-        const float4 e = tab.e[sb];
+        const float2 e = tab.e[sb];
         uint32_t c0, c1;
         if (kFast) {
             float q[8];
@@ -1032,6 +1058,11 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
         } else {
             c0 = codes_half(lo, e.x, e.y);
             c1 = codes_half(hi, e.x, e.y);
+        }
+        if (sw) {   // v[2i] held the block's second chunk
+            const uint32_t t = c0;
+            c0 = c1;
+            c1 = t;
         }
         if (kFull || c < it.c1) {
             int64_t oo;
@@ -1110,6 +1141,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
     constexpr uint32_t kChunks = kFp8 ? kItemChunksFp8 : kItemChunks;
     constexpr int kHalves = kFp8 ? 2 : 1;
     const uint32_t tid = threadIdx.x;
+    const uint32_t sw = kFp8 ? 0u : (tid >> 2) & 1u;   // chunk order within a block (flow_lc)
     const uint32_t stage0 = smem_addr(flow_smem);
     const uint32_t I = a.n_inst, L = a.lead, total = a.total_items;
 
@@ -1188,7 +1220,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
                     for (int j = 0; j < kItemChunksPerThread; j += 2) {
                         // lc even: the block's two chunks lie in one row and one
                         // tile, so one row / column step and one tile-scale load
-                        const uint32_t lc = hoff + flow_lc(j, tid);
+                        const uint32_t lc = hoff + flow_blk(j >> 1, tid);
                         const uint4 cc = *reinterpret_cast<const uint4*>(buf + lc * 8u);
                         const uint32_t c = it.c0 + lc;
                         const uint32_t r = fdiv(c, M.cpr);
@@ -1200,13 +1232,13 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
                 } else {
 #pragma unroll
                     for (int j = 0; j < kItemChunksPerThread; ++j)
-                        v[j] = *reinterpret_cast<const uint4*>(buf + flow_lc(j, tid) * 16u);
+                        v[j] = *reinterpret_cast<const uint4*>(buf + flow_lc(j, tid, sw) * 16u);
                 }
             } else {
                 const char* xb = M.x + (int64_t)it.b * M.x_bs;
 #pragma unroll
                 for (int j = 0; j < kItemChunksPerThread; ++j) {
-                    const uint32_t lc = hoff + flow_lc(j, tid);   // chunk within the item
+                    const uint32_t lc = hoff + flow_lc(j, tid, sw);   // chunk within the item
                     const uint32_t c = it.c0 + lc;
                     v[j] = make_uint4(0u, 0u, 0u, 0u);
                     if (c < it.c1) {
@@ -1244,7 +1276,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
                     // |y| of the pair -- without dequantising
 #pragma unroll
                     for (int j = 0; j < kItemChunksPerThread; j += 2) {
-                        const uint32_t lc = (uint32_t)h * kItemChunks + flow_lc(j, tid);
+                        const uint32_t lc = (uint32_t)h * kItemChunks + flow_blk(j >> 1, tid);
                         const uint4 cc = *reinterpret_cast<const uint4*>(buf + lc * 8u);
                         const uint32_t c = it.c0 + lc;
                         const uint32_t r = fdiv(c, M.cpr);
@@ -1343,18 +1375,18 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         }
         if (!kFp8) {
             if (all_fast && full)
-                flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
+                flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream, sw);
             else
-                flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream);
+                flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream, sw);
         } else {
 #pragma unroll 1
             for (int h = 0; h < kHalves; ++h) {
                 load_half(h, v);
                 if (all_fast && full)
-                    flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream,
+                    flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream, sw,
                                                    (uint32_t)h * kItemChunks);
                 else
-                    flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream,
+                    flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream, sw,
                                                      (uint32_t)h * kItemChunks);
             }
             __syncthreads();   // stage st is free
@@ -1465,6 +1497,10 @@ cudaError_t for_unit_launches(const NvGroup* groups, int n_groups, bool fake, ui
             S.dense_o = dense_rows(o, fake ? o.cols * 2 : o.cols / 2);
             S.vec16_x = (uintptr_t)x.ptr % 16 == 0 && (x.rows <= 1 || x.rstride % 16 == 0) &&
                         (x.batch <= 1 || x.bstride % 16 == 0);
+            S.vec32_x = !G.ts && (uintptr_t)x.ptr % 32 == 0 && (x.rows <= 1 || x.rstride % 32 == 0) &&
+                        (x.batch <= 1 || x.bstride % 32 == 0);
+            S.vec32_o = fake && (uintptr_t)o.ptr % 32 == 0 && (o.rows <= 1 || o.rstride % 32 == 0) &&
+                        (o.batch <= 1 || o.bstride % 32 == 0);
             a.mblk0[n_members + i] = (uint32_t)units;
             units += S.chunks / 2;
         }
@@ -1479,8 +1515,8 @@ cudaError_t for_unit_launches(const NvGroup* groups, int n_groups, bool fake, ui
     return a.n_groups ? run(a) : cudaSuccess;
 }
 
-int unit_grid(const FourSixArgs& a) {
-    const int cap = sm_count(current_device()) * kFourSixCtasPerSm;
+int unit_grid(const FourSixArgs& a, int ctas_per_sm = kFourSixCtasPerSm) {
+    const int cap = sm_count(current_device()) * ctas_per_sm;
     return (int)std::max<int64_t>(1, std::min<int64_t>(cap, (int64_t)((a.total + kThreads - 1) / kThreads)));
 }
 
@@ -1518,7 +1554,7 @@ cudaError_t launch_nvfp4_units_encode(const NvGroup* groups, int n_groups, bool 
     const bool fp8 = n_groups > 0 && groups[0].ts != nullptr;   // every group of a call has the same source
     return for_unit_launches(groups, n_groups, fake, const_cast<uint32_t*>(amax_bits), 2688.0f,
                              [&](const FourSixArgs& a) {
-                                 const int grid = unit_grid(a);
+                                 const int grid = unit_grid(a, kUnitCtasPerSm);
                                  if (fp8)
                                      nvfp4_units_kernel<false, true><<<grid, kThreads, 0, s>>>(a);
                                  else if (fake)
