@@ -67,21 +67,21 @@ struct Sib {
 // The 32 bytes of a 16-element BF16 block at byte offset xo of a member's
 // source: one 256-bit load when the member's blocks are 32-byte aligned
 // (the two halves then leave L2 as one request), else two 128-bit loads.
-__device__ __forceinline__ void ld_block32(const Sib& S, int64_t xo, uint4& lo, uint4& hi) {
-    if (S.vec32_x) {
-        ld_nc_v8(S.x + xo, lo, hi);
+__device__ __forceinline__ void ld_block32(const char* p, int vec32, uint4& lo, uint4& hi) {
+    if (vec32) {
+        ld_nc_v8(p, lo, hi);
     } else {
-        lo = ld_stream_v4(S.x + xo);
-        hi = ld_stream_v4(S.x + xo + 16);
+        lo = ld_stream_v4(p);
+        hi = ld_stream_v4(p + 16);
     }
 }
-// The 32 bytes of a fake-quantised block at byte offset oo of the output.
-__device__ __forceinline__ void st_block32(const Sib& S, int64_t oo, uint4 y0, uint4 y1) {
-    if (S.vec32_o) {
-        st_v8(S.out + oo, y0, y1);
+// The 32 bytes of a fake-quantised block at p.
+__device__ __forceinline__ void st_block32(char* p, int vec32, uint4 y0, uint4 y1) {
+    if (vec32) {
+        st_v8(p, y0, y1);
     } else {
-        st_v4(S.out + oo, y0);
-        st_v4(S.out + oo + 16, y1);
+        st_v4(p, y0);
+        st_v4(p + 16, y1);
     }
 }
 
@@ -480,20 +480,6 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kern
 // issued before the current one is encoded.  kFp8: an FP8 block-wise source
 // whose codes are dequantised in registers, y = bf16(fl(dec(q) s)).
 
-// Block j of member S at batch index b, FP8 block-wise source: its 16 codes
-// (one 16-byte load, or two 8-byte loads for code rows that are only 8-byte
-// aligned) and its tile scale (both chunks of a block lie in one tile).
-__device__ __forceinline__ uint4 unit_fp8_codes(const Sib& S, uint32_t b, uint32_t j, float& s) {
-    const uint32_t c = 2u * j;
-    const uint32_t r = fdiv(c, S.cpr);
-    const uint32_t k = c - r * S.cpr.d;
-    const char* p = S.x + (int64_t)b * S.x_bs + (S.dense_x ? (int64_t)c * 8 : (int64_t)r * S.x_rs + (int64_t)k * 8);
-    s = __ldg(S.ts + (int64_t)b * S.ts_bs + (r >> 7) * S.tn + (k >> 4));
-    if (S.vec16_x) return ld_stream_v4(p);
-    const uint2 c0 = ld_stream_v2(p), c1 = ld_stream_v2(p + 8);
-    return make_uint4(c0.x, c0.y, c1.x, c1.y);
-}
-
 constexpr int kUnitCtasPerSm = 4;
 template <bool kFake, bool kFp8>
 __global__ void __launch_bounds__(kThreads, kUnitCtasPerSm) nvfp4_units_kernel(const FourSixArgs a) {
@@ -523,56 +509,87 @@ __global__ void __launch_bounds__(kThreads, kUnitCtasPerSm) nvfp4_units_kernel(c
         }
         __syncthreads();
         const uint32_t rs = (uint32_t)(start - inst_lo), re = (uint32_t)(u - inst_lo);
-        const uint32_t n = re - rs;
-        int i = 0;
-        int64_t xo = 0, oo = 0;
-        uint4 nlo = make_uint4(0u, 0u, 0u, 0u), nhi = nlo;
-        float nsc = 0.0f;
-        auto fetch = [&](uint32_t r) {
-            i = four_six_member(a, G, r);
-            const uint32_t j = r - a.mblk0[i];
-            four_six_offsets<kFake>(a.m[i], b, j, xo, oo);
-            if (kFp8) {
-                nlo = unit_fp8_codes(a.m[i], b, j, nsc);
-            } else {
-                ld_block32(a.m[i], xo, nlo, nhi);
-            }
-        };
-        if (threadIdx.x < n) fetch(re - 1u - threadIdx.x);
-        for (uint32_t k = threadIdx.x; k < n; k += kThreads) {
-            uint4 lo4 = nlo, hi4 = nhi;
-            const float sc = nsc;
-            const int ic = i;
-            const int64_t ooc = oo;
-            const uint32_t jc = re - 1u - k - a.mblk0[ic];
-            if (k + kThreads < n) fetch(re - 1u - k - kThreads);
-            if (kFp8) {
-                hi4 = fp8_dequant8(make_uint2(lo4.z, lo4.w), sc);
-                lo4 = fp8_dequant8(make_uint2(lo4.x, lo4.y), sc);
-            }
-            const Sib& S = a.m[ic];
-            const uint32_t mw = hmax_abs(amax_word8(lo4), amax_word8(hi4)) & 0x7fff7fffu;
-            const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
-            const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
-            const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
-            const float2 e = tab.e[sb];
-            uint32_t c0, c1;
-            if (all_fast) {
-                float q[8];
-                quotients8<true>(lo4, e.x, e.y, q);
-                c0 = e2m1x8(q);
-                quotients8<true>(hi4, e.x, e.y, q);
-                c1 = e2m1x8(q);
-            } else {
-                c0 = codes_half(lo4, e.x, e.y);
-                c1 = codes_half(hi4, e.x, e.y);
-            }
-            if (kFake) {
-                const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
-                st_block32(S, ooc, dequant_half_h(c0, sb2, gs2), dequant_half_h(c1, sb2, gs2));
-            } else {
-                st_v2(S.out + ooc, make_uint2(c0, c1));   // 8-byte aligned: 2 jc even
-                S.sb[(int64_t)b * (S.chunks >> 1) + jc] = (uint8_t)sb;
+        // the piece's member segments, last first: member i holds units
+        // [mblk0[i], mblk0[i + 1]) of the instance.  Per segment the
+        // member's values are CTA-uniform and read once; its blocks
+        // j = jh - 1 - k, k = tid, tid + kThreads, ..., the next block's
+        // loads issued before the current one is encoded.
+        int i = four_six_member(a, G, re - 1u);
+        for (uint32_t se = re; se > rs; --i) {
+            const Sib& S = a.m[i];
+            const uint32_t m0 = a.mblk0[i];
+            const uint32_t ss = max(rs, m0);
+            const uint32_t jh = se - m0, n = se - ss;
+            se = ss;
+            const char* xb = S.x + (int64_t)b * S.x_bs;
+            char* ob = S.out + (int64_t)b * S.o_bs;
+            uint8_t* sbb = kFake ? nullptr : S.sb + (int64_t)b * (S.chunks >> 1);
+            const float* tsb = kFp8 ? S.ts + (int64_t)b * S.ts_bs : nullptr;
+            const bool dense_x = S.dense_x, dense_o = S.dense_o;
+            const int vec_x = kFp8 ? S.vec16_x : S.vec32_x, vec_o = S.vec32_o;
+            const FastDiv cpr = S.cpr;
+            const int64_t x_rs = S.x_rs, o_rs = S.o_rs;
+            const uint32_t tn = S.tn;
+            // block j: its source bytes (and, FP8, its tile scale) and its output offset
+            auto fetch = [&](uint32_t j, uint4& flo, uint4& fhi, float& fsc, int64_t& foo) {
+                const uint32_t c = 2u * j;   // the block's first chunk; c + 1 is in the same row
+                uint32_t r = 0u, kc = 0u;
+                if (kFp8 || !dense_x || !dense_o) {
+                    r = fdiv(c, cpr);
+                    kc = c - r * cpr.d;
+                }
+                constexpr uint32_t kXb = kFp8 ? 8u : 16u, kOb = kFake ? 16u : 4u;   // bytes per chunk
+                const char* p = xb + (dense_x ? (int64_t)c * kXb : (int64_t)r * x_rs + (int64_t)kc * kXb);
+                foo = dense_o ? (int64_t)c * kOb : (int64_t)r * o_rs + (int64_t)kc * kOb;
+                if (kFp8) {
+                    fsc = __ldg(tsb + (r >> 7) * tn + (kc >> 4));
+                    if (vec_x) {
+                        flo = ld_stream_v4(p);
+                    } else {
+                        const uint2 c0 = ld_stream_v2(p), c1 = ld_stream_v2(p + 8);
+                        flo = make_uint4(c0.x, c0.y, c1.x, c1.y);
+                    }
+                } else {
+                    ld_block32(p, vec_x, flo, fhi);
+                }
+            };
+            uint4 nlo = make_uint4(0u, 0u, 0u, 0u), nhi = nlo;
+            float nsc = 0.0f;
+            int64_t noo = 0;
+            if (threadIdx.x < n) fetch(jh - 1u - threadIdx.x, nlo, nhi, nsc, noo);
+            for (uint32_t k = threadIdx.x; k < n; k += kThreads) {
+                uint4 lo4 = nlo, hi4 = nhi;
+                const float sc = nsc;
+                const int64_t ooc = noo;
+                const uint32_t jc = jh - 1u - k;
+                if (k + kThreads < n) fetch(jc - kThreads, nlo, nhi, nsc, noo);
+                if (kFp8) {
+                    hi4 = fp8_dequant8(make_uint2(lo4.z, lo4.w), sc);
+                    lo4 = fp8_dequant8(make_uint2(lo4.x, lo4.y), sc);
+                }
+                const uint32_t mw = hmax_abs(amax_word8(lo4), amax_word8(hi4)) & 0x7fff7fffu;
+                const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
+                const float ratio = fast6 ? div_fast(amax_b, six_gs, r6) : div_slow(amax_b, six_gs);
+                const uint32_t sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
+                const float2 e = tab.e[sb];
+                uint32_t c0, c1;
+                if (all_fast) {
+                    float q[8];
+                    quotients8<true>(lo4, e.x, e.y, q);
+                    c0 = e2m1x8(q);
+                    quotients8<true>(hi4, e.x, e.y, q);
+                    c1 = e2m1x8(q);
+                } else {
+                    c0 = codes_half(lo4, e.x, e.y);
+                    c1 = codes_half(hi4, e.x, e.y);
+                }
+                if (kFake) {
+                    const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
+                    st_block32(ob + ooc, vec_o, dequant_half_h(c0, sb2, gs2), dequant_half_h(c1, sb2, gs2));
+                } else {
+                    st_v2(ob + ooc, make_uint2(c0, c1));   // 8-byte aligned: 2 jc even
+                    sbb[jc] = (uint8_t)sb;
+                }
             }
         }
         u = start;
@@ -625,7 +642,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_cluster_kernel(const FourSixAr
             const int i = four_six_member(a, G, r);
             int64_t xo, oo;
             four_six_offsets<kFake>(a.m[i], b, r - a.mblk0[i], xo, oo);
-            ld_block32(a.m[i], xo, lo[k], hi[k]);
+            ld_block32(a.m[i].x + xo, a.m[i].vec32_x, lo[k], hi[k]);
         }
         m = max(m, max(amax_bits8(lo[k]), amax_bits8(hi[k])));
     }
@@ -680,7 +697,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_cluster_kernel(const FourSixAr
             const uint32_t c0 = codes_half(lo[k], e.x, e.y), c1 = codes_half(hi[k], e.x, e.y);
             if (kFake) {
                 const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
-                st_block32(S, oo, dequant_half_h(c0, sb2, gs2), dequant_half_h(c1, sb2, gs2));
+                st_block32(S.out + oo, S.vec32_o, dequant_half_h(c0, sb2, gs2), dequant_half_h(c1, sb2, gs2));
             } else {
                 st_v2(S.out + oo, make_uint2(c0, c1));   // 8-byte aligned: 2 j even
                 S.sb[(int64_t)b * (S.chunks >> 1) + j] = (uint8_t)sb;

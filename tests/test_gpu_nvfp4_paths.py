@@ -134,3 +134,28 @@ def test_nvfp4_cluster_grouped_mixed_with_flow(P):
                 assert np.array_equal(u8(packed[g][i]), opk) and np.array_equal(u8(sb[g][i]), osb), (g, i)
                 assert f32bits(gs[g])[0] == np.float32(ogs).view(np.uint32), g
                 assert np.array_equal(u16(fq[g][i]), O.nvfp4_fake_quant(x, A)), (g, i)
+
+
+def test_nvfp4_amax_given_empty_and_strided_members(P):
+    """Quantise / fake-quantise with a given amax over groups whose every
+    instance exceeds the cluster path's limit (the streaming encode over
+    member segments): empty members between and after non-empty ones, a
+    member with padded rows, two batch indices."""
+    shapes = [(2, 200, 512), (2, 0, 512), (2, 130, 512), (2, 0, 512)]
+    xs = [rand_bits(s, seed=4300 + i) for i, s in enumerate(shapes)]
+    A = [np.float32(2.0) * np.float32(O.nvfp4_group_amax([x[b] for x in xs if x.size])) for b in range(2)]
+    amax = torch.tensor(A, dtype=torch.float32, device=DEV)
+    xg = [W.from_bits(x, DEV) if x.size else torch.empty(x.shape, dtype=torch.bfloat16, device=DEV) for x in xs]
+    xg[2] = padded(xs[2], 24)
+    packed, sb, gs = P.nvfp4_quant(xg, amax=amax)
+    fq = P.nvfp4_fake_quant(xg, amax=amax)
+    for b in range(2):
+        for i, x in enumerate(xs):
+            if not x.size:
+                assert packed[i].numel() == 0 and fq[i].numel() == 0
+                continue
+            opk, osb, ogs = O.nvfp4_quant(x[b], A[b])
+            assert f32bits(gs)[b] == np.float32(ogs).view(np.uint32), b
+            assert np.array_equal(u8(packed[i][b]), opk), (b, i)
+            assert np.array_equal(u8(sb[i][b]), osb), (b, i)
+            assert np.array_equal(u16(fq[i][b]), O.nvfp4_fake_quant(x[b], A[b])), (b, i)

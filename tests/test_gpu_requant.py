@@ -149,6 +149,10 @@ def test_fp8_to_nvfp4_codes_only_8_byte_aligned(P):
     A, out, gs = want[0]
     assert np.array_equal(f32bits(g), gs.view(np.uint32))
     assert np.array_equal(u8(pk), out[0][0]) and np.array_equal(u8(sb), out[0][1])
+    # the same with the amax given (the streaming encode reads 8-byte code pairs)
+    pk, sb, g = P.fp8_block_requant_nvfp4(q0, torch.from_numpy(s[0]).to(DEV), amax=torch.from_numpy(A).to(DEV))
+    assert np.array_equal(f32bits(g), gs.view(np.uint32))
+    assert np.array_equal(u8(pk), out[0][0]) and np.array_equal(u8(sb), out[0][1])
     # a batch of two with a batch stride of M * N + 8 bytes
     bs = M * N + 8
     buf2 = torch.zeros(2 * bs, dtype=torch.uint8, device=DEV)
