@@ -418,51 +418,65 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kern
             if (G.amax_out) G.amax_out[b] = A;
         }
         __syncthreads();
-        // units u - 1 - t, u - 1 - t - kThreads, ... down to start; the next
-        // one's two loads are issued before the current one is encoded
+        // the piece's member segments, last first (member i holds units
+        // [mblk0[i], mblk0[i + 1]) of the instance); per segment the
+        // member's values are CTA-uniform and read once; its blocks
+        // j = jh - 1 - k, k = tid, tid + kThreads, ..., the next block's two
+        // loads issued before the current one is encoded
         const uint32_t rs = (uint32_t)(start - inst_lo), re = (uint32_t)(u - inst_lo);
-        const uint32_t n = re - rs;
-        int i = 0;
-        int64_t xo = 0, oo = 0;
-        uint4 nlo = make_uint4(0u, 0u, 0u, 0u), nhi = nlo;
-        if (threadIdx.x < n) {
-            const uint32_t r = re - 1u - threadIdx.x;
-            i = four_six_member(a, G, r);
-            four_six_offsets<kFake>(a.m[i], b, r - a.mblk0[i], xo, oo);
-            nlo = ld_stream_v4(a.m[i].x + xo);
-            nhi = ld_stream_v4(a.m[i].x + xo + 16);
-        }
-        for (uint32_t k = threadIdx.x; k < n; k += kThreads) {
-            const uint4 lo4 = nlo, hi4 = nhi;
-            const int ic = i;
-            const int64_t ooc = oo;
-            const uint32_t jc = re - 1u - k - a.mblk0[ic];   // block within the member
-            if (k + kThreads < n) {
-                const uint32_t r = re - 1u - k - kThreads;
-                i = four_six_member(a, G, r);
-                four_six_offsets<kFake>(a.m[i], b, r - a.mblk0[i], xo, oo);
-                nlo = ld_stream_v4(a.m[i].x + xo);
-                nhi = ld_stream_v4(a.m[i].x + xo + 16);
-            }
-            const Sib& S = a.m[ic];
-            const uint32_t mw = hmax_abs(amax_word8(lo4), amax_word8(hi4)) & 0x7fff7fffu;
-            const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
-            uint64_t xl[4], xh[4];
-            widen8(lo4, xl);
-            widen8(hi4, xh);
-            uint32_t sb6, a0, a1, sb4, b0, b1;
-            uint4 ya0, ya1, yb0, yb1;
-            const float e6 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g6, r6, fast6, tab, gs2, sb6, a0, a1,
-                                                ya0, ya1);
-            const float e4 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g4, r4, fast4, tab, gs2, sb4, b0, b1,
-                                                yb0, yb1);
-            const bool four = e4 < e6;
-            if (kFake) {
-                st_v4(S.out + ooc, four ? yb0 : ya0);
-                st_v4(S.out + ooc + 16, four ? yb1 : ya1);
-            } else {
-                st_v2(S.out + ooc, make_uint2(four ? b0 : a0, four ? b1 : a1));   // 8-byte aligned: 2 jc even
-                S.sb[(int64_t)b * (S.chunks >> 1) + jc] = (uint8_t)(four ? sb4 : sb6);
+        int i = four_six_member(a, G, re - 1u);
+        for (uint32_t se = re; se > rs; --i) {
+            const Sib& S = a.m[i];
+            const uint32_t m0 = a.mblk0[i];
+            const uint32_t ss = max(rs, m0);
+            const uint32_t jh = se - m0, n = se - ss;
+            se = ss;
+            const char* xb = S.x + (int64_t)b * S.x_bs;
+            char* ob = S.out + (int64_t)b * S.o_bs;
+            uint8_t* sbb = kFake ? nullptr : S.sb + (int64_t)b * (S.chunks >> 1);
+            const bool dense_x = S.dense_x, dense_o = S.dense_o;
+            const FastDiv cpr = S.cpr;
+            const int64_t x_rs = S.x_rs, o_rs = S.o_rs;
+            auto fetch = [&](uint32_t j, uint4& flo, uint4& fhi, int64_t& foo) {
+                const uint32_t c = 2u * j;   // the block's first chunk; c + 1 is in the same row
+                uint32_t r = 0u, kc = 0u;
+                if (!dense_x || !dense_o) {
+                    r = fdiv(c, cpr);
+                    kc = c - r * cpr.d;
+                }
+                constexpr uint32_t kOb = kFake ? 16u : 4u;   // output bytes per chunk
+                const char* p = xb + (dense_x ? (int64_t)c * 16 : (int64_t)r * x_rs + (int64_t)kc * 16);
+                foo = dense_o ? (int64_t)c * kOb : (int64_t)r * o_rs + (int64_t)kc * kOb;
+                flo = ld_stream_v4(p);
+                fhi = ld_stream_v4(p + 16);
+            };
+            uint4 nlo = make_uint4(0u, 0u, 0u, 0u), nhi = nlo;
+            int64_t noo = 0;
+            if (threadIdx.x < n) fetch(jh - 1u - threadIdx.x, nlo, nhi, noo);
+            for (uint32_t k = threadIdx.x; k < n; k += kThreads) {
+                const uint4 lo4 = nlo, hi4 = nhi;
+                const int64_t ooc = noo;
+                const uint32_t jc = jh - 1u - k;
+                if (k + kThreads < n) fetch(jc - kThreads, nlo, nhi, noo);
+                const uint32_t mw = hmax_abs(amax_word8(lo4), amax_word8(hi4)) & 0x7fff7fffu;
+                const float amax_b = __uint_as_float(max(mw & 0xffffu, mw >> 16) << 16);
+                uint64_t xl[4], xh[4];
+                widen8(lo4, xl);
+                widen8(hi4, xh);
+                uint32_t sb6, a0, a1, sb4, b0, b1;
+                uint4 ya0, ya1, yb0, yb1;
+                const float e6 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g6, r6, fast6, tab, gs2, sb6, a0, a1,
+                                                    ya0, ya1);
+                const float e4 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g4, r4, fast4, tab, gs2, sb4, b0, b1,
+                                                    yb0, yb1);
+                const bool four = e4 < e6;
+                if (kFake) {
+                    st_v4(ob + ooc, four ? yb0 : ya0);
+                    st_v4(ob + ooc + 16, four ? yb1 : ya1);
+                } else {
+                    st_v2(ob + ooc, make_uint2(four ? b0 : a0, four ? b1 : a1));   // 8-byte aligned: 2 jc even
+                    sbb[jc] = (uint8_t)(four ? sb4 : sb6);
+                }
             }
         }
         u = start;
