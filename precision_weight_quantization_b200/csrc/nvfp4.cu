@@ -492,7 +492,10 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kern
 // backwards one instance piece at a time (the scale table belongs to the
 // instance's gs), one thread per 16-element block, the next block's loads
 // issued before the current one is encoded.  kFp8: an FP8 block-wise source
-// whose codes are dequantised in registers, y = bf16(fl(dec(q) s)).
+// whose codes are dequantised in registers, y = bf16(fl(dec(q) s)).  Four
+// CTAs per SM (at most 64 registers a thread): a block's 32 bytes are one
+// 256-bit access where aligned, and more blocks in flight per thread
+// measured no faster than the fourth CTA.
 
 constexpr int kUnitCtasPerSm = 4;
 template <bool kFake, bool kFp8>
