@@ -133,6 +133,22 @@ def test_fp8_to_nvfp4_siblings(P, shapes, raw):
         assert torch.equal(pk2[i], pk[i]) and torch.equal(sb2[i].view(torch.uint8), sb[i].view(torch.uint8))
 
 
+@pytest.mark.parametrize("pad", [8, 16])   # code rows 8- and 16-byte aligned
+def test_fp8_to_nvfp4_strided_codes_amax_given(P, pad):
+    """Padded (strided) code rows, batched, a sibling pair, with the group
+    amax given: the streaming encode addresses each block through its row
+    and column; codes, block scales and global scales against the oracle."""
+    members = [codes_and_scales(sh, seed=60 + i, raw=True) for i, sh in enumerate([(2, 130, 272), (2, 70, 272)])]
+    A, out, gs = O.fp8_block_requant_nvfp4([m[0] for m in members], [m[1] for m in members])
+    qs = [to_gpu_codes(m[0], pad) for m in members]
+    ss = [torch.from_numpy(m[1]).to(DEV) for m in members]
+    pk, sb, g = P.fp8_block_requant_nvfp4(qs, ss, amax=torch.from_numpy(A).to(DEV))
+    assert np.array_equal(f32bits(g), gs.view(np.uint32))
+    for i in range(2):
+        assert np.array_equal(u8(pk[i]), out[i][0]), i
+        assert np.array_equal(u8(sb[i]), out[i][1]), i
+
+
 def test_fp8_to_nvfp4_codes_only_8_byte_aligned(P):
     """E4M3 code tensors need only 8-byte alignment: dense code rows whose
     base, or whose batch stride, is 8 bytes off a 16-byte boundary are read
