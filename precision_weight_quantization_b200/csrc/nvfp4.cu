@@ -181,6 +181,40 @@ __device__ __forceinline__ void fill_scale_table(ScaleTable& t, float gs) {
     }
 }
 
+// Per block-scale code k, the dequantised magnitudes y(m) =
+// bf16(fl(fl(dec(m) dec(k)) gs)) of the 8 E2M1 magnitude codes m, as
+// dequant_half_h computes them, in byte planes for byte permutes: {low
+// bytes of y(0..3), low bytes of y(4..7), high bytes of y(0..3), high
+// bytes of y(4..7)}.  A fake-quantised block then looks its values up
+// instead of decoding and multiplying each one.
+struct DeqTable {
+    uint4 e[128];
+};
+
+__device__ __forceinline__ void fill_deq_table(DeqTable& t, uint64_t gs2) {
+    for (uint32_t k = threadIdx.x; k < 128u; k += blockDim.x) {
+        const uint4 w = dequant_half_h(0x76543210u, e4m3x2_f16x2(k * 0x101u), gs2);   // y(0), y(1), ..., y(7)
+        t.e[k] = make_uint4(__byte_perm(w.x, w.y, 0x6420u), __byte_perm(w.z, w.w, 0x6420u),
+                            __byte_perm(w.x, w.y, 0x7531u), __byte_perm(w.z, w.w, 0x7531u));
+    }
+}
+
+// The BF16 values of the 8 E2M1 codes of a half block (element 0 in bits
+// 0..3) from the block's DeqTable entry tb, each with the sign of its input
+// value in x: with a positive divisor a code carries its input's sign,
+// signed zeros included, and rounding is symmetric in sign, so y(-m) is
+// -y(m).  Byte permutes pick the magnitude bytes (3-bit indices), then
+// interleave the low and high bytes into BF16 pairs.
+__device__ __forceinline__ uint4 dequant_lookup8(uint32_t codes, uint4 tb, uint4 x) {
+    const uint32_t s0 = codes & 0x7777u, s1 = (codes >> 16) & 0x7777u;
+    const uint32_t l0 = __byte_perm(tb.x, tb.y, s0), h0 = __byte_perm(tb.z, tb.w, s0);
+    const uint32_t l1 = __byte_perm(tb.x, tb.y, s1), h1 = __byte_perm(tb.z, tb.w, s1);
+    return make_uint4(__byte_perm(l0, h0, 0x5140u) | (x.x & 0x80008000u),
+                      __byte_perm(l0, h0, 0x7362u) | (x.y & 0x80008000u),
+                      __byte_perm(l1, h1, 0x5140u) | (x.z & 0x80008000u),
+                      __byte_perm(l1, h1, 0x7362u) | (x.w & 0x80008000u));
+}
+
 // E2M1 codes of one 8-element half block (element 0 in bits 0..3).
 __device__ __forceinline__ uint32_t codes_half(uint4 v, float d, float r) {
     float q[8];
@@ -325,23 +359,26 @@ __device__ __forceinline__ uint32_t codes_neg8(const uint64_t (&x)[4], uint64_t 
 // dequantised values.
 __device__ __forceinline__ float four_six_candidate(uint4 lo, uint4 hi, const uint64_t (&xl)[4],
                                                     const uint64_t (&xh)[4], float amax_b, float t_gs, float rt,
-                                                    bool fast_t, const ScaleTable& tab, uint64_t gs2,
-                                                    uint32_t& sb, uint32_t& c0, uint32_t& c1, uint4& y0,
-                                                    uint4& y1) {
+                                                    bool fast_t, const ScaleTable& tab, const DeqTable& dtab,
+                                                    uint64_t gs2, uint32_t& sb, uint32_t& c0, uint32_t& c1,
+                                                    uint4& y0, uint4& y1) {
     const float ratio = fast_t ? div_fast(amax_b, t_gs, rt) : div_slow(amax_b, t_gs);
     sb = e4m3x2(ratio, 0.0f) & 0x7fu;   // ratio >= 0
     const float2 e = tab.e[sb];
-    if (e.y != 0.0f) {
+    if (e.y != 0.0f) {   // d > 0 finite, so gs is: the table holds the values
         const uint64_t d2 = f32x2(e.x, e.x), nr2 = f32x2(-e.y, -e.y);
         c0 = codes_neg8(xl, d2, nr2);
         c1 = codes_neg8(xh, d2, nr2);
+        const uint4 tb = dtab.e[sb];
+        y0 = dequant_lookup8(c0, tb, lo);
+        y1 = dequant_lookup8(c1, tb, hi);
     } else {
         c0 = codes_half(lo, e.x, e.y);
         c1 = codes_half(hi, e.x, e.y);
+        const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
+        y0 = dequant_half_h(c0, sb2, gs2);
+        y1 = dequant_half_h(c1, sb2, gs2);
     }
-    const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
-    y0 = dequant_half_h(c0, sb2, gs2);
-    y1 = dequant_half_h(c1, sb2, gs2);
     return sse8(xh, y1, sse8(xl, y0, 0.0f));
 }
 
@@ -396,6 +433,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_4over6_amax_kernel(const FourS
 template <bool kFake>
 __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kernel(const FourSixArgs a) {
     __shared__ ScaleTable tab;
+    __shared__ DeqTable dtab;
     uint64_t lo, hi;
     four_six_range(a, lo, hi);
     for (uint64_t u = hi; u > lo;) {
@@ -413,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kern
         const uint64_t gs2 = f32x2(gs, gs);
         __syncthreads();   // the previous piece's table reads are done
         fill_scale_table(tab, gs);
+        fill_deq_table(dtab, gs2);
         if (start == inst_lo && threadIdx.x == 0) {   // the one CTA that holds the instance's first unit
             if (G.gs_out) G.gs_out[b] = gs;
             if (G.amax_out) G.amax_out[b] = A;
@@ -465,9 +504,9 @@ __global__ void __launch_bounds__(kThreads, kFourSixCtasPerSm) nvfp4_4over6_kern
                 widen8(hi4, xh);
                 uint32_t sb6, a0, a1, sb4, b0, b1;
                 uint4 ya0, ya1, yb0, yb1;
-                const float e6 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g6, r6, fast6, tab, gs2, sb6, a0, a1,
+                const float e6 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g6, r6, fast6, tab, dtab, gs2, sb6, a0, a1,
                                                     ya0, ya1);
-                const float e4 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g4, r4, fast4, tab, gs2, sb4, b0, b1,
+                const float e4 = four_six_candidate(lo4, hi4, xl, xh, amax_b, g4, r4, fast4, tab, dtab, gs2, sb4, b0, b1,
                                                     yb0, yb1);
                 const bool four = e4 < e6;
                 if (kFake) {
@@ -1062,8 +1101,9 @@ __device__ __forceinline__ uint32_t flow_lc(int j, uint32_t tid, uint32_t sw) {
 // item exist and both operands are dense.
 template <bool kFake, bool kFast, bool kFull>
 __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThread], const FlowItem& it,
-                                            const FlowMember& M, const ScaleTable& tab, float gs, float six_gs,
-                                            float r6, bool fast6, uint64_t pol, uint32_t sw, uint32_t c_off = 0u) {
+                                            const FlowMember& M, const ScaleTable& tab, const DeqTable& dtab,
+                                            float gs, float six_gs, float r6, bool fast6, uint64_t pol, uint32_t sw,
+                                            uint32_t c_off = 0u) {
     const uint32_t tid = threadIdx.x;
     char* ob = M.out + (int64_t)it.b * M.o_bs;
     uint8_t* sbb = kFake ? nullptr : M.sb + (int64_t)it.b * (M.sf_mma ? M.sf_slab : (int64_t)(M.chunks >> 1));
@@ -1093,6 +1133,12 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
             c0 = codes_half(lo, e.x, e.y);
             c1 = codes_half(hi, e.x, e.y);
         }
+        uint4 ya, yb;   // fake, fast: the values of the codes of lo and hi
+        if (kFake && kFast) {
+            const uint4 tb = dtab.e[sb];
+            ya = dequant_lookup8(c0, tb, lo);
+            yb = dequant_lookup8(c1, tb, hi);
+        }
         if (sw) {   // v[2i] held the block's second chunk
             const uint32_t t = c0;
             c0 = c1;
@@ -1107,9 +1153,16 @@ __device__ __forceinline__ void flow_encode(const uint4 (&v)[kItemChunksPerThrea
                 oo = (int64_t)r * M.o_rs + (int64_t)(c - r * M.cpr.d) * (kFake ? 16 : 4);
             }
             if (kFake) {
-                const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
-                const uint64_t gs2 = f32x2(gs, gs);
-                const uint4 y0 = dequant_half_h(c0, sb2, gs2), y1 = dequant_half_h(c1, sb2, gs2);
+                uint4 y0, y1;
+                if (kFast) {
+                    y0 = sw ? yb : ya;
+                    y1 = sw ? ya : yb;
+                } else {
+                    const uint32_t sb2 = e4m3x2_f16x2(sb * 0x101u);
+                    const uint64_t gs2 = f32x2(gs, gs);
+                    y0 = dequant_half_h(c0, sb2, gs2);
+                    y1 = dequant_half_h(c1, sb2, gs2);
+                }
                 if (M.vec32_o) {
                     st_hint_v8(ob + oo, y0, y1, pol);
                 } else {
@@ -1162,6 +1215,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
     extern __shared__ __align__(128) unsigned char flow_smem[];
     __shared__ FlowTables t;
     __shared__ ScaleTable tab;
+    __shared__ DeqTable dtab;   // fake-quantise only
     __shared__ FlowItem items[kFlowStages + 1];   // item n in slot n % (kFlowStages + 1)
     __shared__ __align__(8) uint64_t bars[kFlowStages];
     __shared__ uint32_t s_amax[2];
@@ -1400,6 +1454,7 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
             // every non-zero block scale gives dec(sb) * gs in [2^-9 gs, 448 gs]
             all_fast = fast6 && __fmul_rn(0x1p-9f, gs) >= 0x1p-64f && __fmul_rn(448.0f, gs) <= 0x1p126f;
             fill_scale_table(tab, gs);
+            if (kFake) fill_deq_table(dtab, f32x2(gs, gs));
             __syncthreads();
             cached = it.inst;
         }
@@ -1409,18 +1464,18 @@ __global__ void __launch_bounds__(kFlowThreads, kFlowCtasPerSm) nvfp4_flow_kerne
         }
         if (!kFp8) {
             if (all_fast && full)
-                flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream, sw);
+                flow_encode<kFake, true, true>(v, it, M, tab, dtab, gs, six_gs, r6, fast6, stream, sw);
             else
-                flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream, sw);
+                flow_encode<kFake, false, false>(v, it, M, tab, dtab, gs, six_gs, r6, fast6, stream, sw);
         } else {
 #pragma unroll 1
             for (int h = 0; h < kHalves; ++h) {
                 load_half(h, v);
                 if (all_fast && full)
-                    flow_encode<kFake, true, true>(v, it, M, tab, gs, six_gs, r6, fast6, stream, sw,
+                    flow_encode<kFake, true, true>(v, it, M, tab, dtab, gs, six_gs, r6, fast6, stream, sw,
                                                    (uint32_t)h * kItemChunks);
                 else
-                    flow_encode<kFake, false, false>(v, it, M, tab, gs, six_gs, r6, fast6, stream, sw,
+                    flow_encode<kFake, false, false>(v, it, M, tab, dtab, gs, six_gs, r6, fast6, stream, sw,
                                                      (uint32_t)h * kItemChunks);
             }
             __syncthreads();   // stage st is free
